@@ -1,0 +1,145 @@
+"""Seeded synthetic inputs for the gated delta rule workloads.
+
+This module holds workload shapes and value distributions only: none of the
+rule's arithmetic.  Both the CUDA path (tests, bench) and the float64 oracle
+are fed from it, so the two sides see bit-identical inputs.
+
+Distributions follow the workload recipe for a Qwen3-Next Gated DeltaNet
+layer (model card "Qwen3-Next-80B-A3B-Instruct", section "Model Overview":
+32 value heads, 16 query/key heads, head dim 128):
+
+* q, k ~ N(0, 1), then L2-normalised per head in fp32, then cast to the
+  workload dtype (so bf16 keys are unit length only up to rounding; the oracle
+  receives the rounded values, not re-normalised ones);
+* v ~ N(0, 1);
+* g = log(alpha) with alpha ~ U(0.9, 1.0) per token and value head (fp32);
+* beta = sigmoid(N(0, 1)) per token and value head (fp32);
+* h0 = 0, or ~N(0, 0.02) where the workload asks for a nonzero start state.
+
+Everything is drawn on the CPU from ``torch.Generator().manual_seed(seed)``.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    seed: int
+    kind: str                    # "prefill" or "decode"
+    B: int                       # batch (prefill without cu_seqlens) or sequences (decode)
+    T: int                       # tokens per sequence (prefill) / decode steps
+    HK: int
+    HV: int
+    dk: int
+    dv: int
+    chunk: int
+    dtype: torch.dtype
+    h0_std: float = 0.0          # 0 -> zero start state
+    varlen: tuple = field(default=())   # (n_seqs, lo, hi) -> packed lengths ~U[lo, hi]
+
+    @property
+    def dtype_name(self) -> str:
+        return {torch.float32: "f32", torch.bfloat16: "bf16"}[self.dtype]
+
+
+WORKLOADS = {
+    "tiny_fp32": Workload("tiny_fp32", 0, "prefill", 1, 128, 1, 2, 32, 32, 16, torch.float32),
+    "layer_prefill_4k": Workload("layer_prefill_4k", 1, "prefill", 1, 4096, 16, 32, 128, 128, 64,
+                                 torch.bfloat16),
+    "long_prefill_64k": Workload("long_prefill_64k", 2, "prefill", 1, 65536, 16, 32, 128, 128, 64,
+                                 torch.bfloat16),
+    "varlen_8": Workload("varlen_8", 3, "prefill", 1, 0, 16, 32, 128, 128, 64, torch.bfloat16,
+                         h0_std=0.02, varlen=(8, 1024, 32768)),
+    "decode_256x64": Workload("decode_256x64", 4, "decode", 256, 64, 16, 32, 128, 128, 1,
+                              torch.bfloat16, h0_std=0.02),
+}
+
+
+def _unit_rows(x: torch.Tensor) -> torch.Tensor:
+    # L2 normalisation of each head vector, in fp32, before the cast
+    return x / x.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+
+
+def draw_lengths(gen: torch.Generator, n: int, lo: int, hi: int) -> list[int]:
+    return [int(x) for x in torch.randint(lo, hi + 1, (n,), generator=gen)]
+
+
+def make_prefill(HK: int, HV: int, dk: int, dv: int, lengths, dtype=torch.bfloat16,
+                 seed: int = 0, h0_std: float = 0.0, packed: bool | None = None,
+                 g_low: float = 0.9, g_high: float = 1.0):
+    """Draw one prefill problem.
+
+    ``lengths`` is a list of per-sequence token counts.  If every length is
+    equal and ``packed`` is not True, tensors are [B,T,H,d] and ``cu_seqlens``
+    is None; otherwise they are packed as [1,Ttot,H,d] with int32 ``cu_seqlens``.
+    Returns a dict of CPU tensors: q,k,v (dtype), g,beta (fp32), h0 (fp32 or
+    None), cu_seqlens (int32 or None).
+    """
+    gen = torch.Generator().manual_seed(seed)
+    lengths = [int(x) for x in lengths]
+    if packed is None:
+        packed = len(set(lengths)) > 1
+    N = len(lengths)
+    Ttot = sum(lengths)
+    q = _unit_rows(torch.randn(Ttot, HK, dk, generator=gen)).to(dtype)
+    k = _unit_rows(torch.randn(Ttot, HK, dk, generator=gen)).to(dtype)
+    v = torch.randn(Ttot, HV, dv, generator=gen).to(dtype)
+    alpha = g_low + (g_high - g_low) * torch.rand(Ttot, HV, generator=gen)
+    g = torch.log(alpha).float()
+    beta = torch.sigmoid(torch.randn(Ttot, HV, generator=gen)).float()
+    h0 = None
+    if h0_std > 0:
+        h0 = (h0_std * torch.randn(N, HV, dv, dk, generator=gen)).float()
+    if packed:
+        cu = torch.zeros(N + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+        shape = lambda x: x.reshape(1, Ttot, *x.shape[1:])
+        return dict(q=shape(q), k=shape(k), v=shape(v), g=shape(g), beta=shape(beta), h0=h0,
+                    cu_seqlens=cu)
+    T = lengths[0] if N else 0
+    shape = lambda x: x.reshape(N, T, *x.shape[1:])
+    return dict(q=shape(q), k=shape(k), v=shape(v), g=shape(g), beta=shape(beta), h0=h0,
+                cu_seqlens=None)
+
+
+def make_decode(N: int, steps: int, HK: int, HV: int, dk: int, dv: int, dtype=torch.bfloat16,
+                seed: int = 0, h0_std: float = 0.02):
+    """Draw ``steps`` successive single-token inputs for N sequences plus a start state.
+
+    Returns q,k [steps,N,HK,dk], v [steps,N,HV,dv], g,beta [steps,N,HV] and
+    state [N,HV,dv,dk] fp32, all CPU tensors.
+    """
+    gen = torch.Generator().manual_seed(seed)
+    q = _unit_rows(torch.randn(steps, N, HK, dk, generator=gen)).to(dtype)
+    k = _unit_rows(torch.randn(steps, N, HK, dk, generator=gen)).to(dtype)
+    v = torch.randn(steps, N, HV, dv, generator=gen).to(dtype)
+    g = torch.log(0.9 + 0.1 * torch.rand(steps, N, HV, generator=gen)).float()
+    beta = torch.sigmoid(torch.randn(steps, N, HV, generator=gen)).float()
+    state = (h0_std * torch.randn(N, HV, dv, dk, generator=gen)).float()
+    return dict(q=q, k=k, v=v, g=g, beta=beta, state=state)
+
+
+def workload_inputs(name: str, steps: int | None = None):
+    """Inputs for one named workload (see ``WORKLOADS``)."""
+    w = WORKLOADS[name]
+    if w.kind == "decode":
+        return make_decode(w.B, steps or w.T, w.HK, w.HV, w.dk, w.dv, w.dtype, w.seed, w.h0_std)
+    if w.varlen:
+        gen = torch.Generator().manual_seed(w.seed)
+        n, lo, hi = w.varlen
+        lengths = draw_lengths(gen, n, lo, hi)
+        return make_prefill(w.HK, w.HV, w.dk, w.dv, lengths, w.dtype, seed=w.seed + 1000,
+                            h0_std=w.h0_std, packed=True)
+    return make_prefill(w.HK, w.HV, w.dk, w.dv, [w.T] * w.B, w.dtype, seed=w.seed,
+                        h0_std=w.h0_std)
+
+
+def varlen_lengths(name: str = "varlen_8") -> list[int]:
+    w = WORKLOADS[name]
+    gen = torch.Generator().manual_seed(w.seed)
+    n, lo, hi = w.varlen
+    return draw_lengths(gen, n, lo, hi)

@@ -1,0 +1,163 @@
+"""Float64 CPU oracle for the gated delta rule (Python side).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this module.  The
+product path (the CUDA library and its binding) never imports it and shares no
+code with it.
+
+The arithmetic lives in ``gdn_oracle.c`` (plain C, float64, one thread per
+(sequence, value head) unit); this module only builds that file with gcc,
+converts inputs to contiguous float64 numpy arrays and calls it.  See the C
+file's header for the rule it follows and the pages it cites:
+
+* the delta rule with decay applied first ("Qwen3-Next", sghael.github.io,
+  section "Correcting a memory instead of adding to it"),
+* 32 value heads reading 16 query/key heads at head dim 128 (model card
+  "Qwen3-Next-80B-A3B-Instruct", section "Model Overview"),
+* read-out after the update, state rows indexed by the value dimension
+  ("The Evolving Transformer / Qwen3-Next", section 01 GatedDeltaNet).
+
+Every function here has its result pinned by ``tests/test_oracle_pins.py``
+against values the pages print, closed forms, invariants and the agreement of
+the two independent forms (sequential definition vs. chunkwise WY form).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB = os.path.join(_HERE, "libgdn_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, no fast-math) into ``libgdn_oracle.so``."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-std=c11", "-fPIC",
+             "-shared", "-pthread", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _bind(lib):
+    lib.gdn_oracle_prefill.restype = ctypes.c_int
+    lib.gdn_oracle_prefill.argtypes = [
+        _dp, _dp, _dp, _dp, _dp, _dp, _i64p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_double, _dp, _dp, ctypes.c_int]
+    lib.gdn_oracle_prefill_chunked.restype = ctypes.c_int
+    lib.gdn_oracle_prefill_chunked.argtypes = [
+        _dp, _dp, _dp, _dp, _dp, _dp, _i64p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, _dp, _dp, ctypes.c_int]
+    lib.gdn_oracle_step.restype = ctypes.c_int
+    lib.gdn_oracle_step.argtypes = [
+        _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_double, _dp]
+    return lib
+
+
+def _load(path=None):
+    """The oracle library; ``path`` selects another build of the same C source
+    (the mutation tests load deliberately broken copies this way)."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor: exact upcast (bf16/fp32 -> fp64 is exact)
+        x = x.detach().to("cpu")
+        import torch
+        x = x.to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_dp)
+
+
+def _flatten_tokens(q, k, v, g, beta, cu_seqlens):
+    """Accept [B,T,H,d] (+ no cu_seqlens) or packed [1,Ttot,H,d] / [Ttot,H,d] + cu_seqlens."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    if q.ndim == 4:
+        B, T = q.shape[0], q.shape[1]
+        q = q.reshape(B * T, *q.shape[2:])
+        k = k.reshape(B * T, *k.shape[2:])
+        v = v.reshape(B * T, *v.shape[2:])
+        g = g.reshape(B * T, -1)
+        beta = beta.reshape(B * T, -1)
+    else:
+        B, T = 1, q.shape[0]
+    if cu_seqlens is None:
+        cu = np.arange(0, B * T + 1, T, dtype=np.int64) if T > 0 else np.zeros(B + 1, np.int64)
+    else:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    return q, k, v, g, beta, cu
+
+
+def prefill(q, k, v, g, beta, h0=None, cu_seqlens=None, scale=1.0, nthreads=0,
+            chunked=False, chunk=64, lib=None):
+    """Run the oracle over a batch.
+
+    Shapes: q,k [B,T,HK,dk]; v [B,T,HV,dv]; g,beta [B,T,HV]; or packed
+    [1,Ttot,...] with ``cu_seqlens`` (N+1 offsets).  h0 [N,HV,dv,dk] or None.
+    Returns (o [Ttot or B*T, HV, dv] float64, hT [N,HV,dv,dk] float64).
+    ``chunked=True`` runs the chunkwise WY form instead of the definition.
+    """
+    q, k, v, g, beta, cu = _flatten_tokens(q, k, v, g, beta, cu_seqlens)
+    Ttot, HK, dk = q.shape
+    HV, dv = v.shape[1], v.shape[2]
+    N = cu.shape[0] - 1
+    h0 = _f64(h0)
+    if h0 is not None:
+        h0 = h0.reshape(N, HV, dv, dk)
+    o = np.zeros((Ttot, HV, dv), dtype=np.float64)
+    hT = np.zeros((N, HV, dv, dk), dtype=np.float64)
+    lib = lib or _load()
+    if chunked:
+        rc = lib.gdn_oracle_prefill_chunked(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+            cu.ctypes.data_as(_i64p), N, HK, HV, dk, dv, int(chunk), float(scale),
+            _ptr(o), _ptr(hT), int(nthreads))
+    else:
+        rc = lib.gdn_oracle_prefill(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+            cu.ctypes.data_as(_i64p), N, HK, HV, dk, dv, float(scale),
+            _ptr(o), _ptr(hT), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (rc={rc})")
+    return o, hT
+
+
+def step(q, k, v, g, beta, state, scale=1.0, lib=None):
+    """One decode token per sequence.  q,k [N,HK,dk]; v [N,HV,dv]; g,beta [N,HV];
+    state [N,HV,dv,dk].  Returns (o [N,HV,dv], new_state) as float64 arrays."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    S = _f64(state).copy()
+    N, HK, dk = q.shape
+    HV, dv = v.shape[1], v.shape[2]
+    o = np.zeros((N, HV, dv), dtype=np.float64)
+    rc = (lib or _load()).gdn_oracle_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                                 N, HK, HV, dk, dv, float(scale), _ptr(o))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (rc={rc})")
+    return o, S

@@ -1,0 +1,316 @@
+"""Checks that pin the float64 oracle to facts fixed by the pages and by mathematics.
+
+Each ``pin_*`` function takes an oracle library handle (``None`` = the normal
+build) and raises AssertionError when the oracle disagrees.  They are run by
+``test_oracle_pins.py`` against the real oracle and by
+``test_oracle_mutants.py`` against deliberately broken copies, to show that a
+plausible mistake (a dropped term, a wrong sign or index, the error term taken
+before the decay, the read-out taken before the update, a transposed operand)
+fails at least one of them.
+
+Sources:
+* worked examples: "Qwen3-Next" (sghael.github.io), section "Correcting a
+  memory instead of adding to it" (fixtures under tests/golden/);
+* head geometry 32 V / 16 QK / 128: model card "Qwen3-Next-80B-A3B-Instruct",
+  section "Model Overview";
+* the rule S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T, o_t = S_t q_t
+  and its invariants: closed forms derived from it (stated per check).
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+
+from oracle import gdn_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _read_fixture(name):
+    s0, rows = None, []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            if parts[0] == "S0":
+                s0 = float(parts[1])
+            else:
+                rows.append([float(x) for x in parts[1:]])
+    return s0, np.array(rows)
+
+
+def _rand_problem(rng, T, HK, HV, dk, dv, unit=True, g_range=(math.log(0.9), 0.0)):
+    q = rng.standard_normal((1, T, HK, dk))
+    k = rng.standard_normal((1, T, HK, dk))
+    if unit:
+        q /= np.linalg.norm(q, axis=-1, keepdims=True)
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((1, T, HV, dv))
+    g = rng.uniform(*g_range, size=(1, T, HV))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((1, T, HV))))
+    return q, k, v, g, beta
+
+
+# ----------------------------------------------------------------------------
+# Values printed on the pages
+# ----------------------------------------------------------------------------
+def pin_worked_example_delta(lib=None):
+    s0, rows = _read_fixture("worked_example_delta.txt")
+    T = len(rows)
+    one = np.ones((1, T, 1, 1))
+    g = rows[:, 0].reshape(1, T, 1)
+    beta = rows[:, 1].reshape(1, T, 1)
+    v = rows[:, 2].reshape(1, T, 1, 1)
+    o, hT = O.prefill(one, one, v, g, beta, h0=np.full((1, 1, 1, 1), s0), lib=lib)
+    assert np.array_equal(o.ravel(), rows[:, 3]), (o.ravel(), rows[:, 3])
+    assert hT.ravel()[0] == rows[-1, 3]
+    # the same through the chunked form and through decode steps
+    oc, _ = O.prefill(one, one, v, g, beta, h0=np.full((1, 1, 1, 1), s0), chunked=True,
+                      chunk=2, lib=lib)
+    assert np.allclose(oc.ravel(), rows[:, 3], rtol=0, atol=1e-12)
+    S = np.full((1, 1, 1, 1), s0)
+    for t in range(T):
+        ot, S = O.step(one[:, t], one[:, t], v[:, t], g[:, t], beta[:, t], S, lib=lib)
+        assert ot.ravel()[0] == rows[t, 3]
+
+
+def pin_worked_example_gated(lib=None):
+    s0, rows = _read_fixture("worked_example_gated.txt")
+    T = len(rows)
+    one = np.ones((1, T, 1, 1))
+    g = np.log(rows[:, 0]).reshape(1, T, 1)
+    beta = rows[:, 1].reshape(1, T, 1)
+    v = rows[:, 2].reshape(1, T, 1, 1)
+    h0 = np.full((1, 1, 1, 1), s0)
+    o, hT = O.prefill(one, one, v, g, beta, h0=h0, lib=lib)
+    assert np.allclose(o.ravel(), rows[:, 3], rtol=0, atol=1e-14), o.ravel()
+    oc, _ = O.prefill(one, one, v, g, beta, h0=h0, chunked=True, chunk=1, lib=lib)
+    assert np.allclose(oc.ravel(), rows[:, 3], rtol=0, atol=1e-14), oc.ravel()
+    ot, _ = O.step(one[:, 0], one[:, 0], v[:, 0], g[:, 0], beta[:, 0], h0, lib=lib)
+    assert np.allclose(ot.ravel(), rows[0, 3], rtol=0, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------
+# Closed forms and invariants of the rule
+# ----------------------------------------------------------------------------
+def pin_converges_closed_form(lib=None):
+    """No decay, one repeated unit key: S_n k = v + (1-b)^n (S_0 k - v) (the page's
+    "converges on 10"), and directions orthogonal to k are never touched."""
+    rng = np.random.default_rng(1)
+    dk, dv, T, b = 5, 3, 12, 0.3
+    kvec = rng.standard_normal(dk); kvec /= np.linalg.norm(kvec)
+    qvec = rng.standard_normal(dk)
+    vvec = rng.standard_normal(dv)
+    S0 = rng.standard_normal((dv, dk))
+    k = np.broadcast_to(kvec, (1, T, 1, dk)).copy()
+    q = np.broadcast_to(qvec, (1, T, 1, dk)).copy()
+    v = np.broadcast_to(vvec, (1, T, 1, dv)).copy()
+    g = np.zeros((1, T, 1)); beta = np.full((1, T, 1), b)
+    for chunked in (False, True):
+        o, hT = O.prefill(q, k, v, g, beta, h0=S0[None, None], chunked=chunked, chunk=5, lib=lib)
+        S = hT[0, 0]
+        expect = vvec + (1 - b) ** T * (S0 @ kvec - vvec)
+        assert np.allclose(S @ kvec, expect, atol=1e-12)
+        perp = qvec - (qvec @ kvec) * kvec
+        assert np.allclose(S @ perp, S0 @ perp, atol=1e-12)
+        # o_t after the update: o_t = S_t q with S_t k following the same closed form
+        for t in range(T):
+            skt = vvec + (1 - b) ** (t + 1) * (S0 @ kvec - vvec)
+            ot = S0 @ perp + skt * (qvec @ kvec)
+            assert np.allclose(o[t, 0], ot, atol=1e-12)
+
+
+def pin_identity_when_no_write(lib=None):
+    """alpha = 1, beta = 0: S never changes and o_t = S_0 q_t."""
+    rng = np.random.default_rng(2)
+    q, k, v, g, beta = _rand_problem(rng, 9, 2, 4, 6, 5)
+    g[:] = 0.0; beta[:] = 0.0
+    h0 = rng.standard_normal((1, 4, 5, 6))
+    for chunked in (False, True):
+        o, hT = O.prefill(q, k, v, g, beta, h0=h0, chunked=chunked, chunk=4, lib=lib)
+        assert np.allclose(hT, h0, atol=1e-13)
+        for h in range(4):
+            expect = q[0, :, h // 2, :] @ h0[0, h].T
+            assert np.allclose(o[:, h], expect, atol=1e-13)
+
+
+def pin_full_write_recalls_value(lib=None):
+    """beta = 1 with a unit key: S_t k_t = v_t exactly, whatever the decay.  dk != dv
+    so a transposed state fails; HK < HV so a wrong head map fails."""
+    rng = np.random.default_rng(3)
+    HK, HV, dk, dv, T = 2, 4, 4, 3, 7
+    q, k, v, g, beta = _rand_problem(rng, T, HK, HV, dk, dv, g_range=(-1.0, 0.0))
+    beta[:] = 1.0
+    h0 = rng.standard_normal((1, HV, dv, dk))
+    S = h0.copy()
+    for t in range(T):
+        _, S = O.step(q[:, t], k[:, t], v[:, t], g[:, t], beta[:, t], S, lib=lib)
+        for h in range(HV):
+            assert np.allclose(S[0, h] @ k[0, t, h // (HV // HK)], v[0, t, h], atol=1e-12)
+    o, hT = O.prefill(q, k, v, g, beta, h0=h0, lib=lib)
+    for h in range(HV):
+        assert np.allclose(hT[0, h] @ k[0, -1, h // (HV // HK)], v[0, -1, h], atol=1e-12)
+    assert np.allclose(hT, S, atol=1e-12)
+
+
+def pin_full_decay_resets(lib=None):
+    """alpha = 0 (g -> -inf): everything before is forgotten, S_t = b_t v_t k_t^T."""
+    rng = np.random.default_rng(4)
+    q, k, v, g, beta = _rand_problem(rng, 6, 1, 2, 5, 4)
+    g[:] = -1.0e4  # exp underflows to exactly 0
+    h0 = rng.standard_normal((1, 2, 4, 5))
+    for chunked in (False, True):
+        o, hT = O.prefill(q, k, v, g, beta, h0=h0, chunked=chunked, chunk=3, lib=lib)
+        for h in range(2):
+            S_last = beta[0, -1, h] * np.outer(v[0, -1, h], k[0, -1, 0])
+            assert np.allclose(hT[0, h], S_last, atol=1e-13)
+            for t in range(6):
+                St = beta[0, t, h] * np.outer(v[0, t, h], k[0, t, 0])
+                assert np.allclose(o[t, h], St @ q[0, t, 0], atol=1e-13)
+
+
+def pin_orthonormal_keys_store(lib=None):
+    """alpha = beta = 1 and the keys run through an orthonormal basis: after the
+    writes S e_j = v_j for each written direction (a plain associative store)."""
+    rng = np.random.default_rng(5)
+    dk, dv = 6, 5
+    # a random orthonormal basis, written in order
+    Qb, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+    keys = Qb.T
+    T = dk
+    k = keys.reshape(1, T, 1, dk)
+    q = rng.standard_normal((1, T, 1, dk))
+    v = rng.standard_normal((1, T, 1, dv))
+    g = np.zeros((1, T, 1)); beta = np.ones((1, T, 1))
+    h0 = rng.standard_normal((1, 1, dv, dk))
+    for chunked in (False, True):
+        _, hT = O.prefill(q, k, v, g, beta, h0=h0, chunked=chunked, chunk=4, lib=lib)
+        assert np.allclose(hT[0, 0] @ keys.T, v[0, :, 0].T, atol=1e-12)
+
+
+def pin_norm_bound(lib=None):
+    """For b in [0,1] and unit k, I - b k k^T has spectral norm <= 1, hence
+    ||S_t||_2 <= a_t ||S_{t-1}||_2 + b_t ||v_t||."""
+    rng = np.random.default_rng(6)
+    q, k, v, g, beta = _rand_problem(rng, 30, 1, 1, 8, 8, g_range=(-0.3, 0.0))
+    S = rng.standard_normal((1, 1, 8, 8))
+    for t in range(30):
+        prev = np.linalg.norm(S[0, 0], 2)
+        _, S = O.step(q[:, t], k[:, t], v[:, t], g[:, t], beta[:, t], S, lib=lib)
+        bound = math.exp(g[0, t, 0]) * prev + beta[0, t, 0] * np.linalg.norm(v[0, t, 0])
+        assert np.linalg.norm(S[0, 0], 2) <= bound * (1 + 1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Two independent forms must agree (brute force on tiny inputs)
+# ----------------------------------------------------------------------------
+def pin_chunked_equals_sequential(lib=None):
+    rng = np.random.default_rng(7)
+    for (T, HK, HV, dk, dv) in [(1, 1, 1, 1, 1), (13, 1, 2, 4, 4), (37, 2, 4, 8, 5),
+                                (64, 1, 2, 8, 8), (50, 2, 2, 3, 7)]:
+        q, k, v, g, beta = _rand_problem(rng, T, HK, HV, dk, dv, g_range=(-0.5, 0.0))
+        h0 = rng.standard_normal((1, HV, dv, dk))
+        o_ref, h_ref = O.prefill(q, k, v, g, beta, h0=h0, lib=lib)
+        for C in (1, 2, 3, 4, 16, max(T, 1)):
+            o, h = O.prefill(q, k, v, g, beta, h0=h0, chunked=True, chunk=C, lib=lib)
+            assert np.allclose(o, o_ref, atol=1e-11, rtol=0), (T, C, np.abs(o - o_ref).max())
+            assert np.allclose(h, h_ref, atol=1e-11, rtol=0), (T, C)
+
+
+def pin_strong_decay_no_overflow(lib=None):
+    """g = -30 on some tokens (decay e^-30): the chunked form must not overflow."""
+    rng = np.random.default_rng(8)
+    q, k, v, g, beta = _rand_problem(rng, 40, 1, 2, 6, 6)
+    g[0, ::7, :] = -30.0
+    g[0, 5, 1] = -80.0
+    o_ref, h_ref = O.prefill(q, k, v, g, beta, lib=lib)
+    o, h = O.prefill(q, k, v, g, beta, chunked=True, chunk=16, lib=lib)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(h))
+    assert np.allclose(o, o_ref, atol=1e-11) and np.allclose(h, h_ref, atol=1e-11)
+
+
+# ----------------------------------------------------------------------------
+# Structure: packing, splitting, decode, linearity, head symmetry
+# ----------------------------------------------------------------------------
+def pin_varlen_equals_separate(lib=None):
+    rng = np.random.default_rng(9)
+    lens = [5, 1, 17, 9]
+    HK, HV, dk, dv = 1, 2, 4, 3
+    parts = [_rand_problem(rng, L, HK, HV, dk, dv) for L in lens]
+    h0 = rng.standard_normal((len(lens), HV, dv, dk))
+    cat = [np.concatenate([p[i] for p in parts], axis=1) for i in range(5)]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    for chunked in (False, True):
+        o, hT = O.prefill(*cat, h0=h0, cu_seqlens=cu, chunked=chunked, chunk=4, lib=lib)
+        for n, p in enumerate(parts):
+            on, hn = O.prefill(*p, h0=h0[n:n + 1], chunked=False, lib=lib)
+            assert np.allclose(o[cu[n]:cu[n + 1]], on, atol=1e-12)
+            assert np.allclose(hT[n], hn[0], atol=1e-12)
+
+
+def pin_split_resume(lib=None):
+    """prefill(T1) then prefill(T2, h0 = hT1) equals prefill(T1 + T2)."""
+    rng = np.random.default_rng(10)
+    q, k, v, g, beta = _rand_problem(rng, 23, 2, 4, 5, 5)
+    h0 = rng.standard_normal((1, 4, 5, 5))
+    o, hT = O.prefill(q, k, v, g, beta, h0=h0, lib=lib)
+    a = [x[:, :10] for x in (q, k, v, g, beta)]
+    b = [x[:, 10:] for x in (q, k, v, g, beta)]
+    o1, h1 = O.prefill(*a, h0=h0, lib=lib)
+    o2, h2 = O.prefill(*b, h0=h1, chunked=True, chunk=4, lib=lib)
+    assert np.allclose(np.concatenate([o1, o2]), o, atol=1e-12)
+    assert np.allclose(h2, hT, atol=1e-12)
+
+
+def pin_decode_equals_prefill(lib=None):
+    rng = np.random.default_rng(11)
+    q, k, v, g, beta = _rand_problem(rng, 11, 2, 4, 6, 6)
+    h0 = rng.standard_normal((1, 4, 6, 6))
+    o, hT = O.prefill(q, k, v, g, beta, h0=h0, chunked=True, chunk=4, lib=lib)
+    S = h0
+    for t in range(11):
+        ot, S = O.step(q[:, t], k[:, t], v[:, t], g[:, t], beta[:, t], S, lib=lib)
+        assert np.allclose(ot[0], o[t], atol=1e-12)
+    assert np.allclose(S, hT, atol=1e-12)
+
+
+def pin_linear_in_values_and_state(lib=None):
+    """For fixed q, k, g, beta the map (V, h0) -> (O, hT) is linear."""
+    rng = np.random.default_rng(12)
+    q, k, v1, g, beta = _rand_problem(rng, 15, 1, 2, 4, 4)
+    v2 = rng.standard_normal(v1.shape)
+    h1 = rng.standard_normal((1, 2, 4, 4)); h2 = rng.standard_normal((1, 2, 4, 4))
+    a, b = 0.7, -1.3
+    oa, ha = O.prefill(q, k, v1, g, beta, h0=h1, lib=lib)
+    ob, hb = O.prefill(q, k, v2, g, beta, h0=h2, lib=lib)
+    oc, hc = O.prefill(q, k, a * v1 + b * v2, g, beta, h0=a * h1 + b * h2, chunked=True,
+                       chunk=4, lib=lib)
+    assert np.allclose(oc, a * oa + b * ob, atol=1e-12)
+    assert np.allclose(hc, a * ha + b * hb, atol=1e-12)
+
+
+def pin_swap_value_heads(lib=None):
+    """The two value heads of one query/key head are interchangeable."""
+    rng = np.random.default_rng(13)
+    q, k, v, g, beta = _rand_problem(rng, 12, 1, 2, 4, 4)
+    h0 = rng.standard_normal((1, 2, 4, 4))
+    o, hT = O.prefill(q, k, v, g, beta, h0=h0, lib=lib)
+    o2, h2 = O.prefill(q, k, v[:, :, ::-1], g[:, :, ::-1], beta[:, :, ::-1],
+                       h0=h0[:, ::-1], lib=lib)
+    assert np.allclose(o2, o[:, ::-1], atol=1e-13)
+    assert np.allclose(h2, hT[:, ::-1], atol=1e-13)
+
+
+def pin_scale_multiplies_readout(lib=None):
+    rng = np.random.default_rng(14)
+    q, k, v, g, beta = _rand_problem(rng, 8, 1, 1, 4, 4)
+    o1, h1 = O.prefill(q, k, v, g, beta, lib=lib)
+    o2, h2 = O.prefill(q, k, v, g, beta, scale=0.25, lib=lib)
+    assert np.allclose(o2, 0.25 * o1, atol=1e-14) and np.allclose(h2, h1, atol=1e-14)
+
+
+ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]
