@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta rule hot path on B200.
+
+Metric: "GDN prefill tokens/s (T=64K, 32 V heads); decode state HBM GB/s vs peak".
+
+One step = one chunkwise prefill (``gdn_chunk_prefill``) of a Qwen3-Next
+Gated DeltaNet layer over one synthetic sequence: B=1, T=65536, 16 query/key
+heads shared by 32 value heads, head dim 128, chunk 64, bf16 q/k/v, fp32
+g/beta/state.  The same run also measures the fused decode step
+(``gdn_recurrent_step``) on 256 sequences x 64 tokens and reports its state
+HBM bandwidth in the ``decode`` object.
+
+Launch: ``python bench.py [--gpus N --steps K --warmup W]``; for N > 1 under
+``torch.distributed.run``, one replica per GPU (each rank runs its own
+sequence; no data-path collective; ``scaling: weak``).  ``--impl reference``
+times the float64 CPU oracle on the host cores instead (the reference arm).
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s (T=64K, 32 V heads); decode state HBM GB/s vs peak"
+WORKLOAD = "long_prefill_64k"
+DECODE_WORKLOAD = "decode_256x64"
+
+# Fallback peaks (only if the measured-peaks file is absent).
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+N_SM = 148
+FP32_FMA_PER_SM_PER_CLK = 128
+
+
+def prefill_flops_per_token(HK, HV, d, C):
+    """Algorithmic FLOPs of the chunkwise form per token: per query/key head the
+    stacked [Q;K] K^T products (4 C d); per value head W, U~ and P U (6 C d) plus
+    the three state products W S^T, Q S^T and U^T K (6 d^2)."""
+    return HK * 4 * C * d + HV * (6 * C * d + 6 * d * d)
+
+
+def prefill_min_bytes_per_token(HK, HV, d, elt=2):
+    """Mandatory HBM bytes per token: read q, k, v, g, beta, write o."""
+    return 2 * HK * d * elt + 2 * HV * d * elt + 2 * HV * 4
+
+
+def decode_bytes_per_step(N, HK, HV, dk, dv, elt=2):
+    """State read + write (fp32) plus q, k, v, o, g, beta."""
+    return 2 * N * HV * dv * dk * 4 + 2 * N * HK * dk * elt + 2 * N * HV * dv * elt + 2 * N * HV * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# DRAM traffic per launch of the dominant kernels, from the ncu captures
+# summarised under profiles/ (dram__bytes_read.sum + dram__bytes_write.sum).
+# Each entry carries the sha256 of the kernel source it was taken on; a changed
+# source reports null.
+NCU_TRAFFIC = {}
+
+
+def kernel_traffic(key, units_scale=1.0):
+    e = NCU_TRAFFIC.get(key)
+    if not e:
+        return None
+    src = os.path.join(ROOT, "linear_attention_recurrence_rule_b200", "csrc", e["source"])
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if h != e["sha256"]:
+        return None
+    return e["bytes"] * units_scale
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.lines = []
+        self.device_index = device_index
+
+    def start(self):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+            sel = ["-i", "GPU-" + uuid if not uuid.startswith("GPU-") else uuid]
+        except Exception:
+            sel = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle_prefill(tokens, seed_offset=0):
+    """Seconds the float64 oracle takes on the first ``tokens`` tokens of the
+    benchmark workload (all 32 value heads), on every host core."""
+    from linear_attention_recurrence_rule_b200.inputs import workload_inputs
+    from oracle import gdn_oracle as O
+    x = workload_inputs(WORKLOAD, tokens=tokens, seed_offset=seed_offset)
+    t0 = time.perf_counter()
+    O.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], nthreads=host_cores())
+    return time.perf_counter() - t0
+
+
+def cpu_sample_tokens(target_s):
+    """Tokens of the workload the oracle processes in about ``target_s`` seconds."""
+    probe = 512
+    dt = max(time_oracle_prefill(probe), 1e-3)
+    tok = int(probe * target_s / dt)
+    return max(512, min(65536, (tok // 256) * 256))
+
+
+def cpu_baseline(target_s=12.0):
+    tok = cpu_sample_tokens(target_s)
+    dt = time_oracle_prefill(tok)
+    return {"value": tok / dt, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+            "sample": f"first {tok} of 65536 tokens of the benchmark workload, all 32 value "
+                      f"heads, float64 token-by-token recurrence, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    tok = cpu_sample_tokens(args.ref_step_seconds)
+    for i in range(args.warmup):
+        time_oracle_prefill(tok)
+    times = [time_oracle_prefill(tok) for _ in range(args.steps)]
+    total = sum(times)
+    value = tok * args.steps / total
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "B": 1, "T": 65536, "HK": 16, "HV": 32, "d": 128,
+                   "chunk": 64, "parallelism": "replicas",
+                   "sample_tokens_per_step": tok},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(),
+                         "kind": "oracle",
+                         "sample": f"first {tok} of 65536 tokens per step, all 32 value heads"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_b200(args):
+    import torch
+    import torch.distributed as dist
+
+    import linear_attention_recurrence_rule_b200 as gdn
+    from linear_attention_recurrence_rule_b200.inputs import WORKLOADS, workload_inputs
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peak_src = load_peaks()
+    w = WORKLOADS[WORKLOAD]
+    x = workload_inputs(WORKLOAD, seed_offset=rank)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    B, T = d["q"].shape[0], d["q"].shape[1]
+    tokens = B * T
+    path = gdn.gdn_chunk_prefill_path(w.dk, w.dv, w.chunk, w.dtype)
+    ws_bytes = gdn.gdn_chunk_prefill_workspace_size(B, T, w.HK, w.HV, w.dk, w.dv, w.chunk,
+                                                    w.dtype, False)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev) if ws_bytes else None
+    o = torch.empty_like(d["v"])
+    hT = torch.empty((B, w.HV, w.dv, w.dk), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 1 if path == 0 else 2
+
+    def step():
+        gdn.gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], chunk=w.chunk, o=o,
+                              hT=hT, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    elapsed_ms = max_over_ranks(elapsed_ms)
+    value = world * tokens * args.steps / (elapsed_ms / 1000.0)
+    mean_launch_s = statistics.mean(launch_ms) / 1000.0
+
+    flops = prefill_flops_per_token(w.HK, w.HV, w.dk, w.chunk) * tokens
+    if path == 1:
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": flops / mean_launch_s / 1e12, "peak": peak,
+                "unit": "TFLOP/s"}
+        kernel_key = "prefill_tc"
+    else:
+        mhz = peaks.get("sm_max_mhz", FALLBACK_PEAKS["sm_max_mhz"])
+        peak = N_SM * FP32_FMA_PER_SM_PER_CLK * 2 * mhz * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": flops / mean_launch_s / 1e12, "peak": peak,
+                "unit": "TFLOP/s"}
+        kernel_key = "prefill_simt"
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = kernel_traffic(kernel_key)
+    roof["peak_source"] = peak_src
+    roof["kernel"] = kernel_key
+
+    # ---- end to end through the public call, host buffers, copies timed ----
+    e2e = None
+    if not args.no_e2e:
+        names = ("q", "k", "v", "g", "beta")
+        host_in = {n: x[n].pin_memory() for n in names}
+        host_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        host_h = torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True)
+        h2d = sum(host_in[n].numel() * host_in[n].element_size() for n in names)
+        d2h = host_o.numel() * host_o.element_size() + host_h.numel() * host_h.element_size()
+        e_steps = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            for n in names:
+                d[n].copy_(host_in[n], non_blocking=True)
+            gdn.gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], chunk=w.chunk, o=o,
+                                  hT=hT, workspace=ws, stream=stream)
+            host_o.copy_(o, non_blocking=True)
+            host_h.copy_(hT, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = max_over_ranks(a.elapsed_time(b))
+        e2e = {"value": world * tokens * e_steps / (e_ms / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps}
+
+    # ---- decode: 256 sequences x 64 single-token steps ----
+    dec = None
+    if not args.no_decode:
+        wd = WORKLOADS[DECODE_WORKLOAD]
+        y = workload_inputs(DECODE_WORKLOAD, seed_offset=rank)
+        dy = {k: v.to(dev) for k, v in y.items()}
+        S = dy["state"].clone()
+        od = torch.empty_like(dy["v"][0])
+
+        def dstep(t):
+            gdn.gdn_recurrent_step(dy["q"][t], dy["k"][t], dy["v"][t], dy["g"][t], dy["beta"][t],
+                                   S, o=od, stream=stream)
+
+        for t in range(max(3, args.warmup)):
+            dstep(t % wd.T)
+        S.copy_(dy["state"])
+        torch.cuda.synchronize()
+        barrier()
+        dsampler = ClockSampler(local)
+        dsampler.start()
+        dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(wd.T)]
+        for t in range(wd.T):
+            dev_ev[t][0].record(stream)
+            dstep(t)
+            dev_ev[t][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        dclocks = dsampler.stop()
+        step_ms = [a_.elapsed_time(b_) for a_, b_ in dev_ev]
+        total_ms = max_over_ranks(dev_ev[0][0].elapsed_time(dev_ev[-1][1]))
+        bytes_step = decode_bytes_per_step(wd.B, wd.HK, wd.HV, wd.dk, wd.dv)
+        mean_s = statistics.mean(step_ms) / 1000.0
+        hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        achieved = bytes_step / mean_s / 1e9
+        dec = {"workload": DECODE_WORKLOAD, "value": world * bytes_step * wd.T / (total_ms / 1e3) / 1e9,
+               "unit": "GB/s", "tokens_per_s": world * wd.B * wd.T / (total_ms / 1e3),
+               "ms_per_step": total_ms / wd.T, "steps": wd.T,
+               "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak,
+                            "unit": "GB/s", "frac": achieved / hbm_peak,
+                            "traffic": kernel_traffic("decode"), "peak_source": peak_src,
+                            "kernel": "decode"},
+               "bytes_per_step": bytes_step, "gpu_launches": wd.T, "clocks": dclocks,
+               "l2": "state 537 MB per step, larger than L2"}
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": 1, "T": 65536, "HK": 16, "HV": 32, "d": 128,
+                       "chunk": 64, "parallelism": "replicas" if world > 1 else "single",
+                       "path": "tcgen05" if path == 1 else "cuda-core",
+                       "l2": "inputs larger than L2 (q,k,v 1.07 GB per step)"},
+            "roofline": roof, "cpu_baseline": base, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "decode": dec,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_b200(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,157 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) gated delta rule library.
+ *
+ * The operation (sources: "Qwen3-Next", sghael.github.io, section "Correcting
+ * a memory instead of adding to it"; model card "Qwen3-Next-80B-A3B-Instruct",
+ * section "Model Overview", Gated DeltaNet heads; "The Evolving Transformer /
+ * Qwen3-Next", section 01 GatedDeltaNet, for the state orientation and the
+ * read-out after the update):
+ *
+ *   For every sequence n and value head h (reading query/key head
+ *   c = floor(h / (HV / HK))), with S a dv x dk fp32 matrix (row = value
+ *   index, column = key index) starting at h0[n][h] (or zero):
+ *
+ *     S_t = alpha_t * S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = scale * S_t q_t            alpha_t = exp(g_t)
+ *
+ *   i.e. the old memory is first shrunk by the decay, then corrected along the
+ *   current key by the write strength beta_t (the page's scalar example:
+ *   6 -> 3 -> 3 + 0.5 * (10 - 3) = 6.5).  q and k are expected to be
+ *   L2-normalised by the caller; the library does not renormalise.
+ *
+ * Conventions shared by every call
+ *   - All pointers are DEVICE pointers of the current CUDA device unless a
+ *     comment says otherwise.  The caller owns every buffer; the library keeps
+ *     no allocation and no global state, never synchronises the stream, and
+ *     returns as soon as the work is enqueued on `stream`.
+ *   - Tensors are dense, row-major, with the last dimension contiguous.
+ *   - dtype selects the element type of q, k, v and o: GDN_F32 (float) or
+ *     GDN_BF16 (__nv_bfloat16).  g, beta, h0, hT and the decode state are
+ *     always fp32.  Internal accumulation and the recurrent state are fp32.
+ *   - Host-checkable problems (NULL where a buffer is required, HV % HK != 0,
+ *     an unsupported shape/dtype/chunk combination, a misaligned base pointer,
+ *     a short workspace) return an error before anything is enqueued.  A failed
+ *     kernel launch returns GDN_ERR_CUDA.  There is no fallback to another
+ *     implementation or to the CPU.
+ *   - The contents of cu_seqlens are a precondition (see below) and are not
+ *     checked on the host.
+ */
+#ifndef GDN_B200_H
+#define GDN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t.  NULL selects the legacy default stream. */
+typedef struct CUstream_st *gdn_stream_t;
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,   /* NULL buffer, non-positive size, HV % HK != 0 ... */
+    GDN_ERR_UNSUPPORTED = 2,   /* valid but not implemented: head dim, chunk, dtype */
+    GDN_ERR_ALIGNMENT = 3,     /* a base pointer is not 16-byte aligned            */
+    GDN_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed       */
+    GDN_ERR_TIMEOUT = 5,       /* a bounded on-device wait gave up (reported through
+                                  the workspace status word, see gdn_read_status)   */
+    GDN_ERR_WORKSPACE = 6      /* workspace missing or smaller than required        */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Short English description of a status code (static storage, never NULL). */
+GDN_API const char *gdn_status_string(gdn_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+GDN_API int gdn_version(void);
+
+/*
+ * Bytes of device workspace gdn_chunk_prefill needs for this problem.
+ * N: number of sequences; T: tokens per sequence without cu_seqlens, else the
+ * packed total; varlen: nonzero when cu_seqlens will be passed.  Returns 0 for
+ * arguments gdn_chunk_prefill would reject.
+ */
+GDN_API size_t gdn_chunk_prefill_workspace_size(int N, int64_t T, int HK, int HV, int dk, int dv,
+                                        int chunk, gdn_dtype dtype, int varlen);
+
+/*
+ * 1 when gdn_chunk_prefill runs this (head dims, chunk, dtype) combination on
+ * the tcgen05 tensor-core path, 0 when it runs on the CUDA-core path, -1 when
+ * the combination is unsupported.  Pure host query.
+ */
+GDN_API int gdn_chunk_prefill_path(int dk, int dv, int chunk, gdn_dtype dtype);
+
+/*
+ * Chunkwise prefill: runs the rule over whole sequences.
+ *
+ * The sequence is cut into chunks of `chunk` tokens (the last one may be
+ * short; chunks restart at every sequence start).  Within a chunk the tokens
+ * are processed in the WY/UT form derived from the recurrence: a chunk-local
+ * running sum G of g, the unit-lower-triangular system (I + A) with
+ * A_ij = beta_i exp(G_i - G_j) k_i.k_j (j < i), intra-chunk products on the
+ * tensor cores, and a sequential pass over chunks that carries the fp32 state.
+ * The result equals the token-by-token recurrence up to rounding.
+ *
+ * Layouts (B = N without cu_seqlens; with cu_seqlens everything is packed as a
+ * single batch row of Ttot = T tokens):
+ *   q, k   [B][T][HK][dk]  dtype          v, o   [B][T][HV][dv]  dtype
+ *   g      [B][T][HV] fp32 (log decay, g <= 0 expected; alpha = exp(g))
+ *   beta   [B][T][HV] fp32 (write strength, expected in [0, 1])
+ *   h0     [N][HV][dv][dk] fp32, or NULL for a zero start state
+ *   hT     [N][HV][dv][dk] fp32 final states, or NULL to skip; may alias h0
+ *   cu_seqlens  NULL, or N+1 int32 device offsets with cu_seqlens[0] = 0,
+ *               non-decreasing, cu_seqlens[N] = T (precondition, unchecked)
+ * Supported: HV % HK == 0; dtype GDN_BF16 or GDN_F32; dk, dv in {32, 64, 128};
+ * chunk in {16, 32, 64}.  (bf16, dk = dv = 128, chunk = 64 runs on the
+ * tcgen05 tensor-core path; other combinations run on the CUDA-core path.)
+ * Alignment: q, k, v, o, h0, hT must be 16-byte aligned.
+ * workspace: device buffer of at least gdn_chunk_prefill_workspace_size(...)
+ * bytes (may be NULL when that size is 0); its contents need no initialisation
+ * and are scratch after the call.  Calls that share a workspace must be
+ * ordered on the device (same stream or synchronised).
+ */
+GDN_API gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *h0, const int32_t *cu_seqlens,
+                             int N, int64_t T, int HK, int HV, int dk, int dv, int chunk,
+                             float scale, gdn_dtype dtype, void *o, float *hT,
+                             void *workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * Fused single-token decode step for N independent sequences: applies one
+ * token of the rule to each sequence's state in place and writes its output.
+ * Every state element is read once and written once (one pass through HBM).
+ *
+ * Layouts:
+ *   q, k   [N][HK][dk] dtype      v, o [N][HV][dv] dtype
+ *   g, beta [N][HV] fp32          state [N][HV][dv][dk] fp32, updated in place
+ * Supported: HV % HK == 0; dtype GDN_BF16 or GDN_F32; dk in {32, 64, 128};
+ * 1 <= dv <= 256.  Alignment: q, k, v, o, state 16-byte aligned.
+ * o must not overlap state.
+ */
+GDN_API gdn_status gdn_recurrent_step(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, float *state, int N, int HK, int HV, int dk,
+                              int dv, float scale, gdn_dtype dtype, void *o,
+                              gdn_stream_t stream);
+
+/*
+ * Reads the device status word a prefill call left in its workspace (HOST
+ * call; synchronises `stream`).  Returns GDN_OK when every on-device wait of
+ * the last call on this workspace completed, GDN_ERR_TIMEOUT when one gave up
+ * (the outputs of that call are then undefined), or GDN_ERR_CUDA.
+ */
+GDN_API gdn_status gdn_read_status(const void *workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_B200_H */

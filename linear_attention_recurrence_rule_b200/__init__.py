@@ -1,0 +1,13 @@
+"""Gated delta rule (Gated DeltaNet core) for NVIDIA B200, sm_100a.
+
+The computation lives in the CUDA library built from ``csrc/`` (C ABI in
+``include/gdn.h``); this package is its thin Python binding plus the seeded
+synthetic input generator used by the tests and the benchmark.
+"""
+from .gdn import (GDN_BF16, GDN_F32, GDNError, gdn_chunk_prefill,  # noqa: F401
+                  gdn_chunk_prefill_path, gdn_chunk_prefill_workspace_size, gdn_read_status, gdn_recurrent_step,
+                  lib_path, load_library, status_string)
+
+__all__ = ["gdn_chunk_prefill", "gdn_recurrent_step", "gdn_chunk_prefill_workspace_size", "gdn_chunk_prefill_path",
+           "gdn_read_status", "status_string", "load_library", "lib_path", "GDNError",
+           "GDN_F32", "GDN_BF16"]

@@ -1,0 +1,126 @@
+// Fused single-token decode step of the gated delta rule.
+//
+// Rule ("Qwen3-Next", sghael.github.io, section "Correcting a memory instead of
+// adding to it": decay first, then correct along the current key; read-out
+// after the update as in "The Evolving Transformer / Qwen3-Next", section 01):
+//
+//   per row i of the dv x dk state S (row = value index):
+//     sk_i = S_i . k          sq_i = S_i . q          (old state)
+//     u_i  = beta * (v_i - alpha * sk_i)
+//     S_i <- alpha * S_i + u_i * k
+//     o_i  = scale * (alpha * sq_i + u_i * (k . q))   (= scale * S_i(new) . q)
+//
+// Every row is independent, so the kernel is a single streaming pass over the
+// fp32 state: each state element is loaded once (128-bit, evict-first) and
+// stored once (128-bit, streaming).  The two dot products of a row are reduced
+// with warp shuffles inside the lanes that hold the row.
+//
+// Work split: one CTA of 8 warps per (sequence, value head).  A row of dk fp32
+// is held by dk/4 lanes (one float4 each); a warp instruction covers 32/(dk/4)
+// rows; each warp issues NB such loads before using any of them, so every lane
+// has NB x 16 B of state in flight.
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int kDecodeWarps = 8;
+constexpr int kDecodeNB = 16;
+
+template <int DK, typename Tin>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+              const float *__restrict__ g, const float *__restrict__ beta, float *state,
+              Tin *__restrict__ o, int HK, int HV, int dv, float scale) {
+    constexpr int LPR = DK / 4;    // lanes per state row
+    constexpr int RPI = 32 / LPR;  // rows per warp instruction
+    const int nh = blockIdx.x;     // n * HV + h
+    const int n = nh / HV, h = nh - n * HV;
+    const int c = h / (HV / HK);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / LPR;
+    const int col = (lane % LPR) * 4;
+
+    const float4 kk = load4(k + ((size_t)n * HK + c) * DK + col);
+    const float4 qq = load4(q + ((size_t)n * HK + c) * DK + col);
+    float kq = dot4(kk, qq);
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    const float alpha = expf(g[nh]);
+    const float b = beta[nh];
+    const Tin *vrow = v + (size_t)nh * dv;
+    Tin *orow = o + (size_t)nh * dv;
+    float *S = state + (size_t)nh * dv * DK;
+
+    constexpr int rows_per_batch = kDecodeWarps * RPI * kDecodeNB;
+    for (int base = 0; base < dv; base += rows_per_batch) {
+        float4 s[kDecodeNB];
+#pragma unroll
+        for (int j = 0; j < kDecodeNB; ++j) {
+            const int row = base + (j * kDecodeWarps + warp) * RPI + sub;
+            s[j] = row < dv ? __ldcs(reinterpret_cast<const float4 *>(S + (size_t)row * DK + col))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < kDecodeNB; ++j) {
+            const int row = base + (j * kDecodeWarps + warp) * RPI + sub;
+            float sk = dot4(s[j], kk), sq = dot4(s[j], qq);
+#pragma unroll
+            for (int off = LPR / 2; off > 0; off >>= 1) {
+                sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            }
+            if (row < dv) {
+                const float u = b * (to_f32(vrow[row]) - alpha * sk);
+                float4 ns;
+                ns.x = fmaf(alpha, s[j].x, u * kk.x);
+                ns.y = fmaf(alpha, s[j].y, u * kk.y);
+                ns.z = fmaf(alpha, s[j].z, u * kk.z);
+                ns.w = fmaf(alpha, s[j].w, u * kk.w);
+                __stcs(reinterpret_cast<float4 *>(S + (size_t)row * DK + col), ns);
+                if ((lane % LPR) == 0) orow[row] = from_f32<Tin>(scale * fmaf(alpha, sq, u * kq));
+            }
+        }
+    }
+}
+
+template <typename Tin>
+cudaError_t launch_typed(const StepArgs &a, cudaStream_t stream) {
+    const dim3 grid((unsigned)((size_t)a.N * a.HV)), block(kDecodeWarps * 32);
+    const Tin *q = static_cast<const Tin *>(a.q);
+    const Tin *k = static_cast<const Tin *>(a.k);
+    const Tin *v = static_cast<const Tin *>(a.v);
+    Tin *o = static_cast<Tin *>(a.o);
+    switch (a.dk) {
+        case 32:
+            decode_kernel<32, Tin><<<grid, block, 0, stream>>>(q, k, v, a.g, a.beta, a.state, o,
+                                                               a.HK, a.HV, a.dv, a.scale);
+            break;
+        case 64:
+            decode_kernel<64, Tin><<<grid, block, 0, stream>>>(q, k, v, a.g, a.beta, a.state, o,
+                                                               a.HK, a.HV, a.dv, a.scale);
+            break;
+        case 128:
+            decode_kernel<128, Tin><<<grid, block, 0, stream>>>(q, k, v, a.g, a.beta, a.state, o,
+                                                                a.HK, a.HV, a.dv, a.scale);
+            break;
+        default:
+            return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_supported(int dk, int dv) {
+    return (dk == 32 || dk == 64 || dk == 128) && dv >= 1 && dv <= 256;
+}
+
+cudaError_t launch_decode(const StepArgs &a, cudaStream_t stream) {
+    if (a.N == 0) return cudaSuccess;
+    return a.dtype == GDN_BF16 ? launch_typed<__nv_bfloat16>(a, stream)
+                               : launch_typed<float>(a, stream);
+}
+
+}  // namespace gdn

@@ -1,0 +1,50 @@
+// Internal launch interface between the C ABI (gdn_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+struct PrefillArgs {
+    const void *q, *k, *v;
+    const float *g, *beta, *h0;
+    const int32_t *cu_seqlens;
+    int N;
+    int64_t T;       // tokens per sequence (no cu_seqlens) or packed total
+    int HK, HV, dk, dv, chunk;
+    float scale;
+    gdn_dtype dtype;
+    void *o;
+    float *hT;
+    void *workspace;
+    size_t workspace_bytes;
+};
+
+struct StepArgs {
+    const void *q, *k, *v;
+    const float *g, *beta;
+    float *state;
+    int N, HK, HV, dk, dv;
+    float scale;
+    gdn_dtype dtype;
+    void *o;
+};
+
+// decode (gdn_decode.cu)
+bool decode_supported(int dk, int dv);
+cudaError_t launch_decode(const StepArgs &a, cudaStream_t stream);
+
+// CUDA-core chunked prefill (gdn_prefill_simt.cu)
+bool prefill_simt_supported(int dk, int dv, int chunk);
+cudaError_t launch_prefill_simt(const PrefillArgs &a, cudaStream_t stream);
+
+// tcgen05 / TMEM / TMA tensor-core prefill (gdn_prefill_tc.cu)
+bool prefill_tc_supported(int dk, int dv, int chunk, gdn_dtype dtype);
+size_t prefill_tc_workspace(int N, int64_t T, int HV, int chunk, bool varlen);
+cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream);
+
+}  // namespace gdn

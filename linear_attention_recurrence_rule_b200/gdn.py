@@ -1,0 +1,206 @@
+"""Thin Python binding of the C ABI in ``include/gdn.h`` (argument marshalling only).
+
+Every step of the computation runs in the CUDA library ``libgdn_b200.so``; this
+module turns torch tensors into device pointers, passes the current CUDA stream
+and raises on a non-OK status.  PyTorch is used for device memory and streams
+only.  If the library is missing, every call raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import _build
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_ALIGNMENT, GDN_ERR_CUDA, \
+    GDN_ERR_TIMEOUT, GDN_ERR_WORKSPACE = range(7)
+GDN_F32, GDN_BF16 = 0, 1
+
+_lock = threading.Lock()
+_handle = None
+
+
+class GDNError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def load_library() -> ctypes.CDLL:
+    """Load ``libgdn_b200.so`` (raises if it has not been built)."""
+    global _handle
+    with _lock:
+        if _handle is None:
+            if not os.path.exists(_build.LIB):
+                raise RuntimeError(
+                    f"CUDA library {_build.LIB} is not built; run "
+                    "`python -c 'import __graft_entry__ as g; g.build()'` first")
+            lib = ctypes.CDLL(_build.LIB)
+            vp, sz, i64, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int
+            lib.gdn_status_string.restype = ctypes.c_char_p
+            lib.gdn_status_string.argtypes = [i32]
+            lib.gdn_version.restype = i32
+            lib.gdn_version.argtypes = []
+            lib.gdn_chunk_prefill_workspace_size.restype = sz
+            lib.gdn_chunk_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32,
+                                                             i32, i32]
+            lib.gdn_chunk_prefill.restype = i32
+            lib.gdn_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+                                              i32, i32, ctypes.c_float, i32, vp, vp, vp, sz, vp]
+            lib.gdn_recurrent_step.restype = i32
+            lib.gdn_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                               ctypes.c_float, i32, vp, vp]
+            lib.gdn_chunk_prefill_path.restype = i32
+            lib.gdn_chunk_prefill_path.argtypes = [i32, i32, i32, i32]
+            lib.gdn_read_status.restype = i32
+            lib.gdn_read_status.argtypes = [vp, sz, vp]
+            _handle = lib
+    return _handle
+
+
+def status_string(status: int) -> str:
+    return load_library().gdn_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def gdn_chunk_prefill_workspace_size(N, T, HK, HV, dk, dv, chunk, dtype, varlen) -> int:
+    code = dtype if isinstance(dtype, int) else _dtype_code(torch.empty(0, dtype=dtype))
+    return int(load_library().gdn_chunk_prefill_workspace_size(
+        int(N), int(T), int(HK), int(HV), int(dk), int(dv), int(chunk), code, int(bool(varlen))))
+
+
+def gdn_chunk_prefill(q, k, v, g, beta, h0=None, cu_seqlens=None, chunk: int = 64,
+                      scale: float = 1.0, o=None, hT=None, workspace=None, stream=None,
+                      output_final_state: bool = True):
+    """Chunkwise prefill through ``gdn_chunk_prefill``.
+
+    q, k [B,T,HK,dk]; v [B,T,HV,dv] (bf16 or fp32); g, beta [B,T,HV] fp32;
+    h0 [N,HV,dv,dk] fp32 or None; cu_seqlens int32 [N+1] (then B == 1) or None.
+    Returns (o [B,T,HV,dv], hT [N,HV,dv,dk] or None).
+    """
+    lib = load_library()
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("expected q,k [B,T,HK,dk] and v [B,T,HV,dv]")
+    B, T, HK, dk = q.shape
+    HV, dv = v.shape[2], v.shape[3]
+    if g.shape != (B, T, HV) or beta.shape != (B, T, HV):
+        raise ValueError("expected g, beta [B,T,HV]")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        if B != 1:
+            raise ValueError("with cu_seqlens the batch dimension must be 1 (packed)")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, dev)
+        if h0.shape != (N, HV, dv, dk):
+            raise ValueError(f"h0 must be [N,HV,dv,dk] = {(N, HV, dv, dk)}")
+    if o is None:
+        o = torch.empty_like(v)
+    else:
+        _need(o, "o", v.dtype, dev)
+    if hT is None and output_final_state:
+        hT = torch.empty((N, HV, dv, dk), dtype=torch.float32, device=dev)
+    elif hT is not None:
+        _need(hT, "hT", torch.float32, dev)
+    code = _dtype_code(q)
+    need = lib.gdn_chunk_prefill_workspace_size(N, T, HK, HV, dk, dv, chunk, code,
+                                                int(cu_seqlens is not None))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.gdn_chunk_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                               _ptr(cu_seqlens), N, T, HK, HV, dk, dv, int(chunk),
+                               float(scale), code, _ptr(o), _ptr(hT), _ptr(workspace),
+                               ws_bytes, _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_chunk_prefill")
+    return o, hT
+
+
+def gdn_recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, o=None, stream=None):
+    """One fused decode token through ``gdn_recurrent_step``; ``state`` is updated in place.
+
+    q, k [N,HK,dk]; v [N,HV,dv] (bf16 or fp32); g, beta [N,HV] fp32;
+    state [N,HV,dv,dk] fp32.  Returns o [N,HV,dv].
+    """
+    lib = load_library()
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(state, "state", torch.float32, dev)
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[0] != q.shape[0]:
+        raise ValueError("expected q,k [N,HK,dk] and v [N,HV,dv]")
+    N, HK, dk = q.shape
+    HV, dv = v.shape[1], v.shape[2]
+    if g.shape != (N, HV) or beta.shape != (N, HV) or state.shape != (N, HV, dv, dk):
+        raise ValueError("expected g,beta [N,HV] and state [N,HV,dv,dk]")
+    if o is None:
+        o = torch.empty_like(v)
+    else:
+        _need(o, "o", v.dtype, dev)
+    st = lib.gdn_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                                N, HK, HV, dk, dv, float(scale), _dtype_code(q), _ptr(o),
+                                _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_recurrent_step")
+    return o
+
+
+def gdn_chunk_prefill_path(dk, dv, chunk, dtype) -> int:
+    """1 = tcgen05 tensor-core path, 0 = CUDA-core path, -1 = unsupported."""
+    code = dtype if isinstance(dtype, int) else _dtype_code(torch.empty(0, dtype=dtype))
+    return int(load_library().gdn_chunk_prefill_path(int(dk), int(dv), int(chunk), code))
+
+
+def gdn_read_status(workspace, stream=None) -> int:
+    """Status word of the last prefill on ``workspace`` (synchronises the stream)."""
+    if workspace is None:
+        return GDN_OK
+    return int(load_library().gdn_read_status(
+        _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream_ptr(stream, workspace.device)))

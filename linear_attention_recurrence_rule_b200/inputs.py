@@ -123,9 +123,15 @@ def make_decode(N: int, steps: int, HK: int, HV: int, dk: int, dv: int, dtype=to
     return dict(q=q, k=k, v=v, g=g, beta=beta, state=state)
 
 
-def workload_inputs(name: str, steps: int | None = None):
-    """Inputs for one named workload (see ``WORKLOADS``)."""
+def workload_inputs(name: str, steps: int | None = None, seed_offset: int = 0,
+                    tokens: int | None = None):
+    """Inputs for one named workload (see ``WORKLOADS``).  ``seed_offset`` gives
+    another draw of the same workload (one per replica); ``tokens`` truncates a
+    single-sequence prefill workload to its first ``tokens`` tokens."""
     w = WORKLOADS[name]
+    if seed_offset:
+        from dataclasses import replace
+        w = replace(w, seed=w.seed + 7919 * seed_offset)
     if w.kind == "decode":
         return make_decode(w.B, steps or w.T, w.HK, w.HV, w.dk, w.dv, w.dtype, w.seed, w.h0_std)
     if w.varlen:
@@ -134,7 +140,8 @@ def workload_inputs(name: str, steps: int | None = None):
         lengths = draw_lengths(gen, n, lo, hi)
         return make_prefill(w.HK, w.HV, w.dk, w.dv, lengths, w.dtype, seed=w.seed + 1000,
                             h0_std=w.h0_std, packed=True)
-    return make_prefill(w.HK, w.HV, w.dk, w.dv, [w.T] * w.B, w.dtype, seed=w.seed,
+    T = w.T if tokens is None else min(int(tokens), w.T)
+    return make_prefill(w.HK, w.HV, w.dk, w.dv, [T] * w.B, w.dtype, seed=w.seed,
                         h0_std=w.h0_std)
 
 

@@ -1,0 +1,110 @@
+"""The C-ABI library loads, exports every symbol include/gdn.h declares, and its
+host-side validation rejects bad arguments before anything reaches a GPU.
+(No compute call is made here: every call below fails validation first.)"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_recurrence_rule_b200 import _build, gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return gdn.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]*?\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_two_calls():
+    syms = declared_symbols()
+    assert "gdn_chunk_prefill" in syms and "gdn_recurrent_step" in syms
+    assert "gdn_chunk_prefill_workspace_size" in syms and "gdn_status_string" in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    handle = ctypes.CDLL(gdn.lib_path())
+    for name in declared_symbols():
+        assert hasattr(handle, name), f"{name} declared in gdn.h but not exported"
+
+
+def test_library_is_sm100a_only():
+    # the build command pins the one target architecture
+    assert _build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = gdn.status_string(code)
+        assert isinstance(s, str) and s
+    assert gdn.status_string(0) == "ok"
+    assert lib.gdn_version() >= 100
+
+
+P = ctypes.c_void_p
+
+
+def fake(addr):
+    return P(addr)  # never dereferenced: validation fails before any launch
+
+
+def prefill_call(lib, **kw):
+    a = dict(q=fake(0x1000), k=fake(0x2000), v=fake(0x3000), g=fake(0x4000), beta=fake(0x5000),
+             h0=None, cu=None, N=1, T=64, HK=1, HV=2, dk=32, dv=32, chunk=16, scale=1.0,
+             dtype=gdn.GDN_F32, o=fake(0x6000), hT=None, ws=None, ws_bytes=0)
+    a.update(kw)
+    return lib.gdn_chunk_prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], a["h0"], a["cu"],
+                                 a["N"], a["T"], a["HK"], a["HV"], a["dk"], a["dv"], a["chunk"],
+                                 a["scale"], a["dtype"], a["o"], a["hT"], a["ws"], a["ws_bytes"],
+                                 None)
+
+
+def test_prefill_validation(lib):
+    assert prefill_call(lib, q=None) == gdn.GDN_ERR_INVALID_ARG
+    assert prefill_call(lib, o=None) == gdn.GDN_ERR_INVALID_ARG
+    assert prefill_call(lib, HV=3, HK=2) == gdn.GDN_ERR_INVALID_ARG
+    assert prefill_call(lib, N=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert prefill_call(lib, dtype=7) == gdn.GDN_ERR_INVALID_ARG
+    assert prefill_call(lib, dk=48) == gdn.GDN_ERR_UNSUPPORTED
+    assert prefill_call(lib, chunk=48) == gdn.GDN_ERR_UNSUPPORTED
+    assert prefill_call(lib, dv=256) == gdn.GDN_ERR_UNSUPPORTED
+    assert prefill_call(lib, q=fake(0x1004)) == gdn.GDN_ERR_ALIGNMENT
+    assert prefill_call(lib, hT=fake(0x7008)) == gdn.GDN_ERR_ALIGNMENT
+    # N == 0 is a valid empty problem: nothing is launched
+    assert prefill_call(lib, N=0) == gdn.GDN_OK
+
+
+def step_call(lib, **kw):
+    a = dict(q=fake(0x1000), k=fake(0x2000), v=fake(0x3000), g=fake(0x4000), beta=fake(0x5000),
+             state=fake(0x6000), N=2, HK=1, HV=2, dk=128, dv=128, scale=1.0,
+             dtype=gdn.GDN_BF16, o=fake(0x7000))
+    a.update(kw)
+    return lib.gdn_recurrent_step(a["q"], a["k"], a["v"], a["g"], a["beta"], a["state"], a["N"],
+                                  a["HK"], a["HV"], a["dk"], a["dv"], a["scale"], a["dtype"],
+                                  a["o"], None)
+
+
+def test_step_validation(lib):
+    assert step_call(lib, state=None) == gdn.GDN_ERR_INVALID_ARG
+    assert step_call(lib, HK=3) == gdn.GDN_ERR_INVALID_ARG
+    assert step_call(lib, dk=100) == gdn.GDN_ERR_UNSUPPORTED
+    assert step_call(lib, dv=300) == gdn.GDN_ERR_UNSUPPORTED
+    assert step_call(lib, state=fake(0x6004)) == gdn.GDN_ERR_ALIGNMENT
+    assert step_call(lib, N=0) == gdn.GDN_OK
+
+
+def test_workspace_size_rejects_bad_shapes(lib):
+    assert gdn.gdn_chunk_prefill_workspace_size(1, 64, 2, 3, 128, 128, 64, gdn.GDN_BF16, 0) == 0
+    assert gdn.gdn_chunk_prefill_workspace_size(-1, 64, 1, 2, 128, 128, 64, gdn.GDN_BF16, 0) == 0
+
+
+def test_read_status_without_workspace(lib):
+    assert lib.gdn_read_status(None, 0, None) == gdn.GDN_OK

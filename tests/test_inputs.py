@@ -1,0 +1,50 @@
+"""The seeded input generator: deterministic, the shapes and distributions the
+workloads state (CPU only)."""
+import math
+
+import torch
+
+from linear_attention_recurrence_rule_b200.inputs import (WORKLOADS, make_decode, make_prefill,
+                                                          varlen_lengths, workload_inputs)
+
+
+def test_deterministic():
+    a = make_prefill(2, 4, 16, 16, [33, 33], torch.bfloat16, seed=5)
+    b = make_prefill(2, 4, 16, 16, [33, 33], torch.bfloat16, seed=5)
+    for k in ("q", "k", "v", "g", "beta"):
+        assert torch.equal(a[k], b[k])
+
+
+def test_distributions():
+    x = make_prefill(4, 8, 128, 128, [2048], torch.float32, seed=1)
+    assert torch.allclose(x["q"].norm(dim=-1), torch.ones(1), atol=1e-5)
+    assert torch.allclose(x["k"].norm(dim=-1), torch.ones(1), atol=1e-5)
+    alpha = x["g"].exp()
+    assert alpha.min() >= 0.9 - 1e-6 and alpha.max() <= 1.0
+    assert x["beta"].min() > 0 and x["beta"].max() < 1
+    assert abs(float(x["v"].std()) - 1.0) < 0.02
+    assert x["h0"] is None and x["cu_seqlens"] is None
+
+
+def test_workload_shapes():
+    assert (WORKLOADS["long_prefill_64k"].T, WORKLOADS["long_prefill_64k"].HV) == (65536, 32)
+    w = WORKLOADS["layer_prefill_4k"]
+    assert (w.HK, w.HV, w.dk, w.dv, w.chunk) == (16, 32, 128, 128, 64)
+    x = workload_inputs("tiny_fp32")
+    assert x["q"].shape == (1, 128, 1, 32) and x["v"].shape == (1, 128, 2, 32)
+    assert x["q"].dtype == torch.float32
+
+
+def test_varlen_lengths_and_packing():
+    lens = varlen_lengths()
+    assert len(lens) == 8 and all(1024 <= L <= 32768 for L in lens)
+    x = make_prefill(1, 2, 8, 8, [3, 0, 5], torch.bfloat16, seed=2, h0_std=0.02, packed=True)
+    assert x["cu_seqlens"].tolist() == [0, 3, 3, 8]
+    assert x["q"].shape == (1, 8, 1, 8) and x["h0"].shape == (3, 2, 8, 8)
+
+
+def test_decode_inputs():
+    x = make_decode(3, 4, 2, 4, 16, 8, torch.bfloat16, seed=1)
+    assert x["q"].shape == (4, 3, 2, 16) and x["v"].shape == (4, 3, 4, 8)
+    assert x["state"].shape == (3, 4, 8, 16) and x["state"].dtype == torch.float32
+    assert math.isclose(float(x["state"].std()), 0.02, rel_tol=0.2)
