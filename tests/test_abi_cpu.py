@@ -2,6 +2,7 @@
 host-side validation rejects bad arguments before anything reaches a GPU.
 (No compute call is made here: every call below fails validation first.)"""
 import ctypes
+import glob
 import os
 import re
 
@@ -10,7 +11,7 @@ import pytest
 from linear_attention_recurrence_rule_b200 import _build, gdn
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "gdn.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 @pytest.fixture(scope="module")
@@ -20,7 +21,7 @@ def lib():
 
 
 def declared_symbols():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]*?\b(gdn_\w+)\s*\(", text)))
 
 
@@ -28,6 +29,7 @@ def test_header_declares_the_two_calls():
     syms = declared_symbols()
     assert "gdn_chunk_prefill" in syms and "gdn_recurrent_step" in syms
     assert "gdn_chunk_prefill_workspace_size" in syms and "gdn_status_string" in syms
+    assert "gdn_selftest_umma" in syms
 
 
 def test_library_exports_every_declared_symbol(lib):
