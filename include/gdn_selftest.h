@@ -22,13 +22,14 @@ extern "C" {
  * Outputs (row-major fp32):
  *   D1 [128][64]  = X Y^T          D2 [128][64] = Z^T R^T
  *   D3 [128][128] = U Z            D4 [128][64] = D0 - S W
+ *   D5 [128][128] = U Z with U read from tensor memory (A operand in TMEM)
  * status (device int) is set to GDN_ERR_TIMEOUT if an on-device wait gave up.
  * X, Y, Z must be 16-byte aligned.  Returns a gdn_status; asynchronous.
  */
 GDN_API int gdn_selftest_umma(const void *X, const void *Y, const void *Z, const void *R,
                               const void *U, const void *S, const void *W, const float *D0,
-                              float *D1, float *D2, float *D3, float *D4, int *status,
-                              gdn_stream_t stream);
+                              float *D1, float *D2, float *D3, float *D4, float *D5,
+                              int *status, gdn_stream_t stream);
 
 #ifdef __cplusplus
 }

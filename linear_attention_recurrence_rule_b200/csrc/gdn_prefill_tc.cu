@@ -21,24 +21,34 @@
 //   X  : D1[128x64]  = [Q;K] K^T            -> rows 0..63: Q K^T, 64..127: K K^T
 //   Wt : DW[a][t]    = sum_s K[s][a] T'[t][s],  T' = T diag(b gamma)
 //   Ut : DU[i][t]    = sum_s V[s][i] T''[t][s], T'' = T diag(b)
-//   O1 : DQ[i][t]    = sum_a S0[i][a] q_t[a]
 //   M1 : DU[i][t]   -= sum_a S0[i][a] W[t][a]   (negated A, accumulate)
-//   M3 : DO[i][t]    = sum_s U[i][s] P[t][s]
-//   M4 : DS[i][a]    = sum_s (U[i][s] gamma_L/gamma_s) K[s][a]
-// with o_t = scale (gamma_t DQ[:, t] + DO[:, t]).
-// and S(fp32, TMEM) = gamma_L S + DS.  q/k/v tiles arrive by TMA (128B
-// swizzle); operands produced on chip are written by threads in the same
-// swizzled layout.  One CTA per (sequence, value head) walks its chunks in
-// order, prefetching the next chunk's tiles while it computes the current one.
-// The UT inverse runs on CUDA cores (column-wise forward substitution).
+//   O1 : DQ[i][t]    = sum_a S0[i][a] q_t[a]
+//   M4 : S[i][a]    += sum_s (U[i][s] gamma_L/gamma_s) K[s][a]   (U from TMEM)
+//   M3 : DO[i][t]    = sum_s U[i][s] P[t][s]                     (U from TMEM)
+// with o_t = scale (gamma_t DQ[:, t] + DO[:, t]).  The fp32 state S lives in
+// tensor memory; before M4 of a chunk it is scaled in place by gamma_L, so M4
+// accumulates the chunk's update straight into it.
+//
+// Work split: one CTA per (sequence, value head); its warps specialise and
+// run the state-independent preparation of chunk c+1 while the sequential
+// chain processes chunk c:
+//   warp 0        TMA producer: q/k tiles (2-stage ring) and the v tile
+//   warp 1        MMA issuer: the warp computes descriptors, one elected lane
+//                 issues every MMA and commit, in dependency order
+//   warps 2..9    chain: U (hi/lo into TMEM), the bf16 copy of S for the
+//                 next chunk, the gamma_L scaling of S, outputs
+//   warps 10..17  prep: A and P from [Q;K]K^T, the UT inverse T (blocked
+//                 16 -> 32 -> 64 on CUDA cores), T', T'' tiles, W
+// Two warps share each TMEM lane quadrant, each taking half of a row's columns.
+// Stages hand over through mbarriers; every wait is bounded and a timeout
+// winds the CTA down and reports GDN_ERR_TIMEOUT in the workspace status word.
 //
 // Precision: q, k, v are exact bf16 operands.  Operands produced on chip from
 // fp32 values (T', T'', P, U and U diag(gamma_L/gamma)) are passed as a bf16
 // pair hi + lo (hi = bf16(x), lo = bf16(x - hi)) and multiplied as hi*y + lo*y
 // (plus the hi*lo cross term where both sides are split), which keeps ~16
 // significant bits; the decay gamma_t of the inter-chunk read-out is applied in
-// fp32 to a separate accumulator instead of being folded into a bf16 copy of q.
-// Only S0 and W enter as single bf16 operands.
+// fp32 to a separate accumulator.  Only S0 and W enter as single bf16 operands.
 #include <cuda.h>
 
 #include "gdn_common.cuh"
@@ -53,38 +63,47 @@ using namespace tc;
 
 constexpr int C = 64;      // chunk
 constexpr int DH = 128;    // head dim (dk = dv)
-constexpr int kThreads = 128;
+constexpr int kTmaWarp = 0, kMmaWarp = 1, kChainWarp0 = 2, kNumChainWarps = 8;
+constexpr int kPrepWarp0 = kChainWarp0 + kNumChainWarps, kNumPrepWarps = 8;
+constexpr int kThreads = 32 * (kPrepWarp0 + kNumPrepWarps);
+constexpr int kPrepThreads = 32 * kNumPrepWarps;
 constexpr uint32_t kWait = 1u << 22;   // polls before an on-device wait gives up
 
-// shared memory layout (bytes from a 1024-aligned base)
+// ---- shared memory layout (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_QK = 0;         // 2 stages x 32 KB: [atom0: Q | K][atom1: Q | K]
 constexpr uint32_t QK_STAGE = 32768;
 constexpr uint32_t OFF_V = 65536;      // 16 KB: [atom0][atom1], 64 rows each
 constexpr uint32_t OFF_S = 81920;      // S0 bf16, 2 atom cols x 128 rows
 constexpr uint32_t OFF_W = 114688;     // W as MN-major B: 128 rows (a) x 64 (t)
-constexpr uint32_t OFF_P = 131072;     // P hi, P lo: 64 rows (t) x 64 (s) each
-// One 64 KB region used twice per chunk: first by the UT inverse (A fp32,
-// then T' and T'' as hi/lo tiles), later by U and U diag(gamma_L/gamma) (hi/lo).
-constexpr uint32_t OFF_UNION = 147456;
-constexpr uint32_t OFF_U = OFF_UNION;            // U hi, U lo     (2 x 16 KB)
-constexpr uint32_t OFF_UB = OFF_UNION + 32768;   // Ub hi, Ub lo   (2 x 16 KB)
-constexpr uint32_t OFF_A = OFF_UNION;            // A fp32 [64][65]
-constexpr uint32_t A_LD = 65;
-constexpr uint32_t OFF_TP = OFF_UNION + 17408;   // T' hi, T' lo   (2 x 8 KB)
-constexpr uint32_t OFF_TPP = OFF_TP + 16384;     // T'' hi, T'' lo (2 x 8 KB)
-constexpr uint32_t OFF_SMALL = OFF_UNION + 65536;  // G, gamma, beta, misc
-constexpr uint32_t OFF_BAR = OFF_SMALL + 4 * 64 * 4;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;   // + alignment slack
-static_assert(OFF_A + 64 * A_LD * 4 <= OFF_TP, "A overlaps T tiles");
-static_assert(OFF_TPP + 16384 <= OFF_SMALL, "T tiles overflow the union region");
+constexpr uint32_t OFF_P = 131072;     // 2 buffers x (P hi, P lo): 64 rows (t) x 64 (s)
+constexpr uint32_t P_BUF = 16384;
+constexpr uint32_t OFF_T = 163840;     // T' hi, T' lo, T'' hi, T'' lo (4 x 8 KB);
+constexpr uint32_t OFF_A = OFF_T;      //   A fp32 [64][64] shares it (dead before T' is written)
+constexpr uint32_t OFF_TF = 196608;    // T fp32 [64][T_LD]
+constexpr uint32_t T_LD = 68;
+constexpr uint32_t OFF_X = OFF_TF + 64 * T_LD * 4;   // inverse scratch: 32 x X_LD fp32
+constexpr uint32_t X_LD = 36;
+constexpr uint32_t OFF_PB = OFF_X + 32 * X_LD * 4;   // prep: beta, gamma, G (3 x 64)
+constexpr uint32_t OFF_BAR = OFF_PB + 3 * 64 * 4 + 64;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
+static_assert(OFF_A + 64 * 64 * 4 <= OFF_T + 32768, "A overflows the T tiles");
+static_assert(OFF_T + 32768 <= OFF_TF, "T tiles overlap T fp32");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// TMEM columns
+// ---- TMEM columns ----
 constexpr uint32_t TM_D1 = 0;      // X, then W^T
-constexpr uint32_t TM_U = 64;
-constexpr uint32_t TM_O = 128;     // U P^T
-constexpr uint32_t TM_Q = 192;     // S0 Q^T
-constexpr uint32_t TM_DS = 256;
-constexpr uint32_t TM_S = 384;
+constexpr uint32_t TM_U = 64;      // U~, then U
+constexpr uint32_t TM_Q = 128;     // S0 Q^T
+constexpr uint32_t TM_O = 192;     // U P^T
+constexpr uint32_t TM_S = 256;     // fp32 state (128 columns)
+constexpr uint32_t TM_UH = 384, TM_UL = 416, TM_BH = 448, TM_BL = 480;  // bf16 A operands
+
+// ---- mbarriers ----
+enum Bar {
+    B_QK_FULL0, B_QK_FULL1, B_QK_FREE0, B_QK_FREE1, B_V_FULL, B_V_FREE,
+    B_X_FULL, B_T_FULL, B_WU_FULL, B_W_FULL, B_S0_FULL, B_U_MMA, B_U_FULL,
+    B_DS_FULL, B_O_FULL, B_Q_FREE, B_P_FREE0, B_P_FREE1, B_COUNT
+};
 
 struct TcParams {
     const float *g, *beta, *h0;
@@ -97,31 +116,106 @@ struct TcParams {
     unsigned int *status;
 };
 
-__device__ __forceinline__ void ld_row64(uint32_t tmem, int warp, uint32_t col, float *v) {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        float t[16];
-        tmem_ld16(tmem_addr(tmem, warp, col + 16 * p), t);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[16 * p + j] = t[j];
+struct Ctx {
+    uint64_t *bars;
+    volatile int *abort_flag;
+    unsigned int *status;
+};
+
+// Bounded wait; on timeout (or if another role already gave up) raises the
+// CTA-wide abort flag and returns false.
+__device__ __forceinline__ bool wait_bar(const Ctx &x, int b, uint32_t parity) {
+    for (uint32_t i = 0; i < kWait; ++i) {
+        if (mbar_try_wait(&x.bars[b], parity)) return true;
+        if ((i & 1023u) == 1023u && *x.abort_flag) return false;
     }
-    tmem_wait_ld();
+    *x.abort_flag = 1;
+    atomicExch(x.status, (unsigned int)GDN_ERR_TIMEOUT);
+    return false;
+}
+__device__ __forceinline__ void arrive(const Ctx &x, int b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&x.bars[b])) : "memory");
+}
+__device__ __forceinline__ void prep_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kPrepThreads) : "memory");
 }
 
-// Row of 64 floats -> hi tile (bf16(x)) and lo tile (bf16(x - hi)), same row.
-__device__ __forceinline__ void st_row64_hilo(uint32_t hi_base, uint32_t lo_base, uint32_t r,
-                                              const float *f) {
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+    float a[16], b[16];
+    tmem_ld16(taddr, a);
+    tmem_ld16(taddr + 16, b);
+    tmem_wait_ld();
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        float hi[8], lo[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            hi[e] = __bfloat162float(__float2bfloat16_rn(f[8 * c + e]));
-            lo[e] = f[8 * c + e] - hi[e];
-        }
-        st_shared_bf16x8(hi_base + sw128_chunk(r, c), hi);
-        st_shared_bf16x8(lo_base + sw128_chunk(r, c), lo);
+    for (int j = 0; j < 16; ++j) {
+        v[j] = a[j];
+        v[16 + j] = b[j];
     }
+}
+__device__ __forceinline__ void tmem_st16w(uint32_t taddr, const uint32_t (&w)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 "
+        "[%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+        "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
+        "r"(w[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st32f(uint32_t taddr, const float *v) {
+    float a[16], b[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        a[j] = v[j];
+        b[j] = v[16 + j];
+    }
+    tmem_st16(taddr, a);
+    tmem_st16(taddr + 16, b);
+}
+// 32 floats -> hi and lo bf16 words (16 each), packed in element order.
+__device__ __forceinline__ void split_pack32(const float *f, uint32_t (&hi)[16],
+                                             uint32_t (&lo)[16]) {
+#pragma unroll
+    for (int w = 0; w < 16; ++w) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(f[2 * w], f[2 * w + 1]);
+        const float2 hf = __bfloat1622float2(h2);
+        hi[w] = *reinterpret_cast<const uint32_t *>(&h2);
+        lo[w] = pack_bf16x2(f[2 * w] - hf.x, f[2 * w + 1] - hf.y);
+    }
+}
+// 8 floats -> hi chunk (bf16(x)) and lo chunk (bf16(x - hi)) at two shared addresses.
+__device__ __forceinline__ void st_chunk_hilo(uint32_t hi_addr, uint32_t lo_addr, const float *f) {
+    float hi[8], lo[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        hi[e] = __bfloat162float(__float2bfloat16_rn(f[e]));
+        lo[e] = f[e] - hi[e];
+    }
+    st_shared_bf16x8(hi_addr, hi);
+    st_shared_bf16x8(lo_addr, lo);
+}
+
+// Chunk-local running sum of g over 64 tokens by one warp: lane l owns
+// tokens 2l and 2l+1 (rows >= L count as g = 0).  Inputs are the two g values
+// of the lane; returns G(2l), G(2l+1).
+__device__ __forceinline__ float2 warp_decay_scan(float g0, float g1) {
+    const int lane = threadIdx.x & 31;
+    float x = g0 + g1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    return make_float2(x - g1, x);
+}
+__device__ __forceinline__ float2 load_g_pair(const float *g, int64_t s0, int L, int HV, int h) {
+    const int lane = threadIdx.x & 31;
+    const int t0 = 2 * lane, t1 = 2 * lane + 1;
+    return make_float2(t0 < L ? g[(s0 + t0) * HV + h] : 0.f, t1 < L ? g[(s0 + t1) * HV + h] : 0.f);
+}
+// Value of token t's G from the scan registers (lane t/2 holds it).
+__device__ __forceinline__ float g_at(float2 G, int t) {
+    const float a = __shfl_sync(0xffffffffu, G.x, t >> 1);
+    const float b = __shfl_sync(0xffffffffu, G.y, t >> 1);
+    return (t & 1) ? b : a;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -132,16 +226,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
-    float *A_s = reinterpret_cast<float *>(sm + OFF_A);
-    float *G_s = reinterpret_cast<float *>(sm + OFF_SMALL);
-    float *gam_s = G_s + 64;
-    float *beta_s = gam_s + 64;
-    float *misc_s = beta_s + 64;
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + OFF_BAR);  // [2]: q/k stages
-    uint64_t *bar_v = bar_tma + 2;
-    uint64_t *bar_mma = bar_tma + 3;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 4);
-    volatile int *abort_s = reinterpret_cast<volatile int *>(bar_tma + 5);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + B_COUNT);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + B_COUNT + 1);
+    const Ctx x{bars, abort_flag, p.status};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x, n = blockIdx.y;
@@ -156,322 +244,481 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         eos = bos + p.T;
     }
     const int nchunks = (int)((eos - bos + C - 1) / C);
+    const size_t sbase = ((size_t)n * HV + h) * (size_t)DH * DH;
+    auto chunk_len = [&](int c) {
+        const int64_t r = eos - (bos + (int64_t)c * C);
+        return (int)(r < C ? r : C);
+    };
 
     if (tid == 0) {
-        mbar_init(&bar_tma[0], 1);
-        mbar_init(&bar_tma[1], 1);
-        mbar_init(bar_v, 1);
-        mbar_init(bar_mma, 1);
-        *abort_s = 0;
+        for (int b = 0; b < B_COUNT; ++b) {
+            uint32_t cnt = 1;
+            if (b == B_T_FULL || b == B_W_FULL) cnt = kNumPrepWarps;
+            if (b == B_S0_FULL || b == B_U_FULL || b == B_Q_FREE) cnt = kNumChainWarps;
+            mbar_init(&bars[b], cnt);
+        }
+        *abort_flag = 0;
         fence_barrier_init();
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
     }
     if (warp == 0) tmem_alloc(tslot, 512);
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    auto issue_tma_qk = [&](int c, int st) {
-        const int s0 = (int)(bos + (int64_t)c * C);
-        uint8_t *qk = sm + OFF_QK + st * QK_STAGE;
-        mbar_arrive_expect_tx(&bar_tma[st], 4 * 8192);
-        tma_load_3d(qk, &tm_q, &bar_tma[st], 0, cqk, s0);
-        tma_load_3d(qk + 16384, &tm_q, &bar_tma[st], 64, cqk, s0);
-        tma_load_3d(qk + 8192, &tm_k, &bar_tma[st], 0, cqk, s0);
-        tma_load_3d(qk + 24576, &tm_k, &bar_tma[st], 64, cqk, s0);
-    };
-    auto issue_tma_v = [&](int c) {
-        const int s0 = (int)(bos + (int64_t)c * C);
-        mbar_arrive_expect_tx(bar_v, 2 * 8192);
-        tma_load_3d(sm + OFF_V, &tm_v, bar_v, 0, h, s0);
-        tma_load_3d(sm + OFF_V + 8192, &tm_v, bar_v, 64, h, s0);
-    };
-
-    // ---- start state: fp32 into TMEM, bf16 into the S0 operand tile ----
-    const size_t sbase = ((size_t)n * HV + h) * (size_t)DH * DH;
-    {
-        const int i = tid;
-#pragma unroll 1
-        for (int q4 = 0; q4 < 8; ++q4) {
-            float v[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                v[j] = p.h0 ? p.h0[sbase + (size_t)i * DH + 16 * q4 + j] : 0.f;
-            tmem_st16(tmem_addr(tmem, warp, TM_S + 16 * q4), v);
-            const uint32_t atom = sb + OFF_S + (q4 >> 2) * 16384;
-            const uint32_t c0 = (q4 & 3) * 2;
-            st_shared_bf16x8(atom + sw128_chunk(i, c0), v);
-            st_shared_bf16x8(atom + sw128_chunk(i, c0 + 1), v + 8);
-        }
-        tmem_wait_st();
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && nchunks > 0) {
-        issue_tma_qk(0, 0);
-        issue_tma_v(0);
-    }
-
-    uint32_t mma_phase = 0;
-    bool ok = true;
-    auto wait_mma = [&]() {
-        if (!mbar_wait(bar_mma, mma_phase, kWait)) ok = false;
-        mma_phase ^= 1;
-        tc_fence_after();
-    };
-
-    for (int c = 0; c < nchunks; ++c) {
-        const int64_t s0 = bos + (int64_t)c * C;
-        const int L = (int)((eos - s0) < C ? (eos - s0) : C);
-        const int st = c & 1;
-        const uint32_t qk = sb + OFF_QK + st * QK_STAGE;
-        const uint32_t vt = sb + OFF_V;
-
-        // ---- decay running sum and write strengths (rows >= L: g = 0, b = 0) ----
-        float gv = 0.f, bv = 0.f;
-        if (tid < C && tid < L) {
-            gv = p.g[(s0 + tid) * HV + h];
-            bv = p.beta[(s0 + tid) * HV + h];
-        }
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, gv, off);
-            if (lane >= off) gv += y;
-        }
-        if (tid == 31) misc_s[0] = gv;
-        __syncthreads();
-        if (tid >= 32 && tid < 64) gv += misc_s[0];
-        if (tid < C) {
-            G_s[tid] = gv;
-            gam_s[tid] = expf(gv);
-            beta_s[tid] = bv;
-        }
-        if (!mbar_wait(&bar_tma[st], (uint32_t)((c >> 1) & 1), kWait)) ok = false;
-        if (!mbar_wait(bar_v, (uint32_t)(c & 1), kWait)) ok = false;
-        if (!ok) *abort_s = 1;
-        __syncthreads();
-        if (*abort_s) break;
-        if (tid == 0 && c + 1 < nchunks) issue_tma_qk(c + 1, st ^ 1);
-
-        // ---- X: [Q;K] K^T ----
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                mma_bf16(tmem + TM_D1, sdesc_sw128(qk + off, 16, 1024),
-                         sdesc_sw128(qk + 8192 + off, 16, 1024), id, k > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        __syncwarp();
-        wait_mma();
-        {
-            float v[64];
-            ld_row64(tmem, warp, TM_D1, v);
-            if (tid < C) {  // P row i = tid
-                const int i = tid;
-                const float Gi = G_s[i];
-#pragma unroll
-                for (int j = 0; j < 64; ++j) v[j] = (j <= i) ? expf(Gi - G_s[j]) * v[j] : 0.f;
-                st_row64_hilo(sb + OFF_P, sb + OFF_P + 8192, i, v);
-            } else {  // A row i = tid - 64
-                const int i = tid - C;
-                const float Gi = G_s[i], bi = beta_s[i];
-#pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    A_s[i * A_LD + j] = (j < i) ? bi * expf(Gi - G_s[j]) * v[j] : 0.f;
+    if (warp == kTmaWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0 && nchunks > 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c & 1;
+                const int s0 = (int)(bos + (int64_t)c * C);
+                if (c >= 2 && !wait_bar(x, B_QK_FREE0 + st, (uint32_t)(((c >> 1) - 1) & 1))) break;
+                uint8_t *qk = sm + OFF_QK + st * QK_STAGE;
+                mbar_arrive_expect_tx(&bars[B_QK_FULL0 + st], 4 * 8192);
+                tma_load_3d(qk, &tm_q, &bars[B_QK_FULL0 + st], 0, cqk, s0);
+                tma_load_3d(qk + 16384, &tm_q, &bars[B_QK_FULL0 + st], 64, cqk, s0);
+                tma_load_3d(qk + 8192, &tm_k, &bars[B_QK_FULL0 + st], 0, cqk, s0);
+                tma_load_3d(qk + 24576, &tm_k, &bars[B_QK_FULL0 + st], 64, cqk, s0);
+                if (c >= 1 && !wait_bar(x, B_V_FREE, (uint32_t)((c - 1) & 1))) break;
+                mbar_arrive_expect_tx(&bars[B_V_FULL], 2 * 8192);
+                tma_load_3d(sm + OFF_V, &tm_v, &bars[B_V_FULL], 0, h, s0);
+                tma_load_3d(sm + OFF_V + 8192, &tm_v, &bars[B_V_FULL], 64, h, s0);
             }
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- UT inverse (threads 0..63, one column each) ----
-        if (tid < C) {
-            const int j = tid;
-            float Tc[64];
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (nchunks > 0) {
+            const uint32_t id_x = idesc_bf16(128, 64, false, false);
+            const uint32_t id_w = idesc_bf16(128, 64, true, false);
+            const uint32_t id_m1 = idesc_bf16(128, 64, false, true, true);
+            const uint32_t id_m4 = idesc_bf16(128, 128, false, true);
+            auto commit = [&](int b) {
+                if (elect_one()) mma_commit(&bars[b]);
+                __syncwarp();
+            };
+            auto issue_x = [&](int c) {
+                const uint32_t qk = sb + OFF_QK + (c & 1) * QK_STAGE;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                float acc = (i == j) ? 1.f : 0.f;
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                    const uint64_t a = sdesc_sw128(qk + off, 16, 1024);
+                    const uint64_t b = sdesc_sw128(qk + 8192 + off, 16, 1024);
+                    if (elect_one()) mma_bf16(tmem + TM_D1, a, b, id_x, k > 0);
+                    __syncwarp();
+                }
+                commit(B_X_FULL);
+            };
+            auto issue_wu = [&](int c) {
+                const uint32_t qk = sb + OFF_QK + (c & 1) * QK_STAGE;
 #pragma unroll
-                for (int m = 0; m < i; ++m) acc = fmaf(-A_s[i * A_LD + m], Tc[m], acc);
-                Tc[i] = acc;
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t ka = sdesc_sw128(qk + 8192 + k * 2048, 16384, 1024);
+                    const uint64_t va = sdesc_sw128(sb + OFF_V + k * 2048, 8192, 1024);
+                    const uint64_t t1h = sdesc_sw128(sb + OFF_T + k * 32, 16, 1024);
+                    const uint64_t t1l = sdesc_sw128(sb + OFF_T + 8192 + k * 32, 16, 1024);
+                    const uint64_t t2h = sdesc_sw128(sb + OFF_T + 16384 + k * 32, 16, 1024);
+                    const uint64_t t2l = sdesc_sw128(sb + OFF_T + 24576 + k * 32, 16, 1024);
+                    if (elect_one()) {
+                        mma_bf16(tmem + TM_D1, ka, t1h, id_w, k > 0);
+                        mma_bf16(tmem + TM_D1, ka, t1l, id_w, 1);
+                        mma_bf16(tmem + TM_U, va, t2h, id_w, k > 0);
+                        mma_bf16(tmem + TM_U, va, t2l, id_w, 1);
+                    }
+                    __syncwarp();
+                }
+                commit(B_WU_FULL);
+                commit(B_V_FREE);
+            };
+            bool ok = wait_bar(x, B_QK_FULL0, 0);
+            if (ok) {
+                tc_fence_after();
+                issue_x(0);
+                ok = wait_bar(x, B_T_FULL, 0) && wait_bar(x, B_V_FULL, 0);
             }
-            const float bj = beta_s[j], bgj = bj * gam_s[j];
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const uint32_t off = sw128_offset(i, j);
-                const float x1 = Tc[i] * bgj, x2 = Tc[i] * bj;
-                const __nv_bfloat16 h1 = __float2bfloat16_rn(x1), h2 = __float2bfloat16_rn(x2);
-                const __nv_bfloat16 l1 = __float2bfloat16_rn(x1 - __bfloat162float(h1));
-                const __nv_bfloat16 l2 = __float2bfloat16_rn(x2 - __bfloat162float(h2));
-                asm volatile("st.shared.b16 [%0], %1;" ::"r"(sb + OFF_TP + off),
-                             "h"(*reinterpret_cast<const unsigned short *>(&h1)));
-                asm volatile("st.shared.b16 [%0], %1;" ::"r"(sb + OFF_TP + 8192 + off),
-                             "h"(*reinterpret_cast<const unsigned short *>(&l1)));
-                asm volatile("st.shared.b16 [%0], %1;" ::"r"(sb + OFF_TPP + off),
-                             "h"(*reinterpret_cast<const unsigned short *>(&h2)));
-                asm volatile("st.shared.b16 [%0], %1;" ::"r"(sb + OFF_TPP + 8192 + off),
-                             "h"(*reinterpret_cast<const unsigned short *>(&l2)));
+            if (ok) {
+                tc_fence_after();
+                issue_wu(0);
             }
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---- W^T, U~^T (T', T'' as hi + lo), S0 Q^T ----
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t idw = idesc_bf16(128, 64, true, false);
+            for (int c = 0; ok && c < nchunks; ++c) {
+                const uint32_t ph = (uint32_t)(c & 1);
+                const uint32_t qk = sb + OFF_QK + (c & 1) * QK_STAGE;
+                if (!wait_bar(x, B_W_FULL, ph) || !wait_bar(x, B_S0_FULL, ph)) break;
+                if (c >= 1 && !wait_bar(x, B_Q_FREE, (uint32_t)((c - 1) & 1))) break;
+                tc_fence_after();
+                // M1: U = U~ - S0 W^T (committed alone: it gates the chain)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t ka = sdesc_sw128(qk + 8192 + k * 2048, 16384, 1024);
-                const uint64_t va = sdesc_sw128(vt + k * 2048, 8192, 1024);
-                mma_bf16(tmem + TM_D1, ka, sdesc_sw128(sb + OFF_TP + k * 32, 16, 1024), idw, k > 0);
-                mma_bf16(tmem + TM_D1, ka, sdesc_sw128(sb + OFF_TP + 8192 + k * 32, 16, 1024), idw, 1);
-                mma_bf16(tmem + TM_U, va, sdesc_sw128(sb + OFF_TPP + k * 32, 16, 1024), idw, k > 0);
-                mma_bf16(tmem + TM_U, va, sdesc_sw128(sb + OFF_TPP + 8192 + k * 32, 16, 1024), idw, 1);
-            }
-            const uint32_t ido = idesc_bf16(128, 64, false, false);
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                    const uint64_t a = sdesc_sw128(sb + OFF_S + off, 16, 1024);
+                    const uint64_t b = sdesc_sw128(sb + OFF_W + k * 2048, 8192, 1024);
+                    if (elect_one()) mma_bf16(tmem + TM_U, a, b, id_m1, 1);
+                    __syncwarp();
+                }
+                commit(B_U_MMA);
+                // O1: S0 Q^T
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                mma_bf16(tmem + TM_Q, sdesc_sw128(sb + OFF_S + off, 16, 1024),
-                         sdesc_sw128(qk + off, 16, 1024), ido, k > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        __syncwarp();
-        wait_mma();
-        {
-            float v[64];
-            ld_row64(tmem, warp, TM_D1, v);  // W^T row a = tid
-            st_row64_sw128(sb + OFF_W, tid, v);
-        }
-        if (tid == 0 && c + 1 < nchunks) issue_tma_v(c + 1);  // V tile consumed by U~
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- U = U~ - S0 W^T (accumulated onto U~ with A negated) ----
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, false, true, true);
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                    const uint64_t a = sdesc_sw128(sb + OFF_S + off, 16, 1024);
+                    const uint64_t b = sdesc_sw128(qk + off, 16, 1024);
+                    if (elect_one()) mma_bf16(tmem + TM_Q, a, b, id_x, k > 0);
+                    __syncwarp();
+                }
+                if (c + 1 < nchunks) {
+                    if (!wait_bar(x, B_QK_FULL0 + ((c + 1) & 1), (uint32_t)(((c + 1) >> 1) & 1)))
+                        break;
+                    tc_fence_after();
+                    issue_x(c + 1);
+                }
+                if (!wait_bar(x, B_U_FULL, ph)) break;
+                tc_fence_after();
+                // M4: S += Ub K (Ub hi/lo from TMEM; S already scaled by gamma_L)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                mma_bf16(tmem + TM_U, sdesc_sw128(sb + OFF_S + off, 16, 1024),
-                         sdesc_sw128(sb + OFF_W + k * 2048, 8192, 1024), id, 1);
-            }
-            mma_commit(bar_mma);
-        }
-        __syncwarp();
-        wait_mma();
-        {
-            float v[64];
-            ld_row64(tmem, warp, TM_U, v);  // U^T row i = tid
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t kb = sdesc_sw128(qk + 8192 + k * 2048, 16384, 1024);
+                    if (elect_one()) {
+                        mma_bf16_ts(tmem + TM_S, tmem + TM_BH + k * 8, kb, id_m4, 1);
+                        mma_bf16_ts(tmem + TM_S, tmem + TM_BL + k * 8, kb, id_m4, 1);
+                    }
+                    __syncwarp();
+                }
+                commit(B_DS_FULL);
+                // M3: DO = U P^T (hi/lo cross terms)
+                const uint32_t pb = sb + OFF_P + (c & 1) * P_BUF;
 #pragma unroll
-            for (int t = 0; t < 64; ++t)
-                if (t >= L) v[t] = 0.f;
-            st_row64_hilo(sb + OFF_U, sb + OFF_U + 16384, tid, v);
-            const float GL = G_s[63];
-#pragma unroll
-            for (int t = 0; t < 64; ++t) v[t] *= expf(GL - G_s[t]);
-            st_row64_hilo(sb + OFF_UB, sb + OFF_UB + 16384, tid, v);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- DO = U P^T (hi/lo cross terms) ; DS = (U diag(gamma_L/gamma)) K ----
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id3 = idesc_bf16(128, 64, false, false);
-            const uint32_t id4 = idesc_bf16(128, 128, false, true);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t uh = sdesc_sw128(sb + OFF_U + k * 32, 16, 1024);
-                const uint64_t ul = sdesc_sw128(sb + OFF_U + 16384 + k * 32, 16, 1024);
-                const uint64_t ph = sdesc_sw128(sb + OFF_P + k * 32, 16, 1024);
-                const uint64_t pl = sdesc_sw128(sb + OFF_P + 8192 + k * 32, 16, 1024);
-                mma_bf16(tmem + TM_O, uh, ph, id3, k > 0);
-                mma_bf16(tmem + TM_O, uh, pl, id3, 1);
-                mma_bf16(tmem + TM_O, ul, ph, id3, 1);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t kb = sdesc_sw128(qk + 8192 + k * 2048, 16384, 1024);
-                mma_bf16(tmem + TM_DS, sdesc_sw128(sb + OFF_UB + k * 32, 16, 1024), kb, id4, k > 0);
-                mma_bf16(tmem + TM_DS, sdesc_sw128(sb + OFF_UB + 16384 + k * 32, 16, 1024), kb, id4, 1);
-            }
-            mma_commit(bar_mma);
-        }
-        __syncwarp();
-        wait_mma();
-        {
-            const int i = tid;
-            float v[64];
-            ld_row64(tmem, warp, TM_O, v);
-            __nv_bfloat16 *orow = p.o + ((size_t)s0 * HV + h) * DH + i;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                float dq[16];
-                tmem_ld16(tmem_addr(tmem, warp, TM_Q + 16 * q4), dq);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int t = 16 * q4 + j;
-                    if (t < L)
-                        orow[(size_t)t * HV * DH] =
-                            __float2bfloat16_rn(p.scale * fmaf(gam_s[t], dq[j], v[t]));
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t ph_d = sdesc_sw128(pb + k * 32, 16, 1024);
+                    const uint64_t pl_d = sdesc_sw128(pb + 8192 + k * 32, 16, 1024);
+                    if (elect_one()) {
+                        mma_bf16_ts(tmem + TM_O, tmem + TM_UH + k * 8, ph_d, id_x, k > 0);
+                        mma_bf16_ts(tmem + TM_O, tmem + TM_UH + k * 8, pl_d, id_x, 1);
+                        mma_bf16_ts(tmem + TM_O, tmem + TM_UL + k * 8, ph_d, id_x, 1);
+                    }
+                    __syncwarp();
+                }
+                commit(B_O_FULL);
+                commit(B_P_FREE0 + (c & 1));
+                commit(B_QK_FREE0 + (c & 1));
+                if (c + 1 < nchunks) {
+                    const uint32_t ph1 = (uint32_t)((c + 1) & 1);
+                    if (!wait_bar(x, B_T_FULL, ph1) || !wait_bar(x, B_V_FULL, ph1)) break;
+                    tc_fence_after();
+                    issue_wu(c + 1);
                 }
             }
-            const float gL = gam_s[63];
-#pragma unroll 1
-            for (int q4 = 0; q4 < 8; ++q4) {
-                float ds[16], s[16];
-                tmem_ld16(tmem_addr(tmem, warp, TM_DS + 16 * q4), ds);
-                tmem_ld16(tmem_addr(tmem, warp, TM_S + 16 * q4), s);
-                tmem_wait_ld();
+        }
+    } else if (warp < kPrepWarp0) {
+        // ------------------------------------------------------------ chain warps
+        const int hh = (warp - kChainWarp0) >> 2;
+        const int i = 32 * (warp & 3) + lane;  // state row (value index)
+        {
+            // start state: fp32 into TMEM (this thread's 64 columns), bf16 copy for S0
+            float v[64];
+            const float *src = p.h0 ? p.h0 + sbase + (size_t)i * DH + hh * 64 : nullptr;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) s[j] = fmaf(gL, s[j], ds[j]);
-                tmem_st16(tmem_addr(tmem, warp, TM_S + 16 * q4), s);
-                const uint32_t atom = sb + OFF_S + (q4 >> 2) * 16384;
-                const uint32_t c0 = (q4 & 3) * 2;
-                st_shared_bf16x8(atom + sw128_chunk(i, c0), s);
-                st_shared_bf16x8(atom + sw128_chunk(i, c0 + 1), s + 8);
+            for (int j = 0; j < 64; j += 4) {
+                const float4 v4 = src ? *reinterpret_cast<const float4 *>(src + j)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[j] = v4.x;
+                v[j + 1] = v4.y;
+                v[j + 2] = v4.z;
+                v[j + 3] = v4.w;
             }
+            st_row64_sw128(sb + OFF_S + hh * 16384, i, v);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) arrive(x, B_S0_FULL);
+            if (nchunks > 0) {
+                // pre-scale by gamma_L of chunk 0
+                const float2 gp = load_g_pair(p.g, bos, chunk_len(0), HV, h);
+                const float gL = expf(__shfl_sync(0xffffffffu, warp_decay_scan(gp.x, gp.y).y, 31));
+#pragma unroll
+                for (int j = 0; j < 64; ++j) v[j] *= gL;
+            }
+            tmem_st32f(tmem_addr(tmem, warp, TM_S + 64 * hh), v);
+            tmem_st32f(tmem_addr(tmem, warp, TM_S + 64 * hh + 32), v + 32);
             tmem_wait_st();
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
+        float2 gnext = nchunks > 0 ? load_g_pair(p.g, bos, chunk_len(0), HV, h) : make_float2(0.f, 0.f);
+        for (int c = 0; c < nchunks; ++c) {
+            const uint32_t ph = (uint32_t)(c & 1);
+            const int64_t s0 = bos + (int64_t)c * C;
+            const int L = chunk_len(c);
+            const float2 G = warp_decay_scan(gnext.x, gnext.y);
+            const float GL = __shfl_sync(0xffffffffu, G.y, 31);
+            if (c + 1 < nchunks) gnext = load_g_pair(p.g, s0 + C, chunk_len(c + 1), HV, h);
+            if (!wait_bar(x, B_U_MMA, ph)) break;
+            tc_fence_after();
+            {  // U epilogue: this thread's 32 tokens t = 32 hh + j of row i
+                float u[32];
+                tmem_ld32(tmem_addr(tmem, warp, TM_U + 32 * hh), u);
+                uint32_t whi[16], wlo[16];
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (32 * hh + j >= L) u[j] = 0.f;
+                split_pack32(u, whi, wlo);
+                tmem_st16w(tmem_addr(tmem, warp, TM_UH + 16 * hh), whi);
+                tmem_st16w(tmem_addr(tmem, warp, TM_UL + 16 * hh), wlo);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) u[j] *= __expf(GL - g_at(G, 32 * hh + j));
+                split_pack32(u, whi, wlo);
+                tmem_st16w(tmem_addr(tmem, warp, TM_BH + 16 * hh), whi);
+                tmem_st16w(tmem_addr(tmem, warp, TM_BL + 16 * hh), wlo);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive(x, B_U_FULL);
+            // decay of the next chunk (for the in-place state scaling)
+            float gLn = 1.f;
+            if (c + 1 < nchunks) {
+                const float2 Gn = warp_decay_scan(gnext.x, gnext.y);
+                gLn = expf(__shfl_sync(0xffffffffu, Gn.y, 31));
+            }
+            if (!wait_bar(x, B_DS_FULL, ph)) break;
+            tc_fence_after();
+            {  // new state: bf16 copy for the next chunk's S0, then scale by its gamma_L
+                float v[64];
+                tmem_ld32(tmem_addr(tmem, warp, TM_S + 64 * hh), v);
+                tmem_ld32(tmem_addr(tmem, warp, TM_S + 64 * hh + 32), v + 32);
+                st_row64_sw128(sb + OFF_S + hh * 16384, i, v);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) arrive(x, B_S0_FULL);
+                if (c + 1 < nchunks) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) v[j] *= gLn;
+                    tmem_st32f(tmem_addr(tmem, warp, TM_S + 64 * hh), v);
+                    tmem_st32f(tmem_addr(tmem, warp, TM_S + 64 * hh + 32), v + 32);
+                    tmem_wait_st();
+                }
+            }
+            if (!wait_bar(x, B_O_FULL, ph)) break;
+            tc_fence_after();
+            {  // output: o_t = scale (gamma_t DQ[i][t] + DO[i][t]) for this thread's 32 tokens
+                float dq[32], dout[32];
+                tmem_ld32(tmem_addr(tmem, warp, TM_Q + 32 * hh), dq);
+                tmem_ld32(tmem_addr(tmem, warp, TM_O + 32 * hh), dout);
+                __nv_bfloat16 *orow = p.o + ((size_t)s0 * HV + h) * DH + i;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int t = 32 * hh + j;
+                    const float gt = __expf(g_at(G, t));
+                    if (t < L)
+                        orow[(size_t)t * HV * DH] =
+                            __float2bfloat16_rn(p.scale * fmaf(gt, dq[j], dout[j]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive(x, B_Q_FREE);
+        }
+        if (!*abort_flag && p.hT) {
+            float v[64];
+            tmem_ld32(tmem_addr(tmem, warp, TM_S + 64 * hh), v);
+            tmem_ld32(tmem_addr(tmem, warp, TM_S + 64 * hh + 32), v + 32);
+            float *dst = p.hT + sbase + (size_t)i * DH + hh * 64;
+#pragma unroll
+            for (int j = 0; j < 64; j += 4)
+                *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        }
+    } else {
+        // ------------------------------------------------------------ prep warps
+        const int pt = tid - 32 * kPrepWarp0;          // 0..255
+        const int r = 32 * (warp & 3) + lane;          // TMEM lane of this thread
+        const int ph2 = (warp - kPrepWarp0) >> 2;      // which half of the row's columns
+        float *beta_s = reinterpret_cast<float *>(sm + OFF_PB);
+        float *gam_p = beta_s + 64;
+        float *G_p = gam_p + 64;
+        float *A_s = reinterpret_cast<float *>(sm + OFF_A);    // [64][64]
+        float *T_s = reinterpret_cast<float *>(sm + OFF_TF);   // [64][T_LD]
+        float *X_s = reinterpret_cast<float *>(sm + OFF_X);    // [32][X_LD]
+        float2 gnext = make_float2(0.f, 0.f), bnext = make_float2(0.f, 0.f);
+        if (warp == kPrepWarp0 && nchunks > 0) {
+            gnext = load_g_pair(p.g, bos, chunk_len(0), HV, h);
+            bnext = load_g_pair(p.beta, bos, chunk_len(0), HV, h);
+        }
+        for (int c = 0; c < nchunks; ++c) {
+            const uint32_t ph = (uint32_t)(c & 1);
+            const int64_t s0 = bos + (int64_t)c * C;
+            if (warp == kPrepWarp0) {
+                const float2 Gv = warp_decay_scan(gnext.x, gnext.y);
+                G_p[2 * lane] = Gv.x;
+                G_p[2 * lane + 1] = Gv.y;
+                gam_p[2 * lane] = expf(Gv.x);
+                gam_p[2 * lane + 1] = expf(Gv.y);
+                beta_s[2 * lane] = bnext.x;
+                beta_s[2 * lane + 1] = bnext.y;
+                if (c + 1 < nchunks) {
+                    gnext = load_g_pair(p.g, s0 + C, chunk_len(c + 1), HV, h);
+                    bnext = load_g_pair(p.beta, s0 + C, chunk_len(c + 1), HV, h);
+                }
+            }
+            bool ok = wait_bar(x, B_X_FULL, ph);
+            if (ok && r < 64 && c >= 2)
+                ok = wait_bar(x, B_P_FREE0 + (c & 1), (uint32_t)(((c >> 1) - 1) & 1));
+            prep_sync();
+            if (*abort_flag) break;
+            tc_fence_after();
+            {  // P rows (r < 64) and A rows (r >= 64) from [Q;K] K^T, 32 columns per thread
+                float v[32];
+                tmem_ld32(tmem_addr(tmem, warp, TM_D1 + 32 * ph2), v);
+                const int row = r & 63;
+                const float Gi = G_p[row];
+                if (r < 64) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = 32 * ph2 + j;
+                        v[j] = (col <= row) ? __expf(Gi - G_p[col]) * v[j] : 0.f;
+                    }
+                    const uint32_t pb = sb + OFF_P + (c & 1) * P_BUF;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const uint32_t off = sw128_chunk(row, 4 * ph2 + cc);
+                        st_chunk_hilo(pb + off, pb + 8192 + off, v + 8 * cc);
+                    }
+                } else {
+                    const float bi = beta_s[row];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = 32 * ph2 + j;
+                        v[j] = (col < row) ? bi * __expf(Gi - G_p[col]) * v[j] : 0.f;
+                    }
+                    float4 *dst = reinterpret_cast<float4 *>(A_s + row * 64 + 32 * ph2);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            prep_sync();
+            // ---- UT inverse, step 1: 16x16 diagonal blocks (threads 0..63) ----
+            if (pt < 64) {
+                const int b = pt >> 4, j = pt & 15, o0 = 16 * b;
+                float xc[16];
+#pragma unroll
+                for (int ii = 0; ii < 16; ++ii) {
+                    const float *arow = A_s + (o0 + ii) * 64 + o0;
+                    float acc0 = (ii == j) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+                    for (int m = 0; m < ii; m += 2) {
+                        acc0 = fmaf(-arow[m], xc[m], acc0);
+                        if (m + 1 < ii) acc1 = fmaf(-arow[m + 1], xc[m + 1], acc1);
+                    }
+                    xc[ii] = acc0 + acc1;
+                    T_s[(o0 + ii) * T_LD + o0 + j] = xc[ii];
+                }
+            }
+            prep_sync();
+            // ---- step 2: within each 32x32 half, T10 = -T11 A10 T00 (16x16 blocks) ----
+            {
+                const int e = pt * 2;                  // 2 consecutive outputs (same row)
+                const int hf = e >> 8, ii = (e >> 4) & 15, j = e & 15;
+                const int r1 = 32 * hf + 16, c0 = 32 * hf;
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const float am = A_s[(r1 + ii) * 64 + c0 + m];
+                    const float t0 = (m >= j) ? T_s[(c0 + m) * T_LD + c0 + j] : 0.f;
+                    const float t1 = (m >= j + 1) ? T_s[(c0 + m) * T_LD + c0 + j + 1] : 0.f;
+                    a0 = fmaf(am, t0, a0);
+                    a1 = fmaf(am, t1, a1);
+                }
+                X_s[(16 * hf + ii) * X_LD + j] = a0;
+                X_s[(16 * hf + ii) * X_LD + j + 1] = a1;
+            }
+            prep_sync();
+            {
+                const int e = pt * 2;
+                const int hf = e >> 8, ii = (e >> 4) & 15, j = e & 15;
+                const int r1 = 32 * hf + 16, c0 = 32 * hf;
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const float tm = (m <= ii) ? T_s[(r1 + ii) * T_LD + r1 + m] : 0.f;
+                    a0 = fmaf(tm, X_s[(16 * hf + m) * X_LD + j], a0);
+                    a1 = fmaf(tm, X_s[(16 * hf + m) * X_LD + j + 1], a1);
+                }
+                T_s[(r1 + ii) * T_LD + c0 + j] = -a0;
+                T_s[(r1 + ii) * T_LD + c0 + j + 1] = -a1;
+            }
+            prep_sync();
+            // ---- step 3: T[32:64][0:32] = -T22 A21 T11 (32x32 blocks), 4 outputs per thread ----
+            {
+                const int ii = pt >> 3, j = (pt & 7) * 4;
+                float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+                for (int m = 0; m < 32; ++m) {
+                    const float am = A_s[(32 + ii) * 64 + m];
+                    const float4 tv = *reinterpret_cast<const float4 *>(T_s + m * T_LD + j);
+                    a[0] = fmaf(am, (m >= j) ? tv.x : 0.f, a[0]);
+                    a[1] = fmaf(am, (m >= j + 1) ? tv.y : 0.f, a[1]);
+                    a[2] = fmaf(am, (m >= j + 2) ? tv.z : 0.f, a[2]);
+                    a[3] = fmaf(am, (m >= j + 3) ? tv.w : 0.f, a[3]);
+                }
+                *reinterpret_cast<float4 *>(X_s + ii * X_LD + j) = make_float4(a[0], a[1], a[2], a[3]);
+            }
+            prep_sync();
+            {
+                const int ii = pt >> 3, j = (pt & 7) * 4;
+                float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+                for (int m = 0; m < 32; ++m) {
+                    const float tm = (m <= ii) ? T_s[(32 + ii) * T_LD + 32 + m] : 0.f;
+                    const float4 xv = *reinterpret_cast<const float4 *>(X_s + m * X_LD + j);
+                    a[0] = fmaf(tm, xv.x, a[0]);
+                    a[1] = fmaf(tm, xv.y, a[1]);
+                    a[2] = fmaf(tm, xv.z, a[2]);
+                    a[3] = fmaf(tm, xv.w, a[3]);
+                }
+                *reinterpret_cast<float4 *>(T_s + (32 + ii) * T_LD + j) =
+                    make_float4(-a[0], -a[1], -a[2], -a[3]);
+            }
+            prep_sync();
+            // ---- T' = T diag(b gamma), T'' = T diag(b) as hi/lo bf16 tiles (rows t, cols s) ----
+            {
+                const int t = pt >> 2, qtr = pt & 3;   // 16 columns: chunks 2 qtr, 2 qtr + 1
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int chunk16 = 2 * qtr + cc;
+                    float a1[8], a2[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int s = 8 * chunk16 + e;
+                        const float tv = (s <= t) ? T_s[t * T_LD + s] : 0.f;
+                        a2[e] = tv * beta_s[s];
+                        a1[e] = a2[e] * gam_p[s];
+                    }
+                    const uint32_t off = sw128_chunk(t, chunk16);
+                    st_chunk_hilo(sb + OFF_T + off, sb + OFF_T + 8192 + off, a1);
+                    st_chunk_hilo(sb + OFF_T + 16384 + off, sb + OFF_T + 24576 + off, a2);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) arrive(x, B_T_FULL);
+            // ---- W epilogue ----
+            ok = wait_bar(x, B_WU_FULL, ph);
+            prep_sync();
+            if (*abort_flag) break;
+            tc_fence_after();
+            {
+                float v[32];
+                tmem_ld32(tmem_addr(tmem, warp, TM_D1 + 32 * ph2), v);  // W^T row a = r
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+                    st_shared_bf16x8(sb + OFF_W + sw128_chunk(r, 4 * ph2 + cc), v + 8 * cc);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive(x, B_W_FULL);
+        }
     }
 
-    if (*abort_s || !ok) {
-        if (tid == 0) atomicExch(p.status, (unsigned int)GDN_ERR_TIMEOUT);
-        // let any copy or MMA still in flight land before TMEM is released
-        if (tid == 0) {
-            mbar_wait(bar_mma, mma_phase, kWait);
-        }
-    } else if (p.hT) {
-        const int i = tid;
-        float *dst = p.hT + sbase + (size_t)i * DH;
-#pragma unroll 1
-        for (int q4 = 0; q4 < 8; ++q4) {
-            float s[16];
-            tmem_ld16(tmem_addr(tmem, warp, TM_S + 16 * q4), s);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; j += 4)
-                *reinterpret_cast<float4 *>(dst + 16 * q4 + j) =
-                    make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
-        }
-    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);
@@ -491,7 +738,6 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
     unsigned int *status = static_cast<unsigned int *>(a.workspace);
     cudaError_t err = cudaMemsetAsync(status, 0, sizeof(unsigned int), stream);
     if (err != cudaSuccess) return err;
-    if (Ttot == 0 && a.hT == nullptr) return cudaSuccess;
     CUtensorMap tq, tk, tv;
     const uint64_t tok = (uint64_t)(Ttot > 0 ? Ttot : 1);
     uint64_t dq[3] = {(uint64_t)DH, (uint64_t)a.HK, tok};

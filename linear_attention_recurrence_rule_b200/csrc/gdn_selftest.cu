@@ -9,6 +9,7 @@
 //   D4 = D0 - S * W S [128x128] (K-major A, thread-written, negated),
 //                   W [128x64] (MN-major B, thread-written), D0 [128x64]
 //                   stored into TMEM by tcgen05.st before accumulating.
+//   D5 = U  * Z     as D3 but with U packed into TMEM (A operand from TMEM).
 // All inputs are row-major bf16 (D0 fp32); outputs row-major fp32.
 #include <cuda.h>
 
@@ -44,7 +45,8 @@ umma_selftest_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_y,
                      const __grid_constant__ CUtensorMap tm_z, const __nv_bfloat16 *R,
                      const __nv_bfloat16 *U, const __nv_bfloat16 *S, const __nv_bfloat16 *W,
-                     const float *D0, float *D1, float *D2, float *D3, float *D4, int *status) {
+                     const float *D0, float *D1, float *D2, float *D3, float *D4, float *D5,
+                     int *status) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -97,6 +99,13 @@ umma_selftest_kernel(const __grid_constant__ CUtensorMap tm_x,
             for (int j = 0; j < 16; ++j) v[j] = D0[i * 64 + p * 16 + j];
             tmem_st16(tmem_addr(tmem, warp, 256 + p * 16), v);
         }
+        // U row i packed two bf16 per column -> TMEM columns 448..479
+        uint32_t w[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+            w[c] = pack_bf16x2(__bfloat162float(U[i * 64 + 2 * c]),
+                               __bfloat162float(U[i * 64 + 2 * c + 1]));
+        tmem_st32(tmem_addr(tmem, warp, 448), w);
         tmem_wait_st();
     }
     fence_proxy_async_smem();
@@ -135,6 +144,11 @@ umma_selftest_kernel(const __grid_constant__ CUtensorMap tm_x,
                 uint64_t b = sdesc_sw128(sbase + OFF_W + k * 2048, 8192, 1024);
                 mma_bf16(tmem + 256, a, b, id4, 1);
             }
+            // D5 = U(TMEM) * Z: A from TMEM, 8 columns per K step of 16
+            for (int k = 0; k < 4; ++k) {
+                uint64_t b = sdesc_sw128(sbase + OFF_Z + k * 2048, 8192, 1024);
+                mma_bf16_ts(tmem + 320, tmem + 448 + k * 8, b, id3, k > 0);
+            }
         }
         mma_commit(bar_mma);
     }
@@ -160,6 +174,9 @@ umma_selftest_kernel(const __grid_constant__ CUtensorMap tm_x,
             tmem_ld16(tmem_addr(tmem, warp, 128 + p * 16), v);
             tmem_wait_ld();
             for (int j = 0; j < 16; ++j) D3[i * 128 + p * 16 + j] = v[j];
+            tmem_ld16(tmem_addr(tmem, warp, 320 + p * 16), v);
+            tmem_wait_ld();
+            for (int j = 0; j < 16; ++j) D5[i * 128 + p * 16 + j] = v[j];
         }
     }
     tc_fence_before();
@@ -179,8 +196,8 @@ bool map2d(CUtensorMap *m, const void *p, uint64_t cols, uint64_t rows, uint32_t
 
 extern "C" int gdn_selftest_umma(const void *X, const void *Y, const void *Z, const void *R,
                                  const void *U, const void *S, const void *W, const float *D0,
-                                 float *D1, float *D2, float *D3, float *D4, int *status,
-                                 gdn_stream_t stream) {
+                                 float *D1, float *D2, float *D3, float *D4, float *D5,
+                                 int *status, gdn_stream_t stream) {
     using namespace gdn;
     CUtensorMap tx, ty, tz;
     if (!map2d(&tx, X, 128, 128, 128) || !map2d(&ty, Y, 128, 64, 64) ||
@@ -194,6 +211,6 @@ extern "C" int gdn_selftest_umma(const void *X, const void *Y, const void *Z, co
     umma_selftest_kernel<<<1, 128, SMEM_BYTES, s>>>(
         tx, ty, tz, static_cast<const __nv_bfloat16 *>(R), static_cast<const __nv_bfloat16 *>(U),
         static_cast<const __nv_bfloat16 *>(S), static_cast<const __nv_bfloat16 *>(W), D0, D1, D2,
-        D3, D4, status);
+        D3, D4, D5, status);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
