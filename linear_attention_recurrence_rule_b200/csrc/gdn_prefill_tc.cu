@@ -67,7 +67,7 @@ constexpr int kTmaWarp = 0, kMmaWarp = 1, kChainWarp0 = 2, kNumChainWarps = 8;
 constexpr int kPrepWarp0 = kChainWarp0 + kNumChainWarps, kNumPrepWarps = 8;
 constexpr int kThreads = 32 * (kPrepWarp0 + kNumPrepWarps);
 constexpr int kPrepThreads = 32 * kNumPrepWarps;
-constexpr uint32_t kWait = 1u << 22;   // polls before an on-device wait gives up
+constexpr uint32_t kWait = 2000;      // sleeping polls (<= ~1 ms each) before a wait gives up
 
 // ---- shared memory layout (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_QK = 0;         // 2 stages x 32 KB: [atom0: Q | K][atom1: Q | K]
@@ -78,15 +78,17 @@ constexpr uint32_t OFF_W = 114688;     // W as MN-major B: 128 rows (a) x 64 (t)
 constexpr uint32_t OFF_P = 131072;     // 2 buffers x (P hi, P lo): 64 rows (t) x 64 (s)
 constexpr uint32_t P_BUF = 16384;
 constexpr uint32_t OFF_T = 163840;     // T' hi, T' lo, T'' hi, T'' lo (4 x 8 KB);
-constexpr uint32_t OFF_A = OFF_T;      //   A fp32 [64][64] shares it (dead before T' is written)
+constexpr uint32_t OFF_A = OFF_T;      //   A fp32 [64][A_LD] shares it (dead before T' is written)
+constexpr uint32_t A_LD = 68;
 constexpr uint32_t OFF_TF = 196608;    // T fp32 [64][T_LD]
 constexpr uint32_t T_LD = 68;
 constexpr uint32_t OFF_X = OFF_TF + 64 * T_LD * 4;   // inverse scratch: 32 x X_LD fp32
 constexpr uint32_t X_LD = 36;
 constexpr uint32_t OFF_PB = OFF_X + 32 * X_LD * 4;   // prep: beta, gamma, G (3 x 64)
-constexpr uint32_t OFF_BAR = OFF_PB + 3 * 64 * 4 + 64;
+constexpr uint32_t OFF_CG = OFF_PB + 3 * 64 * 4;     // per chain warp: G, gamma (2 x 64)
+constexpr uint32_t OFF_BAR = OFF_CG + kNumChainWarps * 128 * 4 + 64;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
-static_assert(OFF_A + 64 * 64 * 4 <= OFF_T + 32768, "A overflows the T tiles");
+static_assert(OFF_A + 64 * A_LD * 4 <= OFF_T + 32768, "A overflows the T tiles");
 static_assert(OFF_T + 32768 <= OFF_TF, "T tiles overlap T fp32");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -126,8 +128,8 @@ struct Ctx {
 // CTA-wide abort flag and returns false.
 __device__ __forceinline__ bool wait_bar(const Ctx &x, int b, uint32_t parity) {
     for (uint32_t i = 0; i < kWait; ++i) {
-        if (mbar_try_wait(&x.bars[b], parity)) return true;
-        if ((i & 1023u) == 1023u && *x.abort_flag) return false;
+        if (mbar_try_wait_sleep(&x.bars[b], parity, 1000000u)) return true;
+        if (*x.abort_flag) return false;
     }
     *x.abort_flag = 1;
     atomicExch(x.status, (unsigned int)GDN_ERR_TIMEOUT);
@@ -210,12 +212,6 @@ __device__ __forceinline__ float2 load_g_pair(const float *g, int64_t s0, int L,
     const int lane = threadIdx.x & 31;
     const int t0 = 2 * lane, t1 = 2 * lane + 1;
     return make_float2(t0 < L ? g[(s0 + t0) * HV + h] : 0.f, t1 < L ? g[(s0 + t1) * HV + h] : 0.f);
-}
-// Value of token t's G from the scan registers (lane t/2 holds it).
-__device__ __forceinline__ float g_at(float2 G, int t) {
-    const float a = __shfl_sync(0xffffffffu, G.x, t >> 1);
-    const float b = __shfl_sync(0xffffffffu, G.y, t >> 1);
-    return (t & 1) ? b : a;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -413,6 +409,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         // ------------------------------------------------------------ chain warps
         const int hh = (warp - kChainWarp0) >> 2;
         const int i = 32 * (warp & 3) + lane;  // state row (value index)
+        float *cg = reinterpret_cast<float *>(sm + OFF_CG) + (warp - kChainWarp0) * 128;  // G, gamma
         {
             // start state: fp32 into TMEM (this thread's 64 columns), bf16 copy for S0
             float v[64];
@@ -446,8 +443,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             const uint32_t ph = (uint32_t)(c & 1);
             const int64_t s0 = bos + (int64_t)c * C;
             const int L = chunk_len(c);
-            const float2 G = warp_decay_scan(gnext.x, gnext.y);
-            const float GL = __shfl_sync(0xffffffffu, G.y, 31);
+            {
+                const float2 G = warp_decay_scan(gnext.x, gnext.y);
+                cg[2 * lane] = G.x;
+                cg[2 * lane + 1] = G.y;
+                cg[64 + 2 * lane] = expf(G.x);
+                cg[64 + 2 * lane + 1] = expf(G.y);
+                __syncwarp();
+            }
+            const float GL = cg[63];
             if (c + 1 < nchunks) gnext = load_g_pair(p.g, s0 + C, chunk_len(c + 1), HV, h);
             if (!wait_bar(x, B_U_MMA, ph)) break;
             tc_fence_after();
@@ -462,7 +466,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tmem_st16w(tmem_addr(tmem, warp, TM_UH + 16 * hh), whi);
                 tmem_st16w(tmem_addr(tmem, warp, TM_UL + 16 * hh), wlo);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) u[j] *= __expf(GL - g_at(G, 32 * hh + j));
+                for (int j = 0; j < 32; ++j) u[j] *= __expf(GL - cg[32 * hh + j]);
                 split_pack32(u, whi, wlo);
                 tmem_st16w(tmem_addr(tmem, warp, TM_BH + 16 * hh), whi);
                 tmem_st16w(tmem_addr(tmem, warp, TM_BL + 16 * hh), wlo);
@@ -505,7 +509,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int t = 32 * hh + j;
-                    const float gt = __expf(g_at(G, t));
+                    const float gt = cg[64 + t];
                     if (t < L)
                         orow[(size_t)t * HV * DH] =
                             __float2bfloat16_rn(p.scale * fmaf(gt, dq[j], dout[j]));
@@ -532,7 +536,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         float *beta_s = reinterpret_cast<float *>(sm + OFF_PB);
         float *gam_p = beta_s + 64;
         float *G_p = gam_p + 64;
-        float *A_s = reinterpret_cast<float *>(sm + OFF_A);    // [64][64]
+        float *A_s = reinterpret_cast<float *>(sm + OFF_A);    // [64][A_LD]
         float *T_s = reinterpret_cast<float *>(sm + OFF_TF);   // [64][T_LD]
         float *X_s = reinterpret_cast<float *>(sm + OFF_X);    // [32][X_LD]
         float2 gnext = make_float2(0.f, 0.f), bnext = make_float2(0.f, 0.f);
@@ -586,7 +590,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const int col = 32 * ph2 + j;
                         v[j] = (col < row) ? bi * __expf(Gi - G_p[col]) * v[j] : 0.f;
                     }
-                    float4 *dst = reinterpret_cast<float4 *>(A_s + row * 64 + 32 * ph2);
+                    float4 *dst = reinterpret_cast<float4 *>(A_s + row * A_LD + 32 * ph2);
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
                         dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
@@ -601,7 +605,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 float xc[16];
 #pragma unroll
                 for (int ii = 0; ii < 16; ++ii) {
-                    const float *arow = A_s + (o0 + ii) * 64 + o0;
+                    const float *arow = A_s + (o0 + ii) * A_LD + o0;
                     float acc0 = (ii == j) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
                     for (int m = 0; m < ii; m += 2) {
@@ -621,7 +625,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 float a0 = 0.f, a1 = 0.f;
 #pragma unroll
                 for (int m = 0; m < 16; ++m) {
-                    const float am = A_s[(r1 + ii) * 64 + c0 + m];
+                    const float am = A_s[(r1 + ii) * A_LD + c0 + m];
                     const float t0 = (m >= j) ? T_s[(c0 + m) * T_LD + c0 + j] : 0.f;
                     const float t1 = (m >= j + 1) ? T_s[(c0 + m) * T_LD + c0 + j + 1] : 0.f;
                     a0 = fmaf(am, t0, a0);
@@ -652,7 +656,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
                 for (int m = 0; m < 32; ++m) {
-                    const float am = A_s[(32 + ii) * 64 + m];
+                    const float am = A_s[(32 + ii) * A_LD + m];
                     const float4 tv = *reinterpret_cast<const float4 *>(T_s + m * T_LD + j);
                     a[0] = fmaf(am, (m >= j) ? tv.x : 0.f, a[0]);
                     a[1] = fmaf(am, (m >= j + 1) ? tv.y : 0.f, a[1]);

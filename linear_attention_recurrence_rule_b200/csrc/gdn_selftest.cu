@@ -23,7 +23,7 @@ namespace {
 
 using namespace tc;
 
-constexpr uint32_t kWait = 1u << 22;
+constexpr uint32_t kWait = 2000;   // sleeping polls of at most ~1 ms each
 
 constexpr uint32_t OFF_X = 0;          // 2 atom cols x 128 rows = 32 KB
 constexpr uint32_t OFF_Y = 32768;      // 2 x 64 rows = 16 KB

@@ -54,11 +54,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: returns false after `limit` unsuccessful polls instead of
-// spinning forever (the caller then records a timeout and winds down).
+// As above, but a thread whose phase is not complete sleeps until it completes
+// or `hint_ns` nanoseconds pass, instead of returning at once: waiting warps
+// then take no issue slots or shared-memory bandwidth from working warps.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: returns false after `limit` unsuccessful sleeping polls (each
+// at most ~1 ms) instead of spinning forever; the caller then records a
+// timeout and winds down.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit) {
     for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     return false;
 }
 
