@@ -59,6 +59,27 @@ def decode_bytes_per_step(N, HK, HV, dk, dv, elt=2):
     return 2 * N * HV * dv * dk * 4 + 2 * N * HK * dk * elt + 2 * N * HV * dv * elt + 2 * N * HV * 4
 
 
+def dist_max(x, device=None):
+    """Max of a host float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(world, units_per_rank, steps, max_ms):
+    """Whole-job throughput: units every rank processed over the slowest rank's time."""
+    return world * units_per_rank * steps / (max_ms / 1000.0)
+
+
+def replica_seed_offset(rank):
+    """Each replica draws its own sequence of the same workload."""
+    return rank
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -247,15 +268,11 @@ def run_b200(args):
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return dist_max(x, dev)
 
     peaks, peak_src = load_peaks()
     w = WORKLOADS[WORKLOAD]
-    x = workload_inputs(WORKLOAD, seed_offset=rank)
+    x = workload_inputs(WORKLOAD, seed_offset=replica_seed_offset(rank), tokens=args.tokens)
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     B, T = d["q"].shape[0], d["q"].shape[1]
     tokens = B * T
@@ -272,7 +289,8 @@ def run_b200(args):
         gdn.gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], chunk=w.chunk, o=o,
                               hT=hT, workspace=ws, stream=stream)
 
-    for _ in range(args.warmup):
+    n_steps = 0 if args.no_prefill else args.steps
+    for _ in range(0 if args.no_prefill else args.warmup):
         step()
     torch.cuda.synchronize()
     barrier()
@@ -280,11 +298,11 @@ def run_b200(args):
     sampler = ClockSampler(local)
     sampler.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+          for _ in range(max(n_steps, 1))]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for i in range(args.steps):
+    for i in range(n_steps):
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
@@ -294,9 +312,9 @@ def run_b200(args):
     torch.cuda.synchronize()
     clocks = sampler.stop()
     elapsed_ms = t0.elapsed_time(t1)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    launch_ms = [a.elapsed_time(b) for a, b in ev[:n_steps]] or [float("nan")]
     elapsed_ms = max_over_ranks(elapsed_ms)
-    value = world * tokens * args.steps / (elapsed_ms / 1000.0)
+    value = aggregate_throughput(world, tokens, n_steps, elapsed_ms) if n_steps else None
     mean_launch_s = statistics.mean(launch_ms) / 1000.0
 
     flops = prefill_flops_per_token(w.HK, w.HV, w.dk, w.chunk) * tokens
@@ -315,10 +333,12 @@ def run_b200(args):
     roof["traffic"] = kernel_traffic(kernel_key)
     roof["peak_source"] = peak_src
     roof["kernel"] = kernel_key
+    if not n_steps:
+        roof = None
 
     # ---- end to end through the public call, host buffers, copies timed ----
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and n_steps:
         names = ("q", "k", "v", "g", "beta")
         host_in = {n: x[n].pin_memory() for n in names}
         host_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
@@ -354,7 +374,7 @@ def run_b200(args):
     dec = None
     if not args.no_decode:
         wd = WORKLOADS[DECODE_WORKLOAD]
-        y = workload_inputs(DECODE_WORKLOAD, seed_offset=rank)
+        y = workload_inputs(DECODE_WORKLOAD, seed_offset=replica_seed_offset(rank))
         dy = {k: v.to(dev) for k, v in y.items()}
         S = dy["state"].clone()
         od = torch.empty_like(dy["v"][0])
@@ -403,14 +423,16 @@ def run_b200(args):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": elapsed_ms / n_steps if n_steps else None, "higher_is_better": True,
+            "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": 1, "T": 65536, "HK": 16, "HV": 32, "d": 128,
+            "config": {"workload": WORKLOAD if tokens == 65536 else f"{WORKLOAD} truncated to {tokens} tokens",
+                       "B": 1, "T": tokens, "HK": 16, "HV": 32, "d": 128,
                        "chunk": 64, "parallelism": "replicas" if world > 1 else "single",
                        "path": "tcgen05" if path == 1 else "cuda-core",
                        "l2": "inputs larger than L2 (q,k,v 1.07 GB per step)"},
             "roofline": roof, "cpu_baseline": base, "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "decode": dec,
+            "gpu_launches": launches_per_step * n_steps, "clocks": clocks, "decode": dec,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -429,6 +451,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="decode measurement only")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="truncate the prefill workload (profiling runs; not a bench line)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     args = ap.parse_args()
