@@ -93,7 +93,14 @@ def load_peaks():
 # summarised under profiles/ (dram__bytes_read.sum + dram__bytes_write.sum).
 # Each entry carries the sha256 of the kernel source it was taken on; a changed
 # source reports null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # full 64K launch: dram__bytes_read.sum 1,091,034,112 + dram__bytes_write.sum 511,872,000
+    "prefill_tc": {"bytes": 1602906112, "source": "gdn_prefill_tc.cu",
+                   "sha256": "87967450ffc86bebf087d8aaab0c3866571a765f39a03aeb40a70a4c2aca7172"},
+    # full decode_256x64 step: 541,205,504 read + 480,342,528 written
+    "decode": {"bytes": 1021548032, "source": "gdn_decode.cu",
+               "sha256": "6bd14494733cc78d5b35f9cc22ae3a4713fce92518aacec935bf3b868656250d"},
+}
 
 
 def kernel_traffic(key, units_scale=1.0):
