@@ -78,7 +78,7 @@ gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v, const 
         const size_t need = gdn::prefill_tc_workspace(N, T, HV, chunk, cu_seqlens != nullptr);
         if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
         if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
-        err = gdn::launch_prefill_tc(a, reinterpret_cast<cudaStream_t>(stream));
+        err = gdn::launch_prefill_cluster(a, reinterpret_cast<cudaStream_t>(stream));
     } else {
         err = gdn::launch_prefill_simt(a, reinterpret_cast<cudaStream_t>(stream));
     }
