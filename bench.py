@@ -94,9 +94,6 @@ def load_peaks():
 # Each entry carries the sha256 of the kernel source it was taken on; a changed
 # source reports null.
 NCU_TRAFFIC = {
-    # full 64K launch: dram__bytes_read.sum 1,091,034,112 + dram__bytes_write.sum 511,872,000
-    "prefill_tc": {"bytes": 1602906112, "source": "gdn_prefill_tc.cu",
-                   "sha256": "87967450ffc86bebf087d8aaab0c3866571a765f39a03aeb40a70a4c2aca7172"},
     # full decode_256x64 step: 541,205,504 read + 480,342,528 written
     "decode": {"bytes": 1021548032, "source": "gdn_decode.cu",
                "sha256": "6bd14494733cc78d5b35f9cc22ae3a4713fce92518aacec935bf3b868656250d"},
@@ -329,7 +326,7 @@ def run_b200(args):
         peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": flops / mean_launch_s / 1e12, "peak": peak,
                 "unit": "TFLOP/s"}
-        kernel_key = "prefill_tc"
+        kernel_key = "prefill_cluster"
     else:
         mhz = peaks.get("sm_max_mhz", FALLBACK_PEAKS["sm_max_mhz"])
         peak = N_SM * FP32_FMA_PER_SM_PER_CLK * 2 * mhz * 1e6 / 1e12

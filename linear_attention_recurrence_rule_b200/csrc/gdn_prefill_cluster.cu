@@ -47,9 +47,9 @@ constexpr int C = 64;
 constexpr int DH = 128;
 constexpr int kNumPrep = 3;
 constexpr int kClusterSize = 1 + kNumPrep;
-constexpr int kThreads = 14 * 32;
+constexpr int kThreads = 18 * 32;
 // chain CTA roles
-constexpr int kCTma = 0, kCMma = 1, kCChain0 = 2, kCNumChain = 8, kCOut0 = 10, kCNumOut = 4;
+constexpr int kCTma = 0, kCMma = 1, kCChain0 = 2, kCNumChain = 8, kCOut0 = 10, kCNumOut = 8;
 // prep CTA roles
 constexpr int kPCtl = 0, kPWork0 = 1, kPNumWork = 8, kPWorkThreads = kPNumWork * 32;
 constexpr uint32_t kWait = 2000;  // sleeping polls (<= ~1 ms each) before a wait gives up
@@ -94,7 +94,7 @@ constexpr uint32_t TP_D1 = 0, TP_U = 64;
 
 enum ChainBar {
     CB_QK_FULL0, CB_QK_FULL1, CB_QK_FREE0, CB_QK_FREE1, CB_R_FULL0, CB_R_FULL1, CB_S0_FULL,
-    CB_U_MMA, CB_U_FULL, CB_DS_FULL, CB_O_FULL, CB_Q_FREE, CB_COUNT
+    CB_U_MMA, CB_U_FULL, CB_U2_FULL, CB_DS_FULL, CB_O_FULL, CB_Q_FREE, CB_COUNT
 };
 enum PrepBar { PB_LD_FULL, PB_X_DONE, PB_T_READY, PB_WU_DONE, PB_EPI_DONE, PB_GO, PB_STAGE_FREE,
                PB_COUNT };
@@ -183,8 +183,6 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                 mbar_arrive_remote(mapa_shared(sb + P_BAR + PB_STAGE_FREE * 8, 1 + c % kNumPrep));
             __syncwarp();
             if (!wt(CB_S0_FULL, ph)) break;
-            if (c >= 1 && !wt(CB_Q_FREE, (uint32_t)((c - 1) & 1))) break;
-            if (!wt(CB_QK_FULL0 + s, (uint32_t)((c >> 1) & 1))) break;
             tc_fence_after();
             // D = S0 W^T (A = S0 from TMEM, B = W MN-major from the receive slot)
 #pragma unroll
@@ -194,7 +192,10 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                 __syncwarp();
             }
             commit(CB_U_MMA);
-            // S0 Q^T
+            // S0 Q^T (its accumulator is free once the output warps read chunk c-1)
+            if (c >= 1 && !wt(CB_Q_FREE, (uint32_t)((c - 1) & 1))) break;
+            if (!wt(CB_QK_FULL0 + s, (uint32_t)((c >> 1) & 1))) break;
+            tc_fence_after();
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const uint64_t b = sdesc_sw128(qst + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024);
@@ -215,6 +216,8 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             }
             commit(CB_DS_FULL);
             // U P^T (hi/lo cross terms)
+            if (!wt(CB_U2_FULL, ph)) break;
+            tc_fence_after();
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const uint64_t ph_d = sdesc_sw128(slot + SL_PH + k * 32, 16, 1024);
@@ -299,19 +302,24 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
                     if (32 * hh + j >= L) u[j] = 0.f;
+                float ub[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) ub[j] = u[j] * __expf(GL - tab[32 * hh + j]);
+                split_pack32(ub, whi, wlo);
+                tmem_st16w(tmem_addr(tmem, warp, TM_BH + 16 * hh), whi);
+                tmem_st16w(tmem_addr(tmem, warp, TM_BL + 16 * hh), wlo);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) local_arrive(&bars[CB_U_FULL]);   // the state update can start
                 split_pack32(u, whi, wlo);
                 tmem_st16w(tmem_addr(tmem, warp, TM_UH + 16 * hh), whi);
                 tmem_st16w(tmem_addr(tmem, warp, TM_UL + 16 * hh), wlo);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) u[j] *= __expf(GL - tab[32 * hh + j]);
-                split_pack32(u, whi, wlo);
-                tmem_st16w(tmem_addr(tmem, warp, TM_BH + 16 * hh), whi);
-                tmem_st16w(tmem_addr(tmem, warp, TM_BL + 16 * hh), wlo);
                 tmem_wait_st();
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) local_arrive(&bars[CB_U_FULL]);
+            if (lane == 0) local_arrive(&bars[CB_U2_FULL]);
             float gLn = 1.f;
             if (c + 1 < nchunks) {
                 const float2 Gn = warp_decay_scan(gnext.x, gnext.y);
@@ -355,6 +363,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
     } else {
         // ------------------------------------------------------------ output warps
         const int qd = warp & 3;
+        const int half = (warp - kCOut0) >> 2;   // tokens 32 half .. 32 half + 31
         const int i0 = 32 * qd;
         float *tab = reinterpret_cast<float *>(sm + C_TAB) + (warp - kCChain0) * 128;
         unsigned short *ost = reinterpret_cast<unsigned short *>(sm + C_OST + (warp - kCOut0) * 512);
@@ -372,8 +381,16 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             if (c + 1 < nchunks) gnext = load_g_pair(p.g, s0 + C, chunk_len(c + 1), HV, h);
             if (!wt(CB_O_FULL, ph)) break;
             tc_fence_after();
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            // every MMA reading the receive slot of chunk c has completed: re-arm it
+            // and release the prep CTA that produces chunk c + 2 into it
+            if (warp == kCOut0 && c + 2 < nchunks) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bars[CB_R_FULL0 + (c & 1)], SLOT);
+                    mbar_arrive_remote(mapa_shared(sb + P_BAR + PB_GO * 8, 1 + (c + 2) % kNumPrep));
+                }
+                __syncwarp();
+            }
+            {
                 float dq[32], dout[32];
                 tmem_ld32(tmem_addr(tmem, warp, TM_Q + 32 * half), dq);
                 tmem_ld32(tmem_addr(tmem, warp, TM_O + 32 * half), dout);
@@ -399,15 +416,6 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             tc_fence_before();
             __syncwarp();
             if (lane == 0) local_arrive(&bars[CB_Q_FREE]);
-            // the receive slot of chunk c is consumed: re-arm it and release the prep
-            // CTA that produces chunk c + 2 into it
-            if (warp == kCOut0 && c + 2 < nchunks) {
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&bars[CB_R_FULL0 + (c & 1)], SLOT);
-                    mbar_arrive_remote(mapa_shared(sb + P_BAR + PB_GO * 8, 1 + (c + 2) % kNumPrep));
-                }
-                __syncwarp();
-            }
         }
     }
 }
@@ -731,7 +739,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (tid == 0) {
         for (int b = 0; b < nbars; ++b) {
             uint32_t cnt = 1;
-            if (rank == 0 && (b == CB_S0_FULL || b == CB_U_FULL)) cnt = kCNumChain;
+            if (rank == 0 && (b == CB_S0_FULL || b == CB_U_FULL || b == CB_U2_FULL)) cnt = kCNumChain;
             if (rank == 0 && b == CB_Q_FREE) cnt = kCNumOut;
             if (rank != 0 && (b == PB_T_READY || b == PB_EPI_DONE)) cnt = kPNumWork;
             mbar_init(&bars[b], cnt);
