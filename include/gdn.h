@@ -126,6 +126,33 @@ GDN_API gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v
                              void *workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_prefill without a caller-provided workspace.  (The source pages
+ * have no counterpart: this is a library convenience, not part of the rule.)
+ *
+ * For callers that cannot allocate device memory -- code running under a
+ * fixed, pre-reserved memory budget, a hot path that must not call cudaMalloc
+ * (it can synchronise the device and stall other streams), or a host API that
+ * offers no workspace.  Same arguments, layouts and results as
+ * gdn_chunk_prefill; the scratch it needs lives in a 256-byte array inside the
+ * library that every device loading the library keeps until the process exits.
+ *   - Problems needing more than 256 bytes of workspace (see
+ *     gdn_chunk_prefill_workspace_size) return GDN_ERR_WORKSPACE.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls on a device share the array and leave their contents in it:
+ *     calls whose work overlaps on the GPU (different streams, not ordered)
+ *     race on it.  Order them on one stream, or use gdn_chunk_prefill with
+ *     separate workspaces.
+ *   - It allocates nothing and calls no allocating routine.
+ */
+GDN_API gdn_status gdn_chunk_prefill_noalloc(const void *q, const void *k, const void *v,
+                                             const float *g, const float *beta, const float *h0,
+                                             const int32_t *cu_seqlens, int N, int64_t T, int HK,
+                                             int HV, int dk, int dv, int chunk, float scale,
+                                             gdn_dtype dtype, void *o, float *hT,
+                                             gdn_stream_t stream);
+
+/*
  * Fused single-token decode step for N independent sequences: applies one
  * token of the rule to each sequence's state in place and writes its output.
  * Every state element is read once and written once (one pass through HBM).
