@@ -65,9 +65,9 @@ constexpr uint32_t SLOT = 65536;
 constexpr uint32_t C_Q = 0;         // 2 stages x 16 KB (q tile, two atom columns)
 constexpr uint32_t C_K = 32768;     // 2 stages x 16 KB
 constexpr uint32_t C_R = 65536;     // 2 receive slots x 64 KB
-constexpr uint32_t C_TAB = C_R + 2 * SLOT;                 // per chain/output warp: G, gamma
-constexpr uint32_t C_OST = C_TAB + (kCNumChain + kCNumOut) * 512;  // output transpose tiles
-constexpr uint32_t C_BAR = C_OST + kCNumOut * 512;
+constexpr uint32_t C_TAB = C_R + 2 * SLOT;  // per chain warp gamma_L/gamma, per output warp gamma
+constexpr uint32_t C_OST = C_TAB + (kCNumChain + kCNumOut) * 512;  // o tile staging (TMA store)
+constexpr uint32_t C_BAR = C_OST + 16384;
 // ---- prep CTA shared memory ----
 constexpr uint32_t P_QK = 0;        // [atom0: Q | K][atom1: Q | K]
 constexpr uint32_t P_V = 32768;
@@ -84,6 +84,7 @@ constexpr uint32_t SMEM_BYTES = (C_BAR > P_BAR ? C_BAR : P_BAR) + 256 + 1024;
 static_assert(P_PB + 3 * 64 * 4 <= P_ST, "prep layout");
 static_assert(64 * A_LD * 4 <= 32768, "A fits the T tiles");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(C_OST % 1024 == 0, "128B-swizzled staging tile alignment");
 
 // ---- TMEM columns ----
 // chain: D = S0 W^T, S0 Q^T, U P^T, S0 (bf16 A operand), S (fp32), U/Ub hi/lo (bf16 A)
@@ -131,13 +132,17 @@ __device__ __forceinline__ void local_arrive(uint64_t *bar) {
 __device__ __forceinline__ void work_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kPWorkThreads) : "memory");
 }
+__device__ __forceinline__ void out_sync() {
+    asm volatile("bar.sync 2, %0;" ::"n"(kCNumOut * 32) : "memory");
+}
 // fp32 U~ tile [i][t]: byte offset of the 16-byte chunk holding t = 4*tc .. 4*tc+3 of row i
 __device__ __forceinline__ uint32_t ut_chunk(uint32_t i, uint32_t tc) {
     return i * 256u + (((tc ^ i) & 15u) << 4);
 }
 
 // ============================================================================ chain CTA
-__device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const ClParams &p,
+__device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_o,
+                          const ClParams &p,
                           uint8_t *sm, uint32_t sb, uint32_t tmem, const Waiter &wt, int h,
                           int n, int64_t bos, int64_t eos, int nchunks) {
     uint64_t *bars = wt.bars;
@@ -178,9 +183,10 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             const uint32_t slot = sb + C_R + s * SLOT;
             const uint32_t qst = sb + C_Q + s * 16384, kst = sb + C_K + s * 16384;
             if (!wt(CB_R_FULL0 + s, (uint32_t)((c >> 1) & 1))) break;
-            // the producing prep CTA may reuse its staging block
+            // the bulk copy out of the producing prep CTA's staging block has completed:
+            // that block may be refilled
             if (elect_one())
-                mbar_arrive_remote(mapa_shared(sb + P_BAR + PB_STAGE_FREE * 8, 1 + c % kNumPrep));
+                mbar_arrive_remote_relaxed(mapa_shared(sb + P_BAR + PB_STAGE_FREE * 8, 1 + c % kNumPrep));
             __syncwarp();
             if (!wt(CB_S0_FULL, ph)) break;
             tc_fence_after();
@@ -236,7 +242,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
         // ------------------------------------------------------------ chain warps
         const int hh = (warp - kCChain0) >> 2;
         const int i = 32 * (warp & 3) + lane;
-        float *tab = reinterpret_cast<float *>(sm + C_TAB) + (warp - kCChain0) * 128;  // G, gamma
+        float *tab = reinterpret_cast<float *>(sm + C_TAB) + (warp - kCChain0) * 128;  // gamma_L/gamma
         {
             float v[64];
             const float *src = p.h0 ? p.h0 + sbase + (size_t)i * DH + hh * 64 : nullptr;
@@ -277,11 +283,11 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             const int L = chunk_len(c);
             {
                 const float2 G = warp_decay_scan(gnext.x, gnext.y);
-                tab[2 * lane] = G.x;
-                tab[2 * lane + 1] = G.y;
+                const float GL = __shfl_sync(0xffffffffu, G.y, 31);
+                tab[2 * lane] = __expf(GL - G.x);
+                tab[2 * lane + 1] = __expf(GL - G.y);
                 __syncwarp();
             }
-            const float GL = tab[63];
             if (c + 1 < nchunks) gnext = load_g_pair(p.g, s0 + C, chunk_len(c + 1), HV, h);
             if (!wt(CB_R_FULL0 + s, (uint32_t)((c >> 1) & 1))) break;
             if (!wt(CB_U_MMA, ph)) break;
@@ -304,7 +310,13 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                     if (32 * hh + j >= L) u[j] = 0.f;
                 float ub[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) ub[j] = u[j] * __expf(GL - tab[32 * hh + j]);
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 f = *reinterpret_cast<const float4 *>(tab + 32 * hh + 4 * q4);
+                    ub[4 * q4] = u[4 * q4] * f.x;
+                    ub[4 * q4 + 1] = u[4 * q4 + 1] * f.y;
+                    ub[4 * q4 + 2] = u[4 * q4 + 2] * f.z;
+                    ub[4 * q4 + 3] = u[4 * q4 + 3] * f.w;
+                }
                 split_pack32(ub, whi, wlo);
                 tmem_st16w(tmem_addr(tmem, warp, TM_BH + 16 * hh), whi);
                 tmem_st16w(tmem_addr(tmem, warp, TM_BL + 16 * hh), wlo);
@@ -362,11 +374,14 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
         }
     } else {
         // ------------------------------------------------------------ output warps
-        const int qd = warp & 3;
         const int half = (warp - kCOut0) >> 2;   // tokens 32 half .. 32 half + 31
-        const int i0 = 32 * qd;
-        float *tab = reinterpret_cast<float *>(sm + C_TAB) + (warp - kCChain0) * 128;
-        unsigned short *ost = reinterpret_cast<unsigned short *>(sm + C_OST + (warp - kCOut0) * 512);
+        const int i = 32 * (warp & 3) + lane;    // value row of this thread
+        float *tab = reinterpret_cast<float *>(sm + C_TAB) + (warp - kCChain0) * 128;  // gamma
+        // o tile [t][i] as two 128B-swizzled 64-column halves, the layout of the store map
+        uint8_t *ost = sm + C_OST;
+        const uint32_t obase = (uint32_t)(i >> 6) * 8192u + (uint32_t)(i & 7) * 2u;
+        const uint32_t ochunk = (uint32_t)((i & 63) >> 3);
+        const bool leader = warp == kCOut0 && lane == 0;
         float2 gnext = nchunks > 0 ? load_g_pair(p.g, bos, chunk_len(0), HV, h) : make_float2(0.f, 0.f);
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t ph = (uint32_t)(c & 1);
@@ -374,8 +389,8 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             const int L = chunk_len(c);
             {
                 const float2 G = warp_decay_scan(gnext.x, gnext.y);
-                tab[64 + 2 * lane] = expf(G.x);
-                tab[64 + 2 * lane + 1] = expf(G.y);
+                tab[2 * lane] = expf(G.x);
+                tab[2 * lane + 1] = expf(G.y);
                 __syncwarp();
             }
             if (c + 1 < nchunks) gnext = load_g_pair(p.g, s0 + C, chunk_len(c + 1), HV, h);
@@ -386,37 +401,54 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             if (warp == kCOut0 && c + 2 < nchunks) {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&bars[CB_R_FULL0 + (c & 1)], SLOT);
-                    mbar_arrive_remote(mapa_shared(sb + P_BAR + PB_GO * 8, 1 + (c + 2) % kNumPrep));
+                    mbar_arrive_remote_relaxed(
+                        mapa_shared(sb + P_BAR + PB_GO * 8, 1 + (c + 2) % kNumPrep));
                 }
                 __syncwarp();
             }
-            {
-                float dq[32], dout[32];
-                tmem_ld32(tmem_addr(tmem, warp, TM_Q + 32 * half), dq);
-                tmem_ld32(tmem_addr(tmem, warp, TM_O + 32 * half), dout);
-#pragma unroll
-                for (int blk = 0; blk < 4; ++blk) {
-#pragma unroll
-                    for (int b = 0; b < 8; ++b) {
-                        const int j = 8 * blk + b;
-                        const float ov = p.scale * fmaf(tab[64 + 32 * half + j], dq[j], dout[j]);
-                        const __nv_bfloat16 bv = __float2bfloat16_rn(ov);
-                        ost[b * 32 + lane] = *reinterpret_cast<const unsigned short *>(&bv);
-                    }
-                    __syncwarp();
-                    const int row = lane >> 2, part = lane & 3;
-                    const int t = 32 * half + 8 * blk + row;
-                    const uint4 val = *reinterpret_cast<const uint4 *>(ost + row * 32 + part * 8);
-                    if (t < L)
-                        *reinterpret_cast<uint4 *>(p.o + ((size_t)(s0 + t) * HV + h) * DH + i0 +
-                                                   part * 8) = val;
-                    __syncwarp();
-                }
-            }
+            float dq[32], dout[32];
+            tmem_ld32(tmem_addr(tmem, warp, TM_Q + 32 * half), dq);
+            tmem_ld32(tmem_addr(tmem, warp, TM_O + 32 * half), dout);
+            // both accumulators are in registers: the next chunk's MMAs may overwrite them
             tc_fence_before();
             __syncwarp();
             if (lane == 0) local_arrive(&bars[CB_Q_FREE]);
+            // the previous chunk's tile store has finished reading the staging tile
+            if (leader) bulk_wait_group_read0();
+            out_sync();
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+                const float4 gm = *reinterpret_cast<const float4 *>(tab + 32 * half + 4 * q4);
+                const float gv[4] = {gm.x, gm.y, gm.z, gm.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 4 * q4 + e, t = 32 * half + j;
+                    const __nv_bfloat16 bv = __float2bfloat16_rn(p.scale * fmaf(gv[e], dq[j], dout[j]));
+                    *reinterpret_cast<__nv_bfloat16 *>(ost + obase + t * 128 +
+                                                       ((ochunk ^ (uint32_t)(t & 7)) << 4)) = bv;
+                }
+            }
+            fence_proxy_async_smem();
+            out_sync();
+            if (L == C) {
+                if (leader) {
+                    tma_store_3d(tm_o, ost, 0, h, (int)s0);
+                    tma_store_3d(tm_o, ost + 8192, 64, h, (int)s0);
+                    bulk_commit_group();
+                }
+            } else {
+                // short last chunk: the rows past the sequence end belong to the next
+                // sequence, so only rows t < L are written, 16 bytes per thread and step
+                for (int e = tid - 32 * kCOut0; e < L * 16; e += kCNumOut * 32) {
+                    const int t = e >> 4, ch = e & 15;
+                    const uint4 val = *reinterpret_cast<const uint4 *>(
+                        ost + (ch >> 3) * 8192 + t * 128 + (((ch & 7) ^ (t & 7)) << 4));
+                    *reinterpret_cast<uint4 *>(p.o + ((size_t)(s0 + t) * HV + h) * DH + ch * 8) = val;
+                }
+            }
         }
+        // the tile stores complete before the CTA (and its shared memory) goes away
+        if (leader) bulk_wait_group0();
     }
 }
 
@@ -712,7 +744,8 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const ClParams p) {
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_o, const ClParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -759,7 +792,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     cluster_sync_all();   // every CTA's barriers are initialised before any remote traffic
 
     if (rank == 0)
-        chain_cta(&tm_q, &tm_k, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
+        chain_cta(&tm_q, &tm_k, &tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
     else
         prep_cta(&tm_q, &tm_k, &tm_v, p, sm, sb, tmem, wt, h, bos, eos, nchunks, rank);
 
@@ -781,7 +814,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     unsigned int *status = static_cast<unsigned int *>(a.workspace);
     cudaError_t err = cudaMemsetAsync(status, 0, sizeof(unsigned int), stream);
     if (err != cudaSuccess) return err;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     const uint64_t tok = (uint64_t)(Ttot > 0 ? Ttot : 1);
     uint64_t dq[3] = {(uint64_t)DH, (uint64_t)a.HK, tok};
     uint64_t sq[2] = {(uint64_t)DH * 2, (uint64_t)a.HK * DH * 2};
@@ -789,7 +822,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     uint64_t sv[2] = {(uint64_t)DH * 2, (uint64_t)a.HV * DH * 2};
     uint32_t box[3] = {64, 1, 64};
     if (!encode_bf16_map(&tq, a.q, 3, dq, sq, box) || !encode_bf16_map(&tk, a.k, 3, dq, sq, box) ||
-        !encode_bf16_map(&tv, a.v, 3, dv, sv, box))
+        !encode_bf16_map(&tv, a.v, 3, dv, sv, box) || !encode_bf16_map(&to, a.o, 3, dv, sv, box))
         return cudaErrorInvalidValue;
     err = cudaFuncSetAttribute(prefill_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)SMEM_BYTES);
@@ -808,7 +841,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, prefill_cluster_kernel, tq, tk, tv, prm);
+    err = cudaLaunchKernelEx(&cfg, prefill_cluster_kernel, tq, tk, tv, to, prm);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }

@@ -25,9 +25,10 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // bf16 tensor of `rank` dims (dims[0] innermost), byte strides of dims 1..rank-1,
-// box dims, 128-byte swizzle, zero fill outside the tensor.
+// box dims, 128-byte swizzle unless told otherwise, zero fill outside the tensor.
 inline bool encode_bf16_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
-                            const uint64_t *strides_bytes, const uint32_t *box) {
+                            const uint64_t *strides_bytes, const uint32_t *box,
+                            CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
@@ -35,7 +36,7 @@ inline bool encode_bf16_map(CUtensorMap *map, const void *base, int rank, const 
                      const_cast<void *>(base), reinterpret_cast<const cuuint64_t *>(dims),
                      reinterpret_cast<const cuuint64_t *>(strides_bytes),
                      reinterpret_cast<const cuuint32_t *>(box), estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
