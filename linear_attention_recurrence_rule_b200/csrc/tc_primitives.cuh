@@ -143,7 +143,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
     return d;
 }
-// Arrive (release, cluster scope) on an mbarrier of another CTA of the cluster.
 // Relaxed arrive on another cluster CTA's mbarrier: a signal that orders none of
 // this thread's own memory operations (a release arrive costs ~1.1-1.5K cycles
 // here).  Use it only where the waiting CTA reads nothing this thread wrote:
@@ -162,6 +161,14 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint3
         "[%3];" ::"r"(dst_cluster),
         "r"(src_cta), "r"(bytes), "r"(mbar_cluster)
         : "memory");
+}
+// Store a word into the shared memory of a cluster CTA (address from mapa_shared).
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// Named barrier `id` over `count` threads (whole warps); every participant waits.
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 // Every thread of every CTA of the cluster.
 __device__ __forceinline__ void cluster_sync_all() {
@@ -282,6 +289,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&w)[32
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&p);
+}
+// 32 lanes x 32 bit, 8 consecutive columns per thread (raw words).
+__device__ __forceinline__ void tmem_st8w(uint32_t taddr, const uint32_t (&w)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+        : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
