@@ -71,35 +71,43 @@ constexpr uint32_t NB_OUT = 4;                        // epilogue warps
 constexpr uint32_t kChainSync = (kCNumEpi + 1) * 32;
 constexpr uint32_t kEpiSync = kCNumEpi * 32;
 
-// ---- one chunk's hand-over block (prep staging == chain receive slot) ----
+// ---- chain receive slot of one chunk: Q and K by TMA, the rest from a prep CTA ----
 constexpr uint32_t SL_WQ = 0;       // [W;Q] K-major: per 64-column half 16 KB, W rows then Q rows
 constexpr uint32_t SL_K = 32768;    // K as loaded (rows t, two 64-column halves), MN-major B
 constexpr uint32_t SL_PH = 49152;   // P hi: 64 rows (t) x 64 (s), K-major
 constexpr uint32_t SL_PL = 57344;   // P lo
 constexpr uint32_t SL_U = 65536;    // U~ fp32 [i][t], 16-byte chunks xor-swizzled by row
 constexpr uint32_t SL_TAB = 98304;  // fp32: gamma_L/gamma_t [64], gamma_t [64], gamma_L
-constexpr uint32_t SLOT = 99328;    // bytes per block (a multiple of 1024: slots stay swizzle-aligned)
+constexpr uint32_t SLOT = 99328;    // bytes per slot (a multiple of 1024: slots stay swizzle-aligned)
+// the prep CTA's staging block (what its bulk copies carry) and where each piece lands
+constexpr uint32_t ST_W = 0;        // W rows, two 64-column halves of 8 KB -> SL_WQ, SL_WQ + 16384
+constexpr uint32_t ST_P = 16384;    // P hi, P lo -> SL_PH
+constexpr uint32_t ST_U = 32768;    // U~ -> SL_U
+constexpr uint32_t ST_TAB = 65536;  // decay table -> SL_TAB
+constexpr uint32_t ST_BYTES = 66560;
+constexpr uint32_t QK_BYTES = 4 * 8192;            // Q and K tiles loaded by the chain CTA
+constexpr uint32_t SLOT_TX = ST_BYTES + QK_BYTES;  // bytes that complete one receive slot
 
 // ---- chain CTA shared memory ----
 constexpr uint32_t C_R = 0;                                 // 2 receive slots
 constexpr uint32_t C_OST = C_R + 2 * SLOT;                  // o tile staging (TMA store)
 constexpr uint32_t C_BAR = C_OST + 16384;
 // ---- prep CTA shared memory ----
-constexpr uint32_t P_QK = 0;        // [Q half 0 | K half 0][Q half 1 | K half 1]
-constexpr uint32_t P_V = 32768;
-constexpr uint32_t P_T = 49152;     // T' hi, T' lo, T'' hi, T'' lo (4 x 8 KB); A fp32 shares it
+// two q/k/v buffers of 48 KB: [Q half 0 | K half 0][Q half 1 | K half 1][V]
+constexpr uint32_t P_QKV = 0, QKV_STRIDE = 49152, QKV_V = 32768;
+constexpr uint32_t P_T = 98304;     // T' hi, T' lo, T'' hi, T'' lo (4 x 8 KB); A fp32 shares it
 constexpr uint32_t A_LD = 68;
-constexpr uint32_t P_TF = 81920;    // T fp32 [64][T_LD]
+constexpr uint32_t P_TF = 131072;   // T fp32 [64][T_LD]
 constexpr uint32_t T_LD = 68;
 constexpr uint32_t P_X = P_TF + 64 * T_LD * 4;
 constexpr uint32_t X_LD = 36;
 constexpr uint32_t P_PB = P_X + 32 * X_LD * 4;             // beta, gamma, G
-constexpr uint32_t P_ST = 105472;   // staging block (SLOT bytes)
-constexpr uint32_t P_BAR = P_ST + SLOT;
+constexpr uint32_t P_ST = 154624;   // staging block (ST_BYTES)
+constexpr uint32_t P_BAR = P_ST + ST_BYTES;
 
 enum ChainBar { CB_R_FULL0, CB_R_FULL1, CB_U_MMA, CB_DS_FULL, CB_O_FULL, CB_DRAIN, CB_COUNT };
-enum PrepBar { PB_LD_FULL, PB_X_DONE, PB_T_READY, PB_WU_DONE, PB_EPI_DONE, PB_GO, PB_STAGE_FREE,
-               PB_DRAIN, PB_COUNT };
+enum PrepBar { PB_LD_FULL0, PB_LD_FULL1, PB_X_DONE, PB_T_READY, PB_WU_DONE, PB_EPI_DONE, PB_GO,
+               PB_STAGE_FREE, PB_DRAIN, PB_COUNT };
 
 // words at the same offset in every CTA: TMEM base, abort flag, slot bookkeeping
 constexpr uint32_t AUX_RAW = (C_BAR + CB_COUNT * 8 > P_BAR + PB_COUNT * 8) ? C_BAR + CB_COUNT * 8
@@ -112,6 +120,7 @@ static_assert(P_PB + 3 * 64 * 4 <= P_ST, "prep layout");
 static_assert(64 * A_LD * 4 <= 32768, "A fits the T tiles");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(C_OST % 1024 == 0 && P_ST % 1024 == 0 && SLOT % 1024 == 0, "swizzle alignment");
+static_assert(P_PB + 3 * 64 * 4 <= P_ST && P_X + 32 * X_LD * 4 <= P_PB, "prep layout");
 
 // ---- TMEM columns ----
 // chain: S0 [W;Q]^T (D = S0 W^T, then S0 Q^T), U P^T, S0 (bf16 A operand), S (fp32),
@@ -170,12 +179,27 @@ __device__ __forceinline__ uint32_t ut_chunk(uint32_t i, uint32_t tc) {
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
 // ============================================================================ chain CTA
-__device__ void chain_cta(const CUtensorMap *tm_o, const ClParams &p, uint8_t *sm, uint32_t sb,
-                          uint32_t tmem, const Waiter &wt, int h, int n, int64_t bos, int64_t eos,
-                          int nchunks) {
+// Q and K tiles of chunk c into its receive slot (completing on that slot's mbarrier)
+__device__ __forceinline__ void load_qk_slot(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                             uint8_t *sm, uint64_t *bars, int c, int cqk,
+                                             int64_t bos) {
+    const int s = c & 1;
+    uint8_t *slot = sm + C_R + s * SLOT;
+    uint64_t *bar = &bars[CB_R_FULL0 + s];
+    const int s0 = (int)(bos + (int64_t)c * C);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        tma_load_3d(slot + SL_WQ + hf * 16384 + 8192, tm_q, bar, 64 * hf, cqk, s0);
+        tma_load_3d(slot + SL_K + hf * 8192, tm_k, bar, 64 * hf, cqk, s0);
+    }
+}
+
+__device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_o,
+                          const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
+                          const Waiter &wt, int h, int n, int64_t bos, int64_t eos, int nchunks) {
     uint64_t *bars = wt.bars;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int HV = p.HV;
+    const int HV = p.HV, cqk = h / (HV / p.HK);
     const size_t sbase = ((size_t)n * HV + h) * (size_t)DH * DH;
     volatile int *armed = reinterpret_cast<volatile int *>(sm + AUX_ARMED);
     volatile int *consumed = reinterpret_cast<volatile int *>(sm + AUX_CONSUMED);
@@ -443,8 +467,9 @@ __device__ void chain_cta(const CUtensorMap *tm_o, const ClParams &p, uint8_t *s
             ok = warp_all(ok && wt(CB_O_FULL, ph));
             if (ok && warp == kCEpi0 && c + 2 < nchunks) {
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&bars[CB_R_FULL0 + (c & 1)], SLOT);
+                    mbar_arrive_expect_tx(&bars[CB_R_FULL0 + (c & 1)], SLOT_TX);
                     *armed = c + 3;
+                    load_qk_slot(tm_q, tm_k, sm, bars, c + 2, cqk, bos);
                     mbar_arrive_remote_relaxed(
                         mapa_shared(sb + P_BAR + PB_GO * 8, 1 + (c + 2) % kNumPrep));
                 }
@@ -501,17 +526,19 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             if (elect_one()) mma_commit(&bars[b]);
             __syncwarp();
         };
-        int issued = 0, landed = 0;    // q/k/v loads issued / waited for
-        auto load = [&](int c) {
+        int issued = 0, landed = 0;    // q/k/v loads issued / waited for (k-th into buffer k & 1)
+        auto load = [&](int k) {
             if (lane == 0) {
-                const int s0 = (int)(bos + (int64_t)c * C);
-                mbar_arrive_expect_tx(&bars[PB_LD_FULL], 6 * 8192);
-                tma_load_3d(sm + P_QK, tm_q, &bars[PB_LD_FULL], 0, cqk, s0);
-                tma_load_3d(sm + P_QK + 16384, tm_q, &bars[PB_LD_FULL], 64, cqk, s0);
-                tma_load_3d(sm + P_QK + 8192, tm_k, &bars[PB_LD_FULL], 0, cqk, s0);
-                tma_load_3d(sm + P_QK + 24576, tm_k, &bars[PB_LD_FULL], 64, cqk, s0);
-                tma_load_3d(sm + P_V, tm_v, &bars[PB_LD_FULL], 0, h, s0);
-                tma_load_3d(sm + P_V + 8192, tm_v, &bars[PB_LD_FULL], 64, h, s0);
+                const int s0 = (int)(bos + (int64_t)chunk_of(k) * C);
+                uint64_t *bar = &bars[PB_LD_FULL0 + (k & 1)];
+                uint8_t *buf = sm + P_QKV + (k & 1) * QKV_STRIDE;
+                mbar_arrive_expect_tx(bar, 6 * 8192);
+                tma_load_3d(buf, tm_q, bar, 0, cqk, s0);
+                tma_load_3d(buf + 16384, tm_q, bar, 64, cqk, s0);
+                tma_load_3d(buf + 8192, tm_k, bar, 0, cqk, s0);
+                tma_load_3d(buf + 24576, tm_k, bar, 64, cqk, s0);
+                tma_load_3d(buf + QKV_V, tm_v, bar, 0, h, s0);
+                tma_load_3d(buf + QKV_V + 8192, tm_v, bar, 64, h, s0);
             }
             __syncwarp();
             ++issued;
@@ -522,19 +549,22 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 tma_prefetch_desc(tm_k);
                 tma_prefetch_desc(tm_v);
             }
-            load(chunk_of(0));
+            load(0);
         }
         for (int k = 0; k < nk; ++k) {
             const int c = chunk_of(k);
             const uint32_t ph = (uint32_t)(k & 1);
-            if (!warp_all(wt(PB_LD_FULL, ph))) break;
+            const uint32_t qkv = sb + P_QKV + (k & 1) * QKV_STRIDE;
+            if (!warp_all(wt(PB_LD_FULL0 + (k & 1), (uint32_t)((k >> 1) & 1)))) break;
             ++landed;
+            // the other buffer's chunk (k - 1) finished its W/U products: load chunk k + 1
+            if (k + 1 < nk) load(k + 1);
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                const uint64_t a = sdesc_sw128(sb + P_QK + off, 16, 1024);
-                const uint64_t b = sdesc_sw128(sb + P_QK + 8192 + off, 16, 1024);
+                const uint64_t a = sdesc_sw128(qkv + off, 16, 1024);
+                const uint64_t b = sdesc_sw128(qkv + 8192 + off, 16, 1024);
                 if (elect_one()) mma_bf16(tmem + TP_D1, a, b, id_x, kk > 0);
                 __syncwarp();
             }
@@ -543,8 +573,8 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ka = sdesc_sw128(sb + P_QK + 8192 + kk * 2048, 16384, 1024);
-                const uint64_t va = sdesc_sw128(sb + P_V + kk * 2048, 8192, 1024);
+                const uint64_t ka = sdesc_sw128(qkv + 8192 + kk * 2048, 16384, 1024);
+                const uint64_t va = sdesc_sw128(qkv + QKV_V + kk * 2048, 8192, 1024);
                 const uint64_t t1h = sdesc_sw128(sb + P_T + kk * 32, 16, 1024);
                 const uint64_t t1l = sdesc_sw128(sb + P_T + 8192 + kk * 32, 16, 1024);
                 const uint64_t t2h = sdesc_sw128(sb + P_T + 16384 + kk * 32, 16, 1024);
@@ -558,8 +588,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 __syncwarp();
             }
             commit(PB_WU_DONE);
-            if (!warp_all(wt(PB_WU_DONE, ph))) break;   // q/k/v tiles are free again
-            if (k + 1 < nk) load(chunk_of(k + 1));
+            if (!warp_all(wt(PB_WU_DONE, ph))) break;   // this buffer's q/k/v tiles are free again
             if (!warp_all(wt(PB_EPI_DONE, ph))) break;
             if (c >= 2) {
                 const int j = first >= 2 ? k : k - 1;   // go arrivals before this chunk
@@ -569,16 +598,18 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 const int s = c & 1;
                 const uint32_t mbar = mapa_shared(sb + C_BAR + (CB_R_FULL0 + s) * 8, 0);
                 const uint32_t dst = mapa_shared(sb + C_R + s * SLOT, 0);
-#pragma unroll
-                for (int part = 0; part < (int)(SL_TAB / 16384); ++part)
-                    bulk_copy_to_cluster(dst + part * 16384, sb + P_ST + part * 16384, 16384, mbar);
-                bulk_copy_to_cluster(dst + SL_TAB, sb + P_ST + SL_TAB, SLOT - SL_TAB, mbar);
+                const uint32_t st = sb + P_ST;
+                bulk_copy_to_cluster(dst + SL_WQ, st + ST_W, 8192, mbar);
+                bulk_copy_to_cluster(dst + SL_WQ + 16384, st + ST_W + 8192, 8192, mbar);
+                bulk_copy_to_cluster(dst + SL_PH, st + ST_P, 16384, mbar);
+                bulk_copy_to_cluster(dst + SL_U, st + ST_U, 32768, mbar);
+                bulk_copy_to_cluster(dst + SL_TAB, st + ST_TAB, ST_BYTES - ST_TAB, mbar);
             }
             __syncwarp();
         }
         // after an abort: a load still in flight lands, and issued MMAs complete,
         // before this CTA's shared and tensor memory are released
-        if (landed < issued) wt.drain(PB_LD_FULL, (uint32_t)(landed & 1));
+        for (int d = landed; d < issued; ++d) wt.drain(PB_LD_FULL0 + (d & 1), (uint32_t)((d >> 1) & 1));
         commit(PB_DRAIN);
         wt.drain(PB_DRAIN, 0);
     } else if (warp < kPWork0 + kPNumWork) {
@@ -611,9 +642,9 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 beta_s[2 * lane] = bp.x;
                 beta_s[2 * lane + 1] = bp.y;
             }
-            // the q/k tiles have landed (read below), the X product is done, and the
-            // staging block's previous contents have been copied out
-            ok = warp_all(ok && wt(PB_LD_FULL, ph) && wt(PB_X_DONE, ph) &&
+            // the X product is done and the staging block's previous contents have
+            // been copied out
+            ok = warp_all(ok && wt(PB_X_DONE, ph) &&
                           (k == 0 || wt(PB_STAGE_FREE, (uint32_t)((k - 1) & 1))));
             named_sync(NB_WORK, kPWorkThreads);
             if (ok) {
@@ -640,7 +671,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         const uint32_t off = sw128_chunk(row, 2 * qtr + cc);
-                        st_chunk_hilo(sb + P_ST + SL_PH + off, sb + P_ST + SL_PL + off, v + 8 * cc);
+                        st_chunk_hilo(sb + P_ST + ST_P + off, sb + P_ST + ST_P + 8192 + off, v + 8 * cc);
                     }
                 } else {
                     const float bi = beta_s[row];
@@ -661,20 +692,10 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 }
                 // decay table of this chunk for the chain CTA
                 if (pt < 64) {
-                    float *tb = reinterpret_cast<float *>(sm + P_ST + SL_TAB);
+                    float *tb = reinterpret_cast<float *>(sm + P_ST + ST_TAB);
                     tb[pt] = __expf(G_p[63] - G_p[pt]);    // gamma_L / gamma_t
                     tb[64 + pt] = gam_p[pt];               // gamma_t
                     if (pt == 0) tb[128] = gam_p[63];      // gamma_L
-                }
-                // Q (next to W in the [W;Q] operand) and K into the staging block
-#pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    const int e = pt + 512 * e4;            // 16-byte chunk 0..2047
-                    const int isk = e >> 10, hf = (e >> 9) & 1, off = (e & 511) * 16;
-                    const uint4 val =
-                        *reinterpret_cast<const uint4 *>(sm + P_QK + hf * 16384 + isk * 8192 + off);
-                    uint8_t *dst = sm + P_ST + (isk ? SL_K + hf * 8192 : SL_WQ + hf * 16384 + 8192) + off;
-                    *reinterpret_cast<uint4 *>(dst) = val;
                 }
             }
             tc_fence_before();
@@ -773,7 +794,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 // W^T row a = r, tokens t = 16 qtr + j -> W rows of the K-major [W;Q] operand
                 tmem_ld16(tmem_addr(tmem, warp, TP_D1 + 16 * qtr), v);
                 tmem_wait_ld();
-                uint8_t *wq = sm + P_ST + SL_WQ + (r >> 6) * 16384 + (r & 7) * 2;
+                uint8_t *wq = sm + P_ST + ST_W + (r >> 6) * 8192 + (r & 7) * 2;
                 const uint32_t wc = (uint32_t)((r & 63) >> 3);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
@@ -784,7 +805,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 // U~^T row i = r, tokens 16 qtr .. (fp32)
                 tmem_ld16(tmem_addr(tmem, warp, TP_U + 16 * qtr), v);
                 tmem_wait_ld();
-                uint8_t *ut = sm + P_ST + SL_U;
+                uint8_t *ut = sm + P_ST + ST_U;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4)
                     *reinterpret_cast<float4 *>(ut + ut_chunk(r, 4 * qtr + q4)) =
@@ -836,7 +857,12 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (rank == 0) {
             // receive slots for chunks 0 and 1 expect their bytes from the start
             const int pre = nchunks < 2 ? nchunks : 2;
-            for (int c = 0; c < pre; ++c) mbar_arrive_expect_tx(&bars[CB_R_FULL0 + c], SLOT);
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            for (int c = 0; c < pre; ++c) {
+                mbar_arrive_expect_tx(&bars[CB_R_FULL0 + c], SLOT_TX);
+                load_qk_slot(&tm_q, &tm_k, sm, bars, c, h / (p.HV / p.HK), bos);
+            }
             *reinterpret_cast<volatile int *>(sm + AUX_ARMED) = pre;
             *reinterpret_cast<volatile int *>(sm + AUX_CONSUMED) = 0;
         }
@@ -849,7 +875,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     cluster_sync_all();   // every CTA's barriers are initialised before any remote traffic
 
     if (rank == 0)
-        chain_cta(&tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
+        chain_cta(&tm_q, &tm_k, &tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
     else
         prep_cta(&tm_q, &tm_k, &tm_v, p, sm, sb, tmem, wt, h, bos, eos, nchunks, rank);
 
