@@ -14,16 +14,18 @@
 // Split by dependence on the state:
 //   prep CTAs (cluster ranks 1..3) take every third chunk and compute the
 //     state-independent part: [Q;K]K^T, A and P, the UT inverse T (blocked
-//     16 -> 32 -> 64 on CUDA cores), W^T and U~^T (tcgen05), and ship one 96 KB
-//     block per chunk -- [W;Q] as one K-major operand, K, P (bf16 hi + lo) and
-//     U~ (fp32) -- into the chain CTA's shared memory with bulk DSMEM copies
-//     that complete on the chain CTA's mbarrier;
+//     16 -> 32 -> 64 on CUDA cores), W^T and U~^T (tcgen05), and ship 65 KB per
+//     chunk -- W (next to Q in one K-major [W;Q] operand), P (bf16 hi + lo),
+//     U~ (fp32) and the chunk's decay table -- into the chain CTA's receive slot
+//     with bulk DSMEM copies that complete on the chain CTA's mbarrier, where
+//     the chain CTA's own TMA loads of the chunk's Q and K also land;
 //   the chain CTA (rank 0) walks the chunks in order: one N = 128 product
 //     S0 [W;Q]^T gives S0 W^T and S0 Q^T together (S0 as a bf16 operand in
 //     tensor memory), U = U~ - S0 W^T, the state update S += (U diag(gamma_L /
 //     gamma)) K accumulated in tensor memory after an in-place gamma_L scaling,
-//     and the outputs U P^T + gamma_t S0 Q^T, staged in shared memory by eight
-//     output warps and written with TMA stores.
+//     and the outputs gamma_t S0 Q^T + U P^T; sixteen epilogue warps share every
+//     epilogue (16 tokens or 32 state columns each) and write chunk c's outputs
+//     while chunk c + 1's first product runs.
 // The chain's critical loop hands over between its epilogue warps and the
 // MMA-issuing warp through named barriers (no sleeping wake-up on that path);
 // tensor-core completions and cross-CTA hand-overs use mbarriers.
@@ -67,9 +69,7 @@ constexpr uint32_t kDrain = 50;    // polls for a drain of in-flight work after 
 // named barriers (0 is __syncthreads)
 constexpr uint32_t NB_WORK = 1;                       // prep workers
 constexpr uint32_t NB_S0 = 1, NB_U = 2, NB_U2 = 3;    // epilogue warps + MMA warp
-constexpr uint32_t NB_OUT = 4;                        // epilogue warps
 constexpr uint32_t kChainSync = (kCNumEpi + 1) * 32;
-constexpr uint32_t kEpiSync = kCNumEpi * 32;
 
 // ---- chain receive slot of one chunk: Q and K by TMA, the rest from a prep CTA ----
 constexpr uint32_t SL_WQ = 0;       // [W;Q] K-major: per 64-column half 16 KB, W rows then Q rows
@@ -90,8 +90,7 @@ constexpr uint32_t SLOT_TX = ST_BYTES + QK_BYTES;  // bytes that complete one re
 
 // ---- chain CTA shared memory ----
 constexpr uint32_t C_R = 0;                                 // 2 receive slots
-constexpr uint32_t C_OST = C_R + 2 * SLOT;                  // o tile staging (TMA store)
-constexpr uint32_t C_BAR = C_OST + 16384;
+constexpr uint32_t C_BAR = C_R + 2 * SLOT;
 // ---- prep CTA shared memory ----
 // two q/k/v buffers of 48 KB: [Q half 0 | K half 0][Q half 1 | K half 1][V]
 constexpr uint32_t P_QKV = 0, QKV_STRIDE = 49152, QKV_V = 32768;
@@ -119,7 +118,7 @@ constexpr uint32_t SMEM_BYTES = AUX + 16 + 1024;
 static_assert(P_PB + 3 * 64 * 4 <= P_ST, "prep layout");
 static_assert(64 * A_LD * 4 <= 32768, "A fits the T tiles");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(C_OST % 1024 == 0 && P_ST % 1024 == 0 && SLOT % 1024 == 0, "swizzle alignment");
+static_assert(P_ST % 1024 == 0 && SLOT % 1024 == 0, "swizzle alignment");
 static_assert(P_PB + 3 * 64 * 4 <= P_ST && P_X + 32 * X_LD * 4 <= P_PB, "prep layout");
 
 // ---- TMEM columns ----
@@ -194,8 +193,7 @@ __device__ __forceinline__ void load_qk_slot(const CUtensorMap *tm_q, const CUte
     }
 }
 
-__device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_o,
-                          const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
+__device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
                           const Waiter &wt, int h, int n, int64_t bos, int64_t eos, int nchunks) {
     uint64_t *bars = wt.bars;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -287,11 +285,6 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
         // 64-token products, state columns 32 part .. 32 part + 31.
         const int part = (warp - kCEpi0) >> 2;
         const int i = 32 * (warp & 3) + lane;
-        // o tile [t][i] as two 128B-swizzled 64-column halves, the layout of the store map
-        uint8_t *ost = sm + C_OST;
-        const uint32_t obase = (uint32_t)(i >> 6) * 8192u + (uint32_t)(i & 7) * 2u;
-        const uint32_t ochunk = (uint32_t)((i & 63) >> 3);
-        const bool leader = warp == kCEpi0 && lane == 0;
         {
             // start state: fp32 (scaled at the start of chunk 0) and its bf16 copy (chunk 0's S0)
             const float *src = p.h0 ? p.h0 + sbase + (size_t)i * DH + 32 * part : nullptr;
@@ -314,51 +307,25 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
         }
         tc_fence_before();
         if (nchunks > 0) named_sync(NB_S0, kChainSync);
-        // the read-out of chunk c is computed at the end of chunk c (8 words of bf16
-        // pairs: tokens 16 part + 2w, 2w + 1) and stored during chunk c + 1
-        auto store_out = [&](const uint32_t (&opk)[8], bool have, int64_t os0, int oL) {
-            // the previous tile store has finished reading the staging tile
-            if (leader) bulk_wait_group_read0();
-            named_sync(NB_OUT, kEpiSync);
-            if (have) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int t = 16 * part + j;
-                    const unsigned short bits = (unsigned short)((j & 1) ? (opk[j >> 1] >> 16) : (opk[j >> 1] & 0xffffu));
-                    *reinterpret_cast<unsigned short *>(ost + obase + t * 128 +
-                                                        ((ochunk ^ (uint32_t)(t & 7)) << 4)) = bits;
-                }
-            }
-            fence_proxy_async_smem();
-            named_sync(NB_OUT, kEpiSync);
-            if (have) {
-                if (oL == C) {
-                    if (leader) {
-                        tma_store_3d(tm_o, ost, 0, h, (int)os0);
-                        tma_store_3d(tm_o, ost + 8192, 64, h, (int)os0);
-                        bulk_commit_group();
-                    }
-                } else {
-                    // short last chunk: the rows past the sequence end belong to the next
-                    // sequence, so only rows t < oL are written, 16 bytes per thread and step
-                    for (int e = tid - 32 * kCEpi0; e < oL * 16; e += kEpiSync) {
-                        const int t = e >> 4, ch = e & 15;
-                        const uint4 val = *reinterpret_cast<const uint4 *>(
-                            ost + (ch >> 3) * 8192 + t * 128 + (((ch & 7) ^ (t & 7)) << 4));
-                        *reinterpret_cast<uint4 *>(p.o + ((size_t)(os0 + t) * HV + h) * DH + ch * 8) = val;
-                    }
-                }
-            }
-        };
         bool ok = true;
-        uint32_t opk[8];
-        bool pend = false;       // the read-out of the previous chunk is waiting to be stored
-        int64_t ps0 = 0;
-        int pL = 0;
+        float dq[16];            // scale * gamma_t * (S0 q_t) of the previous chunk
+        // read-out of chunk cp: o_t = dq + scale (U P^T)_t, written straight from
+        // registers (each warp store covers 32 consecutive value rows of one token)
+        auto read_out = [&](int cp) {
+            const int64_t ps0 = bos + (int64_t)cp * C;
+            const int pL = chunk_len(cp);
+            float dout[16];
+            tmem_ld16(tmem_addr(tmem, warp, TM_O + 16 * part), dout);
+            tmem_wait_ld();
+            __nv_bfloat16 *dst = p.o + ((size_t)(ps0 + 16 * part) * HV + h) * DH + i;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (16 * part + j < pL)
+                    dst[(size_t)j * HV * DH] = __float2bfloat16_rn(fmaf(p.scale, dout[j], dq[j]));
+        };
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t ph = (uint32_t)(c & 1);
             const int s = c & 1;
-            const int64_t s0 = bos + (int64_t)c * C;
             const int L = chunk_len(c);
             const uint8_t *slot = sm + C_R + s * SLOT;
             const float *tab = reinterpret_cast<const float *>(slot + SL_TAB);
@@ -371,6 +338,27 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] *= gL;
                 tmem_st32f(tmem_addr(tmem, warp, TM_S + 32 * part), v);
+            }
+            if (c > 0) {
+                // the previous chunk's U P^T is done: every read of its receive slot is
+                // over, so re-arm that slot and release the prep CTA that produces chunk
+                // c + 1 into it; then write the previous chunk's outputs (its
+                // accumulator is overwritten only after this chunk's second barrier)
+                ok = warp_all(ok && wt(CB_O_FULL, (uint32_t)((c - 1) & 1)));
+                if (ok) {
+                    tc_fence_after();
+                    if (warp == kCEpi0 && c + 1 < nchunks) {
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&bars[CB_R_FULL0 + ((c + 1) & 1)], SLOT_TX);
+                            *armed = c + 2;
+                            load_qk_slot(tm_q, tm_k, sm, bars, c + 1, cqk, bos);
+                            mbar_arrive_remote_relaxed(
+                                mapa_shared(sb + P_BAR + PB_GO * 8, 1 + (c + 1) % kNumPrep));
+                        }
+                        __syncwarp();
+                    }
+                    read_out(c - 1);
+                }
             }
             ok = warp_all(ok && wt(CB_U_MMA, ph));
             float u[16];
@@ -430,11 +418,8 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             }
             tc_fence_before();
             named_sync(NB_U2, kChainSync);    // U P^T can start
-            // the previous chunk's read-out goes out while the state update runs
-            if (pend) store_out(opk, ok, ps0, pL);
             const bool more = c + 1 < nchunks;
             ok = warp_all(ok && wt(CB_DS_FULL, ph));
-            float dq[16];
             if (ok) {
                 tc_fence_after();
                 if (more) {
@@ -446,50 +431,30 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                     for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
                     tmem_st16w(tmem_addr(tmem, warp, TM_S0 + 16 * part), w);
                 }
-                // scale gamma_t S0 q_t of this part's tokens, read before the next
+                // scale * gamma_t * S0 q_t of this part's tokens, read before the next
                 // chunk's MMAs overwrite it (gamma_t from the slot, still held)
                 tmem_ld16(tmem_addr(tmem, warp, TM_Q + 16 * part), dq);
                 tmem_wait_ld();
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const float4 g4 = *reinterpret_cast<const float4 *>(tab + 64 + 16 * part + 4 * q4);
-                    dq[4 * q4] *= g4.x;
-                    dq[4 * q4 + 1] *= g4.y;
-                    dq[4 * q4 + 2] *= g4.z;
-                    dq[4 * q4 + 3] *= g4.w;
+                    dq[4 * q4] *= p.scale * g4.x;
+                    dq[4 * q4 + 1] *= p.scale * g4.y;
+                    dq[4 * q4 + 2] *= p.scale * g4.z;
+                    dq[4 * q4 + 3] *= p.scale * g4.w;
                 }
                 tmem_wait_st();
             }
             tc_fence_before();
             if (more) named_sync(NB_S0, kChainSync);
-            // every read of the receive slot of chunk c is done once the U P^T product
-            // completes: re-arm the slot and release the prep CTA that produces chunk c + 2
-            ok = warp_all(ok && wt(CB_O_FULL, ph));
-            if (ok && warp == kCEpi0 && c + 2 < nchunks) {
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&bars[CB_R_FULL0 + (c & 1)], SLOT_TX);
-                    *armed = c + 3;
-                    load_qk_slot(tm_q, tm_k, sm, bars, c + 2, cqk, bos);
-                    mbar_arrive_remote_relaxed(
-                        mapa_shared(sb + P_BAR + PB_GO * 8, 1 + (c + 2) % kNumPrep));
-                }
-                __syncwarp();
-            }
+        }
+        if (nchunks > 0) {
+            ok = warp_all(ok && wt(CB_O_FULL, (uint32_t)((nchunks - 1) & 1)));
             if (ok) {
                 tc_fence_after();
-                float dout[16];
-                tmem_ld16(tmem_addr(tmem, warp, TM_O + 16 * part), dout);
-                tmem_wait_ld();
-#pragma unroll
-                for (int w = 0; w < 8; ++w)
-                    opk[w] = pack_bf16x2(p.scale * (dq[2 * w] + dout[2 * w]),
-                                         p.scale * (dq[2 * w + 1] + dout[2 * w + 1]));
+                read_out(nchunks - 1);
             }
-            pend = true;
-            ps0 = s0;
-            pL = L;
         }
-        if (pend) store_out(opk, ok, ps0, pL);
         if (ok && p.hT) {
             tc_fence_after();
             float v[32];
@@ -499,8 +464,6 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             for (int j = 0; j < 32; j += 4)
                 *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
-        // the tile stores complete before the CTA (and its shared memory) goes away
-        if (leader) bulk_wait_group0();
     }
 }
 
@@ -822,8 +785,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v,
-                       const __grid_constant__ CUtensorMap tm_o, const ClParams p) {
+                       const __grid_constant__ CUtensorMap tm_v, const ClParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -875,7 +837,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     cluster_sync_all();   // every CTA's barriers are initialised before any remote traffic
 
     if (rank == 0)
-        chain_cta(&tm_q, &tm_k, &tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
+        chain_cta(&tm_q, &tm_k, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
     else
         prep_cta(&tm_q, &tm_k, &tm_v, p, sm, sb, tmem, wt, h, bos, eos, nchunks, rank);
 
@@ -904,7 +866,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     unsigned int *status = static_cast<unsigned int *>(a.workspace);
     cudaError_t err = cudaMemsetAsync(status, 0, sizeof(unsigned int), stream);
     if (err != cudaSuccess) return err;
-    CUtensorMap tq, tk, tv, to;
+    CUtensorMap tq, tk, tv;
     const uint64_t tok = (uint64_t)(Ttot > 0 ? Ttot : 1);
     uint64_t dq[3] = {(uint64_t)DH, (uint64_t)a.HK, tok};
     uint64_t sq[2] = {(uint64_t)DH * 2, (uint64_t)a.HK * DH * 2};
@@ -912,7 +874,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     uint64_t sv[2] = {(uint64_t)DH * 2, (uint64_t)a.HV * DH * 2};
     uint32_t box[3] = {64, 1, 64};
     if (!encode_bf16_map(&tq, a.q, 3, dq, sq, box) || !encode_bf16_map(&tk, a.k, 3, dq, sq, box) ||
-        !encode_bf16_map(&tv, a.v, 3, dv, sv, box) || !encode_bf16_map(&to, a.o, 3, dv, sv, box))
+        !encode_bf16_map(&tv, a.v, 3, dv, sv, box))
         return cudaErrorInvalidValue;
     err = cudaFuncSetAttribute(prefill_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)SMEM_BYTES);
@@ -931,7 +893,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, prefill_cluster_kernel, tq, tk, tv, to, prm);
+    err = cudaLaunchKernelEx(&cfg, prefill_cluster_kernel, tq, tk, tv, prm);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
