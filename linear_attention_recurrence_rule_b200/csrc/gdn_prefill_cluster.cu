@@ -90,7 +90,8 @@ constexpr uint32_t SLOT_TX = ST_BYTES + QK_BYTES;  // bytes that complete one re
 
 // ---- chain CTA shared memory ----
 constexpr uint32_t C_R = 0;                                 // 2 receive slots
-constexpr uint32_t C_BAR = C_R + 2 * SLOT;
+constexpr uint32_t C_OT = C_R + 2 * SLOT;   // per epilogue warp: 16 x 32 bf16 output tile
+constexpr uint32_t C_BAR = C_OT + kCNumEpi * 1024;
 // ---- prep CTA shared memory ----
 // two q/k/v buffers of 48 KB: [Q half 0 | K half 0][Q half 1 | K half 1][V]
 constexpr uint32_t P_QKV = 0, QKV_STRIDE = 49152, QKV_V = 32768;
@@ -147,6 +148,7 @@ struct Waiter {
     uint32_t abort_saddr;   // shared address of the abort flag (same in every CTA)
     // false once the cluster has aborted: the caller then skips its work
     __device__ bool operator()(int b, uint32_t parity) const {
+        if (mbar_test_wait(&bars[b], parity)) return true;   // usually complete already
         if (*abort_flag) return false;
         for (uint32_t i = 0; i < kWait; ++i) {
             if (mbar_try_wait_sleep(&bars[b], parity, 1000000u)) return true;
@@ -193,7 +195,8 @@ __device__ __forceinline__ void load_qk_slot(const CUtensorMap *tm_q, const CUte
     }
 }
 
-__device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
+__device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_o,
+                          const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
                           const Waiter &wt, int h, int n, int64_t bos, int64_t eos, int nchunks) {
     uint64_t *bars = wt.bars;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -309,19 +312,43 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
         if (nchunks > 0) named_sync(NB_S0, kChainSync);
         bool ok = true;
         float dq[16];            // scale * gamma_t * (S0 q_t) of the previous chunk
-        // read-out of chunk cp: o_t = dq + scale (U P^T)_t, written straight from
-        // registers (each warp store covers 32 consecutive value rows of one token)
+        // read-out of chunk cp: o_t = dq + scale (U P^T)_t for this warp's 16 tokens x
+        // 32 value rows, put into a per-warp shared tile [t][i] and written by one
+        // TMA store of the warp (plain 16-byte stores for tokens of a short last chunk)
+        unsigned short *ot = reinterpret_cast<unsigned short *>(sm + C_OT + (warp - kCEpi0) * 1024);
         auto read_out = [&](int cp) {
             const int64_t ps0 = bos + (int64_t)cp * C;
             const int pL = chunk_len(cp);
             float dout[16];
             tmem_ld16(tmem_addr(tmem, warp, TM_O + 16 * part), dout);
+            // the tile's previous store has been read out of shared memory
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
             tmem_wait_ld();
-            __nv_bfloat16 *dst = p.o + ((size_t)(ps0 + 16 * part) * HV + h) * DH + i;
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (16 * part + j < pL)
-                    dst[(size_t)j * HV * DH] = __float2bfloat16_rn(fmaf(p.scale, dout[j], dq[j]));
+            for (int j = 0; j < 16; ++j) {
+                const __nv_bfloat16 b = __float2bfloat16_rn(fmaf(p.scale, dout[j], dq[j]));
+                ot[j * 32 + lane] = *reinterpret_cast<const unsigned short *>(&b);
+            }
+            if (16 * part + 16 <= pL) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(tm_o, ot, 32 * (warp & 3), h, (int)(ps0 + 16 * part));
+                    bulk_commit_group();
+                }
+            } else {
+                __syncwarp();
+#pragma unroll
+                for (int pass = 0; pass < 2; ++pass) {
+                    const int t = 8 * pass + (lane >> 2), c4 = lane & 3;
+                    const uint4 val = *reinterpret_cast<const uint4 *>(ot + t * 32 + c4 * 8);
+                    if (16 * part + t < pL)
+                        *reinterpret_cast<uint4 *>(p.o + ((size_t)(ps0 + 16 * part + t) * HV + h) * DH +
+                                                   32 * (warp & 3) + 8 * c4) = val;
+                }
+            }
+            __syncwarp();
         };
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t ph = (uint32_t)(c & 1);
@@ -455,6 +482,9 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                 read_out(nchunks - 1);
             }
         }
+        // this warp's tile stores complete before the CTA's shared memory is released
+        if (lane == 0) bulk_wait_group0();
+        __syncwarp();
         if (ok && p.hT) {
             tc_fence_after();
             float v[32];
@@ -785,7 +815,8 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const ClParams p) {
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_o, const ClParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -837,7 +868,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     cluster_sync_all();   // every CTA's barriers are initialised before any remote traffic
 
     if (rank == 0)
-        chain_cta(&tm_q, &tm_k, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
+        chain_cta(&tm_q, &tm_k, &tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
     else
         prep_cta(&tm_q, &tm_k, &tm_v, p, sm, sb, tmem, wt, h, bos, eos, nchunks, rank);
 
@@ -866,7 +897,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     unsigned int *status = static_cast<unsigned int *>(a.workspace);
     cudaError_t err = cudaMemsetAsync(status, 0, sizeof(unsigned int), stream);
     if (err != cudaSuccess) return err;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     const uint64_t tok = (uint64_t)(Ttot > 0 ? Ttot : 1);
     uint64_t dq[3] = {(uint64_t)DH, (uint64_t)a.HK, tok};
     uint64_t sq[2] = {(uint64_t)DH * 2, (uint64_t)a.HK * DH * 2};
@@ -875,6 +906,10 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     uint32_t box[3] = {64, 1, 64};
     if (!encode_bf16_map(&tq, a.q, 3, dq, sq, box) || !encode_bf16_map(&tk, a.k, 3, dq, sq, box) ||
         !encode_bf16_map(&tv, a.v, 3, dv, sv, box))
+        return cudaErrorInvalidValue;
+    // o: one warp's 16 tokens x 32 value rows per store, unswizzled 64-byte rows
+    uint32_t obox[3] = {32, 1, 16};
+    if (!encode_bf16_map(&to, a.o, 3, dv, sv, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     err = cudaFuncSetAttribute(prefill_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)SMEM_BYTES);
@@ -893,7 +928,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, prefill_cluster_kernel, tq, tk, tv, prm);
+    err = cudaLaunchKernelEx(&cfg, prefill_cluster_kernel, tq, tk, tv, to, prm);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
