@@ -97,6 +97,9 @@ NCU_TRAFFIC = {
     # full decode_256x64 step: 541,205,504 read + 480,342,528 written
     "decode": {"bytes": 1021548032, "source": "gdn_decode.cu",
                "sha256": "6bd14494733cc78d5b35f9cc22ae3a4713fce92518aacec935bf3b868656250d"},
+    # full long_prefill_64k launch: 1,090,672,640 read + 512,769,536 written
+    "prefill_cluster": {"bytes": 1603442176, "source": "gdn_prefill_cluster.cu",
+                        "sha256": "cd6808b75ff756e9a49491e50c161fc8b246039cf55fd61a2937b56ffbe88224"},
 }
 
 
