@@ -11,7 +11,7 @@ namespace {
 bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool tc_path(int dk, int dv, int chunk, gdn_dtype dt) {
-    return gdn::prefill_tc_supported(dk, dv, chunk, dt);
+    return gdn::prefill_cluster_supported(dk, dv, chunk, dt);
 }
 
 gdn_status check_prefill(const gdn::PrefillArgs &a) {
@@ -59,7 +59,7 @@ int gdn_chunk_prefill_path(int dk, int dv, int chunk, gdn_dtype dtype) {
 size_t gdn_chunk_prefill_workspace_size(int N, int64_t T, int HK, int HV, int dk, int dv,
                                         int chunk, gdn_dtype dtype, int varlen) {
     if (N < 0 || T < 0 || HK <= 0 || HV <= 0 || HV % HK || chunk <= 0) return 0;
-    if (tc_path(dk, dv, chunk, dtype)) return gdn::prefill_tc_workspace(N, T, HV, chunk, varlen != 0);
+    if (tc_path(dk, dv, chunk, dtype)) return gdn::prefill_cluster_workspace(N, T, HV, chunk, varlen != 0);
     return 0;
 }
 
@@ -75,7 +75,7 @@ gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v, const 
     if (N == 0) return GDN_OK;
     cudaError_t err;
     if (tc_path(dk, dv, chunk, dtype)) {
-        const size_t need = gdn::prefill_tc_workspace(N, T, HV, chunk, cu_seqlens != nullptr);
+        const size_t need = gdn::prefill_cluster_workspace(N, T, HV, chunk, cu_seqlens != nullptr);
         if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
         if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
         err = gdn::launch_prefill_cluster(a, reinterpret_cast<cudaStream_t>(stream));

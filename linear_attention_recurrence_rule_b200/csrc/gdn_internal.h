@@ -42,14 +42,12 @@ cudaError_t launch_decode(const StepArgs &a, cudaStream_t stream);
 bool prefill_simt_supported(int dk, int dv, int chunk);
 cudaError_t launch_prefill_simt(const PrefillArgs &a, cudaStream_t stream);
 
-// tcgen05 / TMEM / TMA tensor-core prefill (gdn_prefill_tc.cu)
-bool prefill_tc_supported(int dk, int dv, int chunk, gdn_dtype dtype);
-size_t prefill_tc_workspace(int N, int64_t T, int HV, int chunk, bool varlen);
-cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream);
 
 // cluster (1 chain CTA + 3 prep CTAs per value head) tensor-core prefill
 // (gdn_prefill_cluster.cu)
 bool prefill_cluster_supported(int dk, int dv, int chunk, gdn_dtype dtype);
+// device workspace the cluster prefill needs: the status word of its bounded waits
+size_t prefill_cluster_workspace(int N, int64_t T, int HV, int chunk, bool varlen);
 cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream);
 
 }  // namespace gdn

@@ -891,6 +891,8 @@ bool prefill_cluster_supported(int dk, int dv, int chunk, gdn_dtype dtype) {
     return dtype == GDN_BF16 && dk == DH && dv == DH && chunk == C;
 }
 
+size_t prefill_cluster_workspace(int, int64_t, int, int, bool) { return 256; }
+
 cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     const int64_t Ttot = a.cu_seqlens ? a.T : (int64_t)a.N * a.T;
     if (Ttot >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
