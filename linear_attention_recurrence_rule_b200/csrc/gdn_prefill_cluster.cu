@@ -14,18 +14,20 @@
 // Split by dependence on the state:
 //   prep CTAs (cluster ranks 1..3) take every third chunk and compute the
 //     state-independent part: [Q;K]K^T, A and P, the UT inverse T (blocked
-//     16 -> 32 -> 64 on CUDA cores), W^T and U~^T (tcgen05), and ship 65 KB per
-//     chunk -- W (next to Q in one K-major [W;Q] operand), P (bf16 hi + lo),
-//     U~ (fp32) and the chunk's decay table -- into the chain CTA's receive slot
-//     with bulk DSMEM copies that complete on the chain CTA's mbarrier, where
-//     the chain CTA's own TMA loads of the chunk's Q and K also land;
-//   the chain CTA (rank 0) walks the chunks in order: one N = 128 product
-//     S0 [W;Q]^T gives S0 W^T and S0 Q^T together (S0 as a bf16 operand in
-//     tensor memory), U = U~ - S0 W^T, the state update S += (U diag(gamma_L /
-//     gamma)) K accumulated in tensor memory after an in-place gamma_L scaling,
-//     and the outputs gamma_t S0 Q^T + U P^T; sixteen epilogue warps share every
-//     epilogue (16 tokens or 32 state columns each) and write chunk c's outputs
-//     while chunk c + 1's first product runs.
+//     16 -> 32 -> 64 on CUDA cores), T' = T diag(b gamma) and T'' = T diag(b) as
+//     bf16 hi + lo tiles, W^T = K^T T'^T (tcgen05) and the chunk's decay table.
+//     They ship 49 KB per chunk -- -W (the first rows of a K-major [-W;Q]
+//     operand), P and T'' (hi + lo) and the table -- from one of two staging
+//     blocks into the chain CTA's receive slot with bulk DSMEM copies that
+//     complete on the chain CTA's mbarrier, where the chain's own TMA loads of
+//     the chunk's Q, K and V also land;
+//   the chain CTA (rank 0) walks the chunks in order: U~^T = V^T T''^T goes into
+//     the U accumulator ahead of the chunk, then S0 (-W)^T is added to it and
+//     S0 Q^T formed (S0 as a bf16 operand in tensor memory), the state update
+//     S += (U diag(gamma_L / gamma)) K accumulates in tensor memory after an
+//     in-place gamma_L scaling, and the outputs are gamma_t S0 Q^T + U P^T;
+//     sixteen epilogue warps share every epilogue (16 tokens or 32 state columns
+//     each) and write chunk c's outputs while chunk c + 1's first products run.
 // The chain's critical loop hands over between its epilogue warps and the
 // MMA-issuing warp through named barriers (no sleeping wake-up on that path);
 // tensor-core completions and cross-CTA hand-overs use mbarriers.
@@ -37,8 +39,9 @@
 // are drained (again bounded) before tensor memory is freed.
 //
 // Precision: exact bf16 q/k/v; T', T'', P, U and U diag(gamma_L/gamma) as bf16
-// hi + lo pairs; U~ crosses in fp32; gamma_t of the inter-chunk read-out
-// applied in fp32; only S0 and W are single bf16.
+// hi + lo pairs (U~ = T''V is formed from T'' hi + lo with fp32 accumulation);
+// gamma_t of the inter-chunk read-out applied in fp32; only S0 and W are single
+// bf16.
 #include <cuda.h>
 
 #include "gdn_common.cuh"
@@ -71,43 +74,45 @@ constexpr uint32_t NB_WORK = 1;                       // prep workers
 constexpr uint32_t NB_S0 = 1, NB_U = 2, NB_U2 = 3;    // epilogue warps + MMA warp
 constexpr uint32_t kChainSync = (kCNumEpi + 1) * 32;
 
-// ---- chain receive slot of one chunk: Q and K by TMA, the rest from a prep CTA ----
-constexpr uint32_t SL_WQ = 0;       // [W;Q] K-major: per 64-column half 16 KB, W rows then Q rows
+// ---- chain receive slot of one chunk: Q, K, V by TMA, the rest from a prep CTA ----
+constexpr uint32_t SL_WQ = 0;       // per 64-column half 16 KB: -W rows (t), then Q rows (t); K-major
 constexpr uint32_t SL_K = 32768;    // K as loaded (rows t, two 64-column halves), MN-major B
-constexpr uint32_t SL_PH = 49152;   // P hi: 64 rows (t) x 64 (s), K-major
-constexpr uint32_t SL_PL = 57344;   // P lo
-constexpr uint32_t SL_U = 65536;    // U~ fp32 [i][t], 16-byte chunks xor-swizzled by row
+constexpr uint32_t SL_V = 49152;    // V as loaded (rows t, two 64-column halves), MN-major A
+constexpr uint32_t SL_PH = 65536;   // P hi: 64 rows (t) x 64 (s), K-major
+constexpr uint32_t SL_PL = 73728;   // P lo
+constexpr uint32_t SL_T2H = 81920;  // T'' = T diag(b) hi: 64 rows (t) x 64 (s), K-major
+constexpr uint32_t SL_T2L = 90112;  // T'' lo
 constexpr uint32_t SL_TAB = 98304;  // fp32: gamma_L/gamma_t [64], gamma_t [64], gamma_L
 constexpr uint32_t SLOT = 99328;    // bytes per slot (a multiple of 1024: slots stay swizzle-aligned)
-// the prep CTA's staging block (what its bulk copies carry) and where each piece lands
-constexpr uint32_t ST_W = 0;        // W rows, two 64-column halves of 8 KB -> SL_WQ, SL_WQ + 16384
+// a prep CTA's staging block (what its bulk copies carry) and where each piece lands
+constexpr uint32_t ST_W = 0;        // -W rows, two 64-column halves of 8 KB -> SL_WQ, SL_WQ + 16384
 constexpr uint32_t ST_P = 16384;    // P hi, P lo -> SL_PH
-constexpr uint32_t ST_U = 32768;    // U~ -> SL_U
-constexpr uint32_t ST_TAB = 65536;  // decay table -> SL_TAB
-constexpr uint32_t ST_BYTES = 66560;
-constexpr uint32_t QK_BYTES = 4 * 8192;            // Q and K tiles loaded by the chain CTA
-constexpr uint32_t SLOT_TX = ST_BYTES + QK_BYTES;  // bytes that complete one receive slot
+constexpr uint32_t ST_T2 = 32768;   // T'' hi, T'' lo -> SL_T2H
+constexpr uint32_t ST_TAB = 49152;  // decay table -> SL_TAB
+constexpr uint32_t ST_BYTES = 50176;
+constexpr uint32_t QKV_BYTES = 6 * 8192;            // Q, K and V tiles loaded by the chain CTA
+constexpr uint32_t SLOT_TX = ST_BYTES + QKV_BYTES;  // bytes that complete one receive slot
 
 // ---- chain CTA shared memory ----
 constexpr uint32_t C_R = 0;                                 // 2 receive slots
 constexpr uint32_t C_OT = C_R + 2 * SLOT;   // per epilogue warp: 16 x 32 bf16 output tile
 constexpr uint32_t C_BAR = C_OT + kCNumEpi * 1024;
 // ---- prep CTA shared memory ----
-// two q/k/v buffers of 48 KB: [Q half 0 | K half 0][Q half 1 | K half 1][V]
-constexpr uint32_t P_QKV = 0, QKV_STRIDE = 49152, QKV_V = 32768;
-constexpr uint32_t P_T = 98304;     // T' hi, T' lo, T'' hi, T'' lo (4 x 8 KB); A fp32 shares it
+// two q/k buffers of 32 KB: [Q half 0 | K half 0][Q half 1 | K half 1]
+constexpr uint32_t P_QK = 0, QK_STRIDE = 32768;
+constexpr uint32_t P_T = 65536;     // A fp32 [64][A_LD], then T' hi, T' lo (2 x 8 KB)
 constexpr uint32_t A_LD = 68;
-constexpr uint32_t P_TF = 131072;   // T fp32 [64][T_LD]
+constexpr uint32_t P_TF = P_T + 64 * A_LD * 4;   // T fp32 [64][T_LD]
 constexpr uint32_t T_LD = 68;
 constexpr uint32_t P_X = P_TF + 64 * T_LD * 4;
 constexpr uint32_t X_LD = 36;
 constexpr uint32_t P_PB = P_X + 32 * X_LD * 4;             // beta, gamma, G
-constexpr uint32_t P_ST = 154624;   // staging block (ST_BYTES)
-constexpr uint32_t P_BAR = P_ST + ST_BYTES;
+constexpr uint32_t P_ST = 106496;   // two staging blocks (ST_BYTES each, 1024-aligned)
+constexpr uint32_t P_BAR = P_ST + 2 * ST_BYTES;
 
 enum ChainBar { CB_R_FULL0, CB_R_FULL1, CB_U_MMA, CB_DS_FULL, CB_O_FULL, CB_DRAIN, CB_COUNT };
-enum PrepBar { PB_LD_FULL0, PB_LD_FULL1, PB_X_DONE, PB_T_READY, PB_WU_DONE, PB_EPI_DONE, PB_GO,
-               PB_STAGE_FREE, PB_DRAIN, PB_COUNT };
+enum PrepBar { PB_LD_FULL0, PB_LD_FULL1, PB_X_DONE, PB_T_READY, PB_W_DONE, PB_EPI_DONE, PB_GO,
+               PB_STAGE_FREE0, PB_STAGE_FREE1, PB_DRAIN, PB_COUNT };
 
 // words at the same offset in every CTA: TMEM base, abort flag, slot bookkeeping
 constexpr uint32_t AUX_RAW = (C_BAR + CB_COUNT * 8 > P_BAR + PB_COUNT * 8) ? C_BAR + CB_COUNT * 8
@@ -117,18 +122,18 @@ constexpr uint32_t AUX_TSLOT = AUX, AUX_ABORT = AUX + 4, AUX_ARMED = AUX + 8,
                    AUX_CONSUMED = AUX + 12;
 constexpr uint32_t SMEM_BYTES = AUX + 16 + 1024;
 static_assert(P_PB + 3 * 64 * 4 <= P_ST, "prep layout");
-static_assert(64 * A_LD * 4 <= 32768, "A fits the T tiles");
+static_assert(64 * A_LD * 4 >= 16384, "T' tiles fit where A was");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(P_ST % 1024 == 0 && SLOT % 1024 == 0, "swizzle alignment");
-static_assert(P_PB + 3 * 64 * 4 <= P_ST && P_X + 32 * X_LD * 4 <= P_PB, "prep layout");
+static_assert(P_ST % 1024 == 0 && SLOT % 1024 == 0 && ST_BYTES % 1024 == 0 && P_T % 1024 == 0,
+              "swizzle alignment");
 
 // ---- TMEM columns ----
 // chain: S0 [W;Q]^T (D = S0 W^T, then S0 Q^T), U P^T, S0 (bf16 A operand), S (fp32),
 //        U / U diag(gamma_L/gamma) hi and lo (bf16 A operands)
 constexpr uint32_t TM_D = 0, TM_Q = 64, TM_O = 128, TM_S0 = 192, TM_S = 256;
 constexpr uint32_t TM_UH = 384, TM_UL = 416, TM_BH = 448, TM_BL = 480;
-// prep: [Q;K]K^T then W^T, U~^T
-constexpr uint32_t TP_D1 = 0, TP_U = 64;
+// prep: [Q;K]K^T, then W^T
+constexpr uint32_t TP_D1 = 0;
 
 struct ClParams {
     const float *g, *beta, *h0;
@@ -172,18 +177,14 @@ struct Waiter {
 __device__ __forceinline__ void local_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// fp32 U~ tile [i][t]: byte offset of the 16-byte chunk holding t = 4*tc .. 4*tc+3 of row i
-__device__ __forceinline__ uint32_t ut_chunk(uint32_t i, uint32_t tc) {
-    return i * 256u + (((tc ^ i) & 15u) << 4);
-}
 // the whole warp agrees (wait results are warp-uniform in practice; this makes it certain)
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
 // ============================================================================ chain CTA
-// Q and K tiles of chunk c into its receive slot (completing on that slot's mbarrier)
-__device__ __forceinline__ void load_qk_slot(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
-                                             uint8_t *sm, uint64_t *bars, int c, int cqk,
-                                             int64_t bos) {
+// Q, K and V tiles of chunk c into its receive slot (completing on that slot's mbarrier)
+__device__ __forceinline__ void load_qkv_slot(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                              const CUtensorMap *tm_v, uint8_t *sm, uint64_t *bars,
+                                              int c, int cqk, int h, int64_t bos) {
     const int s = c & 1;
     uint8_t *slot = sm + C_R + s * SLOT;
     uint64_t *bar = &bars[CB_R_FULL0 + s];
@@ -192,11 +193,12 @@ __device__ __forceinline__ void load_qk_slot(const CUtensorMap *tm_q, const CUte
     for (int hf = 0; hf < 2; ++hf) {
         tma_load_3d(slot + SL_WQ + hf * 16384 + 8192, tm_q, bar, 64 * hf, cqk, s0);
         tma_load_3d(slot + SL_K + hf * 8192, tm_k, bar, 64 * hf, cqk, s0);
+        tma_load_3d(slot + SL_V + hf * 8192, tm_v, bar, 64 * hf, h, s0);
     }
 }
 
-__device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_o,
-                          const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
+__device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+                          const CUtensorMap *tm_o, const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
                           const Waiter &wt, int h, int n, int64_t bos, int64_t eos, int nchunks) {
     uint64_t *bars = wt.bars;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -210,37 +212,60 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
     };
     if (warp == kCMma) {
         // ------------------------------------------------------------ MMA warp
-        const uint32_t id_wq = idesc_bf16(128, 128, false, false);
+        const uint32_t id_n64 = idesc_bf16(128, 64, false, false);
         const uint32_t id_s = idesc_bf16(128, 128, false, true);
-        const uint32_t id_o = idesc_bf16(128, 64, false, false);
+        const uint32_t id_u = idesc_bf16(128, 64, true, false);
         auto commit = [&](int b) {
             if (elect_one()) mma_commit(&bars[b]);
             __syncwarp();
         };
-        bool ok = true;
+        // chunk c's receive slot is complete: release the producing prep CTA's
+        // staging block, then U~^T = V^T T''^T into the U accumulator (hi + lo), so
+        // that chunk c's first product only has to add S0 (-W)^T
+        auto take_slot = [&](int c, bool ok_in) -> bool {
+            const bool ok = warp_all(ok_in && wt(CB_R_FULL0 + (c & 1), (uint32_t)((c >> 1) & 1)));
+            if (!ok) return false;
+            const uint32_t slot = sb + C_R + (c & 1) * SLOT;
+            if (lane == 0) *consumed = c + 1;
+            // the bulk copies out of that staging block have completed
+            if (elect_one())
+                mbar_arrive_remote_relaxed(mapa_shared(
+                    sb + P_BAR + (PB_STAGE_FREE0 + ((c / kNumPrep) & 1)) * 8, 1 + c % kNumPrep));
+            __syncwarp();
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t va = sdesc_sw128(slot + SL_V + k * 2048, 8192, 1024);
+                const uint64_t th = sdesc_sw128(slot + SL_T2H + k * 32, 16, 1024);
+                const uint64_t tl = sdesc_sw128(slot + SL_T2L + k * 32, 16, 1024);
+                if (elect_one()) {
+                    mma_bf16(tmem + TM_D, va, th, id_u, k > 0);
+                    mma_bf16(tmem + TM_D, va, tl, id_u, 1);
+                }
+                __syncwarp();
+            }
+            return true;
+        };
+        bool ok = nchunks > 0 ? take_slot(0, true) : true;
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c & 1;
-            const uint32_t slot = sb + C_R + s * SLOT;
+            const uint32_t slot = sb + C_R + (c & 1) * SLOT;
             // S0 of chunk c is in tensor memory, and the epilogue warps have read every
             // accumulator of chunk c - 1 that this chunk's MMAs overwrite
             named_sync(NB_S0, kChainSync);
             tc_fence_after();
-            ok = warp_all(ok && wt(CB_R_FULL0 + s, (uint32_t)((c >> 1) & 1)));
             if (ok) {
-                if (lane == 0) *consumed = c + 1;
-                // the bulk copy out of the producing prep CTA's staging block has
-                // completed: that block may be refilled
-                if (elect_one())
-                    mbar_arrive_remote_relaxed(
-                        mapa_shared(sb + P_BAR + PB_STAGE_FREE * 8, 1 + c % kNumPrep));
-                __syncwarp();
-            }
-            if (ok) {
-                // [S0 W^T | S0 Q^T] = S0 [W;Q]^T (A = S0 from TMEM, B K-major from the slot)
+                // U = U~ + S0 (-W)^T, then S0 Q^T (A = S0 from TMEM, B K-major from the slot)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint64_t b = sdesc_sw128(slot + SL_WQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                    if (elect_one()) mma_bf16_ts(tmem + TM_D, tmem + TM_S0 + 8 * k, b, id_wq, k > 0);
+                    if (elect_one()) mma_bf16_ts(tmem + TM_D, tmem + TM_S0 + 8 * k, b, id_n64, 1);
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t b =
+                        sdesc_sw128(slot + SL_WQ + (k >> 2) * 16384 + 8192 + (k & 3) * 32, 16, 1024);
+                    if (elect_one()) mma_bf16_ts(tmem + TM_Q, tmem + TM_S0 + 8 * k, b, id_n64, k > 0);
                     __syncwarp();
                 }
                 commit(CB_U_MMA);
@@ -269,14 +294,17 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                     const uint64_t ph_d = sdesc_sw128(slot + SL_PH + k * 32, 16, 1024);
                     const uint64_t pl_d = sdesc_sw128(slot + SL_PL + k * 32, 16, 1024);
                     if (elect_one()) {
-                        mma_bf16_ts(tmem + TM_O, tmem + TM_UH + 8 * k, ph_d, id_o, k > 0);
-                        mma_bf16_ts(tmem + TM_O, tmem + TM_UH + 8 * k, pl_d, id_o, 1);
-                        mma_bf16_ts(tmem + TM_O, tmem + TM_UL + 8 * k, ph_d, id_o, 1);
+                        mma_bf16_ts(tmem + TM_O, tmem + TM_UH + 8 * k, ph_d, id_n64, k > 0);
+                        mma_bf16_ts(tmem + TM_O, tmem + TM_UH + 8 * k, pl_d, id_n64, 1);
+                        mma_bf16_ts(tmem + TM_O, tmem + TM_UL + 8 * k, ph_d, id_n64, 1);
                     }
                     __syncwarp();
                 }
                 commit(CB_O_FULL);
             }
+            // the next chunk's U~ (this chunk's U was read before its second barrier);
+            // it runs while this chunk's state update completes
+            if (c + 1 < nchunks) ok = take_slot(c + 1, ok);
         }
         // every MMA issued here has completed before tensor memory is released
         commit(CB_DRAIN);
@@ -378,7 +406,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                         if (lane == 0) {
                             mbar_arrive_expect_tx(&bars[CB_R_FULL0 + ((c + 1) & 1)], SLOT_TX);
                             *armed = c + 2;
-                            load_qk_slot(tm_q, tm_k, sm, bars, c + 1, cqk, bos);
+                            load_qkv_slot(tm_q, tm_k, tm_v, sm, bars, c + 1, cqk, h, bos);
                             mbar_arrive_remote_relaxed(
                                 mapa_shared(sb + P_BAR + PB_GO * 8, 1 + (c + 1) % kNumPrep));
                         }
@@ -391,18 +419,9 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             float u[16];
             if (ok) {
                 tc_fence_after();
-                // U = U~ - S0 W^T for tokens t = 16 part + j of row i
+                // U = U~ - S0 W^T for tokens t = 16 part + j of row i (formed by the MMAs)
                 tmem_ld16(tmem_addr(tmem, warp, TM_D + 16 * part), u);
                 tmem_wait_ld();
-                const uint8_t *ut = slot + SL_U;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 a = *reinterpret_cast<const float4 *>(ut + ut_chunk(i, 4 * part + q4));
-                    u[4 * q4] = a.x - u[4 * q4];
-                    u[4 * q4 + 1] = a.y - u[4 * q4 + 1];
-                    u[4 * q4 + 2] = a.z - u[4 * q4 + 2];
-                    u[4 * q4 + 3] = a.w - u[4 * q4 + 3];
-                }
                 if (L < C) {   // tokens past the sequence end (short last chunk)
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
@@ -519,19 +538,17 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             if (elect_one()) mma_commit(&bars[b]);
             __syncwarp();
         };
-        int issued = 0, landed = 0;    // q/k/v loads issued / waited for (k-th into buffer k & 1)
+        int issued = 0, landed = 0;    // q/k loads issued / waited for (k-th into buffer k & 1)
         auto load = [&](int k) {
             if (lane == 0) {
                 const int s0 = (int)(bos + (int64_t)chunk_of(k) * C);
                 uint64_t *bar = &bars[PB_LD_FULL0 + (k & 1)];
-                uint8_t *buf = sm + P_QKV + (k & 1) * QKV_STRIDE;
-                mbar_arrive_expect_tx(bar, 6 * 8192);
+                uint8_t *buf = sm + P_QK + (k & 1) * QK_STRIDE;
+                mbar_arrive_expect_tx(bar, 4 * 8192);
                 tma_load_3d(buf, tm_q, bar, 0, cqk, s0);
                 tma_load_3d(buf + 16384, tm_q, bar, 64, cqk, s0);
                 tma_load_3d(buf + 8192, tm_k, bar, 0, cqk, s0);
                 tma_load_3d(buf + 24576, tm_k, bar, 64, cqk, s0);
-                tma_load_3d(buf + QKV_V, tm_v, bar, 0, h, s0);
-                tma_load_3d(buf + QKV_V + 8192, tm_v, bar, 64, h, s0);
             }
             __syncwarp();
             ++issued;
@@ -540,17 +557,16 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             if (lane == 0) {
                 tma_prefetch_desc(tm_q);
                 tma_prefetch_desc(tm_k);
-                tma_prefetch_desc(tm_v);
             }
             load(0);
         }
         for (int k = 0; k < nk; ++k) {
             const int c = chunk_of(k);
             const uint32_t ph = (uint32_t)(k & 1);
-            const uint32_t qkv = sb + P_QKV + (k & 1) * QKV_STRIDE;
+            const uint32_t qkv = sb + P_QK + (k & 1) * QK_STRIDE;
             if (!warp_all(wt(PB_LD_FULL0 + (k & 1), (uint32_t)((k >> 1) & 1)))) break;
             ++landed;
-            // the other buffer's chunk (k - 1) finished its W/U products: load chunk k + 1
+            // the other buffer's chunk (k - 1) finished its W product: load chunk k + 1
             if (k + 1 < nk) load(k + 1);
             tc_fence_after();
 #pragma unroll
@@ -564,24 +580,20 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             commit(PB_X_DONE);
             if (!warp_all(wt(PB_T_READY, ph))) break;
             tc_fence_after();
+            // W^T = K^T T'^T (T' = T diag(b gamma) as hi + lo)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t ka = sdesc_sw128(qkv + 8192 + kk * 2048, 16384, 1024);
-                const uint64_t va = sdesc_sw128(qkv + QKV_V + kk * 2048, 8192, 1024);
                 const uint64_t t1h = sdesc_sw128(sb + P_T + kk * 32, 16, 1024);
                 const uint64_t t1l = sdesc_sw128(sb + P_T + 8192 + kk * 32, 16, 1024);
-                const uint64_t t2h = sdesc_sw128(sb + P_T + 16384 + kk * 32, 16, 1024);
-                const uint64_t t2l = sdesc_sw128(sb + P_T + 24576 + kk * 32, 16, 1024);
                 if (elect_one()) {
                     mma_bf16(tmem + TP_D1, ka, t1h, id_w, kk > 0);
                     mma_bf16(tmem + TP_D1, ka, t1l, id_w, 1);
-                    mma_bf16(tmem + TP_U, va, t2h, id_w, kk > 0);
-                    mma_bf16(tmem + TP_U, va, t2l, id_w, 1);
                 }
                 __syncwarp();
             }
-            commit(PB_WU_DONE);
-            if (!warp_all(wt(PB_WU_DONE, ph))) break;   // this buffer's q/k/v tiles are free again
+            commit(PB_W_DONE);
+            if (!warp_all(wt(PB_W_DONE, ph))) break;   // this buffer's q/k tiles are free again
             if (!warp_all(wt(PB_EPI_DONE, ph))) break;
             if (c >= 2) {
                 const int j = first >= 2 ? k : k - 1;   // go arrivals before this chunk
@@ -591,11 +603,11 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 const int s = c & 1;
                 const uint32_t mbar = mapa_shared(sb + C_BAR + (CB_R_FULL0 + s) * 8, 0);
                 const uint32_t dst = mapa_shared(sb + C_R + s * SLOT, 0);
-                const uint32_t st = sb + P_ST;
+                const uint32_t st = sb + P_ST + (k & 1) * ST_BYTES;
                 bulk_copy_to_cluster(dst + SL_WQ, st + ST_W, 8192, mbar);
                 bulk_copy_to_cluster(dst + SL_WQ + 16384, st + ST_W + 8192, 8192, mbar);
                 bulk_copy_to_cluster(dst + SL_PH, st + ST_P, 16384, mbar);
-                bulk_copy_to_cluster(dst + SL_U, st + ST_U, 32768, mbar);
+                bulk_copy_to_cluster(dst + SL_T2H, st + ST_T2, 16384, mbar);
                 bulk_copy_to_cluster(dst + SL_TAB, st + ST_TAB, ST_BYTES - ST_TAB, mbar);
             }
             __syncwarp();
@@ -622,6 +634,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             const uint32_t ph = (uint32_t)(k & 1);
             const int64_t s0 = bos + (int64_t)c * C;
             const int L = chunk_len(c);
+            const uint32_t stb = P_ST + (k & 1) * ST_BYTES;   // this chunk's staging block
             named_sync(NB_WORK, kPWorkThreads);
             if (warp == kPWork0) {
                 const float2 gp = load_g_pair(p.g, s0, L, HV, h);
@@ -635,10 +648,10 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 beta_s[2 * lane] = bp.x;
                 beta_s[2 * lane + 1] = bp.y;
             }
-            // the X product is done and the staging block's previous contents have
-            // been copied out
+            // the X product is done and this staging block's previous contents (chunk
+            // k - 2 of this CTA) have been copied out
             ok = warp_all(ok && wt(PB_X_DONE, ph) &&
-                          (k == 0 || wt(PB_STAGE_FREE, (uint32_t)((k - 1) & 1))));
+                          (k < 2 || wt(PB_STAGE_FREE0 + (k & 1), (uint32_t)(((k >> 1) - 1) & 1))));
             named_sync(NB_WORK, kPWorkThreads);
             if (ok) {
                 tc_fence_after();
@@ -664,7 +677,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         const uint32_t off = sw128_chunk(row, 2 * qtr + cc);
-                        st_chunk_hilo(sb + P_ST + ST_P + off, sb + P_ST + ST_P + 8192 + off, v + 8 * cc);
+                        st_chunk_hilo(sb + stb + ST_P + off, sb + stb + ST_P + 8192 + off, v + 8 * cc);
                     }
                 } else {
                     const float bi = beta_s[row];
@@ -685,7 +698,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 }
                 // decay table of this chunk for the chain CTA
                 if (pt < 64) {
-                    float *tb = reinterpret_cast<float *>(sm + P_ST + ST_TAB);
+                    float *tb = reinterpret_cast<float *>(sm + stb + ST_TAB);
                     tb[pt] = __expf(G_p[63] - G_p[pt]);    // gamma_L / gamma_t
                     tb[64 + pt] = gam_p[pt];               // gamma_t
                     if (pt == 0) tb[128] = gam_p[63];      // gamma_L
@@ -760,7 +773,8 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 *reinterpret_cast<float2 *>(T_s + (32 + ii3) * T_LD + j3) = make_float2(-a0, -a1);
             }
             named_sync(NB_WORK, kPWorkThreads);
-            // ---- T' = T diag(b gamma), T'' = T diag(b) as hi/lo bf16 tiles (A is dead) ----
+            // ---- T' = T diag(b gamma) (for W) and T'' = T diag(b) (shipped) as hi/lo bf16
+            //      tiles; A is dead ----
             if (ok) {
                 const int t = pt >> 3, chunk16 = pt & 7;
                 float a1[8], a2[8];
@@ -773,36 +787,28 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 }
                 const uint32_t off = sw128_chunk(t, chunk16);
                 st_chunk_hilo(sb + P_T + off, sb + P_T + 8192 + off, a1);
-                st_chunk_hilo(sb + P_T + 16384 + off, sb + P_T + 24576 + off, a2);
+                st_chunk_hilo(sb + stb + ST_T2 + off, sb + stb + ST_T2 + 8192 + off, a2);
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) local_arrive(&bars[PB_T_READY]);
-            // ---- W and U~ epilogues into the staging block ----
-            ok = warp_all(ok && wt(PB_WU_DONE, ph));
+            // ---- -W epilogue into the staging block ----
+            ok = warp_all(ok && wt(PB_W_DONE, ph));
             named_sync(NB_WORK, kPWorkThreads);
             if (ok) {
                 tc_fence_after();
                 float v[16];
-                // W^T row a = r, tokens t = 16 qtr + j -> W rows of the K-major [W;Q] operand
+                // W^T row a = r, tokens t = 16 qtr + j -> -W rows of the K-major [-W;Q] operand
                 tmem_ld16(tmem_addr(tmem, warp, TP_D1 + 16 * qtr), v);
                 tmem_wait_ld();
-                uint8_t *wq = sm + P_ST + ST_W + (r >> 6) * 8192 + (r & 7) * 2;
+                uint8_t *wq = sm + stb + ST_W + (r >> 6) * 8192 + (r & 7) * 2;
                 const uint32_t wc = (uint32_t)((r & 63) >> 3);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const int t = 16 * qtr + j;
                     *reinterpret_cast<__nv_bfloat16 *>(wq + t * 128 + ((wc ^ (uint32_t)(t & 7)) << 4)) =
-                        __float2bfloat16_rn(v[j]);
+                        __float2bfloat16_rn(-v[j]);
                 }
-                // U~^T row i = r, tokens 16 qtr .. (fp32)
-                tmem_ld16(tmem_addr(tmem, warp, TP_U + 16 * qtr), v);
-                tmem_wait_ld();
-                uint8_t *ut = sm + P_ST + ST_U;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<float4 *>(ut + ut_chunk(r, 4 * qtr + q4)) =
-                        make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -838,7 +844,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
         eos = bos + p.T;
     }
     const int nchunks = (int)((eos - bos + C - 1) / C);
-    const uint32_t ncols = rank == 0 ? 512u : 128u;
+    const uint32_t ncols = rank == 0 ? 512u : 64u;
 
     if (tid == 0) {
         for (int b = 0; b < nbars; ++b) {
@@ -852,9 +858,10 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             const int pre = nchunks < 2 ? nchunks : 2;
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
             for (int c = 0; c < pre; ++c) {
                 mbar_arrive_expect_tx(&bars[CB_R_FULL0 + c], SLOT_TX);
-                load_qk_slot(&tm_q, &tm_k, sm, bars, c, h / (p.HV / p.HK), bos);
+                load_qkv_slot(&tm_q, &tm_k, &tm_v, sm, bars, c, h / (p.HV / p.HK), h, bos);
             }
             *reinterpret_cast<volatile int *>(sm + AUX_ARMED) = pre;
             *reinterpret_cast<volatile int *>(sm + AUX_CONSUMED) = 0;
@@ -868,7 +875,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     cluster_sync_all();   // every CTA's barriers are initialised before any remote traffic
 
     if (rank == 0)
-        chain_cta(&tm_q, &tm_k, &tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
+        chain_cta(&tm_q, &tm_k, &tm_v, &tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
     else
         prep_cta(&tm_q, &tm_k, &tm_v, p, sm, sb, tmem, wt, h, bos, eos, nchunks, rank);
 
