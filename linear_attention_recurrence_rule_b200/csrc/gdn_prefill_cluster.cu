@@ -177,6 +177,9 @@ struct Waiter {
 __device__ __forceinline__ void local_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// descriptor of the same operand `bytes` further on (the start-address field holds
+// address >> 4; shared addresses stay below 256 KB, so the field cannot overflow)
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 // the whole warp agrees (wait results are warp-uniform in practice; this makes it certain)
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
@@ -213,6 +216,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
     if (warp == kCMma) {
         // ------------------------------------------------------------ MMA warp
         const uint32_t id_n64 = idesc_bf16(128, 64, false, false);
+        const uint32_t id_wq = idesc_bf16(128, 128, false, false);
         const uint32_t id_s = idesc_bf16(128, 128, false, true);
         const uint32_t id_u = idesc_bf16(128, 64, true, false);
         auto commit = [&](int b) {
@@ -233,14 +237,14 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                     sb + P_BAR + (PB_STAGE_FREE0 + ((c / kNumPrep) & 1)) * 8, 1 + c % kNumPrep));
             __syncwarp();
             tc_fence_after();
+            const uint64_t va0 = sdesc_sw128(slot + SL_V, 8192, 1024);
+            const uint64_t th0 = sdesc_sw128(slot + SL_T2H, 16, 1024);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const uint64_t va = sdesc_sw128(slot + SL_V + k * 2048, 8192, 1024);
-                const uint64_t th = sdesc_sw128(slot + SL_T2H + k * 32, 16, 1024);
-                const uint64_t tl = sdesc_sw128(slot + SL_T2L + k * 32, 16, 1024);
                 if (elect_one()) {
-                    mma_bf16(tmem + TM_D, va, th, id_u, k > 0);
-                    mma_bf16(tmem + TM_D, va, tl, id_u, 1);
+                    mma_bf16(tmem + TM_D, desc_add(va0, k * 2048), desc_add(th0, k * 32), id_u, k > 0);
+                    mma_bf16(tmem + TM_D, desc_add(va0, k * 2048), desc_add(th0, SL_T2L - SL_T2H + k * 32),
+                             id_u, 1);
                 }
                 __syncwarp();
             }
@@ -254,18 +258,14 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             named_sync(NB_S0, kChainSync);
             tc_fence_after();
             if (ok) {
-                // U = U~ + S0 (-W)^T, then S0 Q^T (A = S0 from TMEM, B K-major from the slot)
+                // [U | S0 Q^T] = [U~ | 0] + S0 [-W;Q]^T in one N = 128 product (A = S0 from
+                // TMEM, B K-major from the slot; the epilogue warps zeroed S0 Q^T's columns)
+                const uint64_t wq0 = sdesc_sw128(slot + SL_WQ, 16, 1024);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint64_t b = sdesc_sw128(slot + SL_WQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                    if (elect_one()) mma_bf16_ts(tmem + TM_D, tmem + TM_S0 + 8 * k, b, id_n64, 1);
-                    __syncwarp();
-                }
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint64_t b =
-                        sdesc_sw128(slot + SL_WQ + (k >> 2) * 16384 + 8192 + (k & 3) * 32, 16, 1024);
-                    if (elect_one()) mma_bf16_ts(tmem + TM_Q, tmem + TM_S0 + 8 * k, b, id_n64, k > 0);
+                    if (elect_one())
+                        mma_bf16_ts(tmem + TM_D, tmem + TM_S0 + 8 * k,
+                                    desc_add(wq0, (k >> 2) * 16384 + (k & 3) * 32), id_wq, 1);
                     __syncwarp();
                 }
                 commit(CB_U_MMA);
@@ -274,12 +274,12 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             tc_fence_after();
             if (ok) {
                 // S += (U diag(gamma_L/gamma)) K  (hi + lo; K MN-major from the slot)
+                const uint64_t k0 = sdesc_sw128(slot + SL_K, 8192, 1024);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint64_t b = sdesc_sw128(slot + SL_K + k * 2048, 8192, 1024);
                     if (elect_one()) {
-                        mma_bf16_ts(tmem + TM_S, tmem + TM_BH + 8 * k, b, id_s, 1);
-                        mma_bf16_ts(tmem + TM_S, tmem + TM_BL + 8 * k, b, id_s, 1);
+                        mma_bf16_ts(tmem + TM_S, tmem + TM_BH + 8 * k, desc_add(k0, k * 2048), id_s, 1);
+                        mma_bf16_ts(tmem + TM_S, tmem + TM_BL + 8 * k, desc_add(k0, k * 2048), id_s, 1);
                     }
                     __syncwarp();
                 }
@@ -289,10 +289,10 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             tc_fence_after();
             if (ok) {
                 // U P^T (hi/lo cross terms)
+                const uint64_t p0 = sdesc_sw128(slot + SL_PH, 16, 1024);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint64_t ph_d = sdesc_sw128(slot + SL_PH + k * 32, 16, 1024);
-                    const uint64_t pl_d = sdesc_sw128(slot + SL_PL + k * 32, 16, 1024);
+                    const uint64_t ph_d = desc_add(p0, k * 32), pl_d = desc_add(p0, SL_PL - SL_PH + k * 32);
                     if (elect_one()) {
                         mma_bf16_ts(tmem + TM_O, tmem + TM_UH + 8 * k, ph_d, id_n64, k > 0);
                         mma_bf16_ts(tmem + TM_O, tmem + TM_UH + 8 * k, pl_d, id_n64, 1);
@@ -334,6 +334,10 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
             tmem_st16w(tmem_addr(tmem, warp, TM_S0 + 16 * part), w);
             tmem_st32f(tmem_addr(tmem, warp, TM_S + 32 * part), v);
+            // chunk 0's S0 Q^T accumulates onto zero
+#pragma unroll
+            for (int j = 0; j < 16; ++j) w[j] = 0u;
+            tmem_st16w(tmem_addr(tmem, warp, TM_Q + 16 * part), w);
             tmem_wait_st();
         }
         tc_fence_before();
@@ -478,9 +482,16 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                     tmem_st16w(tmem_addr(tmem, warp, TM_S0 + 16 * part), w);
                 }
                 // scale * gamma_t * S0 q_t of this part's tokens, read before the next
-                // chunk's MMAs overwrite it (gamma_t from the slot, still held)
+                // chunk's MMAs overwrite it (gamma_t from the slot, still held); the
+                // columns are zeroed for the next chunk's accumulation
                 tmem_ld16(tmem_addr(tmem, warp, TM_Q + 16 * part), dq);
                 tmem_wait_ld();
+                if (more) {
+                    uint32_t z[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) z[j] = 0u;
+                    tmem_st16w(tmem_addr(tmem, warp, TM_Q + 16 * part), z);
+                }
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const float4 g4 = *reinterpret_cast<const float4 *>(tab + 64 + 16 * part + 4 * q4);
