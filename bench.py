@@ -354,12 +354,15 @@ def run_b200(args):
         d2h = host_o.numel() * host_o.element_size() + host_h.numel() * host_h.element_size()
         e_steps = max(1, min(args.steps, args.e2e_steps))
 
+        # the host-memory entry point streams segments: the copies of one segment
+        # overlap the computation of the next on the public call's three streams
+        h_ws = torch.empty(gdn.gdn_chunk_prefill_host_workspace_size(
+            B, T, w.HK, w.HV, w.dk, w.dv, w.chunk, w.dtype, 0), dtype=torch.uint8, device=dev)
+
         def e2e_step():
-            for n in names:
-                d[n].copy_(host_in[n], non_blocking=True)
-            gdn.gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], chunk=w.chunk, o=o,
-                                  hT=hT, workspace=ws, stream=stream)
-            host_o.copy_(o, non_blocking=True)
+            gdn.gdn_chunk_prefill_host(host_in["q"], host_in["k"], host_in["v"], host_in["g"],
+                                       host_in["beta"], chunk=w.chunk, o=host_o, hT=hT,
+                                       workspace=h_ws, device=dev, stream=stream)
             host_h.copy_(hT, non_blocking=True)
 
         e2e_step()

@@ -21,9 +21,10 @@
  *
  * Conventions shared by every call
  *   - All pointers are DEVICE pointers of the current CUDA device unless a
- *     comment says otherwise.  The caller owns every buffer; the library keeps
- *     no allocation and no global state, never synchronises the stream, and
- *     returns as soon as the work is enqueued on `stream`.
+ *     comment says otherwise (gdn_chunk_prefill_host takes host buffers).  The
+ *     caller owns every buffer; the library keeps no allocation and no global
+ *     state, never synchronises the stream, and returns as soon as the work is
+ *     enqueued.
  *   - Tensors are dense, row-major, with the last dimension contiguous.
  *   - dtype selects the element type of q, k, v and o: GDN_F32 (float) or
  *     GDN_BF16 (__nv_bfloat16).  g, beta, h0, hT and the decode state are
@@ -151,6 +152,53 @@ GDN_API gdn_status gdn_chunk_prefill_noalloc(const void *q, const void *k, const
                                              int HV, int dk, int dv, int chunk, float scale,
                                              gdn_dtype dtype, void *o, float *hT,
                                              gdn_stream_t stream);
+
+/*
+ * Bytes of device workspace gdn_chunk_prefill_host needs (0 for arguments it
+ * would reject).  segment: tokens per segment, 0 selects the default (4096).
+ */
+GDN_API size_t gdn_chunk_prefill_host_workspace_size(int N, int64_t T, int HK, int HV, int dk,
+                                                     int dv, int chunk, gdn_dtype dtype,
+                                                     int64_t segment);
+
+/*
+ * gdn_chunk_prefill for inputs and outputs in HOST memory, streamed.  (The
+ * source pages have no counterpart: a library convenience for prefills whose
+ * data lives on the host.)
+ *
+ * The N sequences of T tokens are processed in segments of `segment` tokens:
+ * while segment s runs on `stream`, the inputs of segment s + 1 are copied in on
+ * `copy_in` and the outputs of segment s - 1 are copied out on `copy_out`; the
+ * state goes from one segment to the next in device memory.  The result equals
+ * gdn_chunk_prefill over the whole sequences (chunks restart at every segment
+ * start, which does not change the result; segments that are multiples of
+ * `chunk` give bit-identical results).
+ *   q, k, v, g, beta, o  HOST pointers, layouts as gdn_chunk_prefill without
+ *                        cu_seqlens ([N][T][H][d]); page-locked memory lets the
+ *                        copies overlap the computation, pageable memory works
+ *                        but serialises them.  16-byte aligned.
+ *   h0, hT               DEVICE pointers [N][HV][dv][dk] fp32, or NULL (zero start
+ *                        state / final state not wanted); hT may alias h0.
+ *   workspace            device buffer of at least
+ *                        gdn_chunk_prefill_host_workspace_size(...) bytes,
+ *                        256-byte aligned; scratch after the call, and the status
+ *                        word of gdn_read_status (sticky over all segments).
+ *   stream, copy_in, copy_out  three caller-owned streams (they may coincide, at
+ *                        the price of overlap).  The call orders itself after work
+ *                        already queued on `stream`, and every copy and kernel it
+ *                        enqueues completes before later work on `stream`.
+ * It creates and destroys 3 * ceil(T / segment) + 1 CUDA events (released by the
+ * runtime once they complete), does not synchronise, and allocates no memory.
+ * Errors as gdn_chunk_prefill; GDN_ERR_CUDA if an enqueue fails part way (the
+ * work already enqueued then still runs).
+ */
+GDN_API gdn_status gdn_chunk_prefill_host(const void *q, const void *k, const void *v,
+                                          const float *g, const float *beta, const float *h0,
+                                          int N, int64_t T, int HK, int HV, int dk, int dv,
+                                          int chunk, float scale, gdn_dtype dtype, void *o,
+                                          float *hT, void *workspace, size_t workspace_bytes,
+                                          int64_t segment, gdn_stream_t stream,
+                                          gdn_stream_t copy_in, gdn_stream_t copy_out);
 
 /*
  * Fused single-token decode step for N independent sequences: applies one

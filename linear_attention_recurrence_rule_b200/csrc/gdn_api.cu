@@ -3,6 +3,8 @@
 // global state; every launch goes to the caller's stream.
 #include <cuda_runtime.h>
 
+#include <new>
+
 #include "gdn.h"
 #include "gdn_internal.h"
 
@@ -29,6 +31,52 @@ gdn_status check_prefill(const gdn::PrefillArgs &a) {
         return GDN_ERR_ALIGNMENT;
     return GDN_OK;
 }
+
+// Validation, workspace check and dispatch of one prefill call (tensor-core path
+// for bf16 / d = 128 / chunk 64, CUDA-core path otherwise).
+gdn_status enqueue_prefill(const gdn::PrefillArgs &a, cudaStream_t stream) {
+    gdn_status st = check_prefill(a);
+    if (st != GDN_OK) return st;
+    if (a.N == 0) return GDN_OK;
+    cudaError_t err;
+    if (tc_path(a.dk, a.dv, a.chunk, a.dtype)) {
+        const size_t need = gdn::prefill_cluster_workspace(a.N, a.T, a.HV, a.chunk, a.cu_seqlens != nullptr);
+        if (need > 0 && (a.workspace == nullptr || a.workspace_bytes < need)) return GDN_ERR_WORKSPACE;
+        if (!aligned16(a.workspace)) return GDN_ERR_ALIGNMENT;
+        err = gdn::launch_prefill_cluster(a, stream);
+    } else {
+        err = gdn::launch_prefill_simt(a, stream);
+    }
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// Device workspace of gdn_chunk_prefill_host: the status word, two input and two
+// output segment buffers (inputs packed q | k | v | g | beta) and two states.
+struct HostPlan {
+    int64_t seg;
+    size_t elt, q_bytes, v_bytes, g_bytes;
+    size_t status, in[2], out[2], st[2], total;
+    static size_t up(size_t x) { return (x + 255) & ~size_t(255); }
+    HostPlan(int N, int64_t T, int HK, int HV, int dk, int dv, gdn_dtype dtype, int64_t segment) {
+        seg = segment > 0 ? segment : 4096;
+        if (T > 0 && seg > T) seg = T;
+        if (seg <= 0) seg = 1;
+        elt = dtype == GDN_BF16 ? 2 : 4;
+        const size_t rows = (size_t)N * (size_t)seg;
+        q_bytes = up(rows * HK * dk * elt);
+        v_bytes = up(rows * HV * dv * elt);
+        g_bytes = up(rows * HV * 4);
+        const size_t in_b = 2 * q_bytes + v_bytes + 2 * g_bytes;
+        const size_t out_b = v_bytes;
+        const size_t st_b = up((size_t)N * HV * dv * dk * 4);
+        status = 0;
+        size_t off = 256;
+        for (int b = 0; b < 2; ++b) { in[b] = off; off += in_b; }
+        for (int b = 0; b < 2; ++b) { out[b] = off; off += out_b; }
+        for (int b = 0; b < 2; ++b) { st[b] = off; off += st_b; }
+        total = off;
+    }
+};
 
 }  // namespace
 
@@ -70,19 +118,113 @@ gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v, const 
                              size_t workspace_bytes, gdn_stream_t stream) {
     gdn::PrefillArgs a{q, k, v, g, beta, h0, cu_seqlens, N, T, HK, HV, dk, dv, chunk,
                        scale, dtype, o, hT, workspace, workspace_bytes};
-    gdn_status st = check_prefill(a);
-    if (st != GDN_OK) return st;
-    if (N == 0) return GDN_OK;
-    cudaError_t err;
-    if (tc_path(dk, dv, chunk, dtype)) {
-        const size_t need = gdn::prefill_cluster_workspace(N, T, HV, chunk, cu_seqlens != nullptr);
-        if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
-        if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
-        err = gdn::launch_prefill_cluster(a, reinterpret_cast<cudaStream_t>(stream));
-    } else {
-        err = gdn::launch_prefill_simt(a, reinterpret_cast<cudaStream_t>(stream));
+    return enqueue_prefill(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t gdn_chunk_prefill_host_workspace_size(int N, int64_t T, int HK, int HV, int dk, int dv,
+                                             int chunk, gdn_dtype dtype, int64_t segment) {
+    if (N <= 0 || T < 0 || HK <= 0 || HV <= 0 || HV % HK || chunk <= 0 || segment < 0) return 0;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return 0;
+    if (gdn_chunk_prefill_path(dk, dv, chunk, dtype) < 0) return 0;
+    return HostPlan(N, T, HK, HV, dk, dv, dtype, segment).total;
+}
+
+gdn_status gdn_chunk_prefill_host(const void *q, const void *k, const void *v, const float *g,
+                                  const float *beta, const float *h0, int N, int64_t T, int HK,
+                                  int HV, int dk, int dv, int chunk, float scale, gdn_dtype dtype,
+                                  void *o, float *hT, void *workspace, size_t workspace_bytes,
+                                  int64_t segment, gdn_stream_t stream, gdn_stream_t copy_in,
+                                  gdn_stream_t copy_out) {
+    // validate the per-segment call once, with device-side stand-ins for the host buffers
+    if (!q || !k || !v || !g || !beta || !o) return GDN_ERR_INVALID_ARG;
+    if (N <= 0 || T < 0 || segment < 0) return GDN_ERR_INVALID_ARG;
+    {
+        gdn::PrefillArgs a{q, k, v, g, beta, h0, nullptr, N, T, HK, HV, dk, dv, chunk,
+                           scale, dtype, o, hT, nullptr, 0};
+        const gdn_status st = check_prefill(a);
+        if (st != GDN_OK) return st;
     }
-    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    const HostPlan plan(N, T, HK, HV, dk, dv, dtype, segment);
+    if (workspace == nullptr || workspace_bytes < plan.total) return GDN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_ALIGNMENT;
+    if (T == 0) return GDN_OK;
+    cudaStream_t sc = reinterpret_cast<cudaStream_t>(stream);
+    cudaStream_t si = reinterpret_cast<cudaStream_t>(copy_in);
+    cudaStream_t so = reinterpret_cast<cudaStream_t>(copy_out);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const int64_t S = plan.seg, nseg = (T + S - 1) / S;
+    // the events that order the three streams; destroyed below once enqueued (the
+    // runtime keeps each alive until it has completed)
+    const int nev = (int)(3 * nseg + 1);
+    cudaEvent_t evs_local[64];
+    cudaEvent_t *evs = nev <= 64 ? evs_local : new (std::nothrow) cudaEvent_t[nev];
+    if (!evs) return GDN_ERR_CUDA;
+    int made = 0;
+    gdn_status result = GDN_OK;
+    for (; made < nev; ++made)
+        if (cudaEventCreateWithFlags(&evs[made], cudaEventDisableTiming) != cudaSuccess) {
+            result = GDN_ERR_CUDA;
+            break;
+        }
+    auto ev_in = [&](int64_t s) { return evs[1 + 3 * s]; };
+    auto ev_done = [&](int64_t s) { return evs[2 + 3 * s]; };
+    auto ev_out = [&](int64_t s) { return evs[3 + 3 * s]; };
+    auto ok = [&](cudaError_t e) {
+        if (e != cudaSuccess && result == GDN_OK) result = GDN_ERR_CUDA;
+        return result == GDN_OK;
+    };
+    const size_t eq = plan.elt * (size_t)HK * dk, ev = plan.elt * (size_t)HV * dv, eg = 4u * HV;
+    // the copy streams start after everything already queued on the compute stream
+    if (result == GDN_OK && ok(cudaEventRecord(evs[0], sc)) && ok(cudaStreamWaitEvent(si, evs[0], 0)))
+        ok(cudaStreamWaitEvent(so, evs[0], 0));
+    if (result == GDN_OK) ok(cudaMemsetAsync(ws + plan.status, 0, sizeof(unsigned int), sc));
+    for (int64_t s = 0; s < nseg && result == GDN_OK; ++s) {
+        const int64_t t0 = s * S, Ls = T - t0 < S ? T - t0 : S;
+        const int b = (int)(s & 1);
+        uint8_t *in = ws + plan.in[b];
+        uint8_t *dq = in, *dk_ = in + plan.q_bytes, *dv_ = dk_ + plan.q_bytes,
+                *dg = dv_ + plan.v_bytes, *db = dg + plan.g_bytes;
+        // inputs of segment s into buffer b (free once segment s - 2 is computed)
+        if (s >= 2 && !ok(cudaStreamWaitEvent(si, ev_done(s - 2), 0))) break;
+        const struct { const void *src; void *dst; size_t row; } cp[5] = {
+            {q, dq, eq}, {k, dk_, eq}, {v, dv_, ev}, {g, dg, eg}, {beta, db, eg}};
+        for (const auto &c : cp)
+            if (!ok(cudaMemcpy2DAsync(c.dst, (size_t)Ls * c.row,
+                                      static_cast<const uint8_t *>(c.src) + (size_t)t0 * c.row,
+                                      (size_t)T * c.row, (size_t)Ls * c.row, (size_t)N,
+                                      cudaMemcpyHostToDevice, si)))
+                break;
+        if (result != GDN_OK || !ok(cudaEventRecord(ev_in(s), si))) break;
+        // segment s: state from the previous segment (or h0), outputs into buffer b
+        // (free once segment s - 2's outputs have been copied out)
+        if (!ok(cudaStreamWaitEvent(sc, ev_in(s), 0))) break;
+        if (s >= 2 && !ok(cudaStreamWaitEvent(sc, ev_out(s - 2), 0))) break;
+        const float *hin = s == 0 ? h0 : reinterpret_cast<const float *>(ws + plan.st[(s - 1) & 1]);
+        float *hout = (s == nseg - 1 && hT) ? hT : reinterpret_cast<float *>(ws + plan.st[b]);
+        uint8_t *out = ws + plan.out[b];
+        gdn::PrefillArgs a{dq, dk_, dv_, reinterpret_cast<const float *>(dg),
+                           reinterpret_cast<const float *>(db), hin, nullptr, N, Ls, HK, HV, dk,
+                           dv, chunk, scale, dtype, out, hout, ws + plan.status, 256};
+        a.keep_status = true;
+        const gdn_status st = enqueue_prefill(a, sc);
+        if (st != GDN_OK) {
+            result = st;
+            break;
+        }
+        if (!ok(cudaEventRecord(ev_done(s), sc))) break;
+        // outputs of segment s back to the host
+        if (!ok(cudaStreamWaitEvent(so, ev_done(s), 0))) break;
+        if (!ok(cudaMemcpy2DAsync(static_cast<uint8_t *>(o) + (size_t)t0 * ev, (size_t)T * ev, out,
+                                  (size_t)Ls * ev, (size_t)Ls * ev, (size_t)N,
+                                  cudaMemcpyDeviceToHost, so)))
+            break;
+        ok(cudaEventRecord(ev_out(s), so));
+    }
+    // everything the call enqueued is ordered before later work on the compute stream
+    if (result == GDN_OK) ok(cudaStreamWaitEvent(sc, ev_out(nseg - 1), 0));
+    for (int i = 0; i < made; ++i) cudaEventDestroy(evs[i]);
+    if (evs != evs_local) delete[] evs;
+    return result;
 }
 
 gdn_status gdn_recurrent_step(const void *q, const void *k, const void *v, const float *g,

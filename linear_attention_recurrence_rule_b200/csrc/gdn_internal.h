@@ -22,6 +22,7 @@ struct PrefillArgs {
     float *hT;
     void *workspace;
     size_t workspace_bytes;
+    bool keep_status = false;   // leave the workspace status word as earlier calls left it
 };
 
 struct StepArgs {

@@ -915,7 +915,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     const int64_t Ttot = a.cu_seqlens ? a.T : (int64_t)a.N * a.T;
     if (Ttot >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     unsigned int *status = static_cast<unsigned int *>(a.workspace);
-    cudaError_t err = cudaMemsetAsync(status, 0, sizeof(unsigned int), stream);
+    cudaError_t err = a.keep_status ? cudaSuccess : cudaMemsetAsync(status, 0, sizeof(unsigned int), stream);
     if (err != cudaSuccess) return err;
     CUtensorMap tq, tk, tv, to;
     const uint64_t tok = (uint64_t)(Ttot > 0 ? Ttot : 1);

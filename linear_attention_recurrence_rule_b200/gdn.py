@@ -61,6 +61,13 @@ def load_library() -> ctypes.CDLL:
             lib.gdn_chunk_prefill_path.argtypes = [i32, i32, i32, i32]
             lib.gdn_read_status.restype = i32
             lib.gdn_read_status.argtypes = [vp, sz, vp]
+            lib.gdn_chunk_prefill_host_workspace_size.restype = sz
+            lib.gdn_chunk_prefill_host_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32,
+                                                                  i32, i32, i64]
+            lib.gdn_chunk_prefill_host.restype = i32
+            lib.gdn_chunk_prefill_host.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                                   i32, i32, i32, ctypes.c_float, i32, vp, vp,
+                                                   vp, sz, i64, vp, vp, vp]
             _handle = lib
     return _handle
 
@@ -204,3 +211,82 @@ def gdn_read_status(workspace, stream=None) -> int:
     return int(load_library().gdn_read_status(
         _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream_ptr(stream, workspace.device)))
+
+
+_copy_streams = {}
+
+
+def _host_need(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def gdn_chunk_prefill_host_workspace_size(N, T, HK, HV, dk, dv, chunk, dtype, segment=0) -> int:
+    code = dtype if isinstance(dtype, int) else _dtype_code(torch.empty(0, dtype=dtype))
+    return int(load_library().gdn_chunk_prefill_host_workspace_size(
+        int(N), int(T), int(HK), int(HV), int(dk), int(dv), int(chunk), code, int(segment)))
+
+
+def gdn_chunk_prefill_host(q, k, v, g, beta, h0=None, chunk: int = 64, scale: float = 1.0,
+                           o=None, hT=None, workspace=None, segment: int = 0, device=None,
+                           stream=None, copy_streams=None, output_final_state: bool = True):
+    """Prefill of host-resident data through ``gdn_chunk_prefill_host``.
+
+    q, k [B,T,HK,dk]; v [B,T,HV,dv]; g, beta [B,T,HV] fp32 -- CPU tensors (pinned
+    memory lets the copies overlap the computation); o: CPU output [B,T,HV,dv]
+    (allocated pinned if None).  h0, hT: CUDA tensors [B,HV,dv,dk] fp32 or None.
+    copy_streams: (copy_in, copy_out) CUDA streams; two cached side streams of the
+    device are used if None.  Returns (o, hT); the results are ready once
+    ``stream`` (default: the current stream) has been synchronised.
+    """
+    lib = load_library()
+    dev = torch.device(device) if device is not None else (
+        h0.device if h0 is not None else torch.device("cuda", torch.cuda.current_device()))
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _host_need(t, name, q.dtype)
+    _host_need(g, "g", torch.float32)
+    _host_need(beta, "beta", torch.float32)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("expected q,k [B,T,HK,dk] and v [B,T,HV,dv]")
+    B, T, HK, dk = q.shape
+    HV, dv = v.shape[2], v.shape[3]
+    if g.shape != (B, T, HV) or beta.shape != (B, T, HV):
+        raise ValueError("expected g, beta [B,T,HV]")
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, dev)
+        if h0.shape != (B, HV, dv, dk):
+            raise ValueError(f"h0 must be [B,HV,dv,dk] = {(B, HV, dv, dk)}")
+    if o is None:
+        o = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+    else:
+        _host_need(o, "o", v.dtype)
+    if hT is None and output_final_state:
+        hT = torch.empty((B, HV, dv, dk), dtype=torch.float32, device=dev)
+    elif hT is not None:
+        _need(hT, "hT", torch.float32, dev)
+    code = _dtype_code(q)
+    need = lib.gdn_chunk_prefill_host_workspace_size(B, T, HK, HV, dk, dv, chunk, code,
+                                                     int(segment))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if copy_streams is None:
+        key = dev.index
+        if key not in _copy_streams:
+            _copy_streams[key] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+        copy_streams = _copy_streams[key]
+    st = lib.gdn_chunk_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), B,
+                                    T, HK, HV, dk, dv, int(chunk), float(scale), code, _ptr(o),
+                                    _ptr(hT), _ptr(workspace), ws_bytes, int(segment),
+                                    _stream_ptr(stream, dev),
+                                    ctypes.c_void_p(copy_streams[0].cuda_stream),
+                                    ctypes.c_void_p(copy_streams[1].cuda_stream))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_chunk_prefill_host")
+    return o, hT
