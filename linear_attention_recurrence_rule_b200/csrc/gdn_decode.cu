@@ -15,10 +15,13 @@
 // stored once (128-bit, streaming).  The two dot products of a row are reduced
 // with warp shuffles inside the lanes that hold the row.
 //
-// Work split: one CTA of 8 warps per (sequence, value head).  A row of dk fp32
-// is held by dk/4 lanes (one float4 each); a warp instruction covers 32/(dk/4)
-// rows; each warp issues NB such loads before using any of them, so every lane
-// has NB x 16 B of state in flight.
+// Work split: CTAs of 8 warps, each owning a band of rows of one (sequence,
+// value head) state (grid.y walks the bands).  A row of dk fp32 is held by dk/4
+// lanes (one float4 each); a warp instruction covers 32/(dk/4) rows; each warp
+// issues NB such loads before using any of them, so every lane has NB x 16 B of
+// state in flight.  Bands of 8 x NB rows (64 at dk = 128) keep CTAs short and
+// several of them resident per SM, so their load, update and store phases
+// overlap.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -26,10 +29,13 @@ namespace gdn {
 namespace {
 
 constexpr int kDecodeWarps = 8;
-constexpr int kDecodeNB = 16;
+constexpr int kDecodeNB = 8;
+
+template <int DK>
+constexpr int band_rows() { return kDecodeWarps * (32 / (DK / 4)) * kDecodeNB; }
 
 template <int DK, typename Tin>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
+__global__ void __launch_bounds__(kDecodeWarps * 32, 3)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ g, const float *__restrict__ beta, float *state,
               Tin *__restrict__ o, int HK, int HV, int dv, float scale) {
@@ -54,7 +60,8 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     float *S = state + (size_t)nh * dv * DK;
 
     constexpr int rows_per_batch = kDecodeWarps * RPI * kDecodeNB;
-    for (int base = 0; base < dv; base += rows_per_batch) {
+    {
+        const int base = blockIdx.y * rows_per_batch;
         float4 s[kDecodeNB];
 #pragma unroll
         for (int j = 0; j < kDecodeNB; ++j) {
@@ -87,7 +94,9 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 
 template <typename Tin>
 cudaError_t launch_typed(const StepArgs &a, cudaStream_t stream) {
-    const dim3 grid((unsigned)((size_t)a.N * a.HV)), block(kDecodeWarps * 32);
+    const int band = a.dk == 128 ? band_rows<128>() : a.dk == 64 ? band_rows<64>() : band_rows<32>();
+    const dim3 grid((unsigned)((size_t)a.N * a.HV), (unsigned)((a.dv + band - 1) / band)),
+        block(kDecodeWarps * 32);
     const Tin *q = static_cast<const Tin *>(a.q);
     const Tin *k = static_cast<const Tin *>(a.k);
     const Tin *v = static_cast<const Tin *>(a.v);

@@ -197,6 +197,24 @@ def test_decode_fp32_tight():
     assert_close(S, Sref, torch.float32, "state")
 
 
+@pytest.mark.parametrize("N,HK,HV,dk,dv,dtype", [
+    (40, 2, 4, 64, 48, torch.float32),     # 160 states: the persistent streaming kernel
+    (37, 1, 4, 32, 200, torch.bfloat16),   # 148 states, rows not a multiple of a pass
+    (300, 2, 4, 128, 128, torch.bfloat16), # several states per SM
+    (9, 1, 2, 128, 256, torch.float32),    # 128 KB states: the register kernel
+])
+def test_decode_streaming_shapes(N, HK, HV, dk, dv, dtype):
+    x = make_decode(N, 2, HK, HV, dk, dv, dtype, seed=11, h0_std=0.3)
+    d = to_dev(x)
+    S = d["state"].clone()
+    Sref = x["state"]
+    for t in range(2):
+        o = gdn_recurrent_step(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], S)
+        o_ref, Sref = O.step(x["q"][t], x["k"][t], x["v"][t], x["g"][t], x["beta"][t], Sref)
+        assert_close(o, o_ref, dtype, f"o step {t}")
+    assert_close(S, Sref, dtype, "state")
+
+
 def test_split_resume_equals_whole():
     x = make_prefill(2, 4, 128, 128, [700], torch.bfloat16, seed=31, h0_std=0.05)
     d = to_dev(x)
