@@ -154,6 +154,17 @@ GDN_API gdn_status gdn_chunk_prefill_noalloc(const void *q, const void *k, const
                                              gdn_stream_t stream);
 
 /*
+ * Opt-in check of a device cu_seqlens array before gdn_chunk_prefill (which
+ * takes its contents as a precondition): one small kernel on `stream` writes to
+ * the DEVICE int *result 0 when cu_seqlens[0] = 0, the entries never decrease
+ * and cu_seqlens[N] = T, else 1 + the first offending index.  Returns
+ * GDN_ERR_INVALID_ARG for NULL pointers or negative sizes, GDN_ERR_CUDA if the
+ * launch fails.
+ */
+GDN_API gdn_status gdn_validate_cu_seqlens(const int32_t *cu_seqlens, int N, int64_t T,
+                                           int *result, gdn_stream_t stream);
+
+/*
  * Bytes of device workspace gdn_chunk_prefill_host needs (0 for arguments it
  * would reject).  segment: tokens per segment, 0 selects the default (4096).
  */

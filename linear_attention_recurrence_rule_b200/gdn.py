@@ -61,6 +61,8 @@ def load_library() -> ctypes.CDLL:
             lib.gdn_chunk_prefill_path.argtypes = [i32, i32, i32, i32]
             lib.gdn_read_status.restype = i32
             lib.gdn_read_status.argtypes = [vp, sz, vp]
+            lib.gdn_validate_cu_seqlens.restype = i32
+            lib.gdn_validate_cu_seqlens.argtypes = [vp, i32, i64, vp, vp]
             lib.gdn_chunk_prefill_host_workspace_size.restype = sz
             lib.gdn_chunk_prefill_host_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32,
                                                                   i32, i32, i64]
@@ -290,3 +292,17 @@ def gdn_chunk_prefill_host(q, k, v, g, beta, h0=None, chunk: int = 64, scale: fl
     if st != GDN_OK:
         raise GDNError(st, "gdn_chunk_prefill_host")
     return o, hT
+
+
+def gdn_validate_cu_seqlens(cu_seqlens, T, stream=None) -> int:
+    """Runs ``gdn_validate_cu_seqlens`` on a device int32 [N+1] tensor and waits for
+    it: 0 when valid, else 1 + the first offending index."""
+    lib = load_library()
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    dev = cu_seqlens.device
+    res = torch.empty(1, dtype=torch.int32, device=dev)
+    st = lib.gdn_validate_cu_seqlens(_ptr(cu_seqlens), cu_seqlens.numel() - 1, int(T), _ptr(res),
+                                     _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_validate_cu_seqlens")
+    return int(res.item())

@@ -161,3 +161,38 @@ def step(q, k, v, g, beta, state, scale=1.0, lib=None):
     if rc != 0:
         raise ValueError(f"oracle rejected the arguments (rc={rc})")
     return o, S
+
+
+def verify(q, k, v, g, beta, state, scale=1.0, lib=None):
+    """K draft tokens per sequence, checked at once (speculative decoding: the
+    main model processes several proposed tokens and keeps those it accepts --
+    "Qwen3-Next", sghael.github.io, section "Speed depends on the serving
+    software").  The rule is applied token after token from ``state``; the
+    outputs of every token and the state after every token are returned, so a
+    caller can roll back to the state after the last accepted token.
+
+    q,k [N,K,HK,dk]; v [N,K,HV,dv]; g,beta [N,K,HV]; state [N,HV,dv,dk].
+    Returns (o [N,K,HV,dv], states [N,K,HV,dv,dk]) float64; ``state`` is not
+    modified.
+    """
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    S = _f64(state).copy()
+    N, K = q.shape[0], q.shape[1]
+    HV, dv, dk = S.shape[1], S.shape[2], S.shape[3]
+    o = np.zeros((N, K, HV, dv), dtype=np.float64)
+    states = np.zeros((N, K, HV, dv, dk), dtype=np.float64)
+    for j in range(K):
+        o[:, j], S = step(q[:, j], k[:, j], v[:, j], g[:, j], beta[:, j], S, scale=scale, lib=lib)
+        states[:, j] = S
+    return o, states
+
+
+def commit(states, accepted, state):
+    """Roll back to the accepted prefix: for each sequence n, the state after its
+    accepted[n] draft tokens (states[n, accepted[n] - 1]), or ``state[n]``
+    unchanged when none was accepted.  Returns the new [N,HV,dv,dk] array."""
+    states, S = _f64(states), _f64(state).copy()
+    for n, a in enumerate(np.asarray(accepted).tolist()):
+        if a > 0:
+            S[n] = states[n, a - 1]
+    return S

@@ -313,4 +313,41 @@ def pin_scale_multiplies_readout(lib=None):
     assert np.allclose(o2, 0.25 * o1, atol=1e-14) and np.allclose(h2, h1, atol=1e-14)
 
 
+def pin_verify_equals_prefill_of_drafts(lib=None):
+    """Checking K drafts at once gives, for every draft j, the outputs and the
+    state that a chunked prefill (the independent WY form) of the first j+1
+    drafts gives from the same start state."""
+    rng = np.random.default_rng(15)
+    N, K, HK, HV, d = 3, 5, 2, 4, 6
+    probs = [_rand_problem(rng, K, HK, HV, d, d) for _ in range(N)]
+    q, k, v, g, beta = (np.concatenate([p_[i] for p_ in probs]) for i in range(5))
+    S0 = rng.standard_normal((N, HV, d, d))
+    o, states = O.verify(q, k, v, g, beta, S0, scale=0.5, lib=lib)
+    assert o.shape == (N, K, HV, d) and states.shape == (N, K, HV, d, d)
+    for n in range(N):
+        for j in range(K):
+            op, hp = O.prefill(q[n:n + 1, :j + 1], k[n:n + 1, :j + 1], v[n:n + 1, :j + 1],
+                               g[n:n + 1, :j + 1], beta[n:n + 1, :j + 1], h0=S0[n:n + 1],
+                               scale=0.5, chunked=True, chunk=2, lib=lib)
+            assert np.allclose(o[n, j], op[j], atol=1e-12)
+            assert np.allclose(states[n, j], hp[0], atol=1e-12)
+
+
+def pin_commit_rolls_back_to_accepted_prefix(lib=None):
+    rng = np.random.default_rng(16)
+    N, K, HV, d = 3, 4, 2, 5
+    probs = [_rand_problem(rng, K, 1, HV, d, d) for _ in range(N)]
+    q, k, v, g, beta = (np.concatenate([p_[i] for p_ in probs]) for i in range(5))
+    S0 = rng.standard_normal((N, HV, d, d))
+    _, states = O.verify(q, k, v, g, beta, S0, lib=lib)
+    accepted = [0, 2, K]
+    S = O.commit(states, accepted, S0)
+    assert np.array_equal(S[0], S0[0])
+    for n in (1, 2):
+        _, hp = O.prefill(q[n:n + 1, :accepted[n]], k[n:n + 1, :accepted[n]],
+                          v[n:n + 1, :accepted[n]], g[n:n + 1, :accepted[n]],
+                          beta[n:n + 1, :accepted[n]], h0=S0[n:n + 1], lib=lib)
+        assert np.allclose(S[n], hp[0], atol=1e-12)
+
+
 ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

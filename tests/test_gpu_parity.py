@@ -230,3 +230,17 @@ def test_split_resume_equals_whole():
     assert_close(torch.cat([o1, o2], 1), o_ref, torch.bfloat16, "split o")
     assert_close(h2, h_ref, torch.bfloat16, "split hT")
     assert_close(o, o_ref, torch.bfloat16, "whole o")
+
+
+def test_validate_cu_seqlens():
+    from linear_attention_recurrence_rule_b200 import gdn_validate_cu_seqlens
+    cu = lambda xs: torch.tensor(xs, dtype=torch.int32, device="cuda")
+    assert gdn_validate_cu_seqlens(cu([0, 5, 5, 12]), 12) == 0
+    assert gdn_validate_cu_seqlens(cu([0]), 0) == 0
+    assert gdn_validate_cu_seqlens(cu([1, 5, 12]), 12) == 1           # does not start at 0
+    assert gdn_validate_cu_seqlens(cu([0, 7, 5, 12]), 12) == 3        # decreases at index 2
+    assert gdn_validate_cu_seqlens(cu([0, 5, 11]), 12) == 3           # does not end at T
+    big = torch.arange(0, 3001 * 4, 4, dtype=torch.int32, device="cuda")
+    assert gdn_validate_cu_seqlens(big, 12000) == 0
+    big[1777] = 0
+    assert gdn_validate_cu_seqlens(big, 12000) == 1778
