@@ -8,7 +8,9 @@ Gated DeltaNet layer over one synthetic sequence: B=1, T=65536, 16 query/key
 heads shared by 32 value heads, head dim 128, chunk 64, bf16 q/k/v, fp32
 g/beta/state.  The same run also measures the fused decode step
 (``gdn_recurrent_step``) on 256 sequences x 64 tokens and reports its state
-HBM bandwidth in the ``decode`` object.
+HBM bandwidth in the ``decode`` object, and the speculative-decoding round
+(``gdn_recurrent_verify`` of 4 drafts per sequence + the commit of the accepted
+prefix) in the ``verify`` object.
 
 Launch: ``python bench.py [--gpus N --steps K --warmup W]``; for N > 1 under
 ``torch.distributed.run``, one replica per GPU (each rank runs its own
@@ -34,6 +36,7 @@ sys.path.insert(0, ROOT)
 METRIC = "GDN prefill tokens/s (T=64K, 32 V heads); decode state HBM GB/s vs peak"
 WORKLOAD = "long_prefill_64k"
 DECODE_WORKLOAD = "decode_256x64"
+VERIFY_WORKLOAD = "verify_256x4"
 
 # Fallback peaks (only if the measured-peaks file is absent).
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
@@ -57,6 +60,104 @@ def prefill_min_bytes_per_token(HK, HV, d, elt=2):
 def decode_bytes_per_step(N, HK, HV, dk, dv, elt=2):
     """State read + write (fp32) plus q, k, v, o, g, beta."""
     return 2 * N * HV * dv * dk * 4 + 2 * N * HK * dk * elt + 2 * N * HV * dv * elt + 2 * N * HV * 4
+
+
+def verify_bytes(N, K, HK, HV, dk, dv, accepted, rollback, elt=2):
+    """Algorithmic HBM bytes of one verify + commit round (state fp32).
+
+    verify: the state read once, q, k, v, o, g, beta of K drafts, plus either
+    every draft's state ("states") or every draft's update vector u ("deltas").
+    commit: the state of each sequence that kept >= 1 draft read and written
+    once; the deltas form also reads k, g and u of the kept drafts, the states
+    form the selected state instead of the current one."""
+    state = HV * dv * dk * 4                      # one sequence
+    io = N * K * (2 * HK * dk * elt + 2 * HV * dv * elt + 2 * HV * 4)
+    kept = sum(1 for a in accepted if 1 <= a <= K)
+    drafts_kept = sum(a for a in accepted if 1 <= a <= K)
+    if rollback == "states":
+        ver = N * state * (1 + K) + io
+        com = kept * 2 * state + N * 4
+    else:
+        ver = N * state + io + N * K * HV * dv * 4
+        com = kept * 2 * state + drafts_kept * (HK * dk * elt + HV * 4 + HV * dv * 4) + N * 4
+    return ver, com
+
+
+def measure_verify(gdn, torch, dev, stream, peaks, peak_src, rank, world, max_over_ranks,
+                   barrier, args):
+    """Speculative-decoding round on the verify_256x4 workload: K=4 drafts per
+    sequence checked in one pass (``gdn_recurrent_verify``), then the accepted
+    prefix kept (``gdn_state_commit_deltas`` / ``gdn_state_commit``).  The
+    acceptance counts are synthetic, ~U{0..K} per sequence from the seed."""
+    from linear_attention_recurrence_rule_b200.inputs import WORKLOADS, workload_inputs
+    name = VERIFY_WORKLOAD
+    wv = WORKLOADS[name]
+    y = workload_inputs(name, seed_offset=replica_seed_offset(rank))
+    dy = {k: v.to(dev) for k, v in y.items()}
+    N, K = wv.B, wv.T
+    gen = torch.Generator().manual_seed(wv.seed + 77 + rank)
+    acc_host = torch.randint(0, K + 1, (N,), generator=gen, dtype=torch.int32)
+    accepted = acc_host.to(dev)
+    S = dy["state"].clone()
+    o = torch.empty_like(dy["v"])
+    u = torch.empty((N, K, wv.HV, wv.dv), dtype=torch.float32, device=dev)
+    states = torch.empty((N, K, wv.HV, wv.dv, wv.dk), dtype=torch.float32, device=dev)
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    out = {"workload": name, "drafts": K, "sequences": N,
+           "accepted_mean": float(acc_host.float().mean()),
+           "acceptance": "synthetic ~U{0..K} per sequence"}
+    rounds = max(1, args.verify_rounds)
+    for form in ("deltas", "states"):
+        def verify():
+            if form == "deltas":
+                gdn.gdn_recurrent_verify(dy["q"], dy["k"], dy["v"], dy["g"], dy["beta"], S, o=o,
+                                         u_out=u, rollback="deltas", stream=stream)
+            else:
+                gdn.gdn_recurrent_verify(dy["q"], dy["k"], dy["v"], dy["g"], dy["beta"], S, o=o,
+                                         states_out=states, rollback="states", stream=stream)
+
+        def commit():
+            if form == "deltas":
+                gdn.gdn_state_commit_deltas(dy["k"], dy["g"], u, accepted, S, stream=stream)
+            else:
+                gdn.gdn_state_commit(states, accepted, S, stream=stream)
+
+        S.copy_(dy["state"])
+        for _ in range(max(3, args.warmup)):
+            verify()
+            commit()
+        S.copy_(dy["state"])
+        torch.cuda.synchronize()
+        barrier()
+        sampler = ClockSampler(int(dev.index or 0))
+        sampler.start()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(rounds)]
+        for r in range(rounds):
+            ev[r][0].record(stream)
+            verify()
+            ev[r][1].record(stream)
+            commit()
+            ev[r][2].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        clocks = sampler.stop()
+        v_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+        c_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+        total_ms = max_over_ranks(ev[0][0].elapsed_time(ev[-1][2]))
+        vb, cb = verify_bytes(N, K, wv.HK, wv.HV, wv.dk, wv.dv, acc_host.tolist(), form)
+        v_gbs = vb / (v_ms / 1e3) / 1e9
+        c_gbs = cb / (c_ms / 1e3) / 1e9
+        out[form] = {
+            "value": world * N * K * rounds / (total_ms / 1e3), "unit": "draft tokens/s",
+            "ms_per_round": total_ms / rounds, "verify_ms": v_ms, "commit_ms": c_ms,
+            "bytes_per_round": vb + cb, "gb_per_s": (vb + cb) / (total_ms / rounds / 1e3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": v_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": v_gbs / hbm_peak, "traffic": None, "peak_source": peak_src,
+                         "kernel": "verify"},
+            "commit_roofline": {"bound": "hbm", "achieved": c_gbs, "peak": hbm_peak,
+                                "unit": "GB/s", "frac": c_gbs / hbm_peak},
+            "gpu_launches": 2 * rounds, "clocks": clocks}
+    return out
 
 
 def dist_max(x, device=None):
@@ -425,6 +526,11 @@ def run_b200(args):
                "bytes_per_step": bytes_step, "gpu_launches": wd.T, "clocks": dclocks,
                "l2": "state 537 MB per step, larger than L2"}
 
+    ver = None
+    if not args.no_verify:
+        ver = measure_verify(gdn, torch, dev, stream, peaks, peak_src, rank, world,
+                             max_over_ranks, barrier, args)
+
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(args.cpu_seconds)
@@ -443,6 +549,7 @@ def run_b200(args):
                        "l2": "inputs larger than L2 (q,k,v 1.07 GB per step)"},
             "roofline": roof, "cpu_baseline": base, "e2e": e2e,
             "gpu_launches": launches_per_step * n_steps, "clocks": clocks, "decode": dec,
+            "verify": ver,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -460,6 +567,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-verify", action="store_true")
+    ap.add_argument("--verify-rounds", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="decode measurement only")
     ap.add_argument("--tokens", type=int, default=None,

@@ -228,6 +228,70 @@ GDN_API gdn_status gdn_recurrent_step(const void *q, const void *k, const void *
                               int dv, float scale, gdn_dtype dtype, void *o,
                               gdn_stream_t stream);
 
+/* Largest number of draft tokens gdn_recurrent_verify takes per sequence. */
+#define GDN_VERIFY_MAX_DRAFTS 16
+
+/*
+ * Multi-token verify step for speculative decoding (Qwen3-Next, "Speed depends
+ * on the serving software": the model checks several proposed tokens at once
+ * and keeps those it agrees with).  For each of N sequences, K draft tokens
+ * are run through the recurrence of gdn_recurrent_step one after another,
+ * starting from `state`, which is only read (once, from HBM, for all K
+ * tokens).  Every token's output is written; for rolling back to the last
+ * accepted draft the call also writes, when the pointer is not NULL:
+ *   states_out  the state AFTER every token (pair with gdn_state_commit), or
+ *   u_out       every token's update vector u_t = beta_t (v_t - alpha_t S_{t-1} k_t),
+ *               with which S_t = alpha_t S_{t-1} + u_t k_t^T (pair with
+ *               gdn_state_commit_deltas: K*dv floats per head instead of K
+ *               states, the cheaper form in HBM traffic).
+ *
+ * Layouts (token t of sequence n is row n*K + t):
+ *   q, k   [N][K][HK][dk] dtype      v, o [N][K][HV][dv] dtype
+ *   g, beta [N][K][HV] fp32          state [N][HV][dv][dk] fp32 (read)
+ *   states_out [N][K][HV][dv][dk] fp32   u_out [N][K][HV][dv] fp32
+ * Supported: as gdn_recurrent_step, and 1 <= K <= GDN_VERIFY_MAX_DRAFTS.
+ * Alignment: q, k, v, o, state, states_out 16-byte aligned, u_out 4-byte.
+ * No output may overlap an input.  K > GDN_VERIFY_MAX_DRAFTS returns
+ * GDN_ERR_UNSUPPORTED.  N == 0 is an empty batch (GDN_OK, nothing launched;
+ * pointers may be NULL).
+ */
+GDN_API gdn_status gdn_recurrent_verify(const void *q, const void *k, const void *v,
+                                        const float *g, const float *beta, const float *state,
+                                        int N, int K, int HK, int HV, int dk, int dv, float scale,
+                                        gdn_dtype dtype, void *o, float *states_out, float *u_out,
+                                        gdn_stream_t stream);
+
+/*
+ * Keeps the accepted drafts after gdn_recurrent_verify (states_out form): for
+ * each sequence n, state[n] <- states[n][accepted[n] - 1] when
+ * 1 <= accepted[n] <= K; state[n] is left unchanged when accepted[n] is 0 (or
+ * out of range, which is not an error: nothing was accepted).  accepted is a
+ * DEVICE array of N int32, so the acceptance decided on the GPU needs no round
+ * trip through the host.
+ * Layouts: states [N][K][HV][dv][dk] fp32, state [N][HV][dv][dk] fp32.
+ * Alignment: states, state 16-byte aligned, accepted 4-byte aligned; dv*dk a
+ * multiple of 4.  N == 0 is an empty batch (GDN_OK; pointers may be NULL).
+ */
+GDN_API gdn_status gdn_state_commit(const float *states, const int32_t *accepted, float *state,
+                                    int N, int K, int HV, int dk, int dv, gdn_stream_t stream);
+
+/*
+ * Keeps the accepted drafts after gdn_recurrent_verify (u_out form), updating
+ * `state` (the verify call's input state) in place: with a = accepted[n],
+ *   S <- (prod_{t<a} alpha_t) S + sum_{t<a} (prod_{t<s<a} alpha_s) u_t k_t^T,
+ * alpha_t = exp(g_t): the recurrence unrolled over the kept tokens.  Each
+ * state element is read and written once.  a == 0 or out of range leaves the
+ * state unchanged.  k and g are the verify call's inputs, u its u_out.
+ * Layouts: k [N][K][HK][dk] dtype, g [N][K][HV] fp32, u [N][K][HV][dv] fp32,
+ * accepted [N] int32 (device), state [N][HV][dv][dk] fp32.
+ * Supported: as gdn_recurrent_verify.  Alignment: k, state 16-byte aligned,
+ * u, accepted 4-byte.  N == 0 is an empty batch (GDN_OK; pointers may be NULL).
+ */
+GDN_API gdn_status gdn_state_commit_deltas(const void *k, const float *g, const float *u,
+                                           const int32_t *accepted, float *state, int N, int K,
+                                           int HK, int HV, int dk, int dv, gdn_dtype dtype,
+                                           gdn_stream_t stream);
+
 /*
  * Reads the device status word a prefill call left in its workspace (HOST
  * call; synchronises `stream`).  Returns GDN_OK when every on-device wait of

@@ -8,9 +8,13 @@
 #include "gdn.h"
 #include "gdn_internal.h"
 
+static_assert(gdn::kVerifyMaxDrafts == GDN_VERIFY_MAX_DRAFTS,
+              "the verify kernels size their shared memory for the declared draft limit");
+
 namespace {
 
 bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool tc_path(int dk, int dv, int chunk, gdn_dtype dt) {
     return gdn::prefill_cluster_supported(dk, dv, chunk, dt);
@@ -241,6 +245,56 @@ gdn_status gdn_recurrent_step(const void *q, const void *k, const void *v, const
     if (N == 0) return GDN_OK;
     gdn::StepArgs a{q, k, v, g, beta, state, N, HK, HV, dk, dv, scale, dtype, o};
     const cudaError_t err = gdn::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_recurrent_verify(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const float *state, int N, int K, int HK, int HV,
+                                int dk, int dv, float scale, gdn_dtype dtype, void *o,
+                                float *states_out, float *u_out, gdn_stream_t stream) {
+    if (N < 0 || K <= 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK)
+        return GDN_ERR_INVALID_ARG;
+    if (N == 0) return GDN_OK;   // empty batch: buffers may be NULL
+    if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (K > GDN_VERIFY_MAX_DRAFTS || (int64_t)N * HV > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
+    if (!gdn::decode_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
+        !aligned16(states_out) || !aligned4(u_out))
+        return GDN_ERR_ALIGNMENT;
+    gdn::VerifyArgs a{q, k, v, g, beta, state, states_out, u_out, N, K, HK, HV, dk, dv, scale,
+                      dtype, o};
+    const cudaError_t err = gdn::launch_verify(a, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_state_commit(const float *states, const int32_t *accepted, float *state, int N, int K,
+                            int HV, int dk, int dv, gdn_stream_t stream) {
+    if (N < 0 || K <= 0 || HV <= 0 || dk <= 0 || dv <= 0) return GDN_ERR_INVALID_ARG;
+    if (N == 0) return GDN_OK;   // empty batch: buffers may be NULL
+    if (!states || !accepted || !state) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)N * HV > 0x7fffffff || ((int64_t)dk * dv) % 4) return GDN_ERR_UNSUPPORTED;
+    if (!aligned16(states) || !aligned16(state) || !aligned4(accepted)) return GDN_ERR_ALIGNMENT;
+    if (N == 0) return GDN_OK;
+    const cudaError_t err = gdn::launch_commit(states, accepted, state, N, K, HV, dv, dk,
+                                               reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_state_commit_deltas(const void *k, const float *g, const float *u,
+                                   const int32_t *accepted, float *state, int N, int K, int HK,
+                                   int HV, int dk, int dv, gdn_dtype dtype, gdn_stream_t stream) {
+    if (N < 0 || K <= 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK)
+        return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (N == 0) return GDN_OK;   // empty batch: buffers may be NULL
+    if (!k || !g || !u || !accepted || !state) return GDN_ERR_INVALID_ARG;
+    if (K > GDN_VERIFY_MAX_DRAFTS || (int64_t)N * HV > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
+    if (!gdn::decode_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
+    if (!aligned16(k) || !aligned16(state) || !aligned4(u) || !aligned4(accepted))
+        return GDN_ERR_ALIGNMENT;
+    gdn::CommitDeltasArgs a{k, g, u, accepted, state, N, K, HK, HV, dk, dv, dtype};
+    const cudaError_t err = gdn::launch_commit_deltas(a, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -35,9 +35,36 @@ struct StepArgs {
     void *o;
 };
 
+struct VerifyArgs {
+    const void *q, *k, *v;
+    const float *g, *beta, *state;
+    float *states, *u;
+    int N, K, HK, HV, dk, dv;
+    float scale;
+    gdn_dtype dtype;
+    void *o;
+};
+
+
 // decode (gdn_decode.cu)
 bool decode_supported(int dk, int dv);
 cudaError_t launch_decode(const StepArgs &a, cudaStream_t stream);
+cudaError_t launch_verify(const VerifyArgs &a, cudaStream_t stream);
+
+// Largest draft count of the verify kernels (GDN_VERIFY_MAX_DRAFTS in gdn.h).
+constexpr int kVerifyMaxDrafts = 16;
+
+struct CommitDeltasArgs {
+    const void *k;
+    const float *g, *u;
+    const int32_t *accepted;
+    float *state;
+    int N, K, HK, HV, dk, dv;
+    gdn_dtype dtype;
+};
+cudaError_t launch_commit_deltas(const CommitDeltasArgs &a, cudaStream_t stream);
+cudaError_t launch_commit(const float *states, const int32_t *accepted, float *state, int N, int K,
+                          int HV, int dv, int dk, cudaStream_t stream);
 
 // CUDA-core chunked prefill (gdn_prefill_simt.cu)
 bool prefill_simt_supported(int dk, int dv, int chunk);

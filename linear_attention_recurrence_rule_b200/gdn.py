@@ -57,6 +57,14 @@ def load_library() -> ctypes.CDLL:
             lib.gdn_recurrent_step.restype = i32
             lib.gdn_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                                ctypes.c_float, i32, vp, vp]
+            lib.gdn_recurrent_verify.restype = i32
+            lib.gdn_recurrent_verify.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                                 i32, ctypes.c_float, i32, vp, vp, vp, vp]
+            lib.gdn_state_commit.restype = i32
+            lib.gdn_state_commit.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
+            lib.gdn_state_commit_deltas.restype = i32
+            lib.gdn_state_commit_deltas.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                                    i32, i32, vp]
             lib.gdn_chunk_prefill_path.restype = i32
             lib.gdn_chunk_prefill_path.argtypes = [i32, i32, i32, i32]
             lib.gdn_read_status.restype = i32
@@ -198,6 +206,112 @@ def gdn_recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, o=None, stre
     if st != GDN_OK:
         raise GDNError(st, "gdn_recurrent_step")
     return o
+
+
+def gdn_recurrent_verify(q, k, v, g, beta, state, scale: float = 1.0, o=None, states_out=None,
+                         u_out=None, rollback="states", stream=None):
+    """K draft tokens per sequence through ``gdn_recurrent_verify``; ``state`` is only read.
+
+    q, k [N,K,HK,dk]; v [N,K,HV,dv] (bf16 or fp32); g, beta [N,K,HV] fp32;
+    state [N,HV,dv,dk] fp32.  ``rollback`` picks what is written for the
+    commit: "states" (states_out [N,K,HV,dv,dk], the state after each draft),
+    "deltas" (u_out [N,K,HV,dv], each draft's update vector), "both" or "none".
+    Returns (o [N,K,HV,dv], states_out or None, u_out or None).
+    """
+    if rollback not in ("states", "deltas", "both", "none"):
+        raise ValueError("rollback must be 'states', 'deltas', 'both' or 'none'")
+    lib = load_library()
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(state, "state", torch.float32, dev)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("expected q,k [N,K,HK,dk] and v [N,K,HV,dv]")
+    N, K, HK, dk = q.shape
+    HV, dv = v.shape[2], v.shape[3]
+    if g.shape != (N, K, HV) or beta.shape != (N, K, HV) or state.shape != (N, HV, dv, dk):
+        raise ValueError("expected g,beta [N,K,HV] and state [N,HV,dv,dk]")
+    if o is None:
+        o = torch.empty_like(v)
+    else:
+        _need(o, "o", v.dtype, dev)
+        if o.shape != v.shape:
+            raise ValueError("o must have the shape of v")
+    if rollback in ("states", "both"):
+        if states_out is None:
+            states_out = torch.empty((N, K, HV, dv, dk), dtype=torch.float32, device=dev)
+        _need(states_out, "states_out", torch.float32, dev)
+        if states_out.shape != (N, K, HV, dv, dk):
+            raise ValueError("expected states_out [N,K,HV,dv,dk]")
+    else:
+        states_out = None
+    if rollback in ("deltas", "both"):
+        if u_out is None:
+            u_out = torch.empty((N, K, HV, dv), dtype=torch.float32, device=dev)
+        _need(u_out, "u_out", torch.float32, dev)
+        if u_out.shape != (N, K, HV, dv):
+            raise ValueError("expected u_out [N,K,HV,dv]")
+    else:
+        u_out = None
+    st = lib.gdn_recurrent_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                                  N, K, HK, HV, dk, dv, float(scale), _dtype_code(q), _ptr(o),
+                                  _ptr(states_out), _ptr(u_out), _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_recurrent_verify")
+    return o, states_out, u_out
+
+
+def gdn_state_commit(states, accepted, state, stream=None):
+    """state[n] <- states[n, accepted[n]-1] for 1 <= accepted[n] <= K (``gdn_state_commit``).
+
+    states [N,K,HV,dv,dk] fp32; accepted [N] int32 on the device; state
+    [N,HV,dv,dk] fp32, updated in place.  Returns state.
+    """
+    lib = load_library()
+    dev = state.device
+    _need(states, "states", torch.float32, dev)
+    _need(accepted, "accepted", torch.int32, dev)
+    _need(state, "state", torch.float32, dev)
+    if states.dim() != 5 or state.shape != (states.shape[0],) + tuple(states.shape[2:]) \
+            or accepted.shape != (states.shape[0],):
+        raise ValueError("expected states [N,K,HV,dv,dk], accepted [N], state [N,HV,dv,dk]")
+    N, K, HV, dv, dk = states.shape
+    st = lib.gdn_state_commit(_ptr(states), _ptr(accepted), _ptr(state), N, K, HV, dk, dv,
+                              _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_state_commit")
+    return state
+
+
+def gdn_state_commit_deltas(k, g, u, accepted, state, stream=None):
+    """In-place roll-back from a verify pass's update vectors (``gdn_state_commit_deltas``).
+
+    k [N,K,HK,dk] (the verify input, bf16 or fp32); g [N,K,HV] fp32; u
+    [N,K,HV,dv] fp32 (verify's u_out); accepted [N] int32 on the device; state
+    [N,HV,dv,dk] fp32 (verify's input state), updated in place.  Returns state.
+    """
+    lib = load_library()
+    dev = state.device
+    _need(k, "k", k.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(u, "u", torch.float32, dev)
+    _need(accepted, "accepted", torch.int32, dev)
+    _need(state, "state", torch.float32, dev)
+    if k.dim() != 4 or u.dim() != 4 or state.dim() != 4:
+        raise ValueError("expected k [N,K,HK,dk], u [N,K,HV,dv], state [N,HV,dv,dk]")
+    N, K, HK, dk = k.shape
+    HV, dv = u.shape[2], u.shape[3]
+    if u.shape[:2] != (N, K) or g.shape != (N, K, HV) or accepted.shape != (N,) \
+            or state.shape != (N, HV, dv, dk):
+        raise ValueError("expected k [N,K,HK,dk], g [N,K,HV], u [N,K,HV,dv], accepted [N], "
+                         "state [N,HV,dv,dk]")
+    st = lib.gdn_state_commit_deltas(_ptr(k), _ptr(g), _ptr(u), _ptr(accepted), _ptr(state), N, K,
+                                     HK, HV, dk, dv, _dtype_code(k), _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_state_commit_deltas")
+    return state
 
 
 def gdn_chunk_prefill_path(dk, dv, chunk, dtype) -> int:

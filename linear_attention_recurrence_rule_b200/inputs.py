@@ -29,9 +29,9 @@ import torch
 class Workload:
     name: str
     seed: int
-    kind: str                    # "prefill" or "decode"
+    kind: str                    # "prefill", "decode" or "verify"
     B: int                       # batch (prefill without cu_seqlens) or sequences (decode)
-    T: int                       # tokens per sequence (prefill) / decode steps
+    T: int                       # tokens per sequence (prefill) / decode steps / drafts (verify)
     HK: int
     HV: int
     dk: int
@@ -56,6 +56,10 @@ WORKLOADS = {
                          h0_std=0.02, varlen=(8, 1024, 32768)),
     "decode_256x64": Workload("decode_256x64", 4, "decode", 256, 64, 16, 32, 128, 128, 1,
                               torch.bfloat16, h0_std=0.02),
+    # speculative decoding: 4 draft tokens per sequence checked at once (the
+    # model factory's multi-token-prediction head proposes 4), decode shapes
+    "verify_256x4": Workload("verify_256x4", 5, "verify", 256, 4, 16, 32, 128, 128, 1,
+                             torch.bfloat16, h0_std=0.02),
 }
 
 
@@ -123,6 +127,17 @@ def make_decode(N: int, steps: int, HK: int, HV: int, dk: int, dv: int, dtype=to
     return dict(q=q, k=k, v=v, g=g, beta=beta, state=state)
 
 
+def make_verify(N: int, K: int, HK: int, HV: int, dk: int, dv: int, dtype=torch.bfloat16,
+                seed: int = 0, h0_std: float = 0.02):
+    """K draft tokens for each of N sequences plus a start state (the draw of
+    ``make_decode`` laid out sequence-major): q,k [N,K,HK,dk], v [N,K,HV,dv],
+    g,beta [N,K,HV] and state [N,HV,dv,dk] fp32, all CPU tensors."""
+    x = make_decode(N, K, HK, HV, dk, dv, dtype, seed, h0_std)
+    out = {n: x[n].transpose(0, 1).contiguous() for n in ("q", "k", "v", "g", "beta")}
+    out["state"] = x["state"]
+    return out
+
+
 def workload_inputs(name: str, steps: int | None = None, seed_offset: int = 0,
                     tokens: int | None = None):
     """Inputs for one named workload (see ``WORKLOADS``).  ``seed_offset`` gives
@@ -134,6 +149,8 @@ def workload_inputs(name: str, steps: int | None = None, seed_offset: int = 0,
         w = replace(w, seed=w.seed + 7919 * seed_offset)
     if w.kind == "decode":
         return make_decode(w.B, steps or w.T, w.HK, w.HV, w.dk, w.dv, w.dtype, w.seed, w.h0_std)
+    if w.kind == "verify":
+        return make_verify(w.B, w.T, w.HK, w.HV, w.dk, w.dv, w.dtype, w.seed, w.h0_std)
     if w.varlen:
         gen = torch.Generator().manual_seed(w.seed)
         n, lo, hi = w.varlen

@@ -110,3 +110,60 @@ def test_workspace_size_rejects_bad_shapes(lib):
 
 def test_read_status_without_workspace(lib):
     assert lib.gdn_read_status(None, 0, None) == gdn.GDN_OK
+
+
+def verify_call(lib, **kw):
+    a = dict(q=fake(0x1000), k=fake(0x2000), v=fake(0x3000), g=fake(0x4000), beta=fake(0x5000),
+             state=fake(0x6000), N=2, K=4, HK=1, HV=2, dk=128, dv=128, scale=1.0,
+             dtype=gdn.GDN_BF16, o=fake(0x7000), states=fake(0x8000), u=fake(0x9000))
+    a.update(kw)
+    return lib.gdn_recurrent_verify(a["q"], a["k"], a["v"], a["g"], a["beta"], a["state"],
+                                    a["N"], a["K"], a["HK"], a["HV"], a["dk"], a["dv"],
+                                    a["scale"], a["dtype"], a["o"], a["states"], a["u"], None)
+
+
+def test_verify_validation(lib):
+    assert verify_call(lib, o=None) == gdn.GDN_ERR_INVALID_ARG
+    assert verify_call(lib, K=0) == gdn.GDN_ERR_INVALID_ARG
+    assert verify_call(lib, HK=3) == gdn.GDN_ERR_INVALID_ARG
+    assert verify_call(lib, K=17) == gdn.GDN_ERR_UNSUPPORTED   # above the draft limit
+    assert verify_call(lib, dk=100) == gdn.GDN_ERR_UNSUPPORTED
+    assert verify_call(lib, states=fake(0x8008)) == gdn.GDN_ERR_ALIGNMENT
+    assert verify_call(lib, u=fake(0x9002)) == gdn.GDN_ERR_ALIGNMENT
+    assert verify_call(lib, N=0) == gdn.GDN_OK
+
+
+def test_commit_validation(lib):
+    def call(**kw):
+        a = dict(states=fake(0x1000), acc=fake(0x2000), state=fake(0x3000), N=2, K=4, HV=2,
+                 dk=128, dv=128)
+        a.update(kw)
+        return lib.gdn_state_commit(a["states"], a["acc"], a["state"], a["N"], a["K"], a["HV"],
+                                    a["dk"], a["dv"], None)
+    assert call(acc=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(K=0) == gdn.GDN_ERR_INVALID_ARG
+    assert call(dk=3, dv=3) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(acc=fake(0x2002)) == gdn.GDN_ERR_ALIGNMENT
+    assert call(N=0) == gdn.GDN_OK
+
+
+def test_verify_and_commit_accept_empty_batch_with_null_buffers(lib):
+    assert verify_call(lib, N=0, q=None, states=None) == gdn.GDN_OK
+    assert lib.gdn_state_commit(None, None, None, 0, 4, 2, 128, 128, None) == gdn.GDN_OK
+
+
+def test_commit_deltas_validation(lib):
+    def call(**kw):
+        a = dict(k=fake(0x1000), g=fake(0x2000), u=fake(0x3000), acc=fake(0x4000),
+                 state=fake(0x5000), N=2, K=4, HK=1, HV=2, dk=128, dv=128, dtype=gdn.GDN_BF16)
+        a.update(kw)
+        return lib.gdn_state_commit_deltas(a["k"], a["g"], a["u"], a["acc"], a["state"], a["N"],
+                                           a["K"], a["HK"], a["HV"], a["dk"], a["dv"], a["dtype"],
+                                           None)
+    assert call(u=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(HK=3) == gdn.GDN_ERR_INVALID_ARG
+    assert call(dtype=9) == gdn.GDN_ERR_INVALID_ARG
+    assert call(K=17) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(dv=300) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(state=fake(0x5004)) == gdn.GDN_ERR_ALIGNMENT
+    assert call(N=0, k=None, u=None) == gdn.GDN_OK

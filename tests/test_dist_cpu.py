@@ -70,3 +70,9 @@ def test_single_process_helpers():
     assert bench.aggregate_throughput(1, 65536, 10, 1000.0) == pytest.approx(655360.0)
     assert bench.prefill_flops_per_token(16, 32, 128, 64) == 5242880
     assert bench.decode_bytes_per_step(256, 16, 32, 128, 128) == 1080098816
+    # verify_256x4 with every draft kept: hand-counted bytes of one round
+    acc = [4] * 256
+    assert bench.verify_bytes(256, 4, 16, 32, 128, 128, acc, "deltas") == (579076096, 1094845440)
+    assert bench.verify_bytes(256, 4, 16, 32, 128, 128, acc, "states") == (2709782528, 1073742848)
+    # nothing kept: the commit touches no state
+    assert bench.verify_bytes(256, 4, 16, 32, 128, 128, [0] * 256, "deltas")[1] == 1024

@@ -1,0 +1,156 @@
+"""Multi-token verify (speculative drafts) and the roll-back commit, through the
+C ABI, against the float64 oracle's ``verify`` and ``commit``."""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_recurrence_rule_b200 import (GDNError, gdn_recurrent_step,
+                                                   gdn_recurrent_verify, gdn_state_commit,
+                                                   gdn_state_commit_deltas)
+from linear_attention_recurrence_rule_b200.inputs import make_verify
+from oracle import gdn_oracle as O
+from parity_util import assert_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+# "both" runs the kernel that carries the state through the drafts (and writes
+# it after each); "deltas" the one that keeps S_0 and unrolls the drafts.
+@pytest.mark.parametrize("rollback", ["both", "deltas"])
+@pytest.mark.parametrize("N,K,HK,HV,dk,dv,dtype", [
+    (5, 1, 2, 4, 64, 48, torch.float32),      # one draft: the decode step
+    (7, 2, 1, 2, 32, 200, torch.bfloat16),    # dv not a multiple of a band
+    (33, 4, 2, 4, 128, 128, torch.bfloat16),  # the model's head shape
+    (6, 5, 1, 2, 128, 128, torch.float32),    # first count past the 4-draft bound
+    (3, 8, 1, 2, 128, 256, torch.float32),    # two bands per state
+    (4, 11, 2, 2, 32, 72, torch.bfloat16),    # a count between the 8 and 16 bounds
+    (4, 16, 2, 4, 64, 64, torch.float32),     # the largest draft count
+])
+def test_verify_matches_oracle(N, K, HK, HV, dk, dv, dtype, rollback):
+    x = make_verify(N, K, HK, HV, dk, dv, dtype, seed=41 + K, h0_std=0.3)
+    d = to_dev(x)
+    state0 = d["state"].clone()
+    o, states, u = gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                                        scale=0.7, rollback=rollback)
+    torch.cuda.synchronize()
+    o_ref, states_ref = O.verify(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state"], scale=0.7)
+    assert torch.equal(d["state"], state0), "verify must not modify the input state"
+    assert_close(o, o_ref, dtype, "o")
+    if rollback == "both":
+        for t in range(K):
+            assert_close(states[:, t], states_ref[:, t], dtype, f"state after draft {t}")
+    else:
+        assert states is None
+    # u_t is the rank-1 update of draft t: S_t - alpha_t S_{t-1} (oracle states)
+    prev = np.concatenate([x["state"].double().numpy()[:, None], states_ref[:, :-1]], 1)
+    alpha = np.exp(x["g"].double().numpy())[..., None, None]
+    k_rep = x["k"].double().numpy().repeat(HV // HK, axis=2)       # [N,K,HV,dk]
+    delta = states_ref - alpha * prev                                 # = u_t k_t^T
+    u_ref = np.einsum("nthvd,nthd->nthv", delta, k_rep) / np.einsum("nthd,nthd->nth", k_rep,
+                                                                     k_rep)[..., None]
+    assert_close(u, u_ref, dtype, "u")
+
+
+def test_verify_one_draft_equals_decode_step():
+    x = make_verify(9, 1, 2, 4, 128, 128, torch.bfloat16, seed=5, h0_std=0.2)
+    d = to_dev(x)
+    o, states, _ = gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"])
+    S = d["state"].clone()
+    o1 = gdn_recurrent_step(d["q"][:, 0].contiguous(), d["k"][:, 0].contiguous(),
+                            d["v"][:, 0].contiguous(), d["g"][:, 0].contiguous(),
+                            d["beta"][:, 0].contiguous(), S)
+    torch.cuda.synchronize()
+    # the same recurrence with the dot products summed in another order: the
+    # states agree to fp32 rounding, the bf16 outputs to one rounding step
+    assert float((states[:, 0] - S).abs().max()) <= 1e-5
+    diff = (o[:, 0].float() - o1.float()).abs()
+    assert bool((diff <= 2.0 ** -7 * o1.float().abs() + 1e-6).all())
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_commit_keeps_accepted_prefix(dtype):
+    N, K = 11, 6
+    x = make_verify(N, K, 1, 2, 64, 96, dtype, seed=8, h0_std=0.3)
+    d = to_dev(x)
+    o, states, u = gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                                        rollback="both")
+    gen = torch.Generator().manual_seed(3)
+    accepted = torch.randint(0, K + 1, (N,), generator=gen, dtype=torch.int32)
+    accepted[0], accepted[1], accepted[2] = 0, K, 1       # none, all, one
+    accepted[3] = K + 2                                   # out of range: treated as none
+    S = d["state"].clone()
+    gdn_state_commit(states, accepted.cuda(), S)
+    torch.cuda.synchronize()
+    # the commit is a copy: bit-exact against the verify output it selects
+    expect = O.commit(states.cpu().double().numpy(),
+                      np.where(accepted.numpy() <= K, accepted.numpy(), 0), d["state"].cpu())
+    assert np.array_equal(S.cpu().double().numpy(), expect)
+    # and the kept state is the oracle's state after the accepted drafts
+    _, states_ref = O.verify(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state"])
+    acc = np.where(accepted.numpy() <= K, accepted.numpy(), 0)
+    assert_close(S, O.commit(states_ref, acc, x["state"]), dtype, "committed state")
+    # the deltas form reaches the same state from u, k and g in place
+    S2 = d["state"].clone()
+    gdn_state_commit_deltas(d["k"], d["g"], u, accepted.cuda(), S2)
+    torch.cuda.synchronize()
+    assert_close(S2, O.commit(states_ref, acc, x["state"]), dtype, "committed state (deltas)")
+    untouched = np.flatnonzero(acc == 0)
+    assert torch.equal(S2[untouched], d["state"][untouched])
+
+
+@pytest.mark.parametrize("N,K,HK,HV,dk,dv,dtype", [
+    (8, 4, 2, 4, 128, 128, torch.bfloat16),
+    (5, 16, 1, 2, 32, 200, torch.float32),    # the largest draft count, ragged band
+    (3, 3, 1, 1, 64, 256, torch.float32),
+])
+def test_commit_deltas_matches_oracle(N, K, HK, HV, dk, dv, dtype):
+    x = make_verify(N, K, HK, HV, dk, dv, dtype, seed=17 + K, h0_std=0.5)
+    d = to_dev(x)
+    _, states_none, u = gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                             d["state"], rollback="deltas")
+    assert states_none is None
+    accepted = (torch.arange(N, dtype=torch.int32) % (K + 1))
+    S = d["state"].clone()
+    gdn_state_commit_deltas(d["k"], d["g"], u, accepted.cuda(), S)
+    torch.cuda.synchronize()
+    _, states_ref = O.verify(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state"])
+    assert_close(S, O.commit(states_ref, accepted.numpy(), x["state"]), dtype, "state")
+
+
+def test_verify_then_commit_all_equals_decode_steps():
+    N, K = 6, 4
+    x = make_verify(N, K, 2, 4, 128, 128, torch.float32, seed=13, h0_std=0.2)
+    d = to_dev(x)
+    o, states, u = gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                                        rollback="both")
+    S = d["state"].clone()
+    gdn_state_commit(states, torch.full((N,), K, dtype=torch.int32, device="cuda"), S)
+    S2 = d["state"].clone()
+    outs = [gdn_recurrent_step(*(d[n][:, t].contiguous() for n in ("q", "k", "v", "g", "beta")),
+                               S2) for t in range(K)]
+    torch.cuda.synchronize()
+    assert_close(o, torch.stack(outs, 1).cpu().double().numpy(), torch.float32, "o")
+    assert_close(S, S2.cpu().double().numpy(), torch.float32, "state")
+    S3 = d["state"].clone()
+    gdn_state_commit_deltas(d["k"], d["g"], u, torch.full((N,), K, dtype=torch.int32,
+                                                          device="cuda"), S3)
+    torch.cuda.synchronize()
+    assert_close(S3, S2.cpu().double().numpy(), torch.float32, "state (deltas)")
+
+
+def test_verify_empty_and_errors():
+    x = make_verify(2, 3, 1, 2, 32, 32, torch.float32, seed=1)
+    d = to_dev(x)
+    e = {n: d[n][:0] for n in ("q", "k", "v", "g", "beta", "state")}
+    o, states, u = gdn_recurrent_verify(e["q"], e["k"], e["v"], e["g"], e["beta"], e["state"],
+                                        rollback="both")
+    assert o.numel() == 0 and states.numel() == 0 and u.numel() == 0
+    gdn_state_commit_deltas(e["k"], e["g"], u, torch.zeros(0, dtype=torch.int32, device="cuda"),
+                            e["state"])
+    with pytest.raises(ValueError):
+        gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"][:, :2].contiguous(), d["beta"],
+                             d["state"])
+    big = make_verify(1, 17, 1, 2, 32, 32, torch.float32, seed=2)
+    b = to_dev(big)
+    with pytest.raises(GDNError):
+        gdn_recurrent_verify(b["q"], b["k"], b["v"], b["g"], b["beta"], b["state"])

@@ -48,3 +48,14 @@ def test_decode_inputs():
     assert x["q"].shape == (4, 3, 2, 16) and x["v"].shape == (4, 3, 4, 8)
     assert x["state"].shape == (3, 4, 8, 16) and x["state"].dtype == torch.float32
     assert math.isclose(float(x["state"].std()), 0.02, rel_tol=0.2)
+
+
+def test_verify_inputs_are_decode_draws_sequence_major():
+    from linear_attention_recurrence_rule_b200.inputs import make_verify
+    x = make_decode(3, 4, 2, 4, 16, 8, torch.bfloat16, seed=1)
+    y = make_verify(3, 4, 2, 4, 16, 8, torch.bfloat16, seed=1)
+    for n in ("q", "k", "v", "g", "beta"):
+        assert torch.equal(y[n], x[n].transpose(0, 1)) and y[n].is_contiguous()
+    assert torch.equal(y["state"], x["state"])
+    w = WORKLOADS["verify_256x4"]
+    assert (w.kind, w.B, w.T, w.HK, w.HV, w.dk) == ("verify", 256, 4, 16, 32, 128)
