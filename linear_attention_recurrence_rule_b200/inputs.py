@@ -138,6 +138,25 @@ def make_verify(N: int, K: int, HK: int, HV: int, dk: int, dv: int, dtype=torch.
     return out
 
 
+def raw_projections(x: dict, seed: int, norm_range=(0.25, 4.0), forget_logit=(3.0, 1.0)):
+    """Turn a generated problem into the raw projections a layer produces before
+    its prologue: every q, k row multiplied by its own positive factor
+    ~U(norm_range) (kept in the problem's dtype), and the gate arrays replaced
+    by logits: ``g`` <- forget logits ~N(forget_logit) (alpha = sigmoid near
+    0.95 at the default), ``beta`` <- write logits ~N(0, 1).  Only random draws
+    and scalings; CPU tensors in, CPU tensors out."""
+    gen = torch.Generator().manual_seed(seed)
+    out = dict(x)
+    for n in ("q", "k"):
+        t = x[n]
+        f = norm_range[0] + (norm_range[1] - norm_range[0]) * torch.rand(
+            t.shape[:-1] + (1,), generator=gen)
+        out[n] = (t.float() * f).to(t.dtype)
+    out["g"] = (forget_logit[0] + forget_logit[1] * torch.randn(x["g"].shape, generator=gen)).float()
+    out["beta"] = torch.randn(x["beta"].shape, generator=gen).float()
+    return out
+
+
 def workload_inputs(name: str, steps: int | None = None, seed_offset: int = 0,
                     tokens: int | None = None):
     """Inputs for one named workload (see ``WORKLOADS``).  ``seed_offset`` gives

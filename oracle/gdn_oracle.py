@@ -15,7 +15,10 @@ file's header for the rule it follows and the pages it cites:
 * 32 value heads reading 16 query/key heads at head dim 128 (model card
   "Qwen3-Next-80B-A3B-Instruct", section "Model Overview"),
 * read-out after the update, state rows indexed by the value dimension
-  ("The Evolving Transformer / Qwen3-Next", section 01 GatedDeltaNet).
+  ("The Evolving Transformer / Qwen3-Next", section 01 GatedDeltaNet),
+* the prologue that turns a layer's raw projections into the rule's inputs
+  (``prologue``, plain numpy: L2-normalised keys and sigmoid gates, same
+  section of the same page).
 
 Every function here has its result pinned by ``tests/test_oracle_pins.py``
 against values the pages print, closed forms, invariants and the agreement of
@@ -196,3 +199,37 @@ def commit(states, accepted, state):
         if a > 0:
             S[n] = states[n, a - 1]
     return S
+
+
+# flags of the input prologue (same values as the C header's GDN_PROLOGUE_*)
+PROLOGUE_NORM_Q = 1
+PROLOGUE_NORM_K = 2
+PROLOGUE_GATE_LOGITS = 4
+NORM_EPS = 1e-12
+
+
+def prologue(q, k, g, beta, flags):
+    """The steps just before the recurrence, in float64 ("The Evolving
+    Transformer / Qwen3-Next", section 01 GatedDeltaNet: keys are L2-normalised
+    along the head dimension; the write strength is a sigmoid of its logit and
+    the forget gate a sigmoid of its own logit).  Reading: one forget logit per
+    token and value head (the hot path's scalar decay per head), and q is
+    normalised like k when asked (the model's "L2-normalised q/k").
+
+    flags & PROLOGUE_NORM_Q: q <- q / max(|q|, 1e-12) over the last axis
+    flags & PROLOGUE_NORM_K: k <- k / max(|k|, 1e-12)
+    flags & PROLOGUE_GATE_LOGITS: ``g`` holds the forget logits a and ``beta``
+        the write logits b; returns g = log sigmoid(a) (so alpha = exp(g) =
+        sigmoid(a)) and beta = sigmoid(b).
+    Returns float64 (q, k, g, beta); inputs of other shapes pass through.
+    """
+    q, k, g, beta = (_f64(x) for x in (q, k, g, beta))
+    if flags & PROLOGUE_NORM_Q:
+        q = q / np.maximum(np.sqrt(np.sum(q * q, axis=-1, keepdims=True)), NORM_EPS)
+    if flags & PROLOGUE_NORM_K:
+        k = k / np.maximum(np.sqrt(np.sum(k * k, axis=-1, keepdims=True)), NORM_EPS)
+    if flags & PROLOGUE_GATE_LOGITS:
+        # log sigmoid(x) = -log(1 + e^-x), evaluated without overflow
+        g = -np.logaddexp(0.0, -g)
+        beta = np.exp(-np.logaddexp(0.0, -beta))
+    return q, k, g, beta

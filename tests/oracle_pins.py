@@ -350,4 +350,69 @@ def pin_commit_rolls_back_to_accepted_prefix(lib=None):
         assert np.allclose(S[n], hp[0], atol=1e-12)
 
 
+# ----------------------------------------------------------------------------
+# The input prologue (L2-normalised keys and queries, sigmoid gates)
+# ----------------------------------------------------------------------------
+def pin_prologue_normalises_rows(lib=None):
+    """Normalised rows have unit length and point along the raw row; each flag
+    touches only its own tensor; a zero row stays zero (no division by 0)."""
+    rng = np.random.default_rng(21)
+    q = rng.standard_normal((2, 5, 3, 7)) * rng.uniform(0.1, 9.0, (2, 5, 3, 1))
+    k = rng.standard_normal((2, 5, 3, 7)) * rng.uniform(0.1, 9.0, (2, 5, 3, 1))
+    k[0, 1, 2] = 0.0
+    g, b = rng.standard_normal((2, 5, 6)), rng.standard_normal((2, 5, 6))
+    qn, kn, g2, b2 = O.prologue(q, k, g, b, O.PROLOGUE_NORM_Q | O.PROLOGUE_NORM_K)
+    assert np.array_equal(g2, g) and np.array_equal(b2, b)
+    assert np.allclose(np.linalg.norm(qn, axis=-1), 1.0, atol=1e-14)
+    nk = np.linalg.norm(kn, axis=-1)
+    assert np.all(kn[0, 1, 2] == 0.0)
+    nk[0, 1, 2] = 1.0
+    assert np.allclose(nk, 1.0, atol=1e-14)
+    # parallel to the raw rows: <x_hat, x> = |x|
+    assert np.allclose(np.sum(qn * q, -1), np.linalg.norm(q, axis=-1), rtol=1e-13)
+    qn2, kn2, _, _ = O.prologue(q, k, g, b, O.PROLOGUE_NORM_K)
+    assert np.array_equal(qn2, q) and np.array_equal(kn2, kn)
+    qn3, kn3, _, _ = O.prologue(q, k, g, b, O.PROLOGUE_NORM_Q)
+    assert np.array_equal(kn3, k) and np.array_equal(qn3, qn)
+
+
+def pin_prologue_gates(lib=None):
+    """beta = sigmoid(b): 1/2 at 0 and beta(b) + beta(-b) = 1; alpha = exp(g) =
+    sigmoid(a): alpha / (1 - alpha) = e^a; the saturated ends stay finite
+    (g -> 0 for a >> 0, g -> a for a << 0)."""
+    a = np.array([-60.0, -3.0, -0.5, 0.0, 0.7, 4.0, 60.0])
+    b = np.array([0.0, 1.0, -1.0, 2.5, -2.5, 30.0, -30.0])
+    _, _, g, beta = O.prologue(np.zeros(2), np.zeros(2), a, b, O.PROLOGUE_GATE_LOGITS)
+    assert beta[0] == 0.5
+    assert abs(beta[1] + beta[2] - 1.0) < 1e-15 and abs(beta[3] + beta[4] - 1.0) < 1e-15
+    assert np.all((beta > 0) & (beta < 1)) and beta[5] > 1 - 1e-12 and beta[6] < 1e-12
+    alpha = np.exp(g)
+    mid = slice(1, 6)
+    assert np.allclose(np.log(alpha[mid] / (1.0 - alpha[mid])), a[mid], atol=1e-12)
+    assert np.all(g <= 0.0) and np.all(np.isfinite(g))
+    assert abs(g[-1]) < 1e-25 and abs(g[0] - a[0]) < 1e-20
+    assert g[3] == -math.log(2.0)
+
+
+def pin_prologue_then_rule_is_scale_free(lib=None):
+    """With both norms on, scaling a token's raw q or k by any positive factor
+    leaves the outputs and state unchanged; with them off, a scaled key changes
+    the result (so the flag really feeds the rule)."""
+    rng = np.random.default_rng(22)
+    q, k, v, _, _ = _rand_problem(rng, 9, 1, 2, 5, 4, unit=False)
+    a = rng.normal(2.0, 1.0, (1, 9, 2))
+    b = rng.standard_normal((1, 9, 2))
+    flags = O.PROLOGUE_NORM_Q | O.PROLOGUE_NORM_K | O.PROLOGUE_GATE_LOGITS
+    s_q = rng.uniform(0.2, 5.0, (1, 9, 1, 1))
+    s_k = rng.uniform(0.2, 5.0, (1, 9, 1, 1))
+    o1, h1 = O.prefill(*O.prologue(q, k, a, b, flags)[:2], v, *O.prologue(q, k, a, b, flags)[2:],
+                       lib=lib)
+    qq, kk, gg, bb = O.prologue(q * s_q, k * s_k, a, b, flags)
+    o2, h2 = O.prefill(qq, kk, v, gg, bb, lib=lib)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(h1, h2, atol=1e-12)
+    q3, k3, g3, b3 = O.prologue(q, k * s_k, a, b, O.PROLOGUE_NORM_Q | O.PROLOGUE_GATE_LOGITS)
+    o3, _ = O.prefill(q3, k3, v, g3, b3, lib=lib)
+    assert not np.allclose(o1, o3, atol=1e-6)
+
+
 ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

@@ -59,3 +59,15 @@ def test_verify_inputs_are_decode_draws_sequence_major():
     assert torch.equal(y["state"], x["state"])
     w = WORKLOADS["verify_256x4"]
     assert (w.kind, w.B, w.T, w.HK, w.HV, w.dk) == ("verify", 256, 4, 16, 32, 128)
+
+
+def test_raw_projections_scale_rows_and_draw_logits():
+    from linear_attention_recurrence_rule_b200.inputs import raw_projections
+    x = make_decode(3, 4, 2, 4, 16, 8, torch.float32, seed=1)
+    y = raw_projections(x, seed=5)
+    ratio = y["k"].norm(dim=-1) / x["k"].norm(dim=-1)
+    assert bool(((ratio >= 0.25) & (ratio <= 4.0)).all()) and float(ratio.std()) > 0.1
+    cos = (y["q"] * x["q"]).sum(-1) / (y["q"].norm(dim=-1) * x["q"].norm(dim=-1))
+    assert torch.allclose(cos, torch.ones_like(cos), atol=1e-6)
+    assert y["g"].shape == x["g"].shape and float(y["g"].mean()) > 2.0
+    assert torch.equal(y["v"], x["v"]) and torch.equal(y["state"], x["state"])

@@ -63,3 +63,57 @@ def test_pins_catch_mutant(tmp_path, name, old, new):
         except ValueError:
             caught.append(pin.__name__)
     assert caught, f"no pin detects the planted mistake {name}"
+
+
+# Mistakes planted in the prologue (plain numpy): each replaces oracle.prologue
+# for the duration of one test and must fail at least one prologue pin.
+def _prologue_mutant(kind):
+    import numpy as np
+    real = O.prologue
+
+    def mutant(q, k, g, beta, flags):
+        q, k, g, beta = (O._f64(x) for x in (q, k, g, beta))
+        if kind == "no_eps" and flags & O.PROLOGUE_NORM_K:
+            k = k / np.sqrt(np.sum(k * k, axis=-1, keepdims=True))
+            return real(q, k, g, beta, flags & ~O.PROLOGUE_NORM_K)
+        if kind == "wrong_axis" and flags & O.PROLOGUE_NORM_Q:
+            q = q / np.maximum(np.sqrt(np.sum(q * q, axis=0, keepdims=True)), 1e-12)
+            return real(q, k, g, beta, flags & ~O.PROLOGUE_NORM_Q)
+        if kind == "flags_swapped":
+            f = flags & ~3
+            f |= (O.PROLOGUE_NORM_K if flags & O.PROLOGUE_NORM_Q else 0)
+            f |= (O.PROLOGUE_NORM_Q if flags & O.PROLOGUE_NORM_K else 0)
+            return real(q, k, g, beta, f)
+        if kind == "forget_gate_sign" and flags & O.PROLOGUE_GATE_LOGITS:
+            qq, kk, _, bb = real(q, k, g, beta, flags)
+            return qq, kk, -np.logaddexp(0.0, g), bb
+        if kind == "write_gate_sign" and flags & O.PROLOGUE_GATE_LOGITS:
+            qq, kk, gg, _ = real(q, k, g, beta, flags)
+            return qq, kk, gg, np.exp(-np.logaddexp(0.0, beta))
+        if kind == "gate_as_alpha" and flags & O.PROLOGUE_GATE_LOGITS:
+            qq, kk, _, bb = real(q, k, g, beta, flags)   # alpha itself returned as g
+            return qq, kk, np.exp(-np.logaddexp(0.0, -g)), bb
+        if kind == "norms_ignored":
+            return real(q, k, g, beta, flags & O.PROLOGUE_GATE_LOGITS)
+        return real(q, k, g, beta, flags)
+    return mutant
+
+
+PROLOGUE_MUTANTS = ["no_eps", "wrong_axis", "flags_swapped", "forget_gate_sign",
+                    "write_gate_sign", "gate_as_alpha", "norms_ignored"]
+
+
+@pytest.mark.parametrize("kind", PROLOGUE_MUTANTS)
+def test_prologue_pins_catch_mutant(monkeypatch, kind):
+    import numpy as np
+    monkeypatch.setattr(O, "prologue", _prologue_mutant(kind))
+    caught = []
+    with np.errstate(all="ignore"):
+        for pin in ALL_PINS:
+            if "prologue" not in pin.__name__:
+                continue
+            try:
+                pin()
+            except (AssertionError, ValueError):
+                caught.append(pin.__name__)
+    assert caught, f"no pin detects the planted prologue mistake {kind}"
