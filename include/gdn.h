@@ -85,6 +85,27 @@ GDN_API size_t gdn_chunk_prefill_workspace_size(int N, int64_t T, int HK, int HV
                                         int chunk, gdn_dtype dtype, int varlen);
 
 /*
+ * Input prologue flags (bitwise OR; 0 = the inputs are already prepared).
+ * They fuse the layer steps just before the rule into the kernels ("The
+ * Evolving Transformer / Qwen3-Next", section 01 GatedDeltaNet: keys are
+ * L2-normalised, the write strength and the forget gate are sigmoids of their
+ * logits; queries are normalised like keys in the model):
+ *   GDN_PROLOGUE_NORM_Q       each q row (per QK head, over dk) is replaced by
+ *                             q / max(|q|, 1e-12), computed in fp32 from the
+ *                             stored values
+ *   GDN_PROLOGUE_NORM_K       the same for k
+ *   GDN_PROLOGUE_GATE_LOGITS  `g` holds forget logits a and `beta` write logits
+ *                             b: alpha = sigmoid(a) (g = log sigmoid(a)) and
+ *                             beta = sigmoid(b)
+ * No normalised copy is written: the norms are folded into the scalings the
+ * kernels already apply.
+ */
+#define GDN_PROLOGUE_NORM_Q 1u
+#define GDN_PROLOGUE_NORM_K 2u
+#define GDN_PROLOGUE_GATE_LOGITS 4u
+#define GDN_PROLOGUE_ALL 7u
+
+/*
  * 1 when gdn_chunk_prefill runs this (head dims, chunk, dtype) combination on
  * the tcgen05 tensor-core path, 0 when it runs on the CUDA-core path, -1 when
  * the combination is unsupported.  Pure host query.
@@ -125,6 +146,20 @@ GDN_API gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v
                              int N, int64_t T, int HK, int HV, int dk, int dv, int chunk,
                              float scale, gdn_dtype dtype, void *o, float *hT,
                              void *workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * gdn_chunk_prefill with the input prologue fused (`prologue`: GDN_PROLOGUE_*
+ * flags; 0 is exactly gdn_chunk_prefill).  With GDN_PROLOGUE_GATE_LOGITS, g
+ * and beta hold the logits (any real values).  Unknown flag bits return
+ * GDN_ERR_INVALID_ARG.
+ */
+GDN_API gdn_status gdn_chunk_prefill_ex(const void *q, const void *k, const void *v,
+                                        const float *g, const float *beta, const float *h0,
+                                        const int32_t *cu_seqlens, int N, int64_t T, int HK,
+                                        int HV, int dk, int dv, int chunk, float scale,
+                                        gdn_dtype dtype, void *o, float *hT, void *workspace,
+                                        size_t workspace_bytes, unsigned prologue,
+                                        gdn_stream_t stream);
 
 /*
  * gdn_chunk_prefill without a caller-provided workspace.  (The source pages
@@ -228,6 +263,17 @@ GDN_API gdn_status gdn_recurrent_step(const void *q, const void *k, const void *
                               int dv, float scale, gdn_dtype dtype, void *o,
                               gdn_stream_t stream);
 
+/*
+ * gdn_recurrent_step with the input prologue fused (`prologue`: GDN_PROLOGUE_*
+ * flags; 0 is exactly gdn_recurrent_step).  Unknown flag bits return
+ * GDN_ERR_INVALID_ARG.
+ */
+GDN_API gdn_status gdn_recurrent_step_ex(const void *q, const void *k, const void *v,
+                                         const float *g, const float *beta, float *state, int N,
+                                         int HK, int HV, int dk, int dv, float scale,
+                                         gdn_dtype dtype, void *o, unsigned prologue,
+                                         gdn_stream_t stream);
+
 /* Largest number of draft tokens gdn_recurrent_verify takes per sequence. */
 #define GDN_VERIFY_MAX_DRAFTS 16
 
@@ -249,6 +295,7 @@ GDN_API gdn_status gdn_recurrent_step(const void *q, const void *k, const void *
  *   q, k   [N][K][HK][dk] dtype      v, o [N][K][HV][dv] dtype
  *   g, beta [N][K][HV] fp32          state [N][HV][dv][dk] fp32 (read)
  *   states_out [N][K][HV][dv][dk] fp32   u_out [N][K][HV][dv] fp32
+ * prologue: GDN_PROLOGUE_* flags applied to every draft (0 = prepared inputs).
  * Supported: as gdn_recurrent_step, and 1 <= K <= GDN_VERIFY_MAX_DRAFTS.
  * Alignment: q, k, v, o, state, states_out 16-byte aligned, u_out 4-byte.
  * No output may overlap an input.  K > GDN_VERIFY_MAX_DRAFTS returns
@@ -259,7 +306,7 @@ GDN_API gdn_status gdn_recurrent_verify(const void *q, const void *k, const void
                                         const float *g, const float *beta, const float *state,
                                         int N, int K, int HK, int HV, int dk, int dv, float scale,
                                         gdn_dtype dtype, void *o, float *states_out, float *u_out,
-                                        gdn_stream_t stream);
+                                        unsigned prologue, gdn_stream_t stream);
 
 /*
  * Keeps the accepted drafts after gdn_recurrent_verify (states_out form): for
@@ -281,7 +328,8 @@ GDN_API gdn_status gdn_state_commit(const float *states, const int32_t *accepted
  *   S <- (prod_{t<a} alpha_t) S + sum_{t<a} (prod_{t<s<a} alpha_s) u_t k_t^T,
  * alpha_t = exp(g_t): the recurrence unrolled over the kept tokens.  Each
  * state element is read and written once.  a == 0 or out of range leaves the
- * state unchanged.  k and g are the verify call's inputs, u its u_out.
+ * state unchanged.  k and g are the verify call's inputs, u its u_out, and
+ * `prologue` the verify call's flags (its NORM_K and GATE_LOGITS bits apply).
  * Layouts: k [N][K][HK][dk] dtype, g [N][K][HV] fp32, u [N][K][HV][dv] fp32,
  * accepted [N] int32 (device), state [N][HV][dv][dk] fp32.
  * Supported: as gdn_recurrent_verify.  Alignment: k, state 16-byte aligned,
@@ -290,7 +338,7 @@ GDN_API gdn_status gdn_state_commit(const float *states, const int32_t *accepted
 GDN_API gdn_status gdn_state_commit_deltas(const void *k, const float *g, const float *u,
                                            const int32_t *accepted, float *state, int N, int K,
                                            int HK, int HV, int dk, int dv, gdn_dtype dtype,
-                                           gdn_stream_t stream);
+                                           unsigned prologue, gdn_stream_t stream);
 
 /*
  * Reads the device status word a prefill call left in its workspace (HOST

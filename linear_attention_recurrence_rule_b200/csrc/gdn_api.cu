@@ -125,6 +125,18 @@ gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v, const 
     return enqueue_prefill(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+gdn_status gdn_chunk_prefill_ex(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const float *h0, const int32_t *cu_seqlens,
+                                int N, int64_t T, int HK, int HV, int dk, int dv, int chunk,
+                                float scale, gdn_dtype dtype, void *o, float *hT, void *workspace,
+                                size_t workspace_bytes, unsigned prologue, gdn_stream_t stream) {
+    if (prologue & ~GDN_PROLOGUE_ALL) return GDN_ERR_INVALID_ARG;
+    gdn::PrefillArgs a{q, k, v, g, beta, h0, cu_seqlens, N, T, HK, HV, dk, dv, chunk,
+                       scale, dtype, o, hT, workspace, workspace_bytes};
+    a.prologue = prologue;
+    return enqueue_prefill(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t gdn_chunk_prefill_host_workspace_size(int N, int64_t T, int HK, int HV, int dk, int dv,
                                              int chunk, gdn_dtype dtype, int64_t segment) {
     if (N <= 0 || T < 0 || HK <= 0 || HV <= 0 || HV % HK || chunk <= 0 || segment < 0) return 0;
@@ -235,6 +247,15 @@ gdn_status gdn_recurrent_step(const void *q, const void *k, const void *v, const
                               const float *beta, float *state, int N, int HK, int HV, int dk,
                               int dv, float scale, gdn_dtype dtype, void *o,
                               gdn_stream_t stream) {
+    return gdn_recurrent_step_ex(q, k, v, g, beta, state, N, HK, HV, dk, dv, scale, dtype, o, 0u,
+                                 stream);
+}
+
+gdn_status gdn_recurrent_step_ex(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, float *state, int N, int HK, int HV, int dk,
+                                 int dv, float scale, gdn_dtype dtype, void *o, unsigned prologue,
+                                 gdn_stream_t stream) {
+    if (prologue & ~GDN_PROLOGUE_ALL) return GDN_ERR_INVALID_ARG;
     if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
     if (N < 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK) return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
@@ -243,7 +264,7 @@ gdn_status gdn_recurrent_step(const void *q, const void *k, const void *v, const
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
         return GDN_ERR_ALIGNMENT;
     if (N == 0) return GDN_OK;
-    gdn::StepArgs a{q, k, v, g, beta, state, N, HK, HV, dk, dv, scale, dtype, o};
+    gdn::StepArgs a{q, k, v, g, beta, state, N, HK, HV, dk, dv, scale, dtype, o, prologue};
     const cudaError_t err = gdn::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -251,7 +272,9 @@ gdn_status gdn_recurrent_step(const void *q, const void *k, const void *v, const
 gdn_status gdn_recurrent_verify(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, const float *state, int N, int K, int HK, int HV,
                                 int dk, int dv, float scale, gdn_dtype dtype, void *o,
-                                float *states_out, float *u_out, gdn_stream_t stream) {
+                                float *states_out, float *u_out, unsigned prologue,
+                                gdn_stream_t stream) {
+    if (prologue & ~GDN_PROLOGUE_ALL) return GDN_ERR_INVALID_ARG;
     if (N < 0 || K <= 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK)
         return GDN_ERR_INVALID_ARG;
     if (N == 0) return GDN_OK;   // empty batch: buffers may be NULL
@@ -263,7 +286,7 @@ gdn_status gdn_recurrent_verify(const void *q, const void *k, const void *v, con
         !aligned16(states_out) || !aligned4(u_out))
         return GDN_ERR_ALIGNMENT;
     gdn::VerifyArgs a{q, k, v, g, beta, state, states_out, u_out, N, K, HK, HV, dk, dv, scale,
-                      dtype, o};
+                      dtype, o, prologue};
     const cudaError_t err = gdn::launch_verify(a, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -283,7 +306,9 @@ gdn_status gdn_state_commit(const float *states, const int32_t *accepted, float 
 
 gdn_status gdn_state_commit_deltas(const void *k, const float *g, const float *u,
                                    const int32_t *accepted, float *state, int N, int K, int HK,
-                                   int HV, int dk, int dv, gdn_dtype dtype, gdn_stream_t stream) {
+                                   int HV, int dk, int dv, gdn_dtype dtype, unsigned prologue,
+                                   gdn_stream_t stream) {
+    if (prologue & ~GDN_PROLOGUE_ALL) return GDN_ERR_INVALID_ARG;
     if (N < 0 || K <= 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK)
         return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
@@ -293,7 +318,7 @@ gdn_status gdn_state_commit_deltas(const void *k, const float *g, const float *u
     if (!gdn::decode_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
     if (!aligned16(k) || !aligned16(state) || !aligned4(u) || !aligned4(accepted))
         return GDN_ERR_ALIGNMENT;
-    gdn::CommitDeltasArgs a{k, g, u, accepted, state, N, K, HK, HV, dk, dv, dtype};
+    gdn::CommitDeltasArgs a{k, g, u, accepted, state, N, K, HK, HV, dk, dv, dtype, prologue};
     const cudaError_t err = gdn::launch_commit_deltas(a, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

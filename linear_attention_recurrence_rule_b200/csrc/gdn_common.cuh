@@ -32,4 +32,17 @@ __device__ __forceinline__ float dot4(float4 a, float4 b) {
     return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
 }
 
+__device__ __forceinline__ float4 scale4(float4 a, float s) {
+    return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
+}
+
+// Input prologue (the layer steps just before the rule): 1 / max(|x|, 1e-12)
+// for an L2-normalised row with squared norm ss, and the sigmoid gates.
+__device__ __forceinline__ float inv_l2norm(float ss) { return 1.f / fmaxf(sqrtf(ss), 1e-12f); }
+__device__ __forceinline__ float gate_sigmoid(float x) { return 1.f / (1.f + expf(-x)); }
+// log sigmoid(x) = min(x, 0) - log(1 + e^-|x|): finite at both ends
+__device__ __forceinline__ float gate_log_sigmoid(float x) {
+    return fminf(x, 0.f) - log1pf(expf(-fabsf(x)));
+}
+
 }  // namespace gdn

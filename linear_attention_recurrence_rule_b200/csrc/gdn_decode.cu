@@ -34,11 +34,11 @@ constexpr int kDecodeNB = 8;
 template <int DK>
 constexpr int band_rows() { return kDecodeWarps * (32 / (DK / 4)) * kDecodeNB; }
 
-template <int DK, typename Tin>
+template <int DK, typename Tin, bool PRO>
 __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ g, const float *__restrict__ beta, float *state,
-              Tin *__restrict__ o, int HK, int HV, int dv, float scale) {
+              Tin *__restrict__ o, int HK, int HV, int dv, float scale, unsigned pro) {
     constexpr int LPR = DK / 4;    // lanes per state row
     constexpr int RPI = 32 / LPR;  // rows per warp instruction
     const int nh = blockIdx.x;     // n * HV + h
@@ -48,13 +48,9 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     const int sub = lane / LPR;
     const int col = (lane % LPR) * 4;
 
-    const float4 kk = load4(k + ((size_t)n * HK + c) * DK + col);
-    const float4 qq = load4(q + ((size_t)n * HK + c) * DK + col);
-    float kq = dot4(kk, qq);
-#pragma unroll
-    for (int off = LPR / 2; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-    const float alpha = expf(g[nh]);
-    const float b = beta[nh];
+    float4 kk = load4(k + ((size_t)n * HK + c) * DK + col);
+    float4 qq = load4(q + ((size_t)n * HK + c) * DK + col);
+    const float graw = g[nh], braw = beta[nh];
     const Tin *vrow = v + (size_t)nh * dv;
     Tin *orow = o + (size_t)nh * dv;
     float *S = state + (size_t)nh * dv * DK;
@@ -62,6 +58,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     constexpr int rows_per_batch = kDecodeWarps * RPI * kDecodeNB;
     {
         const int base = blockIdx.y * rows_per_batch;
+        // the state loads go out first: nothing below them waits on q, k
         float4 s[kDecodeNB];
 #pragma unroll
         for (int j = 0; j < kDecodeNB; ++j) {
@@ -69,6 +66,23 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
             s[j] = row < dv ? __ldcs(reinterpret_cast<const float4 *>(S + (size_t)row * DK + col))
                             : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        if (PRO && (pro & (GDN_PROLOGUE_NORM_Q | GDN_PROLOGUE_NORM_K))) {
+            // the lanes of a row hold the whole q and k: reduce the squared norms there
+            float ssk = dot4(kk, kk), ssq = dot4(qq, qq);
+#pragma unroll
+            for (int off = LPR / 2; off > 0; off >>= 1) {
+                ssk += __shfl_xor_sync(0xffffffffu, ssk, off);
+                ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+            }
+            if (pro & GDN_PROLOGUE_NORM_K) kk = scale4(kk, inv_l2norm(ssk));
+            if (pro & GDN_PROLOGUE_NORM_Q) qq = scale4(qq, inv_l2norm(ssq));
+        }
+        float kq = dot4(kk, qq);
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+        const bool logits = PRO && (pro & GDN_PROLOGUE_GATE_LOGITS) != 0;
+        const float alpha = logits ? gate_sigmoid(graw) : expf(graw);
+        const float b = logits ? gate_sigmoid(braw) : braw;
 #pragma unroll
         for (int j = 0; j < kDecodeNB; ++j) {
             const int row = base + (j * kDecodeWarps + warp) * RPI + sub;
@@ -92,30 +106,25 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     }
 }
 
+template <int DK, typename Tin>
+void launch_dk(const StepArgs &a, dim3 grid, dim3 block, cudaStream_t stream) {
+    auto kern = a.prologue ? decode_kernel<DK, Tin, true> : decode_kernel<DK, Tin, false>;
+    kern<<<grid, block, 0, stream>>>(static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
+                                     static_cast<const Tin *>(a.v), a.g, a.beta, a.state,
+                                     static_cast<Tin *>(a.o), a.HK, a.HV, a.dv, a.scale,
+                                     a.prologue);
+}
+
 template <typename Tin>
 cudaError_t launch_typed(const StepArgs &a, cudaStream_t stream) {
     const int band = a.dk == 128 ? band_rows<128>() : a.dk == 64 ? band_rows<64>() : band_rows<32>();
     const dim3 grid((unsigned)((size_t)a.N * a.HV), (unsigned)((a.dv + band - 1) / band)),
         block(kDecodeWarps * 32);
-    const Tin *q = static_cast<const Tin *>(a.q);
-    const Tin *k = static_cast<const Tin *>(a.k);
-    const Tin *v = static_cast<const Tin *>(a.v);
-    Tin *o = static_cast<Tin *>(a.o);
     switch (a.dk) {
-        case 32:
-            decode_kernel<32, Tin><<<grid, block, 0, stream>>>(q, k, v, a.g, a.beta, a.state, o,
-                                                               a.HK, a.HV, a.dv, a.scale);
-            break;
-        case 64:
-            decode_kernel<64, Tin><<<grid, block, 0, stream>>>(q, k, v, a.g, a.beta, a.state, o,
-                                                               a.HK, a.HV, a.dv, a.scale);
-            break;
-        case 128:
-            decode_kernel<128, Tin><<<grid, block, 0, stream>>>(q, k, v, a.g, a.beta, a.state, o,
-                                                                a.HK, a.HV, a.dv, a.scale);
-            break;
-        default:
-            return cudaErrorInvalidValue;
+        case 32: launch_dk<32, Tin>(a, grid, block, stream); break;
+        case 64: launch_dk<64, Tin>(a, grid, block, stream); break;
+        case 128: launch_dk<128, Tin>(a, grid, block, stream); break;
+        default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }

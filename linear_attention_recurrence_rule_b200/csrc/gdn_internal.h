@@ -23,6 +23,7 @@ struct PrefillArgs {
     void *workspace;
     size_t workspace_bytes;
     bool keep_status = false;   // leave the workspace status word as earlier calls left it
+    unsigned prologue = 0;      // GDN_PROLOGUE_* flags
 };
 
 struct StepArgs {
@@ -33,6 +34,7 @@ struct StepArgs {
     float scale;
     gdn_dtype dtype;
     void *o;
+    unsigned prologue = 0;
 };
 
 struct VerifyArgs {
@@ -43,6 +45,7 @@ struct VerifyArgs {
     float scale;
     gdn_dtype dtype;
     void *o;
+    unsigned prologue = 0;
 };
 
 
@@ -61,6 +64,7 @@ struct CommitDeltasArgs {
     float *state;
     int N, K, HK, HV, dk, dv;
     gdn_dtype dtype;
+    unsigned prologue = 0;
 };
 cudaError_t launch_commit_deltas(const CommitDeltasArgs &a, cudaStream_t stream);
 cudaError_t launch_commit(const float *states, const int32_t *accepted, float *state, int N, int K,

@@ -106,7 +106,7 @@ constexpr uint32_t P_TF = P_T + 64 * A_LD * 4;   // T fp32 [64][T_LD]
 constexpr uint32_t T_LD = 68;
 constexpr uint32_t P_X = P_TF + 64 * T_LD * 4;
 constexpr uint32_t X_LD = 36;
-constexpr uint32_t P_PB = P_X + 32 * X_LD * 4;             // beta, gamma, G
+constexpr uint32_t P_PB = P_X + 32 * X_LD * 4;   // beta, gamma, G, 1/|q|, 1/|k|
 constexpr uint32_t P_ST = 106496;   // two staging blocks (ST_BYTES each, 1024-aligned)
 constexpr uint32_t P_BAR = P_ST + 2 * ST_BYTES;
 
@@ -121,7 +121,7 @@ constexpr uint32_t AUX = (AUX_RAW + 15) & ~15u;
 constexpr uint32_t AUX_TSLOT = AUX, AUX_ABORT = AUX + 4, AUX_ARMED = AUX + 8,
                    AUX_CONSUMED = AUX + 12;
 constexpr uint32_t SMEM_BYTES = AUX + 16 + 1024;
-static_assert(P_PB + 3 * 64 * 4 <= P_ST, "prep layout");
+static_assert(P_PB + 5 * 64 * 4 <= P_ST, "prep layout");
 static_assert(64 * A_LD * 4 >= 16384, "T' tiles fit where A was");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(P_ST % 1024 == 0 && SLOT % 1024 == 0 && ST_BYTES % 1024 == 0 && P_T % 1024 == 0,
@@ -144,6 +144,7 @@ struct ClParams {
     __nv_bfloat16 *o;
     float *hT;
     unsigned int *status;
+    unsigned int prologue;   // GDN_PROLOGUE_* flags
 };
 
 struct Waiter {
@@ -528,6 +529,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
 }
 
 // ============================================================================ prep CTA
+template <bool PRO>
 __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                          const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
                          const Waiter &wt, int h, int64_t bos, int64_t eos, int nchunks,
@@ -636,6 +638,17 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         float *beta_s = reinterpret_cast<float *>(sm + P_PB);
         float *gam_p = beta_s + 64;
         float *G_p = gam_p + 64;
+        // input prologue: 1/|q_t|, 1/|k_t| (L2-normalised rows), folded into the
+        // diagonal scalings below; 1 throughout without it
+        float *rq_p = G_p + 64;
+        float *rk_p = rq_p + 64;
+        const unsigned pro = PRO ? p.prologue : 0u;   // compiled out without the prologue
+        const bool norm_qk = PRO && (pro & (GDN_PROLOGUE_NORM_Q | GDN_PROLOGUE_NORM_K)) != 0;
+        const bool logits = PRO && (pro & GDN_PROLOGUE_GATE_LOGITS) != 0;
+        if (PRO && !norm_qk && pt < 128) (pt < 64 ? rq_p : rk_p)[pt & 63] = 1.f;
+        // 1/|q_t|, 1/|k_t| where the prologue normalises, else exactly 1
+        auto rq = [&](int t) { return PRO ? rq_p[t] : 1.f; };
+        auto rk = [&](int t) { return PRO ? rk_p[t] : 1.f; };
         float *A_s = reinterpret_cast<float *>(sm + P_T);
         float *T_s = reinterpret_cast<float *>(sm + P_TF);
         float *X_s = reinterpret_cast<float *>(sm + P_X);
@@ -648,14 +661,22 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             const uint32_t stb = P_ST + (k & 1) * ST_BYTES;   // this chunk's staging block
             named_sync(NB_WORK, kPWorkThreads);
             if (warp == kPWork0) {
-                const float2 gp = load_g_pair(p.g, s0, L, HV, h);
+                float2 gp = load_g_pair(p.g, s0, L, HV, h);
+                if (logits) {   // g = log sigmoid(a) for the tokens of the chunk
+                    if (2 * lane < L) gp.x = gate_log_sigmoid(gp.x);
+                    if (2 * lane + 1 < L) gp.y = gate_log_sigmoid(gp.y);
+                }
                 const float2 Gv = warp_decay_scan(gp.x, gp.y);
                 G_p[2 * lane] = Gv.x;
                 G_p[2 * lane + 1] = Gv.y;
                 gam_p[2 * lane] = expf(Gv.x);
                 gam_p[2 * lane + 1] = expf(Gv.y);
             } else if (warp == kPWork0 + 1) {
-                const float2 bp = load_g_pair(p.beta, s0, L, HV, h);
+                float2 bp = load_g_pair(p.beta, s0, L, HV, h);
+                if (logits) {   // beta = sigmoid(b)
+                    if (2 * lane < L) bp.x = gate_sigmoid(bp.x);
+                    if (2 * lane + 1 < L) bp.y = gate_sigmoid(bp.y);
+                }
                 beta_s[2 * lane] = bp.x;
                 beta_s[2 * lane + 1] = bp.y;
             }
@@ -663,6 +684,37 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             // k - 2 of this CTA) have been copied out
             ok = warp_all(ok && wt(PB_X_DONE, ph) &&
                           (k < 2 || wt(PB_STAGE_FREE0 + (k & 1), (uint32_t)(((k >> 1) - 1) & 1))));
+            if (norm_qk) {
+                // squared norms of the 64 q and 64 k rows of the landed tiles: four
+                // threads per row, 64 bytes each (the 128B swizzle only permutes the
+                // 16-byte pieces inside a row)
+                ok = warp_all(ok && wt(PB_LD_FULL0 + (k & 1), (uint32_t)((k >> 1) & 1)));
+                if (ok) {
+                    const int qr = pt >> 2, part = pt & 3;
+                    const bool isk = qr >= 64;
+                    const int t = qr & 63;
+                    const uint8_t *rp = sm + P_QK + (k & 1) * QK_STRIDE + (part >> 1) * 16384 +
+                                        (isk ? 8192 : 0) + t * 128 + (part & 1) * 64;
+                    float ss = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(rp + 16 * i);
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(
+                                *reinterpret_cast<const __nv_bfloat162 *>(&ws[e]));
+                            ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                        }
+                    }
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+                    if (part == 0) {
+                        const bool on = (pro & (isk ? GDN_PROLOGUE_NORM_K : GDN_PROLOGUE_NORM_Q)) != 0;
+                        (isk ? rk_p : rq_p)[t] = t < L ? (on ? inv_l2norm(ss) : 1.f) : 0.f;
+                    }
+                }
+            }
             named_sync(NB_WORK, kPWorkThreads);
             if (ok) {
                 tc_fence_after();
@@ -674,6 +726,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 const int row0 = 32 * ((warp & 3) & 1);          // first row of this warp
                 const bool all_masked = 16 * qtr > row0 + 31;    // every column > every row
                 const float Gi = G_p[row];
+                const float ri = r < 64 ? rq(row) : rk(row);
                 if (r < 64) {
                     if (all_masked) {
 #pragma unroll
@@ -682,7 +735,8 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int col = 16 * qtr + j;
-                            v[j] = (col <= row) ? __expf(Gi - G_p[col]) * v[j] : 0.f;
+                            v[j] = (col <= row) ? __expf(Gi - G_p[col]) * (ri * rk(col)) * v[j]
+                                                : 0.f;
                         }
                     }
 #pragma unroll
@@ -691,7 +745,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                         st_chunk_hilo(sb + stb + ST_P + off, sb + stb + ST_P + 8192 + off, v + 8 * cc);
                     }
                 } else {
-                    const float bi = beta_s[row];
+                    const float bi = beta_s[row] * ri;
                     if (all_masked) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) v[j] = 0.f;
@@ -699,7 +753,8 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int col = 16 * qtr + j;
-                            v[j] = (col < row) ? bi * __expf(Gi - G_p[col]) * v[j] : 0.f;
+                            v[j] = (col < row) ? bi * __expf(Gi - G_p[col]) * rk(col) * v[j]
+                                               : 0.f;
                         }
                     }
                     float4 *dst = reinterpret_cast<float4 *>(A_s + row * A_LD + 16 * qtr);
@@ -710,8 +765,8 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 // decay table of this chunk for the chain CTA
                 if (pt < 64) {
                     float *tb = reinterpret_cast<float *>(sm + stb + ST_TAB);
-                    tb[pt] = __expf(G_p[63] - G_p[pt]);    // gamma_L / gamma_t
-                    tb[64 + pt] = gam_p[pt];               // gamma_t
+                    tb[pt] = __expf(G_p[63] - G_p[pt]) * rk(pt);   // gamma_L / gamma_t / |k_t|
+                    tb[64 + pt] = gam_p[pt] * rq(pt);              // gamma_t / |q_t|
                     if (pt == 0) tb[128] = gam_p[63];      // gamma_L
                 }
             }
@@ -794,7 +849,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                     const int s = 8 * chunk16 + e;
                     const float tv = (s <= t) ? T_s[t * T_LD + s] : 0.f;
                     a2[e] = tv * beta_s[s];
-                    a1[e] = a2[e] * gam_p[s];
+                    a1[e] = a2[e] * gam_p[s] * rk(s);
                 }
                 const uint32_t off = sw128_chunk(t, chunk16);
                 st_chunk_hilo(sb + P_T + off, sb + P_T + 8192 + off, a1);
@@ -829,6 +884,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     }
 }
 
+template <bool PRO>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -888,7 +944,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (rank == 0)
         chain_cta(&tm_q, &tm_k, &tm_v, &tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
     else
-        prep_cta(&tm_q, &tm_k, &tm_v, p, sm, sb, tmem, wt, h, bos, eos, nchunks, rank);
+        prep_cta<PRO>(&tm_q, &tm_k, &tm_v, p, sm, sb, tmem, wt, h, bos, eos, nchunks, rank);
 
     tc_fence_before();
     __syncthreads();
@@ -931,11 +987,12 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     uint32_t obox[3] = {32, 1, 16};
     if (!encode_bf16_map(&to, a.o, 3, dv, sv, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    err = cudaFuncSetAttribute(prefill_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kern = a.prologue ? prefill_cluster_kernel<true> : prefill_cluster_kernel<false>;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     ClParams prm{a.g, a.beta, a.h0, a.cu_seqlens, a.T, a.HK, a.HV, a.scale,
-                 static_cast<__nv_bfloat16 *>(a.o), a.hT, status};
+                 static_cast<__nv_bfloat16 *>(a.o), a.hT, status, a.prologue};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(kClusterSize * a.HV), (unsigned)a.N, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -948,7 +1005,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, prefill_cluster_kernel, tq, tk, tv, to, prm);
+    err = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, prm);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }

@@ -45,7 +45,7 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const Tin *__restrict__ v, const float *__restrict__ g,
                     const float *__restrict__ beta, const float *__restrict__ h0,
                     const int32_t *__restrict__ cu, int64_t T, int HK, int HV, int dv,
-                    float scale, Tin *__restrict__ o, float *__restrict__ hT) {
+                    float scale, Tin *__restrict__ o, float *__restrict__ hT, unsigned pro) {
     using L_ = SimtSmem<DK, BV, C>;
     constexpr int KP = L_::KP, CP = L_::CP, NT = kSimtThreads;
     const int tid = threadIdx.x;
@@ -101,14 +101,30 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             Ys[idx] = i < L ? to_f32(v[((size_t)(s0 + i) * HV + h) * dv + e0 + e]) : 0.f;
         }
         if (tid < C) {
-            Gs[tid] = tid < L ? g[(s0 + tid) * HV + h] : 0.f;
-            Bs[tid] = tid < L ? beta[(s0 + tid) * HV + h] : 0.f;
+            // with gate logits: g = log sigmoid(a), beta = sigmoid(b); padding stays 0
+            const bool logits = (pro & GDN_PROLOGUE_GATE_LOGITS) != 0;
+            const float gv = tid < L ? g[(s0 + tid) * HV + h] : 0.f;
+            const float bv = tid < L ? beta[(s0 + tid) * HV + h] : 0.f;
+            Gs[tid] = (logits && tid < L) ? gate_log_sigmoid(gv) : gv;
+            Bs[tid] = (logits && tid < L) ? gate_sigmoid(bv) : bv;
         }
         __syncthreads();
         // ---- chunk-local running sum of the log decay ----
         if (tid == 0) {
             float run = 0.f;
             for (int i = 0; i < L; ++i) { run += Gs[i]; Gs[i] = run; }
+        }
+        // ---- input prologue: L2-normalised q / k rows (one thread per row) ----
+        if (pro & (GDN_PROLOGUE_NORM_Q | GDN_PROLOGUE_NORM_K)) {
+            for (int idx = tid; idx < 2 * L; idx += NT) {
+                const bool is_k = idx >= L;
+                if (!(pro & (is_k ? GDN_PROLOGUE_NORM_K : GDN_PROLOGUE_NORM_Q))) continue;
+                float *row = (is_k ? Ks : Qs) + (idx - (is_k ? L : 0)) * KP;
+                float ss = 0.f;
+                for (int a = 0; a < DK; ++a) ss = fmaf(row[a], row[a], ss);
+                const float r = inv_l2norm(ss);
+                for (int a = 0; a < DK; ++a) row[a] *= r;
+            }
         }
         __syncthreads();
         // ---- A (strictly lower) and P (lower incl. diagonal) ----
@@ -205,7 +221,7 @@ cudaError_t launch_shape(const PrefillArgs &a, cudaStream_t stream) {
     kern<<<grid, block, smem, stream>>>(
         static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
         static_cast<const Tin *>(a.v), a.g, a.beta, a.h0, a.cu_seqlens, a.T, a.HK, a.HV, a.dv,
-        a.scale, static_cast<Tin *>(a.o), a.hT);
+        a.scale, static_cast<Tin *>(a.o), a.hT, a.prologue);
     return cudaGetLastError();
 }
 

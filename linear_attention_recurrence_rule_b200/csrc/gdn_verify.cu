@@ -43,12 +43,42 @@ constexpr int kVerifyRows = 2;   // rows per lane
 template <int DK>
 __host__ __device__ constexpr int verify_band() { return kVerifyWarps * (32 / (DK / (4 * kVerifyF4))) * kVerifyRows; }
 
-template <int DK, typename Tin>
+// Input prologue on rows staged in shared memory: L2-normalise rows [0, nrows),
+// one warp per row.
+template <int DK>
+__device__ __forceinline__ void normalize_rows(float4 (*rows)[DK / 4], int nrows, int warp,
+                                               int lane) {
+    for (int t = warp; t < nrows; t += kVerifyWarps) {
+        float ss = 0.f;
+        for (int j = lane; j < DK / 4; j += 32) ss += dot4(rows[t][j], rows[t][j]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float r = inv_l2norm(ss);
+        for (int j = lane; j < DK / 4; j += 32) rows[t][j] = scale4(rows[t][j], r);
+    }
+}
+
+template <int DK>
+__device__ __forceinline__ void prologue_qk(float4 (*ks)[DK / 4], float4 (*qs)[DK / 4], int K,
+                                            unsigned pro, int warp, int lane) {
+    if (pro & GDN_PROLOGUE_NORM_K) normalize_rows<DK>(ks, K, warp, lane);
+    if (pro & GDN_PROLOGUE_NORM_Q) normalize_rows<DK>(qs, K, warp, lane);
+}
+
+__device__ __forceinline__ float gate_alpha(float g, unsigned pro) {
+    return (pro & GDN_PROLOGUE_GATE_LOGITS) ? gate_sigmoid(g) : expf(g);
+}
+__device__ __forceinline__ float gate_beta(float b, unsigned pro) {
+    return (pro & GDN_PROLOGUE_GATE_LOGITS) ? gate_sigmoid(b) : b;
+}
+
+template <int DK, typename Tin, bool PRO>
 __global__ void __launch_bounds__(kVerifyWarps * 32, 2)
 verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ g, const float *__restrict__ beta,
               const float *__restrict__ state, float *__restrict__ states, float *__restrict__ u_out,
-              Tin *__restrict__ o, int K, int HK, int HV, int dv, float scale) {
+              Tin *__restrict__ o, int K, int HK, int HV, int dv, float scale, unsigned pro_arg) {
+    const unsigned pro = PRO ? pro_arg : 0u;   // compiled out without the prologue
     constexpr int LPR = DK / (4 * kVerifyF4);   // lanes per row: 2, 4, 8
     constexpr int RPW = 32 / LPR;               // rows per warp instruction
     constexpr int BAND = verify_band<DK>();
@@ -86,10 +116,14 @@ verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     }
     if (threadIdx.x < K) {
         const size_t gi = ((size_t)n * K + threadIdx.x) * HV + h;
-        al[threadIdx.x] = expf(g[gi]);
-        be[threadIdx.x] = beta[gi];
+        al[threadIdx.x] = gate_alpha(g[gi], pro);
+        be[threadIdx.x] = gate_beta(beta[gi], pro);
     }
     __syncthreads();
+    if (pro & (GDN_PROLOGUE_NORM_Q | GDN_PROLOGUE_NORM_K)) {
+        prologue_qk<DK>(ks, qs, K, pro, warp, lane);
+        __syncthreads();
+    }
     for (int t = 0; t < K; ++t) {
         float4 kk[kVerifyF4];
         float kq = 0.f;
@@ -155,12 +189,13 @@ verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 // per-row scalars whose coefficients (the K x K Gram products k_j . k_t and
 // k_j . q_t times the decays, times beta and scale) are tabled once per CTA.
 // KT is the compile-time bound on K (4, 8 or 16).
-template <int DK, int KT, typename Tin>
+template <int DK, int KT, typename Tin, bool PRO>
 __global__ void __launch_bounds__(kVerifyWarps * 32, KT <= 4 ? 3 : 2)
 verify_wy_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                  const float *__restrict__ g, const float *__restrict__ beta,
                  const float *__restrict__ state, float *__restrict__ u_out, Tin *__restrict__ o,
-                 int K, int HK, int HV, int dv, float scale) {
+                 int K, int HK, int HV, int dv, float scale, unsigned pro_arg) {
+    const unsigned pro = PRO ? pro_arg : 0u;
     constexpr int LPR = DK / (4 * kVerifyF4);
     constexpr int RPW = 32 / LPR;
     constexpr int BAND = verify_band<DK>();
@@ -199,10 +234,14 @@ verify_wy_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin
     }
     if (threadIdx.x < K) {
         const size_t gi = ((size_t)n * K + threadIdx.x) * HV + h;
-        al[threadIdx.x] = expf(g[gi]);
-        be[threadIdx.x] = beta[gi];
+        al[threadIdx.x] = gate_alpha(g[gi], pro);
+        be[threadIdx.x] = gate_beta(beta[gi], pro);
     }
     __syncthreads();
+    if (pro & (GDN_PROLOGUE_NORM_Q | GDN_PROLOGUE_NORM_K)) {
+        prologue_qk<DK>(ks, qs, K, pro, warp, lane);
+        __syncthreads();
+    }
     // Gram products, one warp per pair
     for (int p = warp; p < 2 * K * K; p += kVerifyWarps) {
         const int which = p / (K * K), rem = p - which * K * K;
@@ -302,11 +341,13 @@ commit_kernel(const float *__restrict__ states, const int32_t *__restrict__ acce
 // element is read and written once; k_t and the scaled u_t of the band sit in
 // shared memory.  Same row layout and bands as the verify kernel; all of a lane's
 // state loads are issued before the staging and the arithmetic.
-template <int DK, typename Tin>
+template <int DK, typename Tin, bool PRO>
 __global__ void __launch_bounds__(kVerifyWarps * 32, 3)
 commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
                      const float *__restrict__ u, const int32_t *__restrict__ accepted,
-                     float *__restrict__ state, int K, int HK, int HV, int dv) {
+                     float *__restrict__ state, int K, int HK, int HV, int dv,
+                     unsigned pro_arg) {
+    const unsigned pro = PRO ? pro_arg : 0u;
     constexpr int LPR = DK / (4 * kVerifyF4);
     constexpr int RPW = 32 / LPR;
     constexpr int BAND = verify_band<DK>();
@@ -337,7 +378,7 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
         float c_run = 1.f;
         for (int t = a - 1; t >= 0; --t) {
             coef[t] = c_run;
-            c_run *= expf(g[((size_t)n * K + t) * HV + h]);
+            c_run *= gate_alpha(g[((size_t)n * K + t) * HV + h], pro);
         }
         coef[kVerifyMaxDrafts] = c_run;
     }
@@ -346,6 +387,7 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
         ks[t][j] = load4(k + (((size_t)n * K + t) * HK + c) * DK + 4 * j);
     }
     __syncthreads();
+    if (pro & GDN_PROLOGUE_NORM_K) normalize_rows<DK>(ks, a, warp, lane);   // read after the next barrier
     for (int i = threadIdx.x; i < a * BAND; i += blockDim.x) {
         const int t = i / BAND, r = i - t * BAND;
         const int row = base + r;
@@ -388,10 +430,11 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
 
 template <int DK, int KT, typename Tin>
 void launch_verify_wy(const VerifyArgs &a, dim3 grid, dim3 block, cudaStream_t stream) {
-    verify_wy_kernel<DK, KT, Tin><<<grid, block, 0, stream>>>(
+    auto kern = a.prologue ? verify_wy_kernel<DK, KT, Tin, true> : verify_wy_kernel<DK, KT, Tin, false>;
+    kern<<<grid, block, 0, stream>>>(
         static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
         static_cast<const Tin *>(a.v), a.g, a.beta, a.state, a.u, static_cast<Tin *>(a.o), a.K,
-        a.HK, a.HV, a.dv, a.scale);
+        a.HK, a.HV, a.dv, a.scale, a.prologue);
 }
 
 template <int DK, typename Tin>
@@ -404,16 +447,21 @@ void launch_verify_wy_k(const VerifyArgs &a, dim3 grid, dim3 block, cudaStream_t
         launch_verify_wy<DK, 16, Tin>(a, grid, block, stream);
 }
 
+template <int DK, typename Tin>
+void launch_verify_seq(const VerifyArgs &a, dim3 grid, dim3 block, cudaStream_t stream) {
+    auto kern = a.prologue ? verify_kernel<DK, Tin, true> : verify_kernel<DK, Tin, false>;
+    kern<<<grid, block, 0, stream>>>(static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
+                                     static_cast<const Tin *>(a.v), a.g, a.beta, a.state,
+                                     a.states, a.u, static_cast<Tin *>(a.o), a.K, a.HK, a.HV,
+                                     a.dv, a.scale, a.prologue);
+}
+
 template <typename Tin>
 cudaError_t launch_verify_typed(const VerifyArgs &a, cudaStream_t stream) {
     const int band = a.dk == 128 ? verify_band<128>() : a.dk == 64 ? verify_band<64>()
                                                                    : verify_band<32>();
     const dim3 grid((unsigned)((size_t)a.N * a.HV), (unsigned)((a.dv + band - 1) / band)),
         block(kVerifyWarps * 32);
-    const Tin *q = static_cast<const Tin *>(a.q);
-    const Tin *k = static_cast<const Tin *>(a.k);
-    const Tin *v = static_cast<const Tin *>(a.v);
-    Tin *o = static_cast<Tin *>(a.o);
     if (a.states == nullptr) {
         // no per-draft states asked for: the state is never updated in registers
         switch (a.dk) {
@@ -425,23 +473,10 @@ cudaError_t launch_verify_typed(const VerifyArgs &a, cudaStream_t stream) {
         return cudaGetLastError();
     }
     switch (a.dk) {
-        case 32:
-            verify_kernel<32, Tin><<<grid, block, 0, stream>>>(q, k, v, a.g, a.beta, a.state, a.states,
-                                                               a.u, o, a.K, a.HK, a.HV, a.dv,
-                                                               a.scale);
-            break;
-        case 64:
-            verify_kernel<64, Tin><<<grid, block, 0, stream>>>(q, k, v, a.g, a.beta, a.state, a.states,
-                                                               a.u, o, a.K, a.HK, a.HV, a.dv,
-                                                               a.scale);
-            break;
-        case 128:
-            verify_kernel<128, Tin><<<grid, block, 0, stream>>>(q, k, v, a.g, a.beta, a.state,
-                                                                a.states, a.u, o, a.K, a.HK, a.HV,
-                                                                a.dv, a.scale);
-            break;
-        default:
-            return cudaErrorInvalidValue;
+        case 32: launch_verify_seq<32, Tin>(a, grid, block, stream); break;
+        case 64: launch_verify_seq<64, Tin>(a, grid, block, stream); break;
+        case 128: launch_verify_seq<128, Tin>(a, grid, block, stream); break;
+        default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }
@@ -454,31 +489,24 @@ cudaError_t launch_verify(const VerifyArgs &a, cudaStream_t stream) {
                                : launch_verify_typed<float>(a, stream);
 }
 
+template <int DK, typename Tin>
+void launch_commit_dk(const CommitDeltasArgs &a, dim3 grid, dim3 block, cudaStream_t stream) {
+    auto kern = a.prologue ? commit_deltas_kernel<DK, Tin, true> : commit_deltas_kernel<DK, Tin, false>;
+    kern<<<grid, block, 0, stream>>>(static_cast<const Tin *>(a.k), a.g, a.u, a.accepted, a.state,
+                                     a.K, a.HK, a.HV, a.dv, a.prologue);
+}
+
 template <typename Tin>
 cudaError_t launch_commit_deltas_typed(const CommitDeltasArgs &a, cudaStream_t stream) {
     const int band = a.dk == 128 ? verify_band<128>() : a.dk == 64 ? verify_band<64>()
                                                                    : verify_band<32>();
     const dim3 grid((unsigned)((size_t)a.N * a.HV), (unsigned)((a.dv + band - 1) / band)),
         block(kVerifyWarps * 32);
-    const Tin *k = static_cast<const Tin *>(a.k);
     switch (a.dk) {
-        case 32:
-            commit_deltas_kernel<32, Tin><<<grid, block, 0, stream>>>(k, a.g, a.u, a.accepted,
-                                                                      a.state, a.K, a.HK, a.HV,
-                                                                      a.dv);
-            break;
-        case 64:
-            commit_deltas_kernel<64, Tin><<<grid, block, 0, stream>>>(k, a.g, a.u, a.accepted,
-                                                                      a.state, a.K, a.HK, a.HV,
-                                                                      a.dv);
-            break;
-        case 128:
-            commit_deltas_kernel<128, Tin><<<grid, block, 0, stream>>>(k, a.g, a.u, a.accepted,
-                                                                       a.state, a.K, a.HK, a.HV,
-                                                                       a.dv);
-            break;
-        default:
-            return cudaErrorInvalidValue;
+        case 32: launch_commit_dk<32, Tin>(a, grid, block, stream); break;
+        case 64: launch_commit_dk<64, Tin>(a, grid, block, stream); break;
+        case 128: launch_commit_dk<128, Tin>(a, grid, block, stream); break;
+        default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }

@@ -18,6 +18,9 @@ from . import _build
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_ALIGNMENT, GDN_ERR_CUDA, \
     GDN_ERR_TIMEOUT, GDN_ERR_WORKSPACE = range(7)
 GDN_F32, GDN_BF16 = 0, 1
+# input prologue flags (GDN_PROLOGUE_* in gdn.h)
+PROLOGUE_NORM_Q, PROLOGUE_NORM_K, PROLOGUE_GATE_LOGITS = 1, 2, 4
+PROLOGUE_ALL = 7
 
 _lock = threading.Lock()
 _handle = None
@@ -54,17 +57,25 @@ def load_library() -> ctypes.CDLL:
             lib.gdn_chunk_prefill.restype = i32
             lib.gdn_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
                                               i32, i32, ctypes.c_float, i32, vp, vp, vp, sz, vp]
+            lib.gdn_chunk_prefill_ex.restype = i32
+            lib.gdn_chunk_prefill_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                                 i32, i32, i32, ctypes.c_float, i32, vp, vp, vp,
+                                                 sz, ctypes.c_uint, vp]
+            lib.gdn_recurrent_step_ex.restype = i32
+            lib.gdn_recurrent_step_ex.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                                  i32, ctypes.c_float, i32, vp, ctypes.c_uint, vp]
             lib.gdn_recurrent_step.restype = i32
             lib.gdn_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                                ctypes.c_float, i32, vp, vp]
             lib.gdn_recurrent_verify.restype = i32
             lib.gdn_recurrent_verify.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
-                                                 i32, ctypes.c_float, i32, vp, vp, vp, vp]
+                                                 i32, ctypes.c_float, i32, vp, vp, vp,
+                                                 ctypes.c_uint, vp]
             lib.gdn_state_commit.restype = i32
             lib.gdn_state_commit.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
             lib.gdn_state_commit_deltas.restype = i32
             lib.gdn_state_commit_deltas.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
-                                                    i32, i32, vp]
+                                                    i32, i32, ctypes.c_uint, vp]
             lib.gdn_chunk_prefill_path.restype = i32
             lib.gdn_chunk_prefill_path.argtypes = [i32, i32, i32, i32]
             lib.gdn_read_status.restype = i32
@@ -124,12 +135,13 @@ def gdn_chunk_prefill_workspace_size(N, T, HK, HV, dk, dv, chunk, dtype, varlen)
 
 def gdn_chunk_prefill(q, k, v, g, beta, h0=None, cu_seqlens=None, chunk: int = 64,
                       scale: float = 1.0, o=None, hT=None, workspace=None, stream=None,
-                      output_final_state: bool = True):
+                      output_final_state: bool = True, prologue: int = 0):
     """Chunkwise prefill through ``gdn_chunk_prefill``.
 
     q, k [B,T,HK,dk]; v [B,T,HV,dv] (bf16 or fp32); g, beta [B,T,HV] fp32;
     h0 [N,HV,dv,dk] fp32 or None; cu_seqlens int32 [N+1] (then B == 1) or None.
-    Returns (o [B,T,HV,dv], hT [N,HV,dv,dk] or None).
+    ``prologue``: PROLOGUE_* flags fused into the kernels (L2-normalised q / k,
+    g and beta given as logits).  Returns (o [B,T,HV,dv], hT [N,HV,dv,dk] or None).
     """
     lib = load_library()
     dev = q.device
@@ -168,20 +180,21 @@ def gdn_chunk_prefill(q, k, v, g, beta, h0=None, cu_seqlens=None, chunk: int = 6
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.gdn_chunk_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
-                               _ptr(cu_seqlens), N, T, HK, HV, dk, dv, int(chunk),
-                               float(scale), code, _ptr(o), _ptr(hT), _ptr(workspace),
-                               ws_bytes, _stream_ptr(stream, dev))
+    st = lib.gdn_chunk_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                  _ptr(cu_seqlens), N, T, HK, HV, dk, dv, int(chunk),
+                                  float(scale), code, _ptr(o), _ptr(hT), _ptr(workspace),
+                                  ws_bytes, int(prologue), _stream_ptr(stream, dev))
     if st != GDN_OK:
         raise GDNError(st, "gdn_chunk_prefill")
     return o, hT
 
 
-def gdn_recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, o=None, stream=None):
+def gdn_recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, o=None, stream=None,
+                       prologue: int = 0):
     """One fused decode token through ``gdn_recurrent_step``; ``state`` is updated in place.
 
     q, k [N,HK,dk]; v [N,HV,dv] (bf16 or fp32); g, beta [N,HV] fp32;
-    state [N,HV,dv,dk] fp32.  Returns o [N,HV,dv].
+    state [N,HV,dv,dk] fp32.  ``prologue``: PROLOGUE_* flags.  Returns o [N,HV,dv].
     """
     lib = load_library()
     dev = q.device
@@ -200,16 +213,16 @@ def gdn_recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, o=None, stre
         o = torch.empty_like(v)
     else:
         _need(o, "o", v.dtype, dev)
-    st = lib.gdn_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
-                                N, HK, HV, dk, dv, float(scale), _dtype_code(q), _ptr(o),
-                                _stream_ptr(stream, dev))
+    st = lib.gdn_recurrent_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                                   N, HK, HV, dk, dv, float(scale), _dtype_code(q), _ptr(o),
+                                   int(prologue), _stream_ptr(stream, dev))
     if st != GDN_OK:
         raise GDNError(st, "gdn_recurrent_step")
     return o
 
 
 def gdn_recurrent_verify(q, k, v, g, beta, state, scale: float = 1.0, o=None, states_out=None,
-                         u_out=None, rollback="states", stream=None):
+                         u_out=None, rollback="states", stream=None, prologue: int = 0):
     """K draft tokens per sequence through ``gdn_recurrent_verify``; ``state`` is only read.
 
     q, k [N,K,HK,dk]; v [N,K,HV,dv] (bf16 or fp32); g, beta [N,K,HV] fp32;
@@ -257,7 +270,8 @@ def gdn_recurrent_verify(q, k, v, g, beta, state, scale: float = 1.0, o=None, st
         u_out = None
     st = lib.gdn_recurrent_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
                                   N, K, HK, HV, dk, dv, float(scale), _dtype_code(q), _ptr(o),
-                                  _ptr(states_out), _ptr(u_out), _stream_ptr(stream, dev))
+                                  _ptr(states_out), _ptr(u_out), int(prologue),
+                                  _stream_ptr(stream, dev))
     if st != GDN_OK:
         raise GDNError(st, "gdn_recurrent_verify")
     return o, states_out, u_out
@@ -285,7 +299,7 @@ def gdn_state_commit(states, accepted, state, stream=None):
     return state
 
 
-def gdn_state_commit_deltas(k, g, u, accepted, state, stream=None):
+def gdn_state_commit_deltas(k, g, u, accepted, state, stream=None, prologue: int = 0):
     """In-place roll-back from a verify pass's update vectors (``gdn_state_commit_deltas``).
 
     k [N,K,HK,dk] (the verify input, bf16 or fp32); g [N,K,HV] fp32; u
@@ -308,7 +322,8 @@ def gdn_state_commit_deltas(k, g, u, accepted, state, stream=None):
         raise ValueError("expected k [N,K,HK,dk], g [N,K,HV], u [N,K,HV,dv], accepted [N], "
                          "state [N,HV,dv,dk]")
     st = lib.gdn_state_commit_deltas(_ptr(k), _ptr(g), _ptr(u), _ptr(accepted), _ptr(state), N, K,
-                                     HK, HV, dk, dv, _dtype_code(k), _stream_ptr(stream, dev))
+                                     HK, HV, dk, dv, _dtype_code(k), int(prologue),
+                                     _stream_ptr(stream, dev))
     if st != GDN_OK:
         raise GDNError(st, "gdn_state_commit_deltas")
     return state

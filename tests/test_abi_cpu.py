@@ -119,7 +119,8 @@ def verify_call(lib, **kw):
     a.update(kw)
     return lib.gdn_recurrent_verify(a["q"], a["k"], a["v"], a["g"], a["beta"], a["state"],
                                     a["N"], a["K"], a["HK"], a["HV"], a["dk"], a["dv"],
-                                    a["scale"], a["dtype"], a["o"], a["states"], a["u"], None)
+                                    a["scale"], a["dtype"], a["o"], a["states"], a["u"],
+                                    a.get("pro", 0), None)
 
 
 def test_verify_validation(lib):
@@ -159,7 +160,7 @@ def test_commit_deltas_validation(lib):
         a.update(kw)
         return lib.gdn_state_commit_deltas(a["k"], a["g"], a["u"], a["acc"], a["state"], a["N"],
                                            a["K"], a["HK"], a["HV"], a["dk"], a["dv"], a["dtype"],
-                                           None)
+                                           a.get("pro", 0), None)
     assert call(u=None) == gdn.GDN_ERR_INVALID_ARG
     assert call(HK=3) == gdn.GDN_ERR_INVALID_ARG
     assert call(dtype=9) == gdn.GDN_ERR_INVALID_ARG
@@ -167,3 +168,23 @@ def test_commit_deltas_validation(lib):
     assert call(dv=300) == gdn.GDN_ERR_UNSUPPORTED
     assert call(state=fake(0x5004)) == gdn.GDN_ERR_ALIGNMENT
     assert call(N=0, k=None, u=None) == gdn.GDN_OK
+    assert call(pro=8) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_prologue_flags_are_validated(lib):
+    assert gdn.PROLOGUE_ALL == gdn.PROLOGUE_NORM_Q | gdn.PROLOGUE_NORM_K | gdn.PROLOGUE_GATE_LOGITS
+    text = "".join(open(h).read() for h in HEADERS)
+    for name, val in (("NORM_Q", 1), ("NORM_K", 2), ("GATE_LOGITS", 4), ("ALL", 7)):
+        assert re.search(rf"#define GDN_PROLOGUE_{name} {val}u", text)
+    a = dict(q=fake(0x1000), k=fake(0x2000), v=fake(0x3000), g=fake(0x4000), beta=fake(0x5000))
+    assert lib.gdn_chunk_prefill_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], None, None, 1, 64,
+                                    1, 2, 32, 32, 16, 1.0, gdn.GDN_F32, fake(0x6000), None, None,
+                                    0, 8, None) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_recurrent_step_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], fake(0x6000), 2,
+                                     1, 2, 128, 128, 1.0, gdn.GDN_BF16, fake(0x7000), 16,
+                                     None) == gdn.GDN_ERR_INVALID_ARG
+    assert verify_call(lib, pro=9) == gdn.GDN_ERR_INVALID_ARG
+    # valid flags still go through the other checks first
+    assert lib.gdn_recurrent_step_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], fake(0x6004), 2,
+                                     1, 2, 128, 128, 1.0, gdn.GDN_BF16, fake(0x7000), 7,
+                                     None) == gdn.GDN_ERR_ALIGNMENT
