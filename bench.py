@@ -152,12 +152,77 @@ def measure_verify(gdn, torch, dev, stream, peaks, peak_src, rank, world, max_ov
             "ms_per_round": total_ms / rounds, "verify_ms": v_ms, "commit_ms": c_ms,
             "bytes_per_round": vb + cb, "gb_per_s": (vb + cb) / (total_ms / rounds / 1e3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": v_gbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": v_gbs / hbm_peak, "traffic": None, "peak_source": peak_src,
-                         "kernel": "verify"},
+                         "frac": v_gbs / hbm_peak, "traffic": kernel_traffic("verify_" + form),
+                         "peak_source": peak_src,
+                         "kernel": "verify_wy" if form == "deltas" else "verify"},
             "commit_roofline": {"bound": "hbm", "achieved": c_gbs, "peak": hbm_peak,
                                 "unit": "GB/s", "frac": c_gbs / hbm_peak},
             "gpu_launches": 2 * rounds, "clocks": clocks}
     return out
+
+
+def measure_prologue(gdn, torch, dev, stream, x, w, ws, o, hT, rank, barrier, max_over_ranks,
+                     plain_s, args):
+    """Prefill (the bench workload) and one decode step (decode_256x64 shapes)
+    with every prologue flag on raw projections: q, k rows of norm ~U(0.25, 4)
+    and gate logits.  Reported beside the plain kernels' times."""
+    from linear_attention_recurrence_rule_b200.inputs import (WORKLOADS, raw_projections,
+                                                              workload_inputs)
+    flags = gdn.PROLOGUE_ALL
+    r = raw_projections(x, seed=900 + rank)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in r.items()}
+    tokens = d["q"].shape[0] * d["q"].shape[1]
+
+    def step():
+        gdn.gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], chunk=w.chunk, o=o,
+                              hT=hT, workspace=ws, stream=stream, prologue=flags)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a_, b_ in ev:
+        a_.record(stream)
+        step()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    pf_s = statistics.mean(a_.elapsed_time(b_) for a_, b_ in ev) / 1e3
+    total_ms = max_over_ranks(ev[0][0].elapsed_time(ev[-1][1]))
+    del d
+    # decode: one step over the decode workload's 256 sequences, raw inputs
+    wd = WORKLOADS[DECODE_WORKLOAD]
+    y = raw_projections(workload_inputs(DECODE_WORKLOAD, steps=8,
+                                        seed_offset=replica_seed_offset(rank)), seed=901 + rank)
+    dy = {k: v.to(dev) for k, v in y.items()}
+    S = dy["state"].clone()
+    od = torch.empty_like(dy["v"][0])
+    res = {}
+    for tag, fl in (("plain", 0), ("prologue", flags)):
+        for t in range(3):
+            gdn.gdn_recurrent_step(dy["q"][t], dy["k"][t], dy["v"][t], dy["g"][t], dy["beta"][t],
+                                   S, o=od, stream=stream, prologue=fl)
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(8)]
+        for t, (a_, b_) in enumerate(evs):
+            a_.record(stream)
+            gdn.gdn_recurrent_step(dy["q"][t], dy["k"][t], dy["v"][t], dy["g"][t], dy["beta"][t],
+                                   S, o=od, stream=stream, prologue=fl)
+            b_.record(stream)
+        torch.cuda.synchronize()
+        res[tag] = statistics.mean(a_.elapsed_time(b_) for a_, b_ in evs)
+    return {"flags": "norm_q|norm_k|gate_logits",
+            "prefill": {"workload": WORKLOAD, "value": tokens * args.steps / (total_ms / 1e3),
+                        "unit": "tokens/s", "ms_per_step": pf_s * 1e3,
+                        "plain_ms_per_step": plain_s * 1e3,
+                        "overhead": pf_s / plain_s - 1.0, "gpu_launches": args.steps},
+            "decode": {"workload": DECODE_WORKLOAD, "ms_per_step": res["prologue"],
+                       "plain_ms_per_step": res["plain"],
+                       "overhead": res["prologue"] / res["plain"] - 1.0, "gpu_launches": 16},
+            "inputs": "raw projections: q, k rows of norm ~U(0.25, 4), forget logits ~N(3, 1), "
+                      "write logits ~N(0, 1)"}
 
 
 def dist_max(x, device=None):
@@ -195,12 +260,18 @@ def load_peaks():
 # Each entry carries the sha256 of the kernel source it was taken on; a changed
 # source reports null.
 NCU_TRAFFIC = {
-    # full decode_256x64 step: 541,150,720 read + 480,181,760 written
-    "decode": {"bytes": 1021332480, "source": "gdn_decode.cu",
-               "sha256": "60331e595882541b536c8af94903466c17d66939204de90625311abbde61cc2b"},
-    # full long_prefill_64k launch: 1,090,708,736 read + 513,699,328 written
-    "prefill_cluster": {"bytes": 1604408064, "source": "gdn_prefill_cluster.cu",
-                        "sha256": "4e2bdccb96be93a00611bfd48ed5816e997a2ff598e5bc8755f01bdde74c5d2c"},
+    # full decode_256x64 step: 541,149,696 read + 477,217,536 written
+    "decode": {"bytes": 1018367232, "source": "gdn_decode.cu",
+               "sha256": "1b91a761970c803c59da9d7895e9892ca047fb13f5922a6be591c74fb54279bd"},
+    # full long_prefill_64k launch: 1,090,729,728 read + 510,220,032 written
+    "prefill_cluster": {"bytes": 1600949760, "source": "gdn_prefill_cluster.cu",
+                        "sha256": "881a325e6d56777fe19db569636ec05bdd86d18a1d8dea300fed5c5991d89ae0"},
+    # verify_256x4, update-vector form: 553,954,304 read + 4,621,312 written
+    "verify_deltas": {"bytes": 558575616, "source": "gdn_verify.cu",
+                      "sha256": "813090dfadf764cb421f435cc4489f27999477e790e4313a689feb6d7590babe"},
+    # verify_256x4, per-draft states: 555,026,944 read + 2,093,037,568 written
+    "verify_states": {"bytes": 2648064512, "source": "gdn_verify.cu",
+                      "sha256": "813090dfadf764cb421f435cc4489f27999477e790e4313a689feb6d7590babe"},
 }
 
 
@@ -526,6 +597,12 @@ def run_b200(args):
                "bytes_per_step": bytes_step, "gpu_launches": wd.T, "clocks": dclocks,
                "l2": "state 537 MB per step, larger than L2"}
 
+    # ---- the fused input prologue: the same prefill and decode on raw projections ----
+    pro = None
+    if not args.no_prologue and n_steps:
+        pro = measure_prologue(gdn, torch, dev, stream, x, w, ws, o, hT, rank, barrier,
+                               max_over_ranks, mean_launch_s, args)
+
     ver = None
     if not args.no_verify:
         ver = measure_verify(gdn, torch, dev, stream, peaks, peak_src, rank, world,
@@ -549,7 +626,7 @@ def run_b200(args):
                        "l2": "inputs larger than L2 (q,k,v 1.07 GB per step)"},
             "roofline": roof, "cpu_baseline": base, "e2e": e2e,
             "gpu_launches": launches_per_step * n_steps, "clocks": clocks, "decode": dec,
-            "verify": ver,
+            "verify": ver, "prologue": pro,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -568,6 +645,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-verify", action="store_true")
+    ap.add_argument("--no-prologue", action="store_true")
     ap.add_argument("--verify-rounds", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="decode measurement only")
