@@ -296,6 +296,10 @@ GDN_API gdn_status gdn_recurrent_step_ex(const void *q, const void *k, const voi
  *   g, beta [N][K][HV] fp32          state [N][HV][dv][dk] fp32 (read)
  *   states_out [N][K][HV][dv][dk] fp32   u_out [N][K][HV][dv] fp32
  * prologue: GDN_PROLOGUE_* flags applied to every draft (0 = prepared inputs).
+ * workspace: device scratch of at least gdn_recurrent_verify_workspace_size()
+ * bytes, 16-byte aligned, needed when states_out is NULL (the update-vector
+ * form builds per (sequence, value head) tables there; ignored otherwise, may
+ * be NULL); missing or too small returns GDN_ERR_WORKSPACE.
  * Supported: as gdn_recurrent_step, and 1 <= K <= GDN_VERIFY_MAX_DRAFTS.
  * Alignment: q, k, v, o, state, states_out 16-byte aligned, u_out 4-byte.
  * No output may overlap an input.  K > GDN_VERIFY_MAX_DRAFTS returns
@@ -306,7 +310,15 @@ GDN_API gdn_status gdn_recurrent_verify(const void *q, const void *k, const void
                                         const float *g, const float *beta, const float *state,
                                         int N, int K, int HK, int HV, int dk, int dv, float scale,
                                         gdn_dtype dtype, void *o, float *states_out, float *u_out,
-                                        unsigned prologue, gdn_stream_t stream);
+                                        unsigned prologue, void *workspace,
+                                        size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * Bytes of device workspace gdn_recurrent_verify needs when states_out is NULL:
+ * (2 K dk + 2 K^2) fp32 words per (sequence, value head), rounded up to 16
+ * bytes.  0 for invalid sizes.  Pure host query.
+ */
+GDN_API size_t gdn_recurrent_verify_workspace_size(int N, int K, int HV, int dk);
 
 /*
  * Keeps the accepted drafts after gdn_recurrent_verify (states_out form): for

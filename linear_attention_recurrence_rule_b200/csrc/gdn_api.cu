@@ -273,7 +273,7 @@ gdn_status gdn_recurrent_verify(const void *q, const void *k, const void *v, con
                                 const float *beta, const float *state, int N, int K, int HK, int HV,
                                 int dk, int dv, float scale, gdn_dtype dtype, void *o,
                                 float *states_out, float *u_out, unsigned prologue,
-                                gdn_stream_t stream) {
+                                void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
     if (prologue & ~GDN_PROLOGUE_ALL) return GDN_ERR_INVALID_ARG;
     if (N < 0 || K <= 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK)
         return GDN_ERR_INVALID_ARG;
@@ -285,10 +285,21 @@ gdn_status gdn_recurrent_verify(const void *q, const void *k, const void *v, con
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
         !aligned16(states_out) || !aligned4(u_out))
         return GDN_ERR_ALIGNMENT;
+    if (!states_out) {   // update-vector form: tables in the workspace
+        if (!workspace ||
+            workspace_bytes < gdn::verify_workspace_floats(N, K, HV, dk) * sizeof(float))
+            return GDN_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
+    }
     gdn::VerifyArgs a{q, k, v, g, beta, state, states_out, u_out, N, K, HK, HV, dk, dv, scale,
-                      dtype, o, prologue};
+                      dtype, o, prologue, workspace, workspace_bytes};
     const cudaError_t err = gdn::launch_verify(a, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+size_t gdn_recurrent_verify_workspace_size(int N, int K, int HV, int dk) {
+    if (N < 0 || K <= 0 || K > GDN_VERIFY_MAX_DRAFTS || HV <= 0 || dk <= 0) return 0;
+    return gdn::verify_workspace_floats(N, K, HV, dk) * sizeof(float);
 }
 
 gdn_status gdn_state_commit(const float *states, const int32_t *accepted, float *state, int N, int K,

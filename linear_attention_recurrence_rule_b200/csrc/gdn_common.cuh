@@ -32,6 +32,19 @@ __device__ __forceinline__ float dot4(float4 a, float4 b) {
     return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
 }
 
+// d = a * b + c on two fp32 lanes at once (sm_100 packed FMA), each lane rounded
+// as a scalar fmaf
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    unsigned long long ua, ub, uc, ud;
+    memcpy(&ua, &a, 8);
+    memcpy(&ub, &b, 8);
+    memcpy(&uc, &c, 8);
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(ud) : "l"(ua), "l"(ub), "l"(uc));
+    float2 d;
+    memcpy(&d, &ud, 8);
+    return d;
+}
+
 __device__ __forceinline__ float4 scale4(float4 a, float s) {
     return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
 }

@@ -46,7 +46,12 @@ struct VerifyArgs {
     gdn_dtype dtype;
     void *o;
     unsigned prologue = 0;
+    void *workspace = nullptr;   // update-vector form: per (sequence, value head) tables
+    size_t workspace_bytes = 0;
 };
+
+// fp32 words of the update-vector form's workspace (gdn_verify.cu)
+size_t verify_workspace_floats(int N, int K, int HV, int dk);
 
 
 // decode (gdn_decode.cu)

@@ -12,12 +12,20 @@
 //     u_i  = beta_t (v_i - alpha_t S_i . k_t)
 //     S_i <- alpha_t S_i + u_i k_t             o_i = scale * S_i(new) . q_t
 //
-// All kernels are single streaming passes over fp32 state bands of one
-// (sequence, value head): CTAs of 8 warps, rows of dk fp32 held by dk/16 lanes
-// with four float4 each (lane l of a row owns float4 l, l + dk/16, ..., so a
-// warp instruction reads whole 128-byte lines), two rows per lane.
+// Kernels: single streaming passes over fp32 state bands (64 rows at dk = 128,
+// 32 KB) of one (sequence, value head), CTAs of 8 warps, rows of dk fp32 held by
+// dk/16 lanes with four float4 each (lane l of a row owns float4 l, l + dk/16,
+// ..., so a warp instruction reads whole 128-byte lines), two rows per lane:
+//   verify_kernel          per-draft states asked for: the band stays in
+//                          registers from draft to draft
+//   verify_setup_kernel +  update vectors only: per-head tables, then a
+//   verify_wy_kernel       persistent pass fed by bulk copies through a ring of
+//                          shared-memory stages (the state is only read)
+//   commit_kernel          copy of the state after the last kept draft
+//   commit_deltas_kernel   in-place rebuild from S_0 and the kept u_t
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
+#include "tc_primitives.cuh"
 
 namespace gdn {
 namespace {
@@ -56,6 +64,16 @@ __device__ __forceinline__ void normalize_rows(float4 (*rows)[DK / 4], int nrows
         const float r = inv_l2norm(ss);
         for (int j = lane; j < DK / 4; j += 32) rows[t][j] = scale4(rows[t][j], r);
     }
+}
+
+template <int DK>
+__device__ __forceinline__ void normalize_row(float4 *row, int lane) {
+    float ss = 0.f;
+    for (int j = lane; j < DK / 4; j += 32) ss += dot4(row[j], row[j]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float r = inv_l2norm(ss);
+    for (int j = lane; j < DK / 4; j += 32) row[j] = scale4(row[j], r);
 }
 
 template <int DK>
@@ -181,140 +199,392 @@ verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 // Verify without the per-draft states (u_out form): the input state S_0 is never
 // updated.  Unrolling S_t = alpha_t S_{t-1} + u_t k_t^T over the drafts (the chunk
 // form of the rule restricted to K tokens), for one row r of the state,
-//   S_{t-1}[r] . k_t = gamma_{t-1} a_t + sum_{j<t}  G(j,t-1) (k_j . k_t) u_j[r]
-//   S_t[r]     . q_t = gamma_t     b_t + sum_{j<=t} G(j,t)   (k_j . q_t) u_j[r]
-// with a_t = S_0[r] . k_t, b_t = S_0[r] . q_t, gamma_t = prod_{s<=t} alpha_s and
-// G(j,t) = prod_{j<s<=t} alpha_s.  So a lane computes the 2K dot products of its
-// rows against S_0 (independent of each other), then a K-step recurrence on
-// per-row scalars whose coefficients (the K x K Gram products k_j . k_t and
-// k_j . q_t times the decays, times beta and scale) are tabled once per CTA.
-// KT is the compile-time bound on K (4, 8 or 16).
+//   u_t = beta_t v_t - a1_t a_t - sum_{j<t} ck_tj u_j,     a_t = S_0[r] . k_t
+//   o_t = b1_t b_t + sum_{j<=t} cq_tj u_j,                 b_t = S_0[r] . q_t
+// with a1_t = beta_t alpha_t gamma_{t-1}, ck_tj = beta_t alpha_t G(j,t-1) (k_j . k_t),
+// b1_t = scale gamma_t, cq_tj = scale G(j,t) (k_j . q_t), gamma_t = prod_{s<=t} alpha_s
+// and G(j,t) = prod_{j<s<=t} alpha_s.  The recurrence is linear: with
+// M = (I + Ck)^-1 (unit lower triangular, K x K),
+//   u = M diag(beta) v - M diag(a1) a,      o = diag(b1) b + Cq u,
+// and a, b are themselves linear in the row S_0[r].  So every output of a row is
+// one dot product of S_0[r] with a vector mixed once per (sequence, value head):
+//   u_t = S_0[r] . k'_t + sum_j Vu_tj v_j[r],   k'_t = -sum_j M_tj a1_j k_j,    Vu = M diag(beta)
+//   o_t = S_0[r] . q'_t + sum_j Vy_tj v_j[r],   q'_t = b1_t q_t + sum_j E_tj k_j,
+//                                               E = -Cq M diag(a1),            Vy = Cq Vu.
+// verify_setup_kernel builds k', q', Vu, Vy per (sequence, value head) into a
+// workspace (one small CTA each, many resident per SM, so their serial K-step
+// loops overlap); verify_wy_kernel streams the state bands and does 2K plain dot
+// products per row.
+
+// workspace: a 16-byte header (word 0: status of the streaming kernel's bounded
+// waits, 0 = ok), then per (sequence, value head) k', q' [K][dk], Vu, Vy [K][K],
+// rounded up to 16 bytes
+constexpr int kWsHeaderFloats = 4;
+__host__ __device__ inline size_t wy_item_floats(int K, int dk) {
+    return ((size_t)2 * K * dk + 2 * (size_t)K * K + 3) & ~(size_t)3;
+}
+
+// one warp per (sequence, value head); a CTA holds a few such warps, each with
+// its own shared-memory slice, and only warp-level syncs
+template <int KT>
+__host__ __device__ constexpr int setup_warps() { return KT <= 8 ? 4 : 2; }
+
+template <int DK, int KT>
+struct SetupSlice {
+    float4 ks[KT][DK / 4], qs[KT][DK / 4];
+    float al[KT], be[KT], a1[KT], b1[KT];
+    float gkk[KT][KT], gkq[KT][KT], ck[KT][KT], cq[KT][KT], Mi[KT][KT], Dm[KT][KT], Em[KT][KT];
+};
+
 template <int DK, int KT, typename Tin, bool PRO>
-__global__ void __launch_bounds__(kVerifyWarps * 32, KT <= 4 ? 3 : 2)
-verify_wy_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
-                 const float *__restrict__ g, const float *__restrict__ beta,
-                 const float *__restrict__ state, float *__restrict__ u_out, Tin *__restrict__ o,
-                 int K, int HK, int HV, int dv, float scale, unsigned pro_arg) {
+__global__ void __launch_bounds__(setup_warps<KT>() * 32)
+verify_setup_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+                    const float *__restrict__ g, const float *__restrict__ beta,
+                    float *__restrict__ ws, int items, int K, int HK, int HV, float scale,
+                    unsigned pro_arg) {
     const unsigned pro = PRO ? pro_arg : 0u;
-    constexpr int LPR = DK / (4 * kVerifyF4);
-    constexpr int RPW = 32 / LPR;
-    constexpr int BAND = verify_band<DK>();
-    __shared__ float4 ks[KT][DK / 4], qs[KT][DK / 4];
-    __shared__ float vs[KT][BAND];
-    __shared__ float al[KT], be[KT];
-    __shared__ float gram[2][KT][KT];      // [0][j][t] = k_j . k_t, [1][j][t] = k_j . q_t
-    __shared__ float ck[KT][KT], cq[KT][KT], a1[KT], b1[KT];
-    const int nh = blockIdx.x;
+    constexpr int D4 = DK / 4;
+    __shared__ SetupSlice<DK, KT> slices[setup_warps<KT>()];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nh = blockIdx.x * setup_warps<KT>() + warp;
+    if (nh >= items) return;   // whole warps only; nothing below syncs the block
+    SetupSlice<DK, KT> &S = slices[warp];
     const int n = nh / HV, h = nh - n * HV;
     const int c = h / (HV / HK);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int sub = lane / LPR, li = lane % LPR;
-    const int base = blockIdx.y * BAND;
-    float4 s[kVerifyRows][kVerifyF4];
-    const float *S = state + (size_t)nh * dv * DK;
-#pragma unroll
-    for (int jr = 0; jr < kVerifyRows; ++jr) {
-        const int row = base + (jr * kVerifyWarps + warp) * RPW + sub;
-#pragma unroll
-        for (int i = 0; i < kVerifyF4; ++i)
-            s[jr][i] = row < dv ? __ldcs(reinterpret_cast<const float4 *>(S + (size_t)row * DK) +
-                                         li + LPR * i)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    for (int idx = threadIdx.x; idx < K * (DK / 4); idx += blockDim.x) {
-        const int t = idx / (DK / 4), j = idx - t * (DK / 4);
+    for (int idx = lane; idx < K * D4; idx += 32) {
+        const int t = idx / D4, j = idx - t * D4;
         const size_t off = (((size_t)n * K + t) * HK + c) * DK + 4 * j;
-        ks[t][j] = load4(k + off);
-        qs[t][j] = load4(q + off);
+        S.ks[t][j] = load4(k + off);
+        S.qs[t][j] = load4(q + off);
     }
-    for (int idx = threadIdx.x; idx < K * BAND; idx += blockDim.x) {
-        const int t = idx / BAND, r = idx - t * BAND;
-        const int row = base + r;
-        vs[t][r] = row < dv ? to_f32(v[(((size_t)n * K + t) * HV + h) * dv + row]) : 0.f;
+    if (lane < K) {
+        const size_t gi = ((size_t)n * K + lane) * HV + h;
+        S.al[lane] = gate_alpha(g[gi], pro);
+        S.be[lane] = gate_beta(beta[gi], pro);
     }
-    if (threadIdx.x < K) {
-        const size_t gi = ((size_t)n * K + threadIdx.x) * HV + h;
-        al[threadIdx.x] = gate_alpha(g[gi], pro);
-        be[threadIdx.x] = gate_beta(beta[gi], pro);
-    }
-    __syncthreads();
-    if (pro & (GDN_PROLOGUE_NORM_Q | GDN_PROLOGUE_NORM_K)) {
-        prologue_qk<DK>(ks, qs, K, pro, warp, lane);
-        __syncthreads();
-    }
-    // Gram products, one warp per pair
-    for (int p = warp; p < 2 * K * K; p += kVerifyWarps) {
+    __syncwarp();
+    if (pro & GDN_PROLOGUE_NORM_K)
+        for (int t = 0; t < K; ++t) normalize_row<DK>(S.ks[t], lane);
+    if (pro & GDN_PROLOGUE_NORM_Q)
+        for (int t = 0; t < K; ++t) normalize_row<DK>(S.qs[t], lane);
+    __syncwarp();
+    // Gram products: one lane per entry, each walking the columns from its own
+    // offset (rows of the same column would share a bank)
+    for (int p = lane; p < 2 * K * K; p += 32) {
         const int which = p / (K * K), rem = p - which * K * K;
         const int j = rem / K, t = rem - j * K;
+        const float4 *a = S.ks[j];
+        const float4 *b = which ? S.qs[t] : S.ks[t];
         float acc = 0.f;
-        for (int f = lane; f < DK / 4; f += 32) acc += dot4(ks[j][f], which ? qs[t][f] : ks[t][f]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) gram[which][j][t] = acc;
+#pragma unroll 8
+        for (int f = 0; f < D4; ++f) {
+            const int fs = (f + lane) & (D4 - 1);
+            acc += dot4(a[fs], b[fs]);
+        }
+        (which ? S.gkq : S.gkk)[j][t] = acc;
     }
-    __syncthreads();
-    if (threadIdx.x < K) {
-        const int t = threadIdx.x;
-        // u_t = beta_t v_t - a1[t] a_t - sum_{j<t} ck[t][j] u_j
+    __syncwarp();
+    if (lane < K) {   // recurrence coefficients, one lane per draft
+        const int t = lane;
         float G = 1.f;   // G(j, t-1), walking j down from t-1
         for (int j = t - 1; j >= 0; --j) {
-            ck[t][j] = be[t] * al[t] * G * gram[0][j][t];
-            G *= al[j];
+            S.ck[t][j] = S.be[t] * S.al[t] * G * S.gkk[j][t];
+            G *= S.al[j];
         }
-        a1[t] = be[t] * al[t] * G;   // G is now gamma_{t-1}
-        // o_t = b1[t] b_t + sum_{j<=t} cq[t][j] u_j
+        S.a1[t] = S.be[t] * S.al[t] * G;   // G is now gamma_{t-1}
         float H = 1.f;   // G(j, t)
         for (int j = t; j >= 0; --j) {
-            cq[t][j] = scale * H * gram[1][j][t];
-            H *= al[j];
+            S.cq[t][j] = scale * H * S.gkq[j][t];
+            H *= S.al[j];
         }
-        b1[t] = scale * H;           // scale * gamma_t
+        S.b1[t] = scale * H;               // scale * gamma_t
+    }
+    __syncwarp();
+    if (lane < K) {   // M = (I + Ck)^-1 by forward substitution, one lane per column
+        const int col = lane;
+        for (int t = 0; t < K; ++t) {
+            float m = (t == col) ? 1.f : 0.f;
+            for (int j = col; j < t; ++j) m = fmaf(-S.ck[t][j], S.Mi[j][col], m);
+            S.Mi[t][col] = t >= col ? m : 0.f;
+        }
+    }
+    __syncwarp();
+    float *out = ws + kWsHeaderFloats + (size_t)nh * wy_item_floats(K, DK);
+    float *vu_out = out + 2 * (size_t)K * DK, *vy_out = vu_out + (size_t)K * K;
+    for (int e = lane; e < K * K; e += 32) {   // D = -M diag(a1), Vu = M diag(beta)
+        const int t = e / K, j = e - t * K;
+        S.Dm[t][j] = -S.Mi[t][j] * S.a1[j];
+        vu_out[e] = S.Mi[t][j] * S.be[j];
+    }
+    __syncwarp();
+    for (int e = lane; e < K * K; e += 32) {   // E = Cq D, Vy = Cq Vu
+        const int t = e / K, i = e - t * K;
+        float ev = 0.f, vv = 0.f;
+        for (int j = i; j <= t; ++j) {
+            ev = fmaf(S.cq[t][j], S.Dm[j][i], ev);
+            vv = fmaf(S.cq[t][j], S.Mi[j][i] * S.be[i], vv);
+        }
+        S.Em[t][i] = ev;
+        vy_out[e] = vv;
+    }
+    __syncwarp();
+    float4 *kp = reinterpret_cast<float4 *>(out), *qp = kp + (size_t)K * D4;
+    for (int idx = lane; idx < K * D4; idx += 32) {   // mixed key and query vectors
+        const int t = idx / D4, f = idx - t * D4;
+        float4 kk = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 qq = scale4(S.qs[t][f], S.b1[t]);
+        for (int j = 0; j <= t; ++j) {
+            const float4 kj = S.ks[j][f];
+            const float d = S.Dm[t][j], e = S.Em[t][j];
+            kk.x = fmaf(d, kj.x, kk.x); kk.y = fmaf(d, kj.y, kk.y);
+            kk.z = fmaf(d, kj.z, kk.z); kk.w = fmaf(d, kj.w, kk.w);
+            qq.x = fmaf(e, kj.x, qq.x); qq.y = fmaf(e, kj.y, qq.y);
+            qq.z = fmaf(e, kj.z, qq.z); qq.w = fmaf(e, kj.w, qq.w);
+        }
+        kp[idx] = kk;
+        qp[idx] = qq;
+    }
+}
+
+// Streaming kernel, persistent: each CTA walks bands b = blockIdx.x + i * gridDim.x
+// of the (sequence, value head, band) list.  Thread 0 keeps NST bands in flight:
+// every band's 32 KB of state rows (contiguous) and its head's tables arrive by
+// 1-D bulk copies into a ring of shared-memory stages, completing on the stage's
+// mbarrier, so the state stream does not stop while the CTA computes.  Per band:
+// 2K dot products per row against S_0, a reduce-scatter over the row's lanes (a
+// lane keeps the upper half of its values where its lane bit is set, the lower
+// half otherwise) and the outputs the lane ends up holding.  One block barrier per
+// band, which also frees the previous band's stage for the next copy.  Waits are
+// bounded: a timeout sets the workspace status word, and the CTA drains its copies
+// in flight (bounded) before it returns.
+constexpr uint32_t kWyWaitLimit = 2000;   // ~2 s of 1 ms sleeping polls
+
+template <int KT>
+__host__ __device__ constexpr int wy_stages() { return KT <= 4 ? 3 : 2; }
+template <int DK, int KT>
+__host__ __device__ constexpr size_t wy_stage_bytes() {
+    return (size_t)verify_band<DK>() * DK * sizeof(float) +
+           ((2 * (size_t)KT * DK + 2 * (size_t)KT * KT + 3) & ~(size_t)3) * sizeof(float);
+}
+template <int DK, int KT>
+__host__ __device__ constexpr size_t wy_smem_bytes() {
+    // stages, the two v buffers [2][KT][BAND] fp32, the stage mbarriers
+    return wy_stages<KT>() * wy_stage_bytes<DK, KT>() +
+           2 * (size_t)KT * verify_band<DK>() * sizeof(float) +
+           wy_stages<KT>() * sizeof(uint64_t) + 16;
+}
+
+template <int DK, int KT, typename Tin>
+__global__ void __launch_bounds__(kVerifyWarps * 32, KT <= 8 ? 2 : 1)
+verify_wy_kernel(const Tin *__restrict__ v, const float *__restrict__ state, float *__restrict__ ws,
+                 float *__restrict__ u_out, Tin *__restrict__ o, int N, int K, int HV, int dv) {
+    constexpr int LPR = DK / (4 * kVerifyF4);   // lanes per row: 2, 4, 8
+    constexpr int RPW = 32 / LPR;
+    constexpr int BAND = verify_band<DK>();
+    constexpr int D4 = DK / 4;
+    constexpr int NV = 2 * KT;                  // partial sums per row: u then o
+    static_assert(NV % LPR == 0, "reduce-scatter needs 2 KT >= lanes per row");
+    constexpr int NL = NV / LPR;                // finished values per lane
+    constexpr int NST = wy_stages<KT>();
+    constexpr size_t SB = wy_stage_bytes<DK, KT>();
+    extern __shared__ __align__(128) uint8_t wy_smem[];
+    // v of a band, loaded one band ahead (plain loads into registers during the
+    // previous band's arithmetic, stored here after it)
+    float *vsm = reinterpret_cast<float *>(wy_smem + NST * SB);   // [2][KT][BAND]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(vsm + 2 * KT * BAND);
+    constexpr int VPT = (KT * BAND + kVerifyWarps * 32 - 1) / (kVerifyWarps * 32);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sub = lane / LPR, li = lane % LPR;
+    const int nbands = (dv + BAND - 1) / BAND;
+    const long long total = (long long)N * HV * nbands;
+    const long long mine = total > blockIdx.x ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const size_t item_floats = wy_item_floats(K, DK);
+    const float *tables = ws + kWsHeaderFloats;
+
+    // (value-head index, band) of this CTA's i-th band, b = blockIdx.x + i * gridDim.x,
+    // advanced by the grid stride without a division per band
+    struct BandIt {
+        int nh, y;
+        __device__ void init(long long b, int nb) {
+            nh = (int)(b / nb);
+            y = (int)(b - (long long)nh * nb);
+        }
+        __device__ void next(int step_nh, int step_y, int nb) {
+            nh += step_nh;
+            y += step_y;
+            if (y >= nb) {
+                y -= nb;
+                ++nh;
+            }
+        }
+    };
+    const int step_nh = (int)(gridDim.x / nbands), step_y = (int)(gridDim.x % nbands);
+    auto band_rows = [&](int y) { return dv - y * BAND < BAND ? dv - y * BAND : BAND; };
+    BandIt it_issue;   // thread 0: the next band to copy in
+    it_issue.init(blockIdx.x, nbands);
+    auto issue = [&](long long i) {   // thread 0: band i of this CTA into stage i % NST
+        const int nh = it_issue.nh, base = it_issue.y * BAND, rows = band_rows(it_issue.y);
+        it_issue.next(step_nh, step_y, nbands);
+        uint8_t *stg = wy_smem + (i % NST) * SB;
+        uint64_t *bar = &bars[i % NST];
+        const uint32_t sbytes = (uint32_t)rows * DK * sizeof(float);
+        const uint32_t tbytes = (uint32_t)(item_floats * sizeof(float));
+        tc::mbar_arrive_expect_tx(bar, sbytes + tbytes);
+        tc::bulk_load_g2s(stg, state + ((size_t)nh * dv + base) * DK, sbytes, bar);
+        tc::bulk_load_g2s(stg + (size_t)BAND * DK * sizeof(float), tables + (size_t)nh * item_floats,
+                          tbytes, bar);
+    };
+    BandIt it_v;   // the band whose v is loaded next
+    it_v.init(blockIdx.x, nbands);
+    auto load_v = [&](float (&vr)[VPT]) {   // v of band it_v, then advance it
+        const int nh = it_v.nh, base = it_v.y * BAND, rows = band_rows(it_v.y);
+        it_v.next(step_nh, step_y, nbands);
+        const int n = nh / HV, h = nh - n * HV;
+#pragma unroll
+        for (int e0 = 0; e0 < VPT; ++e0) {
+            const int e = tid + e0 * kVerifyWarps * 32;
+            const int j = e / BAND, r = e - j * BAND;
+            vr[e0] = (j < K && r < rows) ? to_f32(v[(((size_t)n * K + j) * HV + h) * dv + base + r])
+                                         : 0.f;
+        }
+    };
+    auto store_v = [&](long long i, const float (&vr)[VPT]) {
+        float *dst = vsm + (i & 1) * KT * BAND;
+#pragma unroll
+        for (int e0 = 0; e0 < VPT; ++e0) {
+            const int e = tid + e0 * kVerifyWarps * 32;
+            if (e < KT * BAND) dst[e] = vr[e0];
+        }
+    };
+    if (tid == 0) {
+        for (int st = 0; st < NST; ++st) tc::mbar_init(&bars[st], 1);
+        tc::fence_barrier_init();
+        for (long long i = 0; i < NST && i < mine; ++i) issue(i);
+    }
+    if (mine > 0) {
+        float vr[VPT];
+        load_v(vr);
+        store_v(0, vr);
     }
     __syncthreads();
-    float uh[kVerifyRows][KT];
-#pragma unroll
-    for (int t = 0; t < KT; ++t) {
-        if (t >= K) break;
-        float a[kVerifyRows], b[kVerifyRows];
-#pragma unroll
-        for (int jr = 0; jr < kVerifyRows; ++jr) {
-            a[jr] = 0.f;
-            b[jr] = 0.f;
+    BandIt it;   // the band being computed
+    it.init(blockIdx.x, nbands);
+    long long issued = mine < NST ? mine : NST, done = 0;
+    bool ok = true;
+    for (long long i = 0; i < mine; ++i) {
+        const int st = (int)(i % NST);
+        bool landed = tc::mbar_wait(&bars[st], (uint32_t)((i / NST) & 1), kWyWaitLimit);
+        ok = __syncthreads_and(landed);   // also: every thread is done with band i - 1
+        if (!ok) break;
+        done = i + 1;
+        if (tid == 0 && i >= 1 && i - 1 + NST < mine) {   // band i - 1's stage is free again
+            issue(i - 1 + NST);
+            ++issued;
         }
-#pragma unroll
-        for (int i = 0; i < kVerifyF4; ++i) {
-            const float4 kk = ks[t][li + LPR * i], qq = qs[t][li + LPR * i];
-#pragma unroll
-            for (int jr = 0; jr < kVerifyRows; ++jr) {
-                a[jr] += dot4(s[jr][i], kk);
-                b[jr] += dot4(s[jr][i], qq);
-            }
-        }
-#pragma unroll
-        for (int off = LPR / 2; off > 0; off >>= 1) {
-#pragma unroll
-            for (int jr = 0; jr < kVerifyRows; ++jr) {
-                a[jr] += __shfl_xor_sync(0xffffffffu, a[jr], off);
-                b[jr] += __shfl_xor_sync(0xffffffffu, b[jr], off);
-            }
-        }
-        const size_t nt = (size_t)n * K + t;
+        float vnext[VPT];
+        if (i + 1 < mine) load_v(vnext);   // band i + 1: lands during this band's arithmetic
+        const int nh = it.nh, base = it.y * BAND, rows = band_rows(it.y);
+        it.next(step_nh, step_y, nbands);
+        const int n = nh / HV, h = nh - n * HV;
+        const float *vb = vsm + (i & 1) * KT * BAND;   // [j][r] of this band
+        const uint8_t *stg = wy_smem + st * SB;
+        const float4 *srow = reinterpret_cast<const float4 *>(stg);
+        const float *item = reinterpret_cast<const float *>(stg + (size_t)BAND * DK * sizeof(float));
+        const float4 *kp = reinterpret_cast<const float4 *>(item);
+        const float4 *qp = kp + (size_t)K * D4;
+        const float *vu = item + 2 * (size_t)K * DK, *vy = vu + (size_t)K * K;
+        float4 s[kVerifyRows][kVerifyF4];
 #pragma unroll
         for (int jr = 0; jr < kVerifyRows; ++jr) {
             const int r = (jr * kVerifyWarps + warp) * RPW + sub;
-            float x = be[t] * vs[t][r] - a1[t] * a[jr];
 #pragma unroll
-            for (int j = 0; j < t; ++j) x = fmaf(-ck[t][j], uh[jr][j], x);
-            uh[jr][t] = x;
-            float y = b1[t] * b[jr];
+            for (int q4 = 0; q4 < kVerifyF4; ++q4) s[jr][q4] = srow[r * D4 + li + LPR * q4];
+        }
+        // dot products on packed pairs (even / odd columns), summed once at the end
+        float2 acc2[kVerifyRows][NV];
 #pragma unroll
-            for (int j = 0; j <= t; ++j) y = fmaf(cq[t][j], uh[jr][j], y);
-            const int row = base + r;
-            if (row < dv && li == 0) {
-                o[(nt * HV + h) * dv + row] = from_f32<Tin>(y);
-                if (u_out) u_out[(nt * HV + h) * dv + row] = x;
+        for (int jr = 0; jr < kVerifyRows; ++jr)
+#pragma unroll
+            for (int m = 0; m < NV; ++m) acc2[jr][m] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < KT; ++t) {
+            if (t < K) {
+#pragma unroll
+                for (int q4 = 0; q4 < kVerifyF4; ++q4) {
+                    const float4 kv = kp[t * D4 + li + LPR * q4], qv = qp[t * D4 + li + LPR * q4];
+                    const float2 klo = make_float2(kv.x, kv.y), khi = make_float2(kv.z, kv.w);
+                    const float2 qlo = make_float2(qv.x, qv.y), qhi = make_float2(qv.z, qv.w);
+#pragma unroll
+                    for (int jr = 0; jr < kVerifyRows; ++jr) {
+                        const float4 x = s[jr][q4];
+                        const float2 xlo = make_float2(x.x, x.y), xhi = make_float2(x.z, x.w);
+                        acc2[jr][t] = fma2(xhi, khi, fma2(xlo, klo, acc2[jr][t]));
+                        acc2[jr][KT + t] = fma2(xhi, qhi, fma2(xlo, qlo, acc2[jr][KT + t]));
+                    }
+                }
             }
         }
+        float acc[kVerifyRows][NV];
+#pragma unroll
+        for (int jr = 0; jr < kVerifyRows; ++jr)
+#pragma unroll
+            for (int m = 0; m < NV; ++m) acc[jr][m] = acc2[jr][m].x + acc2[jr][m].y;
+#pragma unroll
+        for (int jr = 0; jr < kVerifyRows; ++jr) {
+            int n_cur = NV;
+#pragma unroll
+            for (int off = LPR / 2; off > 0; off >>= 1) {
+                const bool upper = (li & off) != 0;
+                const int half = n_cur / 2;
+#pragma unroll
+                for (int m = 0; m < NV / 2; ++m) {
+                    if (m < half) {
+                        const float keep = upper ? acc[jr][m + half] : acc[jr][m];
+                        const float send = upper ? acc[jr][m] : acc[jr][m + half];
+                        acc[jr][m] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                    }
+                }
+                n_cur = half;
+            }
+        }
+        int first = 0;   // index of this lane's first finished value
+        {
+            int half = NV / 2;
+#pragma unroll
+            for (int off = LPR / 2; off > 0; off >>= 1) {
+                if (li & off) first += half;
+                half /= 2;
+            }
+        }
+#pragma unroll
+        for (int jr = 0; jr < kVerifyRows; ++jr) {
+            const int r = (jr * kVerifyWarps + warp) * RPW + sub;
+            if (r >= rows) continue;
+            const int row = base + r;
+#pragma unroll
+            for (int m = 0; m < NL; ++m) {
+                const int idx = first + m;
+                const bool is_u = idx < KT;
+                const int t = is_u ? idx : idx - KT;
+                if (t >= K || (is_u && !u_out)) continue;
+                const float *coef = (is_u ? vu : vy) + t * K;
+                float val = acc[jr][m];
+                for (int j = 0; j <= t; ++j) val = fmaf(coef[j], vb[j * BAND + r], val);
+                const size_t ot = (((size_t)n * K + t) * HV + h) * dv + row;
+                if (is_u)
+                    u_out[ot] = val;
+                else
+                    o[ot] = from_f32<Tin>(val);
+            }
+        }
+        if (i + 1 < mine) store_v(i + 1, vnext);   // published by the next band's barrier
+    }
+    if (!ok && tid == 0) {
+        atomicExch(reinterpret_cast<unsigned int *>(ws), 1u);
+        // copies still in flight land before this CTA's shared memory is released
+        for (long long i = done; i < issued; ++i)
+            tc::mbar_wait(&bars[i % NST], (uint32_t)((i / NST) & 1), kWyWaitLimit);
     }
 }
 
@@ -428,13 +698,47 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
     }
 }
 
+int device_sm_count() {
+    static int count = 0;
+    if (count == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            count = 148;
+    }
+    return count;
+}
+
 template <int DK, int KT, typename Tin>
-void launch_verify_wy(const VerifyArgs &a, dim3 grid, dim3 block, cudaStream_t stream) {
-    auto kern = a.prologue ? verify_wy_kernel<DK, KT, Tin, true> : verify_wy_kernel<DK, KT, Tin, false>;
-    kern<<<grid, block, 0, stream>>>(
-        static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
-        static_cast<const Tin *>(a.v), a.g, a.beta, a.state, a.u, static_cast<Tin *>(a.o), a.K,
-        a.HK, a.HV, a.dv, a.scale, a.prologue);
+void launch_verify_wy(const VerifyArgs &a, dim3, dim3 block, cudaStream_t stream) {
+    auto setup = a.prologue ? verify_setup_kernel<DK, KT, Tin, true>
+                            : verify_setup_kernel<DK, KT, Tin, false>;
+    const int items = a.N * a.HV;
+    constexpr int W = setup_warps<KT>();
+    float *ws = static_cast<float *>(a.workspace);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), stream) != cudaSuccess) return;
+    setup<<<(unsigned)((items + W - 1) / W), W * 32, 0, stream>>>(
+        static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k), a.g, a.beta, ws, items, a.K,
+        a.HK, a.HV, a.scale, a.prologue);
+    auto kern = verify_wy_kernel<DK, KT, Tin>;
+    constexpr size_t smem = wy_smem_bytes<DK, KT>();
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return;   // the launch below reports the error
+        attr_set = true;
+    }
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kVerifyWarps * 32, smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const long long bands = (long long)items * ((a.dv + verify_band<DK>() - 1) / verify_band<DK>());
+    const long long slots = (long long)per_sm * device_sm_count();
+    const unsigned grid = (unsigned)(bands < slots ? bands : slots);
+    kern<<<grid, block, smem, stream>>>(static_cast<const Tin *>(a.v), a.state, ws, a.u,
+                                        static_cast<Tin *>(a.o), a.N, a.K, a.HV, a.dv);
 }
 
 template <int DK, typename Tin>
@@ -482,6 +786,10 @@ cudaError_t launch_verify_typed(const VerifyArgs &a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+size_t verify_workspace_floats(int N, int K, int HV, int dk) {
+    return kWsHeaderFloats + (size_t)N * HV * wy_item_floats(K, dk);
+}
 
 cudaError_t launch_verify(const VerifyArgs &a, cudaStream_t stream) {
     if (a.N == 0) return cudaSuccess;

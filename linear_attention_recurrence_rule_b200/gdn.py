@@ -70,7 +70,9 @@ def load_library() -> ctypes.CDLL:
             lib.gdn_recurrent_verify.restype = i32
             lib.gdn_recurrent_verify.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                                  i32, ctypes.c_float, i32, vp, vp, vp,
-                                                 ctypes.c_uint, vp]
+                                                 ctypes.c_uint, vp, sz, vp]
+            lib.gdn_recurrent_verify_workspace_size.restype = sz
+            lib.gdn_recurrent_verify_workspace_size.argtypes = [i32, i32, i32, i32]
             lib.gdn_state_commit.restype = i32
             lib.gdn_state_commit.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
             lib.gdn_state_commit_deltas.restype = i32
@@ -222,13 +224,16 @@ def gdn_recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, o=None, stre
 
 
 def gdn_recurrent_verify(q, k, v, g, beta, state, scale: float = 1.0, o=None, states_out=None,
-                         u_out=None, rollback="states", stream=None, prologue: int = 0):
+                         u_out=None, rollback="states", stream=None, prologue: int = 0,
+                         workspace=None):
     """K draft tokens per sequence through ``gdn_recurrent_verify``; ``state`` is only read.
 
     q, k [N,K,HK,dk]; v [N,K,HV,dv] (bf16 or fp32); g, beta [N,K,HV] fp32;
     state [N,HV,dv,dk] fp32.  ``rollback`` picks what is written for the
     commit: "states" (states_out [N,K,HV,dv,dk], the state after each draft),
     "deltas" (u_out [N,K,HV,dv], each draft's update vector), "both" or "none".
+    Without per-draft states the call needs a device ``workspace`` of
+    ``gdn_recurrent_verify_workspace_size`` bytes (allocated here if not given).
     Returns (o [N,K,HV,dv], states_out or None, u_out or None).
     """
     if rollback not in ("states", "deltas", "both", "none"):
@@ -268,13 +273,27 @@ def gdn_recurrent_verify(q, k, v, g, beta, state, scale: float = 1.0, o=None, st
             raise ValueError("expected u_out [N,K,HV,dv]")
     else:
         u_out = None
+    ws_bytes = 0
+    if states_out is None and N > 0:
+        need = int(lib.gdn_recurrent_verify_workspace_size(N, K, HV, dk))
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        _need(workspace, "workspace", None, dev)
+        ws_bytes = workspace.numel() * workspace.element_size()
     st = lib.gdn_recurrent_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
                                   N, K, HK, HV, dk, dv, float(scale), _dtype_code(q), _ptr(o),
                                   _ptr(states_out), _ptr(u_out), int(prologue),
+                                  _ptr(workspace) if states_out is None else None, ws_bytes,
                                   _stream_ptr(stream, dev))
     if st != GDN_OK:
         raise GDNError(st, "gdn_recurrent_verify")
     return o, states_out, u_out
+
+
+def gdn_recurrent_verify_workspace_size(N, K, HV, dk) -> int:
+    """Bytes of workspace ``gdn_recurrent_verify`` needs without per-draft states."""
+    return int(load_library().gdn_recurrent_verify_workspace_size(int(N), int(K), int(HV),
+                                                                  int(dk)))
 
 
 def gdn_state_commit(states, accepted, state, stream=None):

@@ -120,7 +120,8 @@ def verify_call(lib, **kw):
     return lib.gdn_recurrent_verify(a["q"], a["k"], a["v"], a["g"], a["beta"], a["state"],
                                     a["N"], a["K"], a["HK"], a["HV"], a["dk"], a["dv"],
                                     a["scale"], a["dtype"], a["o"], a["states"], a["u"],
-                                    a.get("pro", 0), None)
+                                    a.get("pro", 0), a.get("ws", None), a.get("ws_bytes", 0),
+                                    None)
 
 
 def test_verify_validation(lib):
@@ -132,6 +133,13 @@ def test_verify_validation(lib):
     assert verify_call(lib, states=fake(0x8008)) == gdn.GDN_ERR_ALIGNMENT
     assert verify_call(lib, u=fake(0x9002)) == gdn.GDN_ERR_ALIGNMENT
     assert verify_call(lib, N=0) == gdn.GDN_OK
+    # the update-vector form (no per-draft states) needs its workspace
+    need = lib.gdn_recurrent_verify_workspace_size(2, 4, 2, 128)
+    assert need == 16 + 2 * 2 * (2 * 4 * 128 + 2 * 16) * 4   # status word + tables
+    assert verify_call(lib, states=None) == gdn.GDN_ERR_WORKSPACE
+    assert verify_call(lib, states=None, ws=fake(0xa000), ws_bytes=need - 4) == gdn.GDN_ERR_WORKSPACE
+    assert verify_call(lib, states=None, ws=fake(0xa008), ws_bytes=need) == gdn.GDN_ERR_ALIGNMENT
+    assert lib.gdn_recurrent_verify_workspace_size(2, 17, 2, 128) == 0
 
 
 def test_commit_validation(lib):
