@@ -4,9 +4,10 @@ import numpy as np
 import pytest
 import torch
 
-from linear_attention_recurrence_rule_b200 import (GDNError, gdn_recurrent_step,
-                                                   gdn_recurrent_verify, gdn_state_commit,
-                                                   gdn_state_commit_deltas)
+from linear_attention_recurrence_rule_b200 import (GDNError, gdn_read_status, gdn_recurrent_step,
+                                                   gdn_recurrent_verify,
+                                                   gdn_recurrent_verify_workspace_size,
+                                                   gdn_state_commit, gdn_state_commit_deltas)
 from linear_attention_recurrence_rule_b200.inputs import make_verify
 from oracle import gdn_oracle as O
 from parity_util import assert_close, to_dev
@@ -106,9 +107,12 @@ def test_commit_keeps_accepted_prefix(dtype):
 def test_commit_deltas_matches_oracle(N, K, HK, HV, dk, dv, dtype):
     x = make_verify(N, K, HK, HV, dk, dv, dtype, seed=17 + K, h0_std=0.5)
     d = to_dev(x)
+    ws = torch.empty(gdn_recurrent_verify_workspace_size(N, K, HV, dk), dtype=torch.uint8,
+                     device="cuda")
     _, states_none, u = gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"], d["beta"],
-                                             d["state"], rollback="deltas")
+                                             d["state"], rollback="deltas", workspace=ws)
     assert states_none is None
+    assert gdn_read_status(ws) == 0   # every bounded wait of the streaming kernel completed
     accepted = (torch.arange(N, dtype=torch.int32) % (K + 1))
     S = d["state"].clone()
     gdn_state_commit_deltas(d["k"], d["g"], u, accepted.cuda(), S)
@@ -150,6 +154,10 @@ def test_verify_empty_and_errors():
     with pytest.raises(ValueError):
         gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"][:, :2].contiguous(), d["beta"],
                              d["state"])
+    with pytest.raises(GDNError):   # update-vector form with a too small workspace
+        gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                             rollback="deltas",
+                             workspace=torch.empty(64, dtype=torch.uint8, device="cuda"))
     big = make_verify(1, 17, 1, 2, 32, 32, torch.float32, seed=2)
     b = to_dev(big)
     with pytest.raises(GDNError):
