@@ -266,12 +266,13 @@ NCU_TRAFFIC = {
     # full long_prefill_64k launch: 1,090,729,728 read + 510,220,032 written
     "prefill_cluster": {"bytes": 1600949760, "source": "gdn_prefill_cluster.cu",
                         "sha256": "881a325e6d56777fe19db569636ec05bdd86d18a1d8dea300fed5c5991d89ae0"},
-    # verify_256x4, update-vector form: 553,954,304 read + 4,621,312 written
-    "verify_deltas": {"bytes": 558575616, "source": "gdn_verify.cu",
-                      "sha256": "813090dfadf764cb421f435cc4489f27999477e790e4313a689feb6d7590babe"},
-    # verify_256x4, per-draft states: 555,026,944 read + 2,093,037,568 written
-    "verify_states": {"bytes": 2648064512, "source": "gdn_verify.cu",
-                      "sha256": "813090dfadf764cb421f435cc4489f27999477e790e4313a689feb6d7590babe"},
+    # verify_256x4, update-vector form, the streaming kernel: 579,884,544 read + 20,452,864
+    # written (its setup kernel adds 8,679,424)
+    "verify_deltas": {"bytes": 600337408, "source": "gdn_verify.cu",
+                      "sha256": "df4c2ca727a96543e20c2179c271f0d17d539afd0e73bb5afe0ff693637fc673"},
+    # verify_256x4, per-draft states: 554,937,088 read + 2,092,974,848 written
+    "verify_states": {"bytes": 2647911936, "source": "gdn_verify.cu",
+                      "sha256": "df4c2ca727a96543e20c2179c271f0d17d539afd0e73bb5afe0ff693637fc673"},
 }
 
 

@@ -148,3 +148,40 @@ def test_gate_logits_saturate_without_nan():
     assert_close(o, o_ref, torch.float32, "o")
     assert_close(hT, h_ref, torch.float32, "hT")
     assert np.all(np.isfinite(h_ref))
+
+
+def test_long_prefill_64k_raw_projections_sampled_heads():
+    """The bench's prologue leg: all 32 value heads of the 64K prefill from raw
+    projections on the GPU; the oracle recomputes one query/key group."""
+    from linear_attention_recurrence_rule_b200.inputs import WORKLOADS, workload_inputs
+    from parity_util import head_slice
+    w = WORKLOADS["long_prefill_64k"]
+    x = raw_projections(workload_inputs("long_prefill_64k"), seed=900)
+    d = to_dev(x)
+    o, hT = gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], chunk=w.chunk,
+                              prologue=PROLOGUE_ALL)
+    torch.cuda.synchronize()
+    sub, vh = head_slice(x, [5], w.HV // w.HK)
+    q, k, g, b = O.prologue(sub["q"], sub["k"], sub["g"], sub["beta"], PROLOGUE_ALL)
+    o_ref, h_ref = O.prefill(q, k, sub["v"], g, b)
+    assert_close(o[0][:, vh], o_ref, torch.bfloat16, "o")
+    assert_close(hT[:, vh], h_ref, torch.bfloat16, "hT")
+
+
+def test_decode_256_raw_projections_sampled_sequences():
+    """One decode step over the decode workload's 256 sequences from raw projections."""
+    from linear_attention_recurrence_rule_b200.inputs import workload_inputs
+    x = raw_projections(workload_inputs("decode_256x64", steps=2), seed=901)
+    d = to_dev(x)
+    S = d["state"].clone()
+    outs = [gdn_recurrent_step(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], S,
+                               prologue=PROLOGUE_ALL) for t in range(2)]
+    torch.cuda.synchronize()
+    seqs = [0, 64, 255]
+    Sref = x["state"][seqs]
+    for t in range(2):
+        q, k, g, b = O.prologue(x["q"][t][seqs], x["k"][t][seqs], x["g"][t][seqs],
+                                x["beta"][t][seqs], PROLOGUE_ALL)
+        o_ref, Sref = O.step(q, k, x["v"][t][seqs], g, b, Sref)
+        assert_close(outs[t][seqs], o_ref, torch.bfloat16, f"o step {t}")
+    assert_close(S[seqs], Sref, torch.bfloat16, "state")

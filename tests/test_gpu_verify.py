@@ -162,3 +162,30 @@ def test_verify_empty_and_errors():
     b = to_dev(big)
     with pytest.raises(GDNError):
         gdn_recurrent_verify(b["q"], b["k"], b["v"], b["g"], b["beta"], b["state"])
+
+
+@pytest.mark.parametrize("rollback", ["deltas", "states"])
+def test_verify_256x4_sampled_sequences(rollback):
+    """The benchmarked round: all 256 sequences x 4 drafts x 32 value heads on the
+    GPU, verify then commit of ~U{0..4} accepted drafts; the oracle follows 5
+    sequences."""
+    from linear_attention_recurrence_rule_b200.inputs import WORKLOADS, workload_inputs
+    w = WORKLOADS["verify_256x4"]
+    x = workload_inputs("verify_256x4")
+    d = to_dev(x)
+    gen = torch.Generator().manual_seed(w.seed + 77)
+    accepted = torch.randint(0, w.T + 1, (w.B,), generator=gen, dtype=torch.int32)
+    o, states, u = gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                                        rollback=rollback)
+    S = d["state"].clone()
+    if rollback == "deltas":
+        gdn_state_commit_deltas(d["k"], d["g"], u, accepted.cuda(), S)
+    else:
+        gdn_state_commit(states, accepted.cuda(), S)
+    torch.cuda.synchronize()
+    seqs = [0, 3, 100, 201, 255]
+    sub = {n: x[n][seqs] for n in ("q", "k", "v", "g", "beta", "state")}
+    o_ref, states_ref = O.verify(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], sub["state"])
+    assert_close(o[seqs], o_ref, torch.bfloat16, "o")
+    assert_close(S[seqs], O.commit(states_ref, accepted[seqs].numpy(), sub["state"]),
+                 torch.bfloat16, "committed state")
