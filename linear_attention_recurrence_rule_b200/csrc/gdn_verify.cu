@@ -699,13 +699,11 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
 }
 
 int device_sm_count() {
-    static int count = 0;
-    if (count == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            count = 148;
-    }
+    int dev = 0, count = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        count < 1)
+        count = 1;
     return count;
 }
 
@@ -722,13 +720,10 @@ void launch_verify_wy(const VerifyArgs &a, dim3, dim3 block, cudaStream_t stream
         a.HK, a.HV, a.scale, a.prologue);
     auto kern = verify_wy_kernel<DK, KT, Tin>;
     constexpr size_t smem = wy_smem_bytes<DK, KT>();
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return;   // the launch below reports the error
-        attr_set = true;
-    }
+    // per device and cheap: set on every launch (a process may drive several GPUs)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return;   // the launch below reports the error
     int per_sm = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kVerifyWarps * 32, smem) !=
             cudaSuccess ||
