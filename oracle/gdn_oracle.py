@@ -233,3 +233,45 @@ def prologue(q, k, g, beta, flags):
         g = -np.logaddexp(0.0, -g)
         beta = np.exp(-np.logaddexp(0.0, -beta))
     return q, k, g, beta
+
+
+def step_row_decay(q, k, v, g_rows, beta, state, scale=1.0):
+    """One decode token with one decay per value row: the forget gate of the
+    teaching code ("The Evolving Transformer / Qwen3-Next", section 01
+    GatedDeltaNet) has one entry per channel of the value dimension and scales
+    the rows of the state.  Row i of every (sequence, value head) state:
+        S_i <- alpha_i S_i                  (decay first, as in the scalar rule)
+        S_i <- S_i + beta (v_i - S_i . k) k^T
+        o_i  = scale * S_i . q
+    q,k [N,HK,dk]; v [N,HV,dv]; g_rows [N,HV,dv] (alpha = exp(g)); beta [N,HV];
+    state [N,HV,dv,dk].  Plain float64 loops; returns (o [N,HV,dv], new_state)."""
+    q, k, v, g_rows, beta = (_f64(x) for x in (q, k, v, g_rows, beta))
+    S = _f64(state).copy()
+    N, HK, dk = q.shape
+    HV, dv = v.shape[1], v.shape[2]
+    o = np.zeros((N, HV, dv))
+    for n in range(N):
+        for h in range(HV):
+            c = h // (HV // HK)
+            kt, qt = k[n, c], q[n, c]
+            for i in range(dv):
+                row = S[n, h, i] * np.exp(g_rows[n, h, i])
+                row = row + beta[n, h] * (v[n, h, i] - row @ kt) * kt
+                S[n, h, i] = row
+                o[n, h, i] = scale * (row @ qt)
+    return o, S
+
+
+def verify_row_decay(q, k, v, g_rows, beta, state, scale=1.0):
+    """``verify`` with one decay per value row: K calls of ``step_row_decay``.
+    q,k [N,K,HK,dk]; v, g_rows [N,K,HV,dv]; beta [N,K,HV]; state [N,HV,dv,dk]."""
+    q, k, v, g_rows, beta = (_f64(x) for x in (q, k, v, g_rows, beta))
+    S = _f64(state).copy()
+    N, K = q.shape[:2]
+    HV, dv, dk = S.shape[1], S.shape[2], S.shape[3]
+    o = np.zeros((N, K, HV, dv))
+    states = np.zeros((N, K, HV, dv, dk))
+    for t in range(K):
+        o[:, t], S = step_row_decay(q[:, t], k[:, t], v[:, t], g_rows[:, t], beta[:, t], S, scale)
+        states[:, t] = S
+    return o, states

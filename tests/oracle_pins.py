@@ -415,4 +415,72 @@ def pin_prologue_then_rule_is_scale_free(lib=None):
     assert not np.allclose(o1, o3, atol=1e-6)
 
 
+# ----------------------------------------------------------------------------
+# One decay per value row (the teaching code's per-channel forget gate)
+# ----------------------------------------------------------------------------
+def pin_row_decay_worked_examples(lib=None):
+    """The pages' scalar examples, one per row of a 2 x 1 state: row 0 without
+    decay goes 6 -> 8 -> 9, row 1 with decay 0.5 goes 6 -> 3 -> 6.5, then (no
+    decay) 6.5 -> 8.25, with the same key, target 10 and write strength 0.5."""
+    S0 = np.array([[[[6.0], [6.0]]]])                      # [N=1][HV=1][dv=2][dk=1]
+    one = np.ones((1, 1, 1))
+    v = np.full((1, 1, 2), 10.0)
+    beta = np.full((1, 1), 0.5)
+    g1 = np.log(np.array([[[1.0, 0.5]]]))
+    _, S1 = O.step_row_decay(one, one, v, g1, beta, S0)
+    assert np.array_equal(S1[0, 0, :, 0], [8.0, 6.5])
+    _, S2 = O.step_row_decay(one, one, v, np.zeros((1, 1, 2)), beta, S1)
+    assert np.array_equal(S2[0, 0, :, 0], [9.0, 8.25])
+
+
+def pin_row_decay_equal_rows_is_the_scalar_rule(lib=None):
+    """All rows of a head sharing one decay reproduce the scalar-decay oracle
+    (the independent C implementation)."""
+    rng = np.random.default_rng(23)
+    N, HK, HV, dk, dv = 3, 2, 4, 5, 6
+    q, k, v, g, beta = _rand_problem(rng, N, HK, HV, dk, dv)
+    q, k, v, g, beta = q[0], k[0], v[0], g[0], beta[0]     # N tokens -> N sequences
+    S0 = rng.standard_normal((N, HV, dv, dk))
+    o1, S1 = O.step(q, k, v, g, beta, S0, scale=0.7, lib=lib)
+    o2, S2 = O.step_row_decay(q, k, v, np.repeat(g[:, :, None], dv, axis=2), beta, S0,
+                              scale=0.7)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(S1, S2, atol=1e-12)
+
+
+def pin_row_decay_rows_are_independent(lib=None):
+    """Permuting the value rows (state rows, values and decays together)
+    permutes the outputs and the new state the same way; changing one row's
+    decay changes only that row."""
+    rng = np.random.default_rng(24)
+    q, k = rng.standard_normal((2, 1, 4)), rng.standard_normal((2, 1, 4))
+    v = rng.standard_normal((2, 2, 5))
+    g = rng.uniform(np.log(0.5), 0.0, (2, 2, 5))
+    beta = rng.uniform(0.1, 0.9, (2, 2))
+    S0 = rng.standard_normal((2, 2, 5, 4))
+    perm = np.array([3, 0, 4, 1, 2])
+    o, S = O.step_row_decay(q, k, v, g, beta, S0)
+    op, Sp = O.step_row_decay(q, k, v[:, :, perm], g[:, :, perm], beta, S0[:, :, perm])
+    assert np.allclose(op, o[:, :, perm], atol=1e-13) and np.allclose(Sp, S[:, :, perm], atol=1e-13)
+    g2 = g.copy()
+    g2[1, 0, 2] -= 0.3
+    o2, S2 = O.step_row_decay(q, k, v, g2, beta, S0)
+    changed = ~np.isclose(S2, S, atol=1e-14).all(axis=-1)
+    assert changed[1, 0, 2] and changed.sum() == 1
+
+
+def pin_verify_row_decay_equals_steps(lib=None):
+    rng = np.random.default_rng(25)
+    N, K, HK, HV, dk, dv = 2, 3, 1, 2, 4, 3
+    q, k = rng.standard_normal((N, K, HK, dk)), rng.standard_normal((N, K, HK, dk))
+    v = rng.standard_normal((N, K, HV, dv))
+    g = rng.uniform(np.log(0.6), 0.0, (N, K, HV, dv))
+    beta = rng.uniform(0.1, 0.9, (N, K, HV))
+    S0 = rng.standard_normal((N, HV, dv, dk))
+    o, states = O.verify_row_decay(q, k, v, g, beta, S0, scale=0.5)
+    S = S0
+    for t in range(K):
+        ot, S = O.step_row_decay(q[:, t], k[:, t], v[:, t], g[:, t], beta[:, t], S, scale=0.5)
+        assert np.array_equal(o[:, t], ot) and np.array_equal(states[:, t], S)
+
+
 ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

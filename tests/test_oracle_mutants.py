@@ -117,3 +117,51 @@ def test_prologue_pins_catch_mutant(monkeypatch, kind):
             except (AssertionError, ValueError):
                 caught.append(pin.__name__)
     assert caught, f"no pin detects the planted prologue mistake {kind}"
+
+
+# Mistakes planted in the per-row-decay step (plain numpy), each caught by a
+# row-decay pin.
+def _row_decay_mutant(kind):
+    import numpy as np
+
+    def mutant(q, k, v, g_rows, beta, state, scale=1.0):
+        q, k, v, g_rows, beta = (O._f64(x) for x in (q, k, v, g_rows, beta))
+        S = O._f64(state).copy()
+        N, HK, dk = q.shape
+        HV, dv = v.shape[1], v.shape[2]
+        o = np.zeros((N, HV, dv))
+        for n in range(N):
+            for h in range(HV):
+                c = h // (HV // HK)
+                kt, qt = k[n, c], q[n, c]
+                a = np.exp(g_rows[n, h])
+                for i in range(dv):
+                    row = S[n, h, i]
+                    if kind == "decay_after_correction":
+                        row = a[i] * (row + beta[n, h] * (v[n, h, i] - row @ kt) * kt)
+                    elif kind == "decay_on_key_columns":
+                        ac = np.resize(a, dk)
+                        row = row * ac
+                        row = row + beta[n, h] * (v[n, h, i] - row @ kt) * kt
+                    elif kind == "first_row_decay_for_all":
+                        row = row * a[0]
+                        row = row + beta[n, h] * (v[n, h, i] - row @ kt) * kt
+                    S[n, h, i] = row
+                    o[n, h, i] = scale * (row @ qt)
+        return o, S
+    return mutant
+
+
+@pytest.mark.parametrize("kind", ["decay_after_correction", "decay_on_key_columns",
+                                  "first_row_decay_for_all"])
+def test_row_decay_pins_catch_mutant(monkeypatch, kind):
+    monkeypatch.setattr(O, "step_row_decay", _row_decay_mutant(kind))
+    caught = []
+    for pin in ALL_PINS:
+        if "row_decay" not in pin.__name__:
+            continue
+        try:
+            pin()
+        except (AssertionError, ValueError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin detects the planted row-decay mistake {kind}"
