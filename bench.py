@@ -199,16 +199,20 @@ def measure_prologue(gdn, torch, dev, stream, x, w, ws, o, hT, rank, barrier, ma
     S = dy["state"].clone()
     od = torch.empty_like(dy["v"][0])
     res = {}
-    for tag, fl in (("plain", 0), ("prologue", flags)):
+    # one decay per value row (the per-channel forget gate), logits from the same draw
+    from linear_attention_recurrence_rule_b200.inputs import row_decays
+    g_rows = row_decays((8,) + tuple(dy["v"].shape[1:]), seed=902 + rank).to(dev)
+    for tag, fl in (("plain", 0), ("prologue", flags), ("row_decay", gdn.ROW_DECAY)):
+        gsel = g_rows if fl & gdn.ROW_DECAY else dy["g"]
         for t in range(3):
-            gdn.gdn_recurrent_step(dy["q"][t], dy["k"][t], dy["v"][t], dy["g"][t], dy["beta"][t],
+            gdn.gdn_recurrent_step(dy["q"][t], dy["k"][t], dy["v"][t], gsel[t], dy["beta"][t],
                                    S, o=od, stream=stream, prologue=fl)
         torch.cuda.synchronize()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(8)]
         for t, (a_, b_) in enumerate(evs):
             a_.record(stream)
-            gdn.gdn_recurrent_step(dy["q"][t], dy["k"][t], dy["v"][t], dy["g"][t], dy["beta"][t],
+            gdn.gdn_recurrent_step(dy["q"][t], dy["k"][t], dy["v"][t], gsel[t], dy["beta"][t],
                                    S, o=od, stream=stream, prologue=fl)
             b_.record(stream)
         torch.cuda.synchronize()
@@ -220,7 +224,11 @@ def measure_prologue(gdn, torch, dev, stream, x, w, ws, o, hT, rank, barrier, ma
                         "overhead": pf_s / plain_s - 1.0, "gpu_launches": args.steps},
             "decode": {"workload": DECODE_WORKLOAD, "ms_per_step": res["prologue"],
                        "plain_ms_per_step": res["plain"],
-                       "overhead": res["prologue"] / res["plain"] - 1.0, "gpu_launches": 16},
+                       "overhead": res["prologue"] / res["plain"] - 1.0, "gpu_launches": 11},
+            "decode_row_decay": {"workload": DECODE_WORKLOAD, "ms_per_step": res["row_decay"],
+                                 "overhead": res["row_decay"] / res["plain"] - 1.0,
+                                 "gpu_launches": 11,
+                                 "decays": "one per value row, alpha ~U(0.8, 1)"},
             "inputs": "raw projections: q, k rows of norm ~U(0.25, 4), forget logits ~N(3, 1), "
                       "write logits ~N(0, 1)"}
 

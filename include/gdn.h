@@ -106,6 +106,22 @@ GDN_API size_t gdn_chunk_prefill_workspace_size(int N, int64_t T, int HK, int HV
 #define GDN_PROLOGUE_ALL 7u
 
 /*
+ * GDN_ROW_DECAY (same flag word): one decay per value row instead of one per
+ * head -- the teaching code's per-channel forget gate, which scales the rows of
+ * the state ("The Evolving Transformer / Qwen3-Next", section 01 GatedDeltaNet).
+ * `g` (or, with GDN_PROLOGUE_GATE_LOGITS, its logits) then has one entry per
+ * value row: [N][HV][dv] for gdn_recurrent_step_ex, [N][K][HV][dv] for
+ * gdn_recurrent_verify and gdn_state_commit_deltas.  Each row i of a state
+ * decays by its own alpha_i before the correction.  Supported by the decode
+ * step, by verify when states_out is given, and by both commits; the chunked
+ * prefill and the update-vector-only verify return GDN_ERR_UNSUPPORTED (their
+ * per-head tables -- the chunk's triangular inverse, the mixed vectors -- would
+ * become per row).
+ */
+#define GDN_ROW_DECAY 8u
+#define GDN_FLAGS_VALID 15u
+
+/*
  * 1 when gdn_chunk_prefill runs this (head dims, chunk, dtype) combination on
  * the tcgen05 tensor-core path, 0 when it runs on the CUDA-core path, -1 when
  * the combination is unsupported.  Pure host query.
@@ -151,7 +167,7 @@ GDN_API gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v
  * gdn_chunk_prefill with the input prologue fused (`prologue`: GDN_PROLOGUE_*
  * flags; 0 is exactly gdn_chunk_prefill).  With GDN_PROLOGUE_GATE_LOGITS, g
  * and beta hold the logits (any real values).  Unknown flag bits return
- * GDN_ERR_INVALID_ARG.
+ * GDN_ERR_INVALID_ARG; GDN_ROW_DECAY returns GDN_ERR_UNSUPPORTED.
  */
 GDN_API gdn_status gdn_chunk_prefill_ex(const void *q, const void *k, const void *v,
                                         const float *g, const float *beta, const float *h0,
@@ -265,7 +281,8 @@ GDN_API gdn_status gdn_recurrent_step(const void *q, const void *k, const void *
 
 /*
  * gdn_recurrent_step with the input prologue fused (`prologue`: GDN_PROLOGUE_*
- * flags; 0 is exactly gdn_recurrent_step).  Unknown flag bits return
+ * flags, and GDN_ROW_DECAY for one decay per value row with g [N][HV][dv];
+ * 0 is exactly gdn_recurrent_step).  Unknown flag bits return
  * GDN_ERR_INVALID_ARG.
  */
 GDN_API gdn_status gdn_recurrent_step_ex(const void *q, const void *k, const void *v,
@@ -295,7 +312,8 @@ GDN_API gdn_status gdn_recurrent_step_ex(const void *q, const void *k, const voi
  *   q, k   [N][K][HK][dk] dtype      v, o [N][K][HV][dv] dtype
  *   g, beta [N][K][HV] fp32          state [N][HV][dv][dk] fp32 (read)
  *   states_out [N][K][HV][dv][dk] fp32   u_out [N][K][HV][dv] fp32
- * prologue: GDN_PROLOGUE_* flags applied to every draft (0 = prepared inputs).
+ * prologue: GDN_PROLOGUE_* flags applied to every draft (0 = prepared inputs);
+ * GDN_ROW_DECAY (g [N][K][HV][dv]) needs states_out, else GDN_ERR_UNSUPPORTED.
  * workspace: device scratch of at least gdn_recurrent_verify_workspace_size()
  * bytes, 16-byte aligned, needed when states_out is NULL (the update-vector
  * form builds per (sequence, value head) tables there; ignored otherwise, may

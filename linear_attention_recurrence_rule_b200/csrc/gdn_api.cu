@@ -130,7 +130,8 @@ gdn_status gdn_chunk_prefill_ex(const void *q, const void *k, const void *v, con
                                 int N, int64_t T, int HK, int HV, int dk, int dv, int chunk,
                                 float scale, gdn_dtype dtype, void *o, float *hT, void *workspace,
                                 size_t workspace_bytes, unsigned prologue, gdn_stream_t stream) {
-    if (prologue & ~GDN_PROLOGUE_ALL) return GDN_ERR_INVALID_ARG;
+    if (prologue & ~GDN_FLAGS_VALID) return GDN_ERR_INVALID_ARG;
+    if (prologue & GDN_ROW_DECAY) return GDN_ERR_UNSUPPORTED;
     gdn::PrefillArgs a{q, k, v, g, beta, h0, cu_seqlens, N, T, HK, HV, dk, dv, chunk,
                        scale, dtype, o, hT, workspace, workspace_bytes};
     a.prologue = prologue;
@@ -255,7 +256,7 @@ gdn_status gdn_recurrent_step_ex(const void *q, const void *k, const void *v, co
                                  const float *beta, float *state, int N, int HK, int HV, int dk,
                                  int dv, float scale, gdn_dtype dtype, void *o, unsigned prologue,
                                  gdn_stream_t stream) {
-    if (prologue & ~GDN_PROLOGUE_ALL) return GDN_ERR_INVALID_ARG;
+    if (prologue & ~GDN_FLAGS_VALID) return GDN_ERR_INVALID_ARG;
     if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
     if (N < 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK) return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
@@ -274,7 +275,7 @@ gdn_status gdn_recurrent_verify(const void *q, const void *k, const void *v, con
                                 int dk, int dv, float scale, gdn_dtype dtype, void *o,
                                 float *states_out, float *u_out, unsigned prologue,
                                 void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
-    if (prologue & ~GDN_PROLOGUE_ALL) return GDN_ERR_INVALID_ARG;
+    if (prologue & ~GDN_FLAGS_VALID) return GDN_ERR_INVALID_ARG;
     if (N < 0 || K <= 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK)
         return GDN_ERR_INVALID_ARG;
     if (N == 0) return GDN_OK;   // empty batch: buffers may be NULL
@@ -285,6 +286,7 @@ gdn_status gdn_recurrent_verify(const void *q, const void *k, const void *v, con
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
         !aligned16(states_out) || !aligned4(u_out))
         return GDN_ERR_ALIGNMENT;
+    if (!states_out && (prologue & GDN_ROW_DECAY)) return GDN_ERR_UNSUPPORTED;
     if (!states_out) {   // update-vector form: tables in the workspace
         if (!workspace ||
             workspace_bytes < gdn::verify_workspace_floats(N, K, HV, dk) * sizeof(float))
@@ -319,7 +321,7 @@ gdn_status gdn_state_commit_deltas(const void *k, const float *g, const float *u
                                    const int32_t *accepted, float *state, int N, int K, int HK,
                                    int HV, int dk, int dv, gdn_dtype dtype, unsigned prologue,
                                    gdn_stream_t stream) {
-    if (prologue & ~GDN_PROLOGUE_ALL) return GDN_ERR_INVALID_ARG;
+    if (prologue & ~GDN_FLAGS_VALID) return GDN_ERR_INVALID_ARG;
     if (N < 0 || K <= 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK)
         return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;

@@ -50,7 +50,8 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 
     float4 kk = load4(k + ((size_t)n * HK + c) * DK + col);
     float4 qq = load4(q + ((size_t)n * HK + c) * DK + col);
-    const float graw = g[nh], braw = beta[nh];
+    const bool rowdec = PRO && (pro & GDN_ROW_DECAY) != 0;   // g: one entry per value row
+    const float graw = rowdec ? 0.f : g[nh], braw = beta[nh];
     const Tin *vrow = v + (size_t)nh * dv;
     Tin *orow = o + (size_t)nh * dv;
     float *S = state + (size_t)nh * dv * DK;
@@ -60,11 +61,13 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         const int base = blockIdx.y * rows_per_batch;
         // the state loads go out first: nothing below them waits on q, k
         float4 s[kDecodeNB];
+        float grow[kDecodeNB];   // per-row decays (GDN_ROW_DECAY), loaded with the state
 #pragma unroll
         for (int j = 0; j < kDecodeNB; ++j) {
             const int row = base + (j * kDecodeWarps + warp) * RPI + sub;
             s[j] = row < dv ? __ldcs(reinterpret_cast<const float4 *>(S + (size_t)row * DK + col))
                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            grow[j] = (rowdec && row < dv) ? g[(size_t)nh * dv + row] : 0.f;
         }
         if (PRO && (pro & (GDN_PROLOGUE_NORM_Q | GDN_PROLOGUE_NORM_K))) {
             // the lanes of a row hold the whole q and k: reduce the squared norms there
@@ -81,7 +84,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
         const bool logits = PRO && (pro & GDN_PROLOGUE_GATE_LOGITS) != 0;
-        const float alpha = logits ? gate_sigmoid(graw) : expf(graw);
+        const float alpha_h = logits ? gate_sigmoid(graw) : expf(graw);
         const float b = logits ? gate_sigmoid(braw) : braw;
 #pragma unroll
         for (int j = 0; j < kDecodeNB; ++j) {
@@ -93,6 +96,8 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
                 sq += __shfl_xor_sync(0xffffffffu, sq, off);
             }
             if (row < dv) {
+                const float alpha = rowdec ? (logits ? gate_sigmoid(grow[j]) : expf(grow[j]))
+                                           : alpha_h;
                 const float u = b * (to_f32(vrow[row]) - alpha * sk);
                 float4 ns;
                 ns.x = fmaf(alpha, s[j].x, u * kk.x);

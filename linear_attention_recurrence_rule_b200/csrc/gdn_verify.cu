@@ -103,6 +103,9 @@ verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     __shared__ float4 ks[kVerifyMaxDrafts][DK / 4], qs[kVerifyMaxDrafts][DK / 4];
     __shared__ float vs[kVerifyMaxDrafts][BAND];
     __shared__ float al[kVerifyMaxDrafts], be[kVerifyMaxDrafts];
+    // per-row decays (GDN_ROW_DECAY), only in the prologue instance
+    __shared__ float ar[PRO ? kVerifyMaxDrafts : 1][PRO ? BAND : 1];
+    const bool rowdec = PRO && (pro & GDN_ROW_DECAY) != 0;
     const int nh = blockIdx.x;
     const int n = nh / HV, h = nh - n * HV;
     const int c = h / (HV / HK);
@@ -131,10 +134,13 @@ verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         const int t = idx / BAND, r = idx - t * BAND;
         const int row = base + r;
         vs[t][r] = row < dv ? to_f32(v[(((size_t)n * K + t) * HV + h) * dv + row]) : 0.f;
+        if (rowdec)
+            ar[t][r] = row < dv ? gate_alpha(g[(((size_t)n * K + t) * HV + h) * dv + row], pro)
+                                : 1.f;
     }
     if (threadIdx.x < K) {
         const size_t gi = ((size_t)n * K + threadIdx.x) * HV + h;
-        al[threadIdx.x] = gate_alpha(g[gi], pro);
+        al[threadIdx.x] = rowdec ? 1.f : gate_alpha(g[gi], pro);
         be[threadIdx.x] = gate_beta(beta[gi], pro);
     }
     __syncthreads();
@@ -152,7 +158,7 @@ verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         }
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-        const float alpha = al[t], b = be[t];
+        const float alpha_h = al[t], b = be[t];
         const size_t nt = (size_t)n * K + t;
         Tin *orow = o + (nt * HV + h) * dv;
         float *Sout = states ? states + (nt * HV + h) * state_elems : nullptr;
@@ -172,6 +178,7 @@ verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
                 sk += __shfl_xor_sync(0xffffffffu, sk, off);
                 sq += __shfl_xor_sync(0xffffffffu, sq, off);
             }
+            const float alpha = rowdec ? ar[t][r] : alpha_h;
             const float u = b * (vs[t][r] - alpha * sk);
 #pragma unroll
             for (int i = 0; i < kVerifyF4; ++i) {
@@ -624,6 +631,8 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
     __shared__ float4 ks[kVerifyMaxDrafts][DK / 4];
     __shared__ float us[kVerifyMaxDrafts][BAND];
     __shared__ float coef[kVerifyMaxDrafts + 1];
+    __shared__ float gr[PRO ? BAND : 1];   // per-row decay products (GDN_ROW_DECAY)
+    const bool rowdec = PRO && (pro & GDN_ROW_DECAY) != 0;
     const int nh = blockIdx.x;
     const int n = nh / HV, h = nh - n * HV;
     const int c = h / (HV / HK);
@@ -643,7 +652,7 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
                                          li + LPR * i)
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && !rowdec) {
         // coef[t] = prod_{t<s<a} alpha_s, coef[K_max] = prod_{s<a} alpha_s
         float c_run = 1.f;
         for (int t = a - 1; t >= 0; --t) {
@@ -658,15 +667,29 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
     }
     __syncthreads();
     if (pro & GDN_PROLOGUE_NORM_K) normalize_rows<DK>(ks, a, warp, lane);   // read after the next barrier
-    for (int i = threadIdx.x; i < a * BAND; i += blockDim.x) {
-        const int t = i / BAND, r = i - t * BAND;
-        const int row = base + r;
-        us[t][r] = row < dv ? coef[t] * u[(((size_t)n * K + t) * HV + h) * dv + row] : 0.f;
+    if (rowdec) {
+        // the same products per value row, one thread per row
+        for (int r = threadIdx.x; r < BAND; r += blockDim.x) {
+            const int row = base + r;
+            float c_run = 1.f;
+            for (int t = a - 1; t >= 0; --t) {
+                const size_t e = (((size_t)n * K + t) * HV + h) * dv + row;
+                us[t][r] = row < dv ? c_run * u[e] : 0.f;
+                if (row < dv) c_run *= gate_alpha(g[e], pro);
+            }
+            gr[r] = c_run;
+        }
+    } else {
+        for (int i = threadIdx.x; i < a * BAND; i += blockDim.x) {
+            const int t = i / BAND, r = i - t * BAND;
+            const int row = base + r;
+            us[t][r] = row < dv ? coef[t] * u[(((size_t)n * K + t) * HV + h) * dv + row] : 0.f;
+        }
     }
     __syncthreads();
-    const float gam = coef[kVerifyMaxDrafts];
 #pragma unroll
     for (int jr = 0; jr < kVerifyRows; ++jr) {
+        const float gam = rowdec ? gr[(jr * kVerifyWarps + warp) * RPW + sub] : coef[kVerifyMaxDrafts];
 #pragma unroll
         for (int i = 0; i < kVerifyF4; ++i) {
             x[jr][i].x *= gam; x[jr][i].y *= gam; x[jr][i].z *= gam; x[jr][i].w *= gam;

@@ -21,6 +21,7 @@ GDN_F32, GDN_BF16 = 0, 1
 # input prologue flags (GDN_PROLOGUE_* in gdn.h)
 PROLOGUE_NORM_Q, PROLOGUE_NORM_K, PROLOGUE_GATE_LOGITS = 1, 2, 4
 PROLOGUE_ALL = 7
+ROW_DECAY = 8   # one decay per value row: g [..., HV, dv] (GDN_ROW_DECAY)
 
 _lock = threading.Lock()
 _handle = None
@@ -209,8 +210,9 @@ def gdn_recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, o=None, stre
         raise ValueError("expected q,k [N,HK,dk] and v [N,HV,dv]")
     N, HK, dk = q.shape
     HV, dv = v.shape[1], v.shape[2]
-    if g.shape != (N, HV) or beta.shape != (N, HV) or state.shape != (N, HV, dv, dk):
-        raise ValueError("expected g,beta [N,HV] and state [N,HV,dv,dk]")
+    g_shape = (N, HV, dv) if prologue & ROW_DECAY else (N, HV)
+    if g.shape != g_shape or beta.shape != (N, HV) or state.shape != (N, HV, dv, dk):
+        raise ValueError(f"expected g {g_shape}, beta [N,HV] and state [N,HV,dv,dk]")
     if o is None:
         o = torch.empty_like(v)
     else:
@@ -249,8 +251,9 @@ def gdn_recurrent_verify(q, k, v, g, beta, state, scale: float = 1.0, o=None, st
         raise ValueError("expected q,k [N,K,HK,dk] and v [N,K,HV,dv]")
     N, K, HK, dk = q.shape
     HV, dv = v.shape[2], v.shape[3]
-    if g.shape != (N, K, HV) or beta.shape != (N, K, HV) or state.shape != (N, HV, dv, dk):
-        raise ValueError("expected g,beta [N,K,HV] and state [N,HV,dv,dk]")
+    g_shape = (N, K, HV, dv) if prologue & ROW_DECAY else (N, K, HV)
+    if g.shape != g_shape or beta.shape != (N, K, HV) or state.shape != (N, HV, dv, dk):
+        raise ValueError(f"expected g {g_shape}, beta [N,K,HV] and state [N,HV,dv,dk]")
     if o is None:
         o = torch.empty_like(v)
     else:
@@ -336,7 +339,8 @@ def gdn_state_commit_deltas(k, g, u, accepted, state, stream=None, prologue: int
         raise ValueError("expected k [N,K,HK,dk], u [N,K,HV,dv], state [N,HV,dv,dk]")
     N, K, HK, dk = k.shape
     HV, dv = u.shape[2], u.shape[3]
-    if u.shape[:2] != (N, K) or g.shape != (N, K, HV) or accepted.shape != (N,) \
+    g_shape = (N, K, HV, dv) if prologue & ROW_DECAY else (N, K, HV)
+    if u.shape[:2] != (N, K) or g.shape != g_shape or accepted.shape != (N,) \
             or state.shape != (N, HV, dv, dk):
         raise ValueError("expected k [N,K,HK,dk], g [N,K,HV], u [N,K,HV,dv], accepted [N], "
                          "state [N,HV,dv,dk]")

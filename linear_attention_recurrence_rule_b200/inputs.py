@@ -157,6 +157,13 @@ def raw_projections(x: dict, seed: int, norm_range=(0.25, 4.0), forget_logit=(3.
     return out
 
 
+def row_decays(shape, seed: int, low: float = 0.8, high: float = 1.0):
+    """One log decay per value row: g = log(alpha), alpha ~U(low, high), fp32,
+    of the given shape ([..., HV, dv]); a random draw only."""
+    gen = torch.Generator().manual_seed(seed)
+    return torch.log(low + (high - low) * torch.rand(tuple(shape), generator=gen)).float()
+
+
 def workload_inputs(name: str, steps: int | None = None, seed_offset: int = 0,
                     tokens: int | None = None):
     """Inputs for one named workload (see ``WORKLOADS``).  ``seed_offset`` gives

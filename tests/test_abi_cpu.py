@@ -176,7 +176,7 @@ def test_commit_deltas_validation(lib):
     assert call(dv=300) == gdn.GDN_ERR_UNSUPPORTED
     assert call(state=fake(0x5004)) == gdn.GDN_ERR_ALIGNMENT
     assert call(N=0, k=None, u=None) == gdn.GDN_OK
-    assert call(pro=8) == gdn.GDN_ERR_INVALID_ARG
+    assert call(pro=16) == gdn.GDN_ERR_INVALID_ARG
 
 
 def test_prologue_flags_are_validated(lib):
@@ -187,11 +187,22 @@ def test_prologue_flags_are_validated(lib):
     a = dict(q=fake(0x1000), k=fake(0x2000), v=fake(0x3000), g=fake(0x4000), beta=fake(0x5000))
     assert lib.gdn_chunk_prefill_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], None, None, 1, 64,
                                     1, 2, 32, 32, 16, 1.0, gdn.GDN_F32, fake(0x6000), None, None,
-                                    0, 8, None) == gdn.GDN_ERR_INVALID_ARG
+                                    0, 16, None) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_recurrent_step_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], fake(0x6000), 2,
                                      1, 2, 128, 128, 1.0, gdn.GDN_BF16, fake(0x7000), 16,
                                      None) == gdn.GDN_ERR_INVALID_ARG
-    assert verify_call(lib, pro=9) == gdn.GDN_ERR_INVALID_ARG
+    assert verify_call(lib, pro=16) == gdn.GDN_ERR_INVALID_ARG
+    # one decay per value row: decode and per-draft-state verify only
+    assert re.search(r"#define GDN_ROW_DECAY 8u", text)
+    assert lib.gdn_chunk_prefill_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], None, None, 1, 64,
+                                    1, 2, 32, 32, 16, 1.0, gdn.GDN_F32, fake(0x6000), None, None,
+                                    0, gdn.ROW_DECAY, None) == gdn.GDN_ERR_UNSUPPORTED
+    need = lib.gdn_recurrent_verify_workspace_size(2, 4, 2, 128)
+    assert verify_call(lib, states=None, ws=fake(0xa000), ws_bytes=need,
+                       pro=gdn.ROW_DECAY) == gdn.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_recurrent_step_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], fake(0x6004), 2,
+                                     1, 2, 128, 128, 1.0, gdn.GDN_BF16, fake(0x7000),
+                                     gdn.ROW_DECAY | 7, None) == gdn.GDN_ERR_ALIGNMENT
     # valid flags still go through the other checks first
     assert lib.gdn_recurrent_step_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], fake(0x6004), 2,
                                      1, 2, 128, 128, 1.0, gdn.GDN_BF16, fake(0x7000), 7,

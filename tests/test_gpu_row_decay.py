@@ -1,0 +1,86 @@
+"""One decay per value row (GDN_ROW_DECAY: the teaching code's per-channel
+forget gate) in the decode step, the per-draft-state verify and both commits,
+through the C ABI, against the float64 oracle's ``step_row_decay`` and
+``verify_row_decay``."""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_recurrence_rule_b200 import (PROLOGUE_ALL, PROLOGUE_GATE_LOGITS, ROW_DECAY,
+                                                   GDNError, gdn_chunk_prefill, gdn_recurrent_step,
+                                                   gdn_recurrent_verify, gdn_state_commit,
+                                                   gdn_state_commit_deltas)
+from linear_attention_recurrence_rule_b200.inputs import (make_decode, make_prefill, make_verify,
+                                                          raw_projections, row_decays)
+from oracle import gdn_oracle as O
+from parity_util import assert_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("extra", [0, PROLOGUE_ALL])
+@pytest.mark.parametrize("N,HK,HV,dk,dv,dtype", [
+    (16, 2, 4, 128, 128, torch.bfloat16),
+    (5, 1, 2, 64, 48, torch.float32),
+    (3, 1, 1, 32, 200, torch.float32),
+])
+def test_decode_row_decay(N, HK, HV, dk, dv, dtype, extra):
+    base = make_decode(N, 3, HK, HV, dk, dv, dtype, seed=81, h0_std=0.3)
+    x = raw_projections(base, seed=82) if extra else base
+    g_rows = row_decays((3, N, HV, dv), seed=83)
+    if extra & PROLOGUE_GATE_LOGITS:   # logits of the same decays: alpha = sigmoid(a)
+        a = torch.exp(g_rows)
+        g_rows = torch.log(a / (1 - a)).float()
+    d = to_dev(x)
+    gd = g_rows.cuda()
+    S = d["state"].clone()
+    Sref = x["state"]
+    flags = ROW_DECAY | extra
+    for t in range(3):
+        o = gdn_recurrent_step(d["q"][t], d["k"][t], d["v"][t], gd[t].contiguous(), d["beta"][t],
+                               S, scale=0.8, prologue=flags)
+        q, k, g, b = O.prologue(x["q"][t], x["k"][t], g_rows[t], x["beta"][t], extra)
+        o_ref, Sref = O.step_row_decay(q, k, x["v"][t], g, b, Sref, scale=0.8)
+        assert_close(o, o_ref, dtype, f"o step {t}")
+    torch.cuda.synchronize()
+    assert_close(S, Sref, dtype, "state")
+
+
+@pytest.mark.parametrize("N,K,HK,HV,dk,dv,dtype", [
+    (9, 4, 2, 4, 128, 128, torch.bfloat16),
+    (4, 7, 1, 2, 64, 96, torch.float32),
+])
+def test_verify_and_commits_row_decay(N, K, HK, HV, dk, dv, dtype):
+    x = make_verify(N, K, HK, HV, dk, dv, dtype, seed=84, h0_std=0.3)
+    g_rows = row_decays((N, K, HV, dv), seed=85)
+    d = to_dev(x)
+    gd = g_rows.cuda()
+    o, states, u = gdn_recurrent_verify(d["q"], d["k"], d["v"], gd, d["beta"], d["state"],
+                                        scale=0.6, rollback="both", prologue=ROW_DECAY)
+    accepted = torch.arange(N, dtype=torch.int32) % (K + 1)
+    S1 = d["state"].clone()
+    gdn_state_commit(states, accepted.cuda(), S1)
+    S2 = d["state"].clone()
+    gdn_state_commit_deltas(d["k"], gd, u, accepted.cuda(), S2, prologue=ROW_DECAY)
+    torch.cuda.synchronize()
+    o_ref, states_ref = O.verify_row_decay(x["q"], x["k"], x["v"], g_rows, x["beta"], x["state"],
+                                           scale=0.6)
+    assert_close(o, o_ref, dtype, "o")
+    for t in range(K):
+        assert_close(states[:, t], states_ref[:, t], dtype, f"state after draft {t}")
+    kept = O.commit(states_ref, accepted.numpy(), x["state"])
+    assert_close(S1, kept, dtype, "committed (copy)")
+    assert_close(S2, kept, dtype, "committed (deltas)")
+
+
+def test_row_decay_unsupported_forms():
+    x = make_prefill(1, 2, 32, 32, [64], torch.float32, seed=86)
+    d = to_dev(x)
+    with pytest.raises(GDNError):
+        gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], chunk=16, prologue=ROW_DECAY)
+    y = make_verify(2, 3, 1, 2, 32, 32, torch.float32, seed=87)
+    e = to_dev(y)
+    g_rows = row_decays((2, 3, 2, 32), seed=88).cuda()
+    with pytest.raises(GDNError):
+        gdn_recurrent_verify(e["q"], e["k"], e["v"], g_rows, e["beta"], e["state"],
+                             rollback="deltas", prologue=ROW_DECAY)
