@@ -268,19 +268,19 @@ def load_peaks():
 # Each entry carries the sha256 of the kernel source it was taken on; a changed
 # source reports null.
 NCU_TRAFFIC = {
-    # full decode_256x64 step: 541,149,696 read + 477,217,536 written
-    "decode": {"bytes": 1018367232, "source": "gdn_decode.cu",
-               "sha256": "1b91a761970c803c59da9d7895e9892ca047fb13f5922a6be591c74fb54279bd"},
-    # full long_prefill_64k launch: 1,090,729,728 read + 510,220,032 written
-    "prefill_cluster": {"bytes": 1600949760, "source": "gdn_prefill_cluster.cu",
+    # full decode_256x64 step: 541,146,880 read + 476,584,192 written
+    "decode": {"bytes": 1017731072, "source": "gdn_decode.cu",
+               "sha256": "2b41374aacd6222f16e152e67df8cb51675c5fc07d35104e4c0cbf61c6d22621"},
+    # full long_prefill_64k launch: 1,090,664,192 read + 510,390,784 written
+    "prefill_cluster": {"bytes": 1601054976, "source": "gdn_prefill_cluster.cu",
                         "sha256": "881a325e6d56777fe19db569636ec05bdd86d18a1d8dea300fed5c5991d89ae0"},
-    # verify_256x4, update-vector form, the streaming kernel: 579,884,544 read + 20,452,864
-    # written (its setup kernel adds 8,679,424)
-    "verify_deltas": {"bytes": 600337408, "source": "gdn_verify.cu",
-                      "sha256": "df4c2ca727a96543e20c2179c271f0d17d539afd0e73bb5afe0ff693637fc673"},
-    # verify_256x4, per-draft states: 554,937,088 read + 2,092,974,848 written
-    "verify_states": {"bytes": 2647911936, "source": "gdn_verify.cu",
-                      "sha256": "df4c2ca727a96543e20c2179c271f0d17d539afd0e73bb5afe0ff693637fc673"},
+    # verify_256x4, update-vector form, the streaming kernel: 579,901,696 read + 21,873,920
+    # written (its setup kernel adds 8,680,192)
+    "verify_deltas": {"bytes": 601775616, "source": "gdn_verify.cu",
+                      "sha256": "f653b5a19667221bcad35290a382fdd867b7d01015b48c9285dce05bd87c36b7"},
+    # verify_256x4, per-draft states: 554,840,832 read + 2,093,378,048 written
+    "verify_states": {"bytes": 2648218880, "source": "gdn_verify.cu",
+                      "sha256": "f653b5a19667221bcad35290a382fdd867b7d01015b48c9285dce05bd87c36b7"},
 }
 
 
