@@ -74,7 +74,11 @@ def verify_bytes(N, K, HK, HV, dk, dv, accepted, rollback, elt=2):
     io = N * K * (2 * HK * dk * elt + 2 * HV * dv * elt + 2 * HV * 4)
     kept = sum(1 for a in accepted if 1 <= a <= K)
     drafts_kept = sum(a for a in accepted if 1 <= a <= K)
-    if rollback == "states":
+    if rollback == "fused":   # commit of the previous round's drafts, then verify, one pass
+        ver = (N * state + kept * state + io + N * K * HV * dv * 4 +
+               drafts_kept * (HK * dk * elt + HV * 4 + HV * dv * 4) + N * 4)
+        com = 0
+    elif rollback == "states":
         ver = N * state * (1 + K) + io
         com = kept * 2 * state + N * 4
     else:
@@ -107,6 +111,48 @@ def measure_verify(gdn, torch, dev, stream, peaks, peak_src, rank, world, max_ov
            "accepted_mean": float(acc_host.float().mean()),
            "acceptance": "synthetic ~U{0..K} per sequence"}
     rounds = max(1, args.verify_rounds)
+    # fused rounds: each call keeps the previous round's accepted drafts, then
+    # verifies this round's (the same draft inputs every round, u alternating)
+    u_alt = torch.empty_like(u)
+    fws = torch.empty(gdn.gdn_recurrent_commit_verify_workspace_size(N, K, K, wv.HV, wv.dk),
+                      dtype=torch.uint8, device=dev)
+
+    def fused_round(prev_u, new_u):
+        gdn.gdn_recurrent_commit_verify(dy["k"], dy["g"], prev_u, accepted, dy["q"], dy["k"],
+                                        dy["v"], dy["g"], dy["beta"], S, o=o, u_out=new_u,
+                                        workspace=fws, stream=stream)
+
+    S.copy_(dy["state"])
+    gdn.gdn_recurrent_verify(dy["q"], dy["k"], dy["v"], dy["g"], dy["beta"], S, o=o, u_out=u,
+                             rollback="deltas", stream=stream)
+    bufs = [u, u_alt]
+    for w_ in range(max(3, args.warmup)):
+        fused_round(bufs[w_ & 1], bufs[(w_ + 1) & 1])
+    torch.cuda.synchronize()
+    barrier()
+    fsampler = ClockSampler(int(dev.index or 0))
+    fsampler.start()
+    fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(rounds)]
+    for r_, (a_, b_) in enumerate(fev):
+        a_.record(stream)
+        fused_round(bufs[r_ & 1], bufs[(r_ + 1) & 1])
+        b_.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    fclocks = fsampler.stop()
+    f_ms = statistics.mean(a_.elapsed_time(b_) for a_, b_ in fev)
+    ftotal = max_over_ranks(fev[0][0].elapsed_time(fev[-1][1]))
+    fb, _ = verify_bytes(N, K, wv.HK, wv.HV, wv.dk, wv.dv, acc_host.tolist(), "fused")
+    f_gbs = fb / (f_ms / 1e3) / 1e9
+    out["fused"] = {
+        "value": world * N * K * rounds / (ftotal / 1e3), "unit": "draft tokens/s",
+        "ms_per_round": ftotal / rounds, "bytes_per_round": fb,
+        "roofline": {"bound": "hbm", "achieved": f_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": f_gbs / hbm_peak, "traffic": None, "peak_source": peak_src,
+                     "kernel": "verify_wy (commit fused)"},
+        "gpu_launches": 2 * rounds, "clocks": fclocks,
+        "call": "gdn_recurrent_commit_verify: previous round's commit + this round's verify"}
     for form in ("deltas", "states"):
         def verify():
             if form == "deltas":

@@ -339,6 +339,36 @@ GDN_API gdn_status gdn_recurrent_verify(const void *q, const void *k, const void
 GDN_API size_t gdn_recurrent_verify_workspace_size(int N, int K, int HV, int dk);
 
 /*
+ * One speculative-decoding round in one pass over the states: first keeps the
+ * previous round's accepted drafts (exactly gdn_state_commit_deltas with prev_k,
+ * prev_g, prev_u, accepted), writing `state` in place for every sequence that kept
+ * at least one draft, then verifies this round's K drafts from the committed
+ * state (exactly gdn_recurrent_verify in its update-vector form: o and u_out, the
+ * latter for the next round's commit).  Each state element is read once, and
+ * written once where a draft was kept -- against three passes for the two calls.
+ *
+ * Layouts: prev_k [N][prev_K][HK][dk] dtype, prev_g [N][prev_K][HV] fp32,
+ * prev_u [N][prev_K][HV][dv] fp32, accepted [N] int32 (device; 0 or out of range
+ * = nothing kept); the rest as gdn_recurrent_verify.  `prologue` applies to both
+ * rounds' drafts (GDN_ROW_DECAY returns GDN_ERR_UNSUPPORTED).
+ * workspace: at least gdn_recurrent_commit_verify_workspace_size() bytes,
+ * 16-byte aligned; its first word is the status of the call's bounded waits
+ * (gdn_read_status).  Supported: as gdn_recurrent_verify, 1 <= prev_K <= 16.
+ */
+GDN_API gdn_status gdn_recurrent_commit_verify(const void *prev_k, const float *prev_g,
+                                               const float *prev_u, const int32_t *accepted,
+                                               int prev_K, const void *q, const void *k,
+                                               const void *v, const float *g, const float *beta,
+                                               float *state, int N, int K, int HK, int HV, int dk,
+                                               int dv, float scale, gdn_dtype dtype, void *o,
+                                               float *u_out, unsigned prologue, void *workspace,
+                                               size_t workspace_bytes, gdn_stream_t stream);
+
+/* Workspace bytes of gdn_recurrent_commit_verify (0 for invalid sizes). */
+GDN_API size_t gdn_recurrent_commit_verify_workspace_size(int N, int prev_K, int K, int HV,
+                                                          int dk);
+
+/*
  * Keeps the accepted drafts after gdn_recurrent_verify (states_out form): for
  * each sequence n, state[n] <- states[n][accepted[n] - 1] when
  * 1 <= accepted[n] <= K; state[n] is left unchanged when accepted[n] is 0 (or

@@ -8,11 +8,13 @@ from .gdn import (GDN_BF16, GDN_F32, GDNError, gdn_chunk_prefill,  # noqa: F401
                   gdn_chunk_prefill_host, gdn_chunk_prefill_host_workspace_size, gdn_validate_cu_seqlens,
                   gdn_chunk_prefill_path, gdn_chunk_prefill_workspace_size, gdn_read_status, gdn_recurrent_step,
                   gdn_recurrent_verify, gdn_recurrent_verify_workspace_size, gdn_state_commit,
+                  gdn_recurrent_commit_verify, gdn_recurrent_commit_verify_workspace_size,
                   gdn_state_commit_deltas,
                   lib_path, load_library, status_string, PROLOGUE_NORM_Q, PROLOGUE_NORM_K,
                   PROLOGUE_GATE_LOGITS, PROLOGUE_ALL, ROW_DECAY)
 
 __all__ = ["gdn_chunk_prefill", "gdn_recurrent_step", "gdn_recurrent_verify", "gdn_recurrent_verify_workspace_size", "gdn_state_commit",
+           "gdn_recurrent_commit_verify", "gdn_recurrent_commit_verify_workspace_size",
            "gdn_state_commit_deltas", "gdn_chunk_prefill_workspace_size", "gdn_chunk_prefill_path",
            "gdn_chunk_prefill_host", "gdn_chunk_prefill_host_workspace_size", "gdn_validate_cu_seqlens",
            "gdn_read_status", "status_string", "load_library", "lib_path", "GDNError",

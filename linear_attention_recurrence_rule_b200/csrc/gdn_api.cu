@@ -299,6 +299,48 @@ gdn_status gdn_recurrent_verify(const void *q, const void *k, const void *v, con
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status gdn_recurrent_commit_verify(const void *prev_k, const float *prev_g, const float *prev_u,
+                                       const int32_t *accepted, int prev_K, const void *q,
+                                       const void *k, const void *v, const float *g,
+                                       const float *beta, float *state, int N, int K, int HK,
+                                       int HV, int dk, int dv, float scale, gdn_dtype dtype,
+                                       void *o, float *u_out, unsigned prologue, void *workspace,
+                                       size_t workspace_bytes, gdn_stream_t stream) {
+    if (prologue & ~GDN_FLAGS_VALID) return GDN_ERR_INVALID_ARG;
+    if (N < 0 || K <= 0 || prev_K <= 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK)
+        return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (N == 0) return GDN_OK;   // empty batch: buffers may be NULL
+    if (!q || !k || !v || !g || !beta || !state || !o || !prev_k || !prev_g || !prev_u || !accepted)
+        return GDN_ERR_INVALID_ARG;
+    if (K > GDN_VERIFY_MAX_DRAFTS || prev_K > GDN_VERIFY_MAX_DRAFTS || (int64_t)N * HV > 0x7fffffff)
+        return GDN_ERR_UNSUPPORTED;
+    if (!gdn::decode_supported(dk, dv) || (prologue & GDN_ROW_DECAY)) return GDN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
+        !aligned16(prev_k) || !aligned4(prev_u) || !aligned4(accepted) || !aligned4(u_out))
+        return GDN_ERR_ALIGNMENT;
+    if (!workspace ||
+        workspace_bytes < gdn::verify_workspace_floats(N, K, HV, dk, prev_K) * sizeof(float))
+        return GDN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
+    gdn::VerifyArgs a{q, k, v, g, beta, state, nullptr, u_out, N, K, HK, HV, dk, dv, scale,
+                      dtype, o, prologue, workspace, workspace_bytes};
+    a.prev_k = prev_k;
+    a.prev_g = prev_g;
+    a.prev_u = prev_u;
+    a.accepted = accepted;
+    a.prev_K = prev_K;
+    const cudaError_t err = gdn::launch_verify(a, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+size_t gdn_recurrent_commit_verify_workspace_size(int N, int prev_K, int K, int HV, int dk) {
+    if (N < 0 || K <= 0 || K > GDN_VERIFY_MAX_DRAFTS || prev_K <= 0 ||
+        prev_K > GDN_VERIFY_MAX_DRAFTS || HV <= 0 || dk <= 0)
+        return 0;
+    return gdn::verify_workspace_floats(N, K, HV, dk, prev_K) * sizeof(float);
+}
+
 size_t gdn_recurrent_verify_workspace_size(int N, int K, int HV, int dk) {
     if (N < 0 || K <= 0 || K > GDN_VERIFY_MAX_DRAFTS || HV <= 0 || dk <= 0) return 0;
     return gdn::verify_workspace_floats(N, K, HV, dk) * sizeof(float);

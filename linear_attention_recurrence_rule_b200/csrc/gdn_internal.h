@@ -48,10 +48,16 @@ struct VerifyArgs {
     unsigned prologue = 0;
     void *workspace = nullptr;   // update-vector form: per (sequence, value head) tables
     size_t workspace_bytes = 0;
+    // fused commit-then-verify (prev_K > 0): the previous round's kept drafts
+    const void *prev_k = nullptr;
+    const float *prev_g = nullptr, *prev_u = nullptr;
+    const int32_t *accepted = nullptr;
+    int prev_K = 0;
 };
 
-// fp32 words of the update-vector form's workspace (gdn_verify.cu)
-size_t verify_workspace_floats(int N, int K, int HV, int dk);
+// fp32 words of the update-vector form's workspace (gdn_verify.cu); prev_K > 0 adds
+// the fused commit's tables
+size_t verify_workspace_floats(int N, int K, int HV, int dk, int prev_K = 0);
 
 
 // decode (gdn_decode.cu)

@@ -230,6 +230,12 @@ constexpr int kWsHeaderFloats = 4;
 __host__ __device__ inline size_t wy_item_floats(int K, int dk) {
     return ((size_t)2 * K * dk + 2 * (size_t)K * K + 3) & ~(size_t)3;
 }
+// fused commit-then-verify: after all the items' tables, per (sequence, value head)
+// the previous round's kept drafts as kt~_t = c_t k_t [Kp][dk] (c_t = prod_{t<s<a}
+// alpha_s), then gamma = prod_{s<a} alpha_s and the kept count a (as int bits)
+__host__ __device__ inline size_t pend_item_floats(int Kp, int dk) {
+    return ((size_t)Kp * dk + 4 + 3) & ~(size_t)3;
+}
 
 // one warp per (sequence, value head); a CTA holds a few such warps, each with
 // its own shared-memory slice, and only warp-level syncs
@@ -248,7 +254,8 @@ __global__ void __launch_bounds__(setup_warps<KT>() * 32)
 verify_setup_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const float *__restrict__ g, const float *__restrict__ beta,
                     float *__restrict__ ws, int items, int K, int HK, int HV, float scale,
-                    unsigned pro_arg) {
+                    unsigned pro_arg, const Tin *__restrict__ pk, const float *__restrict__ pg,
+                    const int32_t *__restrict__ accepted, float *__restrict__ pend, int Kp) {
     const unsigned pro = PRO ? pro_arg : 0u;
     constexpr int D4 = DK / 4;
     __shared__ SetupSlice<DK, KT> slices[setup_warps<KT>()];
@@ -351,6 +358,35 @@ verify_setup_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         kp[idx] = kk;
         qp[idx] = qq;
     }
+    if (pend == nullptr) return;
+    // ---- the previous round's kept drafts (fused commit-then-verify) ----
+    __syncwarp();   // the slice's rows are read by the loop above
+    float *po = pend + (size_t)nh * pend_item_floats(Kp, DK);
+    int a = accepted[n];
+    if (a < 0 || a > Kp) a = 0;
+    for (int idx = lane; idx < a * D4; idx += 32) {
+        const int t = idx / D4, j = idx - t * D4;
+        S.ks[t][j] = load4(pk + (((size_t)n * Kp + t) * HK + c) * DK + 4 * j);
+    }
+    if (lane < a) S.al[lane] = gate_alpha(pg[((size_t)n * Kp + lane) * HV + h], pro);
+    __syncwarp();
+    if (pro & GDN_PROLOGUE_NORM_K)
+        for (int t = 0; t < a; ++t) normalize_row<DK>(S.ks[t], lane);
+    if (lane == 0) {   // c_t = prod_{t<s<a} alpha_s, gamma = prod_{s<a} alpha_s
+        float c_run = 1.f;
+        for (int t = a - 1; t >= 0; --t) {
+            S.a1[t] = c_run;
+            c_run *= S.al[t];
+        }
+        po[(size_t)Kp * DK] = c_run;
+        po[(size_t)Kp * DK + 1] = __int_as_float(a);
+    }
+    __syncwarp();
+    float4 *ko = reinterpret_cast<float4 *>(po);
+    for (int idx = lane; idx < a * D4; idx += 32) {
+        const int t = idx / D4, f = idx - t * D4;
+        ko[idx] = scale4(S.ks[t][f], S.a1[t]);
+    }
 }
 
 // Streaming kernel, persistent: each CTA walks bands b = blockIdx.x + i * gridDim.x
@@ -366,25 +402,27 @@ verify_setup_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 // in flight (bounded) before it returns.
 constexpr uint32_t kWyWaitLimit = 2000;   // ~2 s of 1 ms sleeping polls
 
-template <int KT>
-__host__ __device__ constexpr int wy_stages() { return KT <= 4 ? 3 : 2; }
-template <int DK, int KT>
+template <int KT, bool FUSED>
+__host__ __device__ constexpr int wy_stages() { return (KT <= 4 && !FUSED) ? 3 : 2; }
+template <int DK, int KT, bool FUSED>
 __host__ __device__ constexpr size_t wy_stage_bytes() {
     return (size_t)verify_band<DK>() * DK * sizeof(float) +
-           ((2 * (size_t)KT * DK + 2 * (size_t)KT * KT + 3) & ~(size_t)3) * sizeof(float);
+           ((2 * (size_t)KT * DK + 2 * (size_t)KT * KT + 3) & ~(size_t)3) * sizeof(float) +
+           (FUSED ? (((size_t)KT * DK + 4 + 3) & ~(size_t)3) * sizeof(float) : 0);
 }
-template <int DK, int KT>
+template <int DK, int KT, bool FUSED>
 __host__ __device__ constexpr size_t wy_smem_bytes() {
-    // stages, the two v buffers [2][KT][BAND] fp32, the stage mbarriers
-    return wy_stages<KT>() * wy_stage_bytes<DK, KT>() +
-           2 * (size_t)KT * verify_band<DK>() * sizeof(float) +
-           wy_stages<KT>() * sizeof(uint64_t) + 16;
+    // stages, the v (and, fused, previous u) buffers [2][KT][BAND] fp32, the mbarriers
+    return wy_stages<KT, FUSED>() * wy_stage_bytes<DK, KT, FUSED>() +
+           (FUSED ? 4 : 2) * (size_t)KT * verify_band<DK>() * sizeof(float) +
+           wy_stages<KT, FUSED>() * sizeof(uint64_t) + 16;
 }
 
-template <int DK, int KT, typename Tin>
+template <int DK, int KT, typename Tin, bool FUSED>
 __global__ void __launch_bounds__(kVerifyWarps * 32, KT <= 8 ? 2 : 1)
-verify_wy_kernel(const Tin *__restrict__ v, const float *__restrict__ state, float *__restrict__ ws,
-                 float *__restrict__ u_out, Tin *__restrict__ o, int N, int K, int HV, int dv) {
+verify_wy_kernel(const Tin *__restrict__ v, float *state, float *__restrict__ ws,
+                 float *__restrict__ u_out, Tin *__restrict__ o, int N, int K, int HV, int dv,
+                 const float *__restrict__ prev_u, int Kp) {
     constexpr int LPR = DK / (4 * kVerifyF4);   // lanes per row: 2, 4, 8
     constexpr int RPW = 32 / LPR;
     constexpr int BAND = verify_band<DK>();
@@ -392,13 +430,14 @@ verify_wy_kernel(const Tin *__restrict__ v, const float *__restrict__ state, flo
     constexpr int NV = 2 * KT;                  // partial sums per row: u then o
     static_assert(NV % LPR == 0, "reduce-scatter needs 2 KT >= lanes per row");
     constexpr int NL = NV / LPR;                // finished values per lane
-    constexpr int NST = wy_stages<KT>();
-    constexpr size_t SB = wy_stage_bytes<DK, KT>();
+    constexpr int NST = wy_stages<KT, FUSED>();
+    constexpr size_t SB = wy_stage_bytes<DK, KT, FUSED>();
     extern __shared__ __align__(128) uint8_t wy_smem[];
-    // v of a band, loaded one band ahead (plain loads into registers during the
-    // previous band's arithmetic, stored here after it)
+    // v (and, fused, the previous round's u) of a band, loaded one band ahead (plain
+    // loads into registers during the previous band's arithmetic, stored here after it)
     float *vsm = reinterpret_cast<float *>(wy_smem + NST * SB);   // [2][KT][BAND]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(vsm + 2 * KT * BAND);
+    float *usm = vsm + 2 * KT * BAND;                            // [2][KT][BAND], fused only
+    uint64_t *bars = reinterpret_cast<uint64_t *>(vsm + (FUSED ? 4 : 2) * KT * BAND);
     constexpr int VPT = (KT * BAND + kVerifyWarps * 32 - 1) / (kVerifyWarps * 32);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -408,6 +447,8 @@ verify_wy_kernel(const Tin *__restrict__ v, const float *__restrict__ state, flo
     const long long mine = total > blockIdx.x ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const size_t item_floats = wy_item_floats(K, DK);
     const float *tables = ws + kWsHeaderFloats;
+    const size_t pend_floats = FUSED ? pend_item_floats(Kp, DK) : 0;
+    const float *pend = tables + (size_t)N * HV * item_floats;
 
     // (value-head index, band) of this CTA's i-th band, b = blockIdx.x + i * gridDim.x,
     // advanced by the grid stride without a division per band
@@ -437,14 +478,18 @@ verify_wy_kernel(const Tin *__restrict__ v, const float *__restrict__ state, flo
         uint64_t *bar = &bars[i % NST];
         const uint32_t sbytes = (uint32_t)rows * DK * sizeof(float);
         const uint32_t tbytes = (uint32_t)(item_floats * sizeof(float));
-        tc::mbar_arrive_expect_tx(bar, sbytes + tbytes);
+        const uint32_t pbytes = (uint32_t)(pend_floats * sizeof(float));
+        tc::mbar_arrive_expect_tx(bar, sbytes + tbytes + pbytes);
         tc::bulk_load_g2s(stg, state + ((size_t)nh * dv + base) * DK, sbytes, bar);
         tc::bulk_load_g2s(stg + (size_t)BAND * DK * sizeof(float), tables + (size_t)nh * item_floats,
                           tbytes, bar);
+        if (FUSED)
+            tc::bulk_load_g2s(stg + (size_t)BAND * DK * sizeof(float) + tbytes,
+                              pend + (size_t)nh * pend_floats, pbytes, bar);
     };
     BandIt it_v;   // the band whose v is loaded next
     it_v.init(blockIdx.x, nbands);
-    auto load_v = [&](float (&vr)[VPT]) {   // v of band it_v, then advance it
+    auto load_v = [&](float (&vr)[VPT], float (&ur)[VPT]) {   // band it_v, then advance it
         const int nh = it_v.nh, base = it_v.y * BAND, rows = band_rows(it_v.y);
         it_v.next(step_nh, step_y, nbands);
         const int n = nh / HV, h = nh - n * HV;
@@ -454,14 +499,21 @@ verify_wy_kernel(const Tin *__restrict__ v, const float *__restrict__ state, flo
             const int j = e / BAND, r = e - j * BAND;
             vr[e0] = (j < K && r < rows) ? to_f32(v[(((size_t)n * K + j) * HV + h) * dv + base + r])
                                          : 0.f;
+            if (FUSED)
+                ur[e0] = (j < Kp && r < rows) ? prev_u[(((size_t)n * Kp + j) * HV + h) * dv + base + r]
+                                              : 0.f;
         }
     };
-    auto store_v = [&](long long i, const float (&vr)[VPT]) {
+    auto store_v = [&](long long i, const float (&vr)[VPT], const float (&ur)[VPT]) {
         float *dst = vsm + (i & 1) * KT * BAND;
+        float *udst = usm + (i & 1) * KT * BAND;
 #pragma unroll
         for (int e0 = 0; e0 < VPT; ++e0) {
             const int e = tid + e0 * kVerifyWarps * 32;
-            if (e < KT * BAND) dst[e] = vr[e0];
+            if (e < KT * BAND) {
+                dst[e] = vr[e0];
+                if (FUSED) udst[e] = ur[e0];
+            }
         }
     };
     if (tid == 0) {
@@ -470,9 +522,9 @@ verify_wy_kernel(const Tin *__restrict__ v, const float *__restrict__ state, flo
         for (long long i = 0; i < NST && i < mine; ++i) issue(i);
     }
     if (mine > 0) {
-        float vr[VPT];
-        load_v(vr);
-        store_v(0, vr);
+        float vr[VPT], ur[VPT];
+        load_v(vr, ur);
+        store_v(0, vr, ur);
     }
     __syncthreads();
     BandIt it;   // the band being computed
@@ -489,8 +541,8 @@ verify_wy_kernel(const Tin *__restrict__ v, const float *__restrict__ state, flo
             issue(i - 1 + NST);
             ++issued;
         }
-        float vnext[VPT];
-        if (i + 1 < mine) load_v(vnext);   // band i + 1: lands during this band's arithmetic
+        float vnext[VPT], unext[VPT];
+        if (i + 1 < mine) load_v(vnext, unext);   // band i + 1: lands during this band's arithmetic
         const int nh = it.nh, base = it.y * BAND, rows = band_rows(it.y);
         it.next(step_nh, step_y, nbands);
         const int n = nh / HV, h = nh - n * HV;
@@ -507,6 +559,39 @@ verify_wy_kernel(const Tin *__restrict__ v, const float *__restrict__ state, flo
             const int r = (jr * kVerifyWarps + warp) * RPW + sub;
 #pragma unroll
             for (int q4 = 0; q4 < kVerifyF4; ++q4) s[jr][q4] = srow[r * D4 + li + LPR * q4];
+        }
+        if (FUSED) {
+            // commit the previous round's kept drafts into the band first:
+            // S <- gamma S + sum_{t<a} u_t[r] kt~_t, written back to the state
+            const float *pitem = item + item_floats;
+            const int a = __float_as_int(pitem[(size_t)Kp * DK + 1]);
+            if (a > 0) {
+                const float gam = pitem[(size_t)Kp * DK];
+                const float4 *pkt = reinterpret_cast<const float4 *>(pitem);
+                const float *ub = usm + (i & 1) * KT * BAND;
+#pragma unroll
+                for (int jr = 0; jr < kVerifyRows; ++jr) {
+                    const int r = (jr * kVerifyWarps + warp) * RPW + sub;
+#pragma unroll
+                    for (int q4 = 0; q4 < kVerifyF4; ++q4) s[jr][q4] = scale4(s[jr][q4], gam);
+                    for (int t = 0; t < a; ++t) {
+                        const float f = ub[t * BAND + r];
+#pragma unroll
+                        for (int q4 = 0; q4 < kVerifyF4; ++q4) {
+                            const float4 kk = pkt[t * D4 + li + LPR * q4];
+                            s[jr][q4].x = fmaf(f, kk.x, s[jr][q4].x);
+                            s[jr][q4].y = fmaf(f, kk.y, s[jr][q4].y);
+                            s[jr][q4].z = fmaf(f, kk.z, s[jr][q4].z);
+                            s[jr][q4].w = fmaf(f, kk.w, s[jr][q4].w);
+                        }
+                    }
+                    if (r < rows) {
+                        float4 *dst = reinterpret_cast<float4 *>(state + ((size_t)nh * dv + base + r) * DK);
+#pragma unroll
+                        for (int q4 = 0; q4 < kVerifyF4; ++q4) __stcs(dst + li + LPR * q4, s[jr][q4]);
+                    }
+                }
+            }
         }
         // dot products on packed pairs (even / odd columns), summed once at the end
         float2 acc2[kVerifyRows][NV];
@@ -585,7 +670,7 @@ verify_wy_kernel(const Tin *__restrict__ v, const float *__restrict__ state, flo
                     o[ot] = from_f32<Tin>(val);
             }
         }
-        if (i + 1 < mine) store_v(i + 1, vnext);   // published by the next band's barrier
+        if (i + 1 < mine) store_v(i + 1, vnext, unext);   // published by the next band's barrier
     }
     if (!ok && tid == 0) {
         atomicExch(reinterpret_cast<unsigned int *>(ws), 1u);
@@ -730,19 +815,21 @@ int device_sm_count() {
     return count;
 }
 
-template <int DK, int KT, typename Tin>
-void launch_verify_wy(const VerifyArgs &a, dim3, dim3 block, cudaStream_t stream) {
+template <int DK, int KT, typename Tin, bool FUSED>
+void launch_verify_wy(const VerifyArgs &a, dim3 block, cudaStream_t stream) {
     auto setup = a.prologue ? verify_setup_kernel<DK, KT, Tin, true>
                             : verify_setup_kernel<DK, KT, Tin, false>;
     const int items = a.N * a.HV;
     constexpr int W = setup_warps<KT>();
     float *ws = static_cast<float *>(a.workspace);
+    float *pend = FUSED ? ws + kWsHeaderFloats + (size_t)items * wy_item_floats(a.K, DK) : nullptr;
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), stream) != cudaSuccess) return;
     setup<<<(unsigned)((items + W - 1) / W), W * 32, 0, stream>>>(
         static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k), a.g, a.beta, ws, items, a.K,
-        a.HK, a.HV, a.scale, a.prologue);
-    auto kern = verify_wy_kernel<DK, KT, Tin>;
-    constexpr size_t smem = wy_smem_bytes<DK, KT>();
+        a.HK, a.HV, a.scale, a.prologue, static_cast<const Tin *>(a.prev_k), a.prev_g, a.accepted,
+        pend, a.prev_K);
+    auto kern = verify_wy_kernel<DK, KT, Tin, FUSED>;
+    constexpr size_t smem = wy_smem_bytes<DK, KT, FUSED>();
     // per device and cheap: set on every launch (a process may drive several GPUs)
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
@@ -755,18 +842,24 @@ void launch_verify_wy(const VerifyArgs &a, dim3, dim3 block, cudaStream_t stream
     const long long bands = (long long)items * ((a.dv + verify_band<DK>() - 1) / verify_band<DK>());
     const long long slots = (long long)per_sm * device_sm_count();
     const unsigned grid = (unsigned)(bands < slots ? bands : slots);
-    kern<<<grid, block, smem, stream>>>(static_cast<const Tin *>(a.v), a.state, ws, a.u,
-                                        static_cast<Tin *>(a.o), a.N, a.K, a.HV, a.dv);
+    kern<<<grid, block, smem, stream>>>(static_cast<const Tin *>(a.v), const_cast<float *>(a.state),
+                                        ws, a.u, static_cast<Tin *>(a.o), a.N, a.K, a.HV, a.dv,
+                                        a.prev_u, a.prev_K);
 }
 
 template <int DK, typename Tin>
-void launch_verify_wy_k(const VerifyArgs &a, dim3 grid, dim3 block, cudaStream_t stream) {
-    if (a.K <= 4)
-        launch_verify_wy<DK, 4, Tin>(a, grid, block, stream);
-    else if (a.K <= 8)
-        launch_verify_wy<DK, 8, Tin>(a, grid, block, stream);
+void launch_verify_wy_k(const VerifyArgs &a, dim3 block, cudaStream_t stream) {
+    const int kb = a.K > a.prev_K ? a.K : a.prev_K;   // bound for both rounds' drafts
+    const bool fused = a.prev_K > 0;
+    if (kb <= 4)
+        fused ? launch_verify_wy<DK, 4, Tin, true>(a, block, stream)
+              : launch_verify_wy<DK, 4, Tin, false>(a, block, stream);
+    else if (kb <= 8)
+        fused ? launch_verify_wy<DK, 8, Tin, true>(a, block, stream)
+              : launch_verify_wy<DK, 8, Tin, false>(a, block, stream);
     else
-        launch_verify_wy<DK, 16, Tin>(a, grid, block, stream);
+        fused ? launch_verify_wy<DK, 16, Tin, true>(a, block, stream)
+              : launch_verify_wy<DK, 16, Tin, false>(a, block, stream);
 }
 
 template <int DK, typename Tin>
@@ -787,9 +880,9 @@ cudaError_t launch_verify_typed(const VerifyArgs &a, cudaStream_t stream) {
     if (a.states == nullptr) {
         // no per-draft states asked for: the state is never updated in registers
         switch (a.dk) {
-            case 32: launch_verify_wy_k<32, Tin>(a, grid, block, stream); break;
-            case 64: launch_verify_wy_k<64, Tin>(a, grid, block, stream); break;
-            case 128: launch_verify_wy_k<128, Tin>(a, grid, block, stream); break;
+            case 32: launch_verify_wy_k<32, Tin>(a, block, stream); break;
+            case 64: launch_verify_wy_k<64, Tin>(a, block, stream); break;
+            case 128: launch_verify_wy_k<128, Tin>(a, block, stream); break;
             default: return cudaErrorInvalidValue;
         }
         return cudaGetLastError();
@@ -805,8 +898,9 @@ cudaError_t launch_verify_typed(const VerifyArgs &a, cudaStream_t stream) {
 
 }  // namespace
 
-size_t verify_workspace_floats(int N, int K, int HV, int dk) {
-    return kWsHeaderFloats + (size_t)N * HV * wy_item_floats(K, dk);
+size_t verify_workspace_floats(int N, int K, int HV, int dk, int prev_K) {
+    return kWsHeaderFloats + (size_t)N * HV * wy_item_floats(K, dk) +
+           (prev_K > 0 ? (size_t)N * HV * pend_item_floats(prev_K, dk) : 0);
 }
 
 cudaError_t launch_verify(const VerifyArgs &a, cudaStream_t stream) {

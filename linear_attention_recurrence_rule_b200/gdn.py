@@ -74,6 +74,13 @@ def load_library() -> ctypes.CDLL:
                                                  ctypes.c_uint, vp, sz, vp]
             lib.gdn_recurrent_verify_workspace_size.restype = sz
             lib.gdn_recurrent_verify_workspace_size.argtypes = [i32, i32, i32, i32]
+            lib.gdn_recurrent_commit_verify.restype = i32
+            lib.gdn_recurrent_commit_verify.argtypes = [vp, vp, vp, vp, i32, vp, vp, vp, vp, vp,
+                                                        vp, i32, i32, i32, i32, i32, i32,
+                                                        ctypes.c_float, i32, vp, vp,
+                                                        ctypes.c_uint, vp, sz, vp]
+            lib.gdn_recurrent_commit_verify_workspace_size.restype = sz
+            lib.gdn_recurrent_commit_verify_workspace_size.argtypes = [i32, i32, i32, i32, i32]
             lib.gdn_state_commit.restype = i32
             lib.gdn_state_commit.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
             lib.gdn_state_commit_deltas.restype = i32
@@ -291,6 +298,62 @@ def gdn_recurrent_verify(q, k, v, g, beta, state, scale: float = 1.0, o=None, st
     if st != GDN_OK:
         raise GDNError(st, "gdn_recurrent_verify")
     return o, states_out, u_out
+
+
+def gdn_recurrent_commit_verify(prev_k, prev_g, prev_u, accepted, q, k, v, g, beta, state,
+                                scale: float = 1.0, o=None, u_out=None, workspace=None,
+                                stream=None, prologue: int = 0):
+    """Keep the previous round's accepted drafts, then verify this round's
+    (``gdn_recurrent_commit_verify``): ``state`` is updated in place to the
+    committed state; returns (o [N,K,HV,dv], u_out [N,K,HV,dv]) of this round.
+
+    prev_k [N,Kp,HK,dk]; prev_g [N,Kp,HV]; prev_u [N,Kp,HV,dv] (the previous
+    verify's u_out); accepted [N] int32 on the device; the rest as
+    ``gdn_recurrent_verify``.
+    """
+    lib = load_library()
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v), ("prev_k", prev_k)):
+        _need(t, name, q.dtype, dev)
+    for name, t in (("g", g), ("beta", beta), ("state", state), ("prev_g", prev_g),
+                    ("prev_u", prev_u)):
+        _need(t, name, torch.float32, dev)
+    _need(accepted, "accepted", torch.int32, dev)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("expected q,k [N,K,HK,dk] and v [N,K,HV,dv]")
+    N, K, HK, dk = q.shape
+    HV, dv = v.shape[2], v.shape[3]
+    Kp = prev_k.shape[1] if prev_k.dim() == 4 else -1
+    if (g.shape != (N, K, HV) or beta.shape != (N, K, HV) or state.shape != (N, HV, dv, dk)
+            or prev_k.shape != (N, Kp, HK, dk) or prev_g.shape != (N, Kp, HV)
+            or prev_u.shape != (N, Kp, HV, dv) or accepted.shape != (N,)):
+        raise ValueError("shapes: prev_k [N,Kp,HK,dk], prev_g [N,Kp,HV], prev_u [N,Kp,HV,dv], "
+                         "accepted [N], q,k [N,K,HK,dk], v [N,K,HV,dv], g,beta [N,K,HV], "
+                         "state [N,HV,dv,dk]")
+    if o is None:
+        o = torch.empty_like(v)
+    if u_out is None:
+        u_out = torch.empty((N, K, HV, dv), dtype=torch.float32, device=dev)
+    _need(o, "o", v.dtype, dev)
+    _need(u_out, "u_out", torch.float32, dev)
+    if workspace is None and N > 0:
+        need = int(lib.gdn_recurrent_commit_verify_workspace_size(N, Kp, K, HV, dk))
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.gdn_recurrent_commit_verify(_ptr(prev_k), _ptr(prev_g), _ptr(prev_u), _ptr(accepted),
+                                         Kp, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                         _ptr(state), N, K, HK, HV, dk, dv, float(scale),
+                                         _dtype_code(q), _ptr(o), _ptr(u_out), int(prologue),
+                                         _ptr(workspace), ws_bytes, _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_recurrent_commit_verify")
+    return o, u_out
+
+
+def gdn_recurrent_commit_verify_workspace_size(N, prev_K, K, HV, dk) -> int:
+    """Bytes of workspace ``gdn_recurrent_commit_verify`` needs."""
+    return int(load_library().gdn_recurrent_commit_verify_workspace_size(
+        int(N), int(prev_K), int(K), int(HV), int(dk)))
 
 
 def gdn_recurrent_verify_workspace_size(N, K, HV, dk) -> int:

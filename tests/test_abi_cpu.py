@@ -207,3 +207,29 @@ def test_prologue_flags_are_validated(lib):
     assert lib.gdn_recurrent_step_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], fake(0x6004), 2,
                                      1, 2, 128, 128, 1.0, gdn.GDN_BF16, fake(0x7000), 7,
                                      None) == gdn.GDN_ERR_ALIGNMENT
+
+
+def test_commit_verify_validation(lib):
+    def call(**kw):
+        a = dict(pk=fake(0x1000), pg=fake(0x2000), pu=fake(0x3000), acc=fake(0x4000), Kp=4,
+                 q=fake(0x5000), k=fake(0x6000), v=fake(0x7000), g=fake(0x8000),
+                 beta=fake(0x9000), state=fake(0xa000), N=2, K=4, HK=1, HV=2, dk=128, dv=128,
+                 dtype=gdn.GDN_BF16, o=fake(0xb000), u=fake(0xc000), pro=0, ws=None, ws_bytes=0)
+        a.update(kw)
+        return lib.gdn_recurrent_commit_verify(
+            a["pk"], a["pg"], a["pu"], a["acc"], a["Kp"], a["q"], a["k"], a["v"], a["g"],
+            a["beta"], a["state"], a["N"], a["K"], a["HK"], a["HV"], a["dk"], a["dv"], 1.0,
+            a["dtype"], a["o"], a["u"], a["pro"], a["ws"], a["ws_bytes"], None)
+    # every call below is rejected before anything is enqueued
+    assert call(Kp=0) == gdn.GDN_ERR_INVALID_ARG
+    assert call(pu=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(pro=16) == gdn.GDN_ERR_INVALID_ARG
+    assert call(Kp=17) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(pro=gdn.ROW_DECAY) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(pk=fake(0x1008)) == gdn.GDN_ERR_ALIGNMENT
+    assert call() == gdn.GDN_ERR_WORKSPACE
+    need = lib.gdn_recurrent_commit_verify_workspace_size(2, 4, 4, 2, 128)
+    assert need == 16 + 2 * 2 * ((2 * 4 * 128 + 2 * 16) + (4 * 128 + 4)) * 4
+    assert call(ws=fake(0xd000), ws_bytes=need - 16) == gdn.GDN_ERR_WORKSPACE
+    assert call(ws=fake(0xd008), ws_bytes=need) == gdn.GDN_ERR_ALIGNMENT
+    assert call(N=0, q=None, pk=None) == gdn.GDN_OK

@@ -189,3 +189,49 @@ def test_verify_256x4_sampled_sequences(rollback):
     assert_close(o[seqs], o_ref, torch.bfloat16, "o")
     assert_close(S[seqs], O.commit(states_ref, accepted[seqs].numpy(), sub["state"]),
                  torch.bfloat16, "committed state")
+
+
+@pytest.mark.parametrize("prologue", [0, 7])
+@pytest.mark.parametrize("N,K1,K2,HK,HV,dk,dv,dtype", [
+    (33, 4, 4, 2, 4, 128, 128, torch.bfloat16),   # the benchmarked shapes
+    (5, 3, 6, 1, 2, 64, 48, torch.float32),       # next round's bound (8) above the kept one
+    (4, 16, 2, 2, 2, 32, 200, torch.float32),     # the largest kept round, ragged band
+])
+def test_commit_verify_equals_commit_then_verify(N, K1, K2, HK, HV, dk, dv, dtype, prologue):
+    from linear_attention_recurrence_rule_b200 import (gdn_recurrent_commit_verify,
+                                                       gdn_recurrent_commit_verify_workspace_size)
+    from linear_attention_recurrence_rule_b200.inputs import raw_projections
+    x1 = make_verify(N, K1, HK, HV, dk, dv, dtype, seed=90 + K1, h0_std=0.3)
+    x2 = make_verify(N, K2, HK, HV, dk, dv, dtype, seed=91 + K2, h0_std=0.3)
+    if prologue:
+        x1, x2 = raw_projections(x1, seed=92), raw_projections(x2, seed=93)
+    d1, d2 = to_dev(x1), to_dev(x2)
+    _, _, u1 = gdn_recurrent_verify(d1["q"], d1["k"], d1["v"], d1["g"], d1["beta"], d1["state"],
+                                    rollback="deltas", prologue=prologue)
+    accepted = (torch.arange(N, dtype=torch.int32) * 7) % (K1 + 2)   # includes 0 and K1 + 1
+    S = d1["state"].clone()
+    ws = torch.empty(gdn_recurrent_commit_verify_workspace_size(N, K1, K2, HV, dk),
+                     dtype=torch.uint8, device="cuda")
+    o2, u2 = gdn_recurrent_commit_verify(d1["k"], d1["g"], u1, accepted.cuda(), d2["q"], d2["k"],
+                                         d2["v"], d2["g"], d2["beta"], S, scale=0.9,
+                                         workspace=ws, prologue=prologue)
+    # the same round as two calls on the GPU
+    Sb = d1["state"].clone()
+    gdn_state_commit_deltas(d1["k"], d1["g"], u1, accepted.cuda(), Sb, prologue=prologue)
+    o2b, _, u2b = gdn_recurrent_verify(d2["q"], d2["k"], d2["v"], d2["g"], d2["beta"], Sb,
+                                       scale=0.9, rollback="deltas", prologue=prologue)
+    torch.cuda.synchronize()
+    assert gdn_read_status(ws) == 0
+    # against the oracle: commit of round 1, then verify of round 2
+    q1, k1, g1, b1 = O.prologue(x1["q"], x1["k"], x1["g"], x1["beta"], prologue)
+    _, st1 = O.verify(q1, k1, x1["v"], g1, b1, x1["state"])
+    acc = np.where(accepted.numpy() <= K1, accepted.numpy(), 0)
+    Sc = O.commit(st1, acc, x1["state"])
+    q2, k2, g2, b2 = O.prologue(x2["q"], x2["k"], x2["g"], x2["beta"], prologue)
+    o2_ref, _ = O.verify(q2, k2, x2["v"], g2, b2, Sc, scale=0.9)
+    assert_close(S, Sc, dtype, "committed state")
+    assert_close(o2, o2_ref, dtype, "o")
+    assert_close(o2, o2b.double().cpu().numpy(), dtype, "o vs two calls")
+    assert_close(u2, u2b.double().cpu().numpy(), dtype, "u vs two calls")
+    untouched = np.flatnonzero(acc == 0)
+    assert torch.equal(S[untouched], d1["state"][untouched])
