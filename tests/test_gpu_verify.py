@@ -235,3 +235,31 @@ def test_commit_verify_equals_commit_then_verify(N, K1, K2, HK, HV, dk, dv, dtyp
     assert_close(u2, u2b.double().cpu().numpy(), dtype, "u vs two calls")
     untouched = np.flatnonzero(acc == 0)
     assert torch.equal(S[untouched], d1["state"][untouched])
+
+
+def test_commit_verify_256x4_sampled_sequences():
+    """The benchmarked fused round at full size: 256 sequences x 4 drafts x 32 value
+    heads keep the previous round's ~U{0..4} accepted drafts and verify the next 4;
+    the oracle follows 4 sequences."""
+    from linear_attention_recurrence_rule_b200 import gdn_recurrent_commit_verify
+    from linear_attention_recurrence_rule_b200.inputs import WORKLOADS, workload_inputs
+    w = WORKLOADS["verify_256x4"]
+    x1 = workload_inputs("verify_256x4")
+    x2 = workload_inputs("verify_256x4", seed_offset=1)
+    d1, d2 = to_dev(x1), to_dev(x2)
+    gen = torch.Generator().manual_seed(w.seed + 77)
+    accepted = torch.randint(0, w.T + 1, (w.B,), generator=gen, dtype=torch.int32)
+    _, _, u1 = gdn_recurrent_verify(d1["q"], d1["k"], d1["v"], d1["g"], d1["beta"], d1["state"],
+                                    rollback="deltas")
+    S = d1["state"].clone()
+    o2, _ = gdn_recurrent_commit_verify(d1["k"], d1["g"], u1, accepted.cuda(), d2["q"], d2["k"],
+                                        d2["v"], d2["g"], d2["beta"], S)
+    torch.cuda.synchronize()
+    seqs = [0, 17, 128, 255]
+    s1 = {n: x1[n][seqs] for n in ("q", "k", "v", "g", "beta", "state")}
+    s2 = {n: x2[n][seqs] for n in ("q", "k", "v", "g", "beta")}
+    _, st1 = O.verify(s1["q"], s1["k"], s1["v"], s1["g"], s1["beta"], s1["state"])
+    Sc = O.commit(st1, accepted[seqs].numpy(), s1["state"])
+    o2_ref, _ = O.verify(s2["q"], s2["k"], s2["v"], s2["g"], s2["beta"], Sc)
+    assert_close(S[seqs], Sc, torch.bfloat16, "committed state")
+    assert_close(o2[seqs], o2_ref, torch.bfloat16, "o")
