@@ -463,7 +463,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
         "config": {"workload": WORKLOAD, "B": 1, "T": 65536, "HK": 16, "HV": 32, "d": 128,
-                   "chunk": 64, "parallelism": "replicas",
+                   "chunk": 64, "parallelism": "replicas" if world > 1 else "single",
                    "sample_tokens_per_step": tok},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(),
                          "kind": "oracle",

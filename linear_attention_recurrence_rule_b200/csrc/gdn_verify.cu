@@ -576,13 +576,15 @@ verify_wy_kernel(const Tin *__restrict__ v, float *state, float *__restrict__ ws
                     for (int q4 = 0; q4 < kVerifyF4; ++q4) s[jr][q4] = scale4(s[jr][q4], gam);
                     for (int t = 0; t < a; ++t) {
                         const float f = ub[t * BAND + r];
+                        const float2 ff = make_float2(f, f);
 #pragma unroll
                         for (int q4 = 0; q4 < kVerifyF4; ++q4) {
                             const float4 kk = pkt[t * D4 + li + LPR * q4];
-                            s[jr][q4].x = fmaf(f, kk.x, s[jr][q4].x);
-                            s[jr][q4].y = fmaf(f, kk.y, s[jr][q4].y);
-                            s[jr][q4].z = fmaf(f, kk.z, s[jr][q4].z);
-                            s[jr][q4].w = fmaf(f, kk.w, s[jr][q4].w);
+                            const float2 lo = fma2(ff, make_float2(kk.x, kk.y),
+                                                   make_float2(s[jr][q4].x, s[jr][q4].y));
+                            const float2 hi = fma2(ff, make_float2(kk.z, kk.w),
+                                                   make_float2(s[jr][q4].z, s[jr][q4].w));
+                            s[jr][q4] = make_float4(lo.x, lo.y, hi.x, hi.y);
                         }
                     }
                     if (r < rows) {
