@@ -222,7 +222,7 @@ def test_commit_verify_equals_commit_then_verify(N, K1, K2, HK, HV, dk, dv, dtyp
                                        scale=0.9, rollback="deltas", prologue=prologue)
     torch.cuda.synchronize()
     assert gdn_read_status(ws) == 0
-    # against the oracle: commit of round 1, then verify of round 2
+    # against the oracle: commit of the first drafts, then verify of the second
     q1, k1, g1, b1 = O.prologue(x1["q"], x1["k"], x1["g"], x1["beta"], prologue)
     _, st1 = O.verify(q1, k1, x1["v"], g1, b1, x1["state"])
     acc = np.where(accepted.numpy() <= K1, accepted.numpy(), 0)
