@@ -275,3 +275,34 @@ def verify_row_decay(q, k, v, g_rows, beta, state, scale=1.0):
         o[:, t], S = step_row_decay(q[:, t], k[:, t], v[:, t], g_rows[:, t], beta[:, t], S, scale)
         states[:, t] = S
     return o, states
+
+
+def prefill_row_decay(q, k, v, g_rows, beta, h0=None, cu_seqlens=None, scale=1.0):
+    """Token-by-token prefill with one decay per value row (see ``step_row_decay``),
+    float64, for small problems: q,k [B,T,HK,dk]; v, g_rows [B,T,HV,dv];
+    beta [B,T,HV]; h0 [N,HV,dv,dk] or None; cu_seqlens as in ``prefill``.
+    Returns (o [B*T,HV,dv], hT [N,HV,dv,dk])."""
+    q, k, v, g_rows, beta = (_f64(x) for x in (q, k, v, g_rows, beta))
+    B, T, HK, dk = q.shape
+    HV, dv = v.shape[2], v.shape[3]
+    if cu_seqlens is None:
+        bounds = [(b * T, (b + 1) * T) for b in range(B)]
+    else:
+        cu = np.asarray(_f64(cu_seqlens)).astype(np.int64)
+        bounds = [(int(cu[i]), int(cu[i + 1])) for i in range(len(cu) - 1)]
+    flat = lambda x: x.reshape((B * T,) + x.shape[2:])
+    q, k, v, g_rows, beta = (flat(x) for x in (q, k, v, g_rows, beta))
+    N = len(bounds)
+    S = np.zeros((N, HV, dv, dk)) if h0 is None else _f64(h0).copy()
+    o = np.zeros((B * T, HV, dv))
+    r = HV // HK
+    for n, (s0, s1) in enumerate(bounds):
+        for t in range(s0, s1):
+            for h in range(HV):
+                c = h // r
+                St = S[n, h] * np.exp(g_rows[t, h])[:, None]        # decay each row
+                u = beta[t, h] * (v[t, h] - St @ k[t, c])
+                St = St + np.outer(u, k[t, c])
+                S[n, h] = St
+                o[t, h] = scale * (St @ q[t, c])
+    return o, S

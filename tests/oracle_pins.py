@@ -468,6 +468,28 @@ def pin_row_decay_rows_are_independent(lib=None):
     assert changed[1, 0, 2] and changed.sum() == 1
 
 
+def pin_prefill_row_decay(lib=None):
+    """The sequential prefill with per-row decay equals the scalar C oracle when
+    every row shares its head's decay (packed sequences, nonzero h0), and equals
+    a run of ``step_row_decay`` calls with different decays per row."""
+    rng = np.random.default_rng(26)
+    q, k, v, g, beta = _rand_problem(rng, 9, 2, 4, 5, 3)
+    cu = np.array([0, 4, 9], dtype=np.int32)
+    h0 = rng.standard_normal((2, 4, 3, 5))
+    o1, h1 = O.prefill(q, k, v, g, beta, h0=h0, cu_seqlens=cu, scale=0.8, lib=lib)
+    o2, h2 = O.prefill_row_decay(q, k, v, np.repeat(g[..., None], 3, axis=-1), beta, h0=h0,
+                                 cu_seqlens=cu, scale=0.8)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(h1, h2, atol=1e-12)
+    gr = rng.uniform(np.log(0.5), 0.0, (1, 9, 4, 3))
+    o3, h3 = O.prefill_row_decay(q[:, :4], k[:, :4], v[:, :4], gr[:, :4], beta[:, :4],
+                                 h0=h0[:1], scale=0.8)
+    S = h0[:1]
+    for t in range(4):
+        ot, S = O.step_row_decay(q[:, t], k[:, t], v[:, t], gr[:, t], beta[:, t], S, scale=0.8)
+        assert np.allclose(o3[t], ot[0], atol=1e-13)
+    assert np.allclose(h3, S, atol=1e-13)
+
+
 def pin_verify_row_decay_equals_steps(lib=None):
     rng = np.random.default_rng(25)
     N, K, HK, HV, dk, dv = 2, 3, 1, 2, 4, 3
