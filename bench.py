@@ -263,7 +263,34 @@ def measure_prologue(gdn, torch, dev, stream, x, w, ws, o, hT, rank, barrier, ma
             b_.record(stream)
         torch.cuda.synchronize()
         res[tag] = statistics.mean(a_.elapsed_time(b_) for a_, b_ in evs)
+    # the chunked prefill with one decay per value row (CUDA-core path) on the 4K layer
+    from linear_attention_recurrence_rule_b200.inputs import workload_inputs as _wi
+    wl = WORKLOADS["layer_prefill_4k"]
+    z = {k_: (v_.to(dev) if isinstance(v_, torch.Tensor) else v_)
+         for k_, v_ in _wi("layer_prefill_4k", seed_offset=replica_seed_offset(rank)).items()}
+    gz = row_decays(tuple(z["v"].shape), seed=903 + rank).to(dev)
+    oz = torch.empty_like(z["v"])
+
+    def rd_prefill():
+        gdn.gdn_chunk_prefill(z["q"], z["k"], z["v"], gz, z["beta"], chunk=wl.chunk, o=oz,
+                              stream=stream, prologue=gdn.ROW_DECAY)
+
+    rd_prefill()
+    torch.cuda.synchronize()
+    rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(3)]
+    for a_, b_ in rev:
+        a_.record(stream)
+        rd_prefill()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    rd_ms = statistics.mean(a_.elapsed_time(b_) for a_, b_ in rev)
+    ztok = z["q"].shape[0] * z["q"].shape[1]
     return {"flags": "norm_q|norm_k|gate_logits",
+            "prefill_row_decay": {"workload": "layer_prefill_4k", "path": "cuda-core",
+                                  "ms_per_step": rd_ms, "value": ztok / (rd_ms / 1e3),
+                                  "unit": "tokens/s", "gpu_launches": 4,
+                                  "decays": "one per value row, alpha ~U(0.8, 1)"},
             "prefill": {"workload": WORKLOAD, "value": tokens * args.steps / (total_ms / 1e3),
                         "unit": "tokens/s", "ms_per_step": pf_s * 1e3,
                         "plain_ms_per_step": plain_s * 1e3,

@@ -113,10 +113,11 @@ GDN_API size_t gdn_chunk_prefill_workspace_size(int N, int64_t T, int HK, int HV
  * value row: [N][HV][dv] for gdn_recurrent_step_ex, [N][K][HV][dv] for
  * gdn_recurrent_verify and gdn_state_commit_deltas.  Each row i of a state
  * decays by its own alpha_i before the correction.  Supported by the decode
- * step, by verify when states_out is given, and by both commits; the chunked
- * prefill and the update-vector-only verify return GDN_ERR_UNSUPPORTED (their
- * per-head tables -- the chunk's triangular inverse, the mixed vectors -- would
- * become per row).
+ * step, by verify when states_out is given, by both commits, and by the chunked
+ * prefill (`g` [B][T][HV][dv]) on its CUDA-core path for every supported shape
+ * (the tensor-core path's per-head triangular inverse becomes per row, so it
+ * is not used); the update-vector-only verify and the fused commit-then-verify
+ * return GDN_ERR_UNSUPPORTED (their per-head mixed vectors would become per row).
  */
 #define GDN_ROW_DECAY 8u
 #define GDN_FLAGS_VALID 15u
@@ -167,7 +168,8 @@ GDN_API gdn_status gdn_chunk_prefill(const void *q, const void *k, const void *v
  * gdn_chunk_prefill with the input prologue fused (`prologue`: GDN_PROLOGUE_*
  * flags; 0 is exactly gdn_chunk_prefill).  With GDN_PROLOGUE_GATE_LOGITS, g
  * and beta hold the logits (any real values).  Unknown flag bits return
- * GDN_ERR_INVALID_ARG; GDN_ROW_DECAY returns GDN_ERR_UNSUPPORTED.
+ * GDN_ERR_INVALID_ARG; with GDN_ROW_DECAY (g [B][T][HV][dv]) the call runs on the
+ * CUDA-core path.
  */
 GDN_API gdn_status gdn_chunk_prefill_ex(const void *q, const void *k, const void *v,
                                         const float *g, const float *beta, const float *h0,

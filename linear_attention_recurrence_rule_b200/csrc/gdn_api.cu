@@ -43,7 +43,8 @@ gdn_status enqueue_prefill(const gdn::PrefillArgs &a, cudaStream_t stream) {
     if (st != GDN_OK) return st;
     if (a.N == 0) return GDN_OK;
     cudaError_t err;
-    if (tc_path(a.dk, a.dv, a.chunk, a.dtype)) {
+    // one decay per value row: only the CUDA-core path (a per-row triangular inverse)
+    if (tc_path(a.dk, a.dv, a.chunk, a.dtype) && !(a.prologue & GDN_ROW_DECAY)) {
         const size_t need = gdn::prefill_cluster_workspace(a.N, a.T, a.HV, a.chunk, a.cu_seqlens != nullptr);
         if (need > 0 && (a.workspace == nullptr || a.workspace_bytes < need)) return GDN_ERR_WORKSPACE;
         if (!aligned16(a.workspace)) return GDN_ERR_ALIGNMENT;
@@ -131,7 +132,8 @@ gdn_status gdn_chunk_prefill_ex(const void *q, const void *k, const void *v, con
                                 float scale, gdn_dtype dtype, void *o, float *hT, void *workspace,
                                 size_t workspace_bytes, unsigned prologue, gdn_stream_t stream) {
     if (prologue & ~GDN_FLAGS_VALID) return GDN_ERR_INVALID_ARG;
-    if (prologue & GDN_ROW_DECAY) return GDN_ERR_UNSUPPORTED;
+    if ((prologue & GDN_ROW_DECAY) && !gdn::prefill_simt_supported(dk, dv, chunk))
+        return GDN_ERR_UNSUPPORTED;
     gdn::PrefillArgs a{q, k, v, g, beta, h0, cu_seqlens, N, T, HK, HV, dk, dv, chunk,
                        scale, dtype, o, hT, workspace, workspace_bytes};
     a.prologue = prologue;

@@ -34,7 +34,9 @@ constexpr int kDecodeNB = 8;
 template <int DK>
 constexpr int band_rows() { return kDecodeWarps * (32 / (DK / 4)) * kDecodeNB; }
 
-template <int DK, typename Tin, bool PRO>
+// PRO: the input prologue flags are read; RD (implies PRO): one decay per value
+// row.  Separate instances, so neither costs the paths that do not use it.
+template <int DK, typename Tin, bool PRO, bool RD>
 __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ g, const float *__restrict__ beta, float *state,
@@ -50,7 +52,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 
     float4 kk = load4(k + ((size_t)n * HK + c) * DK + col);
     float4 qq = load4(q + ((size_t)n * HK + c) * DK + col);
-    const bool rowdec = PRO && (pro & GDN_ROW_DECAY) != 0;   // g: one entry per value row
+    constexpr bool rowdec = RD;   // g: one entry per value row
     const float graw = rowdec ? 0.f : g[nh], braw = beta[nh];
     const Tin *vrow = v + (size_t)nh * dv;
     Tin *orow = o + (size_t)nh * dv;
@@ -61,13 +63,13 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         const int base = blockIdx.y * rows_per_batch;
         // the state loads go out first: nothing below them waits on q, k
         float4 s[kDecodeNB];
-        float grow[kDecodeNB];   // per-row decays (GDN_ROW_DECAY), loaded with the state
+        float grow[RD ? kDecodeNB : 1];   // per-row decays (GDN_ROW_DECAY), loaded with the state
 #pragma unroll
         for (int j = 0; j < kDecodeNB; ++j) {
             const int row = base + (j * kDecodeWarps + warp) * RPI + sub;
             s[j] = row < dv ? __ldcs(reinterpret_cast<const float4 *>(S + (size_t)row * DK + col))
                             : make_float4(0.f, 0.f, 0.f, 0.f);
-            grow[j] = (rowdec && row < dv) ? g[(size_t)nh * dv + row] : 0.f;
+            if (RD) grow[RD ? j : 0] = row < dv ? g[(size_t)nh * dv + row] : 0.f;
         }
         if (PRO && (pro & (GDN_PROLOGUE_NORM_Q | GDN_PROLOGUE_NORM_K))) {
             // the lanes of a row hold the whole q and k: reduce the squared norms there
@@ -96,8 +98,9 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
                 sq += __shfl_xor_sync(0xffffffffu, sq, off);
             }
             if (row < dv) {
-                const float alpha = rowdec ? (logits ? gate_sigmoid(grow[j]) : expf(grow[j]))
-                                           : alpha_h;
+                const float alpha =
+                    rowdec ? (logits ? gate_sigmoid(grow[RD ? j : 0]) : expf(grow[RD ? j : 0]))
+                           : alpha_h;
                 const float u = b * (to_f32(vrow[row]) - alpha * sk);
                 float4 ns;
                 ns.x = fmaf(alpha, s[j].x, u * kk.x);
@@ -113,7 +116,9 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 
 template <int DK, typename Tin>
 void launch_dk(const StepArgs &a, dim3 grid, dim3 block, cudaStream_t stream) {
-    auto kern = a.prologue ? decode_kernel<DK, Tin, true> : decode_kernel<DK, Tin, false>;
+    auto kern = (a.prologue & GDN_ROW_DECAY) ? decode_kernel<DK, Tin, true, true>
+                : a.prologue                 ? decode_kernel<DK, Tin, true, false>
+                                             : decode_kernel<DK, Tin, false, false>;
     kern<<<grid, block, 0, stream>>>(static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
                                      static_cast<const Tin *>(a.v), a.g, a.beta, a.state,
                                      static_cast<Tin *>(a.o), a.HK, a.HV, a.dv, a.scale,

@@ -163,8 +163,9 @@ def gdn_chunk_prefill(q, k, v, g, beta, h0=None, cu_seqlens=None, chunk: int = 6
         raise ValueError("expected q,k [B,T,HK,dk] and v [B,T,HV,dv]")
     B, T, HK, dk = q.shape
     HV, dv = v.shape[2], v.shape[3]
-    if g.shape != (B, T, HV) or beta.shape != (B, T, HV):
-        raise ValueError("expected g, beta [B,T,HV]")
+    g_shape = (B, T, HV, dv) if prologue & ROW_DECAY else (B, T, HV)
+    if g.shape != g_shape or beta.shape != (B, T, HV):
+        raise ValueError(f"expected g {g_shape} and beta [B,T,HV]")
     if cu_seqlens is not None:
         _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
         if B != 1:

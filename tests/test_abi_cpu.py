@@ -194,8 +194,9 @@ def test_prologue_flags_are_validated(lib):
     assert verify_call(lib, pro=16) == gdn.GDN_ERR_INVALID_ARG
     # one decay per value row: decode and per-draft-state verify only
     assert re.search(r"#define GDN_ROW_DECAY 8u", text)
+    # (a supported shape would pass validation and launch: only rejected shapes here)
     assert lib.gdn_chunk_prefill_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], None, None, 1, 64,
-                                    1, 2, 32, 32, 16, 1.0, gdn.GDN_F32, fake(0x6000), None, None,
+                                    1, 2, 48, 32, 16, 1.0, gdn.GDN_F32, fake(0x6000), None, None,
                                     0, gdn.ROW_DECAY, None) == gdn.GDN_ERR_UNSUPPORTED
     need = lib.gdn_recurrent_verify_workspace_size(2, 4, 2, 128)
     assert verify_call(lib, states=None, ws=fake(0xa000), ws_bytes=need,

@@ -73,11 +73,35 @@ def test_verify_and_commits_row_decay(N, K, HK, HV, dk, dv, dtype):
     assert_close(S2, kept, dtype, "committed (deltas)")
 
 
-def test_row_decay_unsupported_forms():
-    x = make_prefill(1, 2, 32, 32, [64], torch.float32, seed=86)
+@pytest.mark.parametrize("extra", [0, PROLOGUE_ALL])
+@pytest.mark.parametrize("HK,HV,dk,dv,lengths,chunk,dtype", [
+    (1, 2, 32, 32, [150], 16, torch.float32),
+    (2, 2, 64, 64, [40, 100, 7], 32, torch.float32),         # packed, ragged
+    (2, 4, 128, 128, [130, 130], 64, torch.bfloat16),        # the tensor-core shape
+])
+def test_prefill_row_decay(HK, HV, dk, dv, lengths, chunk, dtype, extra):
+    """The chunked prefill with one decay per value row runs on the CUDA-core
+    path (the tensor-core path's per-head inverse does not apply)."""
+    base = make_prefill(HK, HV, dk, dv, lengths, dtype, seed=86, h0_std=0.2)
+    x = raw_projections(base, seed=87) if extra else base
+    B, T = x["q"].shape[0], x["q"].shape[1]
+    g_rows = row_decays((B, T, HV, dv), seed=88)
+    if extra & PROLOGUE_GATE_LOGITS:
+        a = torch.exp(g_rows)
+        g_rows = torch.log(a / (1 - a)).float()
     d = to_dev(x)
-    with pytest.raises(GDNError):
-        gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], chunk=16, prologue=ROW_DECAY)
+    o, hT = gdn_chunk_prefill(d["q"], d["k"], d["v"], g_rows.cuda(), d["beta"], h0=d["h0"],
+                              cu_seqlens=d["cu_seqlens"], chunk=chunk, scale=0.7,
+                              prologue=ROW_DECAY | extra)
+    torch.cuda.synchronize()
+    q, k, g, b = O.prologue(x["q"], x["k"], g_rows, x["beta"], extra)
+    o_ref, h_ref = O.prefill_row_decay(q, k, x["v"], g, b, h0=x["h0"], cu_seqlens=x["cu_seqlens"],
+                                       scale=0.7)
+    assert_close(o, o_ref, dtype, "o")
+    assert_close(hT, h_ref, dtype, "hT")
+
+
+def test_row_decay_unsupported_forms():
     y = make_verify(2, 3, 1, 2, 32, 32, torch.float32, seed=87)
     e = to_dev(y)
     g_rows = row_decays((2, 3, 2, 32), seed=88).cuda()
