@@ -90,7 +90,7 @@ __device__ __forceinline__ float gate_beta(float b, unsigned pro) {
     return (pro & GDN_PROLOGUE_GATE_LOGITS) ? gate_sigmoid(b) : b;
 }
 
-template <int DK, typename Tin, bool PRO>
+template <int DK, typename Tin, bool PRO, bool RD>
 __global__ void __launch_bounds__(kVerifyWarps * 32, 2)
 verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ g, const float *__restrict__ beta,
@@ -103,9 +103,9 @@ verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     __shared__ float4 ks[kVerifyMaxDrafts][DK / 4], qs[kVerifyMaxDrafts][DK / 4];
     __shared__ float vs[kVerifyMaxDrafts][BAND];
     __shared__ float al[kVerifyMaxDrafts], be[kVerifyMaxDrafts];
-    // per-row decays (GDN_ROW_DECAY), only in the prologue instance
-    __shared__ float ar[PRO ? kVerifyMaxDrafts : 1][PRO ? BAND : 1];
-    const bool rowdec = PRO && (pro & GDN_ROW_DECAY) != 0;
+    // per-row decays (GDN_ROW_DECAY), only in the row-decay instance
+    __shared__ float ar[RD ? kVerifyMaxDrafts : 1][RD ? BAND : 1];
+    constexpr bool rowdec = RD;
     const int nh = blockIdx.x;
     const int n = nh / HV, h = nh - n * HV;
     const int c = h / (HV / HK);
@@ -134,9 +134,9 @@ verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         const int t = idx / BAND, r = idx - t * BAND;
         const int row = base + r;
         vs[t][r] = row < dv ? to_f32(v[(((size_t)n * K + t) * HV + h) * dv + row]) : 0.f;
-        if (rowdec)
-            ar[t][r] = row < dv ? gate_alpha(g[(((size_t)n * K + t) * HV + h) * dv + row], pro)
-                                : 1.f;
+        if (RD)
+            ar[RD ? t : 0][RD ? r : 0] =
+                row < dv ? gate_alpha(g[(((size_t)n * K + t) * HV + h) * dv + row], pro) : 1.f;
     }
     if (threadIdx.x < K) {
         const size_t gi = ((size_t)n * K + threadIdx.x) * HV + h;
@@ -178,7 +178,7 @@ verify_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
                 sk += __shfl_xor_sync(0xffffffffu, sk, off);
                 sq += __shfl_xor_sync(0xffffffffu, sq, off);
             }
-            const float alpha = rowdec ? ar[t][r] : alpha_h;
+            const float alpha = rowdec ? ar[RD ? t : 0][RD ? r : 0] : alpha_h;
             const float u = b * (vs[t][r] - alpha * sk);
 #pragma unroll
             for (int i = 0; i < kVerifyF4; ++i) {
@@ -705,7 +705,7 @@ commit_kernel(const float *__restrict__ states, const int32_t *__restrict__ acce
 // element is read and written once; k_t and the scaled u_t of the band sit in
 // shared memory.  Same row layout and bands as the verify kernel; all of a lane's
 // state loads are issued before the staging and the arithmetic.
-template <int DK, typename Tin, bool PRO>
+template <int DK, typename Tin, bool PRO, bool RD>
 __global__ void __launch_bounds__(kVerifyWarps * 32, 3)
 commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
                      const float *__restrict__ u, const int32_t *__restrict__ accepted,
@@ -718,8 +718,8 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
     __shared__ float4 ks[kVerifyMaxDrafts][DK / 4];
     __shared__ float us[kVerifyMaxDrafts][BAND];
     __shared__ float coef[kVerifyMaxDrafts + 1];
-    __shared__ float gr[PRO ? BAND : 1];   // per-row decay products (GDN_ROW_DECAY)
-    const bool rowdec = PRO && (pro & GDN_ROW_DECAY) != 0;
+    __shared__ float gr[RD ? BAND : 1];   // per-row decay products (GDN_ROW_DECAY)
+    constexpr bool rowdec = RD;
     const int nh = blockIdx.x;
     const int n = nh / HV, h = nh - n * HV;
     const int c = h / (HV / HK);
@@ -764,7 +764,7 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
                 us[t][r] = row < dv ? c_run * u[e] : 0.f;
                 if (row < dv) c_run *= gate_alpha(g[e], pro);
             }
-            gr[r] = c_run;
+            gr[RD ? r : 0] = c_run;
         }
     } else {
         for (int i = threadIdx.x; i < a * BAND; i += blockDim.x) {
@@ -776,7 +776,8 @@ commit_deltas_kernel(const Tin *__restrict__ k, const float *__restrict__ g,
     __syncthreads();
 #pragma unroll
     for (int jr = 0; jr < kVerifyRows; ++jr) {
-        const float gam = rowdec ? gr[(jr * kVerifyWarps + warp) * RPW + sub] : coef[kVerifyMaxDrafts];
+        const float gam =
+            rowdec ? gr[RD ? (jr * kVerifyWarps + warp) * RPW + sub : 0] : coef[kVerifyMaxDrafts];
 #pragma unroll
         for (int i = 0; i < kVerifyF4; ++i) {
             x[jr][i].x *= gam; x[jr][i].y *= gam; x[jr][i].z *= gam; x[jr][i].w *= gam;
@@ -866,7 +867,9 @@ void launch_verify_wy_k(const VerifyArgs &a, dim3 block, cudaStream_t stream) {
 
 template <int DK, typename Tin>
 void launch_verify_seq(const VerifyArgs &a, dim3 grid, dim3 block, cudaStream_t stream) {
-    auto kern = a.prologue ? verify_kernel<DK, Tin, true> : verify_kernel<DK, Tin, false>;
+    auto kern = (a.prologue & GDN_ROW_DECAY) ? verify_kernel<DK, Tin, true, true>
+                : a.prologue                 ? verify_kernel<DK, Tin, true, false>
+                                             : verify_kernel<DK, Tin, false, false>;
     kern<<<grid, block, 0, stream>>>(static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
                                      static_cast<const Tin *>(a.v), a.g, a.beta, a.state,
                                      a.states, a.u, static_cast<Tin *>(a.o), a.K, a.HK, a.HV,
@@ -913,7 +916,9 @@ cudaError_t launch_verify(const VerifyArgs &a, cudaStream_t stream) {
 
 template <int DK, typename Tin>
 void launch_commit_dk(const CommitDeltasArgs &a, dim3 grid, dim3 block, cudaStream_t stream) {
-    auto kern = a.prologue ? commit_deltas_kernel<DK, Tin, true> : commit_deltas_kernel<DK, Tin, false>;
+    auto kern = (a.prologue & GDN_ROW_DECAY) ? commit_deltas_kernel<DK, Tin, true, true>
+                : a.prologue                 ? commit_deltas_kernel<DK, Tin, true, false>
+                                             : commit_deltas_kernel<DK, Tin, false, false>;
     kern<<<grid, block, 0, stream>>>(static_cast<const Tin *>(a.k), a.g, a.u, a.accepted, a.state,
                                      a.K, a.HK, a.HV, a.dv, a.prologue);
 }
