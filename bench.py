@@ -149,8 +149,8 @@ def measure_verify(gdn, torch, dev, stream, peaks, peak_src, rank, world, max_ov
         "value": world * N * K * rounds / (ftotal / 1e3), "unit": "draft tokens/s",
         "ms_per_round": ftotal / rounds, "bytes_per_round": fb,
         "roofline": {"bound": "hbm", "achieved": f_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": f_gbs / hbm_peak, "traffic": None, "peak_source": peak_src,
-                     "kernel": "verify_wy (commit fused)"},
+                     "frac": f_gbs / hbm_peak, "traffic": kernel_traffic("verify_fused"),
+                     "peak_source": peak_src, "kernel": "verify_wy (commit fused)"},
         "gpu_launches": 2 * rounds, "clocks": fclocks,
         "call": "gdn_recurrent_commit_verify: previous round's commit + this round's verify"}
     for form in ("deltas", "states"):
@@ -341,19 +341,23 @@ def load_peaks():
 # Each entry carries the sha256 of the kernel source it was taken on; a changed
 # source reports null.
 NCU_TRAFFIC = {
-    # full decode_256x64 step: 541,146,880 read + 476,584,192 written
-    "decode": {"bytes": 1017731072, "source": "gdn_decode.cu",
-               "sha256": "2b41374aacd6222f16e152e67df8cb51675c5fc07d35104e4c0cbf61c6d22621"},
-    # full long_prefill_64k launch: 1,090,664,192 read + 510,390,784 written
-    "prefill_cluster": {"bytes": 1601054976, "source": "gdn_prefill_cluster.cu",
+    # full decode_256x64 step: 541,153,280 read + 476,171,776 written
+    "decode": {"bytes": 1017325056, "source": "gdn_decode.cu",
+               "sha256": "dbfc71d8d19d220e31d8f0247d1d42e64f4c5c310b09be07c69e4f71ee4d6aa7"},
+    # full long_prefill_64k launch: 1,090,822,656 read + 511,207,936 written
+    "prefill_cluster": {"bytes": 1602030592, "source": "gdn_prefill_cluster.cu",
                         "sha256": "881a325e6d56777fe19db569636ec05bdd86d18a1d8dea300fed5c5991d89ae0"},
-    # verify_256x4, update-vector form, the streaming kernel: 579,901,696 read + 21,873,920
-    # written (its setup kernel adds 8,680,192)
-    "verify_deltas": {"bytes": 601775616, "source": "gdn_verify.cu",
-                      "sha256": "f653b5a19667221bcad35290a382fdd867b7d01015b48c9285dce05bd87c36b7"},
-    # verify_256x4, per-draft states: 554,840,832 read + 2,093,378,048 written
-    "verify_states": {"bytes": 2648218880, "source": "gdn_verify.cu",
-                      "sha256": "f653b5a19667221bcad35290a382fdd867b7d01015b48c9285dce05bd87c36b7"},
+    # verify_256x4, update-vector form, the streaming kernel: 580,045,056 read + 20,497,408
+    # written (its setup kernel adds 8,682,752)
+    "verify_deltas": {"bytes": 600542464, "source": "gdn_verify.cu",
+                      "sha256": "91513df491cd0f01d3b155b705eebd9cac03e5f9dcac91a98a1150bc941ade38"},
+    # verify_256x4, per-draft states: 554,970,880 read + 2,093,050,368 written
+    "verify_states": {"bytes": 2648021248, "source": "gdn_verify.cu",
+                      "sha256": "91513df491cd0f01d3b155b705eebd9cac03e5f9dcac91a98a1150bc941ade38"},
+    # verify_256x4 fused round (previous commit + verify), the streaming kernel:
+    # 613,578,752 read + 382,084,864 written
+    "verify_fused": {"bytes": 995663616, "source": "gdn_verify.cu",
+                     "sha256": "91513df491cd0f01d3b155b705eebd9cac03e5f9dcac91a98a1150bc941ade38"},
 }
 
 
