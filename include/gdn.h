@@ -297,9 +297,9 @@ GDN_API gdn_status gdn_recurrent_step_ex(const void *q, const void *k, const voi
 #define GDN_VERIFY_MAX_DRAFTS 16
 
 /*
- * Multi-token verify step for speculative decoding (Qwen3-Next, "Speed depends
- * on the serving software": the model checks several proposed tokens at once
- * and keeps those it agrees with).  For each of N sequences, K draft tokens
+ * Multi-token verify step for speculative decoding (Qwen3-Next, section "Speed
+ * depends on the serving software": drafted tokens are verified together and
+ * only an accepted prefix is kept).  For each of N sequences, K draft tokens
  * are run through the recurrence of gdn_recurrent_step one after another,
  * starting from `state`, which is only read (once, from HBM, for all K
  * tokens).  Every token's output is written; for rolling back to the last

@@ -2,8 +2,8 @@
 // roll-back calls that keep the accepted prefix.
 //
 // Speculative decoding ("Qwen3-Next", sghael.github.io, section "Speed depends on
-// the serving software"): the model checks several proposed tokens at once and
-// keeps those it agrees with.  For the recurrence that means running K draft
+// the serving software"): drafted tokens are verified together and only an
+// accepted prefix is kept.  For the recurrence that means running K draft
 // tokens through the decode rule from one state, then keeping the state after
 // the last accepted draft.
 //

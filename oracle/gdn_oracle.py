@@ -167,8 +167,8 @@ def step(q, k, v, g, beta, state, scale=1.0, lib=None):
 
 
 def verify(q, k, v, g, beta, state, scale=1.0, lib=None):
-    """K draft tokens per sequence, checked at once (speculative decoding: the
-    main model processes several proposed tokens and keeps those it accepts --
+    """K draft tokens per sequence, checked at once (speculative decoding, where
+    drafted tokens are verified together and only an accepted prefix is kept --
     "Qwen3-Next", sghael.github.io, section "Speed depends on the serving
     software").  The rule is applied token after token from ``state``; the
     outputs of every token and the state after every token are returned, so a

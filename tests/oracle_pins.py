@@ -99,7 +99,8 @@ def pin_worked_example_gated(lib=None):
 # ----------------------------------------------------------------------------
 def pin_converges_closed_form(lib=None):
     """No decay, one repeated unit key: S_n k = v + (1-b)^n (S_0 k - v) (the page's
-    "converges on 10"), and directions orthogonal to k are never touched."""
+    example approaching the target 10), and directions orthogonal to k are never
+    touched."""
     rng = np.random.default_rng(1)
     dk, dv, T, b = 5, 3, 12, 0.3
     kvec = rng.standard_normal(dk); kvec /= np.linalg.norm(kvec)
