@@ -350,14 +350,14 @@ NCU_TRAFFIC = {
     # verify_256x4, update-vector form, the streaming kernel: 580,045,056 read + 20,497,408
     # written (its setup kernel adds 8,682,752)
     "verify_deltas": {"bytes": 600542464, "source": "gdn_verify.cu",
-                      "sha256": "91513df491cd0f01d3b155b705eebd9cac03e5f9dcac91a98a1150bc941ade38"},
+                      "sha256": "06a1ca667c8f672649db772cc989cae84bf6fba0a1cad2bfdee72a098788d42c"},
     # verify_256x4, per-draft states: 554,970,880 read + 2,093,050,368 written
     "verify_states": {"bytes": 2648021248, "source": "gdn_verify.cu",
-                      "sha256": "91513df491cd0f01d3b155b705eebd9cac03e5f9dcac91a98a1150bc941ade38"},
+                      "sha256": "06a1ca667c8f672649db772cc989cae84bf6fba0a1cad2bfdee72a098788d42c"},
     # verify_256x4 fused round (previous commit + verify), the streaming kernel:
     # 613,578,752 read + 382,084,864 written
     "verify_fused": {"bytes": 995663616, "source": "gdn_verify.cu",
-                     "sha256": "91513df491cd0f01d3b155b705eebd9cac03e5f9dcac91a98a1150bc941ade38"},
+                     "sha256": "06a1ca667c8f672649db772cc989cae84bf6fba0a1cad2bfdee72a098788d42c"},
 }
 
 
