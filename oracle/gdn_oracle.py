@@ -306,3 +306,113 @@ def prefill_row_decay(q, k, v, g_rows, beta, h0=None, cu_seqlens=None, scale=1.0
                 S[n, h] = St
                 o[t, h] = scale * (St @ q[t, c])
     return o, S
+
+
+# ----------------------------------------------------------------------------
+# The layer steps around the rule: a short convolution on the values before it
+# and an output gate after it ("Qwen3-Next", sghael.github.io, section "Linear
+# attention with gated delta rule": the values pass through a 1-D convolution
+# that adds local context, and a gate scales what the recurrence returns).
+# The pages give neither the convolution's width nor the gate's form.  Reading:
+#   * a causal depthwise convolution along time, one kernel of width W per
+#     value channel (channel = h * dv + i), tap j multiplying the input W-1-j
+#     tokens back, an optional bias and an optional SiLU after it; inputs
+#     before a sequence's first token come from a carried convolution state
+#     (the last W-1 inputs of the previous call) or are zero;
+#   * an elementwise sigmoid gate on the read-out, o <- o * sigmoid(z), with
+#     one gate logit per output element (the same page's attention layers use
+#     a sigmoid gate).
+# ----------------------------------------------------------------------------
+def silu(x):
+    """x * sigmoid(x) in float64, without overflow for large |x|."""
+    x = _f64(x)
+    return x * np.exp(-np.logaddexp(0.0, -x))
+
+
+def short_conv(x, weight, bias=None, conv_state=None, cu_seqlens=None, activation="none"):
+    """Causal depthwise convolution of each sequence along time.
+
+    x [B,T,C] (B sequences of T tokens) or packed [1,Ttot,C] / [Ttot,C] with
+    ``cu_seqlens`` (N+1 offsets); weight [C,W]; bias [C] or None; conv_state
+    [N,W-1,C] (row m = the input W-1-m tokens before the sequence's first
+    token) or None (zeros).  For token t of a sequence, with x_s = the input at
+    token s (s < 0 read from the state):
+        y_t = bias + sum_{j=0}^{W-1} weight[:, j] * x_{t-(W-1)+j}
+    then SiLU when ``activation == "silu"``.
+    Returns (y [Ttot,C], new_state [N,W-1,C]): the last W-1 inputs of each
+    sequence, taken from the old state where the sequence is shorter than W-1.
+    """
+    x, w = _f64(x), _f64(weight)
+    C, W = w.shape
+    if cu_seqlens is None and x.ndim == 3:
+        B, T = x.shape[0], x.shape[1]
+        bounds = [(b * T, (b + 1) * T) for b in range(B)]
+    else:
+        cu = np.asarray(_f64(cu_seqlens)).astype(np.int64)
+        bounds = [(int(cu[i]), int(cu[i + 1])) for i in range(len(cu) - 1)]
+    x = x.reshape(-1, C)
+    N = len(bounds)
+    hist = np.zeros((N, W - 1, C)) if conv_state is None else _f64(conv_state).reshape(N, W - 1, C)
+    b = np.zeros(C) if bias is None else _f64(bias)
+    y = np.zeros_like(x)
+    new_state = np.zeros((N, W - 1, C))
+    for n, (s0, s1) in enumerate(bounds):
+        L = s1 - s0
+        xs = np.concatenate([hist[n], x[s0:s1]], axis=0)     # tokens s0-(W-1) .. s1-1
+        acc = np.tile(b, (L, 1))
+        for j in range(W):
+            acc = acc + w[:, j] * xs[j:j + L]
+        y[s0:s1] = silu(acc) if activation == "silu" else acc
+        new_state[n] = xs[L:L + W - 1]
+    return y, new_state
+
+
+def output_gate(o, z):
+    """o * sigmoid(z), elementwise, float64 (shapes must match)."""
+    o, z = _f64(o), _f64(z)
+    return o * np.exp(-np.logaddexp(0.0, -z))
+
+
+def layer_prefill(q, k, v, g, beta, conv_weight=None, conv_bias=None, conv_state=None, z=None,
+                  h0=None, cu_seqlens=None, scale=1.0, activation="none", flags=0):
+    """The rule with the steps around it, over whole sequences: the prologue
+    (``flags``), the short convolution on v (when ``conv_weight`` is given),
+    the prefill, and the output gate (when ``z`` is given).  Shapes as in
+    ``prefill``; conv_weight [HV*dv, W]; conv_state [N, W-1, HV*dv]; z like v.
+    Returns (o [Ttot,HV,dv], hT, new_conv_state or None)."""
+    q, k, g, beta = prologue(q, k, g, beta, flags)
+    v = _f64(v)
+    new_cs = None
+    if conv_weight is not None:
+        vs = v.shape
+        C = vs[-2] * vs[-1]
+        if cu_seqlens is None and v.ndim == 4:
+            xv = v.reshape(vs[0], vs[1], C)
+        else:
+            xv = v.reshape(-1, C)
+        vc, new_cs = short_conv(xv, conv_weight, conv_bias, conv_state, cu_seqlens, activation)
+        v = vc.reshape(vs)
+    o, hT = prefill(q, k, v, g, beta, h0=h0, cu_seqlens=cu_seqlens, scale=scale)
+    if z is not None:
+        o = output_gate(o, _f64(z).reshape(o.shape))
+    return o, hT, new_cs
+
+
+def layer_step(q, k, v, g, beta, state, conv_weight=None, conv_bias=None, conv_state=None,
+               z=None, scale=1.0, activation="none", flags=0):
+    """One decode token per sequence with the steps around the rule (see
+    ``layer_prefill``).  q,k [N,HK,dk]; v, z [N,HV,dv]; g, beta [N,HV];
+    state [N,HV,dv,dk]; conv_state [N,W-1,HV*dv].
+    Returns (o [N,HV,dv], new_state, new_conv_state or None)."""
+    q, k, g, beta = prologue(q, k, g, beta, flags)
+    v = _f64(v)
+    new_cs = None
+    if conv_weight is not None:
+        N, HV, dv = v.shape
+        vc, new_cs = short_conv(v.reshape(N, 1, HV * dv), conv_weight, conv_bias, conv_state,
+                                activation=activation)
+        v = vc.reshape(N, HV, dv)
+    o, S = step(q, k, v, g, beta, state, scale=scale)
+    if z is not None:
+        o = output_gate(o, z)
+    return o, S, new_cs

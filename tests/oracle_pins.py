@@ -506,4 +506,127 @@ def pin_verify_row_decay_equals_steps(lib=None):
         assert np.array_equal(o[:, t], ot) and np.array_equal(states[:, t], S)
 
 
+
+# ----------------------------------------------------------------------------
+# The short convolution on the values and the output gate around the rule
+# ("Qwen3-Next", sghael.github.io, section "Linear attention with gated delta
+# rule"; widths and forms are readings, see the oracle's section header)
+# ----------------------------------------------------------------------------
+def pin_short_conv_is_a_library_convolution(lib=None):
+    """Per channel the causal convolution equals numpy's full convolution of the
+    input (with the carried state in front) with the reversed kernel, cut to the
+    sequence's tokens; with no state the missing history is zero."""
+    rng = np.random.default_rng(31)
+    B, T, C, W = 2, 11, 5, 4
+    x = rng.standard_normal((B, T, C))
+    w = rng.standard_normal((C, W))
+    st = rng.standard_normal((B, W - 1, C))
+    y0, _ = O.short_conv(x, w)
+    y1, _ = O.short_conv(x, w, conv_state=st)
+    for b in range(B):
+        for c in range(C):
+            ref0 = np.convolve(x[b, :, c], w[c, ::-1])[:T]
+            full = np.concatenate([st[b, :, c], x[b, :, c]])
+            ref1 = np.convolve(full, w[c, ::-1])[W - 1:W - 1 + T]
+            assert np.allclose(y0[b * T:(b + 1) * T, c], ref0, atol=1e-13)
+            assert np.allclose(y1[b * T:(b + 1) * T, c], ref1, atol=1e-13)
+
+
+def pin_short_conv_impulse_response(lib=None):
+    """A unit impulse at token t0 of channel c comes out as the kernel read
+    backwards: y_{t0+d} = w[c, W-1-d] for d < W, zero before t0 and after
+    t0+W-1 and on every other channel; the bias adds a constant; SiLU maps 0 to
+    0 and 1 to 1/(1+e^-1)."""
+    C, W, T, t0, c = 3, 4, 10, 3, 1
+    w = np.arange(1.0, C * W + 1).reshape(C, W)
+    x = np.zeros((1, T, C))
+    x[0, t0, c] = 1.0
+    y, st = O.short_conv(x, w)
+    expect = np.zeros((T, C))
+    for d in range(W):
+        expect[t0 + d, c] = w[c, W - 1 - d]
+    assert np.array_equal(y, expect)
+    assert np.array_equal(st[0], x[0, T - (W - 1):])
+    bias = np.array([0.5, -1.0, 2.0])
+    yb, _ = O.short_conv(x, w, bias=bias)
+    assert np.array_equal(yb, expect + bias)
+    ys, _ = O.short_conv(x, w, activation="silu")
+    assert ys[0, 0] == 0.0
+    one = np.zeros((1, 1, 1))
+    one[0, 0, 0] = 1.0
+    y1, _ = O.short_conv(one, np.ones((1, 1)), activation="silu")
+    assert abs(y1[0, 0] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-15
+
+
+def pin_short_conv_state_carry(lib=None):
+    """Cutting a sequence anywhere (also before W-1 tokens) and carrying the
+    state gives the same outputs and final state as one call; packed sequences
+    with cu_seqlens equal separate calls, an empty sequence passes its state
+    through unchanged."""
+    rng = np.random.default_rng(32)
+    T, C, W = 9, 3, 4
+    x = rng.standard_normal((1, T, C))
+    w = rng.standard_normal((C, W))
+    b = rng.standard_normal(C)
+    st = rng.standard_normal((1, W - 1, C))
+    y, s_end = O.short_conv(x, w, b, st, activation="silu")
+    for a in range(T + 1):
+        ya, sa = O.short_conv(x[:, :a], w, b, st, activation="silu")
+        yb, sb = O.short_conv(x[:, a:], w, b, sa, activation="silu")
+        assert np.allclose(np.concatenate([ya, yb]), y, atol=1e-14)
+        assert np.allclose(sb, s_end, atol=0.0)
+    lens = [4, 0, 1, 7]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    xp = rng.standard_normal((1, int(cu[-1]), C))
+    stp = rng.standard_normal((len(lens), W - 1, C))
+    yp, sp = O.short_conv(xp, w, b, stp, cu_seqlens=cu)
+    for n, L in enumerate(lens):
+        yn, sn = O.short_conv(xp[:, cu[n]:cu[n + 1]], w, b, stp[n:n + 1])
+        assert np.array_equal(yp[cu[n]:cu[n + 1]], yn) and np.array_equal(sp[n], sn[0])
+    assert np.array_equal(sp[1], stp[1])
+    # one token: the state shifts by one and takes the token last
+    assert np.array_equal(sp[2], np.concatenate([stp[2, 1:], xp[0, 4:5]]))
+
+
+def pin_output_gate(lib=None):
+    """sigmoid(0) = 1/2 halves the read-out; a large positive logit passes it,
+    a large negative one closes it; gate(o, z) + gate(o, -z) = o."""
+    rng = np.random.default_rng(33)
+    o = rng.standard_normal((4, 3, 5))
+    z = rng.standard_normal((4, 3, 5)) * 3.0
+    assert np.array_equal(O.output_gate(o, np.zeros_like(o)), o / 2)
+    assert np.allclose(O.output_gate(o, np.full_like(o, 40.0)), o, rtol=1e-15, atol=0)
+    assert np.all(np.abs(O.output_gate(o, np.full_like(o, -40.0))) < 1e-17 * np.abs(o) + 1e-300)
+    assert np.allclose(O.output_gate(o, z) + O.output_gate(o, -z), o, atol=1e-15)
+    assert np.all(np.abs(O.output_gate(o, z)) <= np.abs(o))
+
+
+def pin_layer_prefill_equals_layer_steps(lib=None):
+    """The layer over a sequence (convolution, rule, gate) equals one decode
+    step per token with both states carried; a pass-through kernel (last tap 1,
+    others 0) with no gate is the plain rule."""
+    rng = np.random.default_rng(34)
+    N, T, HK, HV, dk, dv, W = 2, 6, 1, 2, 4, 3, 4
+    q, k, v, g, beta = _rand_problem(rng, T, HK, HV, dk, dv)
+    q, k, v, g, beta = (np.repeat(a, N, axis=0) * (1.0 + 0.1 * np.arange(N)).reshape(
+        (N,) + (1,) * (a.ndim - 1)) if a is v else np.repeat(a, N, axis=0) for a in (q, k, v, g, beta))
+    w = rng.standard_normal((HV * dv, W))
+    cb = rng.standard_normal(HV * dv)
+    cs = rng.standard_normal((N, W - 1, HV * dv))
+    z = rng.standard_normal((N, T, HV, dv))
+    h0 = rng.standard_normal((N, HV, dv, dk)) * 0.3
+    o, hT, cs_end = O.layer_prefill(q, k, v, g, beta, w, cb, cs, z, h0=h0, scale=0.9,
+                                    activation="silu")
+    S, c = h0, cs
+    for t in range(T):
+        ot, S, c = O.layer_step(q[:, t], k[:, t], v[:, t], g[:, t], beta[:, t], S, w, cb, c,
+                                z[:, t], scale=0.9, activation="silu")
+        assert np.allclose(o.reshape(N, T, HV, dv)[:, t], ot, atol=1e-12)
+    assert np.allclose(hT, S, atol=1e-12) and np.allclose(cs_end, c, atol=0.0)
+    wid = np.zeros((HV * dv, W))
+    wid[:, W - 1] = 1.0
+    o1, h1, _ = O.layer_prefill(q, k, v, g, beta, wid, None, cs, None, h0=h0, scale=0.9)
+    o2, h2 = O.prefill(q, k, v, g, beta, h0=h0, scale=0.9, lib=lib)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(h1, h2, atol=1e-12)
+
 ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

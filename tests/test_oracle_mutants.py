@@ -165,3 +165,81 @@ def test_row_decay_pins_catch_mutant(monkeypatch, kind):
         except (AssertionError, ValueError):
             caught.append(pin.__name__)
     assert caught, f"no pin detects the planted row-decay mistake {kind}"
+
+
+# Mistakes planted in the short convolution and the output gate (plain numpy),
+# each caught by one of their pins.
+def _conv_mutant(kind):
+    import numpy as np
+
+    def mutant(x, weight, bias=None, conv_state=None, cu_seqlens=None, activation="none"):
+        x, w = O._f64(x), O._f64(weight)
+        C, W = w.shape
+        if cu_seqlens is None and x.ndim == 3:
+            B, T = x.shape[0], x.shape[1]
+            bounds = [(b * T, (b + 1) * T) for b in range(B)]
+        else:
+            cu = np.asarray(O._f64(cu_seqlens)).astype(np.int64)
+            bounds = [(int(cu[i]), int(cu[i + 1])) for i in range(len(cu) - 1)]
+        x = x.reshape(-1, C)
+        N = len(bounds)
+        hist = (np.zeros((N, W - 1, C)) if conv_state is None or kind == "state_ignored"
+                else O._f64(conv_state).reshape(N, W - 1, C))
+        b = np.zeros(C) if bias is None or kind == "bias_dropped" else O._f64(bias)
+        y = np.zeros_like(x)
+        new_state = np.zeros((N, W - 1, C))
+        for n, (s0, s1) in enumerate(bounds):
+            L = s1 - s0
+            xs = np.concatenate([hist[n], x[s0:s1]], axis=0)
+            acc = np.tile(b, (L, 1))
+            for j in range(W):
+                wj = w[:, W - 1 - j] if kind == "taps_reversed" else w[:, j]
+                if kind == "one_token_late":
+                    src = np.concatenate([np.zeros((1, C)), xs])[j:j + L]
+                else:
+                    src = xs[j:j + L]
+                acc = acc + wj * src
+            if activation == "silu":
+                acc = (1.0 / (1.0 + np.exp(-acc))) if kind == "silu_as_sigmoid" else O.silu(acc)
+            y[s0:s1] = acc
+            new_state[n] = xs[:W - 1] if kind == "state_from_first_tokens" else xs[L:L + W - 1]
+        return y, new_state
+    return mutant
+
+
+@pytest.mark.parametrize("kind", ["taps_reversed", "one_token_late", "state_ignored",
+                                  "bias_dropped", "silu_as_sigmoid", "state_from_first_tokens"])
+def test_conv_pins_catch_mutant(monkeypatch, kind):
+    monkeypatch.setattr(O, "short_conv", _conv_mutant(kind))
+    caught = []
+    for pin in ALL_PINS:
+        if "conv" not in pin.__name__ and "layer" not in pin.__name__:
+            continue
+        try:
+            pin()
+        except (AssertionError, ValueError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin detects the planted convolution mistake {kind}"
+
+
+@pytest.mark.parametrize("kind", ["tanh_gate", "one_minus_sigmoid", "gate_on_logit_only"])
+def test_gate_pins_catch_mutant(monkeypatch, kind):
+    import numpy as np
+
+    def mutant(o, z):
+        o, z = O._f64(o), O._f64(z)
+        if kind == "tanh_gate":
+            return o * np.tanh(z)
+        if kind == "one_minus_sigmoid":
+            return o * (1.0 - 1.0 / (1.0 + np.exp(-z)))
+        return o + (1.0 / (1.0 + np.exp(-z)))
+    monkeypatch.setattr(O, "output_gate", mutant)
+    caught = []
+    for pin in ALL_PINS:
+        if "gate" not in pin.__name__ and "layer" not in pin.__name__:
+            continue
+        try:
+            pin()
+        except (AssertionError, ValueError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin detects the planted gate mistake {kind}"
