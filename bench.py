@@ -306,6 +306,117 @@ def measure_prologue(gdn, torch, dev, stream, x, w, ws, o, hT, rank, barrier, ma
                       "write logits ~N(0, 1)"}
 
 
+def _time_events(torch, stream, fn, reps, warm=3):
+    """Mean CUDA-event time (ms) of ``fn`` on ``stream`` over ``reps`` launches."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for a_, b_ in ev:
+        a_.record(stream)
+        fn()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(a_.elapsed_time(b_) for a_, b_ in ev)
+
+
+def measure_layer(gdn, torch, dev, stream, x, w, o, hT, rank, peaks, peak_src, plain_s, args):
+    """The layer steps around the rule: the bench prefill with the short
+    convolution on v (width 4, SiLU, carried state) and the output gate, one
+    call; the convolution and the gate kernels alone with their HBM rooflines;
+    and the decode step of decode_256x64 with both fused into it."""
+    from linear_attention_recurrence_rule_b200.inputs import (WORKLOADS, layer_extras,
+                                                              workload_inputs)
+    W = 4
+    B, T, HV, dv = x["v"].shape
+    C = HV * dv
+    ex = layer_extras(B, C, W, tuple(x["v"].shape), torch.bfloat16, seed=950 + rank)
+    e = {k: v.to(dev) for k, v in ex.items()}
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    tokens = B * T
+    ws = torch.empty(gdn.gdn_chunk_prefill_layer_workspace_size(
+        B, T, w.HK, w.HV, w.dk, w.dv, w.chunk, w.dtype, 0, 1), dtype=torch.uint8, device=dev)
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+
+    def layer_prefill():
+        gdn.gdn_chunk_prefill_layer(d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                    conv_weight=e["conv_weight"], conv_bias=e["conv_bias"],
+                                    conv_state=e["conv_state"], z=e["z"], chunk=w.chunk, o=o,
+                                    hT=hT, workspace=ws, stream=stream, silu=True)
+
+    lp_ms = _time_events(torch, stream, layer_prefill, max(args.steps, 3))
+    y = torch.empty_like(d["v"])
+    vin = d["v"].reshape(B, T, C)
+
+    def conv():
+        gdn.gdn_short_conv(vin, e["conv_weight"], e["conv_bias"], e["conv_state"], silu=True,
+                           y=y.reshape(B, T, C), stream=stream)
+
+    cv_ms = _time_events(torch, stream, conv, 10)
+    elt = 2
+    cv_bytes = 2 * tokens * C * elt + 2 * B * (W - 1) * C * elt + C * (W + 1) * 4
+
+    def gate():
+        gdn.gdn_output_gate(o, e["z"], stream=stream)
+
+    gt_ms = _time_events(torch, stream, gate, 10)
+    gt_bytes = 3 * tokens * C * elt
+    del d, y, ws
+    # decode with both steps fused, 256 sequences (decode_256x64 shapes)
+    wd = WORKLOADS[DECODE_WORKLOAD]
+    yd = workload_inputs(DECODE_WORKLOAD, steps=8, seed_offset=replica_seed_offset(rank))
+    dy = {k: v.to(dev) for k, v in yd.items()}
+    exd = layer_extras(wd.B, wd.HV * wd.dv, W, (8, wd.B, wd.HV, wd.dv), torch.bfloat16,
+                       seed=960 + rank)
+    ed = {k: v.to(dev) for k, v in exd.items()}
+    S = dy["state"].clone()
+    od = torch.empty_like(dy["v"][0])
+    it = [0]
+
+    def dstep(layer):
+        t = it[0] % 8
+        it[0] += 1
+        if layer:
+            gdn.gdn_recurrent_step_layer(dy["q"][t], dy["k"][t], dy["v"][t], dy["g"][t],
+                                         dy["beta"][t], S, conv_weight=ed["conv_weight"],
+                                         conv_bias=ed["conv_bias"], conv_state=ed["conv_state"],
+                                         z=ed["z"][t], o=od, stream=stream, silu=True)
+        else:
+            gdn.gdn_recurrent_step(dy["q"][t], dy["k"][t], dy["v"][t], dy["g"][t], dy["beta"][t],
+                                   S, o=od, stream=stream)
+
+    plain_d = _time_events(torch, stream, lambda: dstep(False), 8)
+    layer_d = _time_events(torch, stream, lambda: dstep(True), 8)
+    dbytes = (decode_bytes_per_step(wd.B, wd.HK, wd.HV, wd.dk, wd.dv)
+              + 2 * wd.B * (W - 1) * wd.HV * wd.dv * elt + wd.B * wd.HV * wd.dv * elt)
+    dach = dbytes / (layer_d / 1e3) / 1e9
+    return {"conv": "causal depthwise, width 4, bias, SiLU, carried state",
+            "gate": "o * sigmoid(z)",
+            "prefill": {"workload": WORKLOAD, "ms_per_step": lp_ms,
+                        "value": tokens / (lp_ms / 1e3), "unit": "tokens/s",
+                        "plain_ms_per_step": plain_s * 1e3, "overhead": lp_ms / (plain_s * 1e3) - 1.0,
+                        "gpu_launches": 4},
+            "conv_kernel": {"ms": cv_ms, "bytes": cv_bytes, "gpu_launches": 2,
+                            "roofline": {"bound": "hbm", "achieved": cv_bytes / (cv_ms / 1e3) / 1e9,
+                                         "peak": hbm, "unit": "GB/s",
+                                         "frac": cv_bytes / (cv_ms / 1e3) / 1e9 / hbm,
+                                         "traffic": kernel_traffic("short_conv"),
+                                         "peak_source": peak_src, "kernel": "conv"}},
+            "gate_kernel": {"ms": gt_ms, "bytes": gt_bytes, "gpu_launches": 1,
+                            "roofline": {"bound": "hbm", "achieved": gt_bytes / (gt_ms / 1e3) / 1e9,
+                                         "peak": hbm, "unit": "GB/s",
+                                         "frac": gt_bytes / (gt_ms / 1e3) / 1e9 / hbm,
+                                         "traffic": kernel_traffic("output_gate"),
+                                         "peak_source": peak_src, "kernel": "gate"}},
+            "decode": {"workload": DECODE_WORKLOAD, "ms_per_step": layer_d,
+                       "plain_ms_per_step": plain_d, "overhead": layer_d / plain_d - 1.0,
+                       "bytes_per_step": dbytes, "gpu_launches": 8,
+                       "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
+                                    "frac": dach / hbm, "traffic": kernel_traffic("decode_layer"),
+                                    "peak_source": peak_src, "kernel": "decode (layer instance)"}}}
+
+
 def dist_max(x, device=None):
     """Max of a host float over all ranks (identity when not distributed)."""
     import torch
@@ -689,6 +800,11 @@ def run_b200(args):
         pro = measure_prologue(gdn, torch, dev, stream, x, w, ws, o, hT, rank, barrier,
                                max_over_ranks, mean_launch_s, args)
 
+    lay = None
+    if not args.no_layer and n_steps:
+        lay = measure_layer(gdn, torch, dev, stream, x, w, o, hT, rank, peaks, peak_src,
+                            mean_launch_s, args)
+
     ver = None
     if not args.no_verify:
         ver = measure_verify(gdn, torch, dev, stream, peaks, peak_src, rank, world,
@@ -712,7 +828,7 @@ def run_b200(args):
                        "l2": "inputs larger than L2 (q,k,v 1.07 GB per step)"},
             "roofline": roof, "cpu_baseline": base, "e2e": e2e,
             "gpu_launches": launches_per_step * n_steps, "clocks": clocks, "decode": dec,
-            "verify": ver, "prologue": pro,
+            "verify": ver, "prologue": pro, "layer": lay,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -732,6 +848,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-verify", action="store_true")
     ap.add_argument("--no-prologue", action="store_true")
+    ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--verify-rounds", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="decode measurement only")

@@ -403,6 +403,99 @@ GDN_API gdn_status gdn_state_commit_deltas(const void *k, const float *g, const 
                                            unsigned prologue, gdn_stream_t stream);
 
 /*
+ * ---- The layer steps around the rule -------------------------------------
+ * "Qwen3-Next" (sghael.github.io), section "Linear attention with gated delta
+ * rule": the values pass through a 1-D convolution that adds local context,
+ * and a gate sets how much of the recurrent read-out reaches the output.  The
+ * page gives neither the width nor the gate's form.  Reading used here:
+ *   - a causal depthwise convolution along time, one kernel of `width` taps
+ *     (2..8) per value channel c = h * dv + i (C = HV * dv channels):
+ *       y_t[c] = act(bias[c] + sum_{j<width} weight[c][j] * x_{t-(width-1)+j}[c])
+ *     within each sequence; the inputs before a sequence's first token come
+ *     from its carried convolution state (its last width-1 inputs, raw) or are
+ *     zero; act = identity, or SiLU (x * sigmoid(x)) with GDN_CONV_SILU;
+ *   - an elementwise sigmoid gate on the read-out: o <- o * sigmoid(z), one
+ *     logit per output element.
+ * Convolution state layout: [N][width-1][C] in the call's dtype, row m = the
+ * input width-1-m tokens before the next token (row width-2 the most recent).
+ */
+#define GDN_CONV_SILU 16u
+#define GDN_CONV_MAX_WIDTH 8
+
+/*
+ * Short causal convolution over N sequences of C channels.
+ * x, y [B][T][C] dtype (or packed [T_total][C] with cu_seqlens, as in
+ * gdn_chunk_prefill; T is then the packed total); weight [C][width] fp32;
+ * bias [C] fp32 or NULL; conv_state as above or NULL (zero history, nothing
+ * kept).  When given, conv_state is read as each sequence's history and then
+ * overwritten with its last width-1 inputs (taken from the old state where a
+ * sequence is shorter than width-1; an empty sequence keeps its state).
+ * flags: 0 or GDN_CONV_SILU.  Supported: 2 <= width <= GDN_CONV_MAX_WIDTH, C a
+ * multiple of 8 (bf16) or 4 (fp32).  Alignment: x, y, conv_state 16-byte.
+ * y must not overlap x or conv_state.  Two launches (the convolution, then the
+ * state update when conv_state is given).  N == 0 or no tokens: GDN_OK, and
+ * only the state update runs.
+ */
+GDN_API gdn_status gdn_short_conv(const void *x, const float *weight, const float *bias,
+                                  void *conv_state, const int32_t *cu_seqlens, int N, int64_t T,
+                                  int C, int width, unsigned flags, gdn_dtype dtype, void *y,
+                                  gdn_stream_t stream);
+
+/*
+ * Output gate in place: o <- o * sigmoid(z) over rows x C elements (o and z
+ * the same dtype and layout, e.g. [B][T][HV][dv] with C = HV * dv).
+ * Supported: rows * C a multiple of 8 (bf16) or 4 (fp32).  Alignment: o, z
+ * 16-byte.  rows == 0: GDN_OK, nothing launched.
+ */
+GDN_API gdn_status gdn_output_gate(void *o, const void *z, int64_t rows, int C, gdn_dtype dtype,
+                                   gdn_stream_t stream);
+
+/*
+ * gdn_recurrent_step_ex with the layer steps fused into the same kernel: the
+ * token's v is convolved with each sequence's carried inputs (conv_state
+ * [N][conv_width-1][HV*dv] dtype, updated in place) before the rule, and the
+ * output is gated by sigmoid(z) (z [N][HV][dv] dtype) after it.  conv_weight
+ * [HV*dv][conv_width] fp32 (NULL: no convolution, conv_width ignored),
+ * conv_bias [HV*dv] fp32 or NULL; z NULL: no gate.  flags: GDN_PROLOGUE_*,
+ * GDN_ROW_DECAY and GDN_CONV_SILU.  Supported and aligned as
+ * gdn_recurrent_step_ex, plus 2 <= conv_width <= GDN_CONV_MAX_WIDTH when
+ * conv_weight is given; conv_state, z 2-byte (bf16) or 4-byte (fp32) aligned.
+ */
+GDN_API gdn_status gdn_recurrent_step_layer(const void *q, const void *k, const void *v,
+                                            const float *g, const float *beta, float *state,
+                                            const float *conv_weight, const float *conv_bias,
+                                            void *conv_state, int conv_width, const void *z,
+                                            int N, int HK, int HV, int dk, int dv, float scale,
+                                            gdn_dtype dtype, void *o, unsigned flags,
+                                            gdn_stream_t stream);
+
+/*
+ * Bytes of device workspace gdn_chunk_prefill_layer needs: the convolved
+ * values (when has_conv) after gdn_chunk_prefill's own workspace.
+ */
+GDN_API size_t gdn_chunk_prefill_layer_workspace_size(int N, int64_t T, int HK, int HV, int dk,
+                                                      int dv, int chunk, gdn_dtype dtype,
+                                                      int varlen, int has_conv);
+
+/*
+ * gdn_chunk_prefill_ex with the layer steps: the short convolution of v
+ * (into the workspace; conv_state [N][conv_width-1][HV*dv] updated as in
+ * gdn_short_conv), the prefill on the convolved values, then the output gate
+ * on o.  conv_weight NULL: no convolution; z NULL: no gate.  flags:
+ * GDN_PROLOGUE_*, GDN_ROW_DECAY and GDN_CONV_SILU.  Up to three launch groups
+ * on `stream`; arguments as in gdn_chunk_prefill_ex and gdn_short_conv.
+ */
+GDN_API gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v,
+                                           const float *g, const float *beta, const float *h0,
+                                           const int32_t *cu_seqlens, int N, int64_t T, int HK,
+                                           int HV, int dk, int dv, int chunk, float scale,
+                                           gdn_dtype dtype, void *o, float *hT,
+                                           const float *conv_weight, const float *conv_bias,
+                                           void *conv_state, int conv_width, const void *z,
+                                           unsigned flags, void *workspace,
+                                           size_t workspace_bytes, gdn_stream_t stream);
+
+/*
  * Reads the device status word a prefill call left in its workspace (HOST
  * call; synchronises `stream`).  Returns GDN_OK when every on-device wait of
  * the last call on this workspace completed, GDN_ERR_TIMEOUT when one gave up

@@ -380,6 +380,165 @@ gdn_status gdn_state_commit_deltas(const void *k, const float *g, const float *u
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+// ---- layer steps: short convolution on the values, output gate ----
+
+}  // extern "C"
+
+namespace {
+
+bool aligned_elt(const void *p, gdn_dtype dt) {
+    return dt == GDN_BF16 ? (reinterpret_cast<uintptr_t>(p) & 1u) == 0 : aligned4(p);
+}
+
+// host checks of one short-convolution call (nothing enqueued)
+gdn_status check_conv(const gdn::ConvArgs &a) {
+    if (!a.x || !a.weight || !a.y) return GDN_ERR_INVALID_ARG;
+    if (a.N < 0 || a.T < 0 || a.C <= 0) return GDN_ERR_INVALID_ARG;
+    if (a.dtype != GDN_F32 && a.dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (a.width < 2 || a.width > gdn::kConvMaxWidth) return GDN_ERR_UNSUPPORTED;
+    if (a.C % gdn::conv_vector_channels(a.dtype)) return GDN_ERR_UNSUPPORTED;
+    if (a.C / gdn::conv_vector_channels(a.dtype) > 65535 * 128) return GDN_ERR_UNSUPPORTED;
+    const int64_t tokens = a.cu_seqlens ? a.T : (int64_t)a.N * a.T;
+    if (a.cu_seqlens == nullptr && a.N > 0 && a.T > 0 && tokens / a.N != a.T) return GDN_ERR_INVALID_ARG;
+    if ((tokens + 31) / 32 > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (!aligned16(a.x) || !aligned16(a.y) || !aligned16(a.conv_state)) return GDN_ERR_ALIGNMENT;
+    return GDN_OK;
+}
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t layer_vconv_bytes(int N, int64_t T, int HV, int dv, gdn_dtype dt, bool varlen) {
+    const int64_t tokens = varlen ? T : (int64_t)N * T;
+    return up256((size_t)tokens * (size_t)HV * (size_t)dv * (dt == GDN_BF16 ? 2 : 4));
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_short_conv(const void *x, const float *weight, const float *bias, void *conv_state,
+                          const int32_t *cu_seqlens, int N, int64_t T, int C, int width,
+                          unsigned flags, gdn_dtype dtype, void *y, gdn_stream_t stream) {
+    if (flags & ~GDN_CONV_SILU) return GDN_ERR_INVALID_ARG;
+    gdn::ConvArgs a{x, weight, bias, conv_state, cu_seqlens, N, T, C, width,
+                    (flags & GDN_CONV_SILU) != 0, dtype, y};
+    const gdn_status st = check_conv(a);
+    if (st != GDN_OK) return st;
+    if (N == 0) return GDN_OK;
+    const cudaError_t err = gdn::launch_short_conv(a, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_output_gate(void *o, const void *z, int64_t rows, int C, gdn_dtype dtype,
+                           gdn_stream_t stream) {
+    if (!o || !z || rows < 0 || C <= 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (rows > ((int64_t)1 << 40) / C) return GDN_ERR_INVALID_ARG;
+    const int64_t elems = rows * (int64_t)C;
+    if (elems % gdn::conv_vector_channels(dtype)) return GDN_ERR_UNSUPPORTED;
+    if (!aligned16(o) || !aligned16(z)) return GDN_ERR_ALIGNMENT;
+    if (elems == 0) return GDN_OK;
+    const cudaError_t err =
+        gdn::launch_output_gate(o, z, elems, dtype, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_recurrent_step_layer(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, float *state, const float *conv_weight,
+                                    const float *conv_bias, void *conv_state, int conv_width,
+                                    const void *z, int N, int HK, int HV, int dk, int dv,
+                                    float scale, gdn_dtype dtype, void *o, unsigned flags,
+                                    gdn_stream_t stream) {
+    if (flags & ~(GDN_FLAGS_VALID | GDN_CONV_SILU)) return GDN_ERR_INVALID_ARG;
+    if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
+    if (N < 0 || HK <= 0 || HV <= 0 || dk <= 0 || dv <= 0 || HV % HK) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (conv_weight && !conv_state) return GDN_ERR_INVALID_ARG;
+    if (conv_weight && (conv_width < 2 || conv_width > GDN_CONV_MAX_WIDTH)) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)N * HV > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
+    if (!gdn::decode_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
+        return GDN_ERR_ALIGNMENT;
+    if (!aligned4(conv_weight) || !aligned4(conv_bias) ||
+        (conv_weight && !aligned_elt(conv_state, dtype)) || (z && !aligned_elt(z, dtype)))
+        return GDN_ERR_ALIGNMENT;
+    if (N == 0) return GDN_OK;
+    gdn::StepArgs a{q, k, v, g, beta, state, N, HK, HV, dk, dv, scale, dtype, o,
+                    flags & GDN_FLAGS_VALID};
+    if (conv_weight) {
+        a.conv_w = conv_weight;
+        a.conv_b = conv_bias;
+        a.conv_state = conv_state;
+        a.conv_width = conv_width;
+        a.conv_silu = (flags & GDN_CONV_SILU) != 0;
+    }
+    a.z = z;
+    const cudaError_t err = gdn::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+size_t gdn_chunk_prefill_layer_workspace_size(int N, int64_t T, int HK, int HV, int dk, int dv,
+                                              int chunk, gdn_dtype dtype, int varlen,
+                                              int has_conv) {
+    if (N < 0 || T < 0 || HK <= 0 || HV <= 0 || HV % HK || dv <= 0 || chunk <= 0) return 0;
+    const size_t pre = up256(gdn_chunk_prefill_workspace_size(N, T, HK, HV, dk, dv, chunk, dtype, varlen));
+    return has_conv ? pre + layer_vconv_bytes(N, T, HV, dv, dtype, varlen != 0) : pre;
+}
+
+gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, const float *h0, const int32_t *cu_seqlens,
+                                   int N, int64_t T, int HK, int HV, int dk, int dv, int chunk,
+                                   float scale, gdn_dtype dtype, void *o, float *hT,
+                                   const float *conv_weight, const float *conv_bias,
+                                   void *conv_state, int conv_width, const void *z, unsigned flags,
+                                   void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    if (flags & ~(GDN_FLAGS_VALID | GDN_CONV_SILU)) return GDN_ERR_INVALID_ARG;
+    const unsigned prologue = flags & GDN_FLAGS_VALID;
+    if ((prologue & GDN_ROW_DECAY) && !gdn::prefill_simt_supported(dk, dv, chunk))
+        return GDN_ERR_UNSUPPORTED;
+    gdn::PrefillArgs a{q, k, v, g, beta, h0, cu_seqlens, N, T, HK, HV, dk, dv, chunk,
+                       scale, dtype, o, hT, workspace, workspace_bytes};
+    a.prologue = prologue;
+    gdn_status st = check_prefill(a);
+    if (st != GDN_OK) return st;
+    const bool varlen = cu_seqlens != nullptr;
+    const int64_t tokens = varlen ? T : (int64_t)N * T;
+    if ((size_t)HV * dv > 0x7fffffffu) return GDN_ERR_UNSUPPORTED;
+    const int C = HV * dv;
+    gdn::ConvArgs ca{v, conv_weight, conv_bias, conv_state, cu_seqlens, N, T, C, conv_width,
+                     (flags & GDN_CONV_SILU) != 0, dtype, nullptr};
+    if (conv_weight) {
+        ca.y = o;   // placeholder for the host checks; the real target is the workspace
+        st = check_conv(ca);
+        if (st != GDN_OK) return st;
+    }
+    if (z) {
+        if ((tokens * (int64_t)C) % gdn::conv_vector_channels(dtype)) return GDN_ERR_UNSUPPORTED;
+        if (!aligned16(z)) return GDN_ERR_ALIGNMENT;
+    }
+    if (N == 0) return GDN_OK;
+    // workspace: [prefill's own | convolved values]
+    const size_t pre = up256(gdn::prefill_cluster_supported(dk, dv, chunk, dtype) && !(prologue & GDN_ROW_DECAY)
+                                 ? gdn::prefill_cluster_workspace(N, T, HV, chunk, varlen)
+                                 : 0);
+    const size_t need = conv_weight ? pre + layer_vconv_bytes(N, T, HV, dv, dtype, varlen) : pre;
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (conv_weight) {
+        ca.y = static_cast<char *>(workspace) + pre;
+        if (gdn::launch_short_conv(ca, s) != cudaSuccess) return GDN_ERR_CUDA;
+        a.v = ca.y;
+    }
+    a.workspace_bytes = pre;
+    if (pre == 0) a.workspace = nullptr;
+    st = enqueue_prefill(a, s);
+    if (st != GDN_OK) return st;
+    if (z && gdn::launch_output_gate(o, z, tokens * (int64_t)C, dtype, s) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    return GDN_OK;
+}
+
 gdn_status gdn_read_status(const void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
     if (workspace == nullptr || workspace_bytes < sizeof(unsigned int)) return GDN_OK;
     unsigned int word = 0;

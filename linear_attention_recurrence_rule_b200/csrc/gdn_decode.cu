@@ -22,6 +22,13 @@
 // state in flight.  Bands of 8 x NB rows (64 at dk = 128) keep CTAs short and
 // several of them resident per SM, so their load, update and store phases
 // overlap.
+//
+// The layer instance (gdn_recurrent_step_layer) adds the steps around the rule
+// for one token: the short convolution on v with its carried inputs, and the
+// sigmoid gate on o (readings in gdn_layer.cu).  The band's threads compute the
+// convolved values and gates of its rows into shared memory while the state
+// loads are in flight; the carried inputs (W-1 values per channel) are the
+// only extra HBM traffic besides v, z and the weights.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -34,13 +41,26 @@ constexpr int kDecodeNB = 8;
 template <int DK>
 constexpr int band_rows() { return kDecodeWarps * (32 / (DK / 4)) * kDecodeNB; }
 
+// The layer steps of gdn_recurrent_step_layer: the short convolution on v (its
+// carried inputs updated in place) and the sigmoid gate on o.
+template <typename Tin>
+struct LayerStep {
+    const float *cw, *cb;   // [HV*dv][W], [HV*dv] or null
+    Tin *cs;                // [N][W-1][HV*dv]
+    const Tin *z;           // [N][HV][dv] or null
+    int W;                  // 0: no convolution
+    bool silu;
+};
+
 // PRO: the input prologue flags are read; RD (implies PRO): one decay per value
-// row.  Separate instances, so neither costs the paths that do not use it.
-template <int DK, typename Tin, bool PRO, bool RD>
-__global__ void __launch_bounds__(kDecodeWarps * 32, 3)
+// row; LY (implies PRO): the layer steps.  Separate instances, so none of them
+// costs the paths that do not use it.
+template <int DK, typename Tin, bool PRO, bool RD, bool LY>
+__global__ void __launch_bounds__(kDecodeWarps * 32, LY ? 2 : 3)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ g, const float *__restrict__ beta, float *state,
-              Tin *__restrict__ o, int HK, int HV, int dv, float scale, unsigned pro) {
+              Tin *__restrict__ o, int HK, int HV, int dv, float scale, unsigned pro,
+              LayerStep<Tin> ly) {
     constexpr int LPR = DK / 4;    // lanes per state row
     constexpr int RPI = 32 / LPR;  // rows per warp instruction
     const int nh = blockIdx.x;     // n * HV + h
@@ -70,6 +90,33 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
             s[j] = row < dv ? __ldcs(reinterpret_cast<const float4 *>(S + (size_t)row * DK + col))
                             : make_float4(0.f, 0.f, 0.f, 0.f);
             if (RD) grow[RD ? j : 0] = row < dv ? g[(size_t)nh * dv + row] : 0.f;
+        }
+        // layer steps of this band's rows, while the state loads are in flight: the
+        // convolved value and the output gate of each row, shared by its lanes
+        __shared__ float lyv[LY ? rows_per_batch : 1], lyg[LY ? rows_per_batch : 1];
+        if (LY) {
+            const size_t C = (size_t)HV * dv;
+            for (int r = threadIdx.x; r < rows_per_batch; r += kDecodeWarps * 32) {
+                const int row = base + r;
+                if (row >= dv) continue;
+                const size_t ch = (size_t)h * dv + row;
+                const float vin = to_f32(vrow[row]);
+                float vc = vin;
+                if (ly.W > 0) {
+                    Tin *cs = ly.cs + (size_t)n * (ly.W - 1) * C + ch;
+                    const float *wr = ly.cw + ch * ly.W;
+                    float a = ly.cb ? ly.cb[ch] : 0.f;
+                    for (int m = 0; m < ly.W - 1; ++m) a = fmaf(wr[m], to_f32(cs[m * C]), a);
+                    a = fmaf(wr[ly.W - 1], vin, a);
+                    vc = ly.silu ? a * gate_sigmoid(a) : a;
+                    // the carried inputs move one token on; this token's raw value last
+                    for (int m = 0; m + 1 < ly.W - 1; ++m) cs[m * C] = cs[(m + 1) * C];
+                    cs[(ly.W - 2) * C] = vrow[row];
+                }
+                lyv[r] = vc;
+                lyg[r] = ly.z ? gate_sigmoid(to_f32(ly.z[(size_t)nh * dv + row])) : 1.f;
+            }
+            __syncthreads();
         }
         if (PRO && (pro & (GDN_PROLOGUE_NORM_Q | GDN_PROLOGUE_NORM_K))) {
             // the lanes of a row hold the whole q and k: reduce the squared norms there
@@ -101,14 +148,19 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
                 const float alpha =
                     rowdec ? (logits ? gate_sigmoid(grow[RD ? j : 0]) : expf(grow[RD ? j : 0]))
                            : alpha_h;
-                const float u = b * (to_f32(vrow[row]) - alpha * sk);
+                const float vval = LY ? lyv[LY ? row - base : 0] : to_f32(vrow[row]);
+                const float u = b * (vval - alpha * sk);
                 float4 ns;
                 ns.x = fmaf(alpha, s[j].x, u * kk.x);
                 ns.y = fmaf(alpha, s[j].y, u * kk.y);
                 ns.z = fmaf(alpha, s[j].z, u * kk.z);
                 ns.w = fmaf(alpha, s[j].w, u * kk.w);
                 __stcs(reinterpret_cast<float4 *>(S + (size_t)row * DK + col), ns);
-                if ((lane % LPR) == 0) orow[row] = from_f32<Tin>(scale * fmaf(alpha, sq, u * kq));
+                if ((lane % LPR) == 0) {
+                    float out = scale * fmaf(alpha, sq, u * kq);
+                    if (LY) out *= lyg[LY ? row - base : 0];
+                    orow[row] = from_f32<Tin>(out);
+                }
             }
         }
     }
@@ -116,13 +168,19 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 
 template <int DK, typename Tin>
 void launch_dk(const StepArgs &a, dim3 grid, dim3 block, cudaStream_t stream) {
-    auto kern = (a.prologue & GDN_ROW_DECAY) ? decode_kernel<DK, Tin, true, true>
-                : a.prologue                 ? decode_kernel<DK, Tin, true, false>
-                                             : decode_kernel<DK, Tin, false, false>;
+    const bool layer = a.conv_width > 0 || a.z != nullptr;
+    const bool rd = (a.prologue & GDN_ROW_DECAY) != 0;
+    auto kern = layer ? (rd ? decode_kernel<DK, Tin, true, true, true>
+                            : decode_kernel<DK, Tin, true, false, true>)
+                : rd          ? decode_kernel<DK, Tin, true, true, false>
+                : a.prologue  ? decode_kernel<DK, Tin, true, false, false>
+                              : decode_kernel<DK, Tin, false, false, false>;
+    const LayerStep<Tin> ly{a.conv_w, a.conv_b, static_cast<Tin *>(a.conv_state),
+                            static_cast<const Tin *>(a.z), a.conv_width, a.conv_silu};
     kern<<<grid, block, 0, stream>>>(static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
                                      static_cast<const Tin *>(a.v), a.g, a.beta, a.state,
                                      static_cast<Tin *>(a.o), a.HK, a.HV, a.dv, a.scale,
-                                     a.prologue);
+                                     a.prologue, ly);
 }
 
 template <typename Tin>

@@ -35,6 +35,12 @@ struct StepArgs {
     gdn_dtype dtype;
     void *o;
     unsigned prologue = 0;
+    // layer steps (gdn_recurrent_step_layer): short convolution on v, gate on o
+    const float *conv_w = nullptr, *conv_b = nullptr;   // [HV*dv][conv_width], [HV*dv]
+    void *conv_state = nullptr;                          // [N][conv_width-1][HV*dv], dtype
+    int conv_width = 0;                                  // 0: no convolution
+    bool conv_silu = false;
+    const void *z = nullptr;                             // gate logits [N][HV][dv], dtype
 };
 
 struct VerifyArgs {
@@ -80,6 +86,25 @@ struct CommitDeltasArgs {
 cudaError_t launch_commit_deltas(const CommitDeltasArgs &a, cudaStream_t stream);
 cudaError_t launch_commit(const float *states, const int32_t *accepted, float *state, int N, int K,
                           int HV, int dv, int dk, cudaStream_t stream);
+
+// short convolution on the values and output gate (gdn_layer.cu)
+struct ConvArgs {
+    const void *x;
+    const float *weight, *bias;   // [C][width], [C] or null
+    void *conv_state;             // [N][width-1][C] dtype, in/out, or null (zeros, not kept)
+    const int32_t *cu_seqlens;
+    int N;
+    int64_t T;                    // tokens per sequence (no cu_seqlens) or packed total
+    int C, width;
+    bool silu;
+    gdn_dtype dtype;
+    void *y;
+};
+constexpr int kConvMaxWidth = 8;
+int conv_vector_channels(gdn_dtype dtype);   // channels per 16-byte vector
+cudaError_t launch_short_conv(const ConvArgs &a, cudaStream_t stream);
+cudaError_t launch_output_gate(void *o, const void *z, int64_t elems, gdn_dtype dtype,
+                               cudaStream_t stream);
 
 // CUDA-core chunked prefill (gdn_prefill_simt.cu)
 bool prefill_simt_supported(int dk, int dv, int chunk);

@@ -1,0 +1,317 @@
+// The layer steps around the rule: a short causal convolution on the values
+// before it and a sigmoid gate on its read-out after it ("Qwen3-Next",
+// sghael.github.io, section "Linear attention with gated delta rule": a 1-D
+// convolution over the values adds local context, and a gate sets how much of
+// the recurrent read-out reaches the layer's output).  The page gives neither
+// the width nor the gate's form; the library reads them as
+//   y_t[c] = act(bias[c] + sum_{j<W} w[c][j] x_{t-(W-1)+j}[c])   (W = 2..8)
+// per value channel c = h * dv + i, causal within each sequence, the inputs
+// before a sequence's first token taken from a carried state of its last W-1
+// inputs (zero without one), act = identity or SiLU; and o <- o * sigmoid(z)
+// elementwise.
+//
+// All three kernels are single streaming passes over HBM:
+//  * conv_kernel: a thread owns 16 bytes of channels (8 bf16 / 4 fp32) for a
+//    run of kConvRun tokens and keeps the previous W-1 inputs of its channels
+//    in registers, so each input is read once plus a halo of W-1 tokens per
+//    run, each output written once; loads go out kConvBatch tokens at a time.
+//    A sequence start inside a run resets the window from the carried state.
+//  * conv_state_kernel (launched after it on the same stream): each
+//    sequence's new carried state, its last W-1 inputs (from the old state
+//    where the sequence is shorter than W-1).  A launch of its own, so that
+//    every read of the old state is over before it is overwritten in place.
+//  * gate_kernel: o <- o * sigmoid(z), 16-byte vectors, grid-stride.
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int kConvThreads = 128;
+constexpr int kConvRun = 32;     // tokens per thread
+constexpr int kConvBatch = 8;    // loads in flight per thread
+constexpr int kGateThreads = 256;
+
+// 16 bytes of one dtype as raw words and as floats
+template <typename T> struct Vec16;
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int n = 8;
+    __device__ static void to_float(const uint4 &u, float (&f)[8]) {
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 t = __bfloat1622float2(h[i]);
+            f[2 * i] = t.x;
+            f[2 * i + 1] = t.y;
+        }
+    }
+    __device__ static uint4 from_float(const float (&f)[8]) {
+        uint4 u;
+        uint32_t *w = reinterpret_cast<uint32_t *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        return u;
+    }
+};
+template <> struct Vec16<float> {
+    static constexpr int n = 4;
+    __device__ static void to_float(const uint4 &u, float (&f)[4]) {
+        f[0] = __uint_as_float(u.x);
+        f[1] = __uint_as_float(u.y);
+        f[2] = __uint_as_float(u.z);
+        f[3] = __uint_as_float(u.w);
+    }
+    __device__ static uint4 from_float(const float (&f)[4]) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                          __float_as_uint(f[3]));
+    }
+};
+
+template <typename T>
+__device__ __forceinline__ uint4 ld16(const T *p) { return *reinterpret_cast<const uint4 *>(p); }
+template <typename T>
+__device__ __forceinline__ void st16(T *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+
+// bounds of sequence n
+__device__ __forceinline__ void seq_bounds(const int32_t *cu, int64_t T_per, int n, int64_t &bos,
+                                           int64_t &eos) {
+    if (cu) {
+        bos = cu[n];
+        eos = cu[n + 1];
+    } else {
+        bos = (int64_t)n * T_per;
+        eos = bos + T_per;
+    }
+}
+
+template <typename T, int W>
+__global__ void __launch_bounds__(kConvThreads)
+conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
+            const T *__restrict__ cstate, const int32_t *__restrict__ cu, int N, int64_t T_per,
+            int64_t Ttot, int C, bool silu, T *__restrict__ y) {
+    constexpr int VN = Vec16<T>::n;
+    const int c0 = (blockIdx.y * kConvThreads + threadIdx.x) * VN;
+    if (c0 >= C) return;
+    const int64_t t0 = (int64_t)blockIdx.x * kConvRun;
+    const int64_t t1 = t0 + kConvRun < Ttot ? t0 + kConvRun : Ttot;
+    // the sequence holding token t0: the last n with start <= t0 (empty sequences skipped)
+    int n;
+    if (cu) {
+        int lo = 0, hi = N - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (cu[mid] <= t0) lo = mid;
+            else hi = mid - 1;
+        }
+        n = lo;
+    } else {
+        n = (int)(t0 / T_per);
+    }
+    int64_t bos, eos;
+    seq_bounds(cu, T_per, n, bos, eos);
+
+    float wt[W][VN], b[VN];
+#pragma unroll
+    for (int e = 0; e < VN; ++e) {
+#pragma unroll
+        for (int j = 0; j < W; ++j) wt[j][e] = w[(size_t)(c0 + e) * W + j];
+        b[e] = bias ? bias[c0 + e] : 0.f;
+    }
+    // window: win[m] = the raw input at token t - (W-1) + m, m < W-1 (raw words,
+    // converted where used: half the registers for bf16)
+    uint4 win[W - 1];
+#pragma unroll
+    for (int m = 0; m < W - 1; ++m) {
+        const int64_t s = t0 - (W - 1) + m;
+        if (s >= bos)
+            win[m] = ld16(x + s * C + c0);
+        else if (cstate)
+            win[m] = ld16(cstate + ((size_t)n * (W - 1) + (size_t)(s - bos + W - 1)) * C + c0);
+        else
+            win[m] = make_uint4(0u, 0u, 0u, 0u);   // +0.0 in both dtypes
+    }
+    constexpr int NB = W <= 4 ? kConvBatch : kConvBatch / 2;
+    for (int64_t tb = t0; tb < t1; tb += NB) {
+        uint4 raw[NB];
+#pragma unroll
+        for (int u = 0; u < NB; ++u)
+            if (tb + u < t1) raw[u] = ld16(x + (tb + u) * C + c0);
+#pragma unroll
+        for (int u = 0; u < NB; ++u) {
+            const int64_t t = tb + u;
+            if (t >= t1) break;
+            if (t >= eos) {
+                // a new sequence starts at t (after any empty ones): window from its state
+                do {
+                    ++n;
+                    seq_bounds(cu, T_per, n, bos, eos);
+                } while (eos <= t);
+#pragma unroll
+                for (int m = 0; m < W - 1; ++m)
+                    win[m] = cstate ? ld16(cstate + ((size_t)n * (W - 1) + m) * C + c0)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+            }
+            float acc[VN], f[VN];
+#pragma unroll
+            for (int e = 0; e < VN; ++e) acc[e] = b[e];
+#pragma unroll
+            for (int m = 0; m < W - 1; ++m) {
+                Vec16<T>::to_float(win[m], f);
+#pragma unroll
+                for (int e = 0; e < VN; ++e) acc[e] = fmaf(wt[m][e], f[e], acc[e]);
+            }
+            Vec16<T>::to_float(raw[u], f);
+#pragma unroll
+            for (int e = 0; e < VN; ++e) {
+                const float a = fmaf(wt[W - 1][e], f[e], acc[e]);
+                acc[e] = silu ? a * gate_sigmoid(a) : a;
+            }
+            st16(y + t * C + c0, Vec16<T>::from_float(acc));
+#pragma unroll
+            for (int m = 0; m + 1 < W - 1; ++m) win[m] = win[m + 1];
+            win[W - 2] = raw[u];
+        }
+    }
+}
+
+// new carried state of sequence blockIdx.x: its last W-1 inputs (raw copies)
+template <typename T, int W>
+__global__ void __launch_bounds__(kConvThreads)
+conv_state_kernel(const T *__restrict__ x, T *cstate, const int32_t *__restrict__ cu, int64_t T_per,
+                  int C) {
+    constexpr int VN = Vec16<T>::n;
+    const int c0 = (blockIdx.y * kConvThreads + threadIdx.x) * VN;
+    if (c0 >= C) return;
+    const int n = blockIdx.x;
+    int64_t bos, eos;
+    seq_bounds(cu, T_per, n, bos, eos);
+    const int64_t L = eos - bos;
+    T *st = cstate + (size_t)n * (W - 1) * C + c0;
+    uint4 old[W - 1], nw[W - 1];
+#pragma unroll
+    for (int m = 0; m < W - 1; ++m) old[m] = ld16(st + (size_t)m * C);
+#pragma unroll
+    for (int m = 0; m < W - 1; ++m) {
+        const int64_t s = eos - (W - 1) + m;
+        if (s >= bos) {
+            nw[m] = ld16(x + s * C + c0);
+        } else {
+            // old[m + L] (m + L < W - 1 when s < bos), selected without a dynamic index
+            nw[m] = old[0];
+#pragma unroll
+            for (int r = 1; r < W - 1; ++r)
+                if (r == m + L) nw[m] = old[r];
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < W - 1; ++m) st16(st + (size_t)m * C, nw[m]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kGateThreads)
+gate_kernel(T *o, const T *__restrict__ z, int64_t nvec) {
+    constexpr int VN = Vec16<T>::n;
+    constexpr int U = 4;
+    const int64_t stride = (int64_t)gridDim.x * kGateThreads;
+    for (int64_t i0 = (int64_t)blockIdx.x * kGateThreads + threadIdx.x; i0 < nvec; i0 += U * stride) {
+        uint4 ov[U], zv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < nvec) {
+                ov[u] = __ldcs(reinterpret_cast<const uint4 *>(o) + i);
+                zv[u] = __ldcs(reinterpret_cast<const uint4 *>(z) + i);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < nvec) {
+                float of[VN], zf[VN];
+                Vec16<T>::to_float(ov[u], of);
+                Vec16<T>::to_float(zv[u], zf);
+#pragma unroll
+                for (int e = 0; e < VN; ++e) of[e] *= gate_sigmoid(zf[e]);
+                __stcs(reinterpret_cast<uint4 *>(o) + i, Vec16<T>::from_float(of));
+            }
+        }
+    }
+}
+
+template <typename T, int W>
+cudaError_t launch_conv_w(const ConvArgs &a, cudaStream_t stream) {
+    constexpr int VN = Vec16<T>::n;
+    const int vecs = a.C / VN;
+    const unsigned cblocks = (unsigned)((vecs + kConvThreads - 1) / kConvThreads);
+    const int64_t Ttot = a.cu_seqlens ? a.T : (int64_t)a.N * a.T;
+    const T *x = static_cast<const T *>(a.x);
+    T *cs = static_cast<T *>(a.conv_state);
+    if (Ttot > 0) {
+        const dim3 grid((unsigned)((Ttot + kConvRun - 1) / kConvRun), cblocks);
+        conv_kernel<T, W><<<grid, kConvThreads, 0, stream>>>(
+            x, a.weight, a.bias, cs, a.cu_seqlens, a.N, a.T, Ttot, a.C, a.silu, static_cast<T *>(a.y));
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (cs) {
+        conv_state_kernel<T, W><<<dim3((unsigned)a.N, cblocks), kConvThreads, 0, stream>>>(
+            x, cs, a.cu_seqlens, a.T, a.C);
+        return cudaGetLastError();
+    }
+    return cudaSuccess;
+}
+
+template <typename T>
+cudaError_t launch_conv_t(const ConvArgs &a, cudaStream_t stream) {
+    switch (a.width) {
+        case 2: return launch_conv_w<T, 2>(a, stream);
+        case 3: return launch_conv_w<T, 3>(a, stream);
+        case 4: return launch_conv_w<T, 4>(a, stream);
+        case 5: return launch_conv_w<T, 5>(a, stream);
+        case 6: return launch_conv_w<T, 6>(a, stream);
+        case 7: return launch_conv_w<T, 7>(a, stream);
+        case 8: return launch_conv_w<T, 8>(a, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+int sm_count() {
+    int dev = 0, count = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || count < 1)
+        count = 1;
+    return count;
+}
+
+template <typename T>
+cudaError_t launch_gate_t(void *o, const void *z, int64_t elems, cudaStream_t stream) {
+    const int64_t nvec = elems / Vec16<T>::n;
+    int64_t blocks = (nvec + kGateThreads * 4 - 1) / (kGateThreads * 4);
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    gate_kernel<T><<<(unsigned)blocks, kGateThreads, 0, stream>>>(static_cast<T *>(o),
+                                                                  static_cast<const T *>(z), nvec);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int conv_vector_channels(gdn_dtype dtype) { return dtype == GDN_BF16 ? 8 : 4; }
+
+cudaError_t launch_short_conv(const ConvArgs &a, cudaStream_t stream) {
+    if (a.N == 0) return cudaSuccess;
+    return a.dtype == GDN_BF16 ? launch_conv_t<__nv_bfloat16>(a, stream) : launch_conv_t<float>(a, stream);
+}
+
+cudaError_t launch_output_gate(void *o, const void *z, int64_t elems, gdn_dtype dtype,
+                               cudaStream_t stream) {
+    if (elems == 0) return cudaSuccess;
+    return dtype == GDN_BF16 ? launch_gate_t<__nv_bfloat16>(o, z, elems, stream)
+                             : launch_gate_t<float>(o, z, elems, stream);
+}
+
+}  // namespace gdn

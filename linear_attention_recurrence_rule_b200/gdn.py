@@ -22,6 +22,8 @@ GDN_F32, GDN_BF16 = 0, 1
 PROLOGUE_NORM_Q, PROLOGUE_NORM_K, PROLOGUE_GATE_LOGITS = 1, 2, 4
 PROLOGUE_ALL = 7
 ROW_DECAY = 8   # one decay per value row: g [..., HV, dv] (GDN_ROW_DECAY)
+CONV_SILU = 16  # SiLU after the short convolution (GDN_CONV_SILU)
+CONV_MAX_WIDTH = 8
 
 _lock = threading.Lock()
 _handle = None
@@ -99,6 +101,23 @@ def load_library() -> ctypes.CDLL:
             lib.gdn_chunk_prefill_host.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
                                                    i32, i32, i32, ctypes.c_float, i32, vp, vp,
                                                    vp, sz, i64, vp, vp, vp]
+            lib.gdn_short_conv.restype = i32
+            lib.gdn_short_conv.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, ctypes.c_uint,
+                                           i32, vp, vp]
+            lib.gdn_output_gate.restype = i32
+            lib.gdn_output_gate.argtypes = [vp, vp, i64, i32, i32, vp]
+            lib.gdn_recurrent_step_layer.restype = i32
+            lib.gdn_recurrent_step_layer.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp,
+                                                     i32, i32, i32, i32, i32, ctypes.c_float, i32,
+                                                     vp, ctypes.c_uint, vp]
+            lib.gdn_chunk_prefill_layer_workspace_size.restype = sz
+            lib.gdn_chunk_prefill_layer_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32,
+                                                                   i32, i32, i32, i32]
+            lib.gdn_chunk_prefill_layer.restype = i32
+            lib.gdn_chunk_prefill_layer.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
+                                                    i32, i32, i32, i32, ctypes.c_float, i32, vp,
+                                                    vp, vp, vp, vp, i32, vp, ctypes.c_uint, vp,
+                                                    sz, vp]
             _handle = lib
     return _handle
 
@@ -522,3 +541,191 @@ def gdn_validate_cu_seqlens(cu_seqlens, T, stream=None) -> int:
     if st != GDN_OK:
         raise GDNError(st, "gdn_validate_cu_seqlens")
     return int(res.item())
+
+
+
+# ---- the layer steps around the rule: short convolution on v, output gate ----
+def _conv_args(conv_weight, conv_bias, conv_state, C, N, dtype, dev):
+    """Shape checks of the convolution's weight [C,W], bias [C] and carried state
+    [N,W-1,C]; returns the width (0 without a convolution)."""
+    if conv_weight is None:
+        return 0
+    _need(conv_weight, "conv_weight", torch.float32, dev)
+    if conv_weight.dim() != 2 or conv_weight.shape[0] != C:
+        raise ValueError(f"conv_weight must be [C, width] with C = {C}")
+    W = conv_weight.shape[1]
+    if conv_bias is not None:
+        _need(conv_bias, "conv_bias", torch.float32, dev)
+        if conv_bias.shape != (C,):
+            raise ValueError(f"conv_bias must be [{C}]")
+    if conv_state is not None:
+        _need(conv_state, "conv_state", dtype, dev)
+        if conv_state.shape != (N, W - 1, C):
+            raise ValueError(f"conv_state must be [N, width-1, C] = {(N, W - 1, C)}")
+    return W
+
+
+def gdn_short_conv(x, weight, bias=None, conv_state=None, cu_seqlens=None, silu: bool = False,
+                   y=None, stream=None):
+    """Causal depthwise convolution of each sequence through ``gdn_short_conv``.
+
+    x [B,T,C] (bf16 or fp32; or packed [1,Ttot,C] with cu_seqlens); weight [C,W]
+    fp32; bias [C] fp32 or None; conv_state [N,W-1,C] (x's dtype) or None: read
+    as the history and overwritten with each sequence's last W-1 inputs.
+    Returns y like x.
+    """
+    lib = load_library()
+    dev = x.device
+    _need(x, "x", None, dev)
+    if x.dim() != 3:
+        raise ValueError("expected x [B,T,C]")
+    B, T, C = x.shape
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        if B != 1:
+            raise ValueError("with cu_seqlens the batch dimension must be 1 (packed)")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    W = _conv_args(weight, bias, conv_state, C, N, x.dtype, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    else:
+        _need(y, "y", x.dtype, dev)
+    st = lib.gdn_short_conv(_ptr(x), _ptr(weight), _ptr(bias), _ptr(conv_state),
+                            _ptr(cu_seqlens), N, T, C, W, CONV_SILU if silu else 0,
+                            _dtype_code(x), _ptr(y), _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_short_conv")
+    return y
+
+
+def gdn_output_gate(o, z, stream=None):
+    """o <- o * sigmoid(z) in place through ``gdn_output_gate``; returns o."""
+    lib = load_library()
+    dev = o.device
+    _need(o, "o", None, dev)
+    _need(z, "z", o.dtype, dev)
+    if z.shape != o.shape:
+        raise ValueError("z must have o's shape")
+    C = o.shape[-1] if o.dim() > 0 else 1
+    rows = o.numel() // C if C else 0
+    st = lib.gdn_output_gate(_ptr(o), _ptr(z), rows, C, _dtype_code(o), _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_output_gate")
+    return o
+
+
+def gdn_recurrent_step_layer(q, k, v, g, beta, state, conv_weight=None, conv_bias=None,
+                             conv_state=None, z=None, scale: float = 1.0, o=None, stream=None,
+                             prologue: int = 0, silu: bool = False):
+    """One decode token with the layer steps fused (``gdn_recurrent_step_layer``):
+    v is convolved with the carried inputs ``conv_state`` [N,W-1,HV*dv] (updated
+    in place) and o gated by sigmoid(z) (z [N,HV,dv]).  Other arguments as in
+    ``gdn_recurrent_step``.  Returns o [N,HV,dv]."""
+    lib = load_library()
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(state, "state", torch.float32, dev)
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[0] != q.shape[0]:
+        raise ValueError("expected q,k [N,HK,dk] and v [N,HV,dv]")
+    N, HK, dk = q.shape
+    HV, dv = v.shape[1], v.shape[2]
+    g_shape = (N, HV, dv) if prologue & ROW_DECAY else (N, HV)
+    if g.shape != g_shape or beta.shape != (N, HV) or state.shape != (N, HV, dv, dk):
+        raise ValueError(f"expected g {g_shape}, beta [N,HV] and state [N,HV,dv,dk]")
+    if conv_weight is not None and conv_state is None:
+        raise ValueError("a convolution needs its conv_state")
+    W = _conv_args(conv_weight, conv_bias, conv_state, HV * dv, N, q.dtype, dev)
+    if z is not None:
+        _need(z, "z", q.dtype, dev)
+        if z.shape != v.shape:
+            raise ValueError("z must be [N,HV,dv]")
+    if o is None:
+        o = torch.empty_like(v)
+    else:
+        _need(o, "o", v.dtype, dev)
+    flags = int(prologue) | (CONV_SILU if silu else 0)
+    st = lib.gdn_recurrent_step_layer(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                      _ptr(state), _ptr(conv_weight), _ptr(conv_bias),
+                                      _ptr(conv_state), W, _ptr(z), N, HK, HV, dk, dv,
+                                      float(scale), _dtype_code(q), _ptr(o), flags,
+                                      _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_recurrent_step_layer")
+    return o
+
+
+def gdn_chunk_prefill_layer_workspace_size(N, T, HK, HV, dk, dv, chunk, dtype, varlen,
+                                           has_conv) -> int:
+    code = dtype if isinstance(dtype, int) else _dtype_code(torch.empty(0, dtype=dtype))
+    return int(load_library().gdn_chunk_prefill_layer_workspace_size(
+        int(N), int(T), int(HK), int(HV), int(dk), int(dv), int(chunk), code,
+        int(bool(varlen)), int(bool(has_conv))))
+
+
+def gdn_chunk_prefill_layer(q, k, v, g, beta, h0=None, cu_seqlens=None, conv_weight=None,
+                            conv_bias=None, conv_state=None, z=None, chunk: int = 64,
+                            scale: float = 1.0, o=None, hT=None, workspace=None, stream=None,
+                            output_final_state: bool = True, prologue: int = 0,
+                            silu: bool = False):
+    """Prefill with the layer steps (``gdn_chunk_prefill_layer``): the short
+    convolution of v (``conv_state`` [N,W-1,HV*dv] carried and updated when
+    given), the rule, and the gate o <- o * sigmoid(z) (z like v).  Other
+    arguments as in ``gdn_chunk_prefill``.  Returns (o, hT or None)."""
+    lib = load_library()
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("expected q,k [B,T,HK,dk] and v [B,T,HV,dv]")
+    B, T, HK, dk = q.shape
+    HV, dv = v.shape[2], v.shape[3]
+    g_shape = (B, T, HV, dv) if prologue & ROW_DECAY else (B, T, HV)
+    if g.shape != g_shape or beta.shape != (B, T, HV):
+        raise ValueError(f"expected g {g_shape} and beta [B,T,HV]")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        if B != 1:
+            raise ValueError("with cu_seqlens the batch dimension must be 1 (packed)")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    W = _conv_args(conv_weight, conv_bias, conv_state, HV * dv, N, q.dtype, dev)
+    if z is not None:
+        _need(z, "z", q.dtype, dev)
+        if z.shape != v.shape:
+            raise ValueError("z must have v's shape")
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, dev)
+        if h0.shape != (N, HV, dv, dk):
+            raise ValueError(f"h0 must be [N,HV,dv,dk] = {(N, HV, dv, dk)}")
+    if o is None:
+        o = torch.empty_like(v)
+    else:
+        _need(o, "o", v.dtype, dev)
+    if hT is None and output_final_state:
+        hT = torch.empty((N, HV, dv, dk), dtype=torch.float32, device=dev)
+    elif hT is not None:
+        _need(hT, "hT", torch.float32, dev)
+    code = _dtype_code(q)
+    need = lib.gdn_chunk_prefill_layer_workspace_size(N, T, HK, HV, dk, dv, chunk, code,
+                                                      int(cu_seqlens is not None),
+                                                      int(conv_weight is not None))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    flags = int(prologue) | (CONV_SILU if silu else 0)
+    st = lib.gdn_chunk_prefill_layer(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                     _ptr(cu_seqlens), N, T, HK, HV, dk, dv, int(chunk),
+                                     float(scale), code, _ptr(o), _ptr(hT), _ptr(conv_weight),
+                                     _ptr(conv_bias), _ptr(conv_state), W, _ptr(z), flags,
+                                     _ptr(workspace), ws_bytes, _stream_ptr(stream, dev))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_chunk_prefill_layer")
+    return o, hT

@@ -164,6 +164,19 @@ def row_decays(shape, seed: int, low: float = 0.8, high: float = 1.0):
     return torch.log(low + (high - low) * torch.rand(tuple(shape), generator=gen)).float()
 
 
+def layer_extras(N: int, C: int, width: int, z_shape, dtype=torch.bfloat16, seed: int = 0):
+    """Seeded inputs of the layer steps around the rule (random draws only):
+    short-convolution weights [C, width] ~ N(0, 1/width) and bias [C] ~ N(0, 0.1^2)
+    (fp32), a carried convolution state [N, width-1, C] ~ N(0, 1) and gate
+    logits z of ``z_shape`` ~ N(0, 1), both in ``dtype``."""
+    gen = torch.Generator().manual_seed(seed)
+    w = (torch.randn((C, width), generator=gen) / width ** 0.5).float()
+    b = (0.1 * torch.randn((C,), generator=gen)).float()
+    cs = torch.randn((N, max(width - 1, 0), C), generator=gen).to(dtype)
+    z = torch.randn(tuple(z_shape), generator=gen).to(dtype)
+    return {"conv_weight": w, "conv_bias": b, "conv_state": cs, "z": z}
+
+
 def workload_inputs(name: str, steps: int | None = None, seed_offset: int = 0,
                     tokens: int | None = None):
     """Inputs for one named workload (see ``WORKLOADS``).  ``seed_offset`` gives

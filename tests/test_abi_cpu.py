@@ -234,3 +234,95 @@ def test_commit_verify_validation(lib):
     assert call(ws=fake(0xd000), ws_bytes=need - 16) == gdn.GDN_ERR_WORKSPACE
     assert call(ws=fake(0xd008), ws_bytes=need) == gdn.GDN_ERR_ALIGNMENT
     assert call(N=0, q=None, pk=None) == gdn.GDN_OK
+
+
+# ---- the layer steps (short convolution, output gate); fake pointers never reach a launch
+def conv_call(lib, **kw):
+    a = dict(x=fake(0x1000), w=fake(0x2000), b=None, cs=None, cu=None, N=1, T=64, C=64, W=4,
+             flags=0, dtype=gdn.GDN_BF16, y=fake(0x3000))
+    a.update(kw)
+    return lib.gdn_short_conv(a["x"], a["w"], a["b"], a["cs"], a["cu"], a["N"], a["T"], a["C"],
+                              a["W"], a["flags"], a["dtype"], a["y"], None)
+
+
+def test_short_conv_validation(lib):
+    assert conv_call(lib, flags=32) == gdn.GDN_ERR_INVALID_ARG
+    assert conv_call(lib, x=None) == gdn.GDN_ERR_INVALID_ARG
+    assert conv_call(lib, w=None) == gdn.GDN_ERR_INVALID_ARG
+    assert conv_call(lib, y=None) == gdn.GDN_ERR_INVALID_ARG
+    assert conv_call(lib, N=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert conv_call(lib, C=0) == gdn.GDN_ERR_INVALID_ARG
+    assert conv_call(lib, dtype=7) == gdn.GDN_ERR_INVALID_ARG
+    assert conv_call(lib, W=1) == gdn.GDN_ERR_UNSUPPORTED
+    assert conv_call(lib, W=gdn.CONV_MAX_WIDTH + 1) == gdn.GDN_ERR_UNSUPPORTED
+    assert conv_call(lib, C=12) == gdn.GDN_ERR_UNSUPPORTED                 # bf16: 8 per vector
+    assert conv_call(lib, C=12, dtype=gdn.GDN_F32, x=fake(0x1008)) == gdn.GDN_ERR_ALIGNMENT
+    assert conv_call(lib, cs=fake(0x4004)) == gdn.GDN_ERR_ALIGNMENT
+    assert conv_call(lib, N=0) == gdn.GDN_OK                                # empty batch
+
+
+def test_output_gate_validation(lib):
+    def call(o=fake(0x1000), z=fake(0x2000), rows=4, C=64, dtype=gdn.GDN_F32):
+        return lib.gdn_output_gate(o, z, rows, C, dtype, None)
+    assert call(o=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(z=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(rows=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert call(C=0) == gdn.GDN_ERR_INVALID_ARG
+    assert call(dtype=5) == gdn.GDN_ERR_INVALID_ARG
+    assert call(rows=1, C=3) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(z=fake(0x2004)) == gdn.GDN_ERR_ALIGNMENT
+    assert call(rows=0) == gdn.GDN_OK
+
+
+def step_layer_call(lib, **kw):
+    a = dict(q=fake(0x1000), k=fake(0x2000), v=fake(0x3000), g=fake(0x4000), beta=fake(0x5000),
+             state=fake(0x6000), w=fake(0x7000), b=None, cs=fake(0x8000), W=4, z=fake(0x9000),
+             N=2, HK=1, HV=2, dk=64, dv=64, dtype=gdn.GDN_BF16, o=fake(0xa000), flags=0)
+    a.update(kw)
+    return lib.gdn_recurrent_step_layer(a["q"], a["k"], a["v"], a["g"], a["beta"], a["state"],
+                                        a["w"], a["b"], a["cs"], a["W"], a["z"], a["N"], a["HK"],
+                                        a["HV"], a["dk"], a["dv"], 1.0, a["dtype"], a["o"],
+                                        a["flags"], None)
+
+
+def test_step_layer_validation(lib):
+    assert step_layer_call(lib, flags=32) == gdn.GDN_ERR_INVALID_ARG
+    assert step_layer_call(lib, o=None) == gdn.GDN_ERR_INVALID_ARG
+    assert step_layer_call(lib, cs=None) == gdn.GDN_ERR_INVALID_ARG         # conv without state
+    assert step_layer_call(lib, W=1) == gdn.GDN_ERR_UNSUPPORTED
+    assert step_layer_call(lib, W=9) == gdn.GDN_ERR_UNSUPPORTED
+    assert step_layer_call(lib, dk=48) == gdn.GDN_ERR_UNSUPPORTED
+    assert step_layer_call(lib, z=fake(0x9001)) == gdn.GDN_ERR_ALIGNMENT     # bf16: 2-byte
+    assert step_layer_call(lib, cs=fake(0x8001)) == gdn.GDN_ERR_ALIGNMENT
+    assert step_layer_call(lib, q=fake(0x1008)) == gdn.GDN_ERR_ALIGNMENT
+    assert step_layer_call(lib, N=0) == gdn.GDN_OK
+    assert step_layer_call(lib, N=0, w=None, cs=None, z=None,
+                           flags=gdn.PROLOGUE_ALL | gdn.ROW_DECAY | gdn.CONV_SILU) == gdn.GDN_OK
+
+
+def prefill_layer_call(lib, **kw):
+    a = dict(q=fake(0x1000), k=fake(0x2000), v=fake(0x3000), g=fake(0x4000), beta=fake(0x5000),
+             N=1, T=64, HK=1, HV=2, dk=32, dv=32, chunk=16, dtype=gdn.GDN_F32, o=fake(0x6000),
+             w=fake(0x7000), b=None, cs=None, W=4, z=None, flags=0, ws=None, ws_bytes=0)
+    a.update(kw)
+    return lib.gdn_chunk_prefill_layer(a["q"], a["k"], a["v"], a["g"], a["beta"], None, None,
+                                       a["N"], a["T"], a["HK"], a["HV"], a["dk"], a["dv"],
+                                       a["chunk"], 1.0, a["dtype"], a["o"], None, a["w"], a["b"],
+                                       a["cs"], a["W"], a["z"], a["flags"], a["ws"], a["ws_bytes"],
+                                       None)
+
+
+def test_prefill_layer_validation(lib):
+    assert prefill_layer_call(lib, flags=32) == gdn.GDN_ERR_INVALID_ARG
+    assert prefill_layer_call(lib, q=None) == gdn.GDN_ERR_INVALID_ARG
+    assert prefill_layer_call(lib, dk=48) == gdn.GDN_ERR_UNSUPPORTED
+    assert prefill_layer_call(lib, W=9) == gdn.GDN_ERR_UNSUPPORTED
+    assert prefill_layer_call(lib, z=fake(0x9008)) == gdn.GDN_ERR_ALIGNMENT
+    # the convolved values need workspace: none given
+    assert prefill_layer_call(lib) == gdn.GDN_ERR_WORKSPACE
+    need = lib.gdn_chunk_prefill_layer_workspace_size(1, 64, 1, 2, 32, 32, 16, gdn.GDN_F32, 0, 1)
+    assert need >= 64 * 2 * 32 * 4
+    assert prefill_layer_call(lib, ws=fake(0x10000), ws_bytes=need - 1) == gdn.GDN_ERR_WORKSPACE
+    assert prefill_layer_call(lib, ws=fake(0x10008), ws_bytes=need) == gdn.GDN_ERR_ALIGNMENT
+    assert prefill_layer_call(lib, N=0) == gdn.GDN_OK
+    assert lib.gdn_chunk_prefill_layer_workspace_size(1, 64, 1, 2, 32, 32, 16, gdn.GDN_F32, 0, 0) == 0

@@ -1,0 +1,241 @@
+"""The layer steps around the rule -- the short causal convolution on the values
+and the sigmoid output gate -- through the C ABI, alone and fused into the
+decode step and the prefill, against the float64 oracle's ``short_conv``,
+``output_gate``, ``layer_step`` and ``layer_prefill``."""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_recurrence_rule_b200 import (PROLOGUE_ALL, ROW_DECAY, gdn_chunk_prefill_layer,
+                                                   gdn_output_gate, gdn_recurrent_step_layer,
+                                                   gdn_short_conv)
+from linear_attention_recurrence_rule_b200.inputs import (layer_extras, make_decode, make_prefill,
+                                                          raw_projections, row_decays,
+                                                          workload_inputs)
+from oracle import gdn_oracle as O
+from parity_util import assert_close, head_slice, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def packed_x(lengths, C, dtype, seed):
+    gen = torch.Generator().manual_seed(seed)
+    T = sum(lengths)
+    x = torch.randn(1, T, C, generator=gen).to(dtype)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32)
+    return x, cu
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("width", [2, 4, 8])
+@pytest.mark.parametrize("silu,with_state", [(False, False), (True, True)])
+def test_short_conv_packed_ragged(dtype, width, silu, with_state):
+    # lengths below width-1, around the 32-token runs and an empty sequence
+    lengths = [0, 1, 2, 37, 64, 100, 3, 31, 33]
+    C = 64
+    x, cu = packed_x(lengths, C, dtype, seed=301 + width)
+    ex = layer_extras(len(lengths), C, width, (1,), dtype, seed=302 + width)
+    cs = ex["conv_state"] if with_state else None
+    y_ref, s_ref = O.short_conv(x, ex["conv_weight"], ex["conv_bias"], cs, cu, "silu" if silu else "none")
+    cs_dev = cs.cuda() if with_state else None
+    y = gdn_short_conv(x.cuda(), ex["conv_weight"].cuda(), ex["conv_bias"].cuda(), cs_dev,
+                       cu.cuda(), silu=silu)
+    torch.cuda.synchronize()
+    assert_close(y[0], y_ref, dtype, "y")
+    if with_state:
+        # the new state holds raw inputs: bit-exact copies
+        assert torch.equal(cs_dev.cpu(), torch.from_numpy(s_ref).to(dtype))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_short_conv_batched_no_bias(dtype):
+    B, T, C, W = 3, 70, 96, 4
+    gen = torch.Generator().manual_seed(303)
+    x = torch.randn(B, T, C, generator=gen).to(dtype)
+    ex = layer_extras(B, C, W, (1,), dtype, seed=304)
+    y_ref, s_ref = O.short_conv(x, ex["conv_weight"], None, ex["conv_state"])
+    cs = ex["conv_state"].cuda()
+    y = gdn_short_conv(x.cuda(), ex["conv_weight"].cuda(), None, cs)
+    torch.cuda.synchronize()
+    assert_close(y.reshape(B * T, C), y_ref, dtype, "y")
+    assert torch.equal(cs.cpu(), torch.from_numpy(s_ref).to(dtype))
+
+
+def test_short_conv_bench_size_sampled_channels():
+    # the 64K-token value tensor of the bench (4096 channels); each channel is
+    # independent, so a sample of channels checks the whole launch's indexing
+    w = workload_inputs("long_prefill_64k")
+    x = w["v"].reshape(1, 65536, -1)
+    C = x.shape[-1]
+    ex = layer_extras(1, C, 4, (1,), torch.bfloat16, seed=305)
+    cs = ex["conv_state"].cuda()
+    y = gdn_short_conv(x.cuda(), ex["conv_weight"].cuda(), ex["conv_bias"].cuda(), cs, silu=True)
+    torch.cuda.synchronize()
+    chans = np.r_[0:8, 1000:1008, 2048:2056, C - 8:C]
+    y_ref, s_ref = O.short_conv(x[:, :, chans], ex["conv_weight"][chans], ex["conv_bias"][chans],
+                                ex["conv_state"][:, :, chans], activation="silu")
+    assert_close(y[0][:, chans], y_ref, torch.bfloat16, "y (sampled channels)")
+    assert torch.equal(cs.cpu()[:, :, chans], torch.from_numpy(s_ref).to(torch.bfloat16))
+    assert torch.equal(cs.cpu()[0], x[0, -3:])
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_output_gate(dtype):
+    gen = torch.Generator().manual_seed(306)
+    o = torch.randn(37, 3, 64, generator=gen).to(dtype)
+    z = (3.0 * torch.randn(37, 3, 64, generator=gen)).to(dtype)
+    ref = O.output_gate(o, z)
+    od = o.cuda()
+    gdn_output_gate(od, z.cuda())
+    torch.cuda.synchronize()
+    assert_close(od, ref, dtype, "gated o")
+
+
+def _step_inputs(N, HK, HV, d, dtype, steps, seed, width=4):
+    x = make_decode(N, steps, HK, HV, d, d, dtype, seed=seed)
+    ex = layer_extras(N, HV * d, width, (steps, N, HV, d), dtype, seed=seed + 1)
+    return x, ex
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+@pytest.mark.parametrize("conv,gate,silu", [(True, True, True), (True, False, False),
+                                            (False, True, False)])
+def test_step_layer_matches_oracle(dtype, d, conv, gate, silu):
+    N, HK, HV, steps = 5, 2, 4, 4
+    x, ex = _step_inputs(N, HK, HV, d, dtype, steps, seed=310)
+    S_ref, cs_ref = x["state"].double().numpy(), ex["conv_state"]
+    S, cs = x["state"].cuda(), ex["conv_state"].cuda()
+    w, b = ex["conv_weight"].cuda(), ex["conv_bias"].cuda()
+    for t in range(steps):
+        z = ex["z"][t] if gate else None
+        o = gdn_recurrent_step_layer(x["q"][t].cuda(), x["k"][t].cuda(), x["v"][t].cuda(),
+                                     x["g"][t].cuda(), x["beta"][t].cuda(), S,
+                                     conv_weight=w if conv else None, conv_bias=b if conv else None,
+                                     conv_state=cs if conv else None,
+                                     z=z.cuda() if gate else None, scale=0.8, silu=silu)
+        o_ref, S_ref, cs_new = O.layer_step(x["q"][t], x["k"][t], x["v"][t], x["g"][t],
+                                            x["beta"][t], S_ref,
+                                            ex["conv_weight"] if conv else None, ex["conv_bias"],
+                                            cs_ref, z, scale=0.8,
+                                            activation="silu" if silu else "none")
+        if conv:
+            cs_ref = cs_new
+        torch.cuda.synchronize()
+        assert_close(o, o_ref, dtype, f"o step {t}")
+    assert_close(S, S_ref, dtype, "state")
+    if conv:
+        assert torch.equal(cs.cpu(), torch.from_numpy(cs_ref).to(dtype))
+
+
+def test_step_layer_with_prologue_and_row_decay():
+    N, HK, HV, d, steps = 3, 2, 4, 128, 3
+    x, ex = _step_inputs(N, HK, HV, d, torch.bfloat16, steps, seed=320)
+    raw = raw_projections({k: x[k] for k in ("q", "k", "g", "beta", "v")}, seed=321)
+    gr = row_decays((steps, N, HV, d), seed=322)
+    flags = PROLOGUE_ALL & ~4 | ROW_DECAY     # norms on, decays given as log values per row
+    S_ref, cs_ref = x["state"].double().numpy(), ex["conv_state"]
+    S, cs = x["state"].cuda(), ex["conv_state"].cuda()
+    for t in range(steps):
+        o = gdn_recurrent_step_layer(raw["q"][t].cuda(), raw["k"][t].cuda(), x["v"][t].cuda(),
+                                     gr[t].cuda(), x["beta"][t].cuda(), S,
+                                     conv_weight=ex["conv_weight"].cuda(),
+                                     conv_bias=ex["conv_bias"].cuda(), conv_state=cs,
+                                     z=ex["z"][t].cuda(), prologue=flags, silu=True)
+        qn, kn, _, _ = O.prologue(raw["q"][t], raw["k"][t], x["g"][t], x["beta"][t], flags & 3)
+        vc, cs_ref = O.short_conv(x["v"][t].reshape(N, 1, HV * d), ex["conv_weight"],
+                                  ex["conv_bias"], cs_ref, activation="silu")
+        o_ref, S_ref = O.step_row_decay(qn, kn, vc.reshape(N, HV, d), gr[t], x["beta"][t], S_ref)
+        o_ref = O.output_gate(o_ref, ex["z"][t])
+        torch.cuda.synchronize()
+        assert_close(o, o_ref, torch.bfloat16, f"o step {t}")
+    assert_close(S, S_ref, torch.bfloat16, "state")
+    assert torch.equal(cs.cpu(), torch.from_numpy(cs_ref).to(torch.bfloat16))
+
+
+def _layer_problem(lengths, dtype, d, chunk_seed, HK=2, HV=4, width=4):
+    x = make_prefill(HK, HV, d, d, lengths, dtype, seed=chunk_seed, h0_std=0.05)
+    N = len(lengths)
+    ex = layer_extras(N, HV * d, width, x["v"].shape, dtype, seed=chunk_seed + 1)
+    return x, ex
+
+
+def _run_layer_prefill(x, ex, chunk, silu, conv=True, gate=True, cs=None):
+    d = to_dev(x)
+    return gdn_chunk_prefill_layer(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
+                                   cu_seqlens=d["cu_seqlens"],
+                                   conv_weight=ex["conv_weight"].cuda() if conv else None,
+                                   conv_bias=ex["conv_bias"].cuda() if conv else None,
+                                   conv_state=cs, z=ex["z"].cuda() if gate else None,
+                                   chunk=chunk, scale=0.7, silu=silu)
+
+
+@pytest.mark.parametrize("dtype,d,chunk", [(torch.bfloat16, 128, 64), (torch.float32, 32, 16)])
+@pytest.mark.parametrize("conv,gate", [(True, True), (True, False), (False, True)])
+def test_prefill_layer_matches_oracle(dtype, d, chunk, conv, gate):
+    lengths = [300, 77, 0, 129]
+    x, ex = _layer_problem(lengths, dtype, d, 330)
+    cs = ex["conv_state"].cuda() if conv else None
+    o, hT = _run_layer_prefill(x, ex, chunk, silu=True, conv=conv, gate=gate, cs=cs)
+    torch.cuda.synchronize()
+    o_ref, h_ref, cs_ref = O.layer_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"],
+                                           ex["conv_weight"] if conv else None, ex["conv_bias"],
+                                           ex["conv_state"] if conv else None,
+                                           ex["z"] if gate else None, h0=x["h0"],
+                                           cu_seqlens=x["cu_seqlens"], scale=0.7,
+                                           activation="silu")
+    assert_close(o[0], o_ref, dtype, "o")
+    assert_close(hT, h_ref, dtype, "hT")
+    if conv:
+        assert torch.equal(cs.cpu(), torch.from_numpy(cs_ref).to(dtype))
+
+
+def test_prefill_layer_then_steps_continue_the_sequence():
+    # a layer prefill of the first 150 tokens, then 5 layer decode steps with both
+    # states carried, equals the oracle's layer over all 155 tokens
+    T0, T1, HV, d = 150, 5, 4, 128
+    x, ex = _layer_problem([T0 + T1, T0 + T1], torch.bfloat16, d, 340)
+    o_ref, h_ref, cs_ref = O.layer_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"],
+                                           ex["conv_weight"], ex["conv_bias"], ex["conv_state"],
+                                           ex["z"], h0=x["h0"], scale=0.7, activation="silu")
+    o_ref = o_ref.reshape(2, T0 + T1, HV, d)
+    first = {k: (v[:, :T0].contiguous() if isinstance(v, torch.Tensor) and k != "h0" else v)
+             for k, v in x.items()}
+    ex0 = dict(ex, z=ex["z"][:, :T0].contiguous())
+    cs = ex["conv_state"].cuda()
+    o0, S = _run_layer_prefill(first, ex0, 64, silu=True, cs=cs)
+    torch.cuda.synchronize()
+    assert_close(o0, o_ref[:, :T0], torch.bfloat16, "o (prefill part)")
+    for t in range(T0, T0 + T1):
+        o = gdn_recurrent_step_layer(x["q"][:, t].contiguous().cuda(),
+                                     x["k"][:, t].contiguous().cuda(),
+                                     x["v"][:, t].contiguous().cuda(),
+                                     x["g"][:, t].contiguous().cuda(),
+                                     x["beta"][:, t].contiguous().cuda(), S,
+                                     conv_weight=ex["conv_weight"].cuda(),
+                                     conv_bias=ex["conv_bias"].cuda(), conv_state=cs,
+                                     z=ex["z"][:, t].contiguous().cuda(), scale=0.7, silu=True)
+        torch.cuda.synchronize()
+        assert_close(o, o_ref[:, t], torch.bfloat16, f"o step {t}")
+    assert_close(S, h_ref, torch.bfloat16, "state after the steps")
+    assert torch.equal(cs.cpu(), torch.from_numpy(cs_ref).to(torch.bfloat16))
+
+
+def test_prefill_layer_bench_size_sampled_heads():
+    # the bench's 64K layer prefill (convolution + rule + gate, all 32 value heads
+    # in one call); the oracle checks two query/key heads and their value heads
+    x = workload_inputs("long_prefill_64k")
+    HV, dv = x["v"].shape[2], x["v"].shape[3]
+    ex = layer_extras(1, HV * dv, 4, x["v"].shape, torch.bfloat16, seed=350)
+    cs = ex["conv_state"].cuda()
+    o, hT = _run_layer_prefill(x, ex, 64, silu=True, cs=cs)
+    torch.cuda.synchronize()
+    for qk in ([0], [15]):
+        sub, vh = head_slice(x, qk, HV // x["q"].shape[2])
+        ch = np.concatenate([np.arange(h * dv, (h + 1) * dv) for h in vh])
+        o_ref, h_ref, cs_ref = O.layer_prefill(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"],
+                                               ex["conv_weight"][ch], ex["conv_bias"][ch],
+                                               ex["conv_state"][:, :, ch], ex["z"][:, :, vh],
+                                               h0=sub["h0"], scale=0.7, activation="silu")
+        assert_close(o[0][:, vh], o_ref, torch.bfloat16, f"o heads {vh}")
+        assert_close(hT[:, vh], h_ref, torch.bfloat16, f"hT heads {vh}")
+        assert torch.equal(cs.cpu()[:, :, ch], torch.from_numpy(cs_ref).to(torch.bfloat16))
