@@ -323,9 +323,10 @@ def _time_events(torch, stream, fn, reps, warm=3):
 
 def measure_layer(gdn, torch, dev, stream, x, w, o, hT, rank, peaks, peak_src, plain_s, args):
     """The layer steps around the rule: the bench prefill with the short
-    convolution on v (width 4, SiLU, carried state) and the output gate, one
-    call; the convolution and the gate kernels alone with their HBM rooflines;
-    and the decode step of decode_256x64 with both fused into it."""
+    convolution on v (width 4, SiLU, carried state) and the output gate (fused
+    into the prefill's read-out), one call; the convolution and the standalone
+    gate kernels alone with their HBM rooflines; and the decode step of
+    decode_256x64 with both fused into it."""
     from linear_attention_recurrence_rule_b200.inputs import (WORKLOADS, layer_extras,
                                                               workload_inputs)
     W = 4
@@ -396,7 +397,8 @@ def measure_layer(gdn, torch, dev, stream, x, w, o, hT, rank, peaks, peak_src, p
             "prefill": {"workload": WORKLOAD, "ms_per_step": lp_ms,
                         "value": tokens / (lp_ms / 1e3), "unit": "tokens/s",
                         "plain_ms_per_step": plain_s * 1e3, "overhead": lp_ms / (plain_s * 1e3) - 1.0,
-                        "gpu_launches": 4},
+                        "gpu_launches": 3,
+                        "launches": "convolution + carried state, prefill with the gate in its read-out"},
             "conv_kernel": {"ms": cv_ms, "bytes": cv_bytes, "gpu_launches": 2,
                             "roofline": {"bound": "hbm", "achieved": cv_bytes / (cv_ms / 1e3) / 1e9,
                                          "peak": hbm, "unit": "GB/s",

@@ -479,11 +479,14 @@ GDN_API size_t gdn_chunk_prefill_layer_workspace_size(int N, int64_t T, int HK, 
 
 /*
  * gdn_chunk_prefill_ex with the layer steps: the short convolution of v
- * (into the workspace; conv_state [N][conv_width-1][HV*dv] updated as in
- * gdn_short_conv), the prefill on the convolved values, then the output gate
- * on o.  conv_weight NULL: no convolution; z NULL: no gate.  flags:
- * GDN_PROLOGUE_*, GDN_ROW_DECAY and GDN_CONV_SILU.  Up to three launch groups
- * on `stream`; arguments as in gdn_chunk_prefill_ex and gdn_short_conv.
+ * (gdn_short_conv into the workspace, stored in the call's dtype -- the
+ * tensor-core path takes bf16 operands; conv_state [N][conv_width-1][HV*dv]
+ * updated as there), then the prefill on the convolved values with the output
+ * gate o <- o * sigmoid(z) applied where the prefill writes o (z like v, one
+ * rounding of o).  conv_weight NULL: no convolution; z NULL: no gate.  flags:
+ * GDN_PROLOGUE_*, GDN_ROW_DECAY and GDN_CONV_SILU.  Launches on `stream`: the
+ * convolution's two, then the prefill's one; arguments as in
+ * gdn_chunk_prefill_ex and gdn_short_conv.  z 16-byte aligned.
  */
 GDN_API gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v,
                                            const float *g, const float *beta, const float *h0,

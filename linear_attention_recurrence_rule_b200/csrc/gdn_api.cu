@@ -502,7 +502,6 @@ gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, 
     gdn_status st = check_prefill(a);
     if (st != GDN_OK) return st;
     const bool varlen = cu_seqlens != nullptr;
-    const int64_t tokens = varlen ? T : (int64_t)N * T;
     if ((size_t)HV * dv > 0x7fffffffu) return GDN_ERR_UNSUPPORTED;
     const int C = HV * dv;
     gdn::ConvArgs ca{v, conv_weight, conv_bias, conv_state, cu_seqlens, N, T, C, conv_width,
@@ -512,10 +511,7 @@ gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, 
         st = check_conv(ca);
         if (st != GDN_OK) return st;
     }
-    if (z) {
-        if ((tokens * (int64_t)C) % gdn::conv_vector_channels(dtype)) return GDN_ERR_UNSUPPORTED;
-        if (!aligned16(z)) return GDN_ERR_ALIGNMENT;
-    }
+    if (z && !aligned16(z)) return GDN_ERR_ALIGNMENT;
     if (N == 0) return GDN_OK;
     // workspace: [prefill's own | convolved values]
     const size_t pre = up256(gdn::prefill_cluster_supported(dk, dv, chunk, dtype) && !(prologue & GDN_ROW_DECAY)
@@ -532,11 +528,8 @@ gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, 
     }
     a.workspace_bytes = pre;
     if (pre == 0) a.workspace = nullptr;
-    st = enqueue_prefill(a, s);
-    if (st != GDN_OK) return st;
-    if (z && gdn::launch_output_gate(o, z, tokens * (int64_t)C, dtype, s) != cudaSuccess)
-        return GDN_ERR_CUDA;
-    return GDN_OK;
+    a.z = z;   // the gate is applied in the prefill's read-out, before o is rounded
+    return enqueue_prefill(a, s);
 }
 
 gdn_status gdn_read_status(const void *workspace, size_t workspace_bytes, gdn_stream_t stream) {

@@ -24,6 +24,7 @@ struct PrefillArgs {
     size_t workspace_bytes;
     bool keep_status = false;   // leave the workspace status word as earlier calls left it
     unsigned prologue = 0;      // GDN_PROLOGUE_* flags
+    const void *z = nullptr;    // output gate logits, like o (gdn_chunk_prefill_layer)
 };
 
 struct StepArgs {

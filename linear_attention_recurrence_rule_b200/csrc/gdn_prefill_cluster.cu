@@ -27,7 +27,9 @@
 //     S += (U diag(gamma_L / gamma)) K accumulates in tensor memory after an
 //     in-place gamma_L scaling, and the outputs are gamma_t S0 Q^T + U P^T;
 //     sixteen epilogue warps share every epilogue (16 tokens or 32 state columns
-//     each) and write chunk c's outputs while chunk c + 1's first products run.
+//     each) and write chunk c's outputs while chunk c + 1's first products run
+//     (with the layer's output gate, o * sigmoid(z) before the rounding to bf16;
+//     z loaded while the state is rescaled).
 // The chain's critical loop hands over between its epilogue warps and the
 // MMA-issuing warp through named barriers (no sleeping wake-up on that path);
 // tensor-core completions and cross-CTA hand-overs use mbarriers.
@@ -145,6 +147,7 @@ struct ClParams {
     float *hT;
     unsigned int *status;
     unsigned int prologue;   // GDN_PROLOGUE_* flags
+    const __nv_bfloat16 *z = nullptr;   // output gate logits [tokens][HV][dv] (GT instances)
 };
 
 struct Waiter {
@@ -201,6 +204,9 @@ __device__ __forceinline__ void load_qkv_slot(const CUtensorMap *tm_q, const CUt
     }
 }
 
+// GT: the output gate o <- o * sigmoid(z) is applied in the read-out, before the
+// one rounding to bf16 (z loaded a chunk ahead, while the state is rescaled)
+template <bool GT>
 __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                           const CUtensorMap *tm_o, const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
                           const Waiter &wt, int h, int n, int64_t bos, int64_t eos, int nchunks) {
@@ -345,6 +351,17 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
         if (nchunks > 0) named_sync(NB_S0, kChainSync);
         bool ok = true;
         float dq[16];            // scale * gamma_t * (S0 q_t) of the previous chunk
+        unsigned short zr[GT ? 16 : 1];   // gate logits of the chunk being read out (raw bf16)
+        // gate logits of chunk cp for this warp's 16 tokens x 32 value rows
+        auto load_z = [&](int cp) {
+            const int64_t ps0 = bos + (int64_t)cp * C;
+            const int pL = chunk_len(cp);
+            const unsigned short *zb = reinterpret_cast<const unsigned short *>(p.z) +
+                                       ((size_t)(ps0 + 16 * part) * HV + h) * DH + i;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                zr[GT ? j : 0] = 16 * part + j < pL ? zb[(size_t)j * HV * DH] : (unsigned short)0;
+        };
         // read-out of chunk cp: o_t = dq + scale (U P^T)_t for this warp's 16 tokens x
         // 32 value rows, put into a per-warp shared tile [t][i] and written by one
         // TMA store of the warp (plain 16-byte stores for tokens of a short last chunk)
@@ -360,7 +377,9 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const __nv_bfloat16 b = __float2bfloat16_rn(fmaf(p.scale, dout[j], dq[j]));
+                float out = fmaf(p.scale, dout[j], dq[j]);
+                if (GT) out *= gate_sigmoid(__uint_as_float((uint32_t)zr[GT ? j : 0] << 16));
+                const __nv_bfloat16 b = __float2bfloat16_rn(out);
                 ot[j * 32 + lane] = *reinterpret_cast<const unsigned short *>(&b);
             }
             if (16 * part + 16 <= pL) {
@@ -389,6 +408,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             const int L = chunk_len(c);
             const uint8_t *slot = sm + C_R + s * SLOT;
             const float *tab = reinterpret_cast<const float *>(slot + SL_TAB);
+            if (GT && c > 0) load_z(c - 1);   // in flight while the state is rescaled
             ok = warp_all(ok && wt(CB_R_FULL0 + s, (uint32_t)((c >> 1) & 1)));
             if (ok) {
                 // scale the fp32 state by this chunk's gamma_L before its update
@@ -507,6 +527,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             if (more) named_sync(NB_S0, kChainSync);
         }
         if (nchunks > 0) {
+            if (GT) load_z(nchunks - 1);
             ok = warp_all(ok && wt(CB_O_FULL, (uint32_t)((nchunks - 1) & 1)));
             if (ok) {
                 tc_fence_after();
@@ -884,7 +905,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     }
 }
 
-template <bool PRO>
+template <bool PRO, bool GT>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -942,7 +963,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     cluster_sync_all();   // every CTA's barriers are initialised before any remote traffic
 
     if (rank == 0)
-        chain_cta(&tm_q, &tm_k, &tm_v, &tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
+        chain_cta<GT>(&tm_q, &tm_k, &tm_v, &tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
     else
         prep_cta<PRO>(&tm_q, &tm_k, &tm_v, p, sm, sb, tmem, wt, h, bos, eos, nchunks, rank);
 
@@ -987,12 +1008,14 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     uint32_t obox[3] = {32, 1, 16};
     if (!encode_bf16_map(&to, a.o, 3, dv, sv, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    auto kern = a.prologue ? prefill_cluster_kernel<true> : prefill_cluster_kernel<false>;
+    auto kern = a.z ? (a.prologue ? prefill_cluster_kernel<true, true> : prefill_cluster_kernel<false, true>)
+                    : (a.prologue ? prefill_cluster_kernel<true, false> : prefill_cluster_kernel<false, false>);
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     ClParams prm{a.g, a.beta, a.h0, a.cu_seqlens, a.T, a.HK, a.HV, a.scale,
                  static_cast<__nv_bfloat16 *>(a.o), a.hT, status, a.prologue};
+    prm.z = static_cast<const __nv_bfloat16 *>(a.z);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(kClusterSize * a.HV), (unsigned)a.N, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);

@@ -49,7 +49,8 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const Tin *__restrict__ v, const float *__restrict__ g,
                     const float *__restrict__ beta, const float *__restrict__ h0,
                     const int32_t *__restrict__ cu, int64_t T, int HK, int HV, int dv,
-                    float scale, Tin *__restrict__ o, float *__restrict__ hT, unsigned pro) {
+                    float scale, Tin *__restrict__ o, float *__restrict__ hT, unsigned pro,
+                    const Tin *__restrict__ z) {
     using L_ = SimtSmem<DK, BV, C, RD>;
     constexpr int KP = L_::KP, CP = L_::CP, NT = kSimtThreads;
     const int tid = threadIdx.x;
@@ -215,7 +216,10 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                 for (int j = 0; j <= i; ++j) acc = fmaf(Ps[i * CP + j], Ys[j * BV + e], acc);
                 acc = fmaf(expf(Gs[i]), QSs[idx], acc);
             }
-            o[((size_t)(s0 + i) * HV + h) * dv + e0 + e] = from_f32<Tin>(scale * acc);
+            const size_t oi = ((size_t)(s0 + i) * HV + h) * dv + e0 + e;
+            float out = scale * acc;
+            if (z) out *= gate_sigmoid(to_f32(z[oi]));   // output gate, before the one rounding
+            o[oi] = from_f32<Tin>(out);
         }
         __syncthreads();
         // ---- S_L = gamma_L S0 + sum_j exp(G_L - G_j) u_j k_j^T ----
@@ -253,7 +257,7 @@ cudaError_t launch_shape_rd(const PrefillArgs &a, cudaStream_t stream) {
     kern<<<grid, block, smem, stream>>>(
         static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
         static_cast<const Tin *>(a.v), a.g, a.beta, a.h0, a.cu_seqlens, a.T, a.HK, a.HV, a.dv,
-        a.scale, static_cast<Tin *>(a.o), a.hT, a.prologue);
+        a.scale, static_cast<Tin *>(a.o), a.hT, a.prologue, static_cast<const Tin *>(a.z));
     return cudaGetLastError();
 }
 

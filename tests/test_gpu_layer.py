@@ -169,6 +169,35 @@ def _run_layer_prefill(x, ex, chunk, silu, conv=True, gate=True, cs=None):
                                    chunk=chunk, scale=0.7, silu=silu)
 
 
+def ref_layer(x, ex, conv, gate, dtype, scale, stored=None):
+    """The oracle's layer with the convolved values held in the call's dtype
+    between the convolution and the rule, as the prefill call stores them in its
+    workspace (bf16 values feed the tensor cores).  ``stored`` selects the tokens
+    whose convolved values pass through that storage ([B, T] bool; all when None):
+    the decode step keeps them in fp32 on chip."""
+    v = x["v"]
+    vs = v.shape
+    C = vs[-2] * vs[-1]
+    cs_new = None
+    if conv:
+        xv = v.reshape(vs[0], vs[1], C) if x["cu_seqlens"] is None else v.reshape(1, -1, C)
+        vc, cs_new = O.short_conv(xv, ex["conv_weight"], ex["conv_bias"], ex["conv_state"],
+                                  x["cu_seqlens"], activation="silu")
+        vc = torch.from_numpy(vc.reshape(vs))
+        rounded = vc.to(dtype).double()
+        if stored is None:
+            vc = rounded
+        else:
+            vc = torch.where(stored[:, :, None, None], rounded, vc)
+    else:
+        vc = v
+    o, h = O.prefill(x["q"], x["k"], vc, x["g"], x["beta"], h0=x["h0"],
+                     cu_seqlens=x["cu_seqlens"], scale=scale)
+    if gate:
+        o = O.output_gate(o, ex["z"].reshape(o.shape))
+    return o, h, cs_new
+
+
 @pytest.mark.parametrize("dtype,d,chunk", [(torch.bfloat16, 128, 64), (torch.float32, 32, 16)])
 @pytest.mark.parametrize("conv,gate", [(True, True), (True, False), (False, True)])
 def test_prefill_layer_matches_oracle(dtype, d, chunk, conv, gate):
@@ -177,12 +206,7 @@ def test_prefill_layer_matches_oracle(dtype, d, chunk, conv, gate):
     cs = ex["conv_state"].cuda() if conv else None
     o, hT = _run_layer_prefill(x, ex, chunk, silu=True, conv=conv, gate=gate, cs=cs)
     torch.cuda.synchronize()
-    o_ref, h_ref, cs_ref = O.layer_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"],
-                                           ex["conv_weight"] if conv else None, ex["conv_bias"],
-                                           ex["conv_state"] if conv else None,
-                                           ex["z"] if gate else None, h0=x["h0"],
-                                           cu_seqlens=x["cu_seqlens"], scale=0.7,
-                                           activation="silu")
+    o_ref, h_ref, cs_ref = ref_layer(x, ex, conv, gate, dtype, 0.7)
     assert_close(o[0], o_ref, dtype, "o")
     assert_close(hT, h_ref, dtype, "hT")
     if conv:
@@ -194,9 +218,9 @@ def test_prefill_layer_then_steps_continue_the_sequence():
     # states carried, equals the oracle's layer over all 155 tokens
     T0, T1, HV, d = 150, 5, 4, 128
     x, ex = _layer_problem([T0 + T1, T0 + T1], torch.bfloat16, d, 340)
-    o_ref, h_ref, cs_ref = O.layer_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"],
-                                           ex["conv_weight"], ex["conv_bias"], ex["conv_state"],
-                                           ex["z"], h0=x["h0"], scale=0.7, activation="silu")
+    stored = torch.zeros(2, T0 + T1, dtype=torch.bool)
+    stored[:, :T0] = True          # the prefill part stores its convolved values in bf16
+    o_ref, h_ref, cs_ref = ref_layer(x, ex, True, True, torch.bfloat16, 0.7, stored)
     o_ref = o_ref.reshape(2, T0 + T1, HV, d)
     first = {k: (v[:, :T0].contiguous() if isinstance(v, torch.Tensor) and k != "h0" else v)
              for k, v in x.items()}
@@ -232,10 +256,9 @@ def test_prefill_layer_bench_size_sampled_heads():
     for qk in ([0], [15]):
         sub, vh = head_slice(x, qk, HV // x["q"].shape[2])
         ch = np.concatenate([np.arange(h * dv, (h + 1) * dv) for h in vh])
-        o_ref, h_ref, cs_ref = O.layer_prefill(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"],
-                                               ex["conv_weight"][ch], ex["conv_bias"][ch],
-                                               ex["conv_state"][:, :, ch], ex["z"][:, :, vh],
-                                               h0=sub["h0"], scale=0.7, activation="silu")
+        exs = {"conv_weight": ex["conv_weight"][ch], "conv_bias": ex["conv_bias"][ch],
+               "conv_state": ex["conv_state"][:, :, ch], "z": ex["z"][:, :, vh]}
+        o_ref, h_ref, cs_ref = ref_layer(sub, exs, True, True, torch.bfloat16, 0.7)
         assert_close(o[0][:, vh], o_ref, torch.bfloat16, f"o heads {vh}")
         assert_close(hT[:, vh], h_ref, torch.bfloat16, f"hT heads {vh}")
         assert torch.equal(cs.cpu()[:, :, ch], torch.from_numpy(cs_ref).to(torch.bfloat16))
