@@ -112,7 +112,9 @@ constexpr uint32_t P_PB = P_X + 32 * X_LD * 4;   // beta, gamma, G, 1/|q|, 1/|k|
 constexpr uint32_t P_ST = 106496;   // two staging blocks (ST_BYTES each, 1024-aligned)
 constexpr uint32_t P_BAR = P_ST + 2 * ST_BYTES;
 
-enum ChainBar { CB_R_FULL0, CB_R_FULL1, CB_U_MMA, CB_DS_FULL, CB_O_FULL, CB_DRAIN, CB_COUNT };
+// CB_Z0 + w: epilogue warp w's gate-logit tile has landed in its output tile (GT)
+enum ChainBar { CB_R_FULL0, CB_R_FULL1, CB_U_MMA, CB_DS_FULL, CB_O_FULL, CB_DRAIN, CB_Z0,
+                CB_COUNT = CB_Z0 + 16 };
 enum PrepBar { PB_LD_FULL0, PB_LD_FULL1, PB_X_DONE, PB_T_READY, PB_W_DONE, PB_EPI_DONE, PB_GO,
                PB_STAGE_FREE0, PB_STAGE_FREE1, PB_DRAIN, PB_COUNT };
 
@@ -147,7 +149,6 @@ struct ClParams {
     float *hT;
     unsigned int *status;
     unsigned int prologue;   // GDN_PROLOGUE_* flags
-    const __nv_bfloat16 *z = nullptr;   // output gate logits [tokens][HV][dv] (GT instances)
 };
 
 struct Waiter {
@@ -205,10 +206,12 @@ __device__ __forceinline__ void load_qkv_slot(const CUtensorMap *tm_q, const CUt
 }
 
 // GT: the output gate o <- o * sigmoid(z) is applied in the read-out, before the
-// one rounding to bf16 (z loaded a chunk ahead, while the state is rescaled)
+// one rounding to bf16.  Each epilogue warp TMA-loads its 16 x 32 tile of gate
+// logits into its output tile while the state is rescaled, and the read-out
+// overwrites it in place with the gated outputs.
 template <bool GT>
 __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
-                          const CUtensorMap *tm_o, const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
+                          const CUtensorMap *tm_o, const CUtensorMap *tm_z, const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
                           const Waiter &wt, int h, int n, int64_t bos, int64_t eos, int nchunks) {
     uint64_t *bars = wt.bars;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -351,22 +354,27 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
         if (nchunks > 0) named_sync(NB_S0, kChainSync);
         bool ok = true;
         float dq[16];            // scale * gamma_t * (S0 q_t) of the previous chunk
-        unsigned short zr[GT ? 16 : 1];   // gate logits of the chunk being read out (raw bf16)
-        // gate logits of chunk cp for this warp's 16 tokens x 32 value rows
+        // gate logits of chunk cp for this warp's 16 tokens x 32 value rows, into the
+        // warp's output tile once its previous store has been read (tokens past the
+        // end of the data read as zero; those of a next sequence are never stored)
+        uint32_t zst = 0;   // bit 0: phase of the next gate-logit load; bit 1: one in flight
         auto load_z = [&](int cp) {
-            const int64_t ps0 = bos + (int64_t)cp * C;
-            const int pL = chunk_len(cp);
-            const unsigned short *zb = reinterpret_cast<const unsigned short *>(p.z) +
-                                       ((size_t)(ps0 + 16 * part) * HV + h) * DH + i;
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                zr[GT ? j : 0] = 16 * part + j < pL ? zb[(size_t)j * HV * DH] : (unsigned short)0;
+            if (lane == 0) {
+                uint64_t *zbar = &bars[CB_Z0 + (warp - kCEpi0)];
+                bulk_wait_group_read0();
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(zbar, 1024);
+                tma_load_3d(sm + C_OT + (warp - kCEpi0) * 1024, tm_z, zbar, 32 * (warp & 3), h,
+                            (int)(bos + (int64_t)cp * C + 16 * part));
+            }
+            __syncwarp();
+            zst |= 2u;
         };
         // read-out of chunk cp: o_t = dq + scale (U P^T)_t for this warp's 16 tokens x
         // 32 value rows, put into a per-warp shared tile [t][i] and written by one
         // TMA store of the warp (plain 16-byte stores for tokens of a short last chunk)
         unsigned short *ot = reinterpret_cast<unsigned short *>(sm + C_OT + (warp - kCEpi0) * 1024);
-        auto read_out = [&](int cp) {
+        auto read_out = [&](int cp) -> bool {
             const int64_t ps0 = bos + (int64_t)cp * C;
             const int pL = chunk_len(cp);
             float dout[16];
@@ -374,11 +382,19 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             // the tile's previous store has been read out of shared memory
             if (lane == 0) bulk_wait_group_read0();
             __syncwarp();
+            if (GT) {
+                // the gate logits are in the tile
+                const bool zok = warp_all(wt(CB_Z0 + (warp - kCEpi0), zst & 1u));
+                if (zok) zst = (zst & 1u) ^ 1u;
+                tmem_wait_ld();
+                if (!zok) return false;
+            }
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 float out = fmaf(p.scale, dout[j], dq[j]);
-                if (GT) out *= gate_sigmoid(__uint_as_float((uint32_t)zr[GT ? j : 0] << 16));
+                if (GT)
+                    out *= gate_sigmoid(__uint_as_float((uint32_t)ot[j * 32 + lane] << 16));
                 const __nv_bfloat16 b = __float2bfloat16_rn(out);
                 ot[j * 32 + lane] = *reinterpret_cast<const unsigned short *>(&b);
             }
@@ -401,6 +417,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                 }
             }
             __syncwarp();
+            return true;
         };
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t ph = (uint32_t)(c & 1);
@@ -408,7 +425,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             const int L = chunk_len(c);
             const uint8_t *slot = sm + C_R + s * SLOT;
             const float *tab = reinterpret_cast<const float *>(slot + SL_TAB);
-            if (GT && c > 0) load_z(c - 1);   // in flight while the state is rescaled
+            if (GT && c > 0 && ok) load_z(c - 1);   // in flight while the state is rescaled
             ok = warp_all(ok && wt(CB_R_FULL0 + s, (uint32_t)((c >> 1) & 1)));
             if (ok) {
                 // scale the fp32 state by this chunk's gamma_L before its update
@@ -437,7 +454,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                         }
                         __syncwarp();
                     }
-                    read_out(c - 1);
+                    ok = read_out(c - 1);
                 }
             }
             ok = warp_all(ok && wt(CB_U_MMA, ph));
@@ -527,14 +544,16 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             if (more) named_sync(NB_S0, kChainSync);
         }
         if (nchunks > 0) {
-            if (GT) load_z(nchunks - 1);
+            if (GT && ok) load_z(nchunks - 1);
             ok = warp_all(ok && wt(CB_O_FULL, (uint32_t)((nchunks - 1) & 1)));
             if (ok) {
                 tc_fence_after();
-                read_out(nchunks - 1);
+                ok = read_out(nchunks - 1);
             }
         }
-        // this warp's tile stores complete before the CTA's shared memory is released
+        // a gate-logit load still in flight (after an abort) lands before the
+        // CTA's shared memory is released, and so do this warp's tile stores
+        if (GT && (zst & 2u)) wt.drain(CB_Z0 + (warp - kCEpi0), zst & 1u);
         if (lane == 0) bulk_wait_group0();
         __syncwarp();
         if (ok && p.hT) {
@@ -910,7 +929,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
-                       const __grid_constant__ CUtensorMap tm_o, const ClParams p) {
+                       const __grid_constant__ CUtensorMap tm_o,
+                       const __grid_constant__ CUtensorMap tm_z, const ClParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -963,7 +983,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     cluster_sync_all();   // every CTA's barriers are initialised before any remote traffic
 
     if (rank == 0)
-        chain_cta<GT>(&tm_q, &tm_k, &tm_v, &tm_o, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
+        chain_cta<GT>(&tm_q, &tm_k, &tm_v, &tm_o, &tm_z, p, sm, sb, tmem, wt, h, n, bos, eos, nchunks);
     else
         prep_cta<PRO>(&tm_q, &tm_k, &tm_v, p, sm, sb, tmem, wt, h, bos, eos, nchunks, rank);
 
@@ -1008,6 +1028,10 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     uint32_t obox[3] = {32, 1, 16};
     if (!encode_bf16_map(&to, a.o, 3, dv, sv, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
+    // z (gate logits, o's layout): the same 16 x 32 tiles, loaded into the output tiles
+    CUtensorMap tz = to;
+    if (a.z && !encode_bf16_map(&tz, a.z, 3, dv, sv, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
     auto kern = a.z ? (a.prologue ? prefill_cluster_kernel<true, true> : prefill_cluster_kernel<false, true>)
                     : (a.prologue ? prefill_cluster_kernel<true, false> : prefill_cluster_kernel<false, false>);
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1015,7 +1039,6 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     ClParams prm{a.g, a.beta, a.h0, a.cu_seqlens, a.T, a.HK, a.HV, a.scale,
                  static_cast<__nv_bfloat16 *>(a.o), a.hT, status, a.prologue};
-    prm.z = static_cast<const __nv_bfloat16 *>(a.z);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(kClusterSize * a.HV), (unsigned)a.N, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1028,7 +1051,7 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, prm);
+    err = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, tz, prm);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
