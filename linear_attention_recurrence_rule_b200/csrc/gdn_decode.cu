@@ -56,7 +56,7 @@ struct LayerStep {
 // row; LY (implies PRO): the layer steps.  Separate instances, so none of them
 // costs the paths that do not use it.
 template <int DK, typename Tin, bool PRO, bool RD, bool LY>
-__global__ void __launch_bounds__(kDecodeWarps * 32, LY ? 2 : 3)
+__global__ void __launch_bounds__(kDecodeWarps * 32, 3)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ g, const float *__restrict__ beta, float *state,
               Tin *__restrict__ o, int HK, int HV, int dv, float scale, unsigned pro,
@@ -81,7 +81,51 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     constexpr int rows_per_batch = kDecodeWarps * RPI * kDecodeNB;
     {
         const int base = blockIdx.y * rows_per_batch;
-        // the state loads go out first: nothing below them waits on q, k
+        // layer steps of this band's rows (one row per thread of the first
+        // rows_per_batch / 32 warps, before their own state loads; the other warps'
+        // state loads are in flight meanwhile): the convolved value and the output
+        // gate of each row, shared by its lanes
+        __shared__ float lyv[LY ? rows_per_batch : 1], lyg[LY ? rows_per_batch : 1];
+        if (LY && threadIdx.x < rows_per_batch && base + (int)threadIdx.x < dv) {
+            const size_t C = (size_t)HV * dv;
+            const int r = threadIdx.x;
+            const int row = base + r;
+            const size_t ch = (size_t)h * dv + row;
+            const float vin = to_f32(vrow[row]);
+            float vc = vin;
+            if (ly.W > 0) {
+                // every tap's loads go out together (predicated, not a runtime loop)
+                constexpr int MW = kConvMaxWidth;
+                const int W = ly.W;
+                Tin *cs = ly.cs + (size_t)n * (W - 1) * C + ch;
+                const float *wr = ly.cw + ch * W;
+                Tin hist[MW - 1];
+                float wt[MW];
+#pragma unroll
+                for (int m = 0; m < MW - 1; ++m)
+                    if (m < W - 1) hist[m] = cs[m * C];
+#pragma unroll
+                for (int m = 0; m < MW; ++m)
+                    if (m < W) wt[m] = wr[m];
+                float a = ly.cb ? ly.cb[ch] : 0.f;
+#pragma unroll
+                for (int m = 0; m < MW - 1; ++m)
+                    if (m < W - 1) a = fmaf(wt[m], to_f32(hist[m]), a);
+#pragma unroll
+                for (int m = 0; m < MW; ++m)
+                    if (m == W - 1) a = fmaf(wt[m], vin, a);
+                vc = ly.silu ? a * gate_sigmoid(a) : a;
+                // the carried inputs move one token on; this token's raw value last
+#pragma unroll
+                for (int m = 0; m < MW - 2; ++m)
+                    if (m < W - 2) cs[m * C] = hist[m + 1];
+                cs[(W - 2) * C] = vrow[row];
+            }
+            lyv[r] = vc;
+            lyg[r] = ly.z ? gate_sigmoid(to_f32(ly.z[(size_t)nh * dv + row])) : 1.f;
+        }
+        // the state loads go out first (after the layer steps in the layer
+        // instance's first warps): nothing below them waits on q, k
         float4 s[kDecodeNB];
         float grow[RD ? kDecodeNB : 1];   // per-row decays (GDN_ROW_DECAY), loaded with the state
 #pragma unroll
@@ -91,33 +135,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
                             : make_float4(0.f, 0.f, 0.f, 0.f);
             if (RD) grow[RD ? j : 0] = row < dv ? g[(size_t)nh * dv + row] : 0.f;
         }
-        // layer steps of this band's rows, while the state loads are in flight: the
-        // convolved value and the output gate of each row, shared by its lanes
-        __shared__ float lyv[LY ? rows_per_batch : 1], lyg[LY ? rows_per_batch : 1];
-        if (LY) {
-            const size_t C = (size_t)HV * dv;
-            for (int r = threadIdx.x; r < rows_per_batch; r += kDecodeWarps * 32) {
-                const int row = base + r;
-                if (row >= dv) continue;
-                const size_t ch = (size_t)h * dv + row;
-                const float vin = to_f32(vrow[row]);
-                float vc = vin;
-                if (ly.W > 0) {
-                    Tin *cs = ly.cs + (size_t)n * (ly.W - 1) * C + ch;
-                    const float *wr = ly.cw + ch * ly.W;
-                    float a = ly.cb ? ly.cb[ch] : 0.f;
-                    for (int m = 0; m < ly.W - 1; ++m) a = fmaf(wr[m], to_f32(cs[m * C]), a);
-                    a = fmaf(wr[ly.W - 1], vin, a);
-                    vc = ly.silu ? a * gate_sigmoid(a) : a;
-                    // the carried inputs move one token on; this token's raw value last
-                    for (int m = 0; m + 1 < ly.W - 1; ++m) cs[m * C] = cs[(m + 1) * C];
-                    cs[(ly.W - 2) * C] = vrow[row];
-                }
-                lyv[r] = vc;
-                lyg[r] = ly.z ? gate_sigmoid(to_f32(ly.z[(size_t)nh * dv + row])) : 1.f;
-            }
-            __syncthreads();
-        }
+        if (LY) __syncthreads();   // the band's convolved values and gates are in place
         if (PRO && (pro & (GDN_PROLOGUE_NORM_Q | GDN_PROLOGUE_NORM_K))) {
             // the lanes of a row hold the whole q and k: reduce the squared norms there
             float ssk = dot4(kk, kk), ssq = dot4(qq, qq);

@@ -12,10 +12,12 @@
 //
 // All three kernels are single streaming passes over HBM:
 //  * conv_kernel: a thread owns 16 bytes of channels (8 bf16 / 4 fp32) for a
-//    run of kConvRun tokens and keeps the previous W-1 inputs of its channels
-//    in registers, so each input is read once plus a halo of W-1 tokens per
-//    run, each output written once; loads go out kConvBatch tokens at a time.
-//    A sequence start inside a run resets the window from the carried state.
+//    run of kConvRun tokens: it issues the loads of the W-1 tokens before the
+//    run and of the whole run at once (one round trip), then slides a window of
+//    the previous W-1 inputs in registers.  Each input is read from DRAM once;
+//    the halo rows are re-read from L2, where the neighbouring run's thread has
+//    just brought them.  A sequence start inside a run resets the window from
+//    the carried state.
 //  * conv_state_kernel (launched after it on the same stream): each
 //    sequence's new carried state, its last W-1 inputs (from the old state
 //    where the sequence is shorter than W-1).  A launch of its own, so that
@@ -28,8 +30,8 @@ namespace gdn {
 namespace {
 
 constexpr int kConvThreads = 128;
-constexpr int kConvRun = 32;     // tokens per thread
-constexpr int kConvBatch = 8;    // loads in flight per thread
+constexpr int kConvRun = 8;      // tokens per thread, all loaded at once with the window
+constexpr int kConvBatch = 8;
 constexpr int kGateThreads = 256;
 
 // 16 bytes of one dtype as raw words and as floats
@@ -133,7 +135,7 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
         else
             win[m] = make_uint4(0u, 0u, 0u, 0u);   // +0.0 in both dtypes
     }
-    constexpr int NB = W <= 4 ? kConvBatch : kConvBatch / 2;
+    constexpr int NB = kConvBatch;
     for (int64_t tb = t0; tb < t1; tb += NB) {
         uint4 raw[NB];
 #pragma unroll

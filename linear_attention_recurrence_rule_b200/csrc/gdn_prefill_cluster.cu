@@ -206,9 +206,10 @@ __device__ __forceinline__ void load_qkv_slot(const CUtensorMap *tm_q, const CUt
 }
 
 // GT: the output gate o <- o * sigmoid(z) is applied in the read-out, before the
-// one rounding to bf16.  Each epilogue warp TMA-loads its 16 x 32 tile of gate
-// logits into its output tile while the state is rescaled, and the read-out
-// overwrites it in place with the gated outputs.
+// one rounding to bf16.  Each epilogue warp prefetches its 16 x 32 tile of gate
+// logits into L2 one chunk ahead, TMA-loads it into its output tile while the
+// state is rescaled, and the read-out overwrites it in place with the gated
+// outputs.
 template <bool GT>
 __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                           const CUtensorMap *tm_o, const CUtensorMap *tm_z, const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
@@ -425,7 +426,14 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             const int L = chunk_len(c);
             const uint8_t *slot = sm + C_R + s * SLOT;
             const float *tab = reinterpret_cast<const float *>(slot + SL_TAB);
-            if (GT && c > 0 && ok) load_z(c - 1);   // in flight while the state is rescaled
+            if (GT) {
+                // this chunk's gate logits towards L2 a period ahead of their load, and
+                // the previous chunk's into the output tile (an L2 hit by now), in
+                // flight while the state is rescaled
+                if (lane == 0)
+                    tma_prefetch_l2_3d(tm_z, 32 * (warp & 3), h, (int)(bos + (int64_t)c * C + 16 * part));
+                if (c > 0 && ok) load_z(c - 1);
+            }
             ok = warp_all(ok && wt(CB_R_FULL0 + s, (uint32_t)((c >> 1) & 1)));
             if (ok) {
                 // scale the fp32 state by this chunk's gamma_L before its update
