@@ -337,7 +337,7 @@ def measure_layer(gdn, torch, dev, stream, x, w, o, hT, rank, peaks, peak_src, p
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     tokens = B * T
     ws = torch.empty(gdn.gdn_chunk_prefill_layer_workspace_size(
-        B, T, w.HK, w.HV, w.dk, w.dv, w.chunk, w.dtype, 0, 1), dtype=torch.uint8, device=dev)
+        B, T, w.HK, w.HV, w.dk, w.dv, w.chunk, w.dtype, 0, 1, 1), dtype=torch.uint8, device=dev)
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
 
     def layer_prefill():
@@ -398,8 +398,9 @@ def measure_layer(gdn, torch, dev, stream, x, w, o, hT, rank, peaks, peak_src, p
             "prefill": {"workload": WORKLOAD, "ms_per_step": lp_ms,
                         "value": tokens / (lp_ms / 1e3), "unit": "tokens/s",
                         "plain_ms_per_step": plain_s * 1e3, "overhead": lp_ms / (plain_s * 1e3) - 1.0,
-                        "gpu_launches": 3,
-                        "launches": "convolution + carried state, prefill with the gate in its read-out"},
+                        "gpu_launches": 4,
+                        "launches": "convolution + carried state, gate factors, prefill (gate applied "
+                                    "in its read-out)"},
             "conv_kernel": {"ms": cv_ms, "bytes": cv_bytes, "gpu_launches": 2,
                             "roofline": {"bound": "hbm", "achieved": cv_bytes / (cv_ms / 1e3) / 1e9,
                                          "peak": hbm, "unit": "GB/s",

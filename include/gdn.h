@@ -470,22 +470,26 @@ GDN_API gdn_status gdn_recurrent_step_layer(const void *q, const void *k, const 
                                             gdn_stream_t stream);
 
 /*
- * Bytes of device workspace gdn_chunk_prefill_layer needs: the convolved
- * values (when has_conv) after gdn_chunk_prefill's own workspace.
+ * Bytes of device workspace gdn_chunk_prefill_layer needs: gdn_chunk_prefill's
+ * own workspace, then the convolved values (when has_conv) and the gate factors
+ * sigmoid(z) (when has_gate), each [tokens][HV*dv] of 2 bytes (bf16 calls) or
+ * 4 bytes (fp32 calls).
  */
 GDN_API size_t gdn_chunk_prefill_layer_workspace_size(int N, int64_t T, int HK, int HV, int dk,
                                                       int dv, int chunk, gdn_dtype dtype,
-                                                      int varlen, int has_conv);
+                                                      int varlen, int has_conv, int has_gate);
 
 /*
  * gdn_chunk_prefill_ex with the layer steps: the short convolution of v
  * (gdn_short_conv into the workspace, stored in the call's dtype -- the
  * tensor-core path takes bf16 operands; conv_state [N][conv_width-1][HV*dv]
- * updated as there), then the prefill on the convolved values with the output
- * gate o <- o * sigmoid(z) applied where the prefill writes o (z like v, one
- * rounding of o).  conv_weight NULL: no convolution; z NULL: no gate.  flags:
- * GDN_PROLOGUE_*, GDN_ROW_DECAY and GDN_CONV_SILU.  Launches on `stream`: the
- * convolution's two, then the prefill's one; arguments as in
+ * updated as there), the gate factors sigmoid(z) into the workspace (fp16,
+ * relative error <= 2^-12, for bf16 calls; fp32 for fp32 calls), then the
+ * prefill on the convolved values, which
+ * multiplies o by the factors where it writes o (z like v; o is rounded once).
+ * conv_weight NULL: no convolution; z NULL: no gate.  flags: GDN_PROLOGUE_*,
+ * GDN_ROW_DECAY and GDN_CONV_SILU.  Launches on `stream`: the convolution's
+ * two, the factors' one, the prefill's one; arguments as in
  * gdn_chunk_prefill_ex and gdn_short_conv.  z 16-byte aligned.
  */
 GDN_API gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v,

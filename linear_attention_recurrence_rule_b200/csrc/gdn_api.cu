@@ -479,10 +479,11 @@ gdn_status gdn_recurrent_step_layer(const void *q, const void *k, const void *v,
 
 size_t gdn_chunk_prefill_layer_workspace_size(int N, int64_t T, int HK, int HV, int dk, int dv,
                                               int chunk, gdn_dtype dtype, int varlen,
-                                              int has_conv) {
+                                              int has_conv, int has_gate) {
     if (N < 0 || T < 0 || HK <= 0 || HV <= 0 || HV % HK || dv <= 0 || chunk <= 0) return 0;
     const size_t pre = up256(gdn_chunk_prefill_workspace_size(N, T, HK, HV, dk, dv, chunk, dtype, varlen));
-    return has_conv ? pre + layer_vconv_bytes(N, T, HV, dv, dtype, varlen != 0) : pre;
+    return pre + (has_conv ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen != 0) : 0) +
+           (has_gate ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen != 0) : 0);
 }
 
 gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, const float *g,
@@ -513,11 +514,12 @@ gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, 
     }
     if (z && !aligned16(z)) return GDN_ERR_ALIGNMENT;
     if (N == 0) return GDN_OK;
-    // workspace: [prefill's own | convolved values]
+    // workspace: [prefill's own | convolved values | gate factors (fp16)]
     const size_t pre = up256(gdn::prefill_cluster_supported(dk, dv, chunk, dtype) && !(prologue & GDN_ROW_DECAY)
                                  ? gdn::prefill_cluster_workspace(N, T, HV, chunk, varlen)
                                  : 0);
-    const size_t need = conv_weight ? pre + layer_vconv_bytes(N, T, HV, dv, dtype, varlen) : pre;
+    const size_t vbytes = conv_weight ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen) : 0;
+    const size_t need = pre + vbytes + (z ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen) : 0);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -526,9 +528,17 @@ gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, 
         if (gdn::launch_short_conv(ca, s) != cudaSuccess) return GDN_ERR_CUDA;
         a.v = ca.y;
     }
+    if (z) {
+        // sigmoid(z) factors (fp16 for bf16, fp32 for fp32), applied in the prefill's
+        // read-out before o is rounded
+        void *f = static_cast<char *>(workspace) + pre + vbytes;
+        const int64_t tokens = varlen ? T : (int64_t)N * T;
+        if (gdn::launch_gate_factor(z, f, tokens * (int64_t)C, dtype, s) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        a.gate = f;
+    }
     a.workspace_bytes = pre;
     if (pre == 0) a.workspace = nullptr;
-    a.z = z;   // the gate is applied in the prefill's read-out, before o is rounded
     return enqueue_prefill(a, s);
 }
 

@@ -53,6 +53,13 @@ __device__ __forceinline__ float4 scale4(float4 a, float s) {
 // for an L2-normalised row with squared norm ss, and the sigmoid gates.
 __device__ __forceinline__ float inv_l2norm(float ss) { return 1.f / fmaxf(sqrtf(ss), 1e-12f); }
 __device__ __forceinline__ float gate_sigmoid(float x) { return 1.f / (1.f + expf(-x)); }
+// Sigmoid of the layer steps (output gate, SiLU after the short convolution):
+// hardware exponential and reciprocal, relative error ~1e-6 -- far inside the
+// bf16 and fp32 output tolerances -- at a few instructions, so these steps stay
+// memory-bound.  x is clamped at -80 so the reciprocal never sees an infinity.
+__device__ __forceinline__ float layer_sigmoid(float x) {
+    return __fdividef(1.f, 1.f + __expf(-fmaxf(x, -80.f)));
+}
 // log sigmoid(x) = min(x, 0) - log(1 + e^-|x|): finite at both ends
 __device__ __forceinline__ float gate_log_sigmoid(float x) {
     return fminf(x, 0.f) - log1pf(expf(-fabsf(x)));

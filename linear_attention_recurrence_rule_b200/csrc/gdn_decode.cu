@@ -114,7 +114,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 #pragma unroll
                 for (int m = 0; m < MW; ++m)
                     if (m == W - 1) a = fmaf(wt[m], vin, a);
-                vc = ly.silu ? a * gate_sigmoid(a) : a;
+                vc = ly.silu ? a * layer_sigmoid(a) : a;
                 // the carried inputs move one token on; this token's raw value last
 #pragma unroll
                 for (int m = 0; m < MW - 2; ++m)
@@ -122,7 +122,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
                 cs[(W - 2) * C] = vrow[row];
             }
             lyv[r] = vc;
-            lyg[r] = ly.z ? gate_sigmoid(to_f32(ly.z[(size_t)nh * dv + row])) : 1.f;
+            lyg[r] = ly.z ? layer_sigmoid(to_f32(ly.z[(size_t)nh * dv + row])) : 1.f;
         }
         // the state loads go out first (after the layer steps in the layer
         // instance's first warps): nothing below them waits on q, k

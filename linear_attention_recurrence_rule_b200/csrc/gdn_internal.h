@@ -24,7 +24,8 @@ struct PrefillArgs {
     size_t workspace_bytes;
     bool keep_status = false;   // leave the workspace status word as earlier calls left it
     unsigned prologue = 0;      // GDN_PROLOGUE_* flags
-    const void *z = nullptr;    // output gate logits, like o (gdn_chunk_prefill_layer)
+    const void *gate = nullptr; // output gate factors sigmoid(z), o's layout: fp16 for
+                                // bf16 calls, fp32 for fp32 calls
 };
 
 struct StepArgs {
@@ -105,6 +106,9 @@ constexpr int kConvMaxWidth = 8;
 int conv_vector_channels(gdn_dtype dtype);   // channels per 16-byte vector
 cudaError_t launch_short_conv(const ConvArgs &a, cudaStream_t stream);
 cudaError_t launch_output_gate(void *o, const void *z, int64_t elems, gdn_dtype dtype,
+                               cudaStream_t stream);
+// sigmoid(z) -> fp16 factors (the layer prefill's gate)
+cudaError_t launch_gate_factor(const void *z, void *factors, int64_t elems, gdn_dtype dtype,
                                cudaStream_t stream);
 
 // CUDA-core chunked prefill (gdn_prefill_simt.cu)

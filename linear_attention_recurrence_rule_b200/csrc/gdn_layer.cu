@@ -23,6 +23,13 @@
 //    where the sequence is shorter than W-1).  A launch of its own, so that
 //    every read of the old state is over before it is overwritten in place.
 //  * gate_kernel: o <- o * sigmoid(z), 16-byte vectors, grid-stride.
+//  * gate_factor_kernel: sigmoid(z) -- fp16 (relative error <= 2^-12) for bf16
+//    calls, fp32 for fp32 calls -- the factors the layer prefill's read-out
+//    multiplies by, computed here on every SM at streaming speed rather than on
+//    the prefill's chain SMs, where the special function unit would sit on the
+//    critical path.
+#include <cuda_fp16.h>
+
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -169,7 +176,7 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
 #pragma unroll
             for (int e = 0; e < VN; ++e) {
                 const float a = fmaf(wt[W - 1][e], f[e], acc[e]);
-                acc[e] = silu ? a * gate_sigmoid(a) : a;
+                acc[e] = silu ? a * layer_sigmoid(a) : a;
             }
             st16(y + t * C + c0, Vec16<T>::from_float(acc));
 #pragma unroll
@@ -236,9 +243,30 @@ gate_kernel(T *o, const T *__restrict__ z, int64_t nvec) {
                 Vec16<T>::to_float(ov[u], of);
                 Vec16<T>::to_float(zv[u], zf);
 #pragma unroll
-                for (int e = 0; e < VN; ++e) of[e] *= gate_sigmoid(zf[e]);
+                for (int e = 0; e < VN; ++e) of[e] *= layer_sigmoid(zf[e]);
                 __stcs(reinterpret_cast<uint4 *>(o) + i, Vec16<T>::from_float(of));
             }
+        }
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kGateThreads)
+gate_factor_kernel(const T *__restrict__ z, void *__restrict__ f, int64_t nvec) {
+    constexpr int VN = Vec16<T>::n;
+    const int64_t stride = (int64_t)gridDim.x * kGateThreads;
+    for (int64_t i = (int64_t)blockIdx.x * kGateThreads + threadIdx.x; i < nvec; i += stride) {
+        float zf[VN];
+        Vec16<T>::to_float(__ldcs(reinterpret_cast<const uint4 *>(z) + i), zf);
+        if constexpr (VN == 8) {   // bf16 logits -> fp16 factors
+            __half2 h[VN / 2];
+#pragma unroll
+            for (int e = 0; e < VN / 2; ++e)
+                h[e] = __floats2half2_rn(layer_sigmoid(zf[2 * e]), layer_sigmoid(zf[2 * e + 1]));
+            reinterpret_cast<uint4 *>(f)[i] = *reinterpret_cast<const uint4 *>(h);
+        } else {                   // fp32 logits -> fp32 factors
+            reinterpret_cast<float4 *>(f)[i] = make_float4(layer_sigmoid(zf[0]), layer_sigmoid(zf[1]),
+                                                           layer_sigmoid(zf[2]), layer_sigmoid(zf[3]));
         }
     }
 }
@@ -300,9 +328,28 @@ cudaError_t launch_gate_t(void *o, const void *z, int64_t elems, cudaStream_t st
     return cudaGetLastError();
 }
 
+template <typename T>
+cudaError_t launch_gate_factor_t(const void *z, void *f, int64_t elems, cudaStream_t stream) {
+    const int64_t nvec = elems / Vec16<T>::n;
+    int64_t blocks = (nvec + kGateThreads - 1) / kGateThreads;
+    const int64_t cap = (int64_t)sm_count() * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    gate_factor_kernel<T><<<(unsigned)blocks, kGateThreads, 0, stream>>>(
+        static_cast<const T *>(z), f, nvec);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 int conv_vector_channels(gdn_dtype dtype) { return dtype == GDN_BF16 ? 8 : 4; }
+
+cudaError_t launch_gate_factor(const void *z, void *factors, int64_t elems, gdn_dtype dtype,
+                               cudaStream_t stream) {
+    if (elems == 0) return cudaSuccess;
+    return dtype == GDN_BF16 ? launch_gate_factor_t<__nv_bfloat16>(z, factors, elems, stream)
+                             : launch_gate_factor_t<float>(z, factors, elems, stream);
+}
 
 cudaError_t launch_short_conv(const ConvArgs &a, cudaStream_t stream) {
     if (a.N == 0) return cudaSuccess;

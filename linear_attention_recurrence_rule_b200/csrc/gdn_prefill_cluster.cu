@@ -28,8 +28,8 @@
 //     in-place gamma_L scaling, and the outputs are gamma_t S0 Q^T + U P^T;
 //     sixteen epilogue warps share every epilogue (16 tokens or 32 state columns
 //     each) and write chunk c's outputs while chunk c + 1's first products run
-//     (with the layer's output gate, o * sigmoid(z) before the rounding to bf16;
-//     z loaded while the state is rescaled).
+//     (with the layer's output gate, o * sigmoid(z) before the rounding to bf16,
+//     the fp16 factors loaded while the state is rescaled).
 // The chain's critical loop hands over between its epilogue warps and the
 // MMA-issuing warp through named barriers (no sleeping wake-up on that path);
 // tensor-core completions and cross-CTA hand-overs use mbarriers.
@@ -45,6 +45,7 @@
 // gamma_t of the inter-chunk read-out applied in fp32; only S0 and W are single
 // bf16.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
@@ -206,10 +207,10 @@ __device__ __forceinline__ void load_qkv_slot(const CUtensorMap *tm_q, const CUt
 }
 
 // GT: the output gate o <- o * sigmoid(z) is applied in the read-out, before the
-// one rounding to bf16.  Each epilogue warp prefetches its 16 x 32 tile of gate
-// logits into L2 one chunk ahead, TMA-loads it into its output tile while the
-// state is rescaled, and the read-out overwrites it in place with the gated
-// outputs.
+// one rounding to bf16, from factors sigmoid(z) precomputed in fp16.  Each
+// epilogue warp prefetches its 16 x 32 tile of factors into L2 one chunk ahead,
+// TMA-loads it into its output tile while the state is rescaled, and the
+// read-out overwrites it in place with the gated outputs.
 template <bool GT>
 __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                           const CUtensorMap *tm_o, const CUtensorMap *tm_z, const ClParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
@@ -355,7 +356,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
         if (nchunks > 0) named_sync(NB_S0, kChainSync);
         bool ok = true;
         float dq[16];            // scale * gamma_t * (S0 q_t) of the previous chunk
-        // gate logits of chunk cp for this warp's 16 tokens x 32 value rows, into the
+        // gate factors of chunk cp for this warp's 16 tokens x 32 value rows, into the
         // warp's output tile once its previous store has been read (tokens past the
         // end of the data read as zero; those of a next sequence are never stored)
         uint32_t zst = 0;   // bit 0: phase of the next gate-logit load; bit 1: one in flight
@@ -384,7 +385,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             if (lane == 0) bulk_wait_group_read0();
             __syncwarp();
             if (GT) {
-                // the gate logits are in the tile
+                // the gate factors are in the tile
                 const bool zok = warp_all(wt(CB_Z0 + (warp - kCEpi0), zst & 1u));
                 if (zok) zst = (zst & 1u) ^ 1u;
                 tmem_wait_ld();
@@ -394,8 +395,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 float out = fmaf(p.scale, dout[j], dq[j]);
-                if (GT)
-                    out *= gate_sigmoid(__uint_as_float((uint32_t)ot[j * 32 + lane] << 16));
+                if (GT) out *= __half2float(__ushort_as_half(ot[j * 32 + lane]));
                 const __nv_bfloat16 b = __float2bfloat16_rn(out);
                 ot[j * 32 + lane] = *reinterpret_cast<const unsigned short *>(&b);
             }
@@ -427,7 +427,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             const uint8_t *slot = sm + C_R + s * SLOT;
             const float *tab = reinterpret_cast<const float *>(slot + SL_TAB);
             if (GT) {
-                // this chunk's gate logits towards L2 a period ahead of their load, and
+                // this chunk's gate factors towards L2 a period ahead of their load, and
                 // the previous chunk's into the output tile (an L2 hit by now), in
                 // flight while the state is rescaled
                 if (lane == 0)
@@ -1036,11 +1036,12 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream) {
     uint32_t obox[3] = {32, 1, 16};
     if (!encode_bf16_map(&to, a.o, 3, dv, sv, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    // z (gate logits, o's layout): the same 16 x 32 tiles, loaded into the output tiles
+    // gate factors (fp16, o's layout; copied raw, so the 2-byte map type serves):
+    // the same 16 x 32 tiles, loaded into the output tiles
     CUtensorMap tz = to;
-    if (a.z && !encode_bf16_map(&tz, a.z, 3, dv, sv, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (a.gate && !encode_bf16_map(&tz, a.gate, 3, dv, sv, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    auto kern = a.z ? (a.prologue ? prefill_cluster_kernel<true, true> : prefill_cluster_kernel<false, true>)
+    auto kern = a.gate ? (a.prologue ? prefill_cluster_kernel<true, true> : prefill_cluster_kernel<false, true>)
                     : (a.prologue ? prefill_cluster_kernel<true, false> : prefill_cluster_kernel<false, false>);
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)SMEM_BYTES);

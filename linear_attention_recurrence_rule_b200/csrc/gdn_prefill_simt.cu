@@ -19,6 +19,10 @@
 // State rows are independent, so each CTA carries BV rows of S in shared
 // memory through the sequential loop over chunks; the key-key and query-key
 // products of a chunk are recomputed by each value tile.
+#include <cuda_fp16.h>
+
+#include <type_traits>
+
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
@@ -50,7 +54,7 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const float *__restrict__ beta, const float *__restrict__ h0,
                     const int32_t *__restrict__ cu, int64_t T, int HK, int HV, int dv,
                     float scale, Tin *__restrict__ o, float *__restrict__ hT, unsigned pro,
-                    const Tin *__restrict__ z) {
+                    const void *__restrict__ gate) {
     using L_ = SimtSmem<DK, BV, C, RD>;
     constexpr int KP = L_::KP, CP = L_::CP, NT = kSimtThreads;
     const int tid = threadIdx.x;
@@ -218,7 +222,9 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             }
             const size_t oi = ((size_t)(s0 + i) * HV + h) * dv + e0 + e;
             float out = scale * acc;
-            if (z) out *= gate_sigmoid(to_f32(z[oi]));   // output gate, before the one rounding
+            if (gate)   // output gate, before the one rounding: fp32 factors for fp32, else fp16
+                out *= std::is_same<Tin, float>::value ? static_cast<const float *>(gate)[oi]
+                                                       : __half2float(static_cast<const __half *>(gate)[oi]);
             o[oi] = from_f32<Tin>(out);
         }
         __syncthreads();
@@ -257,7 +263,7 @@ cudaError_t launch_shape_rd(const PrefillArgs &a, cudaStream_t stream) {
     kern<<<grid, block, smem, stream>>>(
         static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
         static_cast<const Tin *>(a.v), a.g, a.beta, a.h0, a.cu_seqlens, a.T, a.HK, a.HV, a.dv,
-        a.scale, static_cast<Tin *>(a.o), a.hT, a.prologue, static_cast<const Tin *>(a.z));
+        a.scale, static_cast<Tin *>(a.o), a.hT, a.prologue, a.gate);
     return cudaGetLastError();
 }
 

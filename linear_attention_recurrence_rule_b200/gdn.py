@@ -112,7 +112,7 @@ def load_library() -> ctypes.CDLL:
                                                      vp, ctypes.c_uint, vp]
             lib.gdn_chunk_prefill_layer_workspace_size.restype = sz
             lib.gdn_chunk_prefill_layer_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32,
-                                                                   i32, i32, i32, i32]
+                                                                   i32, i32, i32, i32, i32]
             lib.gdn_chunk_prefill_layer.restype = i32
             lib.gdn_chunk_prefill_layer.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
                                                     i32, i32, i32, i32, ctypes.c_float, i32, vp,
@@ -660,11 +660,11 @@ def gdn_recurrent_step_layer(q, k, v, g, beta, state, conv_weight=None, conv_bia
 
 
 def gdn_chunk_prefill_layer_workspace_size(N, T, HK, HV, dk, dv, chunk, dtype, varlen,
-                                           has_conv) -> int:
+                                           has_conv, has_gate=False) -> int:
     code = dtype if isinstance(dtype, int) else _dtype_code(torch.empty(0, dtype=dtype))
     return int(load_library().gdn_chunk_prefill_layer_workspace_size(
         int(N), int(T), int(HK), int(HV), int(dk), int(dv), int(chunk), code,
-        int(bool(varlen)), int(bool(has_conv))))
+        int(bool(varlen)), int(bool(has_conv)), int(bool(has_gate))))
 
 
 def gdn_chunk_prefill_layer(q, k, v, g, beta, h0=None, cu_seqlens=None, conv_weight=None,
@@ -716,7 +716,8 @@ def gdn_chunk_prefill_layer(q, k, v, g, beta, h0=None, cu_seqlens=None, conv_wei
     code = _dtype_code(q)
     need = lib.gdn_chunk_prefill_layer_workspace_size(N, T, HK, HV, dk, dv, chunk, code,
                                                       int(cu_seqlens is not None),
-                                                      int(conv_weight is not None))
+                                                      int(conv_weight is not None),
+                                                      int(z is not None))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

@@ -320,9 +320,13 @@ def test_prefill_layer_validation(lib):
     assert prefill_layer_call(lib, z=fake(0x9008)) == gdn.GDN_ERR_ALIGNMENT
     # the convolved values need workspace: none given
     assert prefill_layer_call(lib) == gdn.GDN_ERR_WORKSPACE
-    need = lib.gdn_chunk_prefill_layer_workspace_size(1, 64, 1, 2, 32, 32, 16, gdn.GDN_F32, 0, 1)
+    need = lib.gdn_chunk_prefill_layer_workspace_size(1, 64, 1, 2, 32, 32, 16, gdn.GDN_F32, 0, 1, 0)
     assert need >= 64 * 2 * 32 * 4
     assert prefill_layer_call(lib, ws=fake(0x10000), ws_bytes=need - 1) == gdn.GDN_ERR_WORKSPACE
     assert prefill_layer_call(lib, ws=fake(0x10008), ws_bytes=need) == gdn.GDN_ERR_ALIGNMENT
     assert prefill_layer_call(lib, N=0) == gdn.GDN_OK
-    assert lib.gdn_chunk_prefill_layer_workspace_size(1, 64, 1, 2, 32, 32, 16, gdn.GDN_F32, 0, 0) == 0
+    assert lib.gdn_chunk_prefill_layer_workspace_size(1, 64, 1, 2, 32, 32, 16, gdn.GDN_F32, 0, 0, 0) == 0
+    # the gate factors: fp16, one per output element
+    assert lib.gdn_chunk_prefill_layer_workspace_size(1, 64, 1, 2, 32, 32, 16, gdn.GDN_F32, 0, 0,
+                                                      1) >= 64 * 2 * 32 * 2
+    assert prefill_layer_call(lib, w=None, z=fake(0x9000)) == gdn.GDN_ERR_WORKSPACE
