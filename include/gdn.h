@@ -431,7 +431,8 @@ GDN_API gdn_status gdn_state_commit_deltas(const void *k, const float *g, const 
  * overwritten with its last width-1 inputs (taken from the old state where a
  * sequence is shorter than width-1; an empty sequence keeps its state).
  * flags: 0 or GDN_CONV_SILU.  Supported: 2 <= width <= GDN_CONV_MAX_WIDTH, C a
- * multiple of 8 (bf16) or 4 (fp32).  Alignment: x, y, conv_state 16-byte.
+ * multiple of 8 (bf16) or 4 (fp32).  Alignment: x, y, conv_state, weight
+ * 16-byte; bias 4-byte.
  * y must not overlap x or conv_state.  Two launches (the convolution, then the
  * state update when conv_state is given).  N == 0 or no tokens: GDN_OK, and
  * only the state update runs.

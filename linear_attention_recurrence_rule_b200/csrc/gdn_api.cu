@@ -400,8 +400,11 @@ gdn_status check_conv(const gdn::ConvArgs &a) {
     if (a.C / gdn::conv_vector_channels(a.dtype) > 65535 * 128) return GDN_ERR_UNSUPPORTED;
     const int64_t tokens = a.cu_seqlens ? a.T : (int64_t)a.N * a.T;
     if (a.cu_seqlens == nullptr && a.N > 0 && a.T > 0 && tokens / a.N != a.T) return GDN_ERR_INVALID_ARG;
-    if ((tokens + 7) / 8 > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
-    if (!aligned16(a.x) || !aligned16(a.y) || !aligned16(a.conv_state)) return GDN_ERR_ALIGNMENT;
+    if ((tokens + 7) / 8 * ((a.C / gdn::conv_vector_channels(a.dtype) + 127) / 128) > 0x7fffffffLL)
+        return GDN_ERR_UNSUPPORTED;
+    if (!aligned16(a.x) || !aligned16(a.y) || !aligned16(a.conv_state) || !aligned16(a.weight) ||
+        !aligned4(a.bias))
+        return GDN_ERR_ALIGNMENT;
     return GDN_OK;
 }
 

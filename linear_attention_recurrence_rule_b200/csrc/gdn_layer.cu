@@ -100,11 +100,14 @@ template <typename T, int W>
 __global__ void __launch_bounds__(kConvThreads)
 conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
             const T *__restrict__ cstate, const int32_t *__restrict__ cu, int N, int64_t T_per,
-            int64_t Ttot, int C, bool silu, T *__restrict__ y) {
+            int64_t Ttot, int C, int cblocks, bool silu, T *__restrict__ y) {
     constexpr int VN = Vec16<T>::n;
-    const int c0 = (blockIdx.y * kConvThreads + threadIdx.x) * VN;
+    // the channel blocks of one run are neighbours in the grid, so the blocks
+    // resident at a time read whole token rows
+    const int64_t run = (int64_t)blockIdx.x / cblocks;
+    const int c0 = ((int)(blockIdx.x - run * cblocks) * kConvThreads + threadIdx.x) * VN;
     if (c0 >= C) return;
-    const int64_t t0 = (int64_t)blockIdx.x * kConvRun;
+    const int64_t t0 = run * kConvRun;
     const int64_t t1 = t0 + kConvRun < Ttot ? t0 + kConvRun : Ttot;
     // the sequence holding token t0: the last n with start <= t0 (empty sequences skipped)
     int n;
@@ -122,12 +125,25 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
     int64_t bos, eos;
     seq_bounds(cu, T_per, n, bos, eos);
 
+    // this thread's VN x W weights are contiguous (16-byte aligned: c0 is a multiple of 4)
     float wt[W][VN], b[VN];
+    {
+        float flat[VN * W];
+        const float4 *w4 = reinterpret_cast<const float4 *>(w + (size_t)c0 * W);
 #pragma unroll
-    for (int e = 0; e < VN; ++e) {
+        for (int i = 0; i < VN * W / 4; ++i) {
+            const float4 f = __ldg(w4 + i);
+            flat[4 * i] = f.x;
+            flat[4 * i + 1] = f.y;
+            flat[4 * i + 2] = f.z;
+            flat[4 * i + 3] = f.w;
+        }
 #pragma unroll
-        for (int j = 0; j < W; ++j) wt[j][e] = w[(size_t)(c0 + e) * W + j];
-        b[e] = bias ? bias[c0 + e] : 0.f;
+        for (int e = 0; e < VN; ++e)
+#pragma unroll
+            for (int j = 0; j < W; ++j) wt[j][e] = flat[e * W + j];
+#pragma unroll
+        for (int e = 0; e < VN; ++e) b[e] = bias ? __ldg(bias + c0 + e) : 0.f;
     }
     // window: win[m] = the raw input at token t - (W-1) + m, m < W-1 (raw words,
     // converted where used: half the registers for bf16)
@@ -280,9 +296,10 @@ cudaError_t launch_conv_w(const ConvArgs &a, cudaStream_t stream) {
     const T *x = static_cast<const T *>(a.x);
     T *cs = static_cast<T *>(a.conv_state);
     if (Ttot > 0) {
-        const dim3 grid((unsigned)((Ttot + kConvRun - 1) / kConvRun), cblocks);
+        const unsigned grid = (unsigned)((Ttot + kConvRun - 1) / kConvRun * cblocks);
         conv_kernel<T, W><<<grid, kConvThreads, 0, stream>>>(
-            x, a.weight, a.bias, cs, a.cu_seqlens, a.N, a.T, Ttot, a.C, a.silu, static_cast<T *>(a.y));
+            x, a.weight, a.bias, cs, a.cu_seqlens, a.N, a.T, Ttot, a.C, (int)cblocks, a.silu,
+            static_cast<T *>(a.y));
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -258,6 +258,7 @@ def test_short_conv_validation(lib):
     assert conv_call(lib, C=12) == gdn.GDN_ERR_UNSUPPORTED                 # bf16: 8 per vector
     assert conv_call(lib, C=12, dtype=gdn.GDN_F32, x=fake(0x1008)) == gdn.GDN_ERR_ALIGNMENT
     assert conv_call(lib, cs=fake(0x4004)) == gdn.GDN_ERR_ALIGNMENT
+    assert conv_call(lib, w=fake(0x2004)) == gdn.GDN_ERR_ALIGNMENT
     assert conv_call(lib, N=0) == gdn.GDN_OK                                # empty batch
 
 
