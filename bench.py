@@ -456,12 +456,23 @@ def load_peaks():
 # Each entry carries the sha256 of the kernel source it was taken on; a changed
 # source reports null.
 NCU_TRAFFIC = {
-    # full decode_256x64 step: 541,153,280 read + 476,171,776 written
-    "decode": {"bytes": 1017325056, "source": "gdn_decode.cu",
-               "sha256": "dbfc71d8d19d220e31d8f0247d1d42e64f4c5c310b09be07c69e4f71ee4d6aa7"},
-    # full long_prefill_64k launch: 1,090,822,656 read + 511,207,936 written
-    "prefill_cluster": {"bytes": 1602030592, "source": "gdn_prefill_cluster.cu",
-                        "sha256": "881a325e6d56777fe19db569636ec05bdd86d18a1d8dea300fed5c5991d89ae0"},
+    # full decode_256x64 step: 541,171,712 read + 476,291,072 written
+    "decode": {"bytes": 1017462784, "source": "gdn_decode.cu",
+               "sha256": "342c1ce55a1419f66a4d3b79e1f521987b47cfa44938be1fd8bc6c150858c6b6"},
+    # the same step with the short convolution and the output gate fused (layer
+    # instance): 549,628,160 read + 482,972,928 written
+    "decode_layer": {"bytes": 1032601088, "source": "gdn_decode.cu",
+                     "sha256": "342c1ce55a1419f66a4d3b79e1f521987b47cfa44938be1fd8bc6c150858c6b6"},
+    # full long_prefill_64k launch: 1,090,636,800 read + 510,305,280 written
+    "prefill_cluster": {"bytes": 1600942080, "source": "gdn_prefill_cluster.cu",
+                        "sha256": "4ef0fef23fee2a3208626b5a458640654ce023f7ea5ab71922fbe7ecd21b2990"},
+    # short convolution of the 64K bench values (width 4): 537,046,272 read + 491,637,504
+    # written (its carried-state launch adds 55,552)
+    "short_conv": {"bytes": 1028683776, "source": "gdn_layer.cu",
+                   "sha256": "c640fdfe2850641a190133aa14232aab76e40677826a489bfa756149e4befc5b"},
+    # standalone output gate over the 64K bench outputs: 1,073,752,064 read + 491,309,056 written
+    "output_gate": {"bytes": 1565061120, "source": "gdn_layer.cu",
+                    "sha256": "c640fdfe2850641a190133aa14232aab76e40677826a489bfa756149e4befc5b"},
     # verify_256x4, update-vector form, the streaming kernel: 580,045,056 read + 20,497,408
     # written (its setup kernel adds 8,682,752)
     "verify_deltas": {"bytes": 600542464, "source": "gdn_verify.cu",
