@@ -125,10 +125,8 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
     int64_t bos, eos;
     seq_bounds(cu, T_per, n, bos, eos);
 
-    // this thread's VN x W weights are contiguous (16-byte aligned: c0 is a multiple of 4);
-    // weights, bias, window and sums are kept as channel pairs for packed fp32 FMAs
-    constexpr int VP = VN / 2;
-    float2 wt[W][VP], b[VP];
+    // this thread's VN x W weights are contiguous (16-byte aligned: c0 is a multiple of 4)
+    float wt[W][VN], b[VN];
     {
         float flat[VN * W];
         const float4 *w4 = reinterpret_cast<const float4 *>(w + (size_t)c0 * W);
@@ -141,31 +139,24 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
             flat[4 * i + 3] = f.w;
         }
 #pragma unroll
-        for (int e = 0; e < VP; ++e) {
+        for (int e = 0; e < VN; ++e)
 #pragma unroll
-            for (int j = 0; j < W; ++j) wt[j][e] = make_float2(flat[2 * e * W + j], flat[(2 * e + 1) * W + j]);
-            b[e] = bias ? make_float2(__ldg(bias + c0 + 2 * e), __ldg(bias + c0 + 2 * e + 1))
-                        : make_float2(0.f, 0.f);
-        }
+            for (int j = 0; j < W; ++j) wt[j][e] = flat[e * W + j];
+#pragma unroll
+        for (int e = 0; e < VN; ++e) b[e] = bias ? __ldg(bias + c0 + e) : 0.f;
     }
-    // window: win[m] = the input at token t - (W-1) + m, m < W-1, as floats
-    // (each input converted once)
-    float2 win[W - 1][VP];
-    auto set_win = [&](int m, uint4 raw) {
-        float f[VN];
-        Vec16<T>::to_float(raw, f);
-#pragma unroll
-        for (int e = 0; e < VP; ++e) win[m][e] = make_float2(f[2 * e], f[2 * e + 1]);
-    };
+    // window: win[m] = the raw input at token t - (W-1) + m, m < W-1 (raw words,
+    // converted where used: half the registers for bf16)
+    uint4 win[W - 1];
 #pragma unroll
     for (int m = 0; m < W - 1; ++m) {
         const int64_t s = t0 - (W - 1) + m;
         if (s >= bos)
-            set_win(m, ld16(x + s * C + c0));
+            win[m] = ld16(x + s * C + c0);
         else if (cstate)
-            set_win(m, ld16(cstate + ((size_t)n * (W - 1) + (size_t)(s - bos + W - 1)) * C + c0));
+            win[m] = ld16(cstate + ((size_t)n * (W - 1) + (size_t)(s - bos + W - 1)) * C + c0);
         else
-            set_win(m, make_uint4(0u, 0u, 0u, 0u));   // +0.0 in both dtypes
+            win[m] = make_uint4(0u, 0u, 0u, 0u);   // +0.0 in both dtypes
     }
     constexpr int NB = kConvBatch;
     for (int64_t tb = t0; tb < t1; tb += NB) {
@@ -185,35 +176,28 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
                 } while (eos <= t);
 #pragma unroll
                 for (int m = 0; m < W - 1; ++m)
-                    set_win(m, cstate ? ld16(cstate + ((size_t)n * (W - 1) + m) * C + c0)
-                                      : make_uint4(0u, 0u, 0u, 0u));
+                    win[m] = cstate ? ld16(cstate + ((size_t)n * (W - 1) + m) * C + c0)
+                                    : make_uint4(0u, 0u, 0u, 0u);
             }
-            float xf[VN];
-            Vec16<T>::to_float(raw[u], xf);
-            float2 xv[VP], acc[VP];
+            float acc[VN], f[VN];
 #pragma unroll
-            for (int e = 0; e < VP; ++e) {
-                xv[e] = make_float2(xf[2 * e], xf[2 * e + 1]);
-                acc[e] = b[e];
+            for (int e = 0; e < VN; ++e) acc[e] = b[e];
+#pragma unroll
+            for (int m = 0; m < W - 1; ++m) {
+                Vec16<T>::to_float(win[m], f);
+#pragma unroll
+                for (int e = 0; e < VN; ++e) acc[e] = fmaf(wt[m][e], f[e], acc[e]);
             }
+            Vec16<T>::to_float(raw[u], f);
 #pragma unroll
-            for (int m = 0; m < W - 1; ++m)
-#pragma unroll
-                for (int e = 0; e < VP; ++e) acc[e] = fma2(wt[m][e], win[m][e], acc[e]);
-            float out[VN];
-#pragma unroll
-            for (int e = 0; e < VP; ++e) {
-                const float2 a = fma2(wt[W - 1][e], xv[e], acc[e]);
-                out[2 * e] = silu ? a.x * layer_sigmoid(a.x) : a.x;
-                out[2 * e + 1] = silu ? a.y * layer_sigmoid(a.y) : a.y;
+            for (int e = 0; e < VN; ++e) {
+                const float a = fmaf(wt[W - 1][e], f[e], acc[e]);
+                acc[e] = silu ? a * layer_sigmoid(a) : a;
             }
-            st16(y + t * C + c0, Vec16<T>::from_float(out));
+            st16(y + t * C + c0, Vec16<T>::from_float(acc));
 #pragma unroll
-            for (int m = 0; m + 1 < W - 1; ++m)
-#pragma unroll
-                for (int e = 0; e < VP; ++e) win[m][e] = win[m + 1][e];
-#pragma unroll
-            for (int e = 0; e < VP; ++e) win[W - 2][e] = xv[e];
+            for (int m = 0; m + 1 < W - 1; ++m) win[m] = win[m + 1];
+            win[W - 2] = raw[u];
         }
     }
 }
