@@ -94,12 +94,7 @@ constexpr uint32_t ST_T2 = 32768;   // T'' hi, T'' lo -> SL_T2H
 constexpr uint32_t ST_TAB = 49152;  // decay table -> SL_TAB
 constexpr uint32_t ST_BYTES = 50176;
 constexpr uint32_t QKV_BYTES = 6 * 8192;            // Q, K and V tiles loaded by the chain CTA
-// A receive slot completes in two parts: P (16 KB, read last, by chunk c's U P^T)
-// on its own mbarrier, everything else (Q, K, V, -W, T'', table) on the other, so
-// that part can be re-armed for chunk c + 2 as soon as chunk c's state update is
-// done, ~a read-out earlier than P.
-constexpr uint32_t P_BYTES = 16384;
-constexpr uint32_t SLOT_TX = ST_BYTES - P_BYTES + QKV_BYTES;   // the part without P
+constexpr uint32_t SLOT_TX = ST_BYTES + QKV_BYTES;  // bytes that complete one receive slot
 
 // ---- chain CTA shared memory ----
 constexpr uint32_t C_R = 0;                                 // 2 receive slots
@@ -119,20 +114,18 @@ constexpr uint32_t P_ST = 106496;   // two staging blocks (ST_BYTES each, 1024-a
 constexpr uint32_t P_BAR = P_ST + 2 * ST_BYTES;
 
 // CB_Z0 + w: epilogue warp w's gate-logit tile has landed in its output tile (GT)
-// CB_R_FULLs: a slot's part without P; CB_P_FULLs: its P tiles
-enum ChainBar { CB_R_FULL0, CB_R_FULL1, CB_U_MMA, CB_DS_FULL, CB_O_FULL, CB_DRAIN, CB_P_FULL0,
-                CB_P_FULL1, CB_Z0, CB_COUNT = CB_Z0 + 16 };
-// PB_GO: the slot's part without P may be filled; PB_GOP: its P tiles may be
+enum ChainBar { CB_R_FULL0, CB_R_FULL1, CB_U_MMA, CB_DS_FULL, CB_O_FULL, CB_DRAIN, CB_Z0,
+                CB_COUNT = CB_Z0 + 16 };
 enum PrepBar { PB_LD_FULL0, PB_LD_FULL1, PB_X_DONE, PB_T_READY, PB_W_DONE, PB_EPI_DONE, PB_GO,
-               PB_GOP, PB_STAGE_FREE0, PB_STAGE_FREE1, PB_DRAIN, PB_COUNT };
+               PB_STAGE_FREE0, PB_STAGE_FREE1, PB_DRAIN, PB_COUNT };
 
 // words at the same offset in every CTA: TMEM base, abort flag, slot bookkeeping
 constexpr uint32_t AUX_RAW = (C_BAR + CB_COUNT * 8 > P_BAR + PB_COUNT * 8) ? C_BAR + CB_COUNT * 8
                                                                           : P_BAR + PB_COUNT * 8;
 constexpr uint32_t AUX = (AUX_RAW + 15) & ~15u;
 constexpr uint32_t AUX_TSLOT = AUX, AUX_ABORT = AUX + 4, AUX_ARMED = AUX + 8,
-                   AUX_CONSUMED = AUX + 12, AUX_ARMED_P = AUX + 16, AUX_CONSUMED_P = AUX + 20;
-constexpr uint32_t SMEM_BYTES = AUX + 32 + 1024;
+                   AUX_CONSUMED = AUX + 12;
+constexpr uint32_t SMEM_BYTES = AUX + 16 + 1024;
 static_assert(P_PB + 5 * 64 * 4 <= P_ST, "prep layout");
 static_assert(64 * A_LD * 4 >= 16384, "T' tiles fit where A was");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -228,8 +221,6 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
     const size_t sbase = ((size_t)n * HV + h) * (size_t)DH * DH;
     volatile int *armed = reinterpret_cast<volatile int *>(sm + AUX_ARMED);
     volatile int *consumed = reinterpret_cast<volatile int *>(sm + AUX_CONSUMED);
-    volatile int *armed_p = reinterpret_cast<volatile int *>(sm + AUX_ARMED_P);
-    volatile int *consumed_p = reinterpret_cast<volatile int *>(sm + AUX_CONSUMED_P);
     auto chunk_len = [&](int c) {
         const int64_t r = eos - (bos + (int64_t)c * C);
         return (int)(r < C ? r : C);
@@ -252,6 +243,10 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             if (!ok) return false;
             const uint32_t slot = sb + C_R + (c & 1) * SLOT;
             if (lane == 0) *consumed = c + 1;
+            // the bulk copies out of that staging block have completed
+            if (elect_one())
+                mbar_arrive_remote_relaxed(mapa_shared(
+                    sb + P_BAR + (PB_STAGE_FREE0 + ((c / kNumPrep) & 1)) * 8, 1 + c % kNumPrep));
             __syncwarp();
             tc_fence_after();
             const uint64_t va0 = sdesc_sw128(slot + SL_V, 8192, 1024);
@@ -304,17 +299,6 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             }
             named_sync(NB_U2, kChainSync);    // U (hi, lo) is in TMEM
             tc_fence_after();
-            // the slot's P tiles have landed: every bulk copy out of the producing prep
-            // CTA's staging block has completed, so release it
-            ok = warp_all(ok && wt(CB_P_FULL0 + (c & 1), (uint32_t)((c >> 1) & 1)));
-            if (ok) {
-                if (lane == 0) *consumed_p = c + 1;
-                if (elect_one())
-                    mbar_arrive_remote_relaxed(mapa_shared(
-                        sb + P_BAR + (PB_STAGE_FREE0 + ((c / kNumPrep) & 1)) * 8, 1 + c % kNumPrep));
-                __syncwarp();
-                tc_fence_after();
-            }
             if (ok) {
                 // U P^T (hi/lo cross terms)
                 const uint64_t p0 = sdesc_sw128(slot + SL_PH, 16, 1024);
@@ -442,19 +426,6 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
             const int L = chunk_len(c);
             const uint8_t *slot = sm + C_R + s * SLOT;
             const float *tab = reinterpret_cast<const float *>(slot + SL_TAB);
-            if (c > 0 && c + 1 < nchunks && warp == kCEpi0 && ok) {
-                // chunk c - 1's products that read its slot's Q, K, V, -W and T'' have
-                // completed and every epilogue warp has read its table (the barrier
-                // that started chunk c): re-arm that part of the slot for chunk c + 1
-                // and let the prep CTA producing it fill it
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&bars[CB_R_FULL0 + ((c + 1) & 1)], SLOT_TX);
-                    *armed = c + 2;
-                    load_qkv_slot(tm_q, tm_k, tm_v, sm, bars, c + 1, cqk, h, bos);
-                    mbar_arrive_remote_relaxed(mapa_shared(sb + P_BAR + PB_GO * 8, 1 + (c + 1) % kNumPrep));
-                }
-                __syncwarp();
-            }
             if (GT) {
                 // this chunk's gate factors towards L2 a period ahead of their load, and
                 // the previous chunk's into the output tile (an L2 hit by now), in
@@ -474,19 +445,20 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                 tmem_st32f(tmem_addr(tmem, warp, TM_S + 32 * part), v);
             }
             if (c > 0) {
-                // the previous chunk's U P^T is done: its slot's P tiles are read, so
-                // re-arm them for chunk c + 1 and let the prep CTA send them; then
-                // write the previous chunk's outputs (its accumulator is overwritten
-                // only after this chunk's second barrier)
+                // the previous chunk's U P^T is done: every read of its receive slot is
+                // over, so re-arm that slot and release the prep CTA that produces chunk
+                // c + 1 into it; then write the previous chunk's outputs (its
+                // accumulator is overwritten only after this chunk's second barrier)
                 ok = warp_all(ok && wt(CB_O_FULL, (uint32_t)((c - 1) & 1)));
                 if (ok) {
                     tc_fence_after();
                     if (warp == kCEpi0 && c + 1 < nchunks) {
                         if (lane == 0) {
-                            mbar_arrive_expect_tx(&bars[CB_P_FULL0 + ((c + 1) & 1)], P_BYTES);
-                            *armed_p = c + 2;
+                            mbar_arrive_expect_tx(&bars[CB_R_FULL0 + ((c + 1) & 1)], SLOT_TX);
+                            *armed = c + 2;
+                            load_qkv_slot(tm_q, tm_k, tm_v, sm, bars, c + 1, cqk, h, bos);
                             mbar_arrive_remote_relaxed(
-                                mapa_shared(sb + P_BAR + PB_GOP * 8, 1 + (c + 1) % kNumPrep));
+                                mapa_shared(sb + P_BAR + PB_GO * 8, 1 + (c + 1) % kNumPrep));
                         }
                         __syncwarp();
                     }
@@ -684,23 +656,20 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             commit(PB_W_DONE);
             if (!warp_all(wt(PB_W_DONE, ph))) break;   // this buffer's q/k tiles are free again
             if (!warp_all(wt(PB_EPI_DONE, ph))) break;
-            const int j = first >= 2 ? k : k - 1;   // go arrivals before this chunk
-            if (c >= 2 && !warp_all(wt(PB_GO, (uint32_t)(j & 1)))) break;
-            const int s = c & 1;
-            const uint32_t dst = mapa_shared(sb + C_R + s * SLOT, 0);
-            const uint32_t st = sb + P_ST + (k & 1) * ST_BYTES;
+            if (c >= 2) {
+                const int j = first >= 2 ? k : k - 1;   // go arrivals before this chunk
+                if (!warp_all(wt(PB_GO, (uint32_t)(j & 1)))) break;
+            }
             if (elect_one()) {
+                const int s = c & 1;
                 const uint32_t mbar = mapa_shared(sb + C_BAR + (CB_R_FULL0 + s) * 8, 0);
+                const uint32_t dst = mapa_shared(sb + C_R + s * SLOT, 0);
+                const uint32_t st = sb + P_ST + (k & 1) * ST_BYTES;
                 bulk_copy_to_cluster(dst + SL_WQ, st + ST_W, 8192, mbar);
                 bulk_copy_to_cluster(dst + SL_WQ + 16384, st + ST_W + 8192, 8192, mbar);
+                bulk_copy_to_cluster(dst + SL_PH, st + ST_P, 16384, mbar);
                 bulk_copy_to_cluster(dst + SL_T2H, st + ST_T2, 16384, mbar);
                 bulk_copy_to_cluster(dst + SL_TAB, st + ST_TAB, ST_BYTES - ST_TAB, mbar);
-            }
-            __syncwarp();
-            if (c >= 2 && !warp_all(wt(PB_GOP, (uint32_t)(j & 1)))) break;
-            if (elect_one()) {
-                const uint32_t mbar = mapa_shared(sb + C_BAR + (CB_P_FULL0 + s) * 8, 0);
-                bulk_copy_to_cluster(dst + SL_PH, st + ST_P, P_BYTES, mbar);
             }
             __syncwarp();
         }
@@ -1008,13 +977,10 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             tma_prefetch_desc(&tm_v);
             for (int c = 0; c < pre; ++c) {
                 mbar_arrive_expect_tx(&bars[CB_R_FULL0 + c], SLOT_TX);
-                mbar_arrive_expect_tx(&bars[CB_P_FULL0 + c], P_BYTES);
                 load_qkv_slot(&tm_q, &tm_k, &tm_v, sm, bars, c, h / (p.HV / p.HK), h, bos);
             }
             *reinterpret_cast<volatile int *>(sm + AUX_ARMED) = pre;
             *reinterpret_cast<volatile int *>(sm + AUX_CONSUMED) = 0;
-            *reinterpret_cast<volatile int *>(sm + AUX_ARMED_P) = pre;
-            *reinterpret_cast<volatile int *>(sm + AUX_CONSUMED_P) = 0;
         }
         fence_barrier_init();
     }
@@ -1037,9 +1003,6 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int armed = *reinterpret_cast<volatile int *>(sm + AUX_ARMED);
         for (int d = *reinterpret_cast<volatile int *>(sm + AUX_CONSUMED); d < armed; ++d)
             wt.drain(CB_R_FULL0 + (d & 1), (uint32_t)((d >> 1) & 1));
-        const int armed_p = *reinterpret_cast<volatile int *>(sm + AUX_ARMED_P);
-        for (int d = *reinterpret_cast<volatile int *>(sm + AUX_CONSUMED_P); d < armed_p; ++d)
-            wt.drain(CB_P_FULL0 + (d & 1), (uint32_t)((d >> 1) & 1));
     }
     if (warp == 0) tmem_dealloc(tmem, ncols);
     cluster_sync_all();   // no CTA leaves while another may still address its shared memory
