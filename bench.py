@@ -469,10 +469,10 @@ NCU_TRAFFIC = {
     # short convolution of the 64K bench values (width 4): 537,046,272 read + 491,637,504
     # written (its carried-state launch adds 55,552)
     "short_conv": {"bytes": 1028683776, "source": "gdn_layer.cu",
-                   "sha256": "c640fdfe2850641a190133aa14232aab76e40677826a489bfa756149e4befc5b"},
+                   "sha256": "911934bd0e7a294c493cab767e7a41f34e1b110e7d47ba97e739ee1fe4b5009a"},
     # standalone output gate over the 64K bench outputs: 1,073,752,064 read + 491,309,056 written
     "output_gate": {"bytes": 1565061120, "source": "gdn_layer.cu",
-                    "sha256": "c640fdfe2850641a190133aa14232aab76e40677826a489bfa756149e4befc5b"},
+                    "sha256": "911934bd0e7a294c493cab767e7a41f34e1b110e7d47ba97e739ee1fe4b5009a"},
     # verify_256x4, update-vector form, the streaming kernel: 580,045,056 read + 20,497,408
     # written (its setup kernel adds 8,682,752)
     "verify_deltas": {"bytes": 600542464, "source": "gdn_verify.cu",

@@ -405,9 +405,9 @@ GDN_API gdn_status gdn_state_commit_deltas(const void *k, const float *g, const 
 /*
  * ---- The layer steps around the rule -------------------------------------
  * "Qwen3-Next" (sghael.github.io), section "Linear attention with gated delta
- * rule": the values pass through a 1-D convolution that adds local context,
- * and a gate sets how much of the recurrent read-out reaches the output.  The
- * page gives neither the width nor the gate's form.  Reading used here:
+ * rule", names two further layer steps: the values are mixed with their
+ * recent predecessors by a short convolution before the rule, and its read-out
+ * is scaled by a gate.  The page gives neither the width nor the gate's form.  Reading used here:
  *   - a causal depthwise convolution along time, one kernel of `width` taps
  *     (2..8) per value channel c = h * dv + i (C = HV * dv channels):
  *       y_t[c] = act(bias[c] + sum_{j<width} weight[c][j] * x_{t-(width-1)+j}[c])

@@ -1,9 +1,9 @@
 // The layer steps around the rule: a short causal convolution on the values
 // before it and a sigmoid gate on its read-out after it ("Qwen3-Next",
-// sghael.github.io, section "Linear attention with gated delta rule": a 1-D
-// convolution over the values adds local context, and a gate sets how much of
-// the recurrent read-out reaches the layer's output).  The page gives neither
-// the width nor the gate's form; the library reads them as
+// sghael.github.io, section "Linear attention with gated delta rule", names
+// both: the values are mixed with their recent predecessors, and the rule's
+// read-out is scaled by a gate).  The page gives neither the width nor the
+// gate's form; the library reads them as
 //   y_t[c] = act(bias[c] + sum_{j<W} w[c][j] x_{t-(W-1)+j}[c])   (W = 2..8)
 // per value channel c = h * dv + i, causal within each sequence, the inputs
 // before a sequence's first token taken from a carried state of its last W-1

@@ -311,8 +311,8 @@ def prefill_row_decay(q, k, v, g_rows, beta, h0=None, cu_seqlens=None, scale=1.0
 # ----------------------------------------------------------------------------
 # The layer steps around the rule: a short convolution on the values before it
 # and an output gate after it ("Qwen3-Next", sghael.github.io, section "Linear
-# attention with gated delta rule": the values pass through a 1-D convolution
-# that adds local context, and a gate scales what the recurrence returns).
+# attention with gated delta rule", names both: the values are mixed with their
+# recent predecessors, and what the recurrence returns is scaled by a gate).
 # The pages give neither the convolution's width nor the gate's form.  Reading:
 #   * a causal depthwise convolution along time, one kernel of width W per
 #     value channel (channel = h * dv + i), tap j multiplying the input W-1-j
