@@ -198,9 +198,12 @@ def ref_layer(x, ex, conv, gate, dtype, scale, stored=None, silu=True):
     return o, h, cs_new
 
 
-@pytest.mark.parametrize("dtype,d,chunk", [(torch.bfloat16, 128, 64), (torch.float32, 32, 16)])
+@pytest.mark.parametrize("dtype,d,chunk", [(torch.bfloat16, 128, 64), (torch.float32, 32, 16),
+                                           (torch.bfloat16, 64, 64)])
 @pytest.mark.parametrize("conv,gate", [(True, True), (True, False), (False, True)])
 def test_prefill_layer_matches_oracle(dtype, d, chunk, conv, gate):
+    # bf16 d = 128: tensor-core path; fp32 and bf16 d = 64: CUDA-core path (fp32
+    # gate factors for fp32, fp16 for bf16)
     lengths = [300, 77, 0, 129]
     x, ex = _layer_problem(lengths, dtype, d, 330)
     cs = ex["conv_state"].cuda() if conv else None
@@ -211,6 +214,35 @@ def test_prefill_layer_matches_oracle(dtype, d, chunk, conv, gate):
     assert_close(hT, h_ref, dtype, "hT")
     if conv:
         assert torch.equal(cs.cpu(), torch.from_numpy(cs_ref).to(dtype))
+
+
+def test_prefill_layer_with_prologue_and_row_decay():
+    # raw q/k normalised in the kernel, one decay per value row (CUDA-core path),
+    # convolution and gate: every flag of the layer call at once
+    lengths = [150, 0, 97]
+    x, ex = _layer_problem(lengths, torch.bfloat16, 128, 360)
+    raw = raw_projections(x, seed=361)
+    gr = row_decays(tuple(x["v"].shape), seed=362)
+    flags = (PROLOGUE_ALL & ~4) | ROW_DECAY
+    d = to_dev(dict(x, q=raw["q"], k=raw["k"]))
+    cs = ex["conv_state"].cuda()
+    o, hT = gdn_chunk_prefill_layer(d["q"], d["k"], d["v"], gr.cuda(), d["beta"], h0=d["h0"],
+                                    cu_seqlens=d["cu_seqlens"],
+                                    conv_weight=ex["conv_weight"].cuda(),
+                                    conv_bias=ex["conv_bias"].cuda(), conv_state=cs,
+                                    z=ex["z"].cuda(), scale=0.7, prologue=flags, silu=True)
+    torch.cuda.synchronize()
+    qn, kn, _, _ = O.prologue(raw["q"], raw["k"], x["g"], x["beta"], flags & 3)
+    C = x["v"].shape[2] * x["v"].shape[3]
+    vc, cs_ref = O.short_conv(x["v"].reshape(1, -1, C), ex["conv_weight"], ex["conv_bias"],
+                              ex["conv_state"], x["cu_seqlens"], activation="silu")
+    vc = torch.from_numpy(vc).to(torch.bfloat16).double().reshape(x["v"].shape)
+    o_ref, h_ref = O.prefill_row_decay(qn, kn, vc, gr, x["beta"], h0=x["h0"],
+                                       cu_seqlens=x["cu_seqlens"], scale=0.7)
+    o_ref = O.output_gate(o_ref, ex["z"].reshape(o_ref.shape))
+    assert_close(o[0], o_ref, torch.bfloat16, "o")
+    assert_close(hT, h_ref, torch.bfloat16, "hT")
+    assert torch.equal(cs.cpu(), torch.from_numpy(cs_ref).to(torch.bfloat16))
 
 
 def test_prefill_layer_then_steps_continue_the_sequence():
