@@ -8,9 +8,14 @@ Gated DeltaNet layer over one synthetic sequence: B=1, T=65536, 16 query/key
 heads shared by 32 value heads, head dim 128, chunk 64, bf16 q/k/v, fp32
 g/beta/state.  The same run also measures the fused decode step
 (``gdn_recurrent_step``) on 256 sequences x 64 tokens and reports its state
-HBM bandwidth in the ``decode`` object, and the speculative-decoding round
+HBM bandwidth in the ``decode`` object, the speculative-decoding round
 (``gdn_recurrent_verify`` of 4 drafts per sequence + the commit of the accepted
-prefix) in the ``verify`` object.
+prefix) in the ``verify`` object, the fused input prologue and one decay per
+value row in the ``prologue`` object, and the layer steps around the rule (the
+short convolution on the values and the output gate, in the prefill and in
+the decode step) in the ``layer`` object.  ``--no-decode``, ``--no-verify``,
+``--no-prologue``, ``--no-layer``, ``--no-e2e`` and ``--no-cpu-baseline`` skip
+the respective legs.
 
 Launch: ``python bench.py [--gpus N --steps K --warmup W]``; for N > 1 under
 ``torch.distributed.run``, one replica per GPU (each rank runs its own
