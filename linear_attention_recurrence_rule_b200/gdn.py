@@ -608,8 +608,10 @@ def gdn_output_gate(o, z, stream=None):
     _need(z, "z", o.dtype, dev)
     if z.shape != o.shape:
         raise ValueError("z must have o's shape")
+    if o.numel() == 0:
+        return o
     C = o.shape[-1] if o.dim() > 0 else 1
-    rows = o.numel() // C if C else 0
+    rows = o.numel() // C
     st = lib.gdn_output_gate(_ptr(o), _ptr(z), rows, C, _dtype_code(o), _stream_ptr(stream, dev))
     if st != GDN_OK:
         raise GDNError(st, "gdn_output_gate")
