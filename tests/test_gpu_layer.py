@@ -30,7 +30,7 @@ def packed_x(lengths, C, dtype, seed):
 @pytest.mark.parametrize("width", [2, 4, 8])
 @pytest.mark.parametrize("silu,with_state", [(False, False), (True, True)])
 def test_short_conv_packed_ragged(dtype, width, silu, with_state):
-    # lengths below width-1, around the 32-token runs and an empty sequence
+    # lengths below width-1, runs of 8 tokens crossing sequence starts, an empty sequence
     lengths = [0, 1, 2, 37, 64, 100, 3, 31, 33]
     C = 64
     x, cu = packed_x(lengths, C, dtype, seed=301 + width)
