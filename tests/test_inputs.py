@@ -71,3 +71,19 @@ def test_raw_projections_scale_rows_and_draw_logits():
     assert torch.allclose(cos, torch.ones_like(cos), atol=1e-6)
     assert y["g"].shape == x["g"].shape and float(y["g"].mean()) > 2.0
     assert torch.equal(y["v"], x["v"]) and torch.equal(y["state"], x["state"])
+
+
+def test_layer_extras_shapes_dtypes_and_seed():
+    from linear_attention_recurrence_rule_b200.inputs import layer_extras
+    a = layer_extras(3, 64, 4, (3, 7, 2, 32), torch.bfloat16, seed=9)
+    b = layer_extras(3, 64, 4, (3, 7, 2, 32), torch.bfloat16, seed=9)
+    c = layer_extras(3, 64, 4, (3, 7, 2, 32), torch.bfloat16, seed=10)
+    assert a["conv_weight"].shape == (64, 4) and a["conv_weight"].dtype == torch.float32
+    assert a["conv_bias"].shape == (64,) and a["conv_bias"].dtype == torch.float32
+    assert a["conv_state"].shape == (3, 3, 64) and a["conv_state"].dtype == torch.bfloat16
+    assert a["z"].shape == (3, 7, 2, 32) and a["z"].dtype == torch.bfloat16
+    for k in a:
+        assert torch.equal(a[k], b[k]) and not torch.equal(a[k], c[k])
+    big = layer_extras(1, 4096, 4, (1,), torch.float32, seed=1)
+    assert abs(float(big["conv_weight"].std()) - 0.5) < 0.02      # N(0, 1/W), W = 4
+    assert abs(float(big["conv_bias"].std()) - 0.1) < 0.01
