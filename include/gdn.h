@@ -407,7 +407,8 @@ GDN_API gdn_status gdn_state_commit_deltas(const void *k, const float *g, const 
  * "Qwen3-Next" (sghael.github.io), section "Linear attention with gated delta
  * rule", names two further layer steps: the values are mixed with their
  * recent predecessors by a short convolution before the rule, and its read-out
- * is scaled by a gate.  The page gives neither the width nor the gate's form.  Reading used here:
+ * is scaled by a gate.  The page gives neither the width nor the gate's form.
+ * Reading used here:
  *   - a causal depthwise convolution along time, one kernel of `width` taps
  *     (2..8) per value channel c = h * dv + i (C = HV * dv channels):
  *       y_t[c] = act(bias[c] + sum_{j<width} weight[c][j] * x_{t-(width-1)+j}[c])
@@ -434,8 +435,8 @@ GDN_API gdn_status gdn_state_commit_deltas(const void *k, const float *g, const 
  * multiple of 8 (bf16) or 4 (fp32).  Alignment: x, y, conv_state, weight
  * 16-byte; bias 4-byte.
  * y must not overlap x or conv_state.  Two launches (the convolution, then the
- * state update when conv_state is given).  N == 0 or no tokens: GDN_OK, and
- * only the state update runs.
+ * state update when conv_state is given).  N == 0: GDN_OK, nothing launched;
+ * no tokens: only the state update runs (and keeps every state).
  */
 GDN_API gdn_status gdn_short_conv(const void *x, const float *weight, const float *bias,
                                   void *conv_state, const int32_t *cu_seqlens, int N, int64_t T,
@@ -486,8 +487,8 @@ GDN_API size_t gdn_chunk_prefill_layer_workspace_size(int N, int64_t T, int HK, 
  * tensor-core path takes bf16 operands; conv_state [N][conv_width-1][HV*dv]
  * updated as there), the gate factors sigmoid(z) into the workspace (fp16,
  * relative error <= 2^-12, for bf16 calls; fp32 for fp32 calls), then the
- * prefill on the convolved values, which
- * multiplies o by the factors where it writes o (z like v; o is rounded once).
+ * prefill on the convolved values, which multiplies o by the factors where it
+ * writes o (z like v; o is rounded once).
  * conv_weight NULL: no convolution; z NULL: no gate.  flags: GDN_PROLOGUE_*,
  * GDN_ROW_DECAY and GDN_CONV_SILU.  Launches on `stream`: the convolution's
  * two, the factors' one, the prefill's one; arguments as in
