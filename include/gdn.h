@@ -79,7 +79,12 @@ GDN_API int gdn_version(void);
  * Bytes of device workspace gdn_chunk_prefill needs for this problem.
  * N: number of sequences; T: tokens per sequence without cu_seqlens, else the
  * packed total; varlen: nonzero when cu_seqlens will be passed.  Returns 0 for
- * arguments gdn_chunk_prefill would reject.
+ * arguments gdn_chunk_prefill would reject.  On the tensor-core path (bf16,
+ * dk = dv = 128, chunk 64) the workspace holds a status word and, per SM of the
+ * current device, a ring of six 65 KB chunk records through which the kernel's
+ * prep CTAs hand their results to its chain CTA (~59 MB on a 148-SM B200,
+ * independent of N and T); the size is computed for the device current at the
+ * time of the query.
  */
 GDN_API size_t gdn_chunk_prefill_workspace_size(int N, int64_t T, int HK, int HV, int dk, int dv,
                                         int chunk, gdn_dtype dtype, int varlen);
@@ -186,8 +191,8 @@ GDN_API gdn_status gdn_chunk_prefill_ex(const void *q, const void *k, const void
  * For callers that cannot allocate device memory -- code running under a
  * fixed, pre-reserved memory budget, a hot path that must not call cudaMalloc
  * (it can synchronise the device and stall other streams), or a host API that
- * offers no workspace.  Same arguments, layouts and results as
- * gdn_chunk_prefill; the scratch it needs lives in a 256-byte array inside the
+ * offers no workspace.  Same arguments and layouts as gdn_chunk_prefill;
+ * the scratch it needs lives in a 256-byte array inside the
  * library that every device loading the library keeps until the process exits.
  *   - Problems needing more than 256 bytes of workspace (see
  *     gdn_chunk_prefill_workspace_size) return GDN_ERR_WORKSPACE.
@@ -197,7 +202,15 @@ GDN_API gdn_status gdn_chunk_prefill_ex(const void *q, const void *k, const void
  *     calls whose work overlaps on the GPU (different streams, not ordered)
  *     race on it.  Order them on one stream, or use gdn_chunk_prefill with
  *     separate workspaces.
+ *   - Whether the on-device waits of the last call completed: gdn_read_status
+ *     with a NULL workspace reads the array's status word.
+ *   - The looked-up address belongs to the device's primary context: after
+ *     cudaDeviceReset, do not call it again in the same process.
  *   - It allocates nothing and calls no allocating routine.
+ *   - On the tensor-core path it runs the cluster kernel whose only scratch is
+ *     that status word (gdn_chunk_prefill runs the faster kernel that also needs
+ *     a ring of chunk records in its workspace); its results agree with
+ *     gdn_chunk_prefill's within the bf16 tolerance, not bit for bit.
  */
 GDN_API gdn_status gdn_chunk_prefill_noalloc(const void *q, const void *k, const void *v,
                                              const float *g, const float *beta, const float *h0,
@@ -509,6 +522,9 @@ GDN_API gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const v
  * call; synchronises `stream`).  Returns GDN_OK when every on-device wait of
  * the last call on this workspace completed, GDN_ERR_TIMEOUT when one gave up
  * (the outputs of that call are then undefined), or GDN_ERR_CUDA.
+ * workspace NULL: reads the status word in the library array that
+ * gdn_chunk_prefill_noalloc uses on the current device (the last such call's
+ * waits); GDN_ERR_CUDA when no device is usable.
  */
 GDN_API gdn_status gdn_read_status(const void *workspace, size_t workspace_bytes, gdn_stream_t stream);
 

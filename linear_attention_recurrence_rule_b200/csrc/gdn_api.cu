@@ -17,7 +17,7 @@ bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr
 bool aligned4(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool tc_path(int dk, int dv, int chunk, gdn_dtype dt) {
-    return gdn::prefill_cluster_supported(dk, dv, chunk, dt);
+    return gdn::prefill_ring_supported(dk, dv, chunk, dt);
 }
 
 gdn_status check_prefill(const gdn::PrefillArgs &a) {
@@ -36,33 +36,50 @@ gdn_status check_prefill(const gdn::PrefillArgs &a) {
     return GDN_OK;
 }
 
+}  // namespace
+
+namespace gdn {
+
+size_t prefill_workspace_bytes(const PrefillArgs &a) {
+    if (!tc_path(a.dk, a.dv, a.chunk, a.dtype) || (a.prologue & GDN_ROW_DECAY)) return 0;
+    return a.status_only ? prefill_cluster_workspace(a.N, a.T, a.HV, a.chunk, a.cu_seqlens != nullptr)
+                         : prefill_ring_workspace(a.N, a.T, a.HV, a.chunk, a.cu_seqlens != nullptr);
+}
+
 // Validation, workspace check and dispatch of one prefill call (tensor-core path
 // for bf16 / d = 128 / chunk 64, CUDA-core path otherwise).
-gdn_status enqueue_prefill(const gdn::PrefillArgs &a, cudaStream_t stream) {
+gdn_status enqueue_prefill(const PrefillArgs &a, cudaStream_t stream) {
     gdn_status st = check_prefill(a);
     if (st != GDN_OK) return st;
     if (a.N == 0) return GDN_OK;
     cudaError_t err;
     // one decay per value row: only the CUDA-core path (a per-row triangular inverse)
     if (tc_path(a.dk, a.dv, a.chunk, a.dtype) && !(a.prologue & GDN_ROW_DECAY)) {
-        const size_t need = gdn::prefill_cluster_workspace(a.N, a.T, a.HV, a.chunk, a.cu_seqlens != nullptr);
+        const size_t need = prefill_workspace_bytes(a);
         if (need > 0 && (a.workspace == nullptr || a.workspace_bytes < need)) return GDN_ERR_WORKSPACE;
         if (!aligned16(a.workspace)) return GDN_ERR_ALIGNMENT;
-        err = gdn::launch_prefill_cluster(a, stream);
+        err = a.status_only ? launch_prefill_cluster(a, stream) : launch_prefill_ring(a, stream);
     } else {
-        err = gdn::launch_prefill_simt(a, stream);
+        err = launch_prefill_simt(a, stream);
     }
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
+
+}  // namespace gdn
+
+namespace {
+
+using gdn::enqueue_prefill;
 
 // Device workspace of gdn_chunk_prefill_host: the status word, two input and two
 // output segment buffers (inputs packed q | k | v | g | beta) and two states.
 struct HostPlan {
     int64_t seg;
     size_t elt, q_bytes, v_bytes, g_bytes;
-    size_t status, in[2], out[2], st[2], total;
+    size_t status, pre, in[2], out[2], st[2], total;
     static size_t up(size_t x) { return (x + 255) & ~size_t(255); }
-    HostPlan(int N, int64_t T, int HK, int HV, int dk, int dv, gdn_dtype dtype, int64_t segment) {
+    HostPlan(int N, int64_t T, int HK, int HV, int dk, int dv, int chunk, gdn_dtype dtype,
+             int64_t segment) {
         seg = segment > 0 ? segment : 4096;
         if (T > 0 && seg > T) seg = T;
         if (seg <= 0) seg = 1;
@@ -74,8 +91,18 @@ struct HostPlan {
         const size_t in_b = 2 * q_bytes + v_bytes + 2 * g_bytes;
         const size_t out_b = v_bytes;
         const size_t st_b = up((size_t)N * HV * dv * dk * 4);
+        // the segment prefill's own workspace (status word first) at the start
+        gdn::PrefillArgs a{};
+        a.N = N;
+        a.T = seg;
+        a.HV = HV;
+        a.dk = dk;
+        a.dv = dv;
+        a.chunk = chunk;
+        a.dtype = dtype;
         status = 0;
-        size_t off = 256;
+        pre = up(gdn::prefill_workspace_bytes(a) > 256 ? gdn::prefill_workspace_bytes(a) : 256);
+        size_t off = pre;
         for (int b = 0; b < 2; ++b) { in[b] = off; off += in_b; }
         for (int b = 0; b < 2; ++b) { out[b] = off; off += out_b; }
         for (int b = 0; b < 2; ++b) { st[b] = off; off += st_b; }
@@ -112,7 +139,7 @@ int gdn_chunk_prefill_path(int dk, int dv, int chunk, gdn_dtype dtype) {
 size_t gdn_chunk_prefill_workspace_size(int N, int64_t T, int HK, int HV, int dk, int dv,
                                         int chunk, gdn_dtype dtype, int varlen) {
     if (N < 0 || T < 0 || HK <= 0 || HV <= 0 || HV % HK || chunk <= 0) return 0;
-    if (tc_path(dk, dv, chunk, dtype)) return gdn::prefill_cluster_workspace(N, T, HV, chunk, varlen != 0);
+    if (tc_path(dk, dv, chunk, dtype)) return gdn::prefill_ring_workspace(N, T, HV, chunk, varlen != 0);
     return 0;
 }
 
@@ -145,7 +172,7 @@ size_t gdn_chunk_prefill_host_workspace_size(int N, int64_t T, int HK, int HV, i
     if (N <= 0 || T < 0 || HK <= 0 || HV <= 0 || HV % HK || chunk <= 0 || segment < 0) return 0;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return 0;
     if (gdn_chunk_prefill_path(dk, dv, chunk, dtype) < 0) return 0;
-    return HostPlan(N, T, HK, HV, dk, dv, dtype, segment).total;
+    return HostPlan(N, T, HK, HV, dk, dv, chunk, dtype, segment).total;
 }
 
 gdn_status gdn_chunk_prefill_host(const void *q, const void *k, const void *v, const float *g,
@@ -163,7 +190,7 @@ gdn_status gdn_chunk_prefill_host(const void *q, const void *k, const void *v, c
         const gdn_status st = check_prefill(a);
         if (st != GDN_OK) return st;
     }
-    const HostPlan plan(N, T, HK, HV, dk, dv, dtype, segment);
+    const HostPlan plan(N, T, HK, HV, dk, dv, chunk, dtype, segment);
     if (workspace == nullptr || workspace_bytes < plan.total) return GDN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_ALIGNMENT;
     if (T == 0) return GDN_OK;
@@ -223,7 +250,7 @@ gdn_status gdn_chunk_prefill_host(const void *q, const void *k, const void *v, c
         uint8_t *out = ws + plan.out[b];
         gdn::PrefillArgs a{dq, dk_, dv_, reinterpret_cast<const float *>(dg),
                            reinterpret_cast<const float *>(db), hin, nullptr, N, Ls, HK, HV, dk,
-                           dv, chunk, scale, dtype, out, hout, ws + plan.status, 256};
+                           dv, chunk, scale, dtype, out, hout, ws + plan.status, plan.pre};
         a.keep_status = true;
         const gdn_status st = enqueue_prefill(a, sc);
         if (st != GDN_OK) {
@@ -518,9 +545,7 @@ gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, 
     if (z && !aligned16(z)) return GDN_ERR_ALIGNMENT;
     if (N == 0) return GDN_OK;
     // workspace: [prefill's own | convolved values | gate factors (fp16)]
-    const size_t pre = up256(gdn::prefill_cluster_supported(dk, dv, chunk, dtype) && !(prologue & GDN_ROW_DECAY)
-                                 ? gdn::prefill_cluster_workspace(N, T, HV, chunk, varlen)
-                                 : 0);
+    const size_t pre = up256(gdn::prefill_workspace_bytes(a));
     const size_t vbytes = conv_weight ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen) : 0;
     const size_t need = pre + vbytes + (z ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen) : 0);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
@@ -546,9 +571,11 @@ gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, 
 }
 
 gdn_status gdn_read_status(const void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
-    if (workspace == nullptr || workspace_bytes < sizeof(unsigned int)) return GDN_OK;
-    unsigned int word = 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // NULL: the library array of the workspace-free prefill on the current device
+    if (workspace == nullptr) return gdn::noalloc_read_status(s);
+    if (workspace_bytes < sizeof(unsigned int)) return GDN_OK;
+    unsigned int word = 0;
     if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return GDN_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;

@@ -26,6 +26,8 @@ struct PrefillArgs {
     unsigned prologue = 0;      // GDN_PROLOGUE_* flags
     const void *gate = nullptr; // output gate factors sigmoid(z), o's layout: fp16 for
                                 // bf16 calls, fp32 for fp32 calls
+    bool status_only = false;   // tensor-core path: the kernel whose only scratch is the
+                                // status word (the workspace-free entry point)
 };
 
 struct StepArgs {
@@ -122,5 +124,19 @@ bool prefill_cluster_supported(int dk, int dv, int chunk, gdn_dtype dtype);
 // device workspace the cluster prefill needs: the status word of its bounded waits
 size_t prefill_cluster_workspace(int N, int64_t T, int HV, int chunk, bool varlen);
 cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream);
+
+// tensor-core prefill with the prep results handed over through a ring of chunk
+// records in the workspace (gdn_prefill_ring.cu): the default tensor-core path
+bool prefill_ring_supported(int dk, int dv, int chunk, gdn_dtype dtype);
+// device workspace: the status word and one ring of chunk records per SM id
+size_t prefill_ring_workspace(int N, int64_t T, int HV, int chunk, bool varlen);
+cudaError_t launch_prefill_ring(const PrefillArgs &a, cudaStream_t stream);
+
+// validation, workspace check and dispatch of one prefill call (gdn_api.cu)
+gdn_status enqueue_prefill(const PrefillArgs &a, cudaStream_t stream);
+// workspace bytes of one prefill call (0: none needed)
+size_t prefill_workspace_bytes(const PrefillArgs &a);
+// status word of the workspace-free prefill's library array (gdn_noalloc.cu)
+gdn_status noalloc_read_status(cudaStream_t stream);
 
 }  // namespace gdn

@@ -109,7 +109,9 @@ def test_workspace_size_rejects_bad_shapes(lib):
 
 
 def test_read_status_without_workspace(lib):
-    assert lib.gdn_read_status(None, 0, None) == gdn.GDN_OK
+    # a NULL workspace reads the workspace-free prefill's library array on the
+    # current device: without a usable device that is a CUDA error, not OK
+    assert lib.gdn_read_status(None, 0, None) == gdn.GDN_ERR_CUDA
 
 
 def verify_call(lib, **kw):
