@@ -303,18 +303,11 @@ def test_prefill_layer_bench_size_sampled_heads():
 
 
 def test_prefill_layer_bench_size_silu_values():
-    # With SiLU after the convolution the values have a positive mean, the state
-    # grows a large common component and o = S q stays small beside it: the
-    # single-bf16 S0 operand of the tensor-core read-out (relative error 2^-9 of
-    # |S|) then weighs more against RMS(o).  Bound for this regime: the RMS error
-    # within 2e-2 of RMS(o) as everywhere, the largest element within 1.5 x the
-    # max-norm bound (measured 1.10 x at the 64K bench size).
+    # SiLU after the convolution gives the values a positive mean, so the state
+    # grows a large common component and o = S q stays small beside it; the
+    # tensor-core read-out carries S0 as a bf16 hi + lo pair, which keeps the
+    # 64K layer prefill inside the standard bf16 bound
     for vh, o, o_ref, h, h_ref in _bench_size_layer(silu=True):
-        o_np = o.double().cpu().numpy().reshape(o_ref.shape)
-        diff = np.abs(o_np - o_ref)
-        rms = float(np.sqrt(np.mean(o_ref ** 2)))
-        assert float(np.sqrt(np.mean(diff ** 2))) <= 2e-2 * rms, f"o heads {vh}: RMS error"
-        worst = float((diff / (2e-2 * rms + 2.0 ** -8 * np.abs(o_ref))).max())
-        print(f"heads {vh}: worst max-norm ratio {worst:.3f}")
-        assert worst <= 1.5, f"o heads {vh}: worst ratio {worst:.3f}"
+        assert_close(o, o_ref, torch.bfloat16, f"o heads {vh}")
         assert_close(h, h_ref, torch.bfloat16, f"hT heads {vh}")
+

@@ -11,9 +11,10 @@ from linear_attention_recurrence_rule_b200 import (PROLOGUE_ALL, PROLOGUE_GATE_L
                                                    gdn_recurrent_verify, gdn_state_commit,
                                                    gdn_state_commit_deltas)
 from linear_attention_recurrence_rule_b200.inputs import (make_decode, make_prefill, make_verify,
-                                                          raw_projections, row_decays)
+                                                          raw_projections, row_decays,
+                                                          workload_inputs)
 from oracle import gdn_oracle as O
-from parity_util import assert_close, to_dev
+from parity_util import assert_close, head_slice, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -108,3 +109,23 @@ def test_row_decay_unsupported_forms():
     with pytest.raises(GDNError):
         gdn_recurrent_verify(e["q"], e["k"], e["v"], g_rows, e["beta"], e["state"],
                              rollback="deltas", prologue=ROW_DECAY)
+
+
+def test_prefill_row_decay_bench_size_sampled_heads():
+    """The workload the bench times for one decay per value row: the 4K-token
+    layer (16 query/key heads, 32 value heads, d = 128, bf16) with row decays
+    alpha ~U(0.8, 1), all heads in one call; the oracle checks two query/key
+    heads and their value heads."""
+    x = workload_inputs("layer_prefill_4k")
+    g_rows = row_decays(tuple(x["v"].shape), seed=903)
+    d = to_dev(x)
+    o, hT = gdn_chunk_prefill(d["q"], d["k"], d["v"], g_rows.cuda(), d["beta"], chunk=64,
+                              prologue=ROW_DECAY)
+    torch.cuda.synchronize()
+    HV = x["v"].shape[2]
+    for qk in ([0], [15]):
+        sub, vh = head_slice(x, qk, HV // x["q"].shape[2])
+        o_ref, h_ref = O.prefill_row_decay(sub["q"], sub["k"], sub["v"], g_rows[:, :, vh],
+                                           sub["beta"])
+        assert_close(o[0][:, vh], o_ref, torch.bfloat16, f"o heads {vh}")
+        assert_close(hT[:, vh], h_ref, torch.bfloat16, f"hT heads {vh}")
