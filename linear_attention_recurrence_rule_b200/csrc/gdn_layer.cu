@@ -1,8 +1,8 @@
 // The layer steps around the rule: a short causal convolution on the values
-// before it and a sigmoid gate on its read-out after it ("Qwen3-Next",
-// sghael.github.io, section "Linear attention with gated delta rule", names
-// both: the values are mixed with their recent predecessors, and the rule's
-// read-out is scaled by a gate).  The page gives neither the width nor the
+// before it and a sigmoid gate on its read-out after it ("Qwen3-Next 80B-A3B --
+// The Evolving Transformer", llamasearch.dev, section 01 GatedDeltaNet, names
+// both: a one-dimensional convolution gives the values local context, and a
+// gate sets how much of the rule's read-out reaches the output).  The page gives neither the width nor the
 // gate's form; the library reads them as
 //   y_t[c] = act(bias[c] + sum_{j<W} w[c][j] x_{t-(W-1)+j}[c])   (W = 2..8)
 // per value channel c = h * dv + i, causal within each sequence, the inputs

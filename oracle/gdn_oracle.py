@@ -310,9 +310,10 @@ def prefill_row_decay(q, k, v, g_rows, beta, h0=None, cu_seqlens=None, scale=1.0
 
 # ----------------------------------------------------------------------------
 # The layer steps around the rule: a short convolution on the values before it
-# and an output gate after it ("Qwen3-Next", sghael.github.io, section "Linear
-# attention with gated delta rule", names both: the values are mixed with their
-# recent predecessors, and what the recurrence returns is scaled by a gate).
+# and an output gate after it ("Qwen3-Next 80B-A3B -- The Evolving Transformer",
+# llamasearch.dev, section 01 GatedDeltaNet, names both: a one-dimensional
+# convolution gives the values local context, and a gate sets how much of what
+# the recurrence returns reaches the output).
 # The pages give neither the convolution's width nor the gate's form.  Reading:
 #   * a causal depthwise convolution along time, one kernel of width W per
 #     value channel (channel = h * dv + i), tap j multiplying the input W-1-j

@@ -509,8 +509,8 @@ def pin_verify_row_decay_equals_steps(lib=None):
 
 # ----------------------------------------------------------------------------
 # The short convolution on the values and the output gate around the rule
-# ("Qwen3-Next", sghael.github.io, section "Linear attention with gated delta
-# rule"; widths and forms are readings, see the oracle's section header)
+# ("Qwen3-Next 80B-A3B -- The Evolving Transformer", llamasearch.dev, section 01
+# GatedDeltaNet; widths and forms are readings, see the oracle's section header)
 # ----------------------------------------------------------------------------
 def pin_short_conv_is_a_library_convolution(lib=None):
     """Per channel the causal convolution equals numpy's full convolution of the
