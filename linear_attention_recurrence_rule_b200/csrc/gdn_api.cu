@@ -512,7 +512,8 @@ size_t gdn_chunk_prefill_layer_workspace_size(int N, int64_t T, int HK, int HV, 
                                               int has_conv, int has_gate) {
     if (N < 0 || T < 0 || HK <= 0 || HV <= 0 || HV % HK || dv <= 0 || chunk <= 0) return 0;
     const size_t pre = up256(gdn_chunk_prefill_workspace_size(N, T, HK, HV, dk, dv, chunk, dtype, varlen));
-    return pre + (has_conv ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen != 0) : 0) +
+    const bool vpair = has_conv && tc_path(dk, dv, chunk, dtype);
+    return pre + (has_conv ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen != 0) * (vpair ? 2 : 1) : 0) +
            (has_gate ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen != 0) : 0);
 }
 
@@ -546,15 +547,21 @@ gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, 
     if (N == 0) return GDN_OK;
     // workspace: [prefill's own | convolved values | gate factors (fp16)]
     const size_t pre = up256(gdn::prefill_workspace_bytes(a));
-    const size_t vbytes = conv_weight ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen) : 0;
+    // on the tensor-core path the convolved values go to the rule as a bf16 pair
+    // (values + remainders): their rounding to bf16 alone would weigh on o where the
+    // state has a large common component (SiLU-convolved values)
+    const bool vpair = conv_weight && tc_path(dk, dv, chunk, dtype) && !(prologue & GDN_ROW_DECAY);
+    const size_t vbytes = conv_weight ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen) * (vpair ? 2 : 1) : 0;
     const size_t need = pre + vbytes + (z ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen) : 0);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (conv_weight) {
         ca.y = static_cast<char *>(workspace) + pre;
+        if (vpair) ca.y_lo = static_cast<char *>(workspace) + pre + vbytes / 2;
         if (gdn::launch_short_conv(ca, s) != cudaSuccess) return GDN_ERR_CUDA;
         a.v = ca.y;
+        a.v_lo = ca.y_lo;
     }
     if (z) {
         // sigmoid(z) factors (fp16 for bf16, fp32 for fp32), applied in the prefill's

@@ -28,6 +28,8 @@ struct PrefillArgs {
                                 // bf16 calls, fp32 for fp32 calls
     bool status_only = false;   // tensor-core path: the kernel whose only scratch is the
                                 // status word (the workspace-free entry point)
+    const void *v_lo = nullptr; // bf16 remainders of v (v + v_lo carries it to ~2^-17;
+                                // tensor-core path, the layer prefill's convolved values)
 };
 
 struct StepArgs {
@@ -103,6 +105,7 @@ struct ConvArgs {
     bool silu;
     gdn_dtype dtype;
     void *y;
+    void *y_lo = nullptr;         // bf16 only: y_lo = y_exact - y, a second output
 };
 constexpr int kConvMaxWidth = 8;
 int conv_vector_channels(gdn_dtype dtype);   // channels per 16-byte vector

@@ -100,7 +100,8 @@ template <typename T, int W>
 __global__ void __launch_bounds__(kConvThreads)
 conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
             const T *__restrict__ cstate, const int32_t *__restrict__ cu, int N, int64_t T_per,
-            int64_t Ttot, int C, int cblocks, bool silu, T *__restrict__ y) {
+            int64_t Ttot, int C, int cblocks, bool silu, T *__restrict__ y,
+            T *__restrict__ y_lo) {
     constexpr int VN = Vec16<T>::n;
     // the channel blocks of one run are neighbours in the grid, so the blocks
     // resident at a time read whole token rows
@@ -194,7 +195,17 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
                 const float a = fmaf(wt[W - 1][e], f[e], acc[e]);
                 acc[e] = silu ? a * layer_sigmoid(a) : a;
             }
-            st16(y + t * C + c0, Vec16<T>::from_float(acc));
+            const uint4 yv = Vec16<T>::from_float(acc);
+            st16(y + t * C + c0, yv);
+            if (y_lo) {
+                // the remainder acc - y (exact in fp32) as a second output: the bf16
+                // pair y + y_lo carries the convolved value to ~2^-17 relative
+                float r[VN];
+                Vec16<T>::to_float(yv, r);
+#pragma unroll
+                for (int e = 0; e < VN; ++e) r[e] = acc[e] - r[e];
+                st16(y_lo + t * C + c0, Vec16<T>::from_float(r));
+            }
 #pragma unroll
             for (int m = 0; m + 1 < W - 1; ++m) win[m] = win[m + 1];
             win[W - 2] = raw[u];
@@ -299,7 +310,7 @@ cudaError_t launch_conv_w(const ConvArgs &a, cudaStream_t stream) {
         const unsigned grid = (unsigned)((Ttot + kConvRun - 1) / kConvRun * cblocks);
         conv_kernel<T, W><<<grid, kConvThreads, 0, stream>>>(
             x, a.weight, a.bias, cs, a.cu_seqlens, a.N, a.T, Ttot, a.C, (int)cblocks, a.silu,
-            static_cast<T *>(a.y));
+            static_cast<T *>(a.y), static_cast<T *>(a.y_lo));
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -87,7 +87,8 @@ constexpr uint32_t RS_P = 16384;     // P hi, P lo: 64 rows (t) x 64 (s), K-majo
 constexpr uint32_t RS_TAB = 32768;   // fp32: gamma_L/gamma_t [64], gamma_t [64], gamma_L
 constexpr uint32_t RS_U = 33792;     // U~ fp32, [value row][token], rows UT_LD floats apart
 constexpr uint32_t UT_LD = 68;       // (a padded pitch: 16-byte row reads are conflict-free)
-constexpr uint32_t RS_STAGED = RS_U; // the part staged in the prep CTA's shared memory
+// the parts staged in the prep CTA's shared memory (P and U~ go to the record directly)
+constexpr uint32_t ST_W = 0, ST_TAB = 16384, ST_BYTES = 17408;
 constexpr uint32_t RSLOT = RS_U + DH * UT_LD * 4;   // 68608
 constexpr size_t kRingHeader = 256;  // status word (and padding) before the rings
 
@@ -114,8 +115,9 @@ constexpr uint32_t P_X = P_TF + 64 * T_LD * 4;
 constexpr uint32_t X_LD = 36;
 constexpr uint32_t P_T2 = 138240;                 // T'' hi, T'' lo (B operand of U~^T)
 constexpr uint32_t P_PB = P_T2 + 16384;           // beta, gamma, G, 1/|q|, 1/|k|
-constexpr uint32_t P_ST = 156672;                 // two staging blocks (RS_STAGED bytes each)
-constexpr uint32_t P_BAR = P_ST + 2 * RS_STAGED;
+constexpr uint32_t P_ST = 156672;                 // two staging blocks (ST_BYTES each)
+constexpr uint32_t P_VL = P_ST + 2 * ST_BYTES;    // two v remainder buffers (values given as a pair)
+constexpr uint32_t P_BAR = P_VL + 2 * V_STRIDE;
 
 enum ChainBar { CB_FULL0, CB_FULL1, CB_RING0, CB_FREE0 = CB_RING0 + kRing, CB_FREE1,
                 CB_U, CB_Q, CB_S, CB_O, CB_QREAD, CB_ODRAIN, CB_DRAIN, CB_Z0,
@@ -133,7 +135,8 @@ static_assert(P_X + 32 * X_LD * 4 <= P_T2, "prep layout");
 static_assert(P_PB + 5 * 64 * 4 <= P_ST, "prep layout");
 static_assert(64 * A_LD * 4 >= 16384, "T' tiles fit where A was");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(P_ST % 1024 == 0 && SLOT % 1024 == 0 && RS_STAGED % 1024 == 0 && P_T % 1024 == 0 &&
+static_assert(P_ST % 1024 == 0 && SLOT % 1024 == 0 && ST_BYTES % 1024 == 0 && P_VL % 1024 == 0 &&
+                  P_T % 1024 == 0 &&
                   P_T2 % 1024 == 0 && P_V % 1024 == 0 && C_OT % 1024 == 0,
               "swizzle alignment");
 static_assert(RSLOT % 16 == 0 && RS_U % 16 == 0, "bulk copy alignment");
@@ -158,6 +161,7 @@ struct RingParams {
     uint8_t *rings;          // kRing records per SM id
     int nrings;              // SM ids the rings cover
     unsigned int prologue;   // GDN_PROLOGUE_* flags
+    bool vpair;              // v comes with bf16 remainders (tm_vl): U~ = T''(V + V_lo)
 };
 
 // Release arrive on another cluster CTA's mbarrier: the arriving thread's earlier
@@ -716,7 +720,7 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
 // ============================================================================ prep CTA
 template <bool PRO>
 __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
-                         const RingParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
+                         const CUtensorMap *tm_vl, const RingParams &p, uint8_t *sm, uint32_t sb, uint32_t tmem,
                          const Waiter &wt, int h, int64_t bos, int64_t eos, int nchunks, int rank,
                          uint8_t *ring) {
     uint64_t *bars = wt.bars;
@@ -744,7 +748,12 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 uint64_t *bar = &bars[PB_LD0 + (k & 1)];
                 uint8_t *buf = sm + P_QK + (k & 1) * QK_STRIDE;
                 uint8_t *vb = sm + P_V + (k & 1) * V_STRIDE;
-                mbar_arrive_expect_tx(bar, 6 * 8192);
+                mbar_arrive_expect_tx(bar, (p.vpair ? 8 : 6) * 8192);
+                if (p.vpair) {
+                    uint8_t *vl = sm + P_VL + (k & 1) * V_STRIDE;
+                    tma_load_3d(vl, tm_vl, bar, 0, h, s0);
+                    tma_load_3d(vl + 8192, tm_vl, bar, 64, h, s0);
+                }
                 tma_load_3d(buf, tm_q, bar, 0, cqk, s0);
                 tma_load_3d(buf + 16384, tm_q, bar, 64, cqk, s0);
                 tma_load_3d(buf + 8192, tm_k, bar, 0, cqk, s0);
@@ -778,6 +787,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 tma_prefetch_desc(tm_q);
                 tma_prefetch_desc(tm_k);
                 tma_prefetch_desc(tm_v);
+                if (p.vpair) tma_prefetch_desc(tm_vl);
             }
             load(0);
             if (nk > 1) load(1);
@@ -793,11 +803,14 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             if (k + 1 < nk && !x_product(k + 1)) break;
             if (!warp_all(wt(PB_T, ph))) break;
             tc_fence_after();
-            // W^T = K^T T'^T and U~^T = V^T T''^T (T', T'' as hi + lo)
+            // W^T = K^T T'^T and U~^T = V^T T''^T (T', T'' as hi + lo; V as V + V_lo
+            // when the values come as a pair)
+            const uint32_t vlb = sb + P_VL + (k & 1) * V_STRIDE;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t ka = sdesc_sw128(qkv + 8192 + kk * 2048, 16384, 1024);
                 const uint64_t va = sdesc_sw128(vb + kk * 2048, 8192, 1024);
+                const uint64_t val = sdesc_sw128(vlb + kk * 2048, 8192, 1024);
                 const uint64_t t1h = sdesc_sw128(sb + P_T + kk * 32, 16, 1024);
                 const uint64_t t1l = sdesc_sw128(sb + P_T + 8192 + kk * 32, 16, 1024);
                 const uint64_t t2h = sdesc_sw128(sb + P_T2 + kk * 32, 16, 1024);
@@ -807,6 +820,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                     mma_bf16(tmem + TP_W, ka, t1l, id_w, 1);
                     mma_bf16(tmem + TP_U, va, t2h, id_w, kk > 0);
                     mma_bf16(tmem + TP_U, va, t2l, id_w, 1);
+                    if (p.vpair) mma_bf16(tmem + TP_U, val, t2h, id_w, 1);
                 }
                 __syncwarp();
             }
@@ -818,8 +832,10 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             if (k + 2 < nk) load(k + 2);
             if (lane == 0) {
                 uint8_t *rec = ring + (size_t)(c % kRing) * RSLOT;
+                const uint32_t stg = sb + P_ST + (k & 1) * ST_BYTES;
                 fence_proxy_async_smem();
-                bulk_store_s2g(rec, sb + P_ST + (k & 1) * RS_STAGED, RS_STAGED);
+                bulk_store_s2g(rec + RS_W, stg + ST_W, 16384);
+                bulk_store_s2g(rec + RS_TAB, stg + ST_TAB, ST_BYTES - ST_TAB);
                 bulk_commit_group();
                 bulk_wait_group0();
                 fence_proxy_async_global();
@@ -870,7 +886,8 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             const int c = chunk_of(k);
             const uint32_t ph = (uint32_t)(k & 1);
             const int L = chunk_len(c);
-            const uint32_t stb = P_ST + (k & 1) * RS_STAGED;   // this chunk's staging block
+            const uint32_t stb = P_ST + (k & 1) * ST_BYTES;   // this chunk's staging block
+            uint8_t *rec = ring + (size_t)(c % kRing) * RSLOT;     // and its ring record
             named_sync(NB_WORK, kPWorkThreads);
             float2 gb = gb_next;
             if (warp <= kPWork0 + 1 && k + 1 < nk) gb_next = load_gb(k + 1);
@@ -894,9 +911,11 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 beta_s[2 * lane] = bp.x;
                 beta_s[2 * lane + 1] = bp.y;
             }
-            // the X product is done; this staging block's previous contents (chunk
-            // k - 2) were stored into the ring before chunk k - 1's X product began
+            // the X product is done (this staging block's previous contents, chunk k - 2,
+            // were stored before chunk k's X product began), and the chain has taken
+            // chunk c - kRing out of this ring record
             ok = warp_all(ok && wt(PB_X, ph));
+            if (k >= 2) ok = warp_all(ok && wt(PB_RFREE0 + (k & 1), (uint32_t)(((k >> 1) - 1) & 1)));
             if (norm_qk) {
                 // squared norms of the 64 q and 64 k rows of the landed tiles: four
                 // threads per row, 64 bytes each (the 128B swizzle only permutes the
@@ -954,8 +973,14 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                     }
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
+                        // P hi and lo into the record, as the chain CTA's swizzled operand image
                         const uint32_t off = sw128_chunk(row, 2 * qtr + cc);
-                        st_chunk_hilo(sb + stb + RS_P + off, sb + stb + RS_P + 8192 + off, v + 8 * cc);
+                        uint32_t hw[4], lw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            split_pair(make_float2(v[8 * cc + 2 * e], v[8 * cc + 2 * e + 1]), hw[e], lw[e]);
+                        *reinterpret_cast<uint4 *>(rec + RS_P + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        *reinterpret_cast<uint4 *>(rec + RS_P + 8192 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
                     }
                 } else {
                     const float bi = beta_s[row] * ri;
@@ -977,7 +1002,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 }
                 // decay table of this chunk for the chain CTA
                 if (pt < 64) {
-                    float *tb = reinterpret_cast<float *>(sm + stb + RS_TAB);
+                    float *tb = reinterpret_cast<float *>(sm + stb + ST_TAB);
                     tb[pt] = __expf(G_p[63] - G_p[pt]) * rk(pt);   // gamma_L / gamma_t / |k_t|
                     tb[64 + pt] = gam_p[pt] * rq(pt);              // gamma_t / |q_t|
                     if (pt == 0) tb[128] = gam_p[63];      // gamma_L
@@ -1105,8 +1130,6 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             if (lane == 0) local_arrive(&bars[PB_T]);
             // ---- -W into the staging block, U~ into the ring record ----
             ok = warp_all(ok && wt(PB_WU, ph));
-            // the chain has taken chunk c - kRing out of this ring slot
-            if (k >= 2) ok = warp_all(ok && wt(PB_RFREE0 + (k & 1), (uint32_t)(((k >> 1) - 1) & 1)));
             if (ok) {
                 tc_fence_after();
                 float v[16], u16[16];
@@ -1114,7 +1137,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 tmem_ld16(tmem_addr(tmem, warp, TP_W + 16 * qtr), v);
                 tmem_ld16(tmem_addr(tmem, warp, TP_U + 16 * qtr), u16);
                 tmem_wait_ld();
-                uint8_t *wq = sm + stb + RS_W + (r >> 6) * 8192 + (r & 7) * 2;
+                uint8_t *wq = sm + stb + ST_W + (r >> 6) * 8192 + (r & 7) * 2;
                 const uint32_t wc = (uint32_t)((r & 63) >> 3);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
@@ -1123,8 +1146,7 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                         __float2bfloat16_rn(-v[j]);
                 }
                 // U~^T row i = r, tokens t = 16 qtr + j -> U~[i][t] (64 contiguous bytes per thread)
-                float4 *ur = reinterpret_cast<float4 *>(ring + (size_t)(c % kRing) * RSLOT + RS_U +
-                                                        ((size_t)r * UT_LD + 16 * qtr) * 4);
+                float4 *ur = reinterpret_cast<float4 *>(rec + RS_U + ((size_t)r * UT_LD + 16 * qtr) * 4);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     ur[j] = make_float4(u16[4 * j], u16[4 * j + 1], u16[4 * j + 2], u16[4 * j + 3]);
@@ -1143,8 +1165,9 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 template <bool PRO, bool GT>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                    const __grid_constant__ CUtensorMap tm_z, const RingParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_vl,
+                    const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_z,
+                    const RingParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -1197,7 +1220,7 @@ prefill_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (rank == 0)
         chain_cta<GT>(&tm_q, &tm_k, &tm_o, &tm_z, p, sm, sb, tmem, wt, h, n, bos, eos, nwork, ring);
     else
-        prep_cta<PRO>(&tm_q, &tm_k, &tm_v, p, sm, sb, tmem, wt, h, bos, eos, nwork, rank, ring);
+        prep_cta<PRO>(&tm_q, &tm_k, &tm_v, &tm_vl, p, sm, sb, tmem, wt, h, bos, eos, nwork, rank, ring);
 
     tc_fence_before();
     __syncthreads();
@@ -1243,7 +1266,7 @@ cudaError_t launch_prefill_ring(const PrefillArgs &a, cudaStream_t stream) {
     unsigned int *status = static_cast<unsigned int *>(a.workspace);
     cudaError_t err = a.keep_status ? cudaSuccess : cudaMemsetAsync(status, 0, sizeof(unsigned int), stream);
     if (err != cudaSuccess) return err;
-    CUtensorMap tq, tk, tv, to;
+    CUtensorMap tq, tk, tv, tvl, to;
     const uint64_t tok = (uint64_t)(Ttot > 0 ? Ttot : 1);
     uint64_t dq[3] = {(uint64_t)DH, (uint64_t)a.HK, tok};
     uint64_t sq[2] = {(uint64_t)DH * 2, (uint64_t)a.HK * DH * 2};
@@ -1253,6 +1276,8 @@ cudaError_t launch_prefill_ring(const PrefillArgs &a, cudaStream_t stream) {
     if (!encode_bf16_map(&tq, a.q, 3, dq, sq, box) || !encode_bf16_map(&tk, a.k, 3, dq, sq, box) ||
         !encode_bf16_map(&tv, a.v, 3, dv, sv, box))
         return cudaErrorInvalidValue;
+    tvl = tv;
+    if (a.v_lo && !encode_bf16_map(&tvl, a.v_lo, 3, dv, sv, box)) return cudaErrorInvalidValue;
     // o: one output warp's 32 tokens x 32 value rows per store, unswizzled 64-byte rows
     uint32_t obox[3] = {32, 1, 32};
     if (!encode_bf16_map(&to, a.o, 3, dv, sv, obox, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -1268,7 +1293,8 @@ cudaError_t launch_prefill_ring(const PrefillArgs &a, cudaStream_t stream) {
     RingParams prm{a.g, a.beta, a.h0, a.cu_seqlens, a.T, a.HK, a.HV, a.scale,
                    static_cast<__nv_bfloat16 *>(a.o), a.hT, status,
                    static_cast<uint8_t *>(a.workspace) + kRingHeader,
-                   (int)((a.workspace_bytes - kRingHeader) / ((size_t)kRing * RSLOT)), a.prologue};
+                   (int)((a.workspace_bytes - kRingHeader) / ((size_t)kRing * RSLOT)), a.prologue,
+                   a.v_lo != nullptr};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(kClusterSize * a.HV), (unsigned)a.N, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1281,7 +1307,7 @@ cudaError_t launch_prefill_ring(const PrefillArgs &a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, tz, prm);
+    err = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tvl, to, tz, prm);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
