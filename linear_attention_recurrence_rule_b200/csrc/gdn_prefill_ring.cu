@@ -239,6 +239,56 @@ __device__ __forceinline__ void mul_lds16p(float2 (&v)[8], const float *src) {
         v[2 * q + 1] = mul2(v[2 * q + 1], make_float2(f.z, f.w));
     }
 }
+// ---- warp-level 16x8x8 TF32 products with fp32 accuracy (x = hi + lo, the three
+// products hi*hi + hi*lo + lo*hi), for the small block products of the UT inverse.
+// Fragments (lane = 4g + t): A 16x8 row-major {(g,t), (g+8,t), (g,t+4), (g+8,t+4)},
+// B 8x8 {(k=t, n=g), (k=t+4, n=g)}, D 16x8 {(g,2t), (g,2t+1), (g+8,2t), (g+8,2t+1)}.
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    hi = tf32_rna(x);
+    lo = tf32_rna(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// d += M[r0.., c0..] (16 x 8 of a row-major fp32 matrix, leading dimension ld) *
+//      N[k0.., n0..] (8 x 8), entries where keep_a(row, col) / keep_b(k, n) is false
+//      taken as zero
+template <typename KA, typename KB>
+__device__ __forceinline__ void mma3_smem(float (&d)[4], const float *M, int ld, int r0, int c0,
+                                          const float *N, int ldn, int k0, int n0, KA keep_a,
+                                          KB keep_b) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int ar[4] = {r0 + g, r0 + g + 8, r0 + g, r0 + g + 8};
+    const int ac[4] = {c0 + t, c0 + t, c0 + t + 4, c0 + t + 4};
+    uint32_t ah[4], al[4], bh[2], bl[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        split_tf32(keep_a(ar[i], ac[i]) ? M[ar[i] * ld + ac[i]] : 0.f, ah[i], al[i]);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int kk = k0 + t + 4 * i, nn = n0 + g;
+        split_tf32(keep_b(kk, nn) ? N[kk * ldn + nn] : 0.f, bh[i], bl[i]);
+    }
+    mma_tf32(d, ah, bh);
+    mma_tf32(d, ah, bl);
+    mma_tf32(d, al, bh);
+}
+// D fragment (times s) into a row-major fp32 matrix at (r0, c0)
+__device__ __forceinline__ void store_d(float *M, int ld, int r0, int c0, const float (&d)[4], float s) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2 *>(M + (r0 + g) * ld + c0 + 2 * t) = make_float2(s * d[0], s * d[1]);
+    *reinterpret_cast<float2 *>(M + (r0 + g + 8) * ld + c0 + 2 * t) = make_float2(s * d[2], s * d[3]);
+}
+
 __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
     uint32_t v;
     asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
@@ -1031,74 +1081,49 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 }
             }
             named_sync(NB_WORK, kPWorkThreads);
-            // ---- step 2: within each 32x32 half, T10 = -T11 A10 T00 (one entry per thread) ----
-            const int hf2 = pt >> 8, ii2 = (pt >> 4) & 15, j2 = pt & 15;
-            const int r1 = 32 * hf2 + 16, c0 = 32 * hf2;
-            if (ok) {
-                float a0 = 0.f;
+            // ---- step 2: within each 32x32 half h, T10 = -T11 (A10 T00) (16 x 16 blocks
+            //      at rows 32h + 16, columns 32h); worker warp 2h + j owns columns 8j..8j+7
+            //      of the block: Y = A10 T00 into the block's place in T, then -T11 Y over
+            //      it (the warp reads its columns of Y before writing them) ----
+            const int wi = warp - kPWork0;
+            const auto all = [](int, int) { return true; };
+            if (ok && wi < 4) {
+                const int hh = wi >> 1, nt = wi & 1, r1 = 32 * hh + 16, c0 = 32 * hh;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                // T00 is lower triangular: k-steps below the tile's first column vanish
+                for (int kk = nt; kk < 2; ++kk)
+                    mma3_smem(d, A_s, A_LD, r1, c0 + 8 * kk, T_s, T_LD, c0 + 8 * kk, c0 + 8 * nt, all, all);
+                store_d(T_s, T_LD, r1, c0 + 8 * nt, d, 1.f);
+                __syncwarp();
+                float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float t0 = (m >= j2) ? T_s[(c0 + m) * T_LD + c0 + j2] : 0.f;
-                    a0 = fmaf(A_s[(r1 + ii2) * A_LD + c0 + m], t0, a0);
-                }
-                X_s[(16 * hf2 + ii2) * X_LD + j2] = a0;
+                for (int kk = 0; kk < 2; ++kk)
+                    mma3_smem(e, T_s, T_LD, r1, r1 + 8 * kk, T_s, T_LD, r1 + 8 * kk, c0 + 8 * nt, all, all);
+                __syncwarp();
+                store_d(T_s, T_LD, r1, c0 + 8 * nt, e, -1.f);
             }
             named_sync(NB_WORK, kPWorkThreads);
-            if (ok) {
-                float a0 = 0.f;
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float tm = (m <= ii2) ? T_s[(r1 + ii2) * T_LD + r1 + m] : 0.f;
-                    a0 = fmaf(tm, X_s[(16 * hf2 + m) * X_LD + j2], a0);
-                }
-                T_s[(r1 + ii2) * T_LD + c0 + j2] = -a0;
+            // ---- step 3: T[32:64][0:32] = -T22 (A21 T11); worker warp w < 8 owns the 16 x 8
+            //      tile (rows 16 (w >> 2), columns 8 (w & 3)) of X = A21 T11, then of the
+            //      result.  The blocks above the diagonal that no step wrote (T11 rows
+            //      0..15 x columns 16..31, T22 rows 32..47 x columns 48..63) are masked:
+            //      T11[k][n] = 0 for k < n, T22[m][k] = 0 for k > m ----
+            if (ok && wi < 8) {
+                const int mt = wi >> 2, nt = wi & 3;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int kk = nt; kk < 4; ++kk)
+                    mma3_smem(d, A_s, A_LD, 32 + 16 * mt, 8 * kk, T_s, T_LD, 8 * kk, 8 * nt, all,
+                              [](int k, int n) { return k >= n; });
+                store_d(X_s, X_LD, 16 * mt, 8 * nt, d, 1.f);
             }
             named_sync(NB_WORK, kPWorkThreads);
-            // ---- step 3: T[32:64][0:32] = -T22 (A21 T11); lane j owns a column, warp w
-            //      two rows (warp-uniform, so the triangular bounds do not diverge):
-            //      2w and 2w + 1 for X = A21 T11, then w and 31 - w for the triangular
-            //      T22 X (equal work per warp); operands in groups of four ----
-            const int rw = 2 * (warp - kPWork0);
-            if (ok) {
-                // X = A21 T11 (T11[m][j] = 0 for m < j; its upper block was never written)
-                float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-                for (int m4 = 0; m4 < 32; m4 += 4) {
-                    const float4 a0 = *reinterpret_cast<const float4 *>(A_s + (32 + rw) * A_LD + m4);
-                    const float4 a1 = *reinterpret_cast<const float4 *>(A_s + (33 + rw) * A_LD + m4);
-                    const float aa0[4] = {a0.x, a0.y, a0.z, a0.w}, aa1[4] = {a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int m = m4 + e;
-                        const float tv = (m >= lane) ? T_s[m * T_LD + lane] : 0.f;
-                        x0 = fmaf(aa0[e], tv, x0);
-                        x1 = fmaf(aa1[e], tv, x1);
-                    }
-                }
-                X_s[rw * X_LD + lane] = x0;
-                X_s[(rw + 1) * X_LD + lane] = x1;
-            }
-            named_sync(NB_WORK, kPWorkThreads);
-            if (ok) {
-                // T21 = -T22 X (T22[ii][m] = 0 for m > ii: only m <= ii is read)
-                const int ra = warp - kPWork0, rb = 31 - ra;   // ra < 16 <= rb
-                float y0 = 0.f, y1 = 0.f;
-                for (int m4 = 0; m4 <= rb; m4 += 4) {
-                    const float4 t0 = *reinterpret_cast<const float4 *>(T_s + (32 + ra) * T_LD + 32 + m4);
-                    const float4 t1 = *reinterpret_cast<const float4 *>(T_s + (32 + rb) * T_LD + 32 + m4);
-                    const float tt0[4] = {t0.x, t0.y, t0.z, t0.w}, tt1[4] = {t1.x, t1.y, t1.z, t1.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int m = m4 + e;
-                        // rows of X past rb (none: rb <= 31) and entries of T22 above its
-                        // diagonal (never written) are not used
-                        const float xv = (m <= rb) ? X_s[m * X_LD + lane] : 0.f;
-                        y0 = fmaf(m <= ra ? tt0[e] : 0.f, xv, y0);
-                        y1 = fmaf(m <= rb ? tt1[e] : 0.f, xv, y1);
-                    }
-                }
-                T_s[(32 + ra) * T_LD + lane] = -y0;
-                T_s[(32 + rb) * T_LD + lane] = -y1;
+            if (ok && wi < 8) {
+                const int mt = wi >> 2, nt = wi & 3;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int kk = 0; kk <= 2 * mt + 1; ++kk)
+                    mma3_smem(d, T_s, T_LD, 32 + 16 * mt, 32 + 8 * kk, X_s, X_LD, 8 * kk, 8 * nt,
+                              [](int m, int k) { return k <= m; }, all);
+                store_d(T_s, T_LD, 32 + 16 * mt, 8 * nt, d, -1.f);
             }
             named_sync(NB_WORK, kPWorkThreads);
             // ---- T' = T diag(b gamma) (for W) and T'' = T diag(b) (for U~) as hi/lo
