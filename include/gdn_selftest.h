@@ -31,6 +31,35 @@ GDN_API int gdn_selftest_umma(const void *X, const void *Y, const void *Z, const
                               float *D1, float *D2, float *D3, float *D4, float *D5,
                               int *status, gdn_stream_t stream);
 
+/*
+ * Test-only instance of the tensor-core prefill (bf16, dk = dv = 128, chunk 64;
+ * same layouts as gdn_chunk_prefill, h0 = 0, scale 1) whose first on-device
+ * wait -- before any load, copy or MMA is issued -- has a limit of zero polls
+ * on a barrier that nothing arrives on.  It exercises the library's timeout
+ * path without a real hang: the wait gives up, the status word in `workspace`
+ * becomes GDN_ERR_TIMEOUT (read it with gdn_read_status), every CTA of each
+ * cluster winds down without work, and the kernel returns.  o and hT are then
+ * undefined.  workspace: gdn_chunk_prefill_workspace_size(...) bytes.  Returns
+ * GDN_OK once enqueued, GDN_ERR_INVALID_ARG / GDN_ERR_WORKSPACE / GDN_ERR_CUDA.
+ */
+GDN_API int gdn_selftest_prefill_timeout(const void *q, const void *k, const void *v,
+                                         const float *g, const float *beta, int N, int64_t T,
+                                         int HK, int HV, void *o, float *hT, void *workspace,
+                                         size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * Test-only instance of the update-vector verify's streaming kernel (dk = dv = 128,
+ * K <= 4 drafts, bf16 v/o): its first on-device wait, before any copy is issued,
+ * has a limit of zero polls on a barrier nothing arrives on, so the kernel records
+ * a timeout in the workspace status word (gdn_read_status then returns
+ * GDN_ERR_TIMEOUT) and returns with nothing in flight.  v [N][K][HV][128] bf16,
+ * state [N][HV][128][128] fp32 (only read), o, u_out as gdn_recurrent_verify (left
+ * unwritten); workspace: gdn_recurrent_verify_workspace_size(N, K, HV, 128) bytes.
+ */
+GDN_API int gdn_selftest_verify_timeout(const void *v, const float *state, int N, int K, int HV,
+                                        void *o, float *u_out, void *workspace,
+                                        size_t workspace_bytes, gdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

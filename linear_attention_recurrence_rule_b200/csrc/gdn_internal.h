@@ -76,6 +76,8 @@ size_t verify_workspace_floats(int N, int K, int HV, int dk, int prev_K = 0);
 bool decode_supported(int dk, int dv);
 cudaError_t launch_decode(const StepArgs &a, cudaStream_t stream);
 cudaError_t launch_verify(const VerifyArgs &a, cudaStream_t stream);
+// test-only: the update-vector verify's streaming kernel with a first wait that gives up
+cudaError_t launch_verify_wy_timeout_test(const VerifyArgs &a, cudaStream_t stream);
 
 // Largest draft count of the verify kernels (GDN_VERIFY_MAX_DRAFTS in gdn.h).
 constexpr int kVerifyMaxDrafts = 16;
@@ -133,7 +135,8 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t stream);
 bool prefill_ring_supported(int dk, int dv, int chunk, gdn_dtype dtype);
 // device workspace: the status word and one ring of chunk records per SM id
 size_t prefill_ring_workspace(int N, int64_t T, int HV, int chunk, bool varlen);
-cudaError_t launch_prefill_ring(const PrefillArgs &a, cudaStream_t stream);
+// timeout_test: the test-only instance whose first on-device wait gives up at once
+cudaError_t launch_prefill_ring(const PrefillArgs &a, cudaStream_t stream, bool timeout_test = false);
 
 // validation, workspace check and dispatch of one prefill call (gdn_api.cu)
 gdn_status enqueue_prefill(const PrefillArgs &a, cudaStream_t stream);

@@ -1187,7 +1187,11 @@ __device__ void prep_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     }
 }
 
-template <bool PRO, bool GT>
+// TMO: a test-only instance whose first wait -- before any load, copy or MMA is
+// issued -- has a limit of zero polls on a barrier nothing arrives on, so the
+// timeout path (status word, abort flags in every CTA, every loop running its
+// iterations without work, the drains) runs without a real hang.
+template <bool PRO, bool GT, bool TMO = false>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_vl,
@@ -1236,11 +1240,17 @@ prefill_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t tmem = *tslot;
     cluster_sync_all();   // every CTA's barriers are initialised before any remote traffic
 
+    if (TMO) {
+        // the drain barrier completes only at teardown: a zero-limit wait on it gives up
+        if (rank == 0 && tid == 0 && !mbar_test_wait(&bars[CB_DRAIN], 0u)) wt.abort_all();
+        cluster_sync_all();   // every CTA sees the abort flags before any work starts
+    }
     const int ring_id = (int)ld_cluster_u32(mapa_shared(sb + AUX_RING, 0));
     const bool ring_ok = ring_id >= 0 && ring_id < p.nrings;
     if (!ring_ok && rank == 0 && tid == 0) atomicExch(p.status, (unsigned int)GDN_ERR_CUDA);
     uint8_t *ring = p.rings + (size_t)(ring_ok ? ring_id : 0) * kRing * RSLOT;
-    const int nwork = ring_ok ? nchunks : 0;
+    // after an abort (only the test instance can have one here) no work is issued
+    const int nwork = (ring_ok && !(TMO && *abort_flag)) ? nchunks : 0;
 
     if (rank == 0)
         chain_cta<GT>(&tm_q, &tm_k, &tm_o, &tm_z, p, sm, sb, tmem, wt, h, n, bos, eos, nwork, ring);
@@ -1284,7 +1294,7 @@ size_t prefill_ring_workspace(int, int64_t, int, int, bool) {
     return kRingHeader + nrings * kRing * RSLOT;
 }
 
-cudaError_t launch_prefill_ring(const PrefillArgs &a, cudaStream_t stream) {
+cudaError_t launch_prefill_ring(const PrefillArgs &a, cudaStream_t stream, bool timeout_test) {
     const int64_t Ttot = a.cu_seqlens ? a.T : (int64_t)a.N * a.T;
     if (Ttot >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     if (a.workspace_bytes < kRingHeader + (size_t)kRing * RSLOT) return cudaErrorInvalidValue;
@@ -1313,6 +1323,7 @@ cudaError_t launch_prefill_ring(const PrefillArgs &a, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     auto kern = a.gate ? (a.prologue ? prefill_ring_kernel<true, true> : prefill_ring_kernel<false, true>)
                        : (a.prologue ? prefill_ring_kernel<true, false> : prefill_ring_kernel<false, false>);
+    if (timeout_test) kern = prefill_ring_kernel<false, false, true>;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     RingParams prm{a.g, a.beta, a.h0, a.cu_seqlens, a.T, a.HK, a.HV, a.scale,

@@ -14,6 +14,7 @@
 #include <cuda.h>
 
 #include "gdn.h"
+#include "gdn_internal.h"
 #include "gdn_selftest.h"
 #include "tc_primitives.cuh"
 #include "tma_host.h"
@@ -213,4 +214,33 @@ extern "C" int gdn_selftest_umma(const void *X, const void *Y, const void *Z, co
         static_cast<const __nv_bfloat16 *>(S), static_cast<const __nv_bfloat16 *>(W), D0, D1, D2,
         D3, D4, D5, status);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// Test-only tensor-core prefill whose first on-device wait gives up at once (see
+// gdn_selftest.h): the library's timeout path, exercised without a real hang.
+extern "C" int gdn_selftest_prefill_timeout(const void *q, const void *k, const void *v,
+                                            const float *g, const float *beta, int N, int64_t T,
+                                            int HK, int HV, void *o, float *hT, void *workspace,
+                                            size_t workspace_bytes, gdn_stream_t stream) {
+    if (!q || !k || !v || !g || !beta || !o || !workspace) return GDN_ERR_INVALID_ARG;
+    if (N <= 0 || T <= 0 || HK <= 0 || HV <= 0 || HV % HK) return GDN_ERR_INVALID_ARG;
+    gdn::PrefillArgs a{q, k, v, g, beta, nullptr, nullptr, N, T, HK, HV, 128, 128, 64,
+                       1.0f, GDN_BF16, o, hT, workspace, workspace_bytes};
+    if (workspace_bytes < gdn::prefill_workspace_bytes(a)) return GDN_ERR_WORKSPACE;
+    const cudaError_t err = gdn::launch_prefill_ring(a, reinterpret_cast<cudaStream_t>(stream), true);
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// Test-only update-vector verify streaming kernel whose first wait gives up at once
+// (see gdn_selftest.h).
+extern "C" int gdn_selftest_verify_timeout(const void *v, const float *state, int N, int K, int HV,
+                                           void *o, float *u_out, void *workspace,
+                                           size_t workspace_bytes, gdn_stream_t stream) {
+    if (!v || !state || !o || !workspace) return GDN_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || K > 4 || HV <= 0) return GDN_ERR_INVALID_ARG;
+    if (workspace_bytes < gdn_recurrent_verify_workspace_size(N, K, HV, 128)) return GDN_ERR_WORKSPACE;
+    gdn::VerifyArgs a{nullptr, nullptr, v, nullptr, nullptr, state, nullptr, u_out, N, K, 1, HV, 128, 128,
+                      1.0f, GDN_BF16, o, 0u, workspace, workspace_bytes};
+    const cudaError_t err = gdn::launch_verify_wy_timeout_test(a, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

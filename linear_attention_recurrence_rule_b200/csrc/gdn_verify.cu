@@ -418,7 +418,10 @@ __host__ __device__ constexpr size_t wy_smem_bytes() {
            wy_stages<KT, FUSED>() * sizeof(uint64_t) + 16;
 }
 
-template <int DK, int KT, typename Tin, bool FUSED>
+// TMO: a test-only instance whose first wait -- before thread 0 issues any copy --
+// has a limit of zero polls on a stage barrier nothing has armed: the timeout path
+// (status word, early return with nothing in flight) runs without a real hang.
+template <int DK, int KT, typename Tin, bool FUSED, bool TMO = false>
 __global__ void __launch_bounds__(kVerifyWarps * 32, KT <= 8 ? 2 : 1)
 verify_wy_kernel(const Tin *__restrict__ v, float *state, float *__restrict__ ws,
                  float *__restrict__ u_out, Tin *__restrict__ o, int N, int K, int HV, int dv,
@@ -516,9 +519,23 @@ verify_wy_kernel(const Tin *__restrict__ v, float *state, float *__restrict__ ws
             }
         }
     };
+    if (TMO) {
+        int gave_up = 0;
+        if (tid == 0) {
+            for (int st = 0; st < NST; ++st) tc::mbar_init(&bars[st], 1);
+            tc::fence_barrier_init();
+            if (!tc::mbar_test_wait(&bars[0], 0u)) {
+                atomicExch(reinterpret_cast<unsigned int *>(ws), 1u);
+                gave_up = 1;
+            }
+        }
+        if (__syncthreads_or(gave_up)) return;
+    }
     if (tid == 0) {
-        for (int st = 0; st < NST; ++st) tc::mbar_init(&bars[st], 1);
-        tc::fence_barrier_init();
+        if (!TMO) {
+            for (int st = 0; st < NST; ++st) tc::mbar_init(&bars[st], 1);
+            tc::fence_barrier_init();
+        }
         for (long long i = 0; i < NST && i < mine; ++i) issue(i);
     }
     if (mine > 0) {
@@ -951,6 +968,24 @@ cudaError_t launch_commit(const float *states, const int32_t *accepted, float *s
     const unsigned ys = (unsigned)((elems / 4 + 2047) / 2048);
     commit_kernel<<<dim3((unsigned)((size_t)N * HV), ys), 256, 0, stream>>>(states, accepted, state,
                                                                           K, HV, elems);
+    return cudaGetLastError();
+}
+
+// Test-only: the update-vector streaming kernel (d = 128, up to 4 drafts, bf16) whose
+// first wait gives up at once; the workspace status word reads nonzero afterwards.
+cudaError_t launch_verify_wy_timeout_test(const VerifyArgs &a, cudaStream_t stream) {
+    auto kern = verify_wy_kernel<128, 4, __nv_bfloat16, false, true>;
+    constexpr size_t smem = wy_smem_bytes<128, 4, false>();
+    cudaError_t e = cudaMemsetAsync(a.workspace, 0, sizeof(unsigned int), stream);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long bands = (long long)a.N * a.HV * ((a.dv + verify_band<128>() - 1) / verify_band<128>());
+    const unsigned grid = (unsigned)(bands < device_sm_count() ? bands : device_sm_count());
+    kern<<<grid, kVerifyWarps * 32, smem, stream>>>(
+        static_cast<const __nv_bfloat16 *>(a.v), const_cast<float *>(a.state),
+        static_cast<float *>(a.workspace), a.u, static_cast<__nv_bfloat16 *>(a.o), a.N, a.K, a.HV,
+        a.dv, nullptr, 0);
     return cudaGetLastError();
 }
 

@@ -442,9 +442,13 @@ def gdn_chunk_prefill_path(dk, dv, chunk, dtype) -> int:
 
 
 def gdn_read_status(workspace, stream=None) -> int:
-    """Status word of the last prefill on ``workspace`` (synchronises the stream)."""
+    """Status word of the last prefill on ``workspace`` (synchronises the stream).
+    ``None``: the word in the library array the workspace-free prefill uses on the
+    current device."""
     if workspace is None:
-        return GDN_OK
+        import torch
+        dev = torch.device("cuda", torch.cuda.current_device())
+        return int(load_library().gdn_read_status(None, 0, _stream_ptr(stream, dev)))
     return int(load_library().gdn_read_status(
         _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream_ptr(stream, workspace.device)))

@@ -54,5 +54,7 @@ def test_noalloc_matches_workspace_entry_point(dtype, d, chunk):
                _ptr(o), _ptr(hT), stream)
         assert rc == gdn.GDN_OK, gdn.status_string(rc)
         torch.cuda.synchronize()
+        # every on-device wait of the call completed (the status word in the library array)
+        assert gdn.gdn_read_status(None) == gdn.GDN_OK
         assert_close(o, o_ref64, dtype, f"o, call {call}")
         assert_close(hT, h_ref64, dtype, f"hT, call {call}")
