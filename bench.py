@@ -14,7 +14,7 @@ prefix) in the ``verify`` object, the fused input prologue and one decay per
 value row in the ``prologue`` object, and the layer steps around the rule (the
 short convolution on the values and the output gate, in the prefill and in
 the decode step) in the ``layer`` object.  ``--no-decode``, ``--no-verify``,
-``--no-prologue``, ``--no-layer``, ``--no-e2e`` and ``--no-cpu-baseline`` skip
+``--no-prologue``, ``--no-layer``, ``--no-configs``, ``--no-e2e`` and ``--no-cpu-baseline`` skip
 the respective legs.
 
 Launch: ``python bench.py [--gpus N --steps K --warmup W]``; for N > 1 under
@@ -640,6 +640,66 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def measure_configs(gdn, torch, dev, stream, peaks, peak_src, rank, args):
+    """The other prefill workloads of the suite, each timed on its own (one call per
+    step, CUDA events on the launching stream, 3 warm-up calls): tokens/s and the
+    fraction of the roofline that bounds its path -- the bf16 tensor peak for the
+    tensor-core path, the fp32 FMA peak (148 SMs x 128 FMA x 2 x max clock) for the
+    CUDA-core path.  A step is one launch of ours plus the status-word reset."""
+    from linear_attention_recurrence_rule_b200.inputs import WORKLOADS, workload_inputs
+    out = {}
+    for name in ("layer_prefill_4k", "varlen_8", "tiny_fp32"):
+        w = WORKLOADS[name]
+        x = workload_inputs(name, seed_offset=replica_seed_offset(rank))
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+        cu = d["cu_seqlens"]
+        B, T = d["q"].shape[0], d["q"].shape[1]
+        N = (cu.numel() - 1) if cu is not None else B
+        tokens = B * T
+        ws_b = gdn.gdn_chunk_prefill_workspace_size(N, T if cu is not None else T, w.HK, w.HV, w.dk,
+                                                    w.dv, w.chunk, w.dtype, cu is not None)
+        ws = torch.empty(max(ws_b, 1), dtype=torch.uint8, device=dev) if ws_b else None
+        o = torch.empty_like(d["v"])
+        hT = torch.empty((N, w.HV, w.dv, w.dk), dtype=torch.float32, device=dev)
+
+        def call():
+            gdn.gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
+                                  cu_seqlens=cu, chunk=w.chunk, o=o, hT=hT, workspace=ws,
+                                  stream=stream)
+
+        reps = 10
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        for a_, b_ in evs:
+            a_.record(stream)
+            call()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.median(a_.elapsed_time(b_) for a_, b_ in evs)
+        flops = prefill_flops_per_token(w.HK, w.HV, w.dk, w.chunk) * tokens
+        tc = gdn.gdn_chunk_prefill_path(w.dk, w.dv, w.chunk, w.dtype) == 1
+        if tc:
+            peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+            bound = "tensor"
+        else:
+            mhz = peaks.get("sm_max_mhz", FALLBACK_PEAKS["sm_max_mhz"])
+            peak = N_SM * FP32_FMA_PER_SM_PER_CLK * 2 * mhz * 1e6 / 1e12
+            bound = "alu"
+        achieved = flops / (ms / 1e3) / 1e12
+        out[name] = {"value": tokens / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+                     "tokens": tokens, "sequences": N, "path": "tcgen05" if tc else "cuda-core",
+                     "dtype": "bf16" if w.dtype == torch.bfloat16 else "fp32",
+                     "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
+                                  "unit": "TFLOP/s", "frac": achieved / peak,
+                                  "peak_source": peak_src if tc else "derived (unit counts x max clock)"},
+                     "gpu_launches_per_step": 1,
+                     "h0": "nonzero" if x["h0"] is not None else "zero"}
+    return out
+
+
 def run_b200(args):
     import torch
     import torch.distributed as dist
@@ -718,7 +778,7 @@ def run_b200(args):
         peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": flops / mean_launch_s / 1e12, "peak": peak,
                 "unit": "TFLOP/s"}
-        kernel_key = "prefill_cluster"
+        kernel_key = "prefill_ring"
     else:
         mhz = peaks.get("sm_max_mhz", FALLBACK_PEAKS["sm_max_mhz"])
         peak = N_SM * FP32_FMA_PER_SM_PER_CLK * 2 * mhz * 1e6 / 1e12
@@ -766,8 +826,37 @@ def run_b200(args):
         torch.cuda.synchronize()
         barrier()
         e_ms = max_over_ranks(a.elapsed_time(b))
+        # what the copies alone cost on this machine: the step's inputs host -> device and
+        # its outputs device -> host as plain pinned copies on one stream
+        dbuf = {n: torch.empty(host_in[n].shape, dtype=host_in[n].dtype, device=dev) for n in names}
+        dout = torch.empty(o.shape, dtype=o.dtype, device=dev)
+
+        def timed(fn, reps=3):
+            fn()
+            torch.cuda.synchronize()
+            a_ = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            for _ in range(reps):
+                fn()
+            b_.record(stream)
+            torch.cuda.synchronize()
+            return a_.elapsed_time(b_) / reps
+
+        h2d_ms = timed(lambda: [dbuf[n].copy_(host_in[n], non_blocking=True) for n in names])
+        d2h_ms = timed(lambda: (host_o.copy_(dout, non_blocking=True),
+                                host_h.copy_(hT, non_blocking=True)))
+        serial_ms = h2d_ms + mean_launch_s * 1e3 + d2h_ms
+        step_ms = e_ms / e_steps
         e2e = {"value": world * tokens * e_steps / (e_ms / 1000.0), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
+               "ms_per_step": step_ms, "segments": -(-T // 4096), "segment_tokens": 4096,
+               "h2d_gbs": h2d / (h2d_ms / 1e3) / 1e9, "d2h_gbs": d2h / (d2h_ms / 1e3) / 1e9,
+               "copies_alone_ms": h2d_ms + d2h_ms, "kernel_alone_ms": mean_launch_s * 1e3,
+               "serial_ms": serial_ms,
+               "overlap": (serial_ms - step_ms) / min(h2d_ms + d2h_ms, mean_launch_s * 1e3),
+               "note": "overlap: the part of the smaller of (copies, kernel) hidden behind the "
+                       "other; the step is bound by the host-to-device copy rate"}
 
     # ---- decode: 256 sequences x 64 single-token steps ----
     dec = None
@@ -825,6 +914,10 @@ def run_b200(args):
         lay = measure_layer(gdn, torch, dev, stream, x, w, o, hT, rank, peaks, peak_src,
                             mean_launch_s, args)
 
+    cfgs = None
+    if not args.no_configs:
+        cfgs = measure_configs(gdn, torch, dev, stream, peaks, peak_src, rank, args)
+
     ver = None
     if not args.no_verify:
         ver = measure_verify(gdn, torch, dev, stream, peaks, peak_src, rank, world,
@@ -848,7 +941,7 @@ def run_b200(args):
                        "l2": "inputs larger than L2 (q,k,v 1.07 GB per step)"},
             "roofline": roof, "cpu_baseline": base, "e2e": e2e,
             "gpu_launches": launches_per_step * n_steps, "clocks": clocks, "decode": dec,
-            "verify": ver, "prologue": pro, "layer": lay,
+            "verify": ver, "prologue": pro, "layer": lay, "configs": cfgs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -869,6 +962,7 @@ def main():
     ap.add_argument("--no-verify", action="store_true")
     ap.add_argument("--no-prologue", action="store_true")
     ap.add_argument("--no-layer", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--verify-rounds", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="decode measurement only")

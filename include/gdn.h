@@ -264,8 +264,9 @@ GDN_API size_t gdn_chunk_prefill_host_workspace_size(int N, int64_t T, int HK, i
  *                        the price of overlap).  The call orders itself after work
  *                        already queued on `stream`, and every copy and kernel it
  *                        enqueues completes before later work on `stream`.
- * It creates and destroys 3 * ceil(T / segment) + 1 CUDA events (released by the
- * runtime once they complete), does not synchronise, and allocates no memory.
+ * It creates and destroys 7 CUDA events per call, whatever the number of
+ * segments (released by the runtime once they complete), does not synchronise,
+ * and allocates no memory.
  * Errors as gdn_chunk_prefill; GDN_ERR_CUDA if an enqueue fails part way (the
  * work already enqueued then still runs).
  */

@@ -3,7 +3,6 @@
 // global state; every launch goes to the caller's stream.
 #include <cuda_runtime.h>
 
-#include <new>
 
 #include "gdn.h"
 #include "gdn_internal.h"
@@ -199,12 +198,13 @@ gdn_status gdn_chunk_prefill_host(const void *q, const void *k, const void *v, c
     cudaStream_t so = reinterpret_cast<cudaStream_t>(copy_out);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const int64_t S = plan.seg, nseg = (T + S - 1) / S;
-    // the events that order the three streams; destroyed below once enqueued (the
-    // runtime keeps each alive until it has completed)
-    const int nev = (int)(3 * nseg + 1);
-    cudaEvent_t evs_local[64];
-    cudaEvent_t *evs = nev <= 64 ? evs_local : new (std::nothrow) cudaEvent_t[nev];
-    if (!evs) return GDN_ERR_CUDA;
+    // the events that order the three streams, two of each kind (by segment parity):
+    // a stream wait takes the event's latest record when it is enqueued, and the record
+    // of segment s is the latest one of its pair until segment s + 2 records it again,
+    // after that segment's waits on it are enqueued.  Destroyed below once enqueued
+    // (the runtime keeps each alive until it has completed).
+    constexpr int nev = 7;
+    cudaEvent_t evs[nev];
     int made = 0;
     gdn_status result = GDN_OK;
     for (; made < nev; ++made)
@@ -212,9 +212,9 @@ gdn_status gdn_chunk_prefill_host(const void *q, const void *k, const void *v, c
             result = GDN_ERR_CUDA;
             break;
         }
-    auto ev_in = [&](int64_t s) { return evs[1 + 3 * s]; };
-    auto ev_done = [&](int64_t s) { return evs[2 + 3 * s]; };
-    auto ev_out = [&](int64_t s) { return evs[3 + 3 * s]; };
+    auto ev_in = [&](int64_t s) { return evs[1 + 3 * (s & 1)]; };
+    auto ev_done = [&](int64_t s) { return evs[2 + 3 * (s & 1)]; };
+    auto ev_out = [&](int64_t s) { return evs[3 + 3 * (s & 1)]; };
     auto ok = [&](cudaError_t e) {
         if (e != cudaSuccess && result == GDN_OK) result = GDN_ERR_CUDA;
         return result == GDN_OK;
@@ -269,7 +269,6 @@ gdn_status gdn_chunk_prefill_host(const void *q, const void *k, const void *v, c
     // everything the call enqueued is ordered before later work on the compute stream
     if (result == GDN_OK) ok(cudaStreamWaitEvent(sc, ev_out(nseg - 1), 0));
     for (int i = 0; i < made; ++i) cudaEventDestroy(evs[i]);
-    if (evs != evs_local) delete[] evs;
     return result;
 }
 
