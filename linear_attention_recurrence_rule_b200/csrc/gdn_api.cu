@@ -52,8 +52,11 @@ gdn_status enqueue_prefill(const PrefillArgs &a, cudaStream_t stream) {
     if (st != GDN_OK) return st;
     if (a.N == 0) return GDN_OK;
     cudaError_t err;
-    // one decay per value row: only the CUDA-core path (a per-row triangular inverse)
-    if (tc_path(a.dk, a.dv, a.chunk, a.dtype) && !(a.prologue & GDN_ROW_DECAY)) {
+    // one decay per value row: the row-recurrent CUDA-core kernel (the rows of the
+    // state never mix under that rule)
+    if (a.prologue & GDN_ROW_DECAY) {
+        err = launch_prefill_rows(a, stream);
+    } else if (tc_path(a.dk, a.dv, a.chunk, a.dtype)) {
         const size_t need = prefill_workspace_bytes(a);
         if (need > 0 && (a.workspace == nullptr || a.workspace_bytes < need)) return GDN_ERR_WORKSPACE;
         if (!aligned16(a.workspace)) return GDN_ERR_ALIGNMENT;

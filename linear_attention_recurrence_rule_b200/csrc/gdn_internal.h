@@ -122,6 +122,11 @@ cudaError_t launch_gate_factor(const void *z, void *factors, int64_t elems, gdn_
 bool prefill_simt_supported(int dk, int dv, int chunk);
 cudaError_t launch_prefill_simt(const PrefillArgs &a, cudaStream_t stream);
 
+// one decay per value row (GDN_ROW_DECAY): the recurrence token by token, one lane
+// group per state row (gdn_prefill_rows.cu)
+bool prefill_rows_supported(int dk, int dv);
+cudaError_t launch_prefill_rows(const PrefillArgs &a, cudaStream_t stream);
+
 
 // cluster (1 chain CTA + 3 prep CTAs per value head) tensor-core prefill
 // (gdn_prefill_cluster.cu)

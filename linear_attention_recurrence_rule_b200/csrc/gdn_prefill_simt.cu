@@ -31,7 +31,7 @@ namespace {
 
 constexpr int kSimtThreads = 256;
 
-template <int DK, int BV, int C, bool RD>
+template <int DK, int BV, int C>
 struct SimtSmem {
     static constexpr int KP = DK + 1;  // padded rows: conflict-free column walks
     static constexpr int CP = C + 1;
@@ -39,15 +39,11 @@ struct SimtSmem {
                                      + (size_t)BV * KP    // S rows
                                      + 2 * (size_t)C * CP // A, P
                                      + 3 * (size_t)C * BV // Y/U, K S^T, Q S^T
-                                     + 2 * (size_t)C      // G, beta
-                                     + (RD ? (size_t)C * BV : 0);   // per-row G (row decay)
+                                     + 2 * (size_t)C;     // G, beta
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
-// RD: one decay per value row (GDN_ROW_DECAY, g [..][HV][dv]): the decay factors
-// become per row, so A and P hold the undecayed products and exp(G_i - G_j) is
-// formed per row where they are used; G is a [C][BV] table of per-row running sums.
-template <typename Tin, int DK, int BV, int C, bool RD>
+template <typename Tin, int DK, int BV, int C>
 __global__ void __launch_bounds__(kSimtThreads)
 prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const Tin *__restrict__ v, const float *__restrict__ g,
@@ -55,7 +51,7 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const int32_t *__restrict__ cu, int64_t T, int HK, int HV, int dv,
                     float scale, Tin *__restrict__ o, float *__restrict__ hT, unsigned pro,
                     const void *__restrict__ gate) {
-    using L_ = SimtSmem<DK, BV, C, RD>;
+    using L_ = SimtSmem<DK, BV, C>;
     constexpr int KP = L_::KP, CP = L_::CP, NT = kSimtThreads;
     const int tid = threadIdx.x;
     const int e0 = blockIdx.x * BV;
@@ -82,7 +78,6 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     float *QSs = KSs + C * BV;
     float *Gs = QSs + C * BV;
     float *Bs = Gs + C;
-    float *Gr = Bs + C;   // [C][BV], row decay only
 
     const size_t state_base = ((size_t)n * HV + h) * (size_t)dv * DK;
     for (int idx = tid; idx < BV * DK; idx += NT) {
@@ -113,27 +108,14 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         if (tid < C) {
             // with gate logits: g = log sigmoid(a), beta = sigmoid(b); padding stays 0
             const bool logits = (pro & GDN_PROLOGUE_GATE_LOGITS) != 0;
-            const float gv = (!RD && tid < L) ? g[(s0 + tid) * HV + h] : 0.f;
+            const float gv = tid < L ? g[(s0 + tid) * HV + h] : 0.f;
             const float bv = tid < L ? beta[(s0 + tid) * HV + h] : 0.f;
             Gs[tid] = (logits && tid < L) ? gate_log_sigmoid(gv) : gv;
             Bs[tid] = (logits && tid < L) ? gate_sigmoid(bv) : bv;
         }
-        if (RD) {
-            const bool logits = (pro & GDN_PROLOGUE_GATE_LOGITS) != 0;
-            for (int idx = tid; idx < C * BV; idx += NT) {
-                const int i = idx / BV, e = idx - i * BV;
-                const float gv = i < L ? g[((size_t)(s0 + i) * HV + h) * dv + e0 + e] : 0.f;
-                Gr[idx] = (logits && i < L) ? gate_log_sigmoid(gv) : gv;
-            }
-        }
         __syncthreads();
         // ---- chunk-local running sum of the log decay ----
-        if (RD) {
-            for (int e = tid; e < BV; e += NT) {
-                float run = 0.f;
-                for (int i = 0; i < L; ++i) { run += Gr[i * BV + e]; Gr[i * BV + e] = run; }
-            }
-        } else if (tid == 0) {
+        if (tid == 0) {
             float run = 0.f;
             for (int i = 0; i < L; ++i) { run += Gs[i]; Gs[i] = run; }
         }
@@ -162,7 +144,7 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     kk = fmaf(Ks[i * KP + a], kj, kk);
                     qk = fmaf(Qs[i * KP + a], kj, qk);
                 }
-                const float gam = RD ? 1.f : expf(Gs[i] - Gs[j]);
+                const float gam = expf(Gs[i] - Gs[j]);
                 if (j < i) av = Bs[i] * gam * kk;
                 pv = gam * qk;
             }
@@ -188,21 +170,14 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         // ---- Y_i = b_i (v_i - gamma_i S0 k_i) ----
         for (int idx = tid; idx < C * BV; idx += NT) {
             const int i = idx / BV;
-            const float gi = RD ? Gr[idx] : Gs[i];
-            Ys[idx] = i < L ? Bs[i] * (Ys[idx] - expf(gi) * KSs[idx]) : 0.f;
+            Ys[idx] = i < L ? Bs[i] * (Ys[idx] - expf(Gs[i]) * KSs[idx]) : 0.f;
         }
         __syncthreads();
         // ---- forward substitution: U_i = Y_i - sum_{j<i} A_ij U_j ----
         for (int i = 1; i < L; ++i) {
             for (int e = tid; e < BV; e += NT) {
                 float acc = Ys[i * BV + e];
-                if (RD) {
-                    const float gi = Gr[i * BV + e];
-                    for (int j = 0; j < i; ++j)
-                        acc = fmaf(-As[i * CP + j] * expf(gi - Gr[j * BV + e]), Ys[j * BV + e], acc);
-                } else {
-                    for (int j = 0; j < i; ++j) acc = fmaf(-As[i * CP + j], Ys[j * BV + e], acc);
-                }
+                for (int j = 0; j < i; ++j) acc = fmaf(-As[i * CP + j], Ys[j * BV + e], acc);
                 Ys[i * BV + e] = acc;
             }
             __syncthreads();
@@ -211,15 +186,8 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         for (int idx = tid; idx < L * BV; idx += NT) {
             const int i = idx / BV, e = idx - i * BV;
             float acc = 0.f;
-            if (RD) {
-                const float gi = Gr[i * BV + e];
-                for (int j = 0; j <= i; ++j)
-                    acc = fmaf(Ps[i * CP + j] * expf(gi - Gr[j * BV + e]), Ys[j * BV + e], acc);
-                acc = fmaf(expf(gi), QSs[idx], acc);
-            } else {
-                for (int j = 0; j <= i; ++j) acc = fmaf(Ps[i * CP + j], Ys[j * BV + e], acc);
-                acc = fmaf(expf(Gs[i]), QSs[idx], acc);
-            }
+            for (int j = 0; j <= i; ++j) acc = fmaf(Ps[i * CP + j], Ys[j * BV + e], acc);
+            acc = fmaf(expf(Gs[i]), QSs[idx], acc);
             const size_t oi = ((size_t)(s0 + i) * HV + h) * dv + e0 + e;
             float out = scale * acc;
             if (gate)   // output gate, before the one rounding: fp32 factors for fp32, else fp16
@@ -232,13 +200,13 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         const float GL = Gs[L - 1];
         for (int idx = tid; idx < L * BV; idx += NT) {
             const int j = idx / BV, e = idx - j * BV;
-            Ys[idx] *= RD ? expf(Gr[(L - 1) * BV + e] - Gr[idx]) : expf(GL - Gs[j]);
+            Ys[idx] *= expf(GL - Gs[j]);
         }
         __syncthreads();
         const float gL = expf(GL);
         for (int idx = tid; idx < BV * DK; idx += NT) {
             const int e = idx / DK, a = idx - e * DK;
-            float acc = (RD ? expf(Gr[(L - 1) * BV + e]) : gL) * Ss[e * KP + a];
+            float acc = gL * Ss[e * KP + a];
             for (int j = 0; j < L; ++j) acc = fmaf(Ys[j * BV + e], Ks[j * KP + a], acc);
             Ss[e * KP + a] = acc;
         }
@@ -252,10 +220,10 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     }
 }
 
-template <typename Tin, int DK, int BV, int C, bool RD>
-cudaError_t launch_shape_rd(const PrefillArgs &a, cudaStream_t stream) {
-    constexpr size_t smem = SimtSmem<DK, BV, C, RD>::bytes;
-    auto kern = prefill_simt_kernel<Tin, DK, BV, C, RD>;
+template <typename Tin, int DK, int BV, int C>
+cudaError_t launch_shape(const PrefillArgs &a, cudaStream_t stream) {
+    constexpr size_t smem = SimtSmem<DK, BV, C>::bytes;
+    auto kern = prefill_simt_kernel<Tin, DK, BV, C>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
@@ -265,12 +233,6 @@ cudaError_t launch_shape_rd(const PrefillArgs &a, cudaStream_t stream) {
         static_cast<const Tin *>(a.v), a.g, a.beta, a.h0, a.cu_seqlens, a.T, a.HK, a.HV, a.dv,
         a.scale, static_cast<Tin *>(a.o), a.hT, a.prologue, a.gate);
     return cudaGetLastError();
-}
-
-template <typename Tin, int DK, int BV, int C>
-cudaError_t launch_shape(const PrefillArgs &a, cudaStream_t stream) {
-    return (a.prologue & GDN_ROW_DECAY) ? launch_shape_rd<Tin, DK, BV, C, true>(a, stream)
-                                        : launch_shape_rd<Tin, DK, BV, C, false>(a, stream);
 }
 
 template <typename Tin, int DK>

@@ -79,10 +79,13 @@ def test_verify_and_commits_row_decay(N, K, HK, HV, dk, dv, dtype):
     (1, 2, 32, 32, [150], 16, torch.float32),
     (2, 2, 64, 64, [40, 100, 7], 32, torch.float32),         # packed, ragged
     (2, 4, 128, 128, [130, 130], 64, torch.bfloat16),        # the tensor-core shape
+    (1, 2, 128, 64, [0, 65, 33, 1], 64, torch.bfloat16),     # an empty sequence, dk != dv
+    (1, 4, 64, 128, [97], 16, torch.float32),               # dk != dv the other way
 ])
 def test_prefill_row_decay(HK, HV, dk, dv, lengths, chunk, dtype, extra):
-    """The chunked prefill with one decay per value row runs on the CUDA-core
-    path (the tensor-core path's per-head inverse does not apply)."""
+    """The prefill with one decay per value row runs on the row-recurrent CUDA-core
+    kernel (each state row carried token by token): blocks of 32 tokens with
+    ragged tails, empty sequences, every head-dim pair it takes."""
     base = make_prefill(HK, HV, dk, dv, lengths, dtype, seed=86, h0_std=0.2)
     x = raw_projections(base, seed=87) if extra else base
     B, T = x["q"].shape[0], x["q"].shape[1]
