@@ -846,17 +846,22 @@ def run_b200(args):
         h2d_ms = timed(lambda: [dbuf[n].copy_(host_in[n], non_blocking=True) for n in names])
         d2h_ms = timed(lambda: (host_o.copy_(dout, non_blocking=True),
                                 host_h.copy_(hT, non_blocking=True)))
-        serial_ms = h2d_ms + mean_launch_s * 1e3 + d2h_ms
+        kern_ms = mean_launch_s * 1e3
+        serial_ms = h2d_ms + kern_ms + d2h_ms
+        # with the two copy directions and the kernels all overlapped the step could
+        # take as little as the slowest of the three
+        bound_ms = max(h2d_ms, d2h_ms, kern_ms)
         step_ms = e_ms / e_steps
         e2e = {"value": world * tokens * e_steps / (e_ms / 1000.0), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
                "ms_per_step": step_ms, "segments": -(-T // 4096), "segment_tokens": 4096,
                "h2d_gbs": h2d / (h2d_ms / 1e3) / 1e9, "d2h_gbs": d2h / (d2h_ms / 1e3) / 1e9,
-               "copies_alone_ms": h2d_ms + d2h_ms, "kernel_alone_ms": mean_launch_s * 1e3,
-               "serial_ms": serial_ms,
-               "overlap": (serial_ms - step_ms) / min(h2d_ms + d2h_ms, mean_launch_s * 1e3),
-               "note": "overlap: the part of the smaller of (copies, kernel) hidden behind the "
-                       "other; the step is bound by the host-to-device copy rate"}
+               "h2d_alone_ms": h2d_ms, "d2h_alone_ms": d2h_ms, "kernel_alone_ms": kern_ms,
+               "serial_ms": serial_ms, "bound_ms": bound_ms,
+               "overlap": (serial_ms - step_ms) / (serial_ms - bound_ms),
+               "note": "overlap = (serial - step) / (serial - bound): 0 when the copies and "
+                       "kernels run one after another, 1 when the step takes only its slowest "
+                       "part (here the host-to-device copy of the inputs)"}
 
     # ---- decode: 256 sequences x 64 single-token steps ----
     dec = None
@@ -950,6 +955,43 @@ def run_b200(args):
     return 0
 
 
+PROFILE_CASES = ("ring_4k", "rows_4k", "conv_16k")
+
+
+def run_profile_case(name):
+    """One small case of one kernel for an ncu capture (no timing, no JSON line):
+    a warm-up launch and two more, on inputs of a few hundred MB at most.
+      ring_4k  -- the tensor-core prefill on the 4096-token layer workload
+      rows_4k  -- the one-decay-per-value-row prefill on the same workload
+      conv_16k -- the short convolution (width 4, SiLU, carried state) over the
+                  first 16K tokens' values of the 64K workload (134 MB in, 134 MB out)
+    """
+    import torch
+    from linear_attention_recurrence_rule_b200 import gdn
+    from linear_attention_recurrence_rule_b200.inputs import layer_extras, row_decays, workload_inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if name == "conv_16k":
+        x = workload_inputs("long_prefill_64k", tokens=16384)["v"].reshape(1, 16384, -1).to(dev)
+        ex = layer_extras(1, x.shape[-1], 4, (1,), torch.bfloat16, seed=305)
+        w, b, cs = (ex[k].to(dev) for k in ("conv_weight", "conv_bias", "conv_state"))
+        y = torch.empty_like(x)
+        run = lambda: gdn.gdn_short_conv(x, w, b, cs, silu=True, y=y)   # noqa: E731
+    else:
+        z = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v)
+             for k, v in workload_inputs("layer_prefill_4k").items()}
+        g = row_decays(tuple(z["v"].shape), seed=903).to(dev) if name == "rows_4k" else z["g"]
+        pro = gdn.ROW_DECAY if name == "rows_4k" else 0
+        o = torch.empty_like(z["v"])
+        run = lambda: gdn.gdn_chunk_prefill(z["q"], z["k"], z["v"], g, z["beta"], chunk=64, o=o,   # noqa: E731
+                                            prologue=pro)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    print(f"profile case {name}: 3 launches done")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -970,7 +1012,11 @@ def main():
                     help="truncate the prefill workload (profiling runs; not a bench line)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--profile-case", choices=PROFILE_CASES, default=None,
+                    help="run one small case of one kernel for an ncu capture and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        return run_profile_case(args.profile_case)
     if args.warmup < 3:
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":

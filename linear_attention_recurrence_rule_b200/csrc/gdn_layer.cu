@@ -11,13 +11,16 @@
 // elementwise.
 //
 // All three kernels are single streaming passes over HBM:
-//  * conv_kernel: a thread owns 16 bytes of channels (8 bf16 / 4 fp32) for a
-//    run of kConvRun tokens: it issues the loads of the W-1 tokens before the
-//    run and of the whole run at once (one round trip), then slides a window of
-//    the previous W-1 inputs in registers.  Each input is read from DRAM once;
-//    the halo rows are re-read from L2, where the neighbouring run's thread has
-//    just brought them.  A sequence start inside a run resets the window from
-//    the carried state.
+//  * conv_kernel: a thread owns 16 bytes of channels (8 bf16 / 4 fp32) for one
+//    contiguous segment of tokens (one segment per SM and channel block), with
+//    its weights loaded once.  Its inputs come through a private ring of
+//    kConvStages tiles of kConvTile tokens in shared memory, filled by cp.async
+//    kConvStages - 1 tiles ahead (each thread reads back only what it copied,
+//    so no barrier is involved and 96 KB per SM stay in flight: the load
+//    depth an HBM stream needs), and it slides a window of the previous W-1
+//    inputs in registers.  Each input is read from DRAM once; the W-1 halo rows
+//    before a segment are re-read from L2.  A sequence start inside a segment
+//    resets the window from the carried state.
 //  * conv_state_kernel (launched after it on the same stream): each
 //    sequence's new carried state, its last W-1 inputs (from the old state
 //    where the sequence is shorter than W-1).  A launch of its own, so that
@@ -36,9 +39,10 @@
 namespace gdn {
 namespace {
 
-constexpr int kConvThreads = 128;
-constexpr int kConvRun = 8;      // tokens per thread, all loaded at once with the window
-constexpr int kConvBatch = 8;
+constexpr int kConvThreads = 512;  // 16 warps per SM: the per-token arithmetic needs the latency hiding
+constexpr int kConvTile = 4;     // tokens per tile
+constexpr int kConvStages = 4;   // tiles in a thread's ring (three in flight)
+constexpr size_t kConvSmem = (size_t)kConvStages * kConvTile * kConvThreads * 16;
 constexpr int kGateThreads = 256;
 
 // 16 bytes of one dtype as raw words and as floats
@@ -96,20 +100,26 @@ __device__ __forceinline__ void seq_bounds(const int32_t *cu, int64_t T_per, int
     }
 }
 
+__device__ __forceinline__ void conv_cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+
 template <typename T, int W>
-__global__ void __launch_bounds__(kConvThreads)
+__global__ void __launch_bounds__(kConvThreads, 1)
 conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
             const T *__restrict__ cstate, const int32_t *__restrict__ cu, int N, int64_t T_per,
-            int64_t Ttot, int C, int cblocks, bool silu, T *__restrict__ y,
+            int64_t Ttot, int C, int cblocks, int64_t seg_len, bool silu, T *__restrict__ y,
             T *__restrict__ y_lo) {
     constexpr int VN = Vec16<T>::n;
-    // the channel blocks of one run are neighbours in the grid, so the blocks
-    // resident at a time read whole token rows
-    const int64_t run = (int64_t)blockIdx.x / cblocks;
-    const int c0 = ((int)(blockIdx.x - run * cblocks) * kConvThreads + threadIdx.x) * VN;
-    if (c0 >= C) return;
-    const int64_t t0 = run * kConvRun;
-    const int64_t t1 = t0 + kConvRun < Ttot ? t0 + kConvRun : Ttot;
+    extern __shared__ uint4 ring[];   // [stage][token of the tile][thread]
+    const int seg = (int)(blockIdx.x / cblocks);
+    const int c0 = ((int)(blockIdx.x - seg * cblocks) * kConvThreads + threadIdx.x) * VN;
+    if (c0 >= C) return;   // (no barrier below: every thread works on its own)
+    const int64_t t0 = (int64_t)seg * seg_len;
+    const int64_t t1 = t0 + seg_len < Ttot ? t0 + seg_len : Ttot;
+    if (t0 >= t1) return;
     // the sequence holding token t0: the last n with start <= t0 (empty sequences skipped)
     int n;
     if (cu) {
@@ -125,6 +135,22 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
     }
     int64_t bos, eos;
     seq_bounds(cu, T_per, n, bos, eos);
+
+    // the ring: tile k of the segment into stage k % kConvStages, this thread's 16 bytes
+    // of each token; a commit group per tile (empty past the segment's end)
+    const int ntiles = (int)((t1 - t0 + kConvTile - 1) / kConvTile);
+    auto issue = [&](int k) {
+        const int64_t tb = t0 + (int64_t)k * kConvTile;
+        uint4 *dst = ring + (size_t)(k % kConvStages) * kConvTile * kConvThreads + threadIdx.x;
+        if (k < ntiles) {
+#pragma unroll
+            for (int r = 0; r < kConvTile; ++r)
+                if (tb + r < t1) conv_cp_async16(dst + r * kConvThreads, x + (tb + r) * C + c0);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+#pragma unroll
+    for (int k = 0; k < kConvStages - 1; ++k) issue(k);
 
     // this thread's VN x W weights are contiguous (16-byte aligned: c0 is a multiple of 4)
     float wt[W][VN], b[VN];
@@ -159,16 +185,17 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
         else
             win[m] = make_uint4(0u, 0u, 0u, 0u);   // +0.0 in both dtypes
     }
-    constexpr int NB = kConvBatch;
-    for (int64_t tb = t0; tb < t1; tb += NB) {
-        uint4 raw[NB];
+    for (int k = 0; k < ntiles; ++k) {
+        issue(k + kConvStages - 1);
+        // all but the kConvStages - 1 newest groups are complete: tile k has landed
+        asm volatile("cp.async.wait_group %0;" ::"n"(kConvStages - 1) : "memory");
+        const uint4 *src = ring + (size_t)(k % kConvStages) * kConvTile * kConvThreads + threadIdx.x;
+        const int64_t tb = t0 + (int64_t)k * kConvTile;
 #pragma unroll
-        for (int u = 0; u < NB; ++u)
-            if (tb + u < t1) raw[u] = ld16(x + (tb + u) * C + c0);
-#pragma unroll
-        for (int u = 0; u < NB; ++u) {
+        for (int u = 0; u < kConvTile; ++u) {
             const int64_t t = tb + u;
             if (t >= t1) break;
+            const uint4 cur = src[u * kConvThreads];
             if (t >= eos) {
                 // a new sequence starts at t (after any empty ones): window from its state
                 do {
@@ -189,7 +216,7 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
 #pragma unroll
                 for (int e = 0; e < VN; ++e) acc[e] = fmaf(wt[m][e], f[e], acc[e]);
             }
-            Vec16<T>::to_float(raw[u], f);
+            Vec16<T>::to_float(cur, f);
 #pragma unroll
             for (int e = 0; e < VN; ++e) {
                 const float a = fmaf(wt[W - 1][e], f[e], acc[e]);
@@ -208,9 +235,10 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
             }
 #pragma unroll
             for (int m = 0; m + 1 < W - 1; ++m) win[m] = win[m + 1];
-            win[W - 2] = raw[u];
+            win[W - 2] = cur;
         }
     }
+    // (every group still pending is empty: tiles past the end issue no copy)
 }
 
 // new carried state of sequence blockIdx.x: its last W-1 inputs (raw copies)
@@ -298,6 +326,14 @@ gate_factor_kernel(const T *__restrict__ z, void *__restrict__ f, int64_t nvec) 
     }
 }
 
+int sm_count() {
+    int dev = 0, count = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || count < 1)
+        count = 1;
+    return count;
+}
+
 template <typename T, int W>
 cudaError_t launch_conv_w(const ConvArgs &a, cudaStream_t stream) {
     constexpr int VN = Vec16<T>::n;
@@ -307,11 +343,20 @@ cudaError_t launch_conv_w(const ConvArgs &a, cudaStream_t stream) {
     const T *x = static_cast<const T *>(a.x);
     T *cs = static_cast<T *>(a.conv_state);
     if (Ttot > 0) {
-        const unsigned grid = (unsigned)((Ttot + kConvRun - 1) / kConvRun * cblocks);
-        conv_kernel<T, W><<<grid, kConvThreads, 0, stream>>>(
-            x, a.weight, a.bias, cs, a.cu_seqlens, a.N, a.T, Ttot, a.C, (int)cblocks, a.silu,
-            static_cast<T *>(a.y), static_cast<T *>(a.y_lo));
-        const cudaError_t e = cudaGetLastError();
+        // one segment of tokens per SM and channel block (a multiple of the tile)
+        const int64_t tiles = (Ttot + kConvTile - 1) / kConvTile;
+        int64_t nseg = ((int64_t)sm_count() + cblocks - 1) / cblocks;
+        if (nseg > tiles) nseg = tiles;
+        const int64_t seg_len = (tiles + nseg - 1) / nseg * kConvTile;
+        nseg = (Ttot + seg_len - 1) / seg_len;
+        auto kern = conv_kernel<T, W>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kConvSmem);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)(nseg * cblocks), kConvThreads, kConvSmem, stream>>>(
+            x, a.weight, a.bias, cs, a.cu_seqlens, a.N, a.T, Ttot, a.C, (int)cblocks, seg_len,
+            a.silu, static_cast<T *>(a.y), static_cast<T *>(a.y_lo));
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     if (cs) {
@@ -334,14 +379,6 @@ cudaError_t launch_conv_t(const ConvArgs &a, cudaStream_t stream) {
         case 8: return launch_conv_w<T, 8>(a, stream);
         default: return cudaErrorInvalidValue;
     }
-}
-
-int sm_count() {
-    int dev = 0, count = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || count < 1)
-        count = 1;
-    return count;
 }
 
 template <typename T>

@@ -48,6 +48,23 @@ def test_short_conv_packed_ragged(dtype, width, silu, with_state):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_short_conv_long_segments_cross_sequences(dtype):
+    # ~5K packed tokens: each SM's segment then spans several tiles of its ring, and
+    # sequence starts (and an empty sequence) fall inside segments and tiles
+    lengths = [0, 700, 3, 1500, 1, 2000, 33, 780]
+    C = 64
+    x, cu = packed_x(lengths, C, dtype, seed=311)
+    ex = layer_extras(len(lengths), C, 4, (1,), dtype, seed=312)
+    y_ref, s_ref = O.short_conv(x, ex["conv_weight"], ex["conv_bias"], ex["conv_state"], cu, "silu")
+    cs = ex["conv_state"].cuda()
+    y = gdn_short_conv(x.cuda(), ex["conv_weight"].cuda(), ex["conv_bias"].cuda(), cs, cu.cuda(),
+                       silu=True)
+    torch.cuda.synchronize()
+    assert_close(y[0], y_ref, dtype, "y")
+    assert torch.equal(cs.cpu(), torch.from_numpy(s_ref).to(dtype))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_short_conv_batched_no_bias(dtype):
     B, T, C, W = 3, 70, 96, 4
     gen = torch.Generator().manual_seed(303)
