@@ -42,7 +42,13 @@ namespace {
 constexpr int kConvThreads = 512;  // 16 warps per SM: the per-token arithmetic needs the latency hiding
 constexpr int kConvTile = 4;     // tokens per tile
 constexpr int kConvStages = 4;   // tiles in a thread's ring (three in flight)
-constexpr size_t kConvSmem = (size_t)kConvStages * kConvTile * kConvThreads * 16;
+// bf16 widths 6..8 keep their weights and window in 256 threads' registers
+template <typename T, int W>
+__host__ __device__ constexpr int conv_threads() { return (sizeof(T) == 2 && W >= 6) ? 256 : kConvThreads; }
+template <typename T, int W>
+__host__ __device__ constexpr size_t conv_smem() {
+    return (size_t)kConvStages * kConvTile * conv_threads<T, W>() * 16;
+}
 constexpr int kGateThreads = 256;
 
 // 16 bytes of one dtype as raw words and as floats
@@ -107,15 +113,16 @@ __device__ __forceinline__ void conv_cp_async16(void *dst, const void *src) {
 }
 
 template <typename T, int W>
-__global__ void __launch_bounds__(kConvThreads, 1)
+__global__ void __launch_bounds__(conv_threads<T, W>(), 1)
 conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
             const T *__restrict__ cstate, const int32_t *__restrict__ cu, int N, int64_t T_per,
             int64_t Ttot, int C, int cblocks, int64_t seg_len, bool silu, T *__restrict__ y,
             T *__restrict__ y_lo) {
     constexpr int VN = Vec16<T>::n;
+    constexpr int NT = conv_threads<T, W>();
     extern __shared__ uint4 ring[];   // [stage][token of the tile][thread]
     const int seg = (int)(blockIdx.x / cblocks);
-    const int c0 = ((int)(blockIdx.x - seg * cblocks) * kConvThreads + threadIdx.x) * VN;
+    const int c0 = ((int)(blockIdx.x - seg * cblocks) * NT + threadIdx.x) * VN;
     if (c0 >= C) return;   // (no barrier below: every thread works on its own)
     const int64_t t0 = (int64_t)seg * seg_len;
     const int64_t t1 = t0 + seg_len < Ttot ? t0 + seg_len : Ttot;
@@ -141,11 +148,11 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
     const int ntiles = (int)((t1 - t0 + kConvTile - 1) / kConvTile);
     auto issue = [&](int k) {
         const int64_t tb = t0 + (int64_t)k * kConvTile;
-        uint4 *dst = ring + (size_t)(k % kConvStages) * kConvTile * kConvThreads + threadIdx.x;
+        uint4 *dst = ring + (size_t)(k % kConvStages) * kConvTile * NT + threadIdx.x;
         if (k < ntiles) {
 #pragma unroll
             for (int r = 0; r < kConvTile; ++r)
-                if (tb + r < t1) conv_cp_async16(dst + r * kConvThreads, x + (tb + r) * C + c0);
+                if (tb + r < t1) conv_cp_async16(dst + r * NT, x + (tb + r) * C + c0);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
@@ -153,7 +160,9 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
     for (int k = 0; k < kConvStages - 1; ++k) issue(k);
 
     // this thread's VN x W weights are contiguous (16-byte aligned: c0 is a multiple of 4)
-    float wt[W][VN], b[VN];
+    // weights and bias as channel pairs (the arithmetic runs on packed fp32 pairs)
+    constexpr int VP = VN / 2;
+    float2 wt[W][VP], b[VP];
     {
         float flat[VN * W];
         const float4 *w4 = reinterpret_cast<const float4 *>(w + (size_t)c0 * W);
@@ -166,36 +175,44 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
             flat[4 * i + 3] = f.w;
         }
 #pragma unroll
-        for (int e = 0; e < VN; ++e)
+        for (int e = 0; e < VP; ++e)
 #pragma unroll
-            for (int j = 0; j < W; ++j) wt[j][e] = flat[e * W + j];
+            for (int j = 0; j < W; ++j) wt[j][e] = make_float2(flat[2 * e * W + j], flat[(2 * e + 1) * W + j]);
 #pragma unroll
-        for (int e = 0; e < VN; ++e) b[e] = bias ? __ldg(bias + c0 + e) : 0.f;
+        for (int e = 0; e < VP; ++e)
+            b[e] = bias ? make_float2(__ldg(bias + c0 + 2 * e), __ldg(bias + c0 + 2 * e + 1))
+                        : make_float2(0.f, 0.f);
     }
-    // window: win[m] = the raw input at token t - (W-1) + m, m < W-1 (raw words,
-    // converted where used: half the registers for bf16)
-    uint4 win[W - 1];
+    // window: win[m] = the input at token t - (W-1) + m, m < W-1, as fp32 pairs
+    // (converted once, when it enters)
+    float2 win[W - 1][VP];
+    auto to_pairs = [](const uint4 &u, float2 (&f)[VP]) {
+        float tmp[VN];
+        Vec16<T>::to_float(u, tmp);
+#pragma unroll
+        for (int e = 0; e < VP; ++e) f[e] = make_float2(tmp[2 * e], tmp[2 * e + 1]);
+    };
 #pragma unroll
     for (int m = 0; m < W - 1; ++m) {
         const int64_t s = t0 - (W - 1) + m;
+        uint4 raw = make_uint4(0u, 0u, 0u, 0u);   // +0.0 in both dtypes
         if (s >= bos)
-            win[m] = ld16(x + s * C + c0);
+            raw = ld16(x + s * C + c0);
         else if (cstate)
-            win[m] = ld16(cstate + ((size_t)n * (W - 1) + (size_t)(s - bos + W - 1)) * C + c0);
-        else
-            win[m] = make_uint4(0u, 0u, 0u, 0u);   // +0.0 in both dtypes
+            raw = ld16(cstate + ((size_t)n * (W - 1) + (size_t)(s - bos + W - 1)) * C + c0);
+        to_pairs(raw, win[m]);
     }
     for (int k = 0; k < ntiles; ++k) {
         issue(k + kConvStages - 1);
         // all but the kConvStages - 1 newest groups are complete: tile k has landed
         asm volatile("cp.async.wait_group %0;" ::"n"(kConvStages - 1) : "memory");
-        const uint4 *src = ring + (size_t)(k % kConvStages) * kConvTile * kConvThreads + threadIdx.x;
+        const uint4 *src = ring + (size_t)(k % kConvStages) * kConvTile * NT + threadIdx.x;
         const int64_t tb = t0 + (int64_t)k * kConvTile;
 #pragma unroll
         for (int u = 0; u < kConvTile; ++u) {
             const int64_t t = tb + u;
             if (t >= t1) break;
-            const uint4 cur = src[u * kConvThreads];
+            const uint4 cur = src[u * NT];
             if (t >= eos) {
                 // a new sequence starts at t (after any empty ones): window from its state
                 do {
@@ -204,25 +221,27 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
                 } while (eos <= t);
 #pragma unroll
                 for (int m = 0; m < W - 1; ++m)
-                    win[m] = cstate ? ld16(cstate + ((size_t)n * (W - 1) + m) * C + c0)
-                                    : make_uint4(0u, 0u, 0u, 0u);
+                    to_pairs(cstate ? ld16(cstate + ((size_t)n * (W - 1) + m) * C + c0)
+                                    : make_uint4(0u, 0u, 0u, 0u),
+                             win[m]);
             }
-            float acc[VN], f[VN];
+            float2 cf[VP], acc[VP];
+            to_pairs(cur, cf);
 #pragma unroll
-            for (int e = 0; e < VN; ++e) acc[e] = b[e];
+            for (int e = 0; e < VP; ++e) {
+                float2 a = b[e];
 #pragma unroll
-            for (int m = 0; m < W - 1; ++m) {
-                Vec16<T>::to_float(win[m], f);
-#pragma unroll
-                for (int e = 0; e < VN; ++e) acc[e] = fmaf(wt[m][e], f[e], acc[e]);
+                for (int m = 0; m < W - 1; ++m) a = fma2(wt[m][e], win[m][e], a);
+                a = fma2(wt[W - 1][e], cf[e], a);
+                acc[e] = silu ? make_float2(a.x * layer_sigmoid(a.x), a.y * layer_sigmoid(a.y)) : a;
             }
-            Vec16<T>::to_float(cur, f);
+            float af[VN];
 #pragma unroll
-            for (int e = 0; e < VN; ++e) {
-                const float a = fmaf(wt[W - 1][e], f[e], acc[e]);
-                acc[e] = silu ? a * layer_sigmoid(a) : a;
+            for (int e = 0; e < VP; ++e) {
+                af[2 * e] = acc[e].x;
+                af[2 * e + 1] = acc[e].y;
             }
-            const uint4 yv = Vec16<T>::from_float(acc);
+            const uint4 yv = Vec16<T>::from_float(af);
             st16(y + t * C + c0, yv);
             if (y_lo) {
                 // the remainder acc - y (exact in fp32) as a second output: the bf16
@@ -230,12 +249,15 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
                 float r[VN];
                 Vec16<T>::to_float(yv, r);
 #pragma unroll
-                for (int e = 0; e < VN; ++e) r[e] = acc[e] - r[e];
+                for (int e = 0; e < VN; ++e) r[e] = af[e] - r[e];
                 st16(y_lo + t * C + c0, Vec16<T>::from_float(r));
             }
 #pragma unroll
-            for (int m = 0; m + 1 < W - 1; ++m) win[m] = win[m + 1];
-            win[W - 2] = cur;
+            for (int m = 0; m + 1 < W - 1; ++m)
+#pragma unroll
+                for (int e = 0; e < VP; ++e) win[m][e] = win[m + 1][e];
+#pragma unroll
+            for (int e = 0; e < VP; ++e) win[W - 2][e] = cf[e];
         }
     }
     // (every group still pending is empty: tiles past the end issue no copy)
@@ -344,17 +366,19 @@ cudaError_t launch_conv_w(const ConvArgs &a, cudaStream_t stream) {
     T *cs = static_cast<T *>(a.conv_state);
     if (Ttot > 0) {
         // one segment of tokens per SM and channel block (a multiple of the tile)
+        constexpr int NT = conv_threads<T, W>();
+        constexpr size_t smem = conv_smem<T, W>();
+        const int64_t cb = (vecs + NT - 1) / NT;
         const int64_t tiles = (Ttot + kConvTile - 1) / kConvTile;
-        int64_t nseg = ((int64_t)sm_count() + cblocks - 1) / cblocks;
+        int64_t nseg = ((int64_t)sm_count() + cb - 1) / cb;
         if (nseg > tiles) nseg = tiles;
         const int64_t seg_len = (tiles + nseg - 1) / nseg * kConvTile;
         nseg = (Ttot + seg_len - 1) / seg_len;
         auto kern = conv_kernel<T, W>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kConvSmem);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<(unsigned)(nseg * cblocks), kConvThreads, kConvSmem, stream>>>(
-            x, a.weight, a.bias, cs, a.cu_seqlens, a.N, a.T, Ttot, a.C, (int)cblocks, seg_len,
+        kern<<<(unsigned)(nseg * cb), NT, smem, stream>>>(
+            x, a.weight, a.bias, cs, a.cu_seqlens, a.N, a.T, Ttot, a.C, (int)cb, seg_len,
             a.silu, static_cast<T *>(a.y), static_cast<T *>(a.y_lo));
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

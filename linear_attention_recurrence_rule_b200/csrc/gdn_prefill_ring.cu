@@ -505,6 +505,14 @@ __device__ void chain_cta(const CUtensorMap *tm_q, const CUtensorMap *tm_k, cons
                     tma_load_3d(slot + SL_WQ + hf * 16384 + 8192, tm_q, full, 64 * hf, cqk, s0);
                     tma_load_3d(slot + SL_K + hf * 8192, tm_k, full, 64 * hf, cqk, s0);
                 }
+                // the q/k tiles of chunk c + 2 into L2 ahead of their load
+                if (c + 2 < nchunks) {
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        tma_prefetch_l2_3d(tm_q, 64 * hf, cqk, s0 + 2 * C);
+                        tma_prefetch_l2_3d(tm_k, 64 * hf, cqk, s0 + 2 * C);
+                    }
+                }
             }
             __syncwarp();
             // the prep CTA has published chunk c's record
