@@ -355,11 +355,13 @@ def measure_layer(gdn, torch, dev, stream, x, w, o, hT, rank, peaks, peak_src, p
     y = torch.empty_like(d["v"])
     vin = d["v"].reshape(B, T, C)
 
-    def conv():
-        gdn.gdn_short_conv(vin, e["conv_weight"], e["conv_bias"], e["conv_state"], silu=True,
+    def conv(silu):
+        gdn.gdn_short_conv(vin, e["conv_weight"], e["conv_bias"], e["conv_state"], silu=silu,
                            y=y.reshape(B, T, C), stream=stream)
 
-    cv_ms = _time_events(torch, stream, conv, 10)
+    # the layer's configuration (no activation), then with SiLU
+    cv_ms = _time_events(torch, stream, lambda: conv(False), 10)
+    cvs_ms = _time_events(torch, stream, lambda: conv(True), 10)
     elt = 2
     cv_bytes = 2 * tokens * C * elt + 2 * B * (W - 1) * C * elt + C * (W + 1) * 4
 
@@ -398,20 +400,26 @@ def measure_layer(gdn, torch, dev, stream, x, w, o, hT, rank, peaks, peak_src, p
               + 2 * wd.B * (W - 1) * wd.HV * wd.dv * elt + wd.B * wd.HV * wd.dv * elt)
     dach = dbytes / (layer_d / 1e3) / 1e9
     return {"conv": "causal depthwise, width 4, bias, no activation, carried state "
-                    "(SiLU timed on the standalone kernel)",
+                    "(the standalone kernel also timed with SiLU)",
             "gate": "o * sigmoid(z)",
             "prefill": {"workload": WORKLOAD, "ms_per_step": lp_ms,
                         "value": tokens / (lp_ms / 1e3), "unit": "tokens/s",
                         "plain_ms_per_step": plain_s * 1e3, "overhead": lp_ms / (plain_s * 1e3) - 1.0,
-                        "gpu_launches": 4,
-                        "launches": "convolution + carried state, gate factors, prefill (gate applied "
-                                    "in its read-out)"},
+                        "gpu_launches": 3,
+                        "launches": "convolution with the gate factors in the same pass, carried "
+                                    "state, prefill (gate applied in its read-out)"},
             "conv_kernel": {"ms": cv_ms, "bytes": cv_bytes, "gpu_launches": 2,
                             "roofline": {"bound": "hbm", "achieved": cv_bytes / (cv_ms / 1e3) / 1e9,
                                          "peak": hbm, "unit": "GB/s",
                                          "frac": cv_bytes / (cv_ms / 1e3) / 1e9 / hbm,
                                          "traffic": kernel_traffic("short_conv"),
                                          "peak_source": peak_src, "kernel": "conv"}},
+            "conv_kernel_silu": {"ms": cvs_ms, "bytes": cv_bytes, "gpu_launches": 2,
+                                 "roofline": {"bound": "hbm",
+                                              "achieved": cv_bytes / (cvs_ms / 1e3) / 1e9,
+                                              "peak": hbm, "unit": "GB/s",
+                                              "frac": cv_bytes / (cvs_ms / 1e3) / 1e9 / hbm,
+                                              "peak_source": peak_src, "kernel": "conv with SiLU"}},
             "gate_kernel": {"ms": gt_ms, "bytes": gt_bytes, "gpu_launches": 1,
                             "roofline": {"bound": "hbm", "achieved": gt_bytes / (gt_ms / 1e3) / 1e9,
                                          "peak": hbm, "unit": "GB/s",
@@ -640,6 +648,36 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def measure_s0_pair_cost(gdn, torch, d, w, o, hT, stream, ring_ms):
+    """What carrying S0 as a bf16 hi + lo pair in the read-out costs: the same 64K
+    prefill through the no-allocation entry point, whose tensor-core kernel (the
+    cluster design with a DSMEM hand-over) reads out with a single-bf16 S0.  The
+    two kernels also differ in their hand-over (DSMEM against the L2 ring), so
+    the difference bounds the pair's cost from above."""
+    import ctypes
+    from linear_attention_recurrence_rule_b200 import gdn as core
+    P = ctypes.c_void_p
+    lib = core.load_library()
+    f = lib.gdn_chunk_prefill_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int, P, P, P]
+    B, T = d["q"].shape[0], d["q"].shape[1]
+    sp = P(stream.cuda_stream)
+
+    def call():
+        rc = f(P(d["q"].data_ptr()), P(d["k"].data_ptr()), P(d["v"].data_ptr()), P(d["g"].data_ptr()),
+               P(d["beta"].data_ptr()), None, None, B, T, w.HK, w.HV, w.dk, w.dv, w.chunk, 1.0,
+               core.GDN_BF16, P(o.data_ptr()), P(hT.data_ptr()), sp)
+        if rc != core.GDN_OK:
+            raise RuntimeError(core.status_string(rc))
+
+    ms = _time_events(torch, stream, call, 5)
+    return {"single_bf16_s0_ms": ms, "pair_s0_ms": ring_ms, "difference_ms": ring_ms - ms,
+            "kernels": "prefill_cluster_kernel (no-allocation entry point) against prefill_ring_kernel",
+            "gpu_launches": 1}
+
+
 def measure_configs(gdn, torch, dev, stream, peaks, peak_src, rank, args):
     """The other prefill workloads of the suite, each timed on its own (one call per
     step, CUDA events on the launching stream, 3 warm-up calls): tokens/s and the
@@ -922,6 +960,9 @@ def run_b200(args):
     cfgs = None
     if not args.no_configs:
         cfgs = measure_configs(gdn, torch, dev, stream, peaks, peak_src, rank, args)
+        if path == 1 and n_steps:
+            cfgs["s0_pair_cost"] = measure_s0_pair_cost(gdn, torch, d, w, o, hT, stream,
+                                                        mean_launch_s * 1e3)
 
     ver = None
     if not args.no_verify:

@@ -549,31 +549,35 @@ gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v, 
     if (N == 0) return GDN_OK;
     // workspace: [prefill's own | convolved values | gate factors (fp16)]
     const size_t pre = up256(gdn::prefill_workspace_bytes(a));
-    // on the tensor-core path the convolved values go to the rule as a bf16 pair
-    // (values + remainders): their rounding to bf16 alone would weigh on o where the
-    // state has a large common component (SiLU-convolved values)
-    const bool vpair = conv_weight && tc_path(dk, dv, chunk, dtype) && !(prologue & GDN_ROW_DECAY);
+    // on the tensor-core path SiLU-convolved values go to the rule as a bf16 pair
+    // (values + remainders): their positive mean gives the state a large common
+    // component, beside which the bf16 rounding of the values alone would weigh on
+    // o; without the activation the values are as centred as v and stay single bf16
+    const bool vpair = conv_weight && (flags & GDN_CONV_SILU) && tc_path(dk, dv, chunk, dtype) &&
+                       !(prologue & GDN_ROW_DECAY);
     const size_t vbytes = conv_weight ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen) * (vpair ? 2 : 1) : 0;
     const size_t need = pre + vbytes + (z ? layer_vconv_bytes(N, T, HV, dv, dtype, varlen) : 0);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // sigmoid(z) factors (fp16 for bf16, fp32 for fp32), applied in the prefill's
+    // read-out before o is rounded: formed by the convolution's launch when there is
+    // one (z has v's layout), else by a pass of their own
+    void *f = z ? static_cast<char *>(workspace) + pre + vbytes : nullptr;
     if (conv_weight) {
         ca.y = static_cast<char *>(workspace) + pre;
         if (vpair) ca.y_lo = static_cast<char *>(workspace) + pre + vbytes / 2;
+        ca.z = z;
+        ca.f = f;
         if (gdn::launch_short_conv(ca, s) != cudaSuccess) return GDN_ERR_CUDA;
         a.v = ca.y;
         a.v_lo = ca.y_lo;
-    }
-    if (z) {
-        // sigmoid(z) factors (fp16 for bf16, fp32 for fp32), applied in the prefill's
-        // read-out before o is rounded
-        void *f = static_cast<char *>(workspace) + pre + vbytes;
+    } else if (z) {
         const int64_t tokens = varlen ? T : (int64_t)N * T;
         if (gdn::launch_gate_factor(z, f, tokens * (int64_t)C, dtype, s) != cudaSuccess)
             return GDN_ERR_CUDA;
-        a.gate = f;
     }
+    if (z) a.gate = f;
     a.workspace_bytes = pre;
     if (pre == 0) a.workspace = nullptr;
     return enqueue_prefill(a, s);

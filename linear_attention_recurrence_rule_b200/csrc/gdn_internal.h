@@ -108,6 +108,8 @@ struct ConvArgs {
     gdn_dtype dtype;
     void *y;
     void *y_lo = nullptr;         // bf16 only: y_lo = y_exact - y, a second output
+    const void *z = nullptr;      // gate logits in x's layout [tokens][C] (layer prefill) or null
+    void *f = nullptr;            // their factors sigmoid(z): fp16 for bf16, fp32 for fp32
 };
 constexpr int kConvMaxWidth = 8;
 int conv_vector_channels(gdn_dtype dtype);   // channels per 16-byte vector

@@ -20,7 +20,10 @@
 //    depth an HBM stream needs), and it slides a window of the previous W-1
 //    inputs in registers.  Each input is read from DRAM once; the W-1 halo rows
 //    before a segment are re-read from L2.  A sequence start inside a segment
-//    resets the window from the carried state.
+//    resets the window from the carried state.  For the layer prefill (GZ) the
+//    same threads also turn the gate logits z of their tokens and channels (z has
+//    v's layout) into the factors sigmoid(z): a second stream through the ring,
+//    one launch for both passes.
 //  * conv_state_kernel (launched after it on the same stream): each
 //    sequence's new carried state, its last W-1 inputs (from the old state
 //    where the sequence is shorter than W-1).  A launch of its own, so that
@@ -41,13 +44,16 @@ namespace {
 
 constexpr int kConvThreads = 512;  // 16 warps per SM: the per-token arithmetic needs the latency hiding
 constexpr int kConvTile = 4;     // tokens per tile
-constexpr int kConvStages = 4;   // tiles in a thread's ring (three in flight)
+// tiles in a thread's ring: 4 (three in flight) for the values alone, 3 when the
+// gate logits stream through the same ring
+template <bool GZ>
+__host__ __device__ constexpr int conv_stages() { return GZ ? 3 : 4; }
 // bf16 widths 6..8 keep their weights and window in 256 threads' registers
 template <typename T, int W>
 __host__ __device__ constexpr int conv_threads() { return (sizeof(T) == 2 && W >= 6) ? 256 : kConvThreads; }
-template <typename T, int W>
+template <typename T, int W, bool GZ>
 __host__ __device__ constexpr size_t conv_smem() {
-    return (size_t)kConvStages * kConvTile * conv_threads<T, W>() * 16;
+    return (size_t)conv_stages<GZ>() * kConvTile * conv_threads<T, W>() * 16 * (GZ ? 2 : 1);
 }
 constexpr int kGateThreads = 256;
 
@@ -112,15 +118,17 @@ __device__ __forceinline__ void conv_cp_async16(void *dst, const void *src) {
                  : "memory");
 }
 
-template <typename T, int W>
+template <typename T, int W, bool GZ>
 __global__ void __launch_bounds__(conv_threads<T, W>(), 1)
 conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
             const T *__restrict__ cstate, const int32_t *__restrict__ cu, int N, int64_t T_per,
             int64_t Ttot, int C, int cblocks, int64_t seg_len, bool silu, T *__restrict__ y,
-            T *__restrict__ y_lo) {
+            T *__restrict__ y_lo, const T *__restrict__ z, void *__restrict__ fz) {
     constexpr int VN = Vec16<T>::n;
     constexpr int NT = conv_threads<T, W>();
-    extern __shared__ uint4 ring[];   // [stage][token of the tile][thread]
+    constexpr int NS = conv_stages<GZ>();
+    constexpr int ZOFF = NS * kConvTile * NT;   // the z stream's part of the ring
+    extern __shared__ uint4 ring[];   // [stage][token of the tile][thread] (values, then z)
     const int seg = (int)(blockIdx.x / cblocks);
     const int c0 = ((int)(blockIdx.x - seg * cblocks) * NT + threadIdx.x) * VN;
     if (c0 >= C) return;   // (no barrier below: every thread works on its own)
@@ -143,21 +151,24 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
     int64_t bos, eos;
     seq_bounds(cu, T_per, n, bos, eos);
 
-    // the ring: tile k of the segment into stage k % kConvStages, this thread's 16 bytes
-    // of each token; a commit group per tile (empty past the segment's end)
+    // the ring: tile k of the segment into stage k % NS, this thread's 16 bytes of
+    // each token; a commit group per tile (empty past the segment's end)
     const int ntiles = (int)((t1 - t0 + kConvTile - 1) / kConvTile);
     auto issue = [&](int k) {
         const int64_t tb = t0 + (int64_t)k * kConvTile;
-        uint4 *dst = ring + (size_t)(k % kConvStages) * kConvTile * NT + threadIdx.x;
+        uint4 *dst = ring + (size_t)(k % NS) * kConvTile * NT + threadIdx.x;
         if (k < ntiles) {
 #pragma unroll
             for (int r = 0; r < kConvTile; ++r)
-                if (tb + r < t1) conv_cp_async16(dst + r * NT, x + (tb + r) * C + c0);
+                if (tb + r < t1) {
+                    conv_cp_async16(dst + r * NT, x + (tb + r) * C + c0);
+                    if (GZ) conv_cp_async16(dst + ZOFF + r * NT, z + (tb + r) * C + c0);
+                }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 #pragma unroll
-    for (int k = 0; k < kConvStages - 1; ++k) issue(k);
+    for (int k = 0; k < NS - 1; ++k) issue(k);
 
     // this thread's VN x W weights are contiguous (16-byte aligned: c0 is a multiple of 4)
     // weights and bias as channel pairs (the arithmetic runs on packed fp32 pairs)
@@ -203,10 +214,10 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
         to_pairs(raw, win[m]);
     }
     for (int k = 0; k < ntiles; ++k) {
-        issue(k + kConvStages - 1);
-        // all but the kConvStages - 1 newest groups are complete: tile k has landed
-        asm volatile("cp.async.wait_group %0;" ::"n"(kConvStages - 1) : "memory");
-        const uint4 *src = ring + (size_t)(k % kConvStages) * kConvTile * NT + threadIdx.x;
+        issue(k + NS - 1);
+        // all but the NS - 1 newest groups are complete: tile k has landed
+        asm volatile("cp.async.wait_group %0;" ::"n"(NS - 1) : "memory");
+        const uint4 *src = ring + (size_t)(k % NS) * kConvTile * NT + threadIdx.x;
         const int64_t tb = t0 + (int64_t)k * kConvTile;
 #pragma unroll
         for (int u = 0; u < kConvTile; ++u) {
@@ -258,6 +269,23 @@ conv_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *_
                 for (int e = 0; e < VP; ++e) win[m][e] = win[m + 1][e];
 #pragma unroll
             for (int e = 0; e < VP; ++e) win[W - 2][e] = cf[e];
+            if (GZ) {
+                // gate factors sigmoid(z): fp16 for bf16 logits, fp32 for fp32 ones
+                float zf[VN];
+                Vec16<T>::to_float(src[ZOFF + u * NT], zf);
+                uint4 fv;
+                if constexpr (VN == 8) {
+                    __half2 hh[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        hh[e] = __floats2half2_rn(layer_sigmoid(zf[2 * e]), layer_sigmoid(zf[2 * e + 1]));
+                    fv = *reinterpret_cast<const uint4 *>(hh);
+                } else {
+                    fv = make_uint4(__float_as_uint(layer_sigmoid(zf[0])), __float_as_uint(layer_sigmoid(zf[1])),
+                                    __float_as_uint(layer_sigmoid(zf[2])), __float_as_uint(layer_sigmoid(zf[3])));
+                }
+                *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(fz) + ((size_t)t * C + c0) * sizeof(T)) = fv;
+            }
         }
     }
     // (every group still pending is empty: tiles past the end issue no copy)
@@ -356,6 +384,28 @@ int sm_count() {
     return count;
 }
 
+template <typename T, int W, bool GZ>
+cudaError_t launch_conv_segments(const ConvArgs &a, int64_t Ttot, cudaStream_t stream) {
+    // one segment of tokens per SM and channel block (a multiple of the tile)
+    constexpr int VN = Vec16<T>::n;
+    constexpr int NT = conv_threads<T, W>();
+    constexpr size_t smem = conv_smem<T, W, GZ>();
+    const int64_t cb = (a.C / VN + NT - 1) / NT;
+    const int64_t tiles = (Ttot + kConvTile - 1) / kConvTile;
+    int64_t nseg = ((int64_t)sm_count() + cb - 1) / cb;
+    if (nseg > tiles) nseg = tiles;
+    const int64_t seg_len = (tiles + nseg - 1) / nseg * kConvTile;
+    nseg = (Ttot + seg_len - 1) / seg_len;
+    auto kern = conv_kernel<T, W, GZ>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(nseg * cb), NT, smem, stream>>>(
+        static_cast<const T *>(a.x), a.weight, a.bias, static_cast<const T *>(a.conv_state), a.cu_seqlens,
+        a.N, a.T, Ttot, a.C, (int)cb, seg_len, a.silu, static_cast<T *>(a.y), static_cast<T *>(a.y_lo),
+        static_cast<const T *>(a.z), a.f);
+    return cudaGetLastError();
+}
+
 template <typename T, int W>
 cudaError_t launch_conv_w(const ConvArgs &a, cudaStream_t stream) {
     constexpr int VN = Vec16<T>::n;
@@ -365,22 +415,8 @@ cudaError_t launch_conv_w(const ConvArgs &a, cudaStream_t stream) {
     const T *x = static_cast<const T *>(a.x);
     T *cs = static_cast<T *>(a.conv_state);
     if (Ttot > 0) {
-        // one segment of tokens per SM and channel block (a multiple of the tile)
-        constexpr int NT = conv_threads<T, W>();
-        constexpr size_t smem = conv_smem<T, W>();
-        const int64_t cb = (vecs + NT - 1) / NT;
-        const int64_t tiles = (Ttot + kConvTile - 1) / kConvTile;
-        int64_t nseg = ((int64_t)sm_count() + cb - 1) / cb;
-        if (nseg > tiles) nseg = tiles;
-        const int64_t seg_len = (tiles + nseg - 1) / nseg * kConvTile;
-        nseg = (Ttot + seg_len - 1) / seg_len;
-        auto kern = conv_kernel<T, W>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<(unsigned)(nseg * cb), NT, smem, stream>>>(
-            x, a.weight, a.bias, cs, a.cu_seqlens, a.N, a.T, Ttot, a.C, (int)cb, seg_len,
-            a.silu, static_cast<T *>(a.y), static_cast<T *>(a.y_lo));
-        e = cudaGetLastError();
+        const cudaError_t e = a.z ? launch_conv_segments<T, W, true>(a, Ttot, stream)
+                                  : launch_conv_segments<T, W, false>(a, Ttot, stream);
         if (e != cudaSuccess) return e;
     }
     if (cs) {

@@ -191,8 +191,8 @@ def ref_layer(x, ex, conv, gate, dtype, scale, stored=None, silu=True, pair=Fals
     between the convolution and the rule, as the prefill call stores them in its
     workspace.  ``stored`` selects the tokens whose convolved values pass through
     that storage ([B, T] bool; all when None): the decode step keeps them in fp32
-    on chip.  ``pair``: the tensor-core path, which stores them as a bf16 value +
-    remainder pair (~2^-17 relative), so they are not rounded here."""
+    on chip.  ``pair``: the tensor-core path with SiLU, which stores them as a bf16
+    value + remainder pair (~2^-17 relative), so they are not rounded here."""
     v = x["v"]
     vs = v.shape
     C = vs[-2] * vs[-1]
@@ -307,8 +307,10 @@ def _bench_size_layer(silu):
         ch = np.concatenate([np.arange(h * dv, (h + 1) * dv) for h in vh])
         exs = {"conv_weight": ex["conv_weight"][ch], "conv_bias": ex["conv_bias"][ch],
                "conv_state": ex["conv_state"][:, :, ch], "z": ex["z"][:, :, vh]}
+        # the tensor-core path carries SiLU-convolved values as a bf16 pair, plain
+        # convolved values as single bf16
         o_ref, h_ref, cs_ref = ref_layer(sub, exs, True, True, torch.bfloat16, 0.7, silu=silu,
-                                         pair=True)
+                                         pair=silu)
         yield vh, o[0][:, vh], o_ref, hT[:, vh], h_ref
         assert torch.equal(cs.cpu()[:, :, ch], torch.from_numpy(cs_ref).to(torch.bfloat16))
 
