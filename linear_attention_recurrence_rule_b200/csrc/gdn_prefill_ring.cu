@@ -129,7 +129,9 @@ enum PrepBar { PB_LD0, PB_LD1, PB_X, PB_XREAD, PB_T, PB_WU, PB_EPI, PB_RFREE0, P
 constexpr uint32_t AUX_RAW = (C_BAR + CB_COUNT * 8 > P_BAR + PB_COUNT * 8) ? C_BAR + CB_COUNT * 8
                                                                           : P_BAR + PB_COUNT * 8;
 constexpr uint32_t AUX = (AUX_RAW + 15) & ~15u;
-constexpr uint32_t AUX_TSLOT = AUX, AUX_ABORT = AUX + 4, AUX_RING = AUX + 8, AUX_ARMED = AUX + 12;
+constexpr uint32_t AUX_TSLOT = AUX, AUX_ABORT = AUX + 4, AUX_RING = AUX + 8, AUX_ARMED = AUX + 12,
+                   AUX_SEQ = AUX + 16;
+constexpr int kOrderMax = 1024;   // packed batches up to this many sequences run longest first
 constexpr uint32_t SMEM_BYTES = AUX + 32 + 1024;
 static_assert(P_X + 32 * X_LD * 4 <= P_T2, "prep layout");
 static_assert(P_PB + 5 * 64 * 4 <= P_ST, "prep layout");
@@ -1210,8 +1212,30 @@ prefill_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                               ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     const int rank = (int)cluster_ctarank();
-    const int h = blockIdx.x / kClusterSize, n = blockIdx.y;
+    const int h = blockIdx.x / kClusterSize;
     const int tid = threadIdx.x, warp = tid >> 5;
+    // Packed batches run longest sequence first: row r of the grid (dispatched after
+    // rows 0..r-1) takes the sequence of rank r by decreasing length (ties by index),
+    // so the long chains start in the first wave and the short ones fill the tail.
+    // Every CTA of a cluster derives the same permutation from cu_seqlens.
+    int n = blockIdx.y;
+    if (p.cu && gridDim.y > 1 && gridDim.y <= (unsigned)kOrderMax) {
+        const int N = (int)gridDim.y;
+        volatile int *seq = reinterpret_cast<volatile int *>(sm + AUX_SEQ);
+        if (tid == 0) *seq = n;
+        __syncthreads();
+        for (int m = tid; m < N; m += kThreads) {
+            const int lm = p.cu[m + 1] - p.cu[m];
+            int rk = 0;
+            for (int j = 0; j < N; ++j) {
+                const int lj = p.cu[j + 1] - p.cu[j];
+                rk += (lj > lm || (lj == lm && j < m)) ? 1 : 0;
+            }
+            if (rk == n) *seq = m;
+        }
+        __syncthreads();
+        n = *seq;
+    }
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + (rank == 0 ? C_BAR : P_BAR));
     const int nbars = rank == 0 ? CB_COUNT : PB_COUNT;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + AUX_TSLOT);
