@@ -996,7 +996,7 @@ def run_b200(args):
     return 0
 
 
-PROFILE_CASES = ("ring_4k", "rows_4k", "conv_16k")
+PROFILE_CASES = ("ring_4k", "rows_4k", "conv_16k", "gate_16k")
 
 
 def run_profile_case(name):
@@ -1006,6 +1006,7 @@ def run_profile_case(name):
       rows_4k  -- the one-decay-per-value-row prefill on the same workload
       conv_16k -- the short convolution (width 4, SiLU, carried state) over the
                   first 16K tokens' values of the 64K workload (134 MB in, 134 MB out)
+      gate_16k -- the standalone output gate o <- o sigmoid(z) on 16K x 4096 outputs
     """
     import torch
     from linear_attention_recurrence_rule_b200 import gdn
@@ -1018,6 +1019,10 @@ def run_profile_case(name):
         w, b, cs = (ex[k].to(dev) for k in ("conv_weight", "conv_bias", "conv_state"))
         y = torch.empty_like(x)
         run = lambda: gdn.gdn_short_conv(x, w, b, cs, silu=True, y=y)   # noqa: E731
+    elif name == "gate_16k":
+        o = workload_inputs("long_prefill_64k", tokens=16384)["v"].to(dev)
+        z = layer_extras(1, o.shape[2] * o.shape[3], 4, tuple(o.shape), torch.bfloat16, seed=306)["z"].to(dev)
+        run = lambda: gdn.gdn_output_gate(o, z)   # noqa: E731
     else:
         z = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v)
              for k, v in workload_inputs("layer_prefill_4k").items()}

@@ -118,11 +118,14 @@ GDN_API size_t gdn_chunk_prefill_workspace_size(int N, int64_t T, int HK, int HV
  * value row: [N][HV][dv] for gdn_recurrent_step_ex, [N][K][HV][dv] for
  * gdn_recurrent_verify and gdn_state_commit_deltas.  Each row i of a state
  * decays by its own alpha_i before the correction.  Supported by the decode
- * step, by verify when states_out is given, by both commits, and by the chunked
- * prefill (`g` [B][T][HV][dv]) on its CUDA-core path for every supported shape
- * (the tensor-core path's per-head triangular inverse becomes per row, so it
- * is not used); the update-vector-only verify and the fused commit-then-verify
- * return GDN_ERR_UNSUPPORTED (their per-head mixed vectors would become per row).
+ * step, by verify when states_out is given, by both commits, and by the
+ * prefill (`g` [B][T][HV][dv]) for every supported shape, which then runs the
+ * recurrence token by token on CUDA cores, one lane group per state row (the
+ * rows never mix under this rule; the tensor-core path's per-head triangular
+ * inverse would become one per row, so it is not used; `chunk` is checked but
+ * does not shape that computation); the update-vector-only verify and the fused
+ * commit-then-verify return GDN_ERR_UNSUPPORTED (their per-head mixed vectors
+ * would become per row).
  */
 #define GDN_ROW_DECAY 8u
 #define GDN_FLAGS_VALID 15u
@@ -489,7 +492,8 @@ GDN_API gdn_status gdn_recurrent_step_layer(const void *q, const void *k, const 
  * Bytes of device workspace gdn_chunk_prefill_layer needs: gdn_chunk_prefill's
  * own workspace, then the convolved values (when has_conv) and the gate factors
  * sigmoid(z) (when has_gate), each [tokens][HV*dv] of 2 bytes (bf16 calls) or
- * 4 bytes (fp32 calls).
+ * 4 bytes (fp32 calls); on the tensor-core path the convolved values get room for
+ * a bf16 pair (twice the bytes), which the call uses with GDN_CONV_SILU.
  */
 GDN_API size_t gdn_chunk_prefill_layer_workspace_size(int N, int64_t T, int HK, int HV, int dk,
                                                       int dv, int chunk, gdn_dtype dtype,
@@ -498,15 +502,20 @@ GDN_API size_t gdn_chunk_prefill_layer_workspace_size(int N, int64_t T, int HK, 
 /*
  * gdn_chunk_prefill_ex with the layer steps: the short convolution of v
  * (gdn_short_conv into the workspace, stored in the call's dtype -- the
- * tensor-core path takes bf16 operands; conv_state [N][conv_width-1][HV*dv]
- * updated as there), the gate factors sigmoid(z) into the workspace (fp16,
- * relative error <= 2^-12, for bf16 calls; fp32 for fp32 calls), then the
- * prefill on the convolved values, which multiplies o by the factors where it
- * writes o (z like v; o is rounded once).
+ * tensor-core path takes bf16 operands, and with GDN_CONV_SILU it takes the
+ * convolved values as a bf16 pair value + remainder, ~2^-17 relative, since
+ * SiLU-convolved values give the state a large common component beside which
+ * their rounding would weigh on o; conv_state [N][conv_width-1][HV*dv] updated
+ * as there), the gate factors sigmoid(z) into the workspace (fp16, relative
+ * error <= 2^-12, for bf16 calls; fp32 for fp32 calls; formed in the
+ * convolution's pass when there is one), then the prefill on the convolved
+ * values, which multiplies o by the factors where it writes o (z like v; o is
+ * rounded once).
  * conv_weight NULL: no convolution; z NULL: no gate.  flags: GDN_PROLOGUE_*,
- * GDN_ROW_DECAY and GDN_CONV_SILU.  Launches on `stream`: the convolution's
- * two, the factors' one, the prefill's one; arguments as in
- * gdn_chunk_prefill_ex and gdn_short_conv.  z 16-byte aligned.
+ * GDN_ROW_DECAY and GDN_CONV_SILU.  Launches on `stream`: the convolution's two
+ * (the factors with it) or, without a convolution, the factors' one, then the
+ * prefill's one; arguments as in gdn_chunk_prefill_ex and gdn_short_conv.  z
+ * 16-byte aligned.
  */
 GDN_API gdn_status gdn_chunk_prefill_layer(const void *q, const void *k, const void *v,
                                            const float *g, const float *beta, const float *h0,

@@ -128,6 +128,21 @@ def test_varlen_with_empty_and_short_sequences(dtype):
     assert torch.equal(hT[0].cpu(), x["h0"][0]) and torch.equal(hT[5].cpu(), x["h0"][5])
 
 
+@pytest.mark.parametrize("nseq,maxlen", [(300, 100), (1100, 9)])
+def test_varlen_many_sequences(nseq, maxlen):
+    # many packed sequences with repeated and zero lengths on the tensor-core path:
+    # up to 1024 sequences run longest first (a permutation of the grid rows, ties
+    # by index), more in launch order
+    gen = torch.Generator().manual_seed(12)
+    lengths = torch.randint(0, maxlen + 1, (nseq,), generator=gen).tolist()
+    x = make_prefill(1, 2, 128, 128, lengths, torch.bfloat16, seed=13, h0_std=0.2, packed=True)
+    o, hT, o_ref, h_ref = run_both(x, 64)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(hT, h_ref, torch.bfloat16, "hT")
+    empty = [i for i, n in enumerate(lengths) if n == 0]
+    assert empty and all(torch.equal(hT[i].cpu(), x["h0"][i]) for i in empty)
+
+
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 1000])
 def test_bf16_d128_ragged_lengths(T):
     x = make_prefill(2, 4, 128, 128, [T, T], torch.bfloat16, seed=300 + T, h0_std=0.05)
