@@ -476,27 +476,32 @@ NCU_TRAFFIC = {
     # instance): 549,628,160 read + 482,972,928 written
     "decode_layer": {"bytes": 1032601088, "source": "gdn_decode.cu",
                      "sha256": "342c1ce55a1419f66a4d3b79e1f521987b47cfa44938be1fd8bc6c150858c6b6"},
-    # full long_prefill_64k launch: 1,090,636,800 read + 510,305,280 written
-    "prefill_cluster": {"bytes": 1600942080, "source": "gdn_prefill_cluster.cu",
+    # full long_prefill_64k launch of the ring prefill: 1,102,597,376 read + 514,424,064
+    # written (algorithmic 1,627,389,952)
+    "prefill_ring": {"bytes": 1617021440, "source": "gdn_prefill_ring.cu",
+                     "sha256": "60d3e2431e39242ff1549de34f0749eda08d3036e9c679e38c9be45722cf180b"},
+    # the same workload on the cluster kernel (no-allocation entry point): 1,091,336,960
+    # read + 509,906,688 written
+    "prefill_cluster": {"bytes": 1601243648, "source": "gdn_prefill_cluster.cu",
                         "sha256": "4ef0fef23fee2a3208626b5a458640654ce023f7ea5ab71922fbe7ecd21b2990"},
-    # short convolution of the 64K bench values (width 4): 537,046,272 read + 491,637,504
-    # written (its carried-state launch adds 55,552)
-    "short_conv": {"bytes": 1028683776, "source": "gdn_layer.cu",
-                   "sha256": "911934bd0e7a294c493cab767e7a41f34e1b110e7d47ba97e739ee1fe4b5009a"},
-    # standalone output gate over the 64K bench outputs: 1,073,752,064 read + 491,309,056 written
-    "output_gate": {"bytes": 1565061120, "source": "gdn_layer.cu",
-                    "sha256": "911934bd0e7a294c493cab767e7a41f34e1b110e7d47ba97e739ee1fe4b5009a"},
-    # verify_256x4, update-vector form, the streaming kernel: 580,045,056 read + 20,497,408
+    # short convolution of the 64K bench values (width 4): 540,828,672 read + 483,701,248
+    # written (its carried-state launch adds 55,296)
+    "short_conv": {"bytes": 1024529920, "source": "gdn_layer.cu",
+                   "sha256": "03e2d96c3e8a4dbc194fc0970d48afd7b79fc033f0bb351a248b95dfc9e837bd"},
+    # standalone output gate over the 64K bench outputs: 1,073,846,528 read + 492,012,288 written
+    "output_gate": {"bytes": 1565858816, "source": "gdn_layer.cu",
+                    "sha256": "03e2d96c3e8a4dbc194fc0970d48afd7b79fc033f0bb351a248b95dfc9e837bd"},
+    # verify_256x4, update-vector form, the streaming kernel: 579,929,088 read + 20,496,640
     # written (its setup kernel adds 8,682,752)
-    "verify_deltas": {"bytes": 600542464, "source": "gdn_verify.cu",
-                      "sha256": "06a1ca667c8f672649db772cc989cae84bf6fba0a1cad2bfdee72a098788d42c"},
-    # verify_256x4, per-draft states: 554,970,880 read + 2,093,050,368 written
-    "verify_states": {"bytes": 2648021248, "source": "gdn_verify.cu",
-                      "sha256": "06a1ca667c8f672649db772cc989cae84bf6fba0a1cad2bfdee72a098788d42c"},
+    "verify_deltas": {"bytes": 600425728, "source": "gdn_verify.cu",
+                      "sha256": "c7f25202b049192171c9b1ccb1c71f87366353665b74ab35948b1484488a8892"},
+    # verify_256x4, per-draft states: 554,959,104 read + 2,092,982,784 written
+    "verify_states": {"bytes": 2647941888, "source": "gdn_verify.cu",
+                      "sha256": "c7f25202b049192171c9b1ccb1c71f87366353665b74ab35948b1484488a8892"},
     # verify_256x4 fused round (previous commit + verify), the streaming kernel:
-    # 613,578,752 read + 382,084,864 written
-    "verify_fused": {"bytes": 995663616, "source": "gdn_verify.cu",
-                     "sha256": "06a1ca667c8f672649db772cc989cae84bf6fba0a1cad2bfdee72a098788d42c"},
+    # 613,593,856 read + 382,361,600 written
+    "verify_fused": {"bytes": 995955456, "source": "gdn_verify.cu",
+                     "sha256": "c7f25202b049192171c9b1ccb1c71f87366353665b74ab35948b1484488a8892"},
 }
 
 
