@@ -123,9 +123,11 @@ GDN_API size_t gdn_chunk_prefill_workspace_size(int N, int64_t T, int HK, int HV
  * recurrence token by token on CUDA cores, one lane group per state row (the
  * rows never mix under this rule; the tensor-core path's per-head triangular
  * inverse would become one per row, so it is not used; `chunk` is checked but
- * does not shape that computation); the update-vector-only verify and the fused
- * commit-then-verify return GDN_ERR_UNSUPPORTED (their per-head mixed vectors
- * would become per row).
+ * does not shape that computation).  The update-vector-only verify and the fused
+ * commit-then-verify take it too: their one-pass kernel mixes the drafts per
+ * head, which row decays would make per row, so with GDN_ROW_DECAY the verify
+ * runs the per-draft kernel without writing states, and the fused call runs the
+ * deltas commit and then that verify (two passes over the states).
  */
 #define GDN_ROW_DECAY 8u
 #define GDN_FLAGS_VALID 15u
@@ -332,7 +334,8 @@ GDN_API gdn_status gdn_recurrent_step_ex(const void *q, const void *k, const voi
  *   g, beta [N][K][HV] fp32          state [N][HV][dv][dk] fp32 (read)
  *   states_out [N][K][HV][dv][dk] fp32   u_out [N][K][HV][dv] fp32
  * prologue: GDN_PROLOGUE_* flags applied to every draft (0 = prepared inputs);
- * GDN_ROW_DECAY (g [N][K][HV][dv]) needs states_out, else GDN_ERR_UNSUPPORTED.
+ * GDN_ROW_DECAY: g [N][K][HV][dv]; without states_out it runs the per-draft
+ * kernel writing no states (the workspace is checked but not used).
  * workspace: device scratch of at least gdn_recurrent_verify_workspace_size()
  * bytes, 16-byte aligned, needed when states_out is NULL (the update-vector
  * form builds per (sequence, value head) tables there; ignored otherwise, may
@@ -369,7 +372,8 @@ GDN_API size_t gdn_recurrent_verify_workspace_size(int N, int K, int HV, int dk)
  * Layouts: prev_k [N][prev_K][HK][dk] dtype, prev_g [N][prev_K][HV] fp32,
  * prev_u [N][prev_K][HV][dv] fp32, accepted [N] int32 (device; 0 or out of range
  * = nothing kept); the rest as gdn_recurrent_verify.  `prologue` applies to both
- * rounds' drafts (GDN_ROW_DECAY returns GDN_ERR_UNSUPPORTED).
+ * rounds' drafts; with GDN_ROW_DECAY (prev_g and g with a trailing dv axis) the
+ * call runs gdn_state_commit_deltas and then the verify, two passes.
  * workspace: at least gdn_recurrent_commit_verify_workspace_size() bytes,
  * 16-byte aligned; its first word is the status of the call's bounded waits
  * (gdn_read_status).  Supported: as gdn_recurrent_verify, 1 <= prev_K <= 16.

@@ -317,8 +317,7 @@ gdn_status gdn_recurrent_verify(const void *q, const void *k, const void *v, con
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
         !aligned16(states_out) || !aligned4(u_out))
         return GDN_ERR_ALIGNMENT;
-    if (!states_out && (prologue & GDN_ROW_DECAY)) return GDN_ERR_UNSUPPORTED;
-    if (!states_out) {   // update-vector form: tables in the workspace
+    if (!states_out) {   // update-vector form: tables in the workspace (unused with row decays)
         if (!workspace ||
             workspace_bytes < gdn::verify_workspace_floats(N, K, HV, dk) * sizeof(float))
             return GDN_ERR_WORKSPACE;
@@ -346,7 +345,7 @@ gdn_status gdn_recurrent_commit_verify(const void *prev_k, const float *prev_g, 
         return GDN_ERR_INVALID_ARG;
     if (K > GDN_VERIFY_MAX_DRAFTS || prev_K > GDN_VERIFY_MAX_DRAFTS || (int64_t)N * HV > 0x7fffffff)
         return GDN_ERR_UNSUPPORTED;
-    if (!gdn::decode_supported(dk, dv) || (prologue & GDN_ROW_DECAY)) return GDN_ERR_UNSUPPORTED;
+    if (!gdn::decode_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
         !aligned16(prev_k) || !aligned4(prev_u) || !aligned4(accepted) || !aligned4(u_out))
         return GDN_ERR_ALIGNMENT;
@@ -356,6 +355,16 @@ gdn_status gdn_recurrent_commit_verify(const void *prev_k, const float *prev_g, 
     if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
     gdn::VerifyArgs a{q, k, v, g, beta, state, nullptr, u_out, N, K, HK, HV, dk, dv, scale,
                       dtype, o, prologue, workspace, workspace_bytes};
+    if (prologue & GDN_ROW_DECAY) {
+        // one decay per value row: the previous round's commit from its update vectors,
+        // then this round's verify writing update vectors (two passes over the states;
+        // the one-pass form mixes the drafts per head)
+        gdn::CommitDeltasArgs c{prev_k, prev_g, prev_u, accepted, state, N, prev_K, HK, HV, dk, dv,
+                                dtype, prologue};
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        if (gdn::launch_commit_deltas(c, s) != cudaSuccess) return GDN_ERR_CUDA;
+        return gdn::launch_verify(a, s) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    }
     a.prev_k = prev_k;
     a.prev_g = prev_g;
     a.prev_u = prev_u;

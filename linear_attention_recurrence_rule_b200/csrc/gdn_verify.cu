@@ -899,8 +899,10 @@ cudaError_t launch_verify_typed(const VerifyArgs &a, cudaStream_t stream) {
                                                                    : verify_band<32>();
     const dim3 grid((unsigned)((size_t)a.N * a.HV), (unsigned)((a.dv + band - 1) / band)),
         block(kVerifyWarps * 32);
-    if (a.states == nullptr) {
+    if (a.states == nullptr && !(a.prologue & GDN_ROW_DECAY)) {
         // no per-draft states asked for: the state is never updated in registers
+        // (with one decay per value row the mixed vectors would be per row: that
+        // form runs on the per-draft kernel below, writing no states)
         switch (a.dk) {
             case 32: launch_verify_wy_k<32, Tin>(a, block, stream); break;
             case 64: launch_verify_wy_k<64, Tin>(a, block, stream); break;

@@ -327,9 +327,9 @@ def gdn_recurrent_commit_verify(prev_k, prev_g, prev_u, accepted, q, k, v, g, be
     (``gdn_recurrent_commit_verify``): ``state`` is updated in place to the
     committed state; returns (o [N,K,HV,dv], u_out [N,K,HV,dv]) of this round.
 
-    prev_k [N,Kp,HK,dk]; prev_g [N,Kp,HV]; prev_u [N,Kp,HV,dv] (the previous
-    verify's u_out); accepted [N] int32 on the device; the rest as
-    ``gdn_recurrent_verify``.
+    prev_k [N,Kp,HK,dk]; prev_g [N,Kp,HV] ([N,Kp,HV,dv] with ROW_DECAY, like g);
+    prev_u [N,Kp,HV,dv] (the previous verify's u_out); accepted [N] int32 on the
+    device; the rest as ``gdn_recurrent_verify``.
     """
     lib = load_library()
     dev = q.device
@@ -344,12 +344,13 @@ def gdn_recurrent_commit_verify(prev_k, prev_g, prev_u, accepted, q, k, v, g, be
     N, K, HK, dk = q.shape
     HV, dv = v.shape[2], v.shape[3]
     Kp = prev_k.shape[1] if prev_k.dim() == 4 else -1
-    if (g.shape != (N, K, HV) or beta.shape != (N, K, HV) or state.shape != (N, HV, dv, dk)
-            or prev_k.shape != (N, Kp, HK, dk) or prev_g.shape != (N, Kp, HV)
+    rd = (dv,) if prologue & ROW_DECAY else ()
+    if (g.shape != (N, K, HV) + rd or beta.shape != (N, K, HV) or state.shape != (N, HV, dv, dk)
+            or prev_k.shape != (N, Kp, HK, dk) or prev_g.shape != (N, Kp, HV) + rd
             or prev_u.shape != (N, Kp, HV, dv) or accepted.shape != (N,)):
-        raise ValueError("shapes: prev_k [N,Kp,HK,dk], prev_g [N,Kp,HV], prev_u [N,Kp,HV,dv], "
-                         "accepted [N], q,k [N,K,HK,dk], v [N,K,HV,dv], g,beta [N,K,HV], "
-                         "state [N,HV,dv,dk]")
+        raise ValueError("shapes: prev_k [N,Kp,HK,dk], prev_g [N,Kp,HV(,dv)], prev_u [N,Kp,HV,dv], "
+                         "accepted [N], q,k [N,K,HK,dk], v [N,K,HV,dv], g [N,K,HV(,dv)], "
+                         "beta [N,K,HV], state [N,HV,dv,dk]")
     if o is None:
         o = torch.empty_like(v)
     if u_out is None:

@@ -194,15 +194,16 @@ def test_prologue_flags_are_validated(lib):
                                      1, 2, 128, 128, 1.0, gdn.GDN_BF16, fake(0x7000), 16,
                                      None) == gdn.GDN_ERR_INVALID_ARG
     assert verify_call(lib, pro=16) == gdn.GDN_ERR_INVALID_ARG
-    # one decay per value row: decode and per-draft-state verify only
+    # one decay per value row: accepted by every call; unsupported shapes still rejected
     assert re.search(r"#define GDN_ROW_DECAY 8u", text)
     # (a supported shape would pass validation and launch: only rejected shapes here)
     assert lib.gdn_chunk_prefill_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], None, None, 1, 64,
                                     1, 2, 48, 32, 16, 1.0, gdn.GDN_F32, fake(0x6000), None, None,
                                     0, gdn.ROW_DECAY, None) == gdn.GDN_ERR_UNSUPPORTED
-    need = lib.gdn_recurrent_verify_workspace_size(2, 4, 2, 128)
-    assert verify_call(lib, states=None, ws=fake(0xa000), ws_bytes=need,
-                       pro=gdn.ROW_DECAY) == gdn.GDN_ERR_UNSUPPORTED
+    # the update-vector form with row decays passes the flag checks and stops at the
+    # workspace check (nothing is launched here)
+    assert verify_call(lib, states=None, ws=None, ws_bytes=0,
+                       pro=gdn.ROW_DECAY) == gdn.GDN_ERR_WORKSPACE
     assert lib.gdn_recurrent_step_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], fake(0x6004), 2,
                                      1, 2, 128, 128, 1.0, gdn.GDN_BF16, fake(0x7000),
                                      gdn.ROW_DECAY | 7, None) == gdn.GDN_ERR_ALIGNMENT
@@ -228,7 +229,7 @@ def test_commit_verify_validation(lib):
     assert call(pu=None) == gdn.GDN_ERR_INVALID_ARG
     assert call(pro=16) == gdn.GDN_ERR_INVALID_ARG
     assert call(Kp=17) == gdn.GDN_ERR_UNSUPPORTED
-    assert call(pro=gdn.ROW_DECAY) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(pro=gdn.ROW_DECAY) == gdn.GDN_ERR_WORKSPACE   # row decays accepted
     assert call(pk=fake(0x1008)) == gdn.GDN_ERR_ALIGNMENT
     assert call() == gdn.GDN_ERR_WORKSPACE
     need = lib.gdn_recurrent_commit_verify_workspace_size(2, 4, 4, 2, 128)

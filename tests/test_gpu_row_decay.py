@@ -7,9 +7,9 @@ import pytest
 import torch
 
 from linear_attention_recurrence_rule_b200 import (PROLOGUE_ALL, PROLOGUE_GATE_LOGITS, ROW_DECAY,
-                                                   GDNError, gdn_chunk_prefill, gdn_recurrent_step,
-                                                   gdn_recurrent_verify, gdn_state_commit,
-                                                   gdn_state_commit_deltas)
+                                                   gdn_chunk_prefill, gdn_recurrent_commit_verify,
+                                                   gdn_recurrent_step, gdn_recurrent_verify,
+                                                   gdn_state_commit, gdn_state_commit_deltas)
 from linear_attention_recurrence_rule_b200.inputs import (make_decode, make_prefill, make_verify,
                                                           raw_projections, row_decays,
                                                           workload_inputs)
@@ -105,13 +105,43 @@ def test_prefill_row_decay(HK, HV, dk, dv, lengths, chunk, dtype, extra):
     assert_close(hT, h_ref, dtype, "hT")
 
 
-def test_row_decay_unsupported_forms():
-    y = make_verify(2, 3, 1, 2, 32, 32, torch.float32, seed=87)
-    e = to_dev(y)
-    g_rows = row_decays((2, 3, 2, 32), seed=88).cuda()
-    with pytest.raises(GDNError):
-        gdn_recurrent_verify(e["q"], e["k"], e["v"], g_rows, e["beta"], e["state"],
-                             rollback="deltas", prologue=ROW_DECAY)
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_row_decay_update_vector_forms(dtype, d):
+    """The update-vector verify and the fused commit-then-verify with one decay
+    per value row (they run the per-draft kernel without writing states, the fused
+    round after a commit from the previous round's update vectors)."""
+    N, K, HK, HV = 6, 4, 2, 4
+    x = make_verify(N, K, HK, HV, d, d, dtype, seed=91, h0_std=0.3)
+    g_rows = row_decays((N, K, HV, d), seed=92)
+    dx = to_dev(x)
+    gd = g_rows.cuda()
+    o, _, u = gdn_recurrent_verify(dx["q"], dx["k"], dx["v"], gd, dx["beta"], dx["state"],
+                                   scale=0.6, rollback="deltas", prologue=ROW_DECAY)
+    accepted = torch.tensor([0, 1, 2, 3, 4, 2], dtype=torch.int32)
+    S2 = dx["state"].clone()
+    gdn_state_commit_deltas(dx["k"], gd, u, accepted.cuda(), S2, prologue=ROW_DECAY)
+    torch.cuda.synchronize()
+    o_ref, states_ref = O.verify_row_decay(x["q"], x["k"], x["v"], g_rows, x["beta"], x["state"],
+                                           scale=0.6)
+    assert_close(o, o_ref, dtype, "o")
+    kept = torch.as_tensor(O.commit(states_ref, accepted.numpy(), x["state"])).float()
+    assert_close(S2, kept, dtype, "committed from the update vectors")
+    # next round: this round's commit fused with the verify of new drafts
+    y = make_verify(N, K, HK, HV, d, d, dtype, seed=93, h0_std=0.3)
+    g2 = row_decays((N, K, HV, d), seed=94)
+    dy = to_dev(y)
+    S3 = dx["state"].clone()
+    o2, u2 = gdn_recurrent_commit_verify(dx["k"], gd, u, accepted.cuda(), dy["q"], dy["k"], dy["v"],
+                                         g2.cuda(), dy["beta"], S3, scale=0.6, prologue=ROW_DECAY)
+    torch.cuda.synchronize()
+    assert_close(S3, kept, dtype, "committed state (fused round)")
+    o2_ref, states2_ref = O.verify_row_decay(y["q"], y["k"], y["v"], g2, y["beta"], kept, scale=0.6)
+    assert_close(o2, o2_ref, dtype, "o (fused round)")
+    S4 = S3.clone()
+    gdn_state_commit_deltas(dy["k"], g2.cuda(), u2, torch.full((N,), K, dtype=torch.int32).cuda(), S4,
+                            prologue=ROW_DECAY)
+    torch.cuda.synchronize()
+    assert_close(S4, states2_ref[:, K - 1], dtype, "state after the fused round's drafts")
 
 
 def test_prefill_row_decay_bench_size_sampled_heads():
