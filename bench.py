@@ -494,14 +494,14 @@ NCU_TRAFFIC = {
     # verify_256x4, update-vector form, the streaming kernel: 579,929,088 read + 20,496,640
     # written (its setup kernel adds 8,682,752)
     "verify_deltas": {"bytes": 600425728, "source": "gdn_verify.cu",
-                      "sha256": "8be8a8d3e9e1d05d521c0b21ec80bc3664d346f24e58877a0c724046b6443285"},
+                      "sha256": "29b8b0ee019915d37a69fff499ebabf0aed524cd5bdefdb7f2affbf7bcaa69a2"},
     # verify_256x4, per-draft states: 554,959,104 read + 2,092,982,784 written
     "verify_states": {"bytes": 2647941888, "source": "gdn_verify.cu",
-                      "sha256": "8be8a8d3e9e1d05d521c0b21ec80bc3664d346f24e58877a0c724046b6443285"},
+                      "sha256": "29b8b0ee019915d37a69fff499ebabf0aed524cd5bdefdb7f2affbf7bcaa69a2"},
     # verify_256x4 fused round (previous commit + verify), the streaming kernel:
     # 613,593,856 read + 382,361,600 written
     "verify_fused": {"bytes": 995955456, "source": "gdn_verify.cu",
-                     "sha256": "8be8a8d3e9e1d05d521c0b21ec80bc3664d346f24e58877a0c724046b6443285"},
+                     "sha256": "29b8b0ee019915d37a69fff499ebabf0aed524cd5bdefdb7f2affbf7bcaa69a2"},
 }
 
 

@@ -836,24 +836,26 @@ int device_sm_count() {
 }
 
 template <int DK, int KT, typename Tin, bool FUSED>
-void launch_verify_wy(const VerifyArgs &a, dim3 block, cudaStream_t stream) {
+cudaError_t launch_verify_wy(const VerifyArgs &a, dim3 block, cudaStream_t stream) {
     auto setup = a.prologue ? verify_setup_kernel<DK, KT, Tin, true>
                             : verify_setup_kernel<DK, KT, Tin, false>;
     const int items = a.N * a.HV;
     constexpr int W = setup_warps<KT>();
     float *ws = static_cast<float *>(a.workspace);
     float *pend = FUSED ? ws + kWsHeaderFloats + (size_t)items * wy_item_floats(a.K, DK) : nullptr;
-    if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), stream) != cudaSuccess) return;
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(unsigned int), stream);
+    if (e != cudaSuccess) return e;
     setup<<<(unsigned)((items + W - 1) / W), W * 32, 0, stream>>>(
         static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k), a.g, a.beta, ws, items, a.K,
         a.HK, a.HV, a.scale, a.prologue, static_cast<const Tin *>(a.prev_k), a.prev_g, a.accepted,
         pend, a.prev_K);
     auto kern = verify_wy_kernel<DK, KT, Tin, FUSED>;
     constexpr size_t smem = wy_smem_bytes<DK, KT, FUSED>();
+    e = cudaGetLastError();   // the setup launch
+    if (e != cudaSuccess) return e;
     // per device and cheap: set on every launch (a process may drive several GPUs)
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return;   // the launch below reports the error
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     int per_sm = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kVerifyWarps * 32, smem) !=
             cudaSuccess ||
@@ -865,21 +867,21 @@ void launch_verify_wy(const VerifyArgs &a, dim3 block, cudaStream_t stream) {
     kern<<<grid, block, smem, stream>>>(static_cast<const Tin *>(a.v), const_cast<float *>(a.state),
                                         ws, a.u, static_cast<Tin *>(a.o), a.N, a.K, a.HV, a.dv,
                                         a.prev_u, a.prev_K);
+    return cudaGetLastError();
 }
 
 template <int DK, typename Tin>
-void launch_verify_wy_k(const VerifyArgs &a, dim3 block, cudaStream_t stream) {
+cudaError_t launch_verify_wy_k(const VerifyArgs &a, dim3 block, cudaStream_t stream) {
     const int kb = a.K > a.prev_K ? a.K : a.prev_K;   // bound for both rounds' drafts
     const bool fused = a.prev_K > 0;
     if (kb <= 4)
-        fused ? launch_verify_wy<DK, 4, Tin, true>(a, block, stream)
-              : launch_verify_wy<DK, 4, Tin, false>(a, block, stream);
-    else if (kb <= 8)
-        fused ? launch_verify_wy<DK, 8, Tin, true>(a, block, stream)
-              : launch_verify_wy<DK, 8, Tin, false>(a, block, stream);
-    else
-        fused ? launch_verify_wy<DK, 16, Tin, true>(a, block, stream)
-              : launch_verify_wy<DK, 16, Tin, false>(a, block, stream);
+        return fused ? launch_verify_wy<DK, 4, Tin, true>(a, block, stream)
+                     : launch_verify_wy<DK, 4, Tin, false>(a, block, stream);
+    if (kb <= 8)
+        return fused ? launch_verify_wy<DK, 8, Tin, true>(a, block, stream)
+                     : launch_verify_wy<DK, 8, Tin, false>(a, block, stream);
+    return fused ? launch_verify_wy<DK, 16, Tin, true>(a, block, stream)
+                 : launch_verify_wy<DK, 16, Tin, false>(a, block, stream);
 }
 
 template <int DK, typename Tin>
@@ -904,12 +906,11 @@ cudaError_t launch_verify_typed(const VerifyArgs &a, cudaStream_t stream) {
         // (with one decay per value row the mixed vectors would be per row: that
         // form runs on the per-draft kernel below, writing no states)
         switch (a.dk) {
-            case 32: launch_verify_wy_k<32, Tin>(a, block, stream); break;
-            case 64: launch_verify_wy_k<64, Tin>(a, block, stream); break;
-            case 128: launch_verify_wy_k<128, Tin>(a, block, stream); break;
+            case 32: return launch_verify_wy_k<32, Tin>(a, block, stream);
+            case 64: return launch_verify_wy_k<64, Tin>(a, block, stream);
+            case 128: return launch_verify_wy_k<128, Tin>(a, block, stream);
             default: return cudaErrorInvalidValue;
         }
-        return cudaGetLastError();
     }
     switch (a.dk) {
         case 32: launch_verify_seq<32, Tin>(a, grid, block, stream); break;
