@@ -205,7 +205,7 @@ def measure_verify(gdn, torch, dev, stream, peaks, peak_src, rank, world, max_ov
             "roofline": {"bound": "hbm", "achieved": v_gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": v_gbs / hbm_peak, "traffic": kernel_traffic("verify_" + form),
                          "peak_source": peak_src,
-                         "kernel": "verify_wy" if form == "deltas" else "verify"},
+                         "kernel": "verify_tc" if form == "deltas" else "verify"},
             "commit_roofline": {"bound": "hbm", "achieved": c_gbs, "peak": hbm_peak,
                                 "unit": "GB/s", "frac": c_gbs / hbm_peak},
             "gpu_launches": 2 * rounds, "clocks": clocks}

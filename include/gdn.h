@@ -340,6 +340,11 @@ GDN_API gdn_status gdn_recurrent_step_ex(const void *q, const void *k, const voi
  * bytes, 16-byte aligned, needed when states_out is NULL (the update-vector
  * form builds per (sequence, value head) tables there; ignored otherwise, may
  * be NULL); missing or too small returns GDN_ERR_WORKSPACE.
+ * Precision: the update-vector form with bf16 inputs, dk = dv = 128 and K <= 8
+ * (no row decays) takes the products of the fp32 state with its mixed key and
+ * query vectors on tensor cores, both factors split into bf16 hi + lo parts
+ * (each term exact up to ~2^-17 relative, the order of fp32 accumulation);
+ * every other form accumulates in fp32 on CUDA cores.
  * Supported: as gdn_recurrent_step, and 1 <= K <= GDN_VERIFY_MAX_DRAFTS.
  * Alignment: q, k, v, o, state, states_out 16-byte aligned, u_out 4-byte.
  * No output may overlap an input.  K > GDN_VERIFY_MAX_DRAFTS returns

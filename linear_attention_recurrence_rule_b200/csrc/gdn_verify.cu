@@ -21,11 +21,16 @@
 //   verify_setup_kernel +  update vectors only: per-head tables, then a
 //   verify_wy_kernel       persistent pass fed by bulk copies through a ring of
 //                          shared-memory stages (the state is only read)
+//   verify_tc_kernel       the same products on tensor cores (bf16 inputs,
+//                          dk = dv = 128, up to 8 drafts)
 //   commit_kernel          copy of the state after the last kept draft
 //   commit_deltas_kernel   in-place rebuild from S_0 and the kept u_t
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
+#include <type_traits>
+
 #include "tc_primitives.cuh"
+#include "tma_host.h"
 
 namespace gdn {
 namespace {
@@ -699,6 +704,274 @@ verify_wy_kernel(const Tin *__restrict__ v, float *state, float *__restrict__ ws
     }
 }
 
+// Update vectors on tensor cores (bf16 inputs, dk = dv = 128, K <= 8).  The 2K
+// dot products per state row of the streaming kernel above are, per (sequence,
+// value head), one product of the [128 x 128] state with the 16 mixed vectors
+// (k'_t in row t, q'_t in row 8 + t).  Both factors are split into bf16 hi + lo:
+// the B operand stacks [k'; q'] hi (rows 0..15) over its lo parts (rows
+// 16..31), and D = S_hi B^T + S_lo B^T (N = 32) gives in column n + 16 c the
+// product with part c of mixed vector n, so D[:, n] + D[:, n + 16] is the whole
+// fp32 dot product up to the rounding of the two lo parts (~2^-17 of each
+// term, the order of fp32 accumulation over 128 terms).
+//   * states stream through three 64 KB shared-memory stages by TMA (four
+//     [128 rows x 32 fp32] boxes, 128-byte swizzle); a stage is refilled with
+//     the item three ahead as soon as the CTA has read it;
+//   * thread = tensor-memory lane = state row: warps w and w + 4 take the two
+//     64-column halves of rows 32 (w % 4) .. + 31, split them into bf16 hi / lo
+//     (two per 32-bit column) and store them to tensor memory as the A operand
+//     (two buffers);
+//   * k', q' (fp32 tables of the setup kernel, read one item ahead into
+//     registers) become the swizzled B tile (two buffers);
+//   * one elected thread issues 2 x 8 MMAs (M = 128, N = 32, K = 16) into one
+//     of two accumulators and commits them to an mbarrier;
+//   * the read-out of item i - 1 (accumulator -> registers, plus the K x K
+//     value terms, stores of u and o) runs while the MMAs of item i execute.
+// Waits are bounded: a timeout sets the workspace status word, and the CTA
+// waits (bounded) for its copies and MMAs in flight before it frees its tensor
+// memory and returns.
+constexpr int kTcThreads = 256;
+constexpr int kTcStages = 3;
+constexpr int kTcDrafts = 8;
+constexpr uint32_t kTcStateBytes = 128u * 128u * 4u;   // one fp32 state
+constexpr uint32_t kTcBTile = 8192;                    // [32 x 128] bf16: hi rows, lo rows
+constexpr int kTcCoef = 2 * kTcDrafts * kTcDrafts;    // Vu, Vy, each [8][8]
+// tensor-memory columns: A (hi 64 + lo 64) x 2 buffers, then D (32) x 2
+constexpr uint32_t kTcColA = 0, kTcColD = 256, kTcCols = 512;
+constexpr size_t tc_smem_bytes() {
+    return 1024 + kTcStages * (size_t)kTcStateBytes + 2 * (size_t)kTcBTile +
+           kTcStages * (size_t)kTcCoef * sizeof(float) + (kTcStages + 2) * sizeof(uint64_t) + 16;
+}
+
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = tc::pack_bf16x2(a - hf.x, b - hf.y);
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+verify_tc_kernel(const __grid_constant__ CUtensorMap tm_s, const __nv_bfloat16 *__restrict__ v,
+                 float *__restrict__ ws, float *__restrict__ u_out, __nv_bfloat16 *__restrict__ o,
+                 int N, int K, int HV) {
+    extern __shared__ uint8_t tc_smem_raw[];
+    const uint32_t raw_s = tc::smem_u32(tc_smem_raw);
+    uint8_t *sm = tc_smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
+    uint8_t *stages = sm;                                         // [3][64 KB]
+    uint8_t *btile = sm + kTcStages * (size_t)kTcStateBytes;      // [2][8 KB]
+    float *coef = reinterpret_cast<float *>(btile + 2 * kTcBTile);   // [3][Vu | Vy]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(coef + kTcStages * kTcCoef);   // stages
+    uint64_t *mbar = bars + kTcStages;                                           // MMAs [2]
+    uint32_t *slot = reinterpret_cast<uint32_t *>(mbar + 2);
+    constexpr uint32_t kIdesc = tc::idesc_bf16(128, 32, false, false);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = 32 * (warp & 3) + lane;   // this thread's state row (tensor-memory lane)
+    const int kh = warp >> 2;               // its column half; also: 0 reads out u, 1 o
+    const long long total = (long long)N * HV;
+    const int mine = total > blockIdx.x ? (int)((total - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
+    const size_t item_floats = wy_item_floats(K, 128);
+    const float *tables = ws + kWsHeaderFloats;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+
+    // what item nh needs besides its state, read one item ahead: the thread's
+    // 8 values of [k'; q'] (row tid / 16, columns 8 (tid % 16) ..), one table
+    // coefficient (entry tid of [Vu | Vy] padded to [2][8][8]), and the K values
+    // of v at row r (raw bf16).  Heads < 2^31 (the launcher checks).
+    struct Pre {
+        float4 kq0, kq1;
+        float c;
+        int n, h;
+        unsigned short vr[kTcDrafts];
+    };
+    auto prefetch = [&](int nh, Pre &p) {
+        p.n = nh / HV;
+        p.h = nh - p.n * HV;
+        const float *tab = tables + (size_t)nh * item_floats;
+        const int rr = tid >> 4, t = rr & 7;
+        if (t < K) {
+            const float4 *src = reinterpret_cast<const float4 *>(
+                tab + (size_t)((rr < 8 ? 0 : K) + t) * 128 + (tid & 15) * 8);
+            p.kq0 = __ldg(src);
+            p.kq1 = __ldg(src + 1);
+        } else {
+            p.kq0 = p.kq1 = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        const int ct = (tid >> 3) & 7, cj = tid & 7;
+        p.c = (tid < kTcCoef && ct < K && cj < K)
+                  ? __ldg(tab + 2 * (size_t)K * 128 + (tid >> 6) * K * K + ct * K + cj)
+                  : 0.f;
+        const unsigned short *vs = reinterpret_cast<const unsigned short *>(v) +
+                                   ((size_t)p.n * K * HV + p.h) * 128 + r;
+        const size_t vstride = (size_t)HV * 128;
+#pragma unroll
+        for (int j = 0; j < kTcDrafts; ++j)
+            p.vr[j] = j < K ? __ldg(vs + j * vstride) : (unsigned short)0;
+    };
+    auto issue = [&](int i) {   // thread 0: item i's state into stage i % 3
+        const int nh = (int)blockIdx.x + i * (int)gridDim.x;
+        uint8_t *dst = stages + (size_t)(i % kTcStages) * kTcStateBytes;
+        uint64_t *bar = &bars[i % kTcStages];
+        tc::mbar_arrive_expect_tx(bar, kTcStateBytes);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tc::tma_load_3d(dst + b * 16384, &tm_s, bar, 32 * b, 0, nh);
+    };
+
+    if (tid == 0) {
+        for (int b = 0; b < kTcStages + 2; ++b) tc::mbar_init(&bars[b], 1);
+        tc::fence_barrier_init();
+    }
+    if (warp == 0) tc::tmem_alloc(slot, kTcCols);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *slot;
+    int issued = 0;   // thread 0
+    if (tid == 0)
+        for (; issued < kTcStages && issued < mine; ++issued) issue(issued);
+
+    bool mfail = false;
+    // read-out of item p (sequence n, value head h):
+    //   u_t = S_0[r] . k'_t + sum_{j<=t} Vu[t][j] v_j[r]   (warps 0-3)
+    //   o_t = S_0[r] . q'_t + sum_{j<=t} Vy[t][j] v_j[r]   (warps 4-7)
+    auto readout = [&](int p, int n, int h, const unsigned short (&vv)[kTcDrafts]) {
+        if (!tc::mbar_wait(&mbar[p & 1], (uint32_t)((p >> 1) & 1), kWyWaitLimit)) mfail = true;
+        tc::tc_fence_after();
+        float d0[16], d1[16];
+        const uint32_t dcol = tmem + kTcColD + (uint32_t)(p & 1) * 32u + lane_off;
+        tc::tmem_ld16(dcol, d0);
+        tc::tmem_ld16(dcol + 16u, d1);
+        tc::tmem_wait_ld();
+        const float *cf = coef + (p % kTcStages) * kTcCoef + kh * 64;
+        float vf[kTcDrafts];
+#pragma unroll
+        for (int j = 0; j < kTcDrafts; ++j) vf[j] = __uint_as_float((uint32_t)vv[j] << 16);
+        const size_t obase = ((size_t)n * K * HV + h) * 128 + r, ostride = (size_t)HV * 128;
+#pragma unroll
+        for (int t = 0; t < kTcDrafts; ++t) {
+            if (t < K) {
+                float val = kh ? d0[8 + t] + d1[8 + t] : d0[t] + d1[t];
+#pragma unroll
+                for (int j = 0; j <= t; ++j) val = fmaf(cf[t * kTcDrafts + j], vf[j], val);
+                if (kh == 0) {
+                    if (u_out) u_out[obase + t * ostride] = val;
+                } else {
+                    o[obase + t * ostride] = __float2bfloat16_rn(val);
+                }
+            }
+        }
+    };
+
+    Pre cur, nxt;
+    unsigned short vprev[kTcDrafts];
+    int nprev = 0, hprev = 0;
+    if (mine > 0) prefetch((int)blockIdx.x, cur);
+    bool ok = true;
+    int consumed = 0;   // items whose state landed and whose MMAs were issued
+    for (int i = 0; i < mine; ++i) {
+        if (i + 1 < mine) prefetch((int)blockIdx.x + (i + 1) * (int)gridDim.x, nxt);
+        const int st = i % kTcStages;
+        const bool landed = tc::mbar_wait(&bars[st], (uint32_t)((i / kTcStages) & 1), kWyWaitLimit);
+        // row r, columns [64 kh, 64 kh + 64): boxes 2 kh and 2 kh + 1, 16-byte
+        // chunk c of a row at chunk position c ^ (r % 8)
+        const uint8_t *stg = stages + (size_t)st * kTcStateBytes;
+        float4 x[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int box = 2 * kh + (j >> 3), c = j & 7;
+            x[j] = *reinterpret_cast<const float4 *>(stg + box * 16384 + r * 128 +
+                                                     (((c ^ r) & 7) << 4));
+        }
+        // A operand: hi at columns [0, 64), lo at [64, 128) of this item's buffer,
+        // bf16 pair (2w, 2w + 1) of the row in column w
+        const uint32_t abuf = tmem + kTcColA + (uint32_t)(i & 1) * 128u + lane_off + 32u * kh;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float hw[16], lw[16];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 e = x[8 * half + q];
+                uint32_t h0, l0, h1, l1;
+                split_bf16x2(e.x, e.y, h0, l0);
+                split_bf16x2(e.z, e.w, h1, l1);
+                hw[2 * q] = __uint_as_float(h0);
+                hw[2 * q + 1] = __uint_as_float(h1);
+                lw[2 * q] = __uint_as_float(l0);
+                lw[2 * q + 1] = __uint_as_float(l1);
+            }
+            tc::tmem_st16(abuf + 16u * half, hw);
+            tc::tmem_st16(abuf + 64u + 16u * half, lw);
+        }
+        // B operand: row tid / 16 of [k'; q'], columns 8 (tid % 16) .. + 7, as one
+        // 16-byte chunk of hi row rr and of lo row 16 + rr (64-column atoms of
+        // 32 rows, 4 KB each)
+        {
+            const int rr = tid >> 4, cc = tid & 15;
+            const uint32_t atom = (uint32_t)(cc >> 3) * 4096u;
+            uint8_t *bt = btile + (i & 1) * kTcBTile;
+            uint32_t hb[4], lb[4];
+            split_bf16x2(cur.kq0.x, cur.kq0.y, hb[0], lb[0]);
+            split_bf16x2(cur.kq0.z, cur.kq0.w, hb[1], lb[1]);
+            split_bf16x2(cur.kq1.x, cur.kq1.y, hb[2], lb[2]);
+            split_bf16x2(cur.kq1.z, cur.kq1.w, hb[3], lb[3]);
+            *reinterpret_cast<uint4 *>(bt + atom + tc::sw128_chunk((uint32_t)rr, (uint32_t)cc)) =
+                make_uint4(hb[0], hb[1], hb[2], hb[3]);
+            *reinterpret_cast<uint4 *>(bt + atom + tc::sw128_chunk((uint32_t)(16 + rr), (uint32_t)cc)) =
+                make_uint4(lb[0], lb[1], lb[2], lb[3]);
+        }
+        if (tid < kTcCoef) coef[st * kTcCoef + tid] = cur.c;
+        tc::tmem_wait_st();
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        ok = __syncthreads_and(landed && !mfail);   // also: item i - 1's read-out is done
+        if (!ok) break;
+        consumed = i + 1;
+        if (tid == 0 && issued < mine) {   // stage st has been read: the item 3 ahead
+            issue(issued);
+            ++issued;
+        }
+        if (warp == 0) {
+            tc::tc_fence_after();
+            if (tc::elect_one()) {
+                const uint32_t dacc = tmem + kTcColD + (uint32_t)(i & 1) * 32u;
+                const uint32_t abase = tmem + kTcColA + (uint32_t)(i & 1) * 128u;
+                const uint32_t bbase = tc::smem_u32(btile + (i & 1) * kTcBTile);
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {   // S_hi k-steps, then S_lo k-steps
+                    const int k8 = kk & 7;
+                    const uint64_t bd = tc::sdesc_sw128(
+                        bbase + (uint32_t)(k8 >> 2) * 4096u + (uint32_t)(k8 & 3) * 32u, 16, 1024);
+                    tc::mma_bf16_ts(dacc, abase + (kk >= 8 ? 64u : 0u) + 8u * k8, bd, kIdesc, kk > 0);
+                }
+                tc::mma_commit(&mbar[i & 1]);
+            }
+            __syncwarp();
+        }
+        if (i >= 1) readout(i - 1, nprev, hprev, vprev);
+#pragma unroll
+        for (int j = 0; j < kTcDrafts; ++j) vprev[j] = cur.vr[j];
+        nprev = cur.n;
+        hprev = cur.h;
+        cur = nxt;
+    }
+    if (ok && mine > 0) readout(mine - 1, nprev, hprev, vprev);
+    tc::tc_fence_before();
+    const bool all_ok = __syncthreads_and(ok && !mfail);
+    if (!all_ok && tid == 0) {
+        atomicExch(reinterpret_cast<unsigned int *>(ws), 1u);
+        // copies still in flight land, and the last MMAs complete, before this
+        // CTA's shared and tensor memory are released
+        for (int j = consumed; j < issued; ++j)
+            tc::mbar_wait(&bars[j % kTcStages], (uint32_t)((j / kTcStages) & 1), kWyWaitLimit);
+        if (consumed > 0)
+            tc::mbar_wait(&mbar[(consumed - 1) & 1], (uint32_t)(((consumed - 1) >> 1) & 1), kWyWaitLimit);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, kTcCols);
+    }
+}
+
 // Roll back after verification: state[n] <- states[n][accepted[n] - 1] when
 // 1 <= accepted[n] <= K, unchanged otherwise.
 __global__ void __launch_bounds__(256)
@@ -835,6 +1108,30 @@ int device_sm_count() {
     return count;
 }
 
+// The states of `items` heads as a [items][128][128] fp32 tensor, read in
+// [128 rows x 32 columns] boxes with the 128-byte swizzle.
+bool tc_state_map(CUtensorMap *tm, const float *state, int items) {
+    if ((reinterpret_cast<uintptr_t>(state) & 15) != 0) return false;
+    const uint64_t dims[3] = {128, 128, (uint64_t)items};
+    const uint64_t strides[2] = {128 * sizeof(float), 128 * 128 * sizeof(float)};
+    const uint32_t box[3] = {32, 128, 1};
+    return encode_f32_map(tm, state, 3, dims, strides, box);
+}
+
+cudaError_t launch_verify_tc(const CUtensorMap &tm, const VerifyArgs &a, float *ws, int items,
+                             cudaStream_t stream) {
+    constexpr size_t smem = tc_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(verify_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int sms = device_sm_count();
+    const unsigned grid = (unsigned)(items < sms ? items : sms);
+    verify_tc_kernel<<<grid, kTcThreads, smem, stream>>>(
+        tm, static_cast<const __nv_bfloat16 *>(a.v), ws, a.u, static_cast<__nv_bfloat16 *>(a.o),
+        a.N, a.K, a.HV);
+    return cudaGetLastError();
+}
+
 template <int DK, int KT, typename Tin, bool FUSED>
 cudaError_t launch_verify_wy(const VerifyArgs &a, dim3 block, cudaStream_t stream) {
     auto setup = a.prologue ? verify_setup_kernel<DK, KT, Tin, true>
@@ -853,6 +1150,12 @@ cudaError_t launch_verify_wy(const VerifyArgs &a, dim3 block, cudaStream_t strea
     constexpr size_t smem = wy_smem_bytes<DK, KT, FUSED>();
     e = cudaGetLastError();   // the setup launch
     if (e != cudaSuccess) return e;
+    if constexpr (DK == 128 && KT <= kTcDrafts && !FUSED &&
+                  std::is_same<Tin, __nv_bfloat16>::value) {
+        CUtensorMap tm;
+        if (a.dv == 128 && (long long)a.N * a.HV < (1LL << 31) && tc_state_map(&tm, a.state, items))
+            return launch_verify_tc(tm, a, ws, items, stream);
+    }
     // per device and cheap: set on every launch (a process may drive several GPUs)
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -41,4 +41,20 @@ inline bool encode_bf16_map(CUtensorMap *map, const void *base, int rank, const 
     return r == CUDA_SUCCESS;
 }
 
+// fp32 tensor, otherwise as above.
+inline bool encode_f32_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                           const uint64_t *strides_bytes, const uint32_t *box,
+                           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (cuuint32_t)rank,
+                     const_cast<void *>(base), reinterpret_cast<const cuuint64_t *>(dims),
+                     reinterpret_cast<const cuuint64_t *>(strides_bytes),
+                     reinterpret_cast<const cuuint32_t *>(box), estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace gdn

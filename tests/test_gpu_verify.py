@@ -22,6 +22,8 @@ pytestmark = pytest.mark.gpu
     (5, 1, 2, 4, 64, 48, torch.float32),      # one draft: the decode step
     (7, 2, 1, 2, 32, 200, torch.bfloat16),    # dv not a multiple of a band
     (33, 4, 2, 4, 128, 128, torch.bfloat16),  # the model's head shape
+    (9, 1, 1, 2, 128, 128, torch.bfloat16),   # tensor-core form, one draft
+    (80, 8, 1, 2, 128, 128, torch.bfloat16),  # its largest count, 160 heads: two per CTA
     (6, 5, 1, 2, 128, 128, torch.float32),    # first count past the 4-draft bound
     (3, 8, 1, 2, 128, 256, torch.float32),    # two bands per state
     (4, 11, 2, 2, 32, 72, torch.bfloat16),    # a count between the 8 and 16 bounds
