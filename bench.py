@@ -491,17 +491,17 @@ NCU_TRAFFIC = {
     # standalone output gate over the 64K bench outputs: 1,073,846,528 read + 492,012,288 written
     "output_gate": {"bytes": 1565858816, "source": "gdn_layer.cu",
                     "sha256": "03e2d96c3e8a4dbc194fc0970d48afd7b79fc033f0bb351a248b95dfc9e837bd"},
-    # verify_256x4, update-vector form, the streaming kernel: 579,929,088 read + 20,496,640
-    # written (its setup kernel adds 8,682,752)
-    "verify_deltas": {"bytes": 600425728, "source": "gdn_verify.cu",
-                      "sha256": "29b8b0ee019915d37a69fff499ebabf0aed524cd5bdefdb7f2affbf7bcaa69a2"},
+    # verify_256x4, update-vector form, the tensor-core kernel: 579,903,488 read +
+    # 24,379,904 written (its setup kernel adds 8,682,752)
+    "verify_deltas": {"bytes": 604283392, "source": "gdn_verify.cu",
+                      "sha256": "a286b231a00aee66bf99dcea49f850b1551e49bf3c5e08a9b8e3c37c6e700872"},
     # verify_256x4, per-draft states: 554,959,104 read + 2,092,982,784 written
     "verify_states": {"bytes": 2647941888, "source": "gdn_verify.cu",
-                      "sha256": "29b8b0ee019915d37a69fff499ebabf0aed524cd5bdefdb7f2affbf7bcaa69a2"},
+                      "sha256": "a286b231a00aee66bf99dcea49f850b1551e49bf3c5e08a9b8e3c37c6e700872"},
     # verify_256x4 fused round (previous commit + verify), the streaming kernel:
     # 613,593,856 read + 382,361,600 written
     "verify_fused": {"bytes": 995955456, "source": "gdn_verify.cu",
-                     "sha256": "29b8b0ee019915d37a69fff499ebabf0aed524cd5bdefdb7f2affbf7bcaa69a2"},
+                     "sha256": "a286b231a00aee66bf99dcea49f850b1551e49bf3c5e08a9b8e3c37c6e700872"},
 }
 
 
