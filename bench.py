@@ -494,14 +494,14 @@ NCU_TRAFFIC = {
     # verify_256x4, update-vector form, the tensor-core kernel: 579,903,488 read +
     # 24,379,904 written (its setup kernel adds 8,682,752)
     "verify_deltas": {"bytes": 604283392, "source": "gdn_verify.cu",
-                      "sha256": "a286b231a00aee66bf99dcea49f850b1551e49bf3c5e08a9b8e3c37c6e700872"},
+                      "sha256": "19b8174a5cb7f9ff183a9cf3f22d26aca35eac177b8e8b360788a170159747f9"},
     # verify_256x4, per-draft states: 554,959,104 read + 2,092,982,784 written
     "verify_states": {"bytes": 2647941888, "source": "gdn_verify.cu",
-                      "sha256": "a286b231a00aee66bf99dcea49f850b1551e49bf3c5e08a9b8e3c37c6e700872"},
+                      "sha256": "19b8174a5cb7f9ff183a9cf3f22d26aca35eac177b8e8b360788a170159747f9"},
     # verify_256x4 fused round (previous commit + verify), the streaming kernel:
     # 613,593,856 read + 382,361,600 written
     "verify_fused": {"bytes": 995955456, "source": "gdn_verify.cu",
-                     "sha256": "a286b231a00aee66bf99dcea49f850b1551e49bf3c5e08a9b8e3c37c6e700872"},
+                     "sha256": "19b8174a5cb7f9ff183a9cf3f22d26aca35eac177b8e8b360788a170159747f9"},
 }
 
 

@@ -60,6 +60,18 @@ GDN_API int gdn_selftest_verify_timeout(const void *v, const float *state, int N
                                         void *o, float *u_out, void *workspace,
                                         size_t workspace_bytes, gdn_stream_t stream);
 
+/*
+ * The same for the tensor-core form of the update-vector verify (bf16 v/o,
+ * dk = dv = 128, K <= 8 drafts; the form gdn_recurrent_verify runs for those
+ * shapes): before any copy or MMA is issued, its first wait has a limit of zero
+ * polls on a barrier nothing arrives on; the status word records the timeout, the
+ * CTA frees its tensor memory and returns.  Arguments as gdn_selftest_verify_timeout
+ * (state 16-byte aligned); 1 <= K <= 8.
+ */
+GDN_API int gdn_selftest_verify_tc_timeout(const void *v, const float *state, int N, int K,
+                                           int HV, void *o, float *u_out, void *workspace,
+                                           size_t workspace_bytes, gdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -78,6 +78,7 @@ cudaError_t launch_decode(const StepArgs &a, cudaStream_t stream);
 cudaError_t launch_verify(const VerifyArgs &a, cudaStream_t stream);
 // test-only: the update-vector verify's streaming kernel with a first wait that gives up
 cudaError_t launch_verify_wy_timeout_test(const VerifyArgs &a, cudaStream_t stream);
+cudaError_t launch_verify_tc_timeout_test(const VerifyArgs &a, cudaStream_t stream);
 
 // Largest draft count of the verify kernels (GDN_VERIFY_MAX_DRAFTS in gdn.h).
 constexpr int kVerifyMaxDrafts = 16;

@@ -244,3 +244,17 @@ extern "C" int gdn_selftest_verify_timeout(const void *v, const float *state, in
     const cudaError_t err = gdn::launch_verify_wy_timeout_test(a, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
+
+// Test-only tensor-core update-vector verify kernel whose first wait gives up at
+// once (see gdn_selftest.h).
+extern "C" int gdn_selftest_verify_tc_timeout(const void *v, const float *state, int N, int K,
+                                              int HV, void *o, float *u_out, void *workspace,
+                                              size_t workspace_bytes, gdn_stream_t stream) {
+    if (!v || !state || !o || !workspace) return GDN_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || K > 8 || HV <= 0) return GDN_ERR_INVALID_ARG;
+    if (workspace_bytes < gdn_recurrent_verify_workspace_size(N, K, HV, 128)) return GDN_ERR_WORKSPACE;
+    gdn::VerifyArgs a{nullptr, nullptr, v, nullptr, nullptr, state, nullptr, u_out, N, K, 1, HV, 128, 128,
+                      1.0f, GDN_BF16, o, 0u, workspace, workspace_bytes};
+    const cudaError_t err = gdn::launch_verify_tc_timeout_test(a, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}

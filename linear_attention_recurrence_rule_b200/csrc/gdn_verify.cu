@@ -728,7 +728,9 @@ verify_wy_kernel(const Tin *__restrict__ v, float *state, float *__restrict__ ws
 //     value terms, stores of u and o) runs while the MMAs of item i execute.
 // Waits are bounded: a timeout sets the workspace status word, and the CTA
 // waits (bounded) for its copies and MMAs in flight before it frees its tensor
-// memory and returns.
+// memory and returns.  TMO: a test-only instance whose first wait -- before any
+// copy or MMA is issued -- has a limit of zero polls on a barrier nothing has
+// armed, so the timeout path runs without a real hang.
 constexpr int kTcThreads = 256;
 constexpr int kTcStages = 3;
 constexpr int kTcDrafts = 8;
@@ -749,6 +751,7 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uin
     lo = tc::pack_bf16x2(a - hf.x, b - hf.y);
 }
 
+template <bool TMO = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
 verify_tc_kernel(const __grid_constant__ CUtensorMap tm_s, const __nv_bfloat16 *__restrict__ v,
                  float *__restrict__ ws, float *__restrict__ u_out, __nv_bfloat16 *__restrict__ o,
@@ -825,6 +828,17 @@ verify_tc_kernel(const __grid_constant__ CUtensorMap tm_s, const __nv_bfloat16 *
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *slot;
+    if (TMO) {
+        int gave_up = 0;
+        if (tid == 0 && !tc::mbar_test_wait(&bars[0], 0u)) {
+            atomicExch(reinterpret_cast<unsigned int *>(ws), 1u);
+            gave_up = 1;
+        }
+        if (__syncthreads_or(gave_up)) {
+            if (warp == 0) tc::tmem_dealloc(tmem, kTcCols);
+            return;
+        }
+    }
     int issued = 0;   // thread 0
     if (tid == 0)
         for (; issued < kTcStages && issued < mine; ++issued) issue(issued);
@@ -1121,12 +1135,12 @@ bool tc_state_map(CUtensorMap *tm, const float *state, int items) {
 cudaError_t launch_verify_tc(const CUtensorMap &tm, const VerifyArgs &a, float *ws, int items,
                              cudaStream_t stream) {
     constexpr size_t smem = tc_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(verify_tc_kernel,
+    cudaError_t e = cudaFuncSetAttribute(verify_tc_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int sms = device_sm_count();
     const unsigned grid = (unsigned)(items < sms ? items : sms);
-    verify_tc_kernel<<<grid, kTcThreads, smem, stream>>>(
+    verify_tc_kernel<false><<<grid, kTcThreads, smem, stream>>>(
         tm, static_cast<const __nv_bfloat16 *>(a.v), ws, a.u, static_cast<__nv_bfloat16 *>(a.o),
         a.N, a.K, a.HV);
     return cudaGetLastError();
@@ -1292,6 +1306,28 @@ cudaError_t launch_verify_wy_timeout_test(const VerifyArgs &a, cudaStream_t stre
         static_cast<const __nv_bfloat16 *>(a.v), const_cast<float *>(a.state),
         static_cast<float *>(a.workspace), a.u, static_cast<__nv_bfloat16 *>(a.o), a.N, a.K, a.HV,
         a.dv, nullptr, 0);
+    return cudaGetLastError();
+}
+
+// Test-only: the tensor-core update-vector kernel (d = 128, up to 8 drafts, bf16)
+// whose first wait gives up at once; the workspace status word reads nonzero
+// afterwards.
+cudaError_t launch_verify_tc_timeout_test(const VerifyArgs &a, cudaStream_t stream) {
+    const long long heads = (long long)a.N * a.HV;
+    if (heads >= (1LL << 31)) return cudaErrorInvalidValue;
+    CUtensorMap tm;
+    if (!tc_state_map(&tm, a.state, (int)heads)) return cudaErrorInvalidValue;
+    constexpr size_t smem = tc_smem_bytes();
+    cudaError_t e = cudaMemsetAsync(a.workspace, 0, sizeof(unsigned int), stream);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(verify_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    const int sms = device_sm_count();
+    const unsigned grid = (unsigned)(heads < sms ? heads : sms);
+    verify_tc_kernel<true><<<grid, kTcThreads, smem, stream>>>(
+        tm, static_cast<const __nv_bfloat16 *>(a.v), static_cast<float *>(a.workspace), a.u,
+        static_cast<__nv_bfloat16 *>(a.o), a.N, a.K, a.HV);
     return cudaGetLastError();
 }
 

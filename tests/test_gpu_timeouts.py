@@ -79,3 +79,28 @@ def test_verify_timeout_path_then_normal_call():
     assert gdn.gdn_read_status(ws) == gdn.GDN_OK
     o_ref, _ = O.verify(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state"])
     assert_close(o2, o_ref, torch.bfloat16, "o after the timed-out call")
+
+
+def test_verify_tc_timeout_path_then_normal_call():
+    """The tensor-core update-vector kernel (bf16, d = 128, up to 8 drafts)."""
+    lib = gdn.load_library()
+    f = lib.gdn_selftest_verify_tc_timeout
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, ctypes.c_size_t, P]
+    N, K, HK, HV = 90, 6, 1, 2     # 180 heads: more than one per CTA
+    x = make_verify(N, K, HK, HV, 128, 128, torch.bfloat16, seed=79, h0_std=0.2)
+    d = to_dev(x)
+    need = gdn.gdn_recurrent_verify_workspace_size(N, K, HV, 128)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(d["v"])
+    u = torch.empty(N, K, HV, 128, device="cuda")
+    rc = f(_ptr(d["v"]), _ptr(d["state"]), N, K, HV, _ptr(o), _ptr(u), _ptr(ws), need, _stream())
+    assert rc == gdn.GDN_OK
+    torch.cuda.synchronize()
+    assert gdn.gdn_read_status(ws) == gdn.GDN_ERR_TIMEOUT
+    o2, _, u2 = gdn.gdn_recurrent_verify(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                                         rollback="deltas", workspace=ws)
+    torch.cuda.synchronize()
+    assert gdn.gdn_read_status(ws) == gdn.GDN_OK
+    o_ref, _ = O.verify(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state"])
+    assert_close(o2, o_ref, torch.bfloat16, "o after the timed-out call")
